@@ -1,0 +1,64 @@
+"""Seeded synthetic inputs for the RaZeR hot path (no quantization arithmetic).
+
+The RaZeR pages evaluate on Llama/Qwen weights and activations, which are not
+available here; these generators stand in for them with the shapes and value
+distributions of the standard workloads:
+
+* weights: i.i.d. N(0, std^2) (std 0.02 for Llama-3-8B-shaped layers, 0.015
+  for Llama-3-70B-shaped ones) with 0.1% of the entries, at seeded positions,
+  multiplied by 10 before the cast to fp16;
+* activation vectors for GEMV/GEMM: N(0, 1);
+* online-quantizer activations: rows N(0, 1) with 8 seeded channels scaled
+  x50 to mimic activation outlier channels, cast to bf16.
+
+Everything is generated on the host with ``torch.Generator('cpu')`` so the
+same tensors feed the CPU oracle and the GPU path.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def weight(N: int, K: int, *, std: float = 0.02, seed: int = 0, dtype=torch.float16,
+           outlier_frac: float = 0.001, outlier_mult: float = 10.0) -> torch.Tensor:
+    """[N, K] weight matrix, N(0, std^2) with a seeded 0.1% of entries x10."""
+    g = _gen(seed)
+    w = torch.empty(N * K, dtype=torch.float32)
+    w.normal_(0.0, std, generator=g)
+    n_out = int(round(outlier_frac * N * K))
+    if n_out:
+        pos = torch.randperm(N * K, generator=g)[:n_out]
+        w[pos] *= outlier_mult
+    return w.view(N, K).to(dtype)
+
+
+def vectors(B: int, K: int, *, seed: int = 1, dtype=torch.float16) -> torch.Tensor:
+    """[B, K] activations, N(0, 1)."""
+    g = _gen(seed)
+    x = torch.empty(B, K, dtype=torch.float32)
+    x.normal_(0.0, 1.0, generator=g)
+    return x.to(dtype)
+
+
+def outlier_activations(M: int, K: int, *, seed: int = 2, n_channels: int = 8,
+                        channel_mult: float = 50.0, dtype=torch.bfloat16) -> torch.Tensor:
+    """[M, K] activations: rows N(0, 1), 8 seeded channels scaled x50."""
+    g = _gen(seed)
+    x = torch.empty(M, K, dtype=torch.float32)
+    x.normal_(0.0, 1.0, generator=g)
+    ch = torch.randperm(K, generator=g)[:n_channels]
+    x[:, ch] *= channel_mult
+    return x.to(dtype)
+
+
+def to_numpy_bits(t: torch.Tensor) -> np.ndarray:
+    """Raw 16-bit payload of an fp16/bf16 CPU tensor as a uint16 array."""
+    assert t.dtype in (torch.float16, torch.bfloat16)
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)

@@ -1,0 +1,363 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+* hand-worked rows from the worked example of the RaZeR notes (golden file);
+* library routines: torch float8_e4m3fn decode/encode (OCP E4M3, RNE),
+  numpy float16 / torch bfloat16 rounding, numpy float32 division and a
+  numpy float64 matmul;
+* brute-force enumeration of every code assignment x every special value with
+  exact rationals (fractions.Fraction) on tiny blocks;
+* invariants of the method on synthetic config-like tensors.
+"""
+import itertools
+import math
+import random
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from bit_quantization_razer_b200 import workloads
+from tests.golden_cases import case_tensor, load_cases
+
+FMT = {"weight": 0, "act": 1, "nvfp4": 2}
+
+
+def oracle_input(t: torch.Tensor):
+    import oracle
+
+    if t.dtype == torch.bfloat16:
+        return oracle.Bf16Bits(workloads.to_numpy_bits(t))
+    return t.numpy()
+
+
+# ----------------------------------------------------------------------------
+# hand-worked rows
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("case", load_cases(), ids=lambda c: c["name"])
+def test_worked_rows(orc, case):
+    fmt = FMT[case["fmt"]]
+    x = case_tensor(case)
+    xin = oracle_input(x)
+    ts = orc.tensor_scale(xin, fmt)
+    assert ts == case["ts"]
+    codes, scales, ts2, _ = orc.quantize(xin, fmt)
+    assert ts2 == case["ts"]
+    np.testing.assert_array_equal(codes[0], case["codes"])
+    np.testing.assert_array_equal(scales[0], case["scales"])
+    deq = orc.dequant(codes, scales, ts, fmt, "f32")
+    np.testing.assert_array_equal(deq[0], np.array(case["dequant"], np.float32))
+    ones = np.ones((1, 32), np.float16)
+    y = orc.gemm_ref(ones, codes, scales, ts, fmt)
+    assert y[0, 0] == case["ones"]
+
+
+# ----------------------------------------------------------------------------
+# scale formats
+# ----------------------------------------------------------------------------
+def test_e4m3_decode_matches_torch(orc):
+    codes = torch.arange(0, 127, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([orc.scale_value(1, int(c)) for c in range(127)])
+    np.testing.assert_array_equal(got, ref)
+    assert orc.scale_max(1) == 448.0 and orc.scale_max(2) == 448.0
+
+
+def test_e3m3_decode(orc):
+    vals = np.array([orc.scale_value(0, c) for c in range(64)])
+    # anchors of an E3M3 / bias-3 format with subnormals
+    assert vals[0x00] == 0.0 and vals[0x01] == 1 / 32 and vals[0x07] == 7 / 32
+    assert vals[0x08] == 0.25 and vals[0x18] == 1.0 and vals[0x3F] == 30.0
+    assert np.all(np.diff(vals) > 0)
+    # the normal range (codes e >= 1) is the E4M3 grid on [0.25, 30]: E3M3
+    # code (e, m) has the value of OCP E4M3 code (e + 4, m)
+    e4 = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(8, 64):
+        e, m = c >> 3, c & 7
+        assert vals[c] == e4[((e + 4) << 3) | m]
+    # subnormal spacing 1/32 continues into the first binade
+    np.testing.assert_array_equal(np.diff(vals[:16]), np.full(15, 1 / 32))
+
+
+def _adversarial_scales(hi: float, n_random: int, seed: int):
+    rng = np.random.default_rng(seed)
+    pts = set()
+    e4 = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    grid = sorted(set(float(v) for v in e4 if v <= hi))
+    for a, b in zip(grid[:-1], grid[1:]):
+        mid = np.float32((a + b) / 2)
+        for v in (mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(1e9)), np.float32(a)):
+            pts.add(float(v))
+    pts.update(float(v) for v in rng.uniform(0, hi, n_random).astype(np.float32))
+    pts.update([0.0, float(np.float32(1e-30)), hi])
+    return sorted(pts)
+
+
+def test_e4m3_encode_matches_torch(orc):
+    # torch's float32 -> float8_e4m3fn conversion rounds to nearest even
+    pts = _adversarial_scales(448.0, 4000, 0)
+    t = torch.tensor(pts, dtype=torch.float32)
+    ref = t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([orc.scale_encode(1, p) for p in pts], np.uint8)
+    np.testing.assert_array_equal(got, ref)
+    # above the largest code the nearest value is 448 itself
+    for p in (448.5, 463.9, 464.0, 500.0, 1e30, float("inf")):
+        assert orc.scale_encode(1, p) == 0x7E
+
+
+def test_e3m3_encode(orc):
+    pts = _adversarial_scales(30.0, 4000, 1)
+    for p in pts:
+        got = orc.scale_encode(0, p)
+        if p >= 0.25:
+            # normal range: same grid as E4M3 (torch RNE), code (e-4, m)
+            c4 = int(torch.tensor([p], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+            exp = (((c4 >> 3) - 4) << 3) | (c4 & 7)
+            assert got == min(exp, 0x3F), p
+        else:
+            # subnormal range: round(32 p) with Python's half-to-even round()
+            exp = round(Fraction(p) * 32)
+            assert got == exp, p
+    for p in (30.0, 30.999, 31.0, 32.0, 1e9):
+        assert orc.scale_encode(0, p) == 0x3F
+
+
+# ----------------------------------------------------------------------------
+# element grid
+# ----------------------------------------------------------------------------
+def test_fp4_grid(orc):
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c in range(16):
+        exp = mags[c & 7] * (-1 if c & 8 else 1)
+        if c == 8:
+            assert orc.fp4_value(c, None) == 0.0
+            for v in (5.0, -5.0, 8.0, -8.0):
+                assert orc.fp4_value(c, v) == v
+        else:
+            assert orc.fp4_value(c, None) == exp
+            assert orc.fp4_value(c, 5.0) == exp
+    assert [orc.special_value(0, m) for m in range(4)] == [5.0, -5.0, 8.0, -8.0]
+    assert [orc.special_value(1, m) for m in range(2)] == [5.0, -5.0]
+    assert orc.num_specials(2) == 0
+
+
+# ----------------------------------------------------------------------------
+# 16-bit conversions, tensor scale, division
+# ----------------------------------------------------------------------------
+def test_float_to_16bit_matches_libraries(orc):
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([
+        rng.standard_normal(3000).astype(np.float32) * np.float32(100),
+        rng.standard_normal(1000).astype(np.float32) * np.float32(1e-6),
+        np.array([0.0, -0.0, 65504.0, 1e-8, 6e-5, 2688.0, 0.1], np.float32),
+    ])
+    f16_ref = vals.astype(np.float16).view(np.uint16)
+    bf_ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    for v, a, b in zip(vals, f16_ref, bf_ref):
+        assert orc.float_to_f16_bits(float(v)) == a
+        assert orc.float_to_bf16_bits(float(v)) == b
+    for h in range(0, 0x7C00, 7):
+        assert orc.f16_to_double(h) == float(np.uint16(h).view(np.float16))
+
+
+def test_tensor_scale(orc):
+    w = workloads.weight(64, 256, seed=5)
+    got = orc.tensor_scale(w.numpy(), 0)
+    amax = np.abs(w.numpy().astype(np.float32)).max()
+    assert got == np.float32(amax) / np.float32(180.0)
+    a = workloads.outlier_activations(16, 256, seed=6)
+    got = orc.tensor_scale(oracle_input(a), 1)
+    amax = a.float().abs().max().item()
+    assert got == np.float32(amax) / np.float32(2688.0)
+
+
+def test_scaled_values_match_numpy_division(orc):
+    rng = np.random.default_rng(4)
+    for _ in range(300):
+        x = (rng.standard_normal(16) * rng.uniform(0.001, 3)).astype(np.float32)
+        ts = np.float32(rng.uniform(0.0001, 0.05))
+        for fmt in (0, 1):
+            codes, sb, xs, _ = orc.quantize_block(x, float(ts), fmt)
+            sc = sb & (0x3F if fmt == 0 else 0x7F)
+            s = np.float32(orc.scale_value(fmt, sc))
+            # block scale code = nearest to amax / (6 ts) computed in fp32
+            sf = np.float32(np.abs(x).max()) / np.float32(np.float32(6) * ts)
+            assert sc == orc.scale_encode(fmt, float(sf))
+            if sc:
+                d = np.float32(s * ts)
+                np.testing.assert_array_equal(xs, x / d)
+
+
+# ----------------------------------------------------------------------------
+# brute force over all code assignments with exact rationals
+# ----------------------------------------------------------------------------
+MAGS = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3), Fraction(4), Fraction(6)]
+
+
+def _code_value(code, v):
+    if code == 8:
+        return v
+    m = MAGS[code & 7]
+    return -m if code & 8 else m
+
+
+def brute_force_block(xs, specials):
+    """Minimise the exact SSE over every (special value, code assignment);
+    ties: lowest special index, then smaller magnitude per element (then the
+    lower code, which makes 0 win over the plain -0 code).  Zero entries of
+    xs are fixed to code 0 (the only zero-error code when v != 0)."""
+    nz = [j for j in range(16) if xs[j] != 0]
+    best = None
+    metas = list(enumerate(specials)) if specials else [(0, None)]
+    for meta, v in metas:
+        vv = Fraction(v) if v is not None else Fraction(0)
+        for assign in itertools.product(range(16), repeat=len(nz)):
+            sse = Fraction(0)
+            mags = []
+            for j, c in zip(nz, assign):
+                val = _code_value(c, vv)
+                sse += (Fraction(float(xs[j])) - val) ** 2
+                mags.append((abs(val), c))
+            key = (sse, meta, mags)
+            if best is None or key < best[0]:
+                best = (key, meta, dict(zip(nz, assign)))
+    _, meta, chosen = best
+    codes = [chosen.get(j, 0) for j in range(16)]
+    return meta, codes
+
+
+ADV = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 4.5, 5.0, 5.5, 6.0, 7.0, 7.5, 8.0, 8.5, 9.0, 4.0, 3.0, 0.5]
+
+
+def _tiny_blocks(seed, count, max_nz):
+    rng = random.Random(seed)
+    out = []
+    for _ in range(count):
+        n = rng.randint(1, max_nz)
+        pos = rng.sample(range(16), n)
+        xs = [0.0] * 16
+        for p in pos:
+            kind = rng.random()
+            if kind < 0.5:
+                a = rng.choice(ADV)
+                a = float(np.float32(a))
+                if rng.random() < 0.4:
+                    a = float(np.nextafter(np.float32(a), np.float32(100 if rng.random() < 0.5 else 0)))
+            else:
+                a = float(np.float32(rng.uniform(0, 9)))
+            xs[p] = a if rng.random() < 0.5 else -a
+        out.append(xs)
+    return out
+
+
+@pytest.mark.parametrize("fmt,max_nz,count", [(0, 2, 150), (0, 3, 12), (1, 3, 40), (2, 3, 30)])
+def test_bruteforce_tiny_blocks(orc, fmt, max_nz, count):
+    specials = [orc.special_value(fmt, m) for m in range(orc.num_specials(fmt))]
+    for xs_target in _tiny_blocks(100 + fmt * 10 + max_nz, count, max_nz):
+        # realise X^scaled exactly with ts = 1/8 and a scale of 1/32 (weights:
+        # subnormal E3M3, so |xs| may reach 9) or 1/64 (E4M3 formats), by
+        # padding the block with an element that fixes the block amax
+        if fmt == 0:
+            d = Fraction(1, 32) / 8
+        else:
+            d = Fraction(1, 64) / 8
+        x = [float(Fraction(t) * d) for t in xs_target]
+        codes, sb, xs, _ = orc.quantize_block(np.array(x, np.float32), 0.125, fmt)
+        s = orc.scale_value(fmt, sb & (0x3F if fmt == 0 else 0x7F))
+        if s == 0:
+            assert all(c == 0 for c in codes)
+            continue
+        meta_bf, codes_bf = brute_force_block(xs, specials)
+        meta = (sb >> 6) if fmt == 0 else ((sb >> 7) if fmt == 1 else 0)
+        assert meta == meta_bf, (xs, meta, meta_bf)
+        assert list(codes) == codes_bf, (xs, list(codes), codes_bf)
+
+
+# ----------------------------------------------------------------------------
+# invariants on config-like tensors
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_invariants(orc, fmt):
+    if fmt == 1:
+        x = workloads.outlier_activations(64, 512, seed=11)
+        xin = oracle_input(x)
+        xf = x.float().numpy()
+    else:
+        x = workloads.weight(64, 512, seed=12)
+        xin = x.numpy()
+        xf = x.float().numpy()
+    ts = orc.tensor_scale(xin, fmt)
+    nv = orc.num_specials(fmt)
+    specials = [orc.special_value(fmt, m) for m in range(nv)]
+    max_xs = 0.0
+    for r in range(0, 64, 3):
+        for b in range(512 // 16):
+            blk = xf[r, b * 16:(b + 1) * 16]
+            codes, sb, xs, dl = orc.quantize_block(blk, ts, fmt)
+            max_xs = max(max_xs, float(np.abs(xs).max()))
+            sc = sb & (0x3F if fmt == 0 else 0x7F)
+            meta = (sb >> 6) if fmt == 0 else ((sb >> 7) if fmt == 1 else 0)
+            if fmt == 2:
+                assert 8 not in codes  # 0b1000 never appears in plain NVFP4
+                continue
+            # the chosen value never raises the squared error over plain NVFP4
+            assert dl[meta] <= 0.0
+            assert dl[meta] == min(dl[:nv])
+            a = np.abs(xs.astype(np.float64))
+            in5 = (a > 4.5) & (a <= 5.5)
+            in8 = a > 7
+            if not (in5.any() or (fmt == 0 and in8.any())):
+                assert meta == 0 and not np.any(dl[:nv])
+                assert 8 not in codes
+            # a code 0b1000 decodes to the chosen special value
+            s = orc.scale_value(fmt, sc)
+            for j in range(16):
+                if codes[j] == 8:
+                    assert orc.fp4_value(8, specials[meta]) * s == specials[meta] * s
+                    assert abs(xs[j] - specials[meta]) <= 1.0
+    # with a library-computed tensor scale X^scaled stays below 9 (+ rounding)
+    assert max_xs <= 9.0 * (1 + 2 ** -20)
+
+
+def test_gemm_ref_matches_numpy(orc):
+    w = workloads.weight(48, 256, seed=21)
+    codes, scales, ts, _ = orc.quantize(w.numpy(), 0)
+    x = workloads.vectors(5, 256, seed=22)
+    deq = orc.dequant(codes, scales, 1.0, 0, "f32").astype(np.float64)
+    ref = (x.numpy().astype(np.float64) @ deq.T) * ts
+    got = orc.gemm_ref(x.numpy(), codes, scales, ts, 0)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    sub = orc.gemm_ref(x.numpy(), codes, scales, ts, 0, rows=[4, 1])
+    np.testing.assert_array_equal(sub, got[[4, 1]])
+
+
+def test_dequant_output_types(orc):
+    w = workloads.weight(8, 64, seed=23)
+    codes, scales, ts, _ = orc.quantize(w.numpy(), 0)
+    f32 = orc.dequant(codes, scales, ts, 0, "f32")
+    f16 = orc.dequant(codes, scales, ts, 0, "f16")
+    bf = orc.dequant(codes, scales, ts, 0, "bf16")
+    np.testing.assert_array_equal(f16, f32.astype(np.float16).view(np.uint16))
+    ref_bf = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(bf, ref_bf)
+    # q*s is exact; (q*s)*ts is one binary32 rounding
+    qs = orc.dequant(codes, scales, 1.0, 0, "f32")
+    np.testing.assert_array_equal(f32, qs * np.float32(ts))
+
+
+def test_zero_and_degenerate(orc):
+    z = np.zeros((2, 32), np.float16)
+    codes, scales, ts, _ = orc.quantize(z, 0)
+    assert ts == 0.0 and not codes.any() and not scales.any()
+    # ts <= 0 given by the caller: all-zero output
+    x = workloads.outlier_activations(2, 32, seed=1)
+    codes, scales, _, _ = orc.quantize(oracle_input(x), 1, ts=0.0)
+    assert not codes.any() and not scales.any()
+    # a block of tiny values under a large tensor scale has scale code 0
+    row = np.zeros((1, 32), np.float16)
+    row[0, 0] = 1e-4
+    row[0, 16] = 60000
+    codes, scales, ts, _ = orc.quantize(row, 0)
+    assert scales[0, 0] == 0 and codes[0, :8].sum() == 0
+    with pytest.raises(ValueError):
+        orc.quantize(np.zeros((1, 24), np.float16), 0)
