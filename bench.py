@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Benchmark of the RaZeR hot path on B200.
+
+Workload (one step): the Llama-3-8B decode projections in RaZeR weight format.
+Each step quantizes the three fp16 weight matrices (4096x4096, 14336x4096,
+4096x14336; N(0, 0.02^2) with 0.1% x10 outliers) and runs the W4A16 GEMV at
+batch 1, 4 and 16 (fp16 activations N(0, 1), fp16 outputs) on each of them.
+The GEMVs of step s read the packed weights written by step s-1 (two packed
+sets alternate), so between writing and reading a packed matrix more than
+600 MB of other traffic has passed through the 126 MB L2; the fp16 inputs
+(268 MB) are larger than L2 as well.
+
+value  = algorithmic bytes of all ranks' steps / max-over-ranks device time
+         (quantizer: 2 B read for the amax pass + 2 B read + 0.5625 B written
+         per weight; GEMV: 0.5625 N K + 2 B K + 2 B N bytes per call).
+Breakdown: per-call device times (CUDA events on the launching stream), the
+activation quantizer on 2048x4096 bf16 with outlier channels, and the
+tcgen05 GEMM on the prefill shapes when the library supports it.
+
+--impl reference times the CPU oracle (single thread, as it stands) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RaZeR W4A16 GEMV HBM GB/s & GEMM TFLOP/s vs B200 roofline; quantize GB/s"
+SHAPES = [(4096, 4096), (14336, 4096), (4096, 14336)]  # (N, K) of the Llama-3-8B projections
+BATCHES = [1, 4, 16]
+WORKLOAD = "llama3-8b-decode-w4a16: quantize 3 projections + GEMV B=1,4,16 (fp16)"
+
+
+def quant_bytes(N, K):
+    return N * K * (2 + 2 + 0.5625)
+
+
+def gemv_bytes(B, N, K):
+    return 0.5625 * N * K + 2 * B * K + 2 * B * N
+
+
+def step_bytes():
+    return sum(quant_bytes(N, K) for N, K in SHAPES) + sum(gemv_bytes(B, N, K) for N, K in SHAPES for B in BATCHES)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_quantization_razer_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_hash") != source_hash():
+        return None
+    return d.get("kernels", {}).get(kernel)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = "clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    from bit_quantization_razer_b200 import workloads
+
+    oracle.build()
+    rows_per_shape = 8
+    ws = [workloads.weight(N, K, seed=100 + i) for i, (N, K) in enumerate(SHAPES)]
+    xs = {B: [workloads.vectors(B, K, seed=10 + B) for _, K in SHAPES] for B in BATCHES}
+
+    def one_step():
+        nbytes = 0.0
+        for i, (N, K) in enumerate(SHAPES):
+            w = ws[i]
+            ts = oracle.tensor_scale(w.numpy(), 0)  # full-tensor amax pass
+            sub = w[:rows_per_shape].numpy()
+            codes, scales, _, _ = oracle.quantize(sub, 0, ts=ts)
+            nbytes += N * K * 2 + rows_per_shape * K * 2.5625
+            for B in BATCHES:
+                oracle.gemm_ref(xs[B][i].numpy(), codes, scales, ts, 0)
+                nbytes += gemv_bytes(B, rows_per_shape, K)
+        return nbytes
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    tot = 0.0
+    for _ in range(args.steps):
+        tot += one_step()
+    dt = time.perf_counter() - t0
+    value = tot / dt / 1e9
+    sample = f"per step: full amax pass of each projection + quantize and GEMV (B=1,4,16) of {rows_per_shape} rows of each"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# CUDA arm
+# ---------------------------------------------------------------------------
+def cpu_baseline_sample():
+    """The oracle as it stands, single-threaded, on a bounded sample (~10 s)."""
+    import oracle
+    from bit_quantization_razer_b200 import workloads
+
+    oracle.build()
+    N, K = SHAPES[0]
+    w = workloads.weight(N, K, seed=100)
+    rows = 24
+    x = {B: workloads.vectors(B, K, seed=10 + B) for B in BATCHES}
+    t0 = time.perf_counter()
+    ts = oracle.tensor_scale(w.numpy(), 0)
+    codes, scales, _, _ = oracle.quantize(w[:rows].numpy(), 0, ts=ts)
+    nbytes = N * K * 2 + rows * K * 2.5625
+    for B in BATCHES:
+        oracle.gemm_ref(x[B].numpy(), codes, scales, ts, 0)
+        nbytes += gemv_bytes(B, rows, K)
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"amax pass of the 4096x4096 projection + quantize and GEMV (B=1,4,16) of {rows} rows ({dt:.1f} s)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="razer", choices=["razer", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the breakdown / e2e / GEMM legs")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+
+    import bit_quantization_razer_b200 as R
+    from bit_quantization_razer_b200 import workloads
+
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    R.load()
+    hbm, bf16, bf16_sus, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # inputs (host-generated, seeded), resident in HBM before timing
+    W = [workloads.weight(N, K, seed=100 + i).to(dev) for i, (N, K) in enumerate(SHAPES)]
+    X = {B: [workloads.vectors(B, K, seed=10 + B).to(dev) for _, K in SHAPES] for B in BATCHES}
+    packed = [[(torch.empty((N, K // 2), dtype=torch.uint8, device=dev), torch.empty((N, K // 16), dtype=torch.uint8, device=dev),
+                torch.empty(1, dtype=torch.float32, device=dev)) for N, K in SHAPES] for _ in range(2)]
+    Y = {B: [torch.empty((B, N), dtype=torch.float16, device=dev) for N, _ in SHAPES] for B in BATCHES}
+    wsz = max(R.razer_workspace_size(R.RAZER_OP_GEMV, B, N, K) for N, K in SHAPES for B in BATCHES)
+    ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
+
+    calls = [("quantize", i, None) for i in range(len(SHAPES))] + [("gemv", i, B) for i in range(len(SHAPES)) for B in BATCHES]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+
+    def step(s, record=False):
+        cur, prev = packed[s % 2], packed[(s + 1) % 2]
+        for ci, (kind, i, B) in enumerate(calls):
+            if record:
+                ev[ci][0].record(stream)
+            if kind == "quantize":
+                c, sc, t = cur[i]
+                R.razer_quantize_weights(W[i], "weight", codes=c, scales=sc, ts=t)
+            else:
+                c, sc, t = prev[i]
+                R.razer_gemv(X[B][i], c, sc, t, "weight", torch.float16, out=Y[B][i], workspace=ws)
+            if record:
+                ev[ci][1].record(stream)
+
+    # the first GEMVs read the second packed set: fill it
+    step(1)
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for s in range(args.steps):
+            step(s)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    elapsed_ms = t0.elapsed_time(t1)
+    if pg:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+        pg.barrier()
+    ms_per_step = elapsed_ms / args.steps
+    value = step_bytes() * args.steps * world / (elapsed_ms / 1e3) / 1e9
+
+    # per-call timing (its own loop, so the events do not perturb the step)
+    breakdown = {}
+    times = {c: [] for c in calls}
+    for s in range(max(3, min(args.steps, 10))):
+        step(s, record=True)
+        torch.cuda.synchronize()
+        for ci, c in enumerate(calls):
+            times[c].append(ev[ci][0].elapsed_time(ev[ci][1]))
+    tot_q = tot_g = 0.0
+    by_kind = {}
+    for (kind, i, B), ts_ in times.items():
+        N, K = SHAPES[i]
+        ms = statistics.median(ts_)
+        nb = quant_bytes(N, K) if kind == "quantize" else gemv_bytes(B, N, K)
+        key = f"{kind}_{N}x{K}" + ("" if B is None else f"_b{B}")
+        breakdown[key] = {"ms": ms, "GB/s": nb / ms / 1e6}
+        by_kind.setdefault(kind, [0.0, 0.0])
+        by_kind[kind][0] += ms
+        by_kind[kind][1] += nb
+    dominant = max(by_kind, key=lambda k: by_kind[k][0])
+    dom_ms, dom_bytes = by_kind[dominant]
+    n_calls = len(SHAPES) if dominant == "quantize" else len(SHAPES) * len(BATCHES)
+    achieved = dom_bytes / dom_ms / 1e6  # GB/s, average over that kind's launches
+    kname = "quantize_kernel" if dominant == "quantize" else "gemv_kernel"
+    traffic = traffic_for(kname)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": traffic, "kernel": ("razer_quantize_weights (amax + quantize kernels)" if dominant == "quantize"
+                                               else "razer_gemv (gemv + split-K reduce kernels)"),
+                "algorithmic_bytes_per_call": dom_bytes / n_calls, "peak_source": peak_src}
+
+    extras = {}
+    if not args.no_extras and rank == 0:
+        extras = run_extras(R, workloads, dev, stream, hbm, bf16)
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_extras:
+        e2e = run_e2e(R, workloads, dev, stream, args, world, pg)
+
+    launches_per_step = len(SHAPES) * 3 + len(SHAPES) * len(BATCHES) * 2
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": None, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (268 MB fp16 weights per step); packed weights double-buffered "
+                         "across steps so each GEMV reads weights written one step (600+ MB of traffic) earlier",
+                   "bytes_per_step": step_bytes()},
+        "roofline": roofline,
+        "clocks": clk.summary(),
+        "gpu_launches": launches_per_step * args.steps,
+        "breakdown": breakdown,
+    }
+    line.update(extras)
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sample()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def run_extras(R, workloads, dev, stream, hbm, bf16):
+    import torch
+
+    out = {}
+    # online activation quantizer: 2048 x 4096 bf16, 8 outlier channels x50
+    Xa = [workloads.outlier_activations(2048, 4096, seed=300 + i).to(dev) for i in range(8)]  # 8 x 16.8 MB > L2
+    codes = torch.empty((2048, 2048), dtype=torch.uint8, device=dev)
+    scales = torch.empty((2048, 256), dtype=torch.uint8, device=dev)
+    ts = torch.empty(1, dtype=torch.float32, device=dev)
+    hist = torch.empty(4, dtype=torch.int64, device=dev)
+    for i in range(3):
+        R.razer_quantize_acts(Xa[i], None, "act", codes=codes, scales=scales, ts_out=ts, meta_hist=hist)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 40
+    e0.record(stream)
+    for r in range(reps):
+        R.razer_quantize_acts(Xa[r % 8], None, "act", codes=codes, scales=scales, ts_out=ts, meta_hist=hist)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    n = 2048 * 4096
+    h = hist.cpu().tolist()
+    nblk = n // 16
+    out["act_quantize"] = {"ms": ms, "GB/s_two_pass": n * 4.5625 / ms / 1e6, "GB/s_single_pass_bytes": n * 2.5625 / ms / 1e6,
+                           "frac_two_pass": n * 4.5625 / ms / 1e6 / hbm,
+                           "meta_fraction": {"+5": h[0] / nblk, "-5": h[1] / nblk},
+                           "effective_fraction": {"+5": h[2] / nblk, "-5": h[3] / nblk}}
+    # tcgen05 GEMM on the prefill shapes
+    try:
+        Xg = workloads.vectors(4096, 4096, seed=400, dtype=torch.bfloat16).to(dev)
+        res = {}
+        for N, K in [(4096, 4096), (14336, 4096)]:
+            w = workloads.weight(N, K, seed=401).to(dev)
+            c, s, t = R.razer_quantize_weights(w)
+            Yg = torch.empty((4096, N), dtype=torch.bfloat16, device=dev)
+            for _ in range(3):
+                R.razer_gemm(Xg, c, s, t, "weight", torch.bfloat16, out=Yg)
+            reps = 20
+            e0.record(stream)
+            for _ in range(reps):
+                R.razer_gemm(Xg, c, s, t, "weight", torch.bfloat16, out=Yg)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            tf = 2 * 4096 * N * K / ms / 1e9
+            res[f"{4096}x{N}x{K}"] = {"ms": ms, "TFLOP/s": tf, "frac": tf / bf16}
+        out["gemm"] = res
+    except R.RazerError as e:
+        out["gemm"] = {"unavailable": str(e)}
+    return out
+
+
+def run_e2e(R, workloads, dev, stream, args, world, pg):
+    """Same step through the public API with host (pinned) buffers: the fp16
+    weights are copied in, quantized, the GEMVs run, the outputs come back."""
+    import torch
+
+    Wh = [workloads.weight(N, K, seed=100 + i).pin_memory() for i, (N, K) in enumerate(SHAPES)]
+    Xh = {B: [workloads.vectors(B, K, seed=10 + B).pin_memory() for _, K in SHAPES] for B in BATCHES}
+    Wd = [torch.empty_like(w, device=dev) for w in Wh]
+    Xd = {B: [torch.empty_like(x, device=dev) for x in Xh[B]] for B in BATCHES}
+    Yh = {B: [torch.empty((B, N), dtype=torch.float16).pin_memory() for N, _ in SHAPES] for B in BATCHES}
+    h2d = sum(w.numel() * 2 for w in Wh) + sum(x.numel() * 2 for B in BATCHES for x in Xh[B])
+    d2h = sum(y.numel() * 2 for B in BATCHES for y in Yh[B])
+
+    def step():
+        packed = []
+        for i in range(len(SHAPES)):
+            Wd[i].copy_(Wh[i], non_blocking=True)
+            packed.append(R.razer_quantize_weights(Wd[i]))
+        for i in range(len(SHAPES)):
+            for B in BATCHES:
+                Xd[B][i].copy_(Xh[B][i], non_blocking=True)
+                y = R.razer_gemv(Xd[B][i], *packed[i], "weight", torch.float16)
+                Yh[B][i].copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if pg:
+        tt = torch.tensor([ms], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        ms = float(tt.item())
+    return {"value": step_bytes() * steps * world / (ms / 1e3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps}
+
+
+if __name__ == "__main__":
+    main()

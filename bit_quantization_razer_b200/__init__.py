@@ -1,0 +1,12 @@
+"""RaZeR (Redundant Zero Remapping for NVFP4) hot path for NVIDIA B200 (sm_100a).
+
+The compute runs in librazer.so (CUDA kernels behind the C ABI of
+include/razer.h); this package is its thin Python binding plus the seeded
+synthetic workload generators used by the tests and the benchmark.
+"""
+from .razer import (  # noqa: F401
+    FORMATS, RAZER_BF16, RAZER_F16, RAZER_F32, RAZER_FMT_ACT, RAZER_FMT_NVFP4, RAZER_FMT_WEIGHT,
+    RAZER_OP_GEMM, RAZER_OP_GEMV, RazerError, load, razer_dequant, razer_gemm, razer_gemv,
+    razer_get_device_status, razer_quantize_acts, razer_quantize_weights, razer_status_string,
+    razer_version, razer_workspace_size,
+)

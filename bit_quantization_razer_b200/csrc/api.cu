@@ -1,0 +1,167 @@
+// extern "C" surface of the RaZeR library: argument validation, then the
+// launches of the kernels in quantize.cu / dequant.cu / gemv.cu / gemm.cu.
+// No call allocates memory or synchronises (razer_get_device_status excepted).
+#include "razer_internal.cuh"
+
+namespace razer {
+
+int sm_count()
+{
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+razer_status last_launch_status() { return cudaGetLastError() == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA; }
+
+razer_status run_quantize(const void *x, razer_dtype dt, int64_t R, int64_t K, const float *ts_in, uint8_t *codes,
+                          uint8_t *scales, float *ts_out, unsigned long long *hist, razer_format fmt, cudaStream_t st);
+razer_status run_dequant(const uint8_t *codes, const uint8_t *scales, const float *ts, razer_format fmt, int64_t R, int64_t K,
+                         void *out, razer_dtype dt, cudaStream_t st);
+razer_status run_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                      razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st);
+size_t gemv_workspace_bytes(int64_t B, int64_t N, int64_t K);
+razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                      razer_format wfmt, int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st);
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+static bool valid_fmt(int f) { return f == RAZER_FMT_WEIGHT || f == RAZER_FMT_ACT || f == RAZER_FMT_NVFP4; }
+static bool valid_dt(int d) { return d == RAZER_F16 || d == RAZER_BF16 || d == RAZER_F32; }
+static bool in16(int d) { return d == RAZER_F16 || d == RAZER_BF16; }
+
+// Shared checks of a [R, K] packed tensor.
+static razer_status check_packed(const uint8_t *codes, const uint8_t *scales, int64_t R, int64_t K)
+{
+    if (!codes || !scales) return RAZER_ERR_INVALID_ARG;
+    if (R < 0 || K < 0 || (K % 16) != 0) return RAZER_ERR_SHAPE;
+    if (!aligned(codes, 16) || !aligned(scales, 4)) return RAZER_ERR_ALIGN;
+    return RAZER_OK;
+}
+
+}  // namespace razer
+
+using namespace razer;
+
+extern "C" {
+
+razer_status razer_quantize_weights(const void *W, razer_dtype in_dt, int64_t N, int64_t K, uint8_t *codes, uint8_t *scales,
+                                    float *tensor_scale, razer_format fmt, razer_stream_t stream)
+{
+    if (!W || !tensor_scale) return RAZER_ERR_INVALID_ARG;
+    if (fmt != RAZER_FMT_WEIGHT && fmt != RAZER_FMT_NVFP4) return valid_fmt(fmt) ? RAZER_ERR_UNSUPPORTED : RAZER_ERR_INVALID_ARG;
+    if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(in_dt)) return RAZER_ERR_DTYPE;
+    razer_status st = check_packed(codes, scales, N, K);
+    if (st != RAZER_OK) return st;
+    if (!aligned(W, 16) || !aligned(tensor_scale, 4)) return RAZER_ERR_ALIGN;
+    return run_quantize(W, in_dt, N, K, nullptr, codes, scales, tensor_scale, nullptr, fmt, (cudaStream_t)stream);
+}
+
+razer_status razer_quantize_acts(const void *X, razer_dtype in_dt, int64_t M, int64_t K, const float *ts_in, uint8_t *codes,
+                                 uint8_t *scales, float *ts_out, unsigned long long *meta_hist, razer_format fmt,
+                                 razer_stream_t stream)
+{
+    if (!X || !ts_out) return RAZER_ERR_INVALID_ARG;
+    if (fmt != RAZER_FMT_ACT && fmt != RAZER_FMT_NVFP4) return valid_fmt(fmt) ? RAZER_ERR_UNSUPPORTED : RAZER_ERR_INVALID_ARG;
+    if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(in_dt)) return RAZER_ERR_DTYPE;
+    razer_status st = check_packed(codes, scales, M, K);
+    if (st != RAZER_OK) return st;
+    if (!aligned(X, 16) || !aligned(ts_out, 4) || (ts_in && !aligned(ts_in, 4)) || (meta_hist && !aligned(meta_hist, 8)))
+        return RAZER_ERR_ALIGN;
+    return run_quantize(X, in_dt, M, K, ts_in, codes, scales, ts_out, meta_hist, fmt, (cudaStream_t)stream);
+}
+
+razer_status razer_dequant(const uint8_t *codes, const uint8_t *scales, const float *ts, razer_format fmt, int64_t R, int64_t K,
+                           void *out, razer_dtype out_dt, razer_stream_t stream)
+{
+    if (!ts || !out) return RAZER_ERR_INVALID_ARG;
+    if (!valid_fmt(fmt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    razer_status st = check_packed(codes, scales, R, K);
+    if (st != RAZER_OK) return st;
+    if (!aligned(out, 16) || !aligned(ts, 4)) return RAZER_ERR_ALIGN;
+    return run_dequant(codes, scales, ts, fmt, R, K, out, out_dt, (cudaStream_t)stream);
+}
+
+size_t razer_workspace_size(razer_op op, int64_t M_or_B, int64_t N, int64_t K)
+{
+    if (op == RAZER_OP_GEMV) return gemv_workspace_bytes(M_or_B, N, K);
+    if (op == RAZER_OP_GEMM) return gemm_workspace_bytes(M_or_B, N, K);
+    return 0;
+}
+
+razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                        razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, size_t ws_bytes,
+                        razer_stream_t stream)
+{
+    if (!x || !ts || !y) return RAZER_ERR_INVALID_ARG;
+    if (!valid_fmt(wfmt) || !valid_dt(act_dt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(act_dt)) return RAZER_ERR_DTYPE;
+    razer_status st = check_packed(codes, scales, N, K);
+    if (st != RAZER_OK) return st;
+    if (B < 1 || B > 32 || K % 128 != 0 || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ts, 4)) return RAZER_ERR_ALIGN;
+    if (N == 0 || K == 0) return RAZER_OK;
+    const size_t need = gemv_workspace_bytes(B, N, K);
+    if (need) {
+        if (!workspace || ws_bytes < need) return RAZER_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
+    }
+    return run_gemv(x, act_dt, B, codes, scales, ts, wfmt, N, K, y, out_dt, workspace, (cudaStream_t)stream);
+}
+
+razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                        razer_format wfmt, int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace, size_t ws_bytes,
+                        razer_stream_t stream)
+{
+    if (!X || !ts || !Y) return RAZER_ERR_INVALID_ARG;
+    if (!valid_fmt(wfmt) || !valid_dt(act_dt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(act_dt)) return RAZER_ERR_DTYPE;
+    razer_status st = check_packed(codes, scales, N, K);
+    if (st != RAZER_OK) return st;
+    if (M < 0 || K % 64 != 0 || N % 16 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ts, 4)) return RAZER_ERR_ALIGN;
+    if (M == 0 || N == 0) return RAZER_OK;
+    const size_t need = gemm_workspace_bytes(M, N, K);
+    if (need) {
+        if (!workspace || ws_bytes < need) return RAZER_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
+    }
+    return run_gemm(X, act_dt, M, codes, scales, ts, wfmt, N, K, Y, out_dt, workspace, (cudaStream_t)stream);
+}
+
+razer_status razer_get_device_status(razer_stream_t stream)
+{
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RAZER_ERR_CUDA;
+    unsigned v = 0u, zero = 0u;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return RAZER_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return RAZER_ERR_CUDA;
+    return (razer_status)v;
+}
+
+const char *razer_status_string(razer_status s)
+{
+    switch (s) {
+    case RAZER_OK: return "ok";
+    case RAZER_ERR_INVALID_ARG: return "invalid argument";
+    case RAZER_ERR_SHAPE: return "unsupported shape";
+    case RAZER_ERR_ALIGN: return "misaligned pointer";
+    case RAZER_ERR_DTYPE: return "unsupported element type";
+    case RAZER_ERR_WORKSPACE: return "workspace too small";
+    case RAZER_ERR_UNSUPPORTED: return "unsupported request";
+    case RAZER_ERR_TIMEOUT: return "device-side wait timed out";
+    case RAZER_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+int razer_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,270 @@
+// RaZeR W4A16 GEMV / skinny GEMM (1 <= B <= 32) for sm_100a.
+//
+// y[b, n] = ts * sum_k x[b, k] * (q*s)[n, k]      (RaZeR notes 关键设计 3:
+// weight-only kernels that decode the remapped codes in registers; the
+// small-batch split-K sizing of the same section is done per launch for the
+// 148 SMs of a B200).
+//
+// Design (HBM-bound: 0.5625 byte of weights per multiply-add at B = 1):
+//   * a warp owns 16 weight rows; each step it streams a 16-row x 128-k
+//     slice of codes with one 128-bit load per thread per row (64 contiguous
+//     bytes per row, 4 lanes per row), plus the matching scale bytes;
+//   * each code byte becomes one f16x2 pair with the hardware E2M1 convert,
+//     the redundant-zero codes are turned into the block's special value by
+//     a second convert of an indicator nibble (1.0 where the code is 0b1000)
+//     folded in with one packed FMA, and the block scale is applied with a
+//     packed multiply -- q*s*2^-12 (E3M3) or q*s*2^-8 (E4M3) is exact in fp16;
+//   * the decoded pairs are already in the register layout of the A operand of
+//     the warp-level m16n8k16 tensor-core MMA, so the products accumulate in
+//     fp32 without any shared-memory round trip; the activations form the
+//     n8 operand (B <= 8 uses one MMA per k16, B <= 32 four).  The reduction
+//     order over k within each 16 columns is permuted identically on both
+//     operands, which leaves the sum unchanged;
+//   * split-K partials go to a caller-provided fp32 workspace and a second
+//     small kernel sums them, applies ts (and the 2^12 / 2^8 unbias) and
+//     converts to the output type.
+#include "razer_internal.cuh"
+
+namespace razer {
+
+constexpr int kGemvWarps = 4;
+constexpr int kGemvThreads = kGemvWarps * 32;
+
+__device__ __forceinline__ unsigned cvt_e2m1x2_f16x2(unsigned byte_in_low8)
+{
+    unsigned r;
+    asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b0; }" : "=r"(r) : "r"(byte_in_low8));
+    return r;
+}
+
+__device__ __forceinline__ unsigned hmul2u(unsigned a, unsigned b)
+{
+    unsigned r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ unsigned hfma2u(unsigned a, unsigned b, unsigned c)
+{
+    unsigned r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+// f16x2 -> bf16x2 (exact for the decoded values: at most 7 significant bits,
+// inside the bf16 range)
+__device__ __forceinline__ unsigned f16x2_to_bf16x2(unsigned h)
+{
+    unsigned r;
+    asm("{ .reg .b16 l, h, ol, oh; mov.b32 {l, h}, %1; cvt.rn.bf16.f16 ol, l; cvt.rn.bf16.f16 oh, h; mov.b32 %0, {ol, oh}; }"
+        : "=r"(r)
+        : "r"(h));
+    return r;
+}
+
+// Decode 8 codes of one block (a 32-bit word) into 4 f16x2 pairs of
+// (q * s * 2^-bias): pair b holds nibbles 2b (low half) and 2b+1.
+template <bool BF16>
+__device__ __forceinline__ void decode_word(unsigned w, unsigned s2, unsigned vs2, unsigned (&h)[4])
+{
+    const unsigned a = w & 0x77777777u;
+    const unsigned nz = (a + 0x77777777u) & 0x88888888u;  // bit 3: magnitude != 0
+    const unsigned ind = (w & ~nz & 0x88888888u) >> 2;     // nibble 2 (=1.0) where code == 0b1000
+#pragma unroll
+    for (int b = 0; b < 4; b++) {
+        const unsigned q = cvt_e2m1x2_f16x2(w >> (8 * b));
+        const unsigned i = cvt_e2m1x2_f16x2(ind >> (8 * b));
+        const unsigned r = hfma2u(i, vs2, hmul2u(q, s2));
+        h[b] = BF16 ? f16x2_to_bf16x2(r) : r;
+    }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void mma16816(float (&d)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3, unsigned b0, unsigned b1)
+{
+    if constexpr (BF16) {
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    } else {
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+}
+
+// f16 scale pair and (v * s) pair of one scale byte
+template <int FMT>
+__device__ __forceinline__ void scale_pairs(unsigned sb, unsigned &s2, unsigned &vs2)
+{
+    const unsigned s16 = scale_f16_bits<FMT>(sb);
+    s2 = s16 | (s16 << 16);
+    if constexpr (Fmt<FMT>::kSpecials > 0) {
+        const unsigned meta = sb >> Fmt<FMT>::kMetaShift;
+        const unsigned v16 = ((meta & 2u) ? 0x4800u : 0x4500u) | ((meta & 1u) << 15);  // +-5 or +-8 in fp16
+        vs2 = hmul2u(v16 | (v16 << 16), s2);
+    } else {
+        vs2 = 0u;
+    }
+}
+
+template <int FMT, bool BF16, int NB>
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__restrict__ x, int B, const uint8_t *__restrict__ codes,
+                                                            const uint8_t *__restrict__ scales, int N, int K, int S,
+                                                            float *__restrict__ ws)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int row0 = (blockIdx.x * kGemvWarps + warp) * 16;
+    if (row0 >= N) return;
+    const int s = blockIdx.y;
+    const int chunks = K >> 7;
+    const int c_begin = (int)((int64_t)s * chunks / S), c_end = (int)((int64_t)(s + 1) * chunks / S);
+    const int rA = min(row0 + g, N - 1), rB = min(row0 + g + 8, N - 1);
+    const uint8_t *pa = codes + (size_t)rA * (K >> 1) + 16 * t;
+    const uint8_t *pb = codes + (size_t)rB * (K >> 1) + 16 * t;
+    const uint8_t *sa = scales + (size_t)rA * (K >> 4) + 2 * t;
+    const uint8_t *sbp = scales + (size_t)rB * (K >> 4) + 2 * t;
+
+    float acc[NB][4];
+#pragma unroll
+    for (int j = 0; j < NB; j++) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+
+    for (int c = c_begin; c < c_end; c++) {
+        const uint4 ca = ldg_stream(pa + (size_t)c * 64);
+        const uint4 cb = ldg_stream(pb + (size_t)c * 64);
+        const unsigned sA = *reinterpret_cast<const unsigned short *>(sa + (size_t)c * 8);
+        const unsigned sB = *reinterpret_cast<const unsigned short *>(sbp + (size_t)c * 8);
+        unsigned xw[NB][16];
+#pragma unroll
+        for (int j = 0; j < NB; j++) {
+            const int n = 8 * j + g;
+            if (n < B) {
+                const uint4 *px = reinterpret_cast<const uint4 *>(x + (size_t)n * K + (size_t)c * 128 + 32 * t);
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const uint4 v = __ldg(px + q);
+                    xw[j][4 * q] = v.x;
+                    xw[j][4 * q + 1] = v.y;
+                    xw[j][4 * q + 2] = v.z;
+                    xw[j][4 * q + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 16; q++) xw[j][q] = 0u;
+            }
+        }
+        unsigned s2A[2], vsA[2], s2B[2], vsB[2];
+        scale_pairs<FMT>(sA & 0xFFu, s2A[0], vsA[0]);
+        scale_pairs<FMT>(sA >> 8, s2A[1], vsA[1]);
+        scale_pairs<FMT>(sB & 0xFFu, s2B[0], vsB[0]);
+        scale_pairs<FMT>(sB >> 8, s2B[1], vsB[1]);
+        const unsigned wa[4] = {ca.x, ca.y, ca.z, ca.w};
+        const unsigned wb[4] = {cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+        for (int m = 0; m < 4; m++) {
+            unsigned hA[4], hB[4];
+            decode_word<BF16>(wa[m], s2A[m >> 1], vsA[m >> 1], hA);
+            decode_word<BF16>(wb[m], s2B[m >> 1], vsB[m >> 1], hB);
+#pragma unroll
+            for (int j = 0; j < NB; j++) {
+                mma16816<BF16>(acc[j], hA[0], hB[0], hA[1], hB[1], xw[j][4 * m], xw[j][4 * m + 1]);
+                mma16816<BF16>(acc[j], hA[2], hB[2], hA[3], hB[3], xw[j][4 * m + 2], xw[j][4 * m + 3]);
+            }
+        }
+    }
+
+    // partials: D[g][2t..2t+1] -> rows row0+g, D[g+8][..] -> rows row0+g+8
+    float *wsb = ws + (size_t)s * B * N;
+#pragma unroll
+    for (int j = 0; j < NB; j++) {
+        const int n0 = 8 * j + 2 * t;
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const int row = row0 + g + 8 * h;
+            if (row < N) {
+                if (n0 < B) wsb[(size_t)n0 * N + row] = acc[j][2 * h];
+                if (n0 + 1 < B) wsb[(size_t)(n0 + 1) * N + row] = acc[j][2 * h + 1];
+            }
+        }
+    }
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(256) gemv_reduce_kernel(const float *__restrict__ ws, int S, int64_t BN, const float *__restrict__ ts_p,
+                                                          float unbias, TOut *__restrict__ y)
+{
+    const float scale = __fmul_rn(*ts_p, unbias);
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < BN; i += stride) {
+        float a = 0.0f;
+        for (int s = 0; s < S; s++) a += ws[(size_t)s * BN + i];
+        a = __fmul_rn(a, scale);
+        if constexpr (sizeof(TOut) == 4) y[i] = a;
+        else if constexpr (std::is_same<TOut, __half>::value) y[i] = __float2half_rn(a);
+        else y[i] = __float2bfloat16_rn(a);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Split-K sizing: enough CTAs for ~4 resident 4-warp CTAs per SM, never more
+// splits than 128-wide k chunks (each split keeps at least two chunks when K
+// allows, so the reduction stays small against the weight stream).
+// ---------------------------------------------------------------------------
+int gemv_splits(int64_t B, int64_t N, int64_t K)
+{
+    (void)B;
+    const int64_t ctas_x = ((N + 15) / 16 + kGemvWarps - 1) / kGemvWarps;
+    const int64_t chunks = K / 128;
+    const int64_t target = (int64_t)sm_count() * 4;
+    int64_t S = (target + ctas_x - 1) / ctas_x;
+    const int64_t max_s = chunks >= 4 ? chunks / 2 : (chunks > 0 ? chunks : 1);
+    if (S > max_s) S = max_s;
+    if (S < 1) S = 1;
+    return (int)S;
+}
+
+size_t gemv_workspace_bytes(int64_t B, int64_t N, int64_t K)
+{
+    if (B <= 0 || N <= 0 || K <= 0) return 0;
+    return (size_t)gemv_splits(B, N, K) * (size_t)B * (size_t)N * sizeof(float);
+}
+
+template <int FMT, bool BF16>
+static void launch_gemv_fmt(const void *x, int B, const uint8_t *codes, const uint8_t *scales, int N, int K, int S, float *ws,
+                            cudaStream_t st)
+{
+    dim3 grid((unsigned)(((N + 15) / 16 + kGemvWarps - 1) / kGemvWarps), (unsigned)S);
+    const uint16_t *xp = reinterpret_cast<const uint16_t *>(x);
+    if (B <= 8) gemv_kernel<FMT, BF16, 1><<<grid, kGemvThreads, 0, st>>>(xp, B, codes, scales, N, K, S, ws);
+    else if (B <= 16) gemv_kernel<FMT, BF16, 2><<<grid, kGemvThreads, 0, st>>>(xp, B, codes, scales, N, K, S, ws);
+    else gemv_kernel<FMT, BF16, 4><<<grid, kGemvThreads, 0, st>>>(xp, B, codes, scales, N, K, S, ws);
+}
+
+razer_status run_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                      razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st)
+{
+    const int S = gemv_splits(B, N, K);
+    float *ws = reinterpret_cast<float *>(workspace);
+    const bool bf = act_dt == RAZER_BF16;
+    if (wfmt == RAZER_FMT_WEIGHT) {
+        if (bf) launch_gemv_fmt<RAZER_FMT_WEIGHT, true>(x, (int)B, codes, scales, (int)N, (int)K, S, ws, st);
+        else launch_gemv_fmt<RAZER_FMT_WEIGHT, false>(x, (int)B, codes, scales, (int)N, (int)K, S, ws, st);
+    } else if (wfmt == RAZER_FMT_ACT) {
+        if (bf) launch_gemv_fmt<RAZER_FMT_ACT, true>(x, (int)B, codes, scales, (int)N, (int)K, S, ws, st);
+        else launch_gemv_fmt<RAZER_FMT_ACT, false>(x, (int)B, codes, scales, (int)N, (int)K, S, ws, st);
+    } else {
+        if (bf) launch_gemv_fmt<RAZER_FMT_NVFP4, true>(x, (int)B, codes, scales, (int)N, (int)K, S, ws, st);
+        else launch_gemv_fmt<RAZER_FMT_NVFP4, false>(x, (int)B, codes, scales, (int)N, (int)K, S, ws, st);
+    }
+    const float unbias = wfmt == RAZER_FMT_WEIGHT ? scale_f16_unbias<RAZER_FMT_WEIGHT>() : scale_f16_unbias<RAZER_FMT_ACT>();
+    const int64_t BN = B * N;
+    int64_t g = (BN + 255) / 256;
+    if (g > (int64_t)sm_count() * 8) g = (int64_t)sm_count() * 8;
+    if (g < 1) g = 1;
+    if (out_dt == RAZER_F32) gemv_reduce_kernel<float><<<(int)g, 256, 0, st>>>(ws, S, BN, ts, unbias, reinterpret_cast<float *>(y));
+    else if (out_dt == RAZER_F16) gemv_reduce_kernel<__half><<<(int)g, 256, 0, st>>>(ws, S, BN, ts, unbias, reinterpret_cast<__half *>(y));
+    else gemv_reduce_kernel<__nv_bfloat16><<<(int)g, 256, 0, st>>>(ws, S, BN, ts, unbias, reinterpret_cast<__nv_bfloat16 *>(y));
+    return last_launch_status();
+}
+
+}  // namespace razer

@@ -1,0 +1,9 @@
+// Single translation unit of librazer.so (keeps the device status word and
+// every kernel in one module without relocatable device code).
+#include <type_traits>
+
+#include "api.cu"
+#include "quantize.cu"
+#include "dequant.cu"
+#include "gemv.cu"
+#include "gemm.cu"

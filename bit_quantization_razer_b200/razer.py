@@ -1,0 +1,178 @@
+"""ctypes binding of librazer.so (declared in include/razer.h).
+
+Argument marshalling only: every step of the RaZeR path runs in the CUDA
+kernels of the library.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or a call fails,
+an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librazer.so")
+
+# enums of include/razer.h
+RAZER_OK = 0
+STATUS_NAMES = {
+    0: "RAZER_OK", 1: "RAZER_ERR_INVALID_ARG", 2: "RAZER_ERR_SHAPE", 3: "RAZER_ERR_ALIGN",
+    4: "RAZER_ERR_DTYPE", 5: "RAZER_ERR_WORKSPACE", 6: "RAZER_ERR_UNSUPPORTED",
+    7: "RAZER_ERR_TIMEOUT", 8: "RAZER_ERR_CUDA",
+}
+RAZER_F16, RAZER_BF16, RAZER_F32 = 0, 1, 2
+RAZER_FMT_WEIGHT, RAZER_FMT_ACT, RAZER_FMT_NVFP4 = 0, 1, 2
+RAZER_OP_GEMV, RAZER_OP_GEMM = 0, 1
+FORMATS = {"weight": RAZER_FMT_WEIGHT, "act": RAZER_FMT_ACT, "nvfp4": RAZER_FMT_NVFP4}
+_DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZER_F32}
+
+EXPORTED = (
+    "razer_quantize_weights", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
+)
+
+
+class RazerError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load librazer.so (built in-tree by bit_quantization_razer_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: run `python -m bit_quantization_razer_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    L.razer_quantize_weights.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp]
+    L.razer_quantize_acts.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, vp, i32, vp]
+    L.razer_dequant.argtypes = [vp, vp, vp, i32, i64, i64, vp, i32, vp]
+    L.razer_gemv.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
+    L.razer_gemm.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
+    L.razer_workspace_size.argtypes = [i32, i64, i64, i64]
+    L.razer_workspace_size.restype = sz
+    L.razer_get_device_status.argtypes = [vp]
+    L.razer_status_string.argtypes = [i32]
+    L.razer_status_string.restype = ctypes.c_char_p
+    L.razer_version.argtypes = []
+    for fn in ("razer_quantize_weights", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+               "razer_get_device_status", "razer_version"):
+        getattr(L, fn).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _p(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != RAZER_OK:
+        raise RazerError(fn, status)
+
+
+def _fmt(fmt) -> int:
+    return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def razer_quantize_weights(W: torch.Tensor, fmt="weight", *, codes=None, scales=None, ts=None, stream=None):
+    """Quantize W [N, K] (fp16/bf16, CUDA). Returns (codes [N, K/2] u8,
+    scales [N, K/16] u8, ts [1] f32), all on W's device."""
+    N, K = W.shape
+    dev = W.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    scales = torch.empty((N, K // 16), dtype=torch.uint8, device=dev) if scales is None else scales
+    ts = torch.empty(1, dtype=torch.float32, device=dev) if ts is None else ts
+    st = load().razer_quantize_weights(_p(W), _DT.get(W.dtype, -1), N, K, _p(codes), _p(scales), _p(ts), _fmt(fmt), _stream(stream))
+    _check("razer_quantize_weights", st)
+    return codes, scales, ts
+
+
+def razer_quantize_acts(X: torch.Tensor, ts_in: torch.Tensor | None = None, fmt="act", *, hist: bool = True,
+                        codes=None, scales=None, ts_out=None, meta_hist=None, stream=None):
+    """Quantize activations X [M, K]. ts_in (device f32 [1]) = static scale,
+    None = dynamic. Returns (codes, scales, ts_out, meta_hist [4] i64 or None)."""
+    M, K = X.shape
+    dev = X.device
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    scales = torch.empty((M, K // 16), dtype=torch.uint8, device=dev) if scales is None else scales
+    ts_out = torch.empty(1, dtype=torch.float32, device=dev) if ts_out is None else ts_out
+    if hist and meta_hist is None:
+        meta_hist = torch.empty(4, dtype=torch.int64, device=dev)
+    st = load().razer_quantize_acts(_p(X), _DT.get(X.dtype, -1), M, K, _p(ts_in), _p(codes), _p(scales), _p(ts_out),
+                                    _p(meta_hist) if hist else None, _fmt(fmt), _stream(stream))
+    _check("razer_quantize_acts", st)
+    return codes, scales, ts_out, (meta_hist if hist else None)
+
+
+def razer_dequant(codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight",
+                  out_dtype=torch.float32, *, out=None, stream=None):
+    R, K2 = codes.shape
+    K = 2 * K2
+    out = torch.empty((R, K), dtype=out_dtype, device=codes.device) if out is None else out
+    st = load().razer_dequant(_p(codes), _p(scales), _p(ts), _fmt(fmt), R, K, _p(out), _DT.get(out.dtype, -1), _stream(stream))
+    _check("razer_dequant", st)
+    return out
+
+
+def razer_workspace_size(op: int, m_or_b: int, N: int, K: int) -> int:
+    return int(load().razer_workspace_size(op, m_or_b, N, K))
+
+
+def _workspace(op, m, N, K, dev, workspace):
+    need = razer_workspace_size(op, m, N, K)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    return workspace, (workspace.numel() * workspace.element_size() if workspace is not None else 0)
+
+
+def razer_gemv(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight",
+               out_dtype=torch.float32, *, out=None, workspace=None, stream=None):
+    """y [B, N] = ts * x [B, K] . deq(W [N, K])^T with 1 <= B <= 32."""
+    B, K = x.shape
+    N = codes.shape[0]
+    out = torch.empty((B, N), dtype=out_dtype, device=x.device) if out is None else out
+    workspace, wsb = _workspace(RAZER_OP_GEMV, B, N, K, x.device, workspace)
+    st = load().razer_gemv(_p(x), _DT.get(x.dtype, -1), B, _p(codes), _p(scales), _p(ts), _fmt(fmt), N, K, _p(out),
+                           _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
+    _check("razer_gemv", st)
+    return out
+
+
+def razer_gemm(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight",
+               out_dtype=torch.bfloat16, *, out=None, workspace=None, stream=None):
+    """Y [M, N] = ts * X [M, K] . deq(W [N, K])^T on the tcgen05 tensor cores."""
+    M, K = X.shape
+    N = codes.shape[0]
+    out = torch.empty((M, N), dtype=out_dtype, device=X.device) if out is None else out
+    workspace, wsb = _workspace(RAZER_OP_GEMM, M, N, K, X.device, workspace)
+    st = load().razer_gemm(_p(X), _DT.get(X.dtype, -1), M, _p(codes), _p(scales), _p(ts), _fmt(fmt), N, K, _p(out),
+                           _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
+    _check("razer_gemm", st)
+    return out
+
+
+def razer_get_device_status(stream=None) -> int:
+    """Synchronises the stream; returns and clears the device error word."""
+    return int(load().razer_get_device_status(_stream(stream)))
+
+
+def razer_status_string(status: int) -> str:
+    return load().razer_status_string(status).decode()
+
+
+def razer_version() -> int:
+    return int(load().razer_version())

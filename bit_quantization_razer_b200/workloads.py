@@ -62,3 +62,22 @@ def to_numpy_bits(t: torch.Tensor) -> np.ndarray:
     """Raw 16-bit payload of an fp16/bf16 CPU tensor as a uint16 array."""
     assert t.dtype in (torch.float16, torch.bfloat16)
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def random_packed(N: int, K: int, fmt: str, *, seed: int = 3, max_scale_code: int | None = None):
+    """Random packed weights [N, K] in a RaZeR format: uniform code bytes and
+    uniform scale bytes over every valid magnitude code and meta value (a
+    synthetic stand-in that exercises every decode path, including 0b1000
+    under each special value).  Returns (codes [N, K/2] u8, scales [N, K/16]
+    u8) as CPU tensors."""
+    g = _gen(seed)
+    codes = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.int32).to(torch.uint8)
+    if fmt == "weight":
+        mag = torch.randint(0, 64 if max_scale_code is None else max_scale_code + 1, (N, K // 16), generator=g, dtype=torch.int32)
+        meta = torch.randint(0, 4, (N, K // 16), generator=g, dtype=torch.int32)
+        scales = (mag | (meta << 6)).to(torch.uint8)
+    else:
+        mag = torch.randint(0, 127 if max_scale_code is None else max_scale_code + 1, (N, K // 16), generator=g, dtype=torch.int32)
+        meta = torch.randint(0, 2, (N, K // 16), generator=g, dtype=torch.int32) if fmt == "act" else torch.zeros_like(mag)
+        scales = (mag | (meta << 7)).to(torch.uint8)
+    return codes, scales

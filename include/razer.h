@@ -1,0 +1,182 @@
+/*
+ * razer.h -- C ABI of the B200 (sm_100a) RaZeR hot path.
+ *
+ * RaZeR ("RaZeR: Pushing the Limits of NVFP4 Quantization with Redundant Zero
+ * Remapping") keeps the NVFP4 layout -- 16-element blocks of FP4-E2M1 codes,
+ * one FP8 block scale per block and one FP32 tensor scale -- and reuses two
+ * redundancies: the FP4 code 0b1000 (-0) decodes to a per-block special value
+ * v, and spare bits of the block-scale byte select v.
+ *
+ * Formats (razer_format):
+ *   RAZER_FMT_WEIGHT  scale byte = meta[7:6] | E3M3[5:0] (bias 3, subnormals,
+ *                     max 30); meta 0..3 selects v in {+5, -5, +8, -8}.
+ *                     (RaZeR notes, 关键设计 1: weight scales narrowed to
+ *                     E3M3 free 2 bits; 训练策略: V_w = {+-5, +-8}.)
+ *   RAZER_FMT_ACT     scale byte = meta[7] | E4M3[6:0] (OCP E4M3, max 448);
+ *                     meta 0..1 selects v in {+5, -5}.  (关键设计 1: the
+ *                     activation scale keeps E4M3 and frees its sign bit.)
+ *   RAZER_FMT_NVFP4   scale byte = E4M3[6:0], no remap: 0b1000 means 0.
+ *                     Plain NVFP4, kept as an ablation of the remap.
+ *
+ * Layout (all row-major, blocks along K; K must be a multiple of 16):
+ *   codes  [R, K/2]  uint8, element 2i in the low nibble of byte i
+ *   scales [R, K/16] uint8
+ *   ts     one float in DEVICE memory (the FP32 tensor scale)
+ *   A weight matrix is W [N, K] (output features x input features); the
+ *   products are y = W x per vector, Y = X W^T for matrices.
+ *
+ * Quantizer semantics (关键设计 2; gist.science summary 2.2): with
+ *   ts   = amax(|X|) / (6 * S_max)            (S_max = 30 or 448; fp32)
+ *   s    = nearest scale code to amax_b / (6*ts) (ties to the even code,
+ *          saturating), decoded exactly
+ *   xs   = x / (s * ts)                         (IEEE fp32, nearest-even)
+ * each block picks v* = argmin_{v in V} || round(xs, Q_FP4 u {v}) - xs ||^2
+ * (rounding to the nearest point, ties to the smaller magnitude; the squared
+ * errors are compared exactly; ties go to the lowest meta index) and stores
+ * the codes of round(xs, Q_FP4 u {v*}); every element that rounds to 0 is
+ * coded 0b0000.  A block with scale code 0 (or ts <= 0) is all zeros.
+ * Codes, scale bytes and meta bits are bit-exact against this definition.
+ *
+ * Conventions for every call:
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     keeps none of them after the call returns and allocates nothing.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
+ *     never synchronise; they keep no global state and are thread-safe.
+ *   - Argument errors are reported synchronously through the return value
+ *     and nothing is launched.  A failed launch returns RAZER_ERR_CUDA.
+ *   - Input, code, output and workspace pointers must be 16-byte aligned;
+ *     scale pointers 4-byte aligned; a null pointer where one is required
+ *     gives RAZER_ERR_INVALID_ARG; sizes that are negative, K % 16 != 0, or
+ *     beyond a call's stated range give RAZER_ERR_SHAPE.
+ */
+#ifndef RAZER_H
+#define RAZER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *razer_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    RAZER_OK = 0,
+    RAZER_ERR_INVALID_ARG = 1, /* null pointer, unknown enum value            */
+    RAZER_ERR_SHAPE = 2,       /* negative size, K % 16 != 0, out of range      */
+    RAZER_ERR_ALIGN = 3,       /* pointer alignment below the stated minimum    */
+    RAZER_ERR_DTYPE = 4,       /* unsupported element type for this call        */
+    RAZER_ERR_WORKSPACE = 5,   /* workspace smaller than razer_workspace_size() */
+    RAZER_ERR_UNSUPPORTED = 6, /* valid request this build does not implement   */
+    RAZER_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up            */
+    RAZER_ERR_CUDA = 8         /* CUDA launch / runtime error                   */
+} razer_status;
+
+typedef enum { RAZER_F16 = 0, RAZER_BF16 = 1, RAZER_F32 = 2 } razer_dtype;
+
+typedef enum { RAZER_FMT_WEIGHT = 0, RAZER_FMT_ACT = 1, RAZER_FMT_NVFP4 = 2 } razer_format;
+
+typedef enum { RAZER_OP_GEMV = 0, RAZER_OP_GEMM = 1 } razer_op;
+
+/*
+ * razer_quantize_weights -- offline weight quantizer (RaZeR notes, 关键设计
+ * 1-2: E3M3 block scale, 2 meta bits, per-block argmin over V_w).
+ *   W             [N, K] input, in_dt = RAZER_F16 or RAZER_BF16
+ *   codes         [N, K/2] output
+ *   scales        [N, K/16] output
+ *   tensor_scale  device float, output: ts = amax(|W|) / (6 * S_max); it is
+ *                 also used as scratch for the amax during the call
+ *   fmt           RAZER_FMT_WEIGHT, or RAZER_FMT_NVFP4 for the ablation
+ * N >= 0, K >= 0 (an empty tensor writes ts = 0 and nothing else).
+ */
+razer_status razer_quantize_weights(const void *W, razer_dtype in_dt, int64_t N, int64_t K,
+                                    uint8_t *codes, uint8_t *scales, float *tensor_scale,
+                                    razer_format fmt, razer_stream_t stream);
+
+/*
+ * razer_quantize_acts -- online activation quantizer (关键设计 1-2; the
+ * "double quantization" of 训练策略 / gist.science 2.2: each block is
+ * quantized once per candidate in V_a = {+5, -5} and the smaller error wins).
+ *   X          [M, K] input, in_dt = RAZER_F16 or RAZER_BF16
+ *   ts_in      device float or NULL.  Given: the tensor scale to use (static
+ *              scaling).  NULL: ts is computed from amax(|X|) (dynamic).
+ *   codes      [M, K/2] output;  scales [M, K/16] output
+ *   ts_out     device float, output: the tensor scale used (may equal ts_in)
+ *   meta_hist  device unsigned long long[4] or NULL.  Overwritten with
+ *              [blocks choosing meta 0, blocks choosing meta 1, blocks where
+ *              meta 0 strictly lowered the squared error, same for meta 1].
+ *   fmt        RAZER_FMT_ACT, or RAZER_FMT_NVFP4 for the ablation
+ */
+razer_status razer_quantize_acts(const void *X, razer_dtype in_dt, int64_t M, int64_t K,
+                                 const float *ts_in, uint8_t *codes, uint8_t *scales, float *ts_out,
+                                 unsigned long long *meta_hist, razer_format fmt,
+                                 razer_stream_t stream);
+
+/*
+ * razer_dequant -- decoder (关键设计 3: the special value replaces -0):
+ *   out[r, k] = round_out( (q * s) * ts ),
+ * q*s exact, one fp32 multiply by *ts, one rounding to out_dt (f16 / bf16 /
+ * f32).  Bit-exact.  out is [R, K].
+ */
+razer_status razer_dequant(const uint8_t *codes, const uint8_t *scales, const float *ts,
+                           razer_format fmt, int64_t R, int64_t K, void *out, razer_dtype out_dt,
+                           razer_stream_t stream);
+
+/*
+ * razer_gemv -- W4A16 small-batch product (关键设计 3: weight-only kernels
+ * that decode the remapped codes on the fly):
+ *   y[b, n] = ts * sum_k x[b, k] * (q*s)[n, k],   1 <= B <= 32,
+ * with fp32 accumulation.
+ *   x          [B, K] activations, act_dt = RAZER_F16 or RAZER_BF16
+ *   codes/scales/ts  a weight tensor [N, K] in format wfmt
+ *   y          [B, N] output, out_dt = RAZER_F16, RAZER_BF16 or RAZER_F32
+ *   workspace  device scratch of at least
+ *              razer_workspace_size(RAZER_OP_GEMV, B, N, K) bytes (16-byte
+ *              aligned), or NULL when that size is 0.  Contents on entry are
+ *              ignored.
+ * K must be a multiple of 128 (one 16-byte code chunk per 32 elements, four
+ * chunks per row slice).
+ */
+razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes,
+                        const uint8_t *scales, const float *ts, razer_format wfmt, int64_t N,
+                        int64_t K, void *y, razer_dtype out_dt, void *workspace, size_t ws_bytes,
+                        razer_stream_t stream);
+
+/*
+ * razer_gemm -- W4A16 large-M product on the tcgen05 tensor cores:
+ *   Y[m, n] = ts * sum_k X[m, k] * (q*s)[n, k],   fp32 accumulation.
+ *   X   [M, K] activations, act_dt = RAZER_BF16 or RAZER_F16; the decoded
+ *       weights use the same 16-bit type (q*s is exact in both).
+ *   Y   [M, N] output, out_dt = RAZER_BF16, RAZER_F16 or RAZER_F32
+ *   workspace  as for razer_gemv (size from razer_workspace_size(RAZER_OP_GEMM, M, N, K))
+ * K must be a multiple of 64 and N a multiple of 16.
+ */
+razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes,
+                        const uint8_t *scales, const float *ts, razer_format wfmt, int64_t N,
+                        int64_t K, void *Y, razer_dtype out_dt, void *workspace, size_t ws_bytes,
+                        razer_stream_t stream);
+
+/* Bytes of workspace razer_gemv / razer_gemm need for these sizes (0 when
+ * none); M_or_B is B for RAZER_OP_GEMV and M for RAZER_OP_GEMM. */
+size_t razer_workspace_size(razer_op op, int64_t M_or_B, int64_t N, int64_t K);
+
+/*
+ * razer_get_device_status -- the device-side error word of the current
+ * device: RAZER_OK, or RAZER_ERR_TIMEOUT when a bounded wait inside a kernel
+ * (pipeline barrier of razer_gemm) gave up.  Synchronises `stream`, then
+ * reads and clears the word.
+ */
+razer_status razer_get_device_status(razer_stream_t stream);
+
+/* Static description of a status code. */
+const char *razer_status_string(razer_status status);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+int razer_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RAZER_H */

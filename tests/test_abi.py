@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+include/razer.h declares, and rejects bad arguments before launching anything
+(no compute calls: these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantization_razer_b200 import razer
+from bit_quantization_razer_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return razer.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "razer.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(razer_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "razer_gemv" in names and "razer_quantize_weights" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    for n in razer.EXPORTED:
+        assert n in names
+
+
+def test_status_strings(lib):
+    for s in range(9):
+        assert razer.razer_status_string(s)
+    assert razer.razer_status_string(3) == "misaligned pointer"
+    assert razer.razer_version() >= 100
+
+
+FAKE = ctypes.c_void_p(0x1000)  # 16-byte aligned; never dereferenced (validation fails first)
+ODD = ctypes.c_void_p(0x1001)
+
+
+def test_quantize_validation(lib):
+    q = lib.razer_quantize_weights
+    assert q(None, 0, 4, 32, FAKE, FAKE, FAKE, 0, None) == 1
+    assert q(FAKE, 0, 4, 32, FAKE, FAKE, FAKE, 1, None) == 6       # ACT format is for activations
+    assert q(FAKE, 0, 4, 32, FAKE, FAKE, FAKE, 7, None) == 1       # unknown format
+    assert q(FAKE, 2, 4, 32, FAKE, FAKE, FAKE, 0, None) == 4       # fp32 input not supported
+    assert q(FAKE, 0, 4, 24, FAKE, FAKE, FAKE, 0, None) == 2       # K % 16
+    assert q(FAKE, 0, -1, 32, FAKE, FAKE, FAKE, 0, None) == 2
+    assert q(ODD, 0, 4, 32, FAKE, FAKE, FAKE, 0, None) == 3
+    assert q(FAKE, 0, 4, 32, ODD, FAKE, FAKE, 0, None) == 3
+    a = lib.razer_quantize_acts
+    assert a(FAKE, 1, 4, 32, None, FAKE, FAKE, None, None, 1, None) == 1
+    assert a(FAKE, 1, 4, 32, None, FAKE, FAKE, FAKE, None, 0, None) == 6
+    assert a(FAKE, 1, 4, 32, ODD, FAKE, FAKE, FAKE, None, 1, None) == 3
+
+
+def test_gemv_gemm_validation(lib):
+    g = lib.razer_gemv
+    args = lambda B, N, K, ws=None, wsb=0: (FAKE, 0, B, FAKE, FAKE, FAKE, 0, N, K, FAKE, 2, ws, wsb, None)
+    assert g(*args(0, 64, 128)) == 2
+    assert g(*args(33, 64, 128)) == 2
+    assert g(*args(1, 64, 96)) == 2          # K % 128
+    assert g(*args(1, 64, 128)) == 5         # workspace missing
+    assert g(FAKE, 2, 1, FAKE, FAKE, FAKE, 0, 64, 128, FAKE, 2, None, 0, None) == 4
+    m = lib.razer_gemm
+    assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 64, 96, FAKE, 1, None, 0, None) == 2   # K % 64
+    assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 40, 128, FAKE, 1, None, 0, None) == 2  # N % 16
+    assert m(None, 1, 64, FAKE, FAKE, FAKE, 0, 64, 128, FAKE, 1, None, 0, None) == 1
+    d = lib.razer_dequant
+    assert d(FAKE, FAKE, FAKE, 3, 4, 32, FAKE, 2, None) == 1
+    assert d(FAKE, FAKE, FAKE, 0, 4, 32, FAKE, 5, None) == 1
+    assert d(FAKE, FAKE, FAKE, 0, 4, 32, ODD, 2, None) == 3
+
+
+def test_workspace_size_host_logic(lib):
+    assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, 0, 64, 128) == 0
+    n = razer.razer_workspace_size(razer.RAZER_OP_GEMV, 4, 4096, 4096)
+    assert n > 0 and n % (4 * 4096 * 4) == 0
