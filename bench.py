@@ -194,20 +194,21 @@ def cpu_baseline_sample():
     from bit_quantization_razer_b200 import workloads
 
     oracle.build()
-    N, K = SHAPES[0]
-    w = workloads.weight(N, K, seed=100)
-    rows = 24
-    x = {B: workloads.vectors(B, K, seed=10 + B) for B in BATCHES}
+    ws = [workloads.weight(N, K, seed=100 + i) for i, (N, K) in enumerate(SHAPES)]
+    x = {B: [workloads.vectors(B, K, seed=10 + B) for _, K in SHAPES] for B in BATCHES}
+    rows = 64
     t0 = time.perf_counter()
-    ts = oracle.tensor_scale(w.numpy(), 0)
-    codes, scales, _, _ = oracle.quantize(w[:rows].numpy(), 0, ts=ts)
-    nbytes = N * K * 2 + rows * K * 2.5625
-    for B in BATCHES:
-        oracle.gemm_ref(x[B].numpy(), codes, scales, ts, 0)
-        nbytes += gemv_bytes(B, rows, K)
+    nbytes = 0.0
+    for i, (N, K) in enumerate(SHAPES):
+        ts = oracle.tensor_scale(ws[i].numpy(), 0)
+        codes, scales, _, _ = oracle.quantize(ws[i][:rows].numpy(), 0, ts=ts)
+        nbytes += N * K * 2 + rows * K * 2.5625
+        for B in BATCHES:
+            oracle.gemm_ref(x[B][i].numpy(), codes, scales, ts, 0)
+            nbytes += gemv_bytes(B, rows, K)
     dt = time.perf_counter() - t0
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"amax pass of the 4096x4096 projection + quantize and GEMV (B=1,4,16) of {rows} rows ({dt:.1f} s)"}
+            "sample": f"per projection: full amax pass + quantize and GEMV (B=1,4,16) of {rows} rows ({dt:.1f} s)"}
 
 
 def main():
@@ -218,6 +219,12 @@ def main():
     ap.add_argument("--impl", default="razer", choices=["razer", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the breakdown / e2e / GEMM legs")
+    ap.add_argument("--no-soak", action="store_true", help="skip the 1.5 s pre-timing load for the clock sampler")
+    ap.add_argument("--kernel", choices=["quantize", "act_quantize", "dequant", "gemv", "gemm"],
+                    help="profiling mode: run one call on --shape in a loop (for ncu)")
+    ap.add_argument("--shape", default="4096,4096", help="N,K (gemm: M,N,K)")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -226,6 +233,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.kernel:
+        run_single_kernel(args)
         return
 
     import torch
@@ -283,6 +293,19 @@ def main():
         pg.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        # keep the same load running ~1.5 s first: nvidia-smi needs time to
+        # start and the timed region itself lasts only milliseconds
+        t_end = time.time() + (0.0 if args.no_soak else 1.5)
+        s = 0
+        while time.time() < t_end:
+            step(s)
+            s += 1
+            if s % 8 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -362,6 +385,64 @@ def main():
     if pg:
         pg.barrier()
         pg.destroy_process_group()
+
+
+def run_single_kernel(args):
+    """One API call on one shape, 3 warm-up + --iters timed calls (ncu target)."""
+    import torch
+
+    import bit_quantization_razer_b200 as R
+    from bit_quantization_razer_b200 import workloads
+
+    dev = torch.device("cuda", 0)
+    dims = [int(v) for v in args.shape.split(",")]
+    if args.kernel in ("quantize", "dequant", "gemv"):
+        N, K = dims
+        w = workloads.weight(N, K, seed=1).to(dev)
+        c, s, t = R.razer_quantize_weights(w)
+        x = workloads.vectors(args.batch, K, seed=2).to(dev)
+        y = torch.empty((args.batch, N), dtype=torch.float16, device=dev)
+        out = torch.empty((N, K), dtype=torch.float16, device=dev)
+        wsb = R.razer_workspace_size(R.RAZER_OP_GEMV, args.batch, N, K)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+
+        def call():
+            if args.kernel == "quantize":
+                R.razer_quantize_weights(w, codes=c, scales=s, ts=t)
+            elif args.kernel == "dequant":
+                R.razer_dequant(c, s, t, "weight", torch.float16, out=out)
+            else:
+                R.razer_gemv(x, c, s, t, "weight", torch.float16, out=y, workspace=ws)
+    elif args.kernel == "act_quantize":
+        M, K = dims
+        xa = workloads.outlier_activations(M, K, seed=3).to(dev)
+        c = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        s = torch.empty((M, K // 16), dtype=torch.uint8, device=dev)
+        t = torch.empty(1, dtype=torch.float32, device=dev)
+        h = torch.empty(4, dtype=torch.int64, device=dev)
+
+        def call():
+            R.razer_quantize_acts(xa, None, "act", codes=c, scales=s, ts_out=t, meta_hist=h)
+    else:
+        M, N, K = dims
+        w = workloads.weight(N, K, seed=1).to(dev)
+        c, s, t = R.razer_quantize_weights(w)
+        X = workloads.vectors(M, K, seed=4, dtype=torch.bfloat16).to(dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+        def call():
+            R.razer_gemm(X, c, s, t, "weight", torch.bfloat16, out=Y)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.iters):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel": args.kernel, "shape": dims, "batch": args.batch,
+                      "ms_per_call": e0.elapsed_time(e1) / args.iters}), flush=True)
 
 
 def run_extras(R, workloads, dev, stream, hbm, bf16):

@@ -39,8 +39,9 @@ static bool in16(int d) { return d == RAZER_F16 || d == RAZER_BF16; }
 // Shared checks of a [R, K] packed tensor.
 static razer_status check_packed(const uint8_t *codes, const uint8_t *scales, int64_t R, int64_t K)
 {
-    if (!codes || !scales) return RAZER_ERR_INVALID_ARG;
     if (R < 0 || K < 0 || (K % 16) != 0) return RAZER_ERR_SHAPE;
+    if (R * K == 0) return RAZER_OK;  // empty: pointers may be null
+    if (!codes || !scales) return RAZER_ERR_INVALID_ARG;
     if (!aligned(codes, 16) || !aligned(scales, 4)) return RAZER_ERR_ALIGN;
     return RAZER_OK;
 }
@@ -54,7 +55,7 @@ extern "C" {
 razer_status razer_quantize_weights(const void *W, razer_dtype in_dt, int64_t N, int64_t K, uint8_t *codes, uint8_t *scales,
                                     float *tensor_scale, razer_format fmt, razer_stream_t stream)
 {
-    if (!W || !tensor_scale) return RAZER_ERR_INVALID_ARG;
+    if (!tensor_scale || (!W && N * K > 0)) return RAZER_ERR_INVALID_ARG;
     if (fmt != RAZER_FMT_WEIGHT && fmt != RAZER_FMT_NVFP4) return valid_fmt(fmt) ? RAZER_ERR_UNSUPPORTED : RAZER_ERR_INVALID_ARG;
     if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
     if (!in16(in_dt)) return RAZER_ERR_DTYPE;
@@ -68,7 +69,7 @@ razer_status razer_quantize_acts(const void *X, razer_dtype in_dt, int64_t M, in
                                  uint8_t *scales, float *ts_out, unsigned long long *meta_hist, razer_format fmt,
                                  razer_stream_t stream)
 {
-    if (!X || !ts_out) return RAZER_ERR_INVALID_ARG;
+    if (!ts_out || (!X && M * K > 0)) return RAZER_ERR_INVALID_ARG;
     if (fmt != RAZER_FMT_ACT && fmt != RAZER_FMT_NVFP4) return valid_fmt(fmt) ? RAZER_ERR_UNSUPPORTED : RAZER_ERR_INVALID_ARG;
     if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
     if (!in16(in_dt)) return RAZER_ERR_DTYPE;
@@ -82,7 +83,7 @@ razer_status razer_quantize_acts(const void *X, razer_dtype in_dt, int64_t M, in
 razer_status razer_dequant(const uint8_t *codes, const uint8_t *scales, const float *ts, razer_format fmt, int64_t R, int64_t K,
                            void *out, razer_dtype out_dt, razer_stream_t stream)
 {
-    if (!ts || !out) return RAZER_ERR_INVALID_ARG;
+    if (!ts || (!out && R * K > 0)) return RAZER_ERR_INVALID_ARG;
     if (!valid_fmt(fmt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
     razer_status st = check_packed(codes, scales, R, K);
     if (st != RAZER_OK) return st;
