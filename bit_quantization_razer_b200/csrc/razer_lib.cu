@@ -7,3 +7,4 @@
 #include "dequant.cu"
 #include "gemv.cu"
 #include "gemm.cu"
+#include "gemv_noalloc.cu"

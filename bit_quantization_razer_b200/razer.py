@@ -31,6 +31,7 @@ _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZE
 EXPORTED = (
     "razer_quantize_weights", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
+    "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
 )
 
 
@@ -57,6 +58,10 @@ def load() -> ctypes.CDLL:
     L.razer_dequant.argtypes = [vp, vp, vp, i32, i64, i64, vp, i32, vp]
     L.razer_gemv.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_gemm.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
+    L.razer_gemv_noalloc.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp]
+    L.razer_gemv_noalloc.restype = ctypes.c_int
+    L.razer_gemv_noalloc_max_scratch.argtypes = []
+    L.razer_gemv_noalloc_max_scratch.restype = sz
     L.razer_workspace_size.argtypes = [i32, i64, i64, i64]
     L.razer_workspace_size.restype = sz
     L.razer_get_device_status.argtypes = [vp]
@@ -150,6 +155,23 @@ def razer_gemv(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: t
                            _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
     _check("razer_gemv", st)
     return out
+
+
+def razer_gemv_noalloc(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight",
+                       out_dtype=torch.float32, *, out=None, stream=None):
+    """razer_gemv without a workspace: the split-K scratch is a fixed array
+    inside the library (for callers that cannot allocate device memory)."""
+    B, K = x.shape
+    N = codes.shape[0]
+    out = torch.empty((B, N), dtype=out_dtype, device=x.device) if out is None else out
+    st = load().razer_gemv_noalloc(_p(x), _DT.get(x.dtype, -1), B, _p(codes), _p(scales), _p(ts), _fmt(fmt), N, K,
+                                   _p(out), _DT.get(out.dtype, -1), _stream(stream))
+    _check("razer_gemv_noalloc", st)
+    return out
+
+
+def razer_gemv_noalloc_max_scratch() -> int:
+    return int(load().razer_gemv_noalloc_max_scratch())
 
 
 def razer_gemm(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight",

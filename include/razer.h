@@ -157,6 +157,33 @@ razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint
                         int64_t K, void *Y, razer_dtype out_dt, void *workspace, size_t ws_bytes,
                         razer_stream_t stream);
 
+/*
+ * razer_gemv_noalloc -- razer_gemv for callers that cannot allocate device
+ * memory (the paper has no counterpart: this is a deployment convenience).
+ * Some callers cannot call cudaMalloc at all, e.g. a runtime that gives every
+ * byte of the GPU to its own pool up front or code under a fixed static
+ * memory budget, so they cannot hand razer_gemv a workspace.  This entry point
+ * takes the same arguments minus the workspace and uses a fixed scratch array
+ * inside the library instead (razer_gemv_noalloc_max_scratch() bytes, held on
+ * every GPU that loads the library until the process exits).
+ *   - It allocates nothing.  Its first call on a device looks up the device
+ *     address of the array (with that device current); make that first call
+ *     before any stream capture.
+ *   - Sizes whose scratch need (razer_workspace_size(RAZER_OP_GEMV, B, N, K))
+ *     exceeds the maximum are rejected with RAZER_ERR_WORKSPACE.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls whose kernels can
+ *     overlap on the GPU -- e.g. on two unordered streams -- race on it; order
+ *     them on one stream.
+ * Results equal razer_gemv's for the same inputs.
+ */
+razer_status razer_gemv_noalloc(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes,
+                                const uint8_t *scales, const float *ts, razer_format wfmt, int64_t N,
+                                int64_t K, void *y, razer_dtype out_dt, razer_stream_t stream);
+
+/* Size in bytes of the fixed scratch array used by razer_gemv_noalloc. */
+size_t razer_gemv_noalloc_max_scratch(void);
+
 /* Bytes of workspace razer_gemv / razer_gemm need for these sizes (0 when
  * none); M_or_B is B for RAZER_OP_GEMV and M for RAZER_OP_GEMM. */
 size_t razer_workspace_size(razer_op op, int64_t M_or_B, int64_t N, int64_t K);
