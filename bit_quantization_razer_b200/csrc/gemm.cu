@@ -1,20 +1,534 @@
 // RaZeR W4A16 GEMM on the tcgen05 tensor cores (sm_100a).
+//
+//   Y[m, n] = ts * sum_k X[m, k] * (q*s)[n, k]
+//
+// (RaZeR notes 关键设计 3: weight-only kernels that decode the remapped codes
+// on the fly; gist.science summary 2.3.)  The contraction is dense, so it runs
+// on the 5th-generation tensor cores:
+//   * CTA tile 256 (M) x 256 (N), k-step 64.  Two UMMA instructions of
+//     M = 128 share one decoded weight tile, so every weight is decoded once
+//     per 256 activation rows (half the decode work per SM of a 128-row tile).
+//   * warp 0: TMA producer of the X tiles (K-major, 128-byte swizzle);
+//     warp 1: TMEM allocator and the single MMA-issuing thread;
+//     warps 2-5: decoders -- they stream the packed codes and scale bytes with
+//     128-bit loads (one stage ahead), decode to 16-bit q*s and write the
+//     UMMA canonical K-major 128B-swizzled layout with 16-byte stores; after
+//     the k loop they are the epilogue (tcgen05.ld, * ts, convert, store).
+//   * fp32 accumulators: two 128 x 256 tiles = all 512 TMEM columns.
+//   * 3-stage mbarrier pipeline; every wait is bounded (~2 s of globaltimer):
+//     on expiry the kernel records RAZER_ERR_TIMEOUT in the device status word,
+//     the other roles stop at their next wait, in-flight TMA loads are waited
+//     for (bounded), and the TMEM is freed before the CTA exits.
+// Decode exactness: q (E2M1 with the redundant zero replaced by v) is exact in
+// fp16; q*s*2^-8 (E3M3) or q*s*2^-4 (E4M3) is an exact fp16 product in the
+// normal range; for bf16 activations q*s is formed in fp32 (exact) and packed
+// to bf16 (exact: at most 7 significant bits).
+#include <cuda.h>
+
 #include "razer_internal.cuh"
 
 namespace razer {
+namespace gemm {
+
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
+constexpr int kThreads = 192;
+constexpr uint32_t A_HALF_BYTES = 128 * BK * 2;               // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;                     // 32 KB
+constexpr uint32_t STAGE_BYTES = 2 * A_HALF_BYTES + B_BYTES;  // 64 KB
+constexpr uint32_t BAR_BYTES = 256;
+constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: false when this CTA has given up (timeout here or elsewhere).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    uint64_t t0 = 0;
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 31u) == 31u) {
+            if (*abort_flag) return false;
+            const uint64_t t = globaltimer();
+            if (t0 == 0) t0 = t;
+            else if (t - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                set_device_status(RAZER_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// Lane 0 waits, the whole warp gets the result (keeps the warp converged for
+// the .aligned tcgen05 instructions that follow).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// UMMA shared-memory descriptor of a K-major, 128B-swizzled tile whose
+// 8-row groups are 1024 bytes apart (rows of 128 bytes).
+__device__ __forceinline__ uint64_t smem_desc_k128(uint32_t addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);  // start address
+    d |= (uint64_t)1 << 16;                   // leading byte offset (unused for 128B swizzle)
+    d |= (uint64_t)(1024 >> 4) << 32;         // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                   // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;                   // 128-byte swizzle
+    return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, K-major A and B.
+__host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N)
+{
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(dtmem), "l"(adesc),
+        "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,"
+        "%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]),
+          "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ unsigned cvt_e2m1x2(unsigned w)
+{
+    unsigned r;
+    asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b0; }" : "=r"(r) : "r"(w));
+    return r;
+}
+__device__ __forceinline__ unsigned prmt(unsigned a, unsigned b, unsigned sel)
+{
+    unsigned r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+__device__ __forceinline__ unsigned hmul2(unsigned a, unsigned b)
+{
+    unsigned r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Per-block decode constants of one scale byte.
+struct BlockK {
+    unsigned s16x2;  // fp16 pair of s * 2^-bias (fp16 path)
+    float s32;       // exact s (bf16 path)
+    unsigned v16x2;  // fp16 pair of v (0 when the format has no remap)
+};
+
+template <int FMT, bool BF16>
+__device__ __forceinline__ BlockK block_consts(unsigned sb)
+{
+    BlockK k;
+    if constexpr (BF16) {
+        k.s32 = decode_scale<FMT>(sb);
+        k.s16x2 = 0u;
+    } else {
+        const unsigned s16 = scale_f16_bits<FMT>(sb);  // s * 2^-12 (E3M3) or s * 2^-8 (E4M3)
+        k.s16x2 = hmul2(s16 | (s16 << 16), 0x4C004C00u);  // * 16 (exact): keeps q*s in the fp16 normal range
+        k.s32 = 0.0f;
+    }
+    if constexpr (Fmt<FMT>::kSpecials > 0) {
+        const unsigned meta = sb >> Fmt<FMT>::kMetaShift;
+        const unsigned v16 = ((meta & 2u) ? 0x4800u : 0x4500u) | ((meta & 1u) << 15);
+        k.v16x2 = v16 | (v16 << 16);
+    } else {
+        k.v16x2 = 0u;
+    }
+    return k;
+}
+
+// Decode one 32-bit word (8 codes of one block) into 4 packed 16-bit pairs.
+template <int FMT, bool BF16>
+__device__ __forceinline__ uint4 decode_word(unsigned w, const BlockK &k)
+{
+    // bit 3 of each nibble set where the code is 0b1000 (the redundant zero)
+    const unsigned is8 = w & ~((w & 0x77777777u) + 0x77777777u) & 0x88888888u;
+    const unsigned is8s = is8 << 4;
+    unsigned out[4];
+#pragma unroll
+    for (int b = 0; b < 4; b++) {
+        unsigned q = cvt_e2m1x2(w >> (8 * b));
+        if constexpr (Fmt<FMT>::kSpecials > 0) {
+            // 0xFFFF in each half whose code is 0b1000, from the nibble sign bits
+            const unsigned sel = (0x88CCu + 0x1111u * (unsigned)b);
+            const unsigned mask = prmt(is8, is8s, sel);
+            q = (q & ~mask) | (k.v16x2 & mask);
+        }
+        if constexpr (BF16) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&q));
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(f.x, k.s32), __fmul_rn(f.y, k.s32));
+            out[b] = *reinterpret_cast<unsigned *>(&h2);
+        } else {
+            out[b] = hmul2(q, k.s16x2);
+        }
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+template <int FMT, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                const float *__restrict__ ts_p, float unbias, int M, int N, int K, void *__restrict__ Y, int out_dt)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *bars = smem + STAGES * STAGE_BYTES;
+    const uint32_t full_a = smem_addr(bars);              // STAGES x 8
+    const uint32_t full_b = full_a + 8 * STAGES;          // STAGES x 8
+    const uint32_t empty = full_b + 8 * STAGES;           // STAGES x 8
+    const uint32_t acc_full = empty + 8 * STAGES;         // 8
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(bars + 128);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 136);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+    const int KB = K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; s++) {
+            mbar_init(full_a + 8 * s, 1);
+            mbar_init(full_b + 8 * s, 4);  // one arrival per decoder warp
+            mbar_init(empty + 8 * s, 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_addr((const void *)tmem_slot)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (X tiles) ----------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < KB; kb++) {
+                const int s = kb % STAGES;
+                const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+                if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort_flag)) break;
+                const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
+                mbar_expect_tx(full_a + 8 * s, 2 * A_HALF_BYTES);
+                tma_load_2d(a0, &tmap_x, kb * BK, m0, full_a + 8 * s);
+                tma_load_2d(a0 + A_HALF_BYTES, &tmap_x, kb * BK, m0 + 128, full_a + 8 * s);
+                issued = kb + 1;
+            }
+            if (*abort_flag) {
+                // let the loads already issued land before the CTA exits (bounded)
+                const uint64_t t0 = globaltimer();
+                for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; kb++) {
+                    const int s = kb % STAGES;
+                    const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+                    while (!mbar_try_wait(full_a + 8 * s, ph) && globaltimer() - t0 < kTimeoutNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f16(BF16, 128, BN);
+            bool ok = true;
+            for (int kb = 0; kb < KB && ok; kb++) {
+                const int s = kb % STAGES;
+                const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+                ok = mbar_wait(full_a + 8 * s, ph, abort_flag) && mbar_wait(full_b + 8 * s, ph, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
+                const uint32_t b0 = a0 + 2 * A_HALF_BYTES;
+#pragma unroll
+                for (int k = 0; k < BK / 16; k++) {
+                    const uint64_t bd = smem_desc_k128(b0 + 32 * k);
+                    const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                    umma_f16(tmem, smem_desc_k128(a0 + 32 * k), bd, idesc, acc);
+                    umma_f16(tmem + 256, smem_desc_k128(a0 + A_HALF_BYTES + 32 * k), bd, idesc, acc);
+                }
+                umma_commit(empty + 8 * s);
+            }
+            umma_commit(acc_full);
+            if (!ok) {
+                // stopped early: let the MMAs already issued finish (bounded)
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(acc_full, 0) && globaltimer() - t0 < kTimeoutNs) {
+                }
+            }
+        }
+    } else {
+        // ---------------- decoders, then epilogue ----------------
+        const int t = threadIdx.x - 64;  // 0..127
+        const int rows[2] = {t, t + 128};
+        const uint8_t *crow[2];
+        const uint8_t *srow[2];
+        bool valid[2];
+#pragma unroll
+        for (int r = 0; r < 2; r++) {
+            const int n = n0 + rows[r];
+            valid[r] = n < N;
+            const int nn = valid[r] ? n : (N - 1);
+            crow[r] = codes + (size_t)nn * (K >> 1);
+            srow[r] = scales + (size_t)nn * (K >> 4);
+        }
+        uint4 cc[2][2];
+        unsigned sc[2];
+        auto load_stage = [&](int kb) {
+#pragma unroll
+            for (int r = 0; r < 2; r++) {
+                cc[r][0] = ldg_stream(crow[r] + (size_t)kb * 32);
+                cc[r][1] = ldg_stream(crow[r] + (size_t)kb * 32 + 16);
+                sc[r] = __ldg(reinterpret_cast<const unsigned *>(srow[r] + (size_t)kb * 4));
+            }
+        };
+        load_stage(0);
+        bool ok = true;
+        for (int kb = 0; kb < KB; kb++) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+            uint4 cur[2][2] = {{cc[0][0], cc[0][1]}, {cc[1][0], cc[1][1]}};
+            unsigned cur_s[2] = {sc[0], sc[1]};
+            if (kb + 1 < KB) load_stage(kb + 1);
+            if (!mbar_wait_warp(empty + 8 * s, ph ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            uint8_t *btile = smem + s * STAGE_BYTES + 2 * A_HALF_BYTES;
+#pragma unroll
+            for (int r = 0; r < 2; r++) {
+                const int row = rows[r];
+                uint8_t *rbase = btile + (row >> 3) * 1024 + (row & 7) * 128;
+                const unsigned words[8] = {cur[r][0].x, cur[r][0].y, cur[r][0].z, cur[r][0].w,
+                                           cur[r][1].x, cur[r][1].y, cur[r][1].z, cur[r][1].w};
+#pragma unroll
+                for (int blk = 0; blk < 4; blk++) {
+                    const BlockK kc = block_consts<FMT, BF16>(valid[r] ? ((cur_s[r] >> (8 * blk)) & 0xFFu) : 0u);
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const int j = 2 * blk + h;  // 16-byte chunk = 8 elements
+                        uint4 v = decode_word<FMT, BF16>(valid[r] ? words[j] : 0u, kc);
+                        *reinterpret_cast<uint4 *>(rbase + ((j ^ (row & 7)) << 4)) = v;
+                    }
+                }
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full_b + 8 * s);
+        }
+
+        // epilogue: TMEM lanes 32*(warp%4) .. +31 of both accumulators
+        if (ok && mbar_wait_warp(acc_full, 0, abort_flag) && !*abort_flag) {
+            tc_fence_after();
+            const int q = warp & 3;
+            const float scale = __fmul_rn(*ts_p, unbias);
+#pragma unroll 1
+            for (int half = 0; half < 2; half++) {
+                const int m = m0 + half * 128 + q * 32 + lane;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c0), v);
+                    const int n = n0 + c0;
+                    if (m < M && n < N && n + 32 > N) {
+                        for (int i = 0; i < N - n; i++) {
+                            const float a = v[i] * scale;
+                            if (out_dt == RAZER_F32) reinterpret_cast<float *>(Y)[(size_t)m * N + n + i] = a;
+                            else if (out_dt == RAZER_BF16) reinterpret_cast<__nv_bfloat16 *>(Y)[(size_t)m * N + n + i] = __float2bfloat16_rn(a);
+                            else reinterpret_cast<__half *>(Y)[(size_t)m * N + n + i] = __float2half_rn(a);
+                        }
+                    } else if (m < M && n < N) {
+                        if (out_dt == RAZER_F32) {
+                            float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(Y) + (size_t)m * N + n);
+#pragma unroll
+                            for (int i = 0; i < 8; i++)
+                                dst[i] = make_float4(v[4 * i] * scale, v[4 * i + 1] * scale, v[4 * i + 2] * scale, v[4 * i + 3] * scale);
+                        } else {
+                            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(Y) + (size_t)m * N + n);
+#pragma unroll
+                            for (int i = 0; i < 4; i++) {
+                                unsigned p[4];
+#pragma unroll
+                                for (int e = 0; e < 4; e++) {
+                                    const float a = v[8 * i + 2 * e] * scale, b = v[8 * i + 2 * e + 1] * scale;
+                                    if (out_dt == RAZER_BF16) {
+                                        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+                                        p[e] = *reinterpret_cast<unsigned *>(&h);
+                                    } else {
+                                        __half2 h = __floats2half2_rn(a, b);
+                                        p[e] = *reinterpret_cast<unsigned *>(&h);
+                                    }
+                                }
+                                dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncwarp();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *, const cuuint64_t *,
+                                  const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int FMT, bool BF16>
+static razer_status launch(const CUtensorMap &map, const uint8_t *codes, const uint8_t *scales, const float *ts, float unbias, int M,
+                           int N, int K, void *Y, razer_dtype out_dt, cudaStream_t st)
+{
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(gemm_kernel<FMT, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess)
+            return RAZER_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt);
+    return last_launch_status();
+}
+
+}  // namespace gemm
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
-    (void)M; (void)N; (void)K;
+    (void)M;
+    (void)N;
+    (void)K;
     return 0;
 }
 
 razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
                       razer_format wfmt, int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st)
 {
-    (void)X; (void)act_dt; (void)M; (void)codes; (void)scales; (void)ts; (void)wfmt; (void)N; (void)K; (void)Y; (void)out_dt;
-    (void)workspace; (void)st;
-    return RAZER_ERR_UNSUPPORTED;
+    (void)workspace;
+    using namespace gemm;
+    if (K == 0) {
+        const size_t esz = out_dt == RAZER_F32 ? 4 : 2;
+        return cudaMemsetAsync(Y, 0, (size_t)M * (size_t)N * esz, st) == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return RAZER_ERR_CUDA;
+    const bool bf = act_dt == RAZER_BF16;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, 128u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (enc(&map, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return RAZER_ERR_CUDA;
+    // q*s carries 2^-8 (E3M3) / 2^-4 (E4M3) on the fp16 path; exact s on the bf16 path
+    const float unbias = bf ? 1.0f : (wfmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f);
+    const int m = (int)M, n = (int)N, k = (int)K;
+    if (wfmt == RAZER_FMT_WEIGHT)
+        return bf ? launch<RAZER_FMT_WEIGHT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
+                  : launch<RAZER_FMT_WEIGHT, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
+    if (wfmt == RAZER_FMT_ACT)
+        return bf ? launch<RAZER_FMT_ACT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
+                  : launch<RAZER_FMT_ACT, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
+    return bf ? launch<RAZER_FMT_NVFP4, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
+              : launch<RAZER_FMT_NVFP4, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
 }
 
 }  // namespace razer

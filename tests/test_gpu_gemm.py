@@ -1,0 +1,86 @@
+"""tcgen05 GEMM against the oracle's double-accumulated product."""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantization_razer_b200 as R
+from bit_quantization_razer_b200 import workloads
+from tests.gpu_helpers import FMT_ID, REL_TOL, assert_close_typed, cuda, oracle_in, rel_err
+
+pytestmark = [pytest.mark.gpu, cuda]
+DEV = "cuda:0"
+
+
+def gemm(X, codes, scales, ts, fmt, out_dtype=torch.float32):
+    Y = R.razer_gemm(X.to(DEV), codes.to(DEV), scales.to(DEV), torch.tensor([ts], dtype=torch.float32, device=DEV),
+                     fmt, out_dtype)
+    torch.cuda.synchronize()
+    assert R.razer_get_device_status() == 0
+    return Y
+
+
+def test_gemm_small_single_tile(orc):
+    M, N, K = 128, 256, 128
+    codes, scales = workloads.random_packed(N, K, "weight", seed=70, max_scale_code=40)
+    X = workloads.vectors(M, K, seed=71, dtype=torch.bfloat16)
+    ref = orc.gemm_ref(oracle_in(X), codes.numpy(), scales.numpy(), 0.25, 0)
+    Y = gemm(X, codes, scales, 0.25, "weight")
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
+
+
+@pytest.mark.parametrize("fmt", ["weight", "act", "nvfp4"])
+@pytest.mark.parametrize("xdt", [torch.bfloat16, torch.float16])
+def test_gemm_ragged_multi_tile(orc, fmt, xdt):
+    # M tail (300 rows), N not a multiple of 32, 3 k-steps (one pass over the stages)
+    M, N, K = 300, 272, 192
+    codes, scales = workloads.random_packed(N, K, fmt, seed=72, max_scale_code=None)
+    X = workloads.vectors(M, K, seed=73, dtype=xdt)
+    ts = 0.0371
+    ref = orc.gemm_ref(oracle_in(X), codes.numpy(), scales.numpy(), ts, FMT_ID[fmt])
+    Y = gemm(X, codes, scales, ts, fmt)
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
+
+
+def test_gemm_oracle_quantized_weights(orc):
+    # realistic weights quantized by the oracle; 8 k-steps wrap the 3-stage ring
+    w = workloads.weight(512, 512, std=0.02, seed=74)
+    codes, scales, ts, _ = orc.quantize(w.numpy(), 0)
+    X = workloads.vectors(512, 512, seed=75, dtype=torch.bfloat16)
+    ref = orc.gemm_ref(oracle_in(X), codes, scales, ts, 0)
+    for odt in (torch.float32, torch.bfloat16, torch.float16):
+        Y = gemm(X, torch.from_numpy(codes), torch.from_numpy(scales), ts, "weight", odt)
+        assert_close_typed(Y, ref)
+
+
+def test_gemm_one_hot_rows_equal_dequant(orc):
+    codes, scales = workloads.random_packed(256, 128, "weight", seed=76)
+    deq = orc.dequant(codes.numpy(), scales.numpy(), 0.5, 0, "f32")
+    X = torch.zeros(256, 128, dtype=torch.bfloat16)
+    for m in range(256):
+        X[m, m % 128] = 1.0
+    Y = gemm(X, codes, scales, 0.5, "weight").cpu().numpy()
+    for m in (0, 5, 127, 128, 200, 255):
+        np.testing.assert_array_equal(Y[m], deq[:, m % 128])
+
+
+@pytest.mark.parametrize("M,N,K,rows", [(4096, 4096, 4096, 96), (4096, 14336, 4096, 24), (2048, 4096, 14336, 24)])
+def test_gemm_prefill_shapes_sampled(orc, M, N, K, rows):
+    codes, scales = workloads.random_packed(N, K, "weight", seed=M + N + K, max_scale_code=40)
+    X = workloads.vectors(M, K, seed=77, dtype=torch.bfloat16)
+    ts = 0.0045
+    Y = gemm(X, codes, scales, ts, "weight").cpu().numpy()
+    sel = np.sort(np.random.default_rng(2).choice(M, rows, replace=False))
+    ref = orc.gemm_ref(oracle_in(X[sel]), codes.numpy(), scales.numpy(), ts, 0)
+    assert rel_err(Y[sel], ref) <= REL_TOL
+
+
+def test_gemm_k_zero_and_errors():
+    codes = torch.zeros(32, 0, dtype=torch.uint8, device=DEV)
+    scales = torch.zeros(32, 0, dtype=torch.uint8, device=DEV)
+    X = torch.zeros(8, 0, dtype=torch.bfloat16, device=DEV)
+    Y = R.razer_gemm(X, codes, scales, torch.ones(1, device=DEV), "weight", torch.float32)
+    torch.cuda.synchronize()
+    assert not Y.any()
+    c, s = workloads.random_packed(48, 96, "weight", seed=1)
+    with pytest.raises(R.RazerError):  # K % 64
+        R.razer_gemm(torch.zeros(8, 96, dtype=torch.bfloat16, device=DEV), c.to(DEV), s.to(DEV), torch.ones(1, device=DEV))
