@@ -102,14 +102,18 @@ razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint
                         razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, size_t ws_bytes,
                         razer_stream_t stream)
 {
-    if (!x || !ts || !y) return RAZER_ERR_INVALID_ARG;
+    if (!ts || (!x && K > 0) || (!y && N > 0)) return RAZER_ERR_INVALID_ARG;
     if (!valid_fmt(wfmt) || !valid_dt(act_dt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
     if (!in16(act_dt)) return RAZER_ERR_DTYPE;
     razer_status st = check_packed(codes, scales, N, K);
     if (st != RAZER_OK) return st;
     if (B < 1 || B > 32 || K % 128 != 0 || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
     if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ts, 4)) return RAZER_ERR_ALIGN;
-    if (N == 0 || K == 0) return RAZER_OK;
+    if (N == 0) return RAZER_OK;
+    if (K == 0)  // empty sums: y = 0
+        return cudaMemsetAsync(y, 0, (size_t)B * (size_t)N * (out_dt == RAZER_F32 ? 4 : 2), (cudaStream_t)stream) == cudaSuccess
+                   ? RAZER_OK
+                   : RAZER_ERR_CUDA;
     const size_t need = gemv_workspace_bytes(B, N, K);
     if (need) {
         if (!workspace || ws_bytes < need) return RAZER_ERR_WORKSPACE;
@@ -122,7 +126,7 @@ razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint
                         razer_format wfmt, int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace, size_t ws_bytes,
                         razer_stream_t stream)
 {
-    if (!X || !ts || !Y) return RAZER_ERR_INVALID_ARG;
+    if (!ts || (!X && M * K > 0) || (!Y && M * N > 0)) return RAZER_ERR_INVALID_ARG;
     if (!valid_fmt(wfmt) || !valid_dt(act_dt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
     if (!in16(act_dt)) return RAZER_ERR_DTYPE;
     razer_status st = check_packed(codes, scales, N, K);
