@@ -10,7 +10,8 @@
 //     per 256 activation rows (half the decode work per SM of a 128-row tile).
 //   * warp 0: TMA producer of the X tiles (K-major, 128-byte swizzle);
 //     warp 1: TMEM allocator and the single MMA-issuing thread;
-//     warps 2-5: decoders -- they stream the packed codes and scale bytes with
+//     warps 2-9: decoders, one weight row per thread, two warps per scheduler
+//     -- they stream the packed codes and scale bytes with
 //     128-bit loads (one stage ahead), decode to 16-bit q*s and write the
 //     UMMA canonical K-major 128B-swizzled layout with 16-byte stores; after
 //     the k loop they are the epilogue (tcgen05.ld, * ts, convert, store).
@@ -21,8 +22,8 @@
 //     for (bounded), and the TMEM is freed before the CTA exits.
 // Decode exactness: q (E2M1 with the redundant zero replaced by v) is exact in
 // fp16; q*s*2^-8 (E3M3) or q*s*2^-4 (E4M3) is an exact fp16 product in the
-// normal range; for bf16 activations q*s is formed in fp32 (exact) and packed
-// to bf16 (exact: at most 7 significant bits).
+// normal range, which converts exactly to bf16 (at most 7 significant bits)
+// for bf16 activations.
 #include <cuda.h>
 
 #include "razer_internal.cuh"
@@ -31,7 +32,8 @@ namespace razer {
 namespace gemm {
 
 constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
-constexpr int kThreads = 192;
+constexpr int kDecodeWarps = 8;  // two per scheduler
+constexpr int kThreads = 64 + 32 * kDecodeWarps;
 constexpr uint32_t A_HALF_BYTES = 128 * BK * 2;               // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;                     // 32 KB
 constexpr uint32_t STAGE_BYTES = 2 * A_HALF_BYTES + B_BYTES;  // 64 KB
@@ -191,10 +193,7 @@ template <int FMT, bool BF16>
 __device__ __forceinline__ BlockK block_consts(unsigned sb)
 {
     BlockK k;
-    if constexpr (BF16) {
-        k.s32 = decode_scale<FMT>(sb);
-        k.s16x2 = 0u;
-    } else {
+    {
         const unsigned s16 = scale_f16_bits<FMT>(sb);  // s * 2^-12 (E3M3) or s * 2^-8 (E4M3)
         k.s16x2 = hmul2(s16 | (s16 << 16), 0x4C004C00u);  // * 16 (exact): keeps q*s in the fp16 normal range
         k.s32 = 0.0f;
@@ -226,12 +225,13 @@ __device__ __forceinline__ uint4 decode_word(unsigned w, const BlockK &k)
             const unsigned mask = prmt(is8, is8s, sel);
             q = (q & ~mask) | (k.v16x2 & mask);
         }
+        const unsigned p = hmul2(q, k.s16x2);  // exact q*s*2^-bias in fp16
         if constexpr (BF16) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&q));
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(f.x, k.s32), __fmul_rn(f.y, k.s32));
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&p));
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(f.x, f.y);  // exact
             out[b] = *reinterpret_cast<unsigned *>(&h2);
         } else {
-            out[b] = hmul2(q, k.s16x2);
+            out[b] = p;
         }
     }
     return make_uint4(out[0], out[1], out[2], out[3]);
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
             mbar_init(full_a + 8 * s, 1);
-            mbar_init(full_b + 8 * s, 4);  // one arrival per decoder warp
+            mbar_init(full_b + 8 * s, kDecodeWarps);  // one arrival per decoder warp
             mbar_init(empty + 8 * s, 1);
         }
         mbar_init(acc_full, 1);
@@ -332,57 +332,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- decoders, then epilogue ----------------
-        const int t = threadIdx.x - 64;  // 0..127
-        const int rows[2] = {t, t + 128};
-        const uint8_t *crow[2];
-        const uint8_t *srow[2];
-        bool valid[2];
-#pragma unroll
-        for (int r = 0; r < 2; r++) {
-            const int n = n0 + rows[r];
-            valid[r] = n < N;
-            const int nn = valid[r] ? n : (N - 1);
-            crow[r] = codes + (size_t)nn * (K >> 1);
-            srow[r] = scales + (size_t)nn * (K >> 4);
-        }
-        uint4 cc[2][2];
-        unsigned sc[2];
+        const int row = threadIdx.x - 64;  // 0..255: one weight row per thread
+        const int n = n0 + row;
+        const bool valid = n < N;
+        const uint8_t *crow = codes + (size_t)(valid ? n : (N - 1)) * (K >> 1);
+        const uint8_t *srow = scales + (size_t)(valid ? n : (N - 1)) * (K >> 4);
+        uint4 cc0, cc1;
+        unsigned sc;
         auto load_stage = [&](int kb) {
-#pragma unroll
-            for (int r = 0; r < 2; r++) {
-                cc[r][0] = ldg_stream(crow[r] + (size_t)kb * 32);
-                cc[r][1] = ldg_stream(crow[r] + (size_t)kb * 32 + 16);
-                sc[r] = __ldg(reinterpret_cast<const unsigned *>(srow[r] + (size_t)kb * 4));
-            }
+            cc0 = ldg_stream(crow + (size_t)kb * 32);
+            cc1 = ldg_stream(crow + (size_t)kb * 32 + 16);
+            sc = __ldg(reinterpret_cast<const unsigned *>(srow + (size_t)kb * 4));
         };
         load_stage(0);
         bool ok = true;
         for (int kb = 0; kb < KB; kb++) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            uint4 cur[2][2] = {{cc[0][0], cc[0][1]}, {cc[1][0], cc[1][1]}};
-            unsigned cur_s[2] = {sc[0], sc[1]};
+            const uint4 c0 = cc0, c1 = cc1;
+            const unsigned cs = valid ? sc : 0u;
             if (kb + 1 < KB) load_stage(kb + 1);
             if (!mbar_wait_warp(empty + 8 * s, ph ^ 1u, abort_flag)) {
                 ok = false;
                 break;
             }
-            uint8_t *btile = smem + s * STAGE_BYTES + 2 * A_HALF_BYTES;
+            uint8_t *rbase = smem + s * STAGE_BYTES + 2 * A_HALF_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+            const unsigned words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-            for (int r = 0; r < 2; r++) {
-                const int row = rows[r];
-                uint8_t *rbase = btile + (row >> 3) * 1024 + (row & 7) * 128;
-                const unsigned words[8] = {cur[r][0].x, cur[r][0].y, cur[r][0].z, cur[r][0].w,
-                                           cur[r][1].x, cur[r][1].y, cur[r][1].z, cur[r][1].w};
+            for (int blk = 0; blk < 4; blk++) {
+                const BlockK kc = block_consts<FMT, BF16>((cs >> (8 * blk)) & 0xFFu);
 #pragma unroll
-                for (int blk = 0; blk < 4; blk++) {
-                    const BlockK kc = block_consts<FMT, BF16>(valid[r] ? ((cur_s[r] >> (8 * blk)) & 0xFFu) : 0u);
-#pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        const int j = 2 * blk + h;  // 16-byte chunk = 8 elements
-                        uint4 v = decode_word<FMT, BF16>(valid[r] ? words[j] : 0u, kc);
-                        *reinterpret_cast<uint4 *>(rbase + ((j ^ (row & 7)) << 4)) = v;
-                    }
+                for (int h = 0; h < 2; h++) {
+                    const int j = 2 * blk + h;  // 16-byte chunk = 8 elements
+                    const uint4 v = decode_word<FMT, BF16>(words[j], kc);
+                    *reinterpret_cast<uint4 *>(rbase + ((j ^ (row & 7)) << 4)) = v;
                 }
             }
             fence_proxy_async();
@@ -390,16 +373,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(full_b + 8 * s);
         }
 
-        // epilogue: TMEM lanes 32*(warp%4) .. +31 of both accumulators
+        // epilogue: TMEM lanes 32*(warp%4) .. +31; the two warps of a lane
+        // quarter split the 256 columns of each accumulator
         if (ok && mbar_wait_warp(acc_full, 0, abort_flag) && !*abort_flag) {
             tc_fence_after();
             const int q = warp & 3;
+            const int cbeg = (warp - 2) < 4 ? 0 : BN / 2;
             const float scale = __fmul_rn(*ts_p, unbias);
 #pragma unroll 1
             for (int half = 0; half < 2; half++) {
                 const int m = m0 + half * 128 + q * 32 + lane;
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
+                for (int c0 = cbeg; c0 < cbeg + BN / 2; c0 += 32) {
                     float v[32];
                     tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c0), v);
                     const int n = n0 + c0;
@@ -518,8 +503,8 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return RAZER_ERR_CUDA;
-    // q*s carries 2^-8 (E3M3) / 2^-4 (E4M3) on the fp16 path; exact s on the bf16 path
-    const float unbias = bf ? 1.0f : (wfmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f);
+    // the decoded q*s carries 2^-8 (E3M3) / 2^-4 (E4M3); undone in the epilogue
+    const float unbias = wfmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f;
     const int m = (int)M, n = (int)N, k = (int)K;
     if (wfmt == RAZER_FMT_WEIGHT)
         return bf ? launch<RAZER_FMT_WEIGHT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)

@@ -9,11 +9,11 @@
 //   * a warp owns 16 weight rows; each step it streams a 16-row x 128-k
 //     slice of codes with one 128-bit load per thread per row (64 contiguous
 //     bytes per row, 4 lanes per row), plus the matching scale bytes;
-//   * each code byte becomes one f16x2 pair with the hardware E2M1 convert,
-//     the redundant-zero codes are turned into the block's special value by
-//     a second convert of an indicator nibble (1.0 where the code is 0b1000)
-//     folded in with one packed FMA, and the block scale is applied with a
-//     packed multiply -- q*s*2^-12 (E3M3) or q*s*2^-8 (E4M3) is exact in fp16;
+//   * each code byte becomes one f16x2 pair with the hardware E2M1 convert;
+//     the redundant-zero codes are replaced by the block's special value with
+//     a byte permute (sign replication of the nibble's bit 3) and one bitwise
+//     select, and the block scale is applied with a packed multiply --
+//     q*s*2^-12 (E3M3) or q*s*2^-8 (E4M3) is exact in fp16;
 //   * the decoded pairs are already in the register layout of the A operand of
 //     the warp-level m16n8k16 tensor-core MMA, so the products accumulate in
 //     fp32 without any shared-memory round trip; the activations form the
@@ -44,13 +44,6 @@ __device__ __forceinline__ unsigned hmul2u(unsigned a, unsigned b)
     return r;
 }
 
-__device__ __forceinline__ unsigned hfma2u(unsigned a, unsigned b, unsigned c)
-{
-    unsigned r;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-    return r;
-}
-
 // f16x2 -> bf16x2 (exact for the decoded values: at most 7 significant bits,
 // inside the bf16 range)
 __device__ __forceinline__ unsigned f16x2_to_bf16x2(unsigned h)
@@ -62,19 +55,33 @@ __device__ __forceinline__ unsigned f16x2_to_bf16x2(unsigned h)
     return r;
 }
 
-// Decode 8 codes of one block (a 32-bit word) into 4 f16x2 pairs of
-// (q * s * 2^-bias): pair b holds nibbles 2b (low half) and 2b+1.
-template <bool BF16>
-__device__ __forceinline__ void decode_word(unsigned w, unsigned s2, unsigned vs2, unsigned (&h)[4])
+__device__ __forceinline__ unsigned prmt(unsigned a, unsigned b, unsigned sel)
 {
-    const unsigned a = w & 0x77777777u;
-    const unsigned nz = (a + 0x77777777u) & 0x88888888u;  // bit 3: magnitude != 0
-    const unsigned ind = (w & ~nz & 0x88888888u) >> 2;     // nibble 2 (=1.0) where code == 0b1000
+    unsigned r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Decode 8 codes of one block (a 32-bit word) into 4 packed pairs of
+// (q * s * 2^-bias): pair b holds nibbles 2b (low half) and 2b+1.  The
+// 0b1000 codes become v: bit 3 of each such nibble is spread over its 16-bit
+// half with a byte permute (sign replication) and selects v's fp16 pattern.
+template <int FMT, bool BF16>
+__device__ __forceinline__ void decode_word(unsigned w, unsigned s2, unsigned v2, unsigned (&h)[4])
+{
+    unsigned is8 = 0u, is8s = 0u;
+    if constexpr (Fmt<FMT>::kSpecials > 0) {
+        is8 = w & ~((w & 0x77777777u) + 0x77777777u) & 0x88888888u;
+        is8s = is8 << 4;
+    }
 #pragma unroll
     for (int b = 0; b < 4; b++) {
-        const unsigned q = cvt_e2m1x2_f16x2(w >> (8 * b));
-        const unsigned i = cvt_e2m1x2_f16x2(ind >> (8 * b));
-        const unsigned r = hfma2u(i, vs2, hmul2u(q, s2));
+        unsigned q = cvt_e2m1x2_f16x2(w >> (8 * b));
+        if constexpr (Fmt<FMT>::kSpecials > 0) {
+            const unsigned m = prmt(is8, is8s, 0x88CCu + 0x1111u * (unsigned)b);
+            q = (q & ~m) | (v2 & m);
+        }
+        const unsigned r = hmul2u(q, s2);
         h[b] = BF16 ? f16x2_to_bf16x2(r) : r;
     }
 }
@@ -93,18 +100,26 @@ __device__ __forceinline__ void mma16816(float (&d)[4], unsigned a0, unsigned a1
     }
 }
 
-// f16 scale pair and (v * s) pair of one scale byte
+// fp16 scale pairs and special-value pairs of the two blocks held in the low
+// 16 bits of sb (one scale byte per block).
 template <int FMT>
-__device__ __forceinline__ void scale_pairs(unsigned sb, unsigned &s2, unsigned &vs2)
+__device__ __forceinline__ void scale_pairs2(unsigned sb, unsigned (&s2)[2], unsigned (&v2)[2])
 {
-    const unsigned s16 = scale_f16_bits<FMT>(sb);
-    s2 = s16 | (s16 << 16);
+    const unsigned x = prmt(sb, 0u, 0x4140u);  // 16-bit lanes: byte 0, byte 1
+    const unsigned mag = Fmt<FMT>::kMagMask * 0x10001u;
+    const unsigned sx = (x & mag) << 7;         // fp16 of s * 2^-12 (E3M3) or s * 2^-8 (E4M3)
+    s2[0] = prmt(sx, 0u, 0x1010u);
+    s2[1] = prmt(sx, 0u, 0x3232u);
     if constexpr (Fmt<FMT>::kSpecials > 0) {
-        const unsigned meta = sb >> Fmt<FMT>::kMetaShift;
-        const unsigned v16 = ((meta & 2u) ? 0x4800u : 0x4500u) | ((meta & 1u) << 15);  // +-5 or +-8 in fp16
-        vs2 = hmul2u(v16 | (v16 << 16), s2);
+        // fp16 high bytes of +5, -5, +8, -8 indexed by the meta value
+        constexpr unsigned kVHigh = 0xC848C545u;
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            const unsigned meta = (x >> (16 * b + Fmt<FMT>::kMetaShift)) & 3u;
+            v2[b] = prmt(kVHigh, 0u, 0x4040u + meta * 0x1010u);
+        }
     } else {
-        vs2 = 0u;
+        v2[0] = v2[1] = 0u;
     }
 }
 
@@ -129,11 +144,19 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
 #pragma unroll
     for (int j = 0; j < NB; j++) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
 
+    uint4 na = make_uint4(0u, 0u, 0u, 0u), nb = na;
+    unsigned nsA = 0u, nsB = 0u;
+    auto load = [&](int c) {
+        na = ldg_stream(pa + (size_t)c * 64);
+        nb = ldg_stream(pb + (size_t)c * 64);
+        nsA = *reinterpret_cast<const unsigned short *>(sa + (size_t)c * 8);
+        nsB = *reinterpret_cast<const unsigned short *>(sbp + (size_t)c * 8);
+    };
+    if (c_begin < c_end) load(c_begin);
     for (int c = c_begin; c < c_end; c++) {
-        const uint4 ca = ldg_stream(pa + (size_t)c * 64);
-        const uint4 cb = ldg_stream(pb + (size_t)c * 64);
-        const unsigned sA = *reinterpret_cast<const unsigned short *>(sa + (size_t)c * 8);
-        const unsigned sB = *reinterpret_cast<const unsigned short *>(sbp + (size_t)c * 8);
+        const uint4 ca = na, cb = nb;
+        const unsigned sA = nsA, sB = nsB;
+        if (c + 1 < c_end) load(c + 1);  // one chunk of codes in flight ahead
         unsigned xw[NB][16];
 #pragma unroll
         for (int j = 0; j < NB; j++) {
@@ -153,18 +176,16 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
                 for (int q = 0; q < 16; q++) xw[j][q] = 0u;
             }
         }
-        unsigned s2A[2], vsA[2], s2B[2], vsB[2];
-        scale_pairs<FMT>(sA & 0xFFu, s2A[0], vsA[0]);
-        scale_pairs<FMT>(sA >> 8, s2A[1], vsA[1]);
-        scale_pairs<FMT>(sB & 0xFFu, s2B[0], vsB[0]);
-        scale_pairs<FMT>(sB >> 8, s2B[1], vsB[1]);
+        unsigned s2A[2], vA[2], s2B[2], vB[2];
+        scale_pairs2<FMT>(sA, s2A, vA);
+        scale_pairs2<FMT>(sB, s2B, vB);
         const unsigned wa[4] = {ca.x, ca.y, ca.z, ca.w};
         const unsigned wb[4] = {cb.x, cb.y, cb.z, cb.w};
 #pragma unroll
         for (int m = 0; m < 4; m++) {
             unsigned hA[4], hB[4];
-            decode_word<BF16>(wa[m], s2A[m >> 1], vsA[m >> 1], hA);
-            decode_word<BF16>(wb[m], s2B[m >> 1], vsB[m >> 1], hB);
+            decode_word<FMT, BF16>(wa[m], s2A[m >> 1], vA[m >> 1], hA);
+            decode_word<FMT, BF16>(wb[m], s2B[m >> 1], vB[m >> 1], hB);
 #pragma unroll
             for (int j = 0; j < NB; j++) {
                 mma16816<BF16>(acc[j], hA[0], hB[0], hA[1], hB[1], xw[j][4 * m], xw[j][4 * m + 1]);
@@ -206,7 +227,7 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float *__restric
 }
 
 // ---------------------------------------------------------------------------
-// Split-K sizing: enough CTAs for ~4 resident 4-warp CTAs per SM, never more
+// Split-K sizing: enough CTAs for ~8 resident 4-warp CTAs per SM, never more
 // splits than 128-wide k chunks (each split keeps at least two chunks when K
 // allows, so the reduction stays small against the weight stream).
 // ---------------------------------------------------------------------------
@@ -215,7 +236,7 @@ int gemv_splits(int64_t B, int64_t N, int64_t K)
     (void)B;
     const int64_t ctas_x = ((N + 15) / 16 + kGemvWarps - 1) / kGemvWarps;
     const int64_t chunks = K / 128;
-    const int64_t target = (int64_t)sm_count() * 4;
+    const int64_t target = (int64_t)sm_count() * 8;
     int64_t S = (target + ctas_x - 1) / ctas_x;
     const int64_t max_s = chunks >= 4 ? chunks / 2 : (chunks > 0 ? chunks : 1);
     if (S > max_s) S = max_s;

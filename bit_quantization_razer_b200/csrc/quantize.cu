@@ -14,6 +14,8 @@
 //     16-bit input significand and every binary32 divisor significand, so the
 //     result is the IEEE quotient (blocks with d outside [2^-90, 2^90] take
 //     the plain IEEE divide);
+//   * the plain E2M1 codes (ties to the smaller magnitude) come from two
+//     hardware conversions and a 3-operation select per 8 codes (fix_codes);
 //   * the squared-error comparison of the candidates is exact: only elements
 //     whose nearest point changes contribute, each term (q - v)(2 xs - q - v)
 //     is a multiple of 2^-20 computed exactly in binary32, and the partial
@@ -22,16 +24,52 @@
 
 namespace razer {
 
-// Plain E2M1 magnitude code of a = |xs|, nearest with ties to the smaller
-// magnitude.  For a >= 1 the code is a half-down rounding of the binary32
-// bit pattern to one mantissa bit (adding 2^21 - 1 then truncating rounds
-// ties down); below 1 the two thresholds are compared directly.
-__device__ __forceinline__ unsigned e2m1_mag_code(float a)
+// Packed binary32 pair arithmetic (two lanes per instruction on sm_100a).
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
 {
-    unsigned u = __float_as_uint(a);
-    unsigned hi = min(((u + 0x1FFFFFu) >> 22) - 252u, 7u);
-    unsigned lo = (unsigned)(a > 0.25f) + (unsigned)(a > 0.75f);
-    return a >= 1.0f ? hi : lo;
+    float2 d;
+    asm("{ .reg .b64 A, B, D; mov.b64 A, {%2, %3}; mov.b64 B, {%4, %5}; mul.rn.f32x2 D, A, B; mov.b64 {%0, %1}, D; }"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{ .reg .b64 A, B, C, D; mov.b64 A, {%2, %3}; mov.b64 B, {%4, %5}; mov.b64 C, {%6, %7}; fma.rn.f32x2 D, A, B, C; mov.b64 {%0, %1}, D; }"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// Hardware E2M1 conversion (round to nearest even, saturating) of 8 values
+// into one word: nibble j holds the code of v[j].
+__device__ __forceinline__ unsigned cvt_e2m1x8(const float *v)
+{
+    unsigned w;
+    asm("{ .reg .b8 b0, b1, b2, b3;"
+        " cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;"
+        " cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;"
+        " cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;"
+        " cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;"
+        " mov.b32 %0, {b0, b1, b2, b3}; }"
+        : "=r"(w)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return w;
+}
+
+// Plain E2M1 codes with ties to the SMALLER magnitude from two hardware
+// conversions (ties to even): c1 of xs and c2 of pred(xs) = xs * (1 - 2^-24)
+// (one ulp toward zero).  They differ only when a midpoint lies in
+// [pred(xs), xs]; the two codes are then adjacent and the right one is the
+// odd one (tests/test_e2m1_tie_identity.py checks this for every binary32 in
+// [0, 16]).  Finally the codes of values that rounded to -0 become 0b0000.
+__device__ __forceinline__ unsigned fix_codes(unsigned c1, unsigned c2)
+{
+    const unsigned odd = (c1 & 0x11111111u) * 15u;  // whole nibble set where c1 is odd
+    const unsigned w = (c1 & odd) | (c2 & ~odd);
+    const unsigned z = w & ~((w & 0x77777777u) + 0x77777777u) & 0x88888888u;  // nibbles == 0b1000
+    return w & ~z;
 }
 
 struct BlockOut {
@@ -67,38 +105,59 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], float t
     float xs[16];
     if (d >= 0x1p-90f && d <= 0x1p90f) {
         const float y = __frcp_rn(d);
+        const float2 y2 = make_float2(y, y), nd2 = make_float2(-d, -d);
 #pragma unroll
-        for (int j = 0; j < 16; j++) {
-            const float q = __fmul_rn(x[j], y);
-            const float r = __fmaf_rn(-q, d, x[j]);
-            xs[j] = __fmaf_rn(r, y, q);
+        for (int j = 0; j < 16; j += 2) {
+            const float2 xv = make_float2(x[j], x[j + 1]);
+            const float2 q = mul2(xv, y2);
+            const float2 r = fma2(q, nd2, xv);
+            const float2 q2 = fma2(r, y2, q);
+            xs[j] = q2.x;
+            xs[j + 1] = q2.y;
         }
     } else {
 #pragma unroll
         for (int j = 0; j < 16; j++) xs[j] = __fdiv_rn(x[j], d);
     }
 
+    // plain codes (ties to the smaller magnitude, 0b1000 never produced)
+    float pv[16];
+    const float2 down = make_float2(1.0f - 0x1p-24f, 1.0f - 0x1p-24f);
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+        const float2 p = mul2(make_float2(xs[j], xs[j + 1]), down);
+        pv[j] = p.x;
+        pv[j + 1] = p.y;
+    }
+    unsigned w0 = fix_codes(cvt_e2m1x8(xs), cvt_e2m1x8(pv));
+    unsigned w1 = fix_codes(cvt_e2m1x8(xs + 8), cvt_e2m1x8(pv + 8));
+
     unsigned meta = 0u;
     if constexpr (F::kSpecials > 0) {
         // v = +5 / -5: an element changes only inside (4.5, 5.5] (resp.
-        // [-5.5, -4.5)), where the error difference is |2 xs -+ 10| - 1 in
-        // [-1, 0].  2 xs -+ 10 is exact there (Sterbenz), and outside the
-        // region the clamped term is exactly 0.  Terms are multiples of
-        // 2^-20 and |sum| <= 16, so the binary32 sums are exact.
-        float dp5 = 0.0f, dn5 = 0.0f;
+        // [-5.5, -4.5)), where the squared-error difference is
+        // t = |2|xs| - 10| - 1 in [-1, 0]; outside, the clamped t is exactly 0.
+        // In the region 2|xs| - 10 is exact (Sterbenz) and t is a multiple of
+        // 2^-20.  A = sum t and B = sum copysign(t, xs) are exact binary32 sums
+        // (|A|, |B| <= 16); then the +5 sum is (A - B) / 2 and the -5 sum is
+        // (A + B) / 2, both exact.
+        float A = 0.0f, Bs = 0.0f;
 #pragma unroll
         for (int j = 0; j < 16; j++) {
-            dp5 = __fadd_rn(dp5, fminf(__fadd_rn(fabsf(__fmaf_rn(2.0f, xs[j], -10.0f)), -1.0f), 0.0f));
-            dn5 = __fadd_rn(dn5, fminf(__fadd_rn(fabsf(__fmaf_rn(2.0f, xs[j], 10.0f)), -1.0f), 0.0f));
+            const float e = __fmaf_rn(2.0f, fabsf(xs[j]), -10.0f);
+            const float t = fminf(__fadd_rn(fabsf(e), -1.0f), 0.0f);
+            A = __fadd_rn(A, t);
+            Bs = __fadd_rn(Bs, copysignf(t, xs[j]));
         }
+        const float dp5 = __fmul_rn(__fsub_rn(A, Bs), 0.5f);
+        const float dn5 = __fmul_rn(__fadd_rn(A, Bs), 0.5f);
         float best = dp5;
         if (dn5 < best) { best = dn5; meta = 1u; }
         if constexpr (F::kSpecials == 4) {
             // v = +8 / -8 changes an element only when |xs| > 7.  With a
             // normal scale code |xs| <= 6 / (1 - 2^-4) < 7, so only blocks with
             // a subnormal scale code (sc < 8) can use them; there |xs| <= 9
-            // and the terms 2*(7 - |xs|)*2 = 28 - 4|xs| are summed exactly as
-            // integers in units of 2^-20 together with the +-5 terms.
+            // and the terms are summed exactly as integers in units of 2^-20.
             if (sc < 8u) {
                 int ip5 = 0, in5 = 0, ip8 = 0, in8 = 0;
 #pragma unroll
@@ -121,26 +180,29 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], float t
             }
         }
         o.effective = best < 0.0f;
+
+        // final encode against Q_FP4 u {v*}: elements nearest to v* take
+        // 0b1000.  As binary32 bit patterns, the region of v* is one interval:
+        // +5: (4.5, 5.5], -5: [-5.5, -4.5), +8: (7, inf], -8: [-inf, -7).
+        unsigned lo, span;
+        if (meta < 2u) {
+            lo = 0x40900001u;             // just above 4.5
+            span = 0x40B00000u - lo;       // up to 5.5
+        } else {
+            lo = 0x40E00001u;              // just above 7
+            span = 0x7F800000u - lo;       // up to +inf
+        }
+        if (meta & 1u) lo |= 0x80000000u;  // negative special value
+        unsigned o0 = 0u, o1 = 0u;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            o0 |= (__float_as_uint(xs[j]) - lo <= span) ? (8u << (4 * j)) : 0u;
+            o1 |= (__float_as_uint(xs[j + 8]) - lo <= span) ? (8u << (4 * j)) : 0u;
+        }
+        w0 = (w0 & ~((o0 >> 3) * 15u)) | o0;
+        w1 = (w1 & ~((o1 >> 3) * 15u)) | o1;
     }
 
-    // final encode against Q_FP4 u {v*}
-    const float v = special_value((int)meta);
-    const float vsign = v < 0.0f ? -1.0f : 1.0f;
-    const float rlo = fabsf(v) == 5.0f ? 4.5f : 7.0f;
-    const float rhi = fabsf(v) == 5.0f ? 5.5f : 3.0e38f;
-    unsigned w0 = 0u, w1 = 0u;
-#pragma unroll
-    for (int j = 0; j < 16; j++) {
-        const float a = fabsf(xs[j]);
-        const unsigned c = e2m1_mag_code(a);
-        unsigned code = (c != 0u && xs[j] < 0.0f) ? (c | 8u) : c;
-        if constexpr (F::kSpecials > 0) {
-            const float sx = xs[j] * vsign;  // exact (multiplication by +-1)
-            if (sx > rlo && sx <= rhi) code = 8u;
-        }
-        if (j < 8) w0 |= code << (4 * j);
-        else w1 |= code << (4 * (j - 8));
-    }
     o.packed = make_uint2(w0, w1);
     o.meta = meta;
     o.sbyte = sc | (meta << F::kMetaShift);
