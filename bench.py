@@ -267,27 +267,31 @@ def main():
     wsz = max(R.razer_workspace_size(R.RAZER_OP_GEMV, B, N, K) for N, K in SHAPES for B in BATCHES)
     ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
 
-    calls = [("quantize", i, None) for i in range(len(SHAPES))] + [("gemv", i, B) for i in range(len(SHAPES)) for B in BATCHES]
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
-
-    def step(s, record=False):
+    def step(s):
         cur, prev = packed[s % 2], packed[(s + 1) % 2]
-        for ci, (kind, i, B) in enumerate(calls):
-            if record:
-                ev[ci][0].record(stream)
-            if kind == "quantize":
-                c, sc, t = cur[i]
-                R.razer_quantize_weights(W[i], "weight", codes=c, scales=sc, ts=t)
-            else:
-                c, sc, t = prev[i]
+        for i in range(len(SHAPES)):
+            c, sc, t = cur[i]
+            R.razer_quantize_weights(W[i], "weight", codes=c, scales=sc, ts=t)
+        for i in range(len(SHAPES)):
+            c, sc, t = prev[i]
+            for B in BATCHES:
                 R.razer_gemv(X[B][i], c, sc, t, "weight", torch.float16, out=Y[B][i], workspace=ws)
-            if record:
-                ev[ci][1].record(stream)
 
-    # the first GEMVs read the second packed set: fill it
+    # the first GEMVs read the second packed set: fill it; warm every path
     step(1)
     for s in range(args.warmup):
         step(s)
+    torch.cuda.synchronize()
+    # one CUDA graph per step parity (the launches of a step replay without
+    # host overhead; the work inside is unchanged)
+    graphs = []
+    for par in range(2):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(par)
+        graphs.append(g)
+    for s in range(3):
+        graphs[s % 2].replay()
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
@@ -298,9 +302,9 @@ def main():
         t_end = time.time() + (0.0 if args.no_soak else 1.5)
         s = 0
         while time.time() < t_end:
-            step(s)
+            graphs[s % 2].replay()
             s += 1
-            if s % 8 == 0:
+            if s % 16 == 0:
                 torch.cuda.synchronize()
         torch.cuda.synchronize()
         if pg:
@@ -310,7 +314,7 @@ def main():
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for s in range(args.steps):
-            step(s)
+            graphs[s % 2].replay()
         t1.record(stream)
         torch.cuda.synchronize()
     elapsed_ms = t0.elapsed_time(t1)
@@ -322,35 +326,50 @@ def main():
     ms_per_step = elapsed_ms / args.steps
     value = step_bytes() * args.steps * world / (elapsed_ms / 1e3) / 1e9
 
-    # per-call timing (its own loop, so the events do not perturb the step)
-    breakdown = {}
-    times = {c: [] for c in calls}
-    for s in range(max(3, min(args.steps, 10))):
-        step(s, record=True)
-        torch.cuda.synchronize()
-        for ci, c in enumerate(calls):
-            times[c].append(ev[ci][0].elapsed_time(ev[ci][1]))
-    tot_q = tot_g = 0.0
-    by_kind = {}
-    for (kind, i, B), ts_ in times.items():
-        N, K = SHAPES[i]
-        ms = statistics.median(ts_)
-        nb = quant_bytes(N, K) if kind == "quantize" else gemv_bytes(B, N, K)
-        key = f"{kind}_{N}x{K}" + ("" if B is None else f"_b{B}")
-        breakdown[key] = {"ms": ms, "GB/s": nb / ms / 1e6}
-        by_kind.setdefault(kind, [0.0, 0.0])
-        by_kind[kind][0] += ms
-        by_kind[kind][1] += nb
+    # per-call device time: a graph of back-to-back calls of one kind, each on
+    # its own copy of the operands so that the copies together exceed L2
+    l2 = 126 * 2 ** 20
+    breakdown, by_kind = {}, {}
+    for i, (N, K) in enumerate(SHAPES):
+        ncopy = max(2, -(-2 * l2 // (N * K * 2)))
+        Wc = [W[i]] + [W[i].clone() for _ in range(ncopy - 1)]
+        outs = [(torch.empty_like(packed[0][i][0]), torch.empty_like(packed[0][i][1]), torch.empty_like(packed[0][i][2]))
+                for _ in range(ncopy)]
+        for r in range(ncopy):
+            R.razer_quantize_weights(Wc[r], "weight", codes=outs[r][0], scales=outs[r][1], ts=outs[r][2])
+        ms = time_graph(lambda: [R.razer_quantize_weights(Wc[r], "weight", codes=outs[r][0], scales=outs[r][1], ts=outs[r][2])
+                                 for r in range(ncopy)], ncopy, stream)
+        nb = quant_bytes(N, K)
+        breakdown[f"quantize_{N}x{K}"] = {"ms": ms, "GB/s": nb / ms / 1e6}
+        by_kind.setdefault("quantize", [0.0, 0.0, 0])
+        by_kind["quantize"][0] += ms
+        by_kind["quantize"][1] += nb
+        by_kind["quantize"][2] += 1
+        del Wc
+        npk = max(2, -(-2 * l2 // (N * K * 9 // 16)))
+        pk = [outs[r % len(outs)] for r in range(npk)]
+        pk = [(c.clone(), sc.clone(), t.clone()) for (c, sc, t) in pk]
+        for B in BATCHES:
+            ms = time_graph(lambda: [R.razer_gemv(X[B][i], *pk[r], "weight", torch.float16, out=Y[B][i], workspace=ws)
+                                     for r in range(npk)], npk, stream)
+            nb = gemv_bytes(B, N, K)
+            breakdown[f"gemv_{N}x{K}_b{B}"] = {"ms": ms, "GB/s": nb / ms / 1e6}
+            by_kind.setdefault("gemv", [0.0, 0.0, 0])
+            by_kind["gemv"][0] += ms
+            by_kind["gemv"][1] += nb
+            by_kind["gemv"][2] += 1
+        del pk, outs
+    torch.cuda.empty_cache()
     dominant = max(by_kind, key=lambda k: by_kind[k][0])
-    dom_ms, dom_bytes = by_kind[dominant]
-    n_calls = len(SHAPES) if dominant == "quantize" else len(SHAPES) * len(BATCHES)
-    achieved = dom_bytes / dom_ms / 1e6  # GB/s, average over that kind's launches
+    dom_ms, dom_bytes, n_calls = by_kind[dominant]
+    achieved = dom_bytes / dom_ms / 1e6  # GB/s over that kind's calls
     kname = "quantize_kernel" if dominant == "quantize" else "gemv_kernel"
     traffic = traffic_for(kname)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": traffic, "kernel": ("razer_quantize_weights (amax + quantize kernels)" if dominant == "quantize"
                                                else "razer_gemv (gemv + split-K reduce kernels)"),
-                "algorithmic_bytes_per_call": dom_bytes / n_calls, "peak_source": peak_src}
+                "algorithmic_bytes_per_call": dom_bytes / n_calls, "peak_source": peak_src,
+                "timing": "CUDA events around CUDA-graph replays of back-to-back calls on operand copies larger than L2"}
 
     extras = {}
     if not args.no_extras and rank == 0:
@@ -445,6 +464,30 @@ def run_single_kernel(args):
                       "ms_per_call": e0.elapsed_time(e1) / args.iters}), flush=True)
 
 
+def time_graph(fn, ncalls, stream, reps=5):
+    """Median device time of one call: fn() issues `ncalls` calls; they are
+    captured into one CUDA graph, replayed `reps` times between events."""
+    import torch
+
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(reps):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / ncalls)
+    del g
+    return statistics.median(times)
+
+
 def run_extras(R, workloads, dev, stream, hbm, bf16):
     import torch
 
@@ -455,16 +498,9 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
     scales = torch.empty((2048, 256), dtype=torch.uint8, device=dev)
     ts = torch.empty(1, dtype=torch.float32, device=dev)
     hist = torch.empty(4, dtype=torch.int64, device=dev)
-    for i in range(3):
-        R.razer_quantize_acts(Xa[i], None, "act", codes=codes, scales=scales, ts_out=ts, meta_hist=hist)
+    ms = time_graph(lambda: [R.razer_quantize_acts(Xa[r], None, "act", codes=codes, scales=scales, ts_out=ts, meta_hist=hist)
+                             for r in range(8)], 8, stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 40
-    e0.record(stream)
-    for r in range(reps):
-        R.razer_quantize_acts(Xa[r % 8], None, "act", codes=codes, scales=scales, ts_out=ts, meta_hist=hist)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
     n = 2048 * 4096
     h = hist.cpu().tolist()
     nblk = n // 16

@@ -116,7 +116,7 @@ __device__ __forceinline__ void scale_pairs2(unsigned sb, unsigned (&s2)[2], uns
 #pragma unroll
         for (int b = 0; b < 2; b++) {
             const unsigned meta = (x >> (16 * b + Fmt<FMT>::kMetaShift)) & 3u;
-            v2[b] = prmt(kVHigh, 0u, 0x4040u + meta * 0x1010u);
+            v2[b] = prmt(kVHigh, 0u, 0x0404u + meta * 0x1010u);  // bytes: 0, table[meta], 0, table[meta]
         }
     } else {
         v2[0] = v2[1] = 0u;
