@@ -163,16 +163,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ unsigned cvt_e2m1x2(unsigned w)
+template <int L>
+__device__ __forceinline__ unsigned cvt_lane(unsigned w)
 {
     unsigned r;
-    asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b0; }" : "=r"(r) : "r"(w));
-    return r;
-}
-__device__ __forceinline__ unsigned prmt(unsigned a, unsigned b, unsigned sel)
-{
-    unsigned r;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    if constexpr (L == 0) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b0; }" : "=r"(r) : "r"(w));
+    if constexpr (L == 1) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b1; }" : "=r"(r) : "r"(w));
+    if constexpr (L == 2) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b2; }" : "=r"(r) : "r"(w));
+    if constexpr (L == 3) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b3; }" : "=r"(r) : "r"(w));
     return r;
 }
 __device__ __forceinline__ unsigned hmul2(unsigned a, unsigned b)
@@ -181,60 +179,62 @@ __device__ __forceinline__ unsigned hmul2(unsigned a, unsigned b)
     asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
+__device__ __forceinline__ unsigned hfma2(unsigned a, unsigned b, unsigned c)
+{
+    unsigned r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
 
-// Per-block decode constants of one scale byte.
+// Per-block decode constants of one scale byte (fp16 pairs).
 struct BlockK {
-    unsigned s16x2;  // fp16 pair of s * 2^-bias (fp16 path)
-    float s32;       // exact s (bf16 path)
-    unsigned v16x2;  // fp16 pair of v (0 when the format has no remap)
+    unsigned s2;   // s * 2^-bias
+    unsigned vs2;  // v * s * 2^-bias (0 when the format has no remap)
 };
 
-template <int FMT, bool BF16>
+template <int FMT>
 __device__ __forceinline__ BlockK block_consts(unsigned sb)
 {
     BlockK k;
-    {
-        const unsigned s16 = scale_f16_bits<FMT>(sb);  // s * 2^-12 (E3M3) or s * 2^-8 (E4M3)
-        k.s16x2 = hmul2(s16 | (s16 << 16), 0x4C004C00u);  // * 16 (exact): keeps q*s in the fp16 normal range
-        k.s32 = 0.0f;
-    }
+    const unsigned s16 = scale_f16_bits<FMT>(sb);        // s * 2^-12 (E3M3) or s * 2^-8 (E4M3)
+    k.s2 = hmul2(s16 | (s16 << 16), 0x4C004C00u);       // * 16 (exact): keeps q*s in the fp16 normal range
     if constexpr (Fmt<FMT>::kSpecials > 0) {
         const unsigned meta = sb >> Fmt<FMT>::kMetaShift;
         const unsigned v16 = ((meta & 2u) ? 0x4800u : 0x4500u) | ((meta & 1u) << 15);
-        k.v16x2 = v16 | (v16 << 16);
+        k.vs2 = hmul2(v16 | (v16 << 16), k.s2);
     } else {
-        k.v16x2 = 0u;
+        k.vs2 = 0u;
     }
     return k;
 }
 
-// Decode one 32-bit word (8 codes of one block) into 4 packed 16-bit pairs.
+// Decode one 32-bit word (8 codes of one block) into 4 packed 16-bit pairs of
+// q*s*2^-bias.  The redundant-zero codes (converted to -0) receive v*s through
+// the convert of an indicator word (code of 1.0 where the code is 0b1000)
+// folded in with a packed FMA.
 template <int FMT, bool BF16>
 __device__ __forceinline__ uint4 decode_word(unsigned w, const BlockK &k)
 {
-    // bit 3 of each nibble set where the code is 0b1000 (the redundant zero)
-    const unsigned is8 = w & ~((w & 0x77777777u) + 0x77777777u) & 0x88888888u;
-    const unsigned is8s = is8 << 4;
-    unsigned out[4];
+    unsigned p[4] = {cvt_lane<0>(w), cvt_lane<1>(w), cvt_lane<2>(w), cvt_lane<3>(w)};
+    if constexpr (Fmt<FMT>::kSpecials > 0) {
+        const unsigned t = (w & 0x77777777u) + 0x77777777u;
+        const unsigned ind = __umulhi(w & ~t & 0x88888888u, 0x40000000u);  // nibble 0b0010 where the code is 0b1000
+        const unsigned i[4] = {cvt_lane<0>(ind), cvt_lane<1>(ind), cvt_lane<2>(ind), cvt_lane<3>(ind)};
 #pragma unroll
-    for (int b = 0; b < 4; b++) {
-        unsigned q = cvt_e2m1x2(w >> (8 * b));
-        if constexpr (Fmt<FMT>::kSpecials > 0) {
-            // 0xFFFF in each half whose code is 0b1000, from the nibble sign bits
-            const unsigned sel = (0x88CCu + 0x1111u * (unsigned)b);
-            const unsigned mask = prmt(is8, is8s, sel);
-            q = (q & ~mask) | (k.v16x2 & mask);
-        }
-        const unsigned p = hmul2(q, k.s16x2);  // exact q*s*2^-bias in fp16
-        if constexpr (BF16) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&p));
+        for (int b = 0; b < 4; b++) p[b] = hfma2(i[b], k.vs2, hmul2(p[b], k.s2));
+    } else {
+#pragma unroll
+        for (int b = 0; b < 4; b++) p[b] = hmul2(p[b], k.s2);
+    }
+    if constexpr (BF16) {
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&p[b]));
             __nv_bfloat162 h2 = __floats2bfloat162_rn(f.x, f.y);  // exact
-            out[b] = *reinterpret_cast<unsigned *>(&h2);
-        } else {
-            out[b] = p;
+            p[b] = *reinterpret_cast<unsigned *>(&h2);
         }
     }
-    return make_uint4(out[0], out[1], out[2], out[3]);
+    return make_uint4(p[0], p[1], p[2], p[3]);
 }
 
 template <int FMT, bool BF16>
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const unsigned words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
             for (int blk = 0; blk < 4; blk++) {
-                const BlockK kc = block_consts<FMT, BF16>((cs >> (8 * blk)) & 0xFFu);
+                const BlockK kc = block_consts<FMT>((cs >> (8 * blk)) & 0xFFu);
 #pragma unroll
                 for (int h = 0; h < 2; h++) {
                     const int j = 2 * blk + h;  // 16-byte chunk = 8 elements

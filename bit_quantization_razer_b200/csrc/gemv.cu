@@ -10,10 +10,11 @@
 //     slice of codes with one 128-bit load per thread per row (64 contiguous
 //     bytes per row, 4 lanes per row), plus the matching scale bytes;
 //   * each code byte becomes one f16x2 pair with the hardware E2M1 convert;
-//     the redundant-zero codes are replaced by the block's special value with
-//     a byte permute (sign replication of the nibble's bit 3) and one bitwise
-//     select, and the block scale is applied with a packed multiply --
-//     q*s*2^-12 (E3M3) or q*s*2^-8 (E4M3) is exact in fp16;
+//     the redundant-zero codes receive v*s through the convert of an
+//     indicator word folded in with one packed FMA, and the block scale is a
+//     packed multiply -- q*s*2^-12 (E3M3) or q*s*2^-8 (E4M3) is exact in fp16
+//     (the integer / convert work runs on the half-rate ALU pipe, which bounds
+//     this kernel, so the decode keeps it to 11 operations per 8 codes);
 //   * the decoded pairs are already in the register layout of the A operand of
 //     the warp-level m16n8k16 tensor-core MMA, so the products accumulate in
 //     fp32 without any shared-memory round trip; the activations form the
@@ -30,10 +31,23 @@ namespace razer {
 constexpr int kGemvWarps = 4;
 constexpr int kGemvThreads = kGemvWarps * 32;
 
-__device__ __forceinline__ unsigned cvt_e2m1x2_f16x2(unsigned byte_in_low8)
+// E2M1 pair -> f16x2 of byte lane L of w (the convert reads the byte lane
+// directly, no shift).
+template <int L>
+__device__ __forceinline__ unsigned cvt_lane(unsigned w)
 {
     unsigned r;
-    asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b0; }" : "=r"(r) : "r"(byte_in_low8));
+    if constexpr (L == 0) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b0; }" : "=r"(r) : "r"(w));
+    if constexpr (L == 1) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b1; }" : "=r"(r) : "r"(w));
+    if constexpr (L == 2) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b2; }" : "=r"(r) : "r"(w));
+    if constexpr (L == 3) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b3; }" : "=r"(r) : "r"(w));
+    return r;
+}
+
+__device__ __forceinline__ unsigned hfma2u(unsigned a, unsigned b, unsigned c)
+{
+    unsigned r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
     return r;
 }
 
@@ -64,25 +78,31 @@ __device__ __forceinline__ unsigned prmt(unsigned a, unsigned b, unsigned sel)
 
 // Decode 8 codes of one block (a 32-bit word) into 4 packed pairs of
 // (q * s * 2^-bias): pair b holds nibbles 2b (low half) and 2b+1.  The
-// 0b1000 codes become v: bit 3 of each such nibble is spread over its 16-bit
-// half with a byte permute (sign replication) and selects v's fp16 pattern.
+// redundant-zero codes (0b1000, converted to -0) receive v*s through a
+// second conversion of an indicator word holding the code of 1.0 (0b0010)
+// exactly where the code is 0b1000, folded in with one packed FMA.  Integer
+// and conversion work shares the half-rate ALU pipe, so the indicator shift
+// is a high multiply (FMA pipe) and the converts read byte lanes directly.
 template <int FMT, bool BF16>
-__device__ __forceinline__ void decode_word(unsigned w, unsigned s2, unsigned v2, unsigned (&h)[4])
+__device__ __forceinline__ void decode_word(unsigned w, unsigned s2, unsigned vs2, unsigned (&h)[4])
 {
-    unsigned is8 = 0u, is8s = 0u;
+    unsigned q[4] = {cvt_lane<0>(w), cvt_lane<1>(w), cvt_lane<2>(w), cvt_lane<3>(w)};
     if constexpr (Fmt<FMT>::kSpecials > 0) {
-        is8 = w & ~((w & 0x77777777u) + 0x77777777u) & 0x88888888u;
-        is8s = is8 << 4;
-    }
+        const unsigned t = (w & 0x77777777u) + 0x77777777u;       // bit 3 set where the magnitude is non-zero
+        const unsigned is8 = w & ~t & 0x88888888u;                 // bit 3 set where the code is 0b1000
+        const unsigned ind = __umulhi(is8, 0x40000000u);          // is8 >> 2: nibble 0b0010 (= 1.0)
+        const unsigned i[4] = {cvt_lane<0>(ind), cvt_lane<1>(ind), cvt_lane<2>(ind), cvt_lane<3>(ind)};
 #pragma unroll
-    for (int b = 0; b < 4; b++) {
-        unsigned q = cvt_e2m1x2_f16x2(w >> (8 * b));
-        if constexpr (Fmt<FMT>::kSpecials > 0) {
-            const unsigned m = prmt(is8, is8s, 0x88CCu + 0x1111u * (unsigned)b);
-            q = (q & ~m) | (v2 & m);
+        for (int b = 0; b < 4; b++) {
+            const unsigned r = hfma2u(i[b], vs2, hmul2u(q[b], s2));
+            h[b] = BF16 ? f16x2_to_bf16x2(r) : r;
         }
-        const unsigned r = hmul2u(q, s2);
-        h[b] = BF16 ? f16x2_to_bf16x2(r) : r;
+    } else {
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+            const unsigned r = hmul2u(q[b], s2);
+            h[b] = BF16 ? f16x2_to_bf16x2(r) : r;
+        }
     }
 }
 
@@ -100,8 +120,8 @@ __device__ __forceinline__ void mma16816(float (&d)[4], unsigned a0, unsigned a1
     }
 }
 
-// fp16 scale pairs and special-value pairs of the two blocks held in the low
-// 16 bits of sb (one scale byte per block).
+// fp16 pairs of s * 2^-bias and of v * s * 2^-bias for the two blocks held in
+// the low 16 bits of sb (one scale byte per block).
 template <int FMT>
 __device__ __forceinline__ void scale_pairs2(unsigned sb, unsigned (&s2)[2], unsigned (&v2)[2])
 {
@@ -116,7 +136,7 @@ __device__ __forceinline__ void scale_pairs2(unsigned sb, unsigned (&s2)[2], uns
 #pragma unroll
         for (int b = 0; b < 2; b++) {
             const unsigned meta = (x >> (16 * b + Fmt<FMT>::kMetaShift)) & 3u;
-            v2[b] = prmt(kVHigh, 0u, 0x0404u + meta * 0x1010u);  // bytes: 0, table[meta], 0, table[meta]
+            v2[b] = hmul2u(prmt(kVHigh, 0u, 0x0404u + meta * 0x1010u), s2[b]);  // fp16 pair of v * s * 2^-bias
         }
     } else {
         v2[0] = v2[1] = 0u;

@@ -182,22 +182,31 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], float t
         o.effective = best < 0.0f;
 
         // final encode against Q_FP4 u {v*}: elements nearest to v* take
-        // 0b1000.  As binary32 bit patterns, the region of v* is one interval:
-        // +5: (4.5, 5.5], -5: [-5.5, -4.5), +8: (7, inf], -8: [-inf, -7).
-        unsigned lo, span;
-        if (meta < 2u) {
-            lo = 0x40900001u;             // just above 4.5
-            span = 0x40B00000u - lo;       // up to 5.5
-        } else {
-            lo = 0x40E00001u;              // just above 7
-            span = 0x7F800000u - lo;       // up to +inf
-        }
-        if (meta & 1u) lo |= 0x80000000u;  // negative special value
+        // 0b1000.  For v* = +-5 the region is e = 2 xs - 2 v* in (-1, 1]
+        // (xs in (4.5, 5.5] resp. [-5.5, -4.5)); there e is an exact multiple
+        // of 2^-20, so the test is |e - 2^-22| < 1, i.e. the sign bit of
+        // r = |e - 2^-22| - 1.  The sign bits are gathered into the nibble
+        // mask with integer multiply-adds, keeping this pass off the
+        // half-rate ALU pipe.
         unsigned o0 = 0u, o1 = 0u;
+        if (meta < 2u) {
+            const float two_v = (meta & 1u) ? -10.0f : 10.0f;
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-            o0 |= (__float_as_uint(xs[j]) - lo <= span) ? (8u << (4 * j)) : 0u;
-            o1 |= (__float_as_uint(xs[j + 8]) - lo <= span) ? (8u << (4 * j)) : 0u;
+            for (int j = 0; j < 16; j++) {
+                const float e = __fmaf_rn(2.0f, xs[j], -two_v);
+                const float r = __fadd_rn(fabsf(__fadd_rn(e, -0x1p-22f)), -1.0f);
+                const unsigned neg = __umulhi(__float_as_uint(r), 2u);  // sign bit of r
+                if (j < 8) o0 = neg * (8u << (4 * j)) + o0;
+                else o1 = neg * (8u << (4 * (j - 8))) + o1;
+            }
+        } else {
+            // +8 (7, inf] / -8 [-inf, -7): one interval of bit patterns each
+            const unsigned lo = 0x40E00001u | ((meta & 1u) << 31), span = 0x7F800000u - 0x40E00001u;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                o0 |= (__float_as_uint(xs[j]) - lo <= span) ? (8u << (4 * j)) : 0u;
+                o1 |= (__float_as_uint(xs[j + 8]) - lo <= span) ? (8u << (4 * j)) : 0u;
+            }
         }
         w0 = (w0 & ~((o0 >> 3) * 15u)) | o0;
         w1 = (w1 & ~((o1 >> 3) * 15u)) | o1;
