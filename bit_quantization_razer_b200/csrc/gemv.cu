@@ -6,9 +6,11 @@
 // 148 SMs of a B200).
 //
 // Design (HBM-bound: 0.5625 byte of weights per multiply-add at B = 1):
-//   * a warp owns 16 weight rows; each step it streams a 16-row x 128-k
-//     slice of codes with one 128-bit load per thread per row (64 contiguous
-//     bytes per row, 4 lanes per row), plus the matching scale bytes;
+//   * a warp owns 16 weight rows; each step consumes a 16-row x 128-k slice of
+//     codes (64 contiguous bytes per row, 4 lanes per row) plus the matching
+//     scale bytes, streamed through a 4-stage per-warp shared-memory ring with
+//     16-byte cp.async copies, so three slices per warp are in flight without
+//     holding registers;
 //   * each code byte becomes one f16x2 pair with the hardware E2M1 convert;
 //     the redundant-zero codes receive v*s through the convert of an
 //     indicator word folded in with one packed FMA, and the block scale is a
@@ -143,11 +145,29 @@ __device__ __forceinline__ void scale_pairs2(unsigned sb, unsigned (&s2)[2], uns
     }
 }
 
+constexpr int kRing = 4;                          // stages per warp ring
+constexpr int kCodeBytes = 16 * 64;               // 16 rows x 64 bytes per chunk
+constexpr int kScaleBytes = 16 * 8;               // 16 rows x 8 scale bytes
+constexpr int kStageBytes = kCodeBytes + kScaleBytes;
+constexpr int kGemvSmem = kGemvWarps * kRing * kStageBytes;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int FMT, bool BF16, int NB>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__restrict__ x, int B, const uint8_t *__restrict__ codes,
                                                             const uint8_t *__restrict__ scales, int N, int K, int S,
                                                             float *__restrict__ ws)
 {
+    extern __shared__ __align__(16) uint8_t gemv_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int row0 = (blockIdx.x * kGemvWarps + warp) * 16;
     if (row0 >= N) return;
@@ -157,32 +177,49 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
     const int rA = min(row0 + g, N - 1), rB = min(row0 + g + 8, N - 1);
     const uint8_t *pa = codes + (size_t)rA * (K >> 1) + 16 * t;
     const uint8_t *pb = codes + (size_t)rB * (K >> 1) + 16 * t;
-    const uint8_t *sa = scales + (size_t)rA * (K >> 4) + 2 * t;
-    const uint8_t *sbp = scales + (size_t)rB * (K >> 4) + 2 * t;
+    const uint8_t *sa = scales + (size_t)rA * (K >> 4);
+    const uint8_t *sbp = scales + (size_t)rB * (K >> 4);
+
+    // this warp's ring: stage = [16 rows x 64 B of codes][16 rows x 8 B of scales]
+    uint8_t *ring = gemv_smem + warp * (kRing * kStageBytes);
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    auto issue = [&](int c, int slot) {
+        if (c < c_end) {
+            const uint32_t st = ring_s + slot * kStageBytes;
+            cp_async16(st + g * 64 + 16 * t, pa + (size_t)c * 64);
+            cp_async16(st + (g + 8) * 64 + 16 * t, pb + (size_t)c * 64);
+            if (t < 2) {  // 8 scale bytes per row (scales are only 4-byte aligned)
+                cp_async4(st + kCodeBytes + g * 8 + 4 * t, sa + (size_t)c * 8 + 4 * t);
+                cp_async4(st + kCodeBytes + (g + 8) * 8 + 4 * t, sbp + (size_t)c * 8 + 4 * t);
+            }
+        }
+        cp_async_commit();  // one group per chunk (possibly empty) keeps the counting uniform
+    };
 
     float acc[NB][4];
 #pragma unroll
     for (int j = 0; j < NB; j++) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
 
-    uint4 na = make_uint4(0u, 0u, 0u, 0u), nb = na;
-    unsigned nsA = 0u, nsB = 0u;
-    auto load = [&](int c) {
-        na = ldg_stream(pa + (size_t)c * 64);
-        nb = ldg_stream(pb + (size_t)c * 64);
-        nsA = *reinterpret_cast<const unsigned short *>(sa + (size_t)c * 8);
-        nsB = *reinterpret_cast<const unsigned short *>(sbp + (size_t)c * 8);
-    };
-    if (c_begin < c_end) load(c_begin);
+#pragma unroll
+    for (int i = 0; i < kRing - 1; i++) issue(c_begin + i, i);
     for (int c = c_begin; c < c_end; c++) {
-        const uint4 ca = na, cb = nb;
-        const unsigned sA = nsA, sB = nsB;
-        if (c + 1 < c_end) load(c + 1);  // one chunk of codes in flight ahead
+        const int i = c - c_begin;
+        __syncwarp();  // every lane is done with the slot refilled next
+        issue(c + kRing - 1, (i + kRing - 1) % kRing);
+        cp_async_wait<kRing - 1>();  // this chunk's group has landed
+        __syncwarp();                // scale bytes were copied by lanes t < 2 of each row group
+        const uint8_t *st = ring + (i % kRing) * kStageBytes;
+        const uint4 ca = *reinterpret_cast<const uint4 *>(st + g * 64 + 16 * t);
+        const uint4 cb = *reinterpret_cast<const uint4 *>(st + (g + 8) * 64 + 16 * t);
+        const unsigned sA = *reinterpret_cast<const unsigned short *>(st + kCodeBytes + g * 8 + 2 * t);
+        const unsigned sB = *reinterpret_cast<const unsigned short *>(st + kCodeBytes + (g + 8) * 8 + 2 * t);
         unsigned xw[NB][16];
 #pragma unroll
         for (int j = 0; j < NB; j++) {
             const int n = 8 * j + g;
             if (n < B) {
                 const uint4 *px = reinterpret_cast<const uint4 *>(x + (size_t)n * K + (size_t)c * 128 + 32 * t);
+                if (c + 1 < c_end) asm volatile("prefetch.global.L1 [%0];" ::"l"(px + 16));  // next chunk's activations
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
                     const uint4 v = __ldg(px + q);
@@ -213,6 +250,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
             }
         }
     }
+    cp_async_wait<0>();
 
     // partials: D[g][2t..2t+1] -> rows row0+g, D[g+8][..] -> rows row0+g+8
     float *wsb = ws + (size_t)s * B * N;
@@ -276,9 +314,9 @@ static void launch_gemv_fmt(const void *x, int B, const uint8_t *codes, const ui
 {
     dim3 grid((unsigned)(((N + 15) / 16 + kGemvWarps - 1) / kGemvWarps), (unsigned)S);
     const uint16_t *xp = reinterpret_cast<const uint16_t *>(x);
-    if (B <= 8) gemv_kernel<FMT, BF16, 1><<<grid, kGemvThreads, 0, st>>>(xp, B, codes, scales, N, K, S, ws);
-    else if (B <= 16) gemv_kernel<FMT, BF16, 2><<<grid, kGemvThreads, 0, st>>>(xp, B, codes, scales, N, K, S, ws);
-    else gemv_kernel<FMT, BF16, 4><<<grid, kGemvThreads, 0, st>>>(xp, B, codes, scales, N, K, S, ws);
+    if (B <= 8) gemv_kernel<FMT, BF16, 1><<<grid, kGemvThreads, kGemvSmem, st>>>(xp, B, codes, scales, N, K, S, ws);
+    else if (B <= 16) gemv_kernel<FMT, BF16, 2><<<grid, kGemvThreads, kGemvSmem, st>>>(xp, B, codes, scales, N, K, S, ws);
+    else gemv_kernel<FMT, BF16, 4><<<grid, kGemvThreads, kGemvSmem, st>>>(xp, B, codes, scales, N, K, S, ws);
 }
 
 razer_status run_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,

@@ -182,19 +182,21 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], float t
         o.effective = best < 0.0f;
 
         // final encode against Q_FP4 u {v*}: elements nearest to v* take
-        // 0b1000.  For v* = +-5 the region is e = 2 xs - 2 v* in (-1, 1]
-        // (xs in (4.5, 5.5] resp. [-5.5, -4.5)); there e is an exact multiple
-        // of 2^-20, so the test is |e - 2^-22| < 1, i.e. the sign bit of
-        // r = |e - 2^-22| - 1.  The sign bits are gathered into the nibble
-        // mask with integer multiply-adds, keeping this pass off the
-        // half-rate ALU pipe.
+        // 0b1000.  For v* = +5 the region is xs in (4.5, 5.5], i.e.
+        // e = 2 xs - 10 in (-1, 1]; for v* = -5 it is [-5.5, -4.5), i.e.
+        // e = 2 xs + 10 in [-1, 1) (ties go to the smaller magnitude).  There e
+        // is an exact multiple of 2^-20, so the test is |e -+ 2^-22| < 1, the
+        // sign bit of r = |e -+ 2^-22| - 1.  The sign bits are gathered into
+        // the nibble mask with integer multiply-adds, keeping this pass off
+        // the half-rate ALU pipe.
         unsigned o0 = 0u, o1 = 0u;
         if (meta < 2u) {
             const float two_v = (meta & 1u) ? -10.0f : 10.0f;
+            const float nudge = (meta & 1u) ? 0x1p-22f : -0x1p-22f;
 #pragma unroll
             for (int j = 0; j < 16; j++) {
                 const float e = __fmaf_rn(2.0f, xs[j], -two_v);
-                const float r = __fadd_rn(fabsf(__fadd_rn(e, -0x1p-22f)), -1.0f);
+                const float r = __fadd_rn(fabsf(__fadd_rn(e, nudge)), -1.0f);
                 const unsigned neg = __umulhi(__float_as_uint(r), 2u);  // sign bit of r
                 if (j < 8) o0 = neg * (8u << (4 * j)) + o0;
                 else o1 = neg * (8u << (4 * (j - 8))) + o1;
