@@ -128,18 +128,18 @@ template <int FMT>
 __device__ __forceinline__ void scale_pairs2(unsigned sb, unsigned (&s2)[2], unsigned (&v2)[2])
 {
     const unsigned x = prmt(sb, 0u, 0x4140u);  // 16-bit lanes: byte 0, byte 1
-    const unsigned mag = Fmt<FMT>::kMagMask * 0x10001u;
-    const unsigned sx = (x & mag) << 7;         // fp16 of s * 2^-12 (E3M3) or s * 2^-8 (E4M3)
+    const unsigned sx = (x & (Fmt<FMT>::kMagMask * 0x10001u)) << 7;  // fp16 [s0, s1] * 2^-12 (E3M3) / 2^-8 (E4M3)
     s2[0] = prmt(sx, 0u, 0x1010u);
     s2[1] = prmt(sx, 0u, 0x3232u);
     if constexpr (Fmt<FMT>::kSpecials > 0) {
-        // fp16 high bytes of +5, -5, +8, -8 indexed by the meta value
+        // fp16 high bytes of +5, -5, +8, -8 indexed by the meta value; one
+        // permute builds [v0, v1] for both blocks
         constexpr unsigned kVHigh = 0xC848C545u;
-#pragma unroll
-        for (int b = 0; b < 2; b++) {
-            const unsigned meta = (x >> (16 * b + Fmt<FMT>::kMetaShift)) & 3u;
-            v2[b] = hmul2u(prmt(kVHigh, 0u, 0x0404u + meta * 0x1010u), s2[b]);  // fp16 pair of v * s * 2^-bias
-        }
+        const unsigned m = (x >> Fmt<FMT>::kMetaShift) & 0x00030003u;  // meta0 | meta1 << 16
+        const unsigned sel = 0x0404u | ((m & 3u) << 4) | ((m >> 16) << 12);
+        const unsigned vs = hmul2u(prmt(kVHigh, 0u, sel), sx);          // [v0 * s0, v1 * s1]
+        v2[0] = prmt(vs, 0u, 0x1010u);
+        v2[1] = prmt(vs, 0u, 0x3232u);
     } else {
         v2[0] = v2[1] = 0u;
     }
@@ -200,6 +200,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
 #pragma unroll
     for (int j = 0; j < NB; j++) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
 
+    unsigned xw[NB][16];
+#pragma unroll
+    for (int j = 0; j < NB; j++)
+#pragma unroll
+        for (int q = 0; q < 16; q++) xw[j][q] = 0u;
+
 #pragma unroll
     for (int i = 0; i < kRing - 1; i++) issue(c_begin + i, i);
     for (int c = c_begin; c < c_end; c++) {
@@ -213,12 +219,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
         const uint4 cb = *reinterpret_cast<const uint4 *>(st + (g + 8) * 64 + 16 * t);
         const unsigned sA = *reinterpret_cast<const unsigned short *>(st + kCodeBytes + g * 8 + 2 * t);
         const unsigned sB = *reinterpret_cast<const unsigned short *>(st + kCodeBytes + (g + 8) * 8 + 2 * t);
-        unsigned xw[NB][16];
 #pragma unroll
         for (int j = 0; j < NB; j++) {
-            const int n = 8 * j + g;
-            if (n < B) {
-                const uint4 *px = reinterpret_cast<const uint4 *>(x + (size_t)n * K + (size_t)c * 128 + 32 * t);
+            if (8 * j + g < B) {  // lanes past the batch keep their zero fragments
+                const uint4 *px = reinterpret_cast<const uint4 *>(x + (size_t)(8 * j + g) * K + (size_t)c * 128 + 32 * t);
                 if (c + 1 < c_end) asm volatile("prefetch.global.L1 [%0];" ::"l"(px + 16));  // next chunk's activations
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
@@ -228,9 +232,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
                     xw[j][4 * q + 2] = v.z;
                     xw[j][4 * q + 3] = v.w;
                 }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 16; q++) xw[j][q] = 0u;
             }
         }
         unsigned s2A[2], vA[2], s2B[2], vB[2];
