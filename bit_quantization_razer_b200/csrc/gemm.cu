@@ -10,8 +10,8 @@
 //     per 256 activation rows (half the decode work per SM of a 128-row tile).
 //   * warp 0: TMA producer of the X tiles (K-major, 128-byte swizzle);
 //     warp 1: TMEM allocator and the single MMA-issuing thread;
-//     warps 2-9: decoders, one weight row per thread, two warps per scheduler
-//     -- they stream the packed codes and scale bytes with
+//     warps 2-17: decoders, half a weight row per thread, four warps per
+//     scheduler (decode is latency-bound) -- they stream the codes and scales with
 //     128-bit loads (one stage ahead), decode to 16-bit q*s and write the
 //     UMMA canonical K-major 128B-swizzled layout with 16-byte stores; after
 //     the k loop they are the epilogue (tcgen05.ld, * ts, convert, store).
@@ -32,7 +32,7 @@ namespace razer {
 namespace gemm {
 
 constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
-constexpr int kDecodeWarps = 8;  // two per scheduler
+constexpr int kDecodeWarps = 16;  // four per scheduler; each thread decodes half a weight row
 constexpr int kThreads = 64 + 32 * kDecodeWarps;
 constexpr uint32_t A_HALF_BYTES = 128 * BK * 2;               // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;                     // 32 KB
@@ -332,24 +332,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- decoders, then epilogue ----------------
-        const int row = threadIdx.x - 64;  // 0..255: one weight row per thread
+        const int row = (threadIdx.x - 64) & (BN - 1);  // 0..255
+        const int hk = (threadIdx.x - 64) >> 8;          // which 32-element half of the k-step
         const int n = n0 + row;
         const bool valid = n < N;
-        const uint8_t *crow = codes + (size_t)(valid ? n : (N - 1)) * (K >> 1);
-        const uint8_t *srow = scales + (size_t)(valid ? n : (N - 1)) * (K >> 4);
-        uint4 cc0, cc1;
+        const uint8_t *crow = codes + (size_t)(valid ? n : (N - 1)) * (K >> 1) + 16 * hk;
+        const uint8_t *srow = scales + (size_t)(valid ? n : (N - 1)) * (K >> 4) + 2 * hk;
+        uint4 cc;
         unsigned sc;
         auto load_stage = [&](int kb) {
-            cc0 = ldg_stream(crow + (size_t)kb * 32);
-            cc1 = ldg_stream(crow + (size_t)kb * 32 + 16);
-            sc = __ldg(reinterpret_cast<const unsigned *>(srow + (size_t)kb * 4));
+            cc = ldg_stream(crow + (size_t)kb * 32);
+            sc = *reinterpret_cast<const unsigned short *>(srow + (size_t)kb * 4);
         };
         load_stage(0);
         bool ok = true;
         for (int kb = 0; kb < KB; kb++) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            const uint4 c0 = cc0, c1 = cc1;
+            const uint4 c0 = cc;
             const unsigned cs = valid ? sc : 0u;
             if (kb + 1 < KB) load_stage(kb + 1);
             if (!mbar_wait_warp(empty + 8 * s, ph ^ 1u, abort_flag)) {
@@ -357,14 +357,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             uint8_t *rbase = smem + s * STAGE_BYTES + 2 * A_HALF_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
-            const unsigned words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            const unsigned words[4] = {c0.x, c0.y, c0.z, c0.w};
 #pragma unroll
-            for (int blk = 0; blk < 4; blk++) {
+            for (int blk = 0; blk < 2; blk++) {
                 const BlockK kc = block_consts<FMT>((cs >> (8 * blk)) & 0xFFu);
 #pragma unroll
                 for (int h = 0; h < 2; h++) {
-                    const int j = 2 * blk + h;  // 16-byte chunk = 8 elements
-                    const uint4 v = decode_word<FMT, BF16>(words[j], kc);
+                    const int j = 4 * hk + 2 * blk + h;  // 16-byte chunk = 8 elements
+                    const uint4 v = decode_word<FMT, BF16>(words[2 * blk + h], kc);
                     *reinterpret_cast<uint4 *>(rbase + ((j ^ (row & 7)) << 4)) = v;
                 }
             }
@@ -373,18 +373,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(full_b + 8 * s);
         }
 
-        // epilogue: TMEM lanes 32*(warp%4) .. +31; the two warps of a lane
+        // epilogue: TMEM lanes 32*(warp%4) .. +31; the four warps of a lane
         // quarter split the 256 columns of each accumulator
         if (ok && mbar_wait_warp(acc_full, 0, abort_flag) && !*abort_flag) {
             tc_fence_after();
             const int q = warp & 3;
-            const int cbeg = (warp - 2) < 4 ? 0 : BN / 2;
+            const int cbeg = ((warp - 2) >> 2) * (BN / 4);
             const float scale = __fmul_rn(*ts_p, unbias);
 #pragma unroll 1
             for (int half = 0; half < 2; half++) {
                 const int m = m0 + half * 128 + q * 32 + lane;
 #pragma unroll 1
-                for (int c0 = cbeg; c0 < cbeg + BN / 2; c0 += 32) {
+                for (int c0 = cbeg; c0 < cbeg + BN / 4; c0 += 32) {
                     float v[32];
                     tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c0), v);
                     const int n = n0 + c0;

@@ -148,8 +148,9 @@ __device__ __forceinline__ void scale_pairs2(unsigned sb, unsigned (&s2)[2], uns
 constexpr int kRing = 4;                          // stages per warp ring
 constexpr int kCodeBytes = 16 * 64;               // 16 rows x 64 bytes per chunk
 constexpr int kScaleBytes = 16 * 8;               // 16 rows x 8 scale bytes
-constexpr int kStageBytes = kCodeBytes + kScaleBytes;
-constexpr int kGemvSmem = kGemvWarps * kRing * kStageBytes;
+constexpr int kXRowBytes = 128 * 2;               // one activation row of a chunk
+// stage = codes | scales | activations (B <= 8 rows, only when NB == 1)
+__host__ __device__ constexpr int gemv_stage_bytes(int xrows) { return kCodeBytes + kScaleBytes + xrows * kXRowBytes; }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
 {
@@ -180,17 +181,26 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
     const uint8_t *sa = scales + (size_t)rA * (K >> 4);
     const uint8_t *sbp = scales + (size_t)rB * (K >> 4);
 
-    // this warp's ring: stage = [16 rows x 64 B of codes][16 rows x 8 B of scales]
-    uint8_t *ring = gemv_smem + warp * (kRing * kStageBytes);
+    // this warp's ring: stage = [16 rows x 64 B of codes][16 rows x 8 B of
+    // scales][activation rows of the chunk, B <= 8 only]
+    const int xrows = NB == 1 ? B : 0;
+    const int stage_bytes = gemv_stage_bytes(xrows);
+    uint8_t *ring = gemv_smem + warp * (kRing * stage_bytes);
     const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
     auto issue = [&](int c, int slot) {
         if (c < c_end) {
-            const uint32_t st = ring_s + slot * kStageBytes;
+            const uint32_t st = ring_s + slot * stage_bytes;
             cp_async16(st + g * 64 + 16 * t, pa + (size_t)c * 64);
             cp_async16(st + (g + 8) * 64 + 16 * t, pb + (size_t)c * 64);
             if (t < 2) {  // 8 scale bytes per row (scales are only 4-byte aligned)
                 cp_async4(st + kCodeBytes + g * 8 + 4 * t, sa + (size_t)c * 8 + 4 * t);
                 cp_async4(st + kCodeBytes + (g + 8) * 8 + 4 * t, sbp + (size_t)c * 8 + 4 * t);
+            }
+            if (NB == 1 && g < B) {  // this lane's 64 activation bytes
+                const uint8_t *src = reinterpret_cast<const uint8_t *>(x + (size_t)g * K + (size_t)c * 128 + 32 * t);
+                const uint32_t dst = st + kCodeBytes + kScaleBytes + g * kXRowBytes + 64 * t;
+#pragma unroll
+                for (int q = 0; q < 4; q++) cp_async16(dst + 16 * q, src + 16 * q);
             }
         }
         cp_async_commit();  // one group per chunk (possibly empty) keeps the counting uniform
@@ -214,7 +224,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
         issue(c + kRing - 1, (i + kRing - 1) % kRing);
         cp_async_wait<kRing - 1>();  // this chunk's group has landed
         __syncwarp();                // scale bytes were copied by lanes t < 2 of each row group
-        const uint8_t *st = ring + (i % kRing) * kStageBytes;
+        const uint8_t *st = ring + (i % kRing) * stage_bytes;
         const uint4 ca = *reinterpret_cast<const uint4 *>(st + g * 64 + 16 * t);
         const uint4 cb = *reinterpret_cast<const uint4 *>(st + (g + 8) * 64 + 16 * t);
         const unsigned sA = *reinterpret_cast<const unsigned short *>(st + kCodeBytes + g * 8 + 2 * t);
@@ -222,11 +232,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
 #pragma unroll
         for (int j = 0; j < NB; j++) {
             if (8 * j + g < B) {  // lanes past the batch keep their zero fragments
-                const uint4 *px = reinterpret_cast<const uint4 *>(x + (size_t)(8 * j + g) * K + (size_t)c * 128 + 32 * t);
-                if (c + 1 < c_end) asm volatile("prefetch.global.L1 [%0];" ::"l"(px + 16));  // next chunk's activations
+                const uint4 *px = NB == 1 ? reinterpret_cast<const uint4 *>(st + kCodeBytes + kScaleBytes + g * kXRowBytes + 64 * t)
+                                          : reinterpret_cast<const uint4 *>(x + (size_t)(8 * j + g) * K + (size_t)c * 128 + 32 * t);
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
-                    const uint4 v = __ldg(px + q);
+                    const uint4 v = NB == 1 ? px[q] : __ldg(px + q);
                     xw[j][4 * q] = v.x;
                     xw[j][4 * q + 1] = v.y;
                     xw[j][4 * q + 2] = v.z;
@@ -315,9 +325,18 @@ static void launch_gemv_fmt(const void *x, int B, const uint8_t *codes, const ui
 {
     dim3 grid((unsigned)(((N + 15) / 16 + kGemvWarps - 1) / kGemvWarps), (unsigned)S);
     const uint16_t *xp = reinterpret_cast<const uint16_t *>(x);
-    if (B <= 8) gemv_kernel<FMT, BF16, 1><<<grid, kGemvThreads, kGemvSmem, st>>>(xp, B, codes, scales, N, K, S, ws);
-    else if (B <= 16) gemv_kernel<FMT, BF16, 2><<<grid, kGemvThreads, kGemvSmem, st>>>(xp, B, codes, scales, N, K, S, ws);
-    else gemv_kernel<FMT, BF16, 4><<<grid, kGemvThreads, kGemvSmem, st>>>(xp, B, codes, scales, N, K, S, ws);
+    const int smem1 = kGemvWarps * kRing * gemv_stage_bytes(B), smem0 = kGemvWarps * kRing * gemv_stage_bytes(0);
+    static bool attr_done[64] = {false};  // per device: allow up to 8 activation rows in the ring (> 48 KB)
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        cudaFuncSetAttribute(gemv_kernel<FMT, BF16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGemvWarps * kRing * gemv_stage_bytes(8));
+        attr_done[dev] = true;
+    }
+    if (B <= 8) gemv_kernel<FMT, BF16, 1><<<grid, kGemvThreads, smem1, st>>>(xp, B, codes, scales, N, K, S, ws);
+    else if (B <= 16) gemv_kernel<FMT, BF16, 2><<<grid, kGemvThreads, smem0, st>>>(xp, B, codes, scales, N, K, S, ws);
+    else gemv_kernel<FMT, BF16, 4><<<grid, kGemvThreads, smem0, st>>>(xp, B, codes, scales, N, K, S, ws);
 }
 
 razer_status run_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
