@@ -10,9 +10,10 @@
 //     per 256 activation rows (half the decode work per SM of a 128-row tile).
 //   * warp 0: TMA producer of the X tiles (K-major, 128-byte swizzle);
 //     warp 1: TMEM allocator and the single MMA-issuing thread;
-//     warps 2-17: decoders, half a weight row per thread, four warps per
-//     scheduler (decode is latency-bound) -- they stream the codes and scales with
-//     128-bit loads (one stage ahead), decode to 16-bit q*s and write the
+//     warps 2-9: decoders, one weight row per thread, two warps per
+//     scheduler -- the producer's TMA also brings each stage's raw code tile
+//     (256 rows x 32 bytes) into shared memory; the decoders read it with
+//     conflict-free 16-byte loads, decode to 16-bit q*s and write the
 //     UMMA canonical K-major 128B-swizzled layout with 16-byte stores; after
 //     the k loop they are the epilogue (tcgen05.ld, * ts, convert, store).
 //   * fp32 accumulators: two 128 x 256 tiles = all 512 TMEM columns.
@@ -32,11 +33,16 @@ namespace razer {
 namespace gemm {
 
 constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
-constexpr int kDecodeWarps = 16;  // four per scheduler; each thread decodes half a weight row
+#ifndef RAZER_GEMM_DECODE_WARPS
+#define RAZER_GEMM_DECODE_WARPS 8
+#endif
+constexpr int kDecodeWarps = RAZER_GEMM_DECODE_WARPS;  // 8: a row per thread; 16: half a row per thread
+constexpr int kHalvesPerThread = 16 / kDecodeWarps;
 constexpr int kThreads = 64 + 32 * kDecodeWarps;
 constexpr uint32_t A_HALF_BYTES = 128 * BK * 2;               // 16 KB
-constexpr uint32_t B_BYTES = BN * BK * 2;                     // 32 KB
-constexpr uint32_t STAGE_BYTES = 2 * A_HALF_BYTES + B_BYTES;  // 64 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;                     // 32 KB (decoded weights)
+constexpr uint32_t CODE_BYTES = BN * BK / 2;                  // 8 KB (raw codes, by TMA)
+constexpr uint32_t STAGE_BYTES = 2 * A_HALF_BYTES + B_BYTES + CODE_BYTES;  // 72 KB
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
 constexpr uint64_t kTimeoutNs = 2000000000ull;
@@ -99,6 +105,7 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, vo
     int ok = 0;
     if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) (void)mbar_try_wait(bar, parity);  // completed phase: every lane acquires it
     __syncwarp();
     return ok != 0;
 }
@@ -239,7 +246,7 @@ __device__ __forceinline__ uint4 decode_word(unsigned w, const BlockK &k)
 
 template <int FMT, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c, const uint8_t *__restrict__ scales,
                 const float *__restrict__ ts_p, float unbias, int M, int N, int K, void *__restrict__ Y, int out_dt)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -284,9 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
                 if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort_flag)) break;
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
-                mbar_expect_tx(full_a + 8 * s, 2 * A_HALF_BYTES);
+                mbar_expect_tx(full_a + 8 * s, 2 * A_HALF_BYTES + CODE_BYTES);
                 tma_load_2d(a0, &tmap_x, kb * BK, m0, full_a + 8 * s);
                 tma_load_2d(a0 + A_HALF_BYTES, &tmap_x, kb * BK, m0 + 128, full_a + 8 * s);
+                tma_load_2d(a0 + 2 * A_HALF_BYTES + B_BYTES, &tmap_c, kb * (BK / 2), n0, full_a + 8 * s);  // raw codes [256 x 32 B]
                 issued = kb + 1;
             }
             if (*abort_flag) {
@@ -333,39 +341,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---------------- decoders, then epilogue ----------------
         const int row = (threadIdx.x - 64) & (BN - 1);  // 0..255
-        const int hk = (threadIdx.x - 64) >> 8;          // which 32-element half of the k-step
+        const int hk0 = kHalvesPerThread == 1 ? ((threadIdx.x - 64) >> 8) : 0;  // first 32-element half of the k-step
         const int n = n0 + row;
         const bool valid = n < N;
-        const uint8_t *crow = codes + (size_t)(valid ? n : (N - 1)) * (K >> 1) + 16 * hk;
-        const uint8_t *srow = scales + (size_t)(valid ? n : (N - 1)) * (K >> 4) + 2 * hk;
-        uint4 cc;
+        const uint8_t *srow = scales + (size_t)(valid ? n : (N - 1)) * (K >> 4) + 2 * hk0;
         unsigned sc;
-        auto load_stage = [&](int kb) {
-            cc = ldg_stream(crow + (size_t)kb * 32);
-            sc = *reinterpret_cast<const unsigned short *>(srow + (size_t)kb * 4);
+        auto load_scales = [&](int kb) {
+            sc = kHalvesPerThread == 1 ? (unsigned)*reinterpret_cast<const unsigned short *>(srow + (size_t)kb * 4)
+                                       : *reinterpret_cast<const unsigned *>(srow + (size_t)kb * 4);
         };
-        load_stage(0);
+        load_scales(0);
         bool ok = true;
         for (int kb = 0; kb < KB; kb++) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            const uint4 c0 = cc;
             const unsigned cs = valid ? sc : 0u;
-            if (kb + 1 < KB) load_stage(kb + 1);
-            if (!mbar_wait_warp(empty + 8 * s, ph ^ 1u, abort_flag)) {
+            if (kb + 1 < KB) load_scales(kb + 1);
+            // the producer refills a slot only after the MMAs released it, so
+            // the arrival of this stage's TMA also means the B slot is free
+            if (!mbar_wait_warp(full_a + 8 * s, ph, abort_flag)) {
                 ok = false;
                 break;
             }
-            uint8_t *rbase = smem + s * STAGE_BYTES + 2 * A_HALF_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
-            const unsigned words[4] = {c0.x, c0.y, c0.z, c0.w};
+            uint8_t *stage = smem + s * STAGE_BYTES;
+            uint8_t *rbase = stage + 2 * A_HALF_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+            // raw codes of this row: 32 bytes; the two 16-byte halves are read
+            // in an order (by bit 2 of the row) that keeps 8 consecutive rows
+            // on distinct banks
+            const uint8_t *crow = stage + 2 * A_HALF_BYTES + B_BYTES + row * 32;
+            uint4 c0[kHalvesPerThread];
+            if (kHalvesPerThread == 1) {
+                c0[0] = *reinterpret_cast<const uint4 *>(crow + 16 * hk0);
+            } else {
+                const int f = (row >> 2) & 1;
+                c0[f] = *reinterpret_cast<const uint4 *>(crow + 16 * f);
+                c0[f ^ 1] = *reinterpret_cast<const uint4 *>(crow + 16 * (f ^ 1));
+            }
 #pragma unroll
-            for (int blk = 0; blk < 2; blk++) {
-                const BlockK kc = block_consts<FMT>((cs >> (8 * blk)) & 0xFFu);
+            for (int h = 0; h < kHalvesPerThread; h++) {
+                const unsigned words[4] = {c0[h].x, c0[h].y, c0[h].z, c0[h].w};
 #pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    const int j = 4 * hk + 2 * blk + h;  // 16-byte chunk = 8 elements
-                    const uint4 v = decode_word<FMT, BF16>(words[2 * blk + h], kc);
-                    *reinterpret_cast<uint4 *>(rbase + ((j ^ (row & 7)) << 4)) = v;
+                for (int blk = 0; blk < 2; blk++) {
+                    const BlockK kc = block_consts<FMT>((cs >> (8 * (2 * h + blk))) & 0xFFu);
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const int j = 4 * (hk0 + h) + 2 * blk + e;  // 16-byte chunk = 8 elements
+                        const uint4 v = decode_word<FMT, BF16>(words[2 * blk + e], kc);
+                        *reinterpret_cast<uint4 *>(rbase + ((j ^ (row & 7)) << 4)) = v;
+                    }
                 }
             }
             fence_proxy_async();
@@ -373,18 +396,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(full_b + 8 * s);
         }
 
-        // epilogue: TMEM lanes 32*(warp%4) .. +31; the four warps of a lane
-        // quarter split the 256 columns of each accumulator
+        // epilogue: TMEM lanes 32*(warp%4) .. +31; the warps of a lane quarter
+        // split the 256 columns of each accumulator
         if (ok && mbar_wait_warp(acc_full, 0, abort_flag) && !*abort_flag) {
             tc_fence_after();
             const int q = warp & 3;
-            const int cbeg = ((warp - 2) >> 2) * (BN / 4);
+            const int cbeg = ((warp - 2) >> 2) * (BN * 4 / kDecodeWarps);
             const float scale = __fmul_rn(*ts_p, unbias);
 #pragma unroll 1
             for (int half = 0; half < 2; half++) {
                 const int m = m0 + half * 128 + q * 32 + lane;
 #pragma unroll 1
-                for (int c0 = cbeg; c0 < cbeg + BN / 4; c0 += 32) {
+                for (int c0 = cbeg; c0 < cbeg + BN * 4 / kDecodeWarps; c0 += 32) {
                     float v[32];
                     tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c0), v);
                     const int n = n0 + c0;
@@ -456,8 +479,8 @@ static EncodeTiledFn encode_fn()
 }
 
 template <int FMT, bool BF16>
-static razer_status launch(const CUtensorMap &map, const uint8_t *codes, const uint8_t *scales, const float *ts, float unbias, int M,
-                           int N, int K, void *Y, razer_dtype out_dt, cudaStream_t st)
+static razer_status launch(const CUtensorMap &map, const CUtensorMap &cmap, const uint8_t *scales, const float *ts, float unbias,
+                           int M, int N, int K, void *Y, razer_dtype out_dt, cudaStream_t st)
 {
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -468,7 +491,7 @@ static razer_status launch(const CUtensorMap &map, const uint8_t *codes, const u
         attr_set[dev] = true;
     }
     dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt);
+    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, cmap, scales, ts, unbias, M, N, K, Y, (int)out_dt);
     return last_launch_status();
 }
 
@@ -503,17 +526,26 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return RAZER_ERR_CUDA;
+    // raw codes [N rows, K/2 bytes]: one 256-row x 32-byte box per k-step
+    CUtensorMap cmap;
+    const cuuint64_t cdims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+    const cuuint64_t cstrides[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t cbox[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)BN};
+    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), cdims, cstrides, cbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return RAZER_ERR_CUDA;
     // the decoded q*s carries 2^-8 (E3M3) / 2^-4 (E4M3); undone in the epilogue
     const float unbias = wfmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f;
     const int m = (int)M, n = (int)N, k = (int)K;
     if (wfmt == RAZER_FMT_WEIGHT)
-        return bf ? launch<RAZER_FMT_WEIGHT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
-                  : launch<RAZER_FMT_WEIGHT, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
+        return bf ? launch<RAZER_FMT_WEIGHT, true>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st)
+                  : launch<RAZER_FMT_WEIGHT, false>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st);
     if (wfmt == RAZER_FMT_ACT)
-        return bf ? launch<RAZER_FMT_ACT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
-                  : launch<RAZER_FMT_ACT, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
-    return bf ? launch<RAZER_FMT_NVFP4, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
-              : launch<RAZER_FMT_NVFP4, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
+        return bf ? launch<RAZER_FMT_ACT, true>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st)
+                  : launch<RAZER_FMT_ACT, false>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st);
+    return bf ? launch<RAZER_FMT_NVFP4, true>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st)
+              : launch<RAZER_FMT_NVFP4, false>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st);
 }
 
 }  // namespace razer
