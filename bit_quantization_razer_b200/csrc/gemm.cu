@@ -10,10 +10,11 @@
 //     per 256 activation rows (half the decode work per SM of a 128-row tile).
 //   * warp 0: TMA producer of the X tiles (K-major, 128-byte swizzle);
 //     warp 1: TMEM allocator and the single MMA-issuing thread;
-//     warps 2-9: decoders, one weight row per thread, two warps per
-//     scheduler -- the producer's TMA also brings each stage's raw code tile
-//     (256 rows x 32 bytes) into shared memory; the decoders read it with
-//     conflict-free 16-byte loads, decode to 16-bit q*s and write the
+//     warp 2: TMA producer of the raw code tiles (256 rows x 32 bytes per
+//     k-step) into their own 4-deep ring, so codes run ahead of the X tiles;
+//     warps 3-10: decoders, one weight row per thread, two warps per
+//     scheduler -- they read the codes with conflict-free 16-byte shared
+//     loads, decode to 16-bit q*s and write the
 //     UMMA canonical K-major 128B-swizzled layout with 16-byte stores; after
 //     the k loop they are the epilogue (tcgen05.ld, * ts, convert, store).
 //   * fp32 accumulators: two 128 x 256 tiles = all 512 TMEM columns.
@@ -38,13 +39,15 @@ constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
 #endif
 constexpr int kDecodeWarps = RAZER_GEMM_DECODE_WARPS;  // 8: a row per thread; 16: half a row per thread
 constexpr int kHalvesPerThread = 16 / kDecodeWarps;
-constexpr int kThreads = 64 + 32 * kDecodeWarps;
+constexpr int kFirstDecodeWarp = 3;  // warp 0: X TMA, 1: MMA, 2: code TMA
+constexpr int kThreads = 32 * kFirstDecodeWarp + 32 * kDecodeWarps;
 constexpr uint32_t A_HALF_BYTES = 128 * BK * 2;               // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;                     // 32 KB (decoded weights)
-constexpr uint32_t CODE_BYTES = BN * BK / 2;                  // 8 KB (raw codes, by TMA)
-constexpr uint32_t STAGE_BYTES = 2 * A_HALF_BYTES + B_BYTES + CODE_BYTES;  // 72 KB
+constexpr uint32_t CODE_BYTES = BN * BK / 2;                  // 8 KB (raw codes of a k-step, by TMA)
+constexpr int CODE_STAGES = 4;                                // codes run ahead in their own ring
+constexpr uint32_t STAGE_BYTES = 2 * A_HALF_BYTES + B_BYTES;  // 64 KB
 constexpr uint32_t BAR_BYTES = 256;
-constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + CODE_STAGES * CODE_BYTES + BAR_BYTES + 1024;  // + alignment slack
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -251,13 +254,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *bars = smem + STAGES * STAGE_BYTES;
+    uint8_t *code_ring = smem + STAGES * STAGE_BYTES;
+    uint8_t *bars = code_ring + CODE_STAGES * CODE_BYTES;
     const uint32_t full_a = smem_addr(bars);              // STAGES x 8
     const uint32_t full_b = full_a + 8 * STAGES;          // STAGES x 8
     const uint32_t empty = full_b + 8 * STAGES;           // STAGES x 8
     const uint32_t acc_full = empty + 8 * STAGES;         // 8
-    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(bars + 128);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 136);
+    const uint32_t code_full = acc_full + 8;              // CODE_STAGES x 8
+    const uint32_t code_empty = code_full + 8 * CODE_STAGES;  // CODE_STAGES x 8
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(bars + 192);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 200);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
@@ -270,6 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(empty + 8 * s, 1);
         }
         mbar_init(acc_full, 1);
+        for (int s = 0; s < CODE_STAGES; s++) {
+            mbar_init(code_full + 8 * s, 1);
+            mbar_init(code_empty + 8 * s, kDecodeWarps);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -291,10 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
                 if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort_flag)) break;
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
-                mbar_expect_tx(full_a + 8 * s, 2 * A_HALF_BYTES + CODE_BYTES);
+                mbar_expect_tx(full_a + 8 * s, 2 * A_HALF_BYTES);
                 tma_load_2d(a0, &tmap_x, kb * BK, m0, full_a + 8 * s);
                 tma_load_2d(a0 + A_HALF_BYTES, &tmap_x, kb * BK, m0 + 128, full_a + 8 * s);
-                tma_load_2d(a0 + 2 * A_HALF_BYTES + B_BYTES, &tmap_c, kb * (BK / 2), n0, full_a + 8 * s);  // raw codes [256 x 32 B]
                 issued = kb + 1;
             }
             if (*abort_flag) {
@@ -338,10 +347,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+    } else if (warp == 2) {
+        // ---------------- TMA producer (raw code tiles, own ring) ----------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < KB; kb++) {
+                const int s = kb % CODE_STAGES;
+                const uint32_t ph = (uint32_t)(kb / CODE_STAGES) & 1u;
+                if (!mbar_wait(code_empty + 8 * s, ph ^ 1u, abort_flag)) break;
+                mbar_expect_tx(code_full + 8 * s, CODE_BYTES);
+                tma_load_2d(smem_addr(code_ring + s * CODE_BYTES), &tmap_c, kb * (BK / 2), n0, code_full + 8 * s);
+                issued = kb + 1;
+            }
+            if (*abort_flag) {
+                const uint64_t t0 = globaltimer();
+                for (int kb = (issued > CODE_STAGES ? issued - CODE_STAGES : 0); kb < issued; kb++) {
+                    const int s = kb % CODE_STAGES;
+                    const uint32_t ph = (uint32_t)(kb / CODE_STAGES) & 1u;
+                    while (!mbar_try_wait(code_full + 8 * s, ph) && globaltimer() - t0 < kTimeoutNs) {
+                    }
+                }
+            }
+        }
     } else {
         // ---------------- decoders, then epilogue ----------------
-        const int row = (threadIdx.x - 64) & (BN - 1);  // 0..255
-        const int hk0 = kHalvesPerThread == 1 ? ((threadIdx.x - 64) >> 8) : 0;  // first 32-element half of the k-step
+        const int dt = threadIdx.x - 32 * kFirstDecodeWarp;  // 0 .. 32*kDecodeWarps-1
+        const int row = dt & (BN - 1);                      // 0..255
+        const int hk0 = kHalvesPerThread == 1 ? (dt >> 8) : 0;  // first 32-element half of the k-step
         const int n = n0 + row;
         const bool valid = n < N;
         const uint8_t *srow = scales + (size_t)(valid ? n : (N - 1)) * (K >> 4) + 2 * hk0;
@@ -355,20 +387,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < KB; kb++) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+            const int cs_slot = kb % CODE_STAGES;
+            const uint32_t cph = (uint32_t)(kb / CODE_STAGES) & 1u;
             const unsigned cs = valid ? sc : 0u;
             if (kb + 1 < KB) load_scales(kb + 1);
-            // the producer refills a slot only after the MMAs released it, so
-            // the arrival of this stage's TMA also means the B slot is free
-            if (!mbar_wait_warp(full_a + 8 * s, ph, abort_flag)) {
+            // raw codes of this row (32 bytes) from the code ring; the two
+            // 16-byte halves are read in an order (bit 2 of the row) that keeps
+            // 8 consecutive rows on distinct banks
+            if (!mbar_wait_warp(code_full + 8 * cs_slot, cph, abort_flag)) {
                 ok = false;
                 break;
             }
-            uint8_t *stage = smem + s * STAGE_BYTES;
-            uint8_t *rbase = stage + 2 * A_HALF_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
-            // raw codes of this row: 32 bytes; the two 16-byte halves are read
-            // in an order (by bit 2 of the row) that keeps 8 consecutive rows
-            // on distinct banks
-            const uint8_t *crow = stage + 2 * A_HALF_BYTES + B_BYTES + row * 32;
+            const uint8_t *crow = code_ring + cs_slot * CODE_BYTES + row * 32;
             uint4 c0[kHalvesPerThread];
             if (kHalvesPerThread == 1) {
                 c0[0] = *reinterpret_cast<const uint4 *>(crow + 16 * hk0);
@@ -377,6 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 c0[f] = *reinterpret_cast<const uint4 *>(crow + 16 * f);
                 c0[f ^ 1] = *reinterpret_cast<const uint4 *>(crow + 16 * (f ^ 1));
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(code_empty + 8 * cs_slot);  // this warp is done with the code slot
+            // the decoded tile goes into B slot s once the MMAs released it
+            if (!mbar_wait_warp(empty + 8 * s, ph ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            uint8_t *rbase = smem + s * STAGE_BYTES + 2 * A_HALF_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
             for (int h = 0; h < kHalvesPerThread; h++) {
                 const unsigned words[4] = {c0[h].x, c0[h].y, c0[h].z, c0[h].w};
@@ -401,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && mbar_wait_warp(acc_full, 0, abort_flag) && !*abort_flag) {
             tc_fence_after();
             const int q = warp & 3;
-            const int cbeg = ((warp - 2) >> 2) * (BN * 4 / kDecodeWarps);
+            const int cbeg = ((warp - kFirstDecodeWarp) >> 2) * (BN * 4 / kDecodeWarps);
             const float scale = __fmul_rn(*ts_p, unbias);
 #pragma unroll 1
             for (int half = 0; half < 2; half++) {
