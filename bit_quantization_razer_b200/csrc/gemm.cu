@@ -10,11 +10,10 @@
 //     per 256 activation rows (half the decode work per SM of a 128-row tile).
 //   * warp 0: TMA producer of the X tiles (K-major, 128-byte swizzle);
 //     warp 1: TMEM allocator and the single MMA-issuing thread;
-//     warp 2: TMA producer of the raw code tiles (256 rows x 32 bytes per
-//     k-step) into their own 4-deep ring, so codes run ahead of the X tiles;
-//     warps 3-10: decoders, one weight row per thread, two warps per
-//     scheduler -- they read the codes with conflict-free 16-byte shared
-//     loads, decode to 16-bit q*s and write the
+//     warps 2-9: decoders, one weight row per thread, two warps per
+//     scheduler -- they stream the packed codes and scale bytes with
+//     128-bit loads (two k-steps ahead, in registers), decode to 16-bit q*s
+//     and write the
 //     UMMA canonical K-major 128B-swizzled layout with 16-byte stores; after
 //     the k loop they are the epilogue (tcgen05.ld, * ts, convert, store).
 //   * fp32 accumulators: two 128 x 256 tiles = all 512 TMEM columns.
@@ -39,15 +38,13 @@ constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
 #endif
 constexpr int kDecodeWarps = RAZER_GEMM_DECODE_WARPS;  // 8: a row per thread; 16: half a row per thread
 constexpr int kHalvesPerThread = 16 / kDecodeWarps;
-constexpr int kFirstDecodeWarp = 3;  // warp 0: X TMA, 1: MMA, 2: code TMA
+constexpr int kFirstDecodeWarp = 2;  // warp 0: X TMA, 1: MMA
 constexpr int kThreads = 32 * kFirstDecodeWarp + 32 * kDecodeWarps;
 constexpr uint32_t A_HALF_BYTES = 128 * BK * 2;               // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;                     // 32 KB (decoded weights)
-constexpr uint32_t CODE_BYTES = BN * BK / 2;                  // 8 KB (raw codes of a k-step, by TMA)
-constexpr int CODE_STAGES = 4;                                // codes run ahead in their own ring
 constexpr uint32_t STAGE_BYTES = 2 * A_HALF_BYTES + B_BYTES;  // 64 KB
 constexpr uint32_t BAR_BYTES = 256;
-constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + CODE_STAGES * CODE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -249,19 +246,16 @@ __device__ __forceinline__ uint4 decode_word(unsigned w, const BlockK &k)
 
 template <int FMT, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c, const uint8_t *__restrict__ scales,
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
                 const float *__restrict__ ts_p, float unbias, int M, int N, int K, void *__restrict__ Y, int out_dt)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *code_ring = smem + STAGES * STAGE_BYTES;
-    uint8_t *bars = code_ring + CODE_STAGES * CODE_BYTES;
+    uint8_t *bars = smem + STAGES * STAGE_BYTES;
     const uint32_t full_a = smem_addr(bars);              // STAGES x 8
     const uint32_t full_b = full_a + 8 * STAGES;          // STAGES x 8
     const uint32_t empty = full_b + 8 * STAGES;           // STAGES x 8
     const uint32_t acc_full = empty + 8 * STAGES;         // 8
-    const uint32_t code_full = acc_full + 8;              // CODE_STAGES x 8
-    const uint32_t code_empty = code_full + 8 * CODE_STAGES;  // CODE_STAGES x 8
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(bars + 192);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 200);
 
@@ -276,10 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(empty + 8 * s, 1);
         }
         mbar_init(acc_full, 1);
-        for (int s = 0; s < CODE_STAGES; s++) {
-            mbar_init(code_full + 8 * s, 1);
-            mbar_init(code_empty + 8 * s, kDecodeWarps);
-        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -347,28 +337,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp == 2) {
-        // ---------------- TMA producer (raw code tiles, own ring) ----------------
-        if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < KB; kb++) {
-                const int s = kb % CODE_STAGES;
-                const uint32_t ph = (uint32_t)(kb / CODE_STAGES) & 1u;
-                if (!mbar_wait(code_empty + 8 * s, ph ^ 1u, abort_flag)) break;
-                mbar_expect_tx(code_full + 8 * s, CODE_BYTES);
-                tma_load_2d(smem_addr(code_ring + s * CODE_BYTES), &tmap_c, kb * (BK / 2), n0, code_full + 8 * s);
-                issued = kb + 1;
-            }
-            if (*abort_flag) {
-                const uint64_t t0 = globaltimer();
-                for (int kb = (issued > CODE_STAGES ? issued - CODE_STAGES : 0); kb < issued; kb++) {
-                    const int s = kb % CODE_STAGES;
-                    const uint32_t ph = (uint32_t)(kb / CODE_STAGES) & 1u;
-                    while (!mbar_try_wait(code_full + 8 * s, ph) && globaltimer() - t0 < kTimeoutNs) {
-                    }
-                }
-            }
-        }
     } else {
         // ---------------- decoders, then epilogue ----------------
         const int dt = threadIdx.x - 32 * kFirstDecodeWarp;  // 0 .. 32*kDecodeWarps-1
@@ -376,39 +344,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hk0 = kHalvesPerThread == 1 ? (dt >> 8) : 0;  // first 32-element half of the k-step
         const int n = n0 + row;
         const bool valid = n < N;
+        const uint8_t *crow = codes + (size_t)(valid ? n : (N - 1)) * (K >> 1) + 16 * hk0;
         const uint8_t *srow = scales + (size_t)(valid ? n : (N - 1)) * (K >> 4) + 2 * hk0;
-        unsigned sc;
-        auto load_scales = [&](int kb) {
-            sc = kHalvesPerThread == 1 ? (unsigned)*reinterpret_cast<const unsigned short *>(srow + (size_t)kb * 4)
-                                       : *reinterpret_cast<const unsigned *>(srow + (size_t)kb * 4);
+        // codes and scale bytes of the next two k-steps are in flight in
+        // registers, so a global-load latency is covered by two decode steps
+        struct Regs {
+            uint4 c[kHalvesPerThread];
+            unsigned s;
         };
-        load_scales(0);
+        auto load_stage = [&](int kb, Regs &r) {
+#pragma unroll
+            for (int h = 0; h < kHalvesPerThread; h++) r.c[h] = ldg_stream(crow + (size_t)kb * 32 + 16 * h);
+            r.s = kHalvesPerThread == 1 ? (unsigned)*reinterpret_cast<const unsigned short *>(srow + (size_t)kb * 4)
+                                        : *reinterpret_cast<const unsigned *>(srow + (size_t)kb * 4);
+        };
+        Regs r0, r1;
+        load_stage(0, r0);
+        if (KB > 1) load_stage(1, r1);
         bool ok = true;
         for (int kb = 0; kb < KB; kb++) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            const int cs_slot = kb % CODE_STAGES;
-            const uint32_t cph = (uint32_t)(kb / CODE_STAGES) & 1u;
-            const unsigned cs = valid ? sc : 0u;
-            if (kb + 1 < KB) load_scales(kb + 1);
-            // raw codes of this row (32 bytes) from the code ring; the two
-            // 16-byte halves are read in an order (bit 2 of the row) that keeps
-            // 8 consecutive rows on distinct banks
-            if (!mbar_wait_warp(code_full + 8 * cs_slot, cph, abort_flag)) {
-                ok = false;
-                break;
-            }
-            const uint8_t *crow = code_ring + cs_slot * CODE_BYTES + row * 32;
             uint4 c0[kHalvesPerThread];
-            if (kHalvesPerThread == 1) {
-                c0[0] = *reinterpret_cast<const uint4 *>(crow + 16 * hk0);
-            } else {
-                const int f = (row >> 2) & 1;
-                c0[f] = *reinterpret_cast<const uint4 *>(crow + 16 * f);
-                c0[f ^ 1] = *reinterpret_cast<const uint4 *>(crow + 16 * (f ^ 1));
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(code_empty + 8 * cs_slot);  // this warp is done with the code slot
+#pragma unroll
+            for (int h = 0; h < kHalvesPerThread; h++) c0[h] = r0.c[h];
+            const unsigned cs = valid ? r0.s : 0u;
+            r0 = r1;
+            if (kb + 2 < KB) load_stage(kb + 2, r1);
             // the decoded tile goes into B slot s once the MMAs released it
             if (!mbar_wait_warp(empty + 8 * s, ph ^ 1u, abort_flag)) {
                 ok = false;
@@ -517,7 +479,7 @@ static EncodeTiledFn encode_fn()
 }
 
 template <int FMT, bool BF16>
-static razer_status launch(const CUtensorMap &map, const CUtensorMap &cmap, const uint8_t *scales, const float *ts, float unbias,
+static razer_status launch(const CUtensorMap &map, const uint8_t *codes, const uint8_t *scales, const float *ts, float unbias,
                            int M, int N, int K, void *Y, razer_dtype out_dt, cudaStream_t st)
 {
     static bool attr_set[64] = {false};
@@ -529,7 +491,7 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &cmap, cons
         attr_set[dev] = true;
     }
     dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, cmap, scales, ts, unbias, M, N, K, Y, (int)out_dt);
+    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt);
     return last_launch_status();
 }
 
@@ -564,26 +526,17 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return RAZER_ERR_CUDA;
-    // raw codes [N rows, K/2 bytes]: one 256-row x 32-byte box per k-step
-    CUtensorMap cmap;
-    const cuuint64_t cdims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
-    const cuuint64_t cstrides[1] = {(cuuint64_t)(K / 2)};
-    const cuuint32_t cbox[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)BN};
-    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), cdims, cstrides, cbox, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return RAZER_ERR_CUDA;
     // the decoded q*s carries 2^-8 (E3M3) / 2^-4 (E4M3); undone in the epilogue
     const float unbias = wfmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f;
     const int m = (int)M, n = (int)N, k = (int)K;
     if (wfmt == RAZER_FMT_WEIGHT)
-        return bf ? launch<RAZER_FMT_WEIGHT, true>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st)
-                  : launch<RAZER_FMT_WEIGHT, false>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st);
+        return bf ? launch<RAZER_FMT_WEIGHT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
+                  : launch<RAZER_FMT_WEIGHT, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
     if (wfmt == RAZER_FMT_ACT)
-        return bf ? launch<RAZER_FMT_ACT, true>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st)
-                  : launch<RAZER_FMT_ACT, false>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st);
-    return bf ? launch<RAZER_FMT_NVFP4, true>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st)
-              : launch<RAZER_FMT_NVFP4, false>(map, cmap, scales, ts, unbias, m, n, k, Y, out_dt, st);
+        return bf ? launch<RAZER_FMT_ACT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
+                  : launch<RAZER_FMT_ACT, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
+    return bf ? launch<RAZER_FMT_NVFP4, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
+              : launch<RAZER_FMT_NVFP4, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
 }
 
 }  // namespace razer
