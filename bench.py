@@ -53,6 +53,15 @@ def step_bytes():
     return sum(quant_bytes(N, K) for N, K in SHAPES) + sum(gemv_bytes(B, N, K) for N, K in SHAPES for B in BATCHES)
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """Max of a per-rank number (device time in ms) over all ranks."""
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -319,9 +328,7 @@ def main():
         torch.cuda.synchronize()
     elapsed_ms = t0.elapsed_time(t1)
     if pg:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+        elapsed_ms = max_over_ranks(elapsed_ms, pg, dev)
         pg.barrier()
     ms_per_step = elapsed_ms / args.steps
     value = step_bytes() * args.steps * world / (elapsed_ms / 1e3) / 1e9
@@ -571,9 +578,7 @@ def run_e2e(R, workloads, dev, stream, args, world, pg):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     if pg:
-        tt = torch.tensor([ms], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, pg, dev)
     return {"value": step_bytes() * steps * world / (ms / 1e3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps}
 

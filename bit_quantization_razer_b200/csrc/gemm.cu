@@ -26,6 +26,7 @@
 // normal range, which converts exactly to bf16 (at most 7 significant bits)
 // for bf16 activations.
 #include <cuda.h>
+#include <cstdlib>
 
 #include "razer_internal.cuh"
 
@@ -247,7 +248,8 @@ __device__ __forceinline__ uint4 decode_word(unsigned w, const BlockK &k)
 template <int FMT, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
-                const float *__restrict__ ts_p, float unbias, int M, int N, int K, void *__restrict__ Y, int out_dt)
+                const float *__restrict__ ts_p, float unbias, int M, int N, int K, void *__restrict__ Y, int out_dt,
+                int inject_stall)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -393,7 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async();
             __syncwarp();
-            if (lane == 0) mbar_arrive(full_b + 8 * s);
+            // fault injection (tests only): a decoder warp that never arrives
+            // makes the MMA thread's bounded wait run out
+            if (lane == 0 && !(inject_stall && warp == kFirstDecodeWarp)) mbar_arrive(full_b + 8 * s);
         }
 
         // epilogue: TMEM lanes 32*(warp%4) .. +31; the warps of a lane quarter
@@ -491,7 +495,11 @@ static razer_status launch(const CUtensorMap &map, const uint8_t *codes, const u
         attr_set[dev] = true;
     }
     dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt);
+    // RAZER_FAULT_INJECT_STALL=1 (tests only) withholds one decoder warp's
+    // arrivals so that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
+    const char *inj = getenv("RAZER_FAULT_INJECT_STALL");
+    const int inject = (inj && inj[0] == '1') ? 1 : 0;
+    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt, inject);
     return last_launch_status();
 }
 

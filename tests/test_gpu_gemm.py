@@ -84,3 +84,26 @@ def test_gemm_k_zero_and_errors():
     c, s = workloads.random_packed(48, 96, "weight", seed=1)
     with pytest.raises(R.RazerError):  # K % 64
         R.razer_gemm(torch.zeros(8, 96, dtype=torch.bfloat16, device=DEV), c.to(DEV), s.to(DEV), torch.ones(1, device=DEV))
+
+
+def test_gemm_bounded_wait_times_out_and_reports(monkeypatch):
+    """A decoder warp that never arrives (host-side fault injection) makes the
+    MMA thread's bounded wait expire: the kernel stops, frees its tensor
+    memory, and the device status word reports RAZER_ERR_TIMEOUT; the context
+    stays usable."""
+    codes, scales = workloads.random_packed(256, 64, "weight", seed=90)
+    X = workloads.vectors(256, 64, seed=91, dtype=torch.bfloat16).to(DEV)
+    c, s = codes.to(DEV), scales.to(DEV)
+    ts = torch.ones(1, device=DEV)
+    assert R.razer_get_device_status() == 0
+    monkeypatch.setenv("RAZER_FAULT_INJECT_STALL", "1")
+    R.razer_gemm(X, c, s, ts, "weight", torch.float32)
+    assert R.razer_get_device_status() == 7  # RAZER_ERR_TIMEOUT, read and cleared
+    monkeypatch.delenv("RAZER_FAULT_INJECT_STALL")
+    assert R.razer_get_device_status() == 0
+    # the next call works normally
+    Y = R.razer_gemm(X, c, s, ts, "weight", torch.float32)
+    torch.cuda.synchronize()
+    import oracle
+    ref = oracle.gemm_ref(oracle_in(X.cpu()), codes.numpy(), scales.numpy(), 1.0, 0)
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
