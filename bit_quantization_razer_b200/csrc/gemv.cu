@@ -26,6 +26,8 @@
 //   * split-K partials go to a caller-provided fp32 workspace and a second
 //     small kernel sums them, applies ts (and the 2^12 / 2^8 unbias) and
 //     converts to the output type.
+#include <algorithm>
+
 #include "razer_internal.cuh"
 
 namespace razer {
@@ -61,14 +63,13 @@ __device__ __forceinline__ unsigned hmul2u(unsigned a, unsigned b)
 }
 
 // f16x2 -> bf16x2 (exact for the decoded values: at most 7 significant bits,
-// inside the bf16 range)
+// inside the bf16 range).  Through fp32: the direct 16-bit convert is a slow
+// instruction on this GPU, the f16 -> f32 converts and the f32 pair pack are not.
 __device__ __forceinline__ unsigned f16x2_to_bf16x2(unsigned h)
 {
-    unsigned r;
-    asm("{ .reg .b16 l, h, ol, oh; mov.b32 {l, h}, %1; cvt.rn.bf16.f16 ol, l; cvt.rn.bf16.f16 oh, h; mov.b32 %0, {ol, oh}; }"
-        : "=r"(r)
-        : "r"(h));
-    return r;
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+    __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<unsigned *>(&b);
 }
 
 __device__ __forceinline__ unsigned prmt(unsigned a, unsigned b, unsigned sel)
@@ -142,6 +143,31 @@ __device__ __forceinline__ void scale_pairs2(unsigned sb, unsigned (&s2)[2], uns
         v2[1] = prmt(vs, 0u, 0x3232u);
     } else {
         v2[0] = v2[1] = 0u;
+    }
+}
+
+// One 16-row x 128-k slice: ca / cb are this lane's 16 code bytes of MMA
+// rows g and g+8 (32 codes = two blocks each), sA / sB their two scale bytes,
+// xw the activation fragments of the same 32 k (zero for batch rows past B).
+template <int FMT, bool BF16, int NB>
+__device__ __forceinline__ void slice_mma(const uint4 &ca, const uint4 &cb, unsigned sA, unsigned sB, const unsigned (&xw)[NB][16],
+                                          float (&acc)[NB][4])
+{
+    unsigned s2A[2], vA[2], s2B[2], vB[2];
+    scale_pairs2<FMT>(sA, s2A, vA);
+    scale_pairs2<FMT>(sB, s2B, vB);
+    const unsigned wa[4] = {ca.x, ca.y, ca.z, ca.w};
+    const unsigned wb[4] = {cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+        unsigned hA[4], hB[4];
+        decode_word<FMT, BF16>(wa[m], s2A[m >> 1], vA[m >> 1], hA);
+        decode_word<FMT, BF16>(wb[m], s2B[m >> 1], vB[m >> 1], hB);
+#pragma unroll
+        for (int j = 0; j < NB; j++) {
+            mma16816<BF16>(acc[j], hA[0], hB[0], hA[1], hB[1], xw[j][4 * m], xw[j][4 * m + 1]);
+            mma16816<BF16>(acc[j], hA[2], hB[2], hA[3], hB[3], xw[j][4 * m + 2], xw[j][4 * m + 3]);
+        }
     }
 }
 
@@ -244,22 +270,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *__re
                 }
             }
         }
-        unsigned s2A[2], vA[2], s2B[2], vB[2];
-        scale_pairs2<FMT>(sA, s2A, vA);
-        scale_pairs2<FMT>(sB, s2B, vB);
-        const unsigned wa[4] = {ca.x, ca.y, ca.z, ca.w};
-        const unsigned wb[4] = {cb.x, cb.y, cb.z, cb.w};
-#pragma unroll
-        for (int m = 0; m < 4; m++) {
-            unsigned hA[4], hB[4];
-            decode_word<FMT, BF16>(wa[m], s2A[m >> 1], vA[m >> 1], hA);
-            decode_word<FMT, BF16>(wb[m], s2B[m >> 1], vB[m >> 1], hB);
-#pragma unroll
-            for (int j = 0; j < NB; j++) {
-                mma16816<BF16>(acc[j], hA[0], hB[0], hA[1], hB[1], xw[j][4 * m], xw[j][4 * m + 1]);
-                mma16816<BF16>(acc[j], hA[2], hB[2], hA[3], hB[3], xw[j][4 * m + 2], xw[j][4 * m + 3]);
-            }
-        }
+        slice_mma<FMT, BF16, NB>(ca, cb, sA, sB, xw, acc);
     }
     cp_async_wait<0>();
 
@@ -313,10 +324,18 @@ int gemv_splits(int64_t B, int64_t N, int64_t K)
     return (int)S;
 }
 
+bool gemv_tma_eligible(int64_t B, int64_t N, int64_t K);
+size_t gemv_tma_workspace_bytes(int64_t B, int64_t N, int64_t K);
+razer_status run_gemv_tma(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                          razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st);
+
 size_t gemv_workspace_bytes(int64_t B, int64_t N, int64_t K)
 {
     if (B <= 0 || N <= 0 || K <= 0) return 0;
-    return (size_t)gemv_splits(B, N, K) * (size_t)B * (size_t)N * sizeof(float);
+    // the per-warp kernel also serves eligible shapes whose scale pointer is
+    // only 4-byte aligned (a tensor map needs 16), so size for both
+    const size_t split = (size_t)gemv_splits(B, N, K) * (size_t)B * (size_t)N * sizeof(float);
+    return gemv_tma_eligible(B, N, K) ? std::max(split, gemv_tma_workspace_bytes(B, N, K)) : split;
 }
 
 template <int FMT, bool BF16>
@@ -342,6 +361,8 @@ static void launch_gemv_fmt(const void *x, int B, const uint8_t *codes, const ui
 razer_status run_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
                       razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st)
 {
+    if (gemv_tma_eligible(B, N, K) && (reinterpret_cast<uintptr_t>(scales) & 15) == 0)
+        return run_gemv_tma(x, act_dt, B, codes, scales, ts, wfmt, N, K, y, out_dt, workspace, st);
     const int S = gemv_splits(B, N, K);
     float *ws = reinterpret_cast<float *>(workspace);
     const bool bf = act_dt == RAZER_BF16;

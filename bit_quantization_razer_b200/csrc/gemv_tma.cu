@@ -1,0 +1,483 @@
+// RaZeR W4A16 GEMV / skinny GEMM (1 <= B <= 32), bulk-tensor pipeline for
+// sm_100a; taken when K % 256 == 0 (the scale rows are then 16-byte strided,
+// as a tensor map requires) and the scale pointer is 16-byte aligned.
+//
+// y[b, n] = ts * sum_k x[b, k] * (q*s)[n, k]     (RaZeR notes 关键设计 3:
+// weight-only kernels that decode the remapped codes in registers, and
+// split-K sized for the machine -- here one persistent CTA per SM.)
+//
+//   * Work = 128-row tiles x 128-k half-units, flattened tile-major and cut
+//     into one contiguous range per CTA ("stream-K"): every SM streams the
+//     same number of weight bytes, whatever N and K, and there is no tail
+//     wave.
+//   * Warp 0 (one lane) is the TMA producer.  Per 256-k stage it loads the
+//     code tile (128 rows x 128 B, 128-byte swizzle), the scale tile
+//     (128 x 16 B) and the B activation rows (B x 512 B) into an S-deep
+//     shared-memory ring guarded by full / empty mbarriers.
+//   * The consumer warps each own 16 * kMT rows of the tile and one 128-k half
+//     of every stage; they run the register decode and warp-level m16n8k16
+//     MMAs of the split-K kernel (the kMT row tiles share the activation
+//     fragments).  The MMA rows g = 2p and 2p+1 (one 128-bit shared-load
+//     phase) map to tile rows p and p+4, whose swizzled 16-byte chunks sit in
+//     opposite halves of the banks, so the code loads are conflict-free.
+//   * When a CTA finishes its part of a tile, the consumers drop their fp32
+//     partials into one of two shared-memory hand-over buffers and go on with
+//     the next tile at once.  Warp 1 (the epilogue warp) adds the two k-halves
+//     and either writes y (the CTA covered the whole tile) or stores the sum in
+//     slot (cta + tile) of the workspace -- the slot index grows along the
+//     flattened order, so it is unique.  A small second kernel, launched as a
+//     programmatic dependent of the first (it is resident and waiting while
+//     the first drains), sums the slots of the shared tiles in CTA order --
+//     deterministic --, applies ts and converts.  Both kernels wait on their
+//     predecessor in the stream (griddepcontrol.wait) before reading memory it
+//     may have written.
+//   * Every mbarrier wait is bounded; on expiry the CTA records
+//     RAZER_ERR_TIMEOUT, stops waiting, keeps its control flow (and its
+//     arrivals) uniform, and the producer lets its in-flight loads land
+//     before it exits.
+#include <algorithm>
+
+#include "razer_internal.cuh"
+#include "sm100_async.cuh"
+
+namespace razer {
+namespace gemv_tma {
+
+#ifndef RAZER_GEMV_MT
+#define RAZER_GEMV_MT 2
+#endif
+constexpr int kMT = RAZER_GEMV_MT;                  // 16-row MMA tiles per consumer warp (1 or 2)
+constexpr int kTileRows = 128;
+constexpr int kRowGroups = kTileRows / (16 * kMT);  // consumer warps per k-half
+constexpr int kConsumerWarps = 2 * kRowGroups;      // one per (row group, 128-k half of a stage)
+constexpr int kFirstConsumer = 2;                   // warp 0: TMA producer, warp 1: epilogue
+constexpr int kThreads = 32 * (kFirstConsumer + kConsumerWarps);
+constexpr int kCodeBytes = kTileRows * 128;         // 128 rows x 256 codes
+constexpr int kScaleBytes = kTileRows * 16;         // 128 rows x 16 blocks
+constexpr int kMaxStages = 8;
+constexpr int kBarBytes = 256;
+constexpr int kSmemLimit = 227 * 1024;
+
+__host__ __device__ constexpr int stage_bytes(int B) { return (kCodeBytes + kScaleBytes + B * 512 + 1023) / 1024 * 1024; }
+// two hand-over buffers of [k-half][B][128 rows] fp32 partials
+__host__ __device__ constexpr int part_bytes(int B) { return 2 * 2 * B * kTileRows * 4; }
+__host__ __device__ constexpr int num_stages(int B)
+{
+    return (kSmemLimit - 1024 - kBarBytes - part_bytes(B)) / stage_bytes(B) > kMaxStages
+               ? kMaxStages
+               : (kSmemLimit - 1024 - kBarBytes - part_bytes(B)) / stage_bytes(B);
+}
+__host__ __device__ constexpr int smem_bytes(int B) { return num_stages(B) * stage_bytes(B) + part_bytes(B) + kBarBytes + 1024; }
+
+// first half-unit of CTA c's range
+__host__ __device__ __forceinline__ int range_start(int c, int U, int G) { return (int)((int64_t)c * U / G); }
+// the CTA whose range holds half-unit p (ranges are never empty: G <= U)
+__host__ __device__ __forceinline__ int range_owner(int p, int U, int G) { return (int)(((int64_t)(p + 1) * G - 1) / U); }
+
+// tile row of MMA row g (and g + 8 -> +8): rows 2p, 2p+1 -> p, p+4
+__device__ __forceinline__ int tile_row(int g) { return (g >> 1) | ((g & 1) << 2); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t a)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ unsigned lds16(uint32_t a)
+{
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned *p, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void store_out(void *y, int out_dt, size_t i, float v)
+{
+    if (out_dt == RAZER_F32) reinterpret_cast<float *>(y)[i] = v;
+    else if (out_dt == RAZER_F16) reinterpret_cast<__half *>(y)[i] = __float2half_rn(v);
+    else reinterpret_cast<__nv_bfloat16 *>(y)[i] = __float2bfloat16_rn(v);
+}
+
+// wait that returns at once when the phase is complete (the common case)
+__device__ __forceinline__ void wait_phase(uint32_t bar, uint32_t ph, volatile int *flags)
+{
+    if (!mbar_try_wait(bar, ph)) (void)mbar_wait(bar, ph, flags);  // on abort: carry on, results are void
+}
+
+template <int FMT, bool BF16, int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemv_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
+                    const __grid_constant__ CUtensorMap tm_x, int B, int N, int UK2, int U, int stages, int stage_sz,
+                    float *__restrict__ ws, const float *__restrict__ ts_p, float unbias, void *__restrict__ y, int out_dt)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *part = reinterpret_cast<float *>(smem + stages * stage_sz);  // [2 buffers][2 k-halves][B][128]
+    uint8_t *bars = smem + stages * stage_sz + 2 * 2 * B * kTileRows * 4;
+    const uint32_t full = smem_addr(bars), empty = full + 8 * kMaxStages;
+    const uint32_t pfull = empty + 8 * kMaxStages, pempty = pfull + 16;
+    volatile int *flags = reinterpret_cast<volatile int *>(bars + 16 * kMaxStages + 32);  // [0] abort
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int p_begin = range_start(c, U, G), p_end = range_start(c + 1, U, G);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; s++) {
+            mbar_init(full + 8 * s, 1);
+            mbar_init(empty + 8 * s, kConsumerWarps);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(pfull + 8 * b, kConsumerWarps);
+            mbar_init(pempty + 8 * b, 1);
+        }
+        flags[0] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    // the reduction kernel may be scheduled now (it waits for this grid to finish)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (warp == 0) {
+        // ------------------------- TMA producer -------------------------
+        if (lane == 0) {
+            // inputs may come from the previous kernel in the stream
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            const uint32_t tx = (uint32_t)(kCodeBytes + kScaleBytes + B * 512);
+            int s = 0, issued = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int p = p_begin; p < p_end && ok;) {
+                const int r = p / UK2;
+                const int pe = min(p_end, (r + 1) * UK2);
+                const int h0 = p - r * UK2, h1 = pe - r * UK2;
+                for (int j = h0 >> 1; j < (h1 + 1) >> 1; j++) {
+                    if (!mbar_wait(empty + 8 * s, ph ^ 1u, flags)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t dst = smem_addr(smem + s * stage_sz);
+                    mbar_expect_tx(full + 8 * s, tx);
+                    tma_load_2d(dst, &tm_codes, j * 128, r * kTileRows, full + 8 * s);
+                    tma_load_2d(dst + kCodeBytes, &tm_scales, j * 16, r * kTileRows, full + 8 * s);
+                    tma_load_2d(dst + kCodeBytes + kScaleBytes, &tm_x, j * 256, 0, full + 8 * s);
+                    issued++;
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                p = pe;
+            }
+            // the loads issued last into each stage land before this warp (and,
+            // on an abort, the CTA) goes away
+            for (int i = issued > stages ? issued - stages : 0; i < issued; i++) {
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(full + 8 * (i % stages), (uint32_t)(i / stages) & 1u) && globaltimer() - t0 < kTimeoutNs) {
+                }
+            }
+        }
+        return;
+    }
+
+    if (warp == 1) {
+        // ------------------------- epilogue -------------------------
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        const float oscale = __fmul_rn(*ts_p, unbias);
+        const int slot_elems = B * kTileRows;
+        int q = 0;
+        for (int p = p_begin; p < p_end; q++) {
+            const int r = p / UK2;
+            const int pe = min(p_end, (r + 1) * UK2);
+            const int buf = q & 1;
+            wait_phase(pfull + 8 * buf, (uint32_t)(q >> 1) & 1u, flags);
+            const float *h0p = part + buf * 2 * slot_elems, *h1p = h0p + slot_elems;
+            const int c_first = range_owner(r * UK2, U, G), c_last = range_owner((r + 1) * UK2 - 1, U, G);
+            const int row_base = r * kTileRows;
+            // lane owns float4 e4 = lane + 32 i (i < B) of the [B][128] tile
+            const float4 *h0v = reinterpret_cast<const float4 *>(h0p), *h1v = reinterpret_cast<const float4 *>(h1p);
+            if (c_first == c_last) {
+                for (int i = 0; i < B; i++) {
+                    const int e4 = lane + 32 * i;
+                    const float4 a = h0v[e4], b4 = h1v[e4];
+                    const float v[4] = {a.x + b4.x, a.y + b4.y, a.z + b4.z, a.w + b4.w};
+                    const int b = e4 >> 5, row = row_base + 4 * (e4 & 31);
+#pragma unroll
+                    for (int u = 0; u < 4; u++)
+                        if (row + u < N) store_out(y, out_dt, (size_t)b * N + row + u, __fmul_rn(v[u], oscale));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pempty + 8 * buf);
+            } else {
+                float4 *slot = reinterpret_cast<float4 *>(ws + (size_t)(c + r) * slot_elems);
+                for (int i = 0; i < B; i++) {
+                    const int e4 = lane + 32 * i;
+                    const float4 a = h0v[e4], b4 = h1v[e4];
+                    slot[e4] = make_float4(a.x + b4.x, a.y + b4.y, a.z + b4.z, a.w + b4.w);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pempty + 8 * buf);
+            }
+            p = pe;
+        }
+        return;
+    }
+
+    // ------------------------- consumers -------------------------
+    // warp (rg, kh): rows 16 kMT rg .. 16 kMT (rg + 1) - 1 of the tile, k-half kh
+    // of every 256-k stage
+    const int cw = warp - kFirstConsumer, rg = cw >> 1, kh = cw & 1, g = lane >> 2, t = lane & 3;
+    const int pr = tile_row(g);
+    const int cc = t + 4 * kh;  // this lane's 16-byte chunk of the 128-byte code row
+    const int R0 = 16 * kMT * rg + pr;  // tile row of MMA row g of the first 16-row tile
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t offA = (uint32_t)(R0 * 128 + ((cc ^ pr) << 4));  // + 1024 for row g + 8, + 2048 per 16-row tile
+    const uint32_t offS = (uint32_t)(kCodeBytes + R0 * 16 + 2 * cc);  // + 128 for row g + 8, + 256 per tile
+    const uint32_t offX = (uint32_t)(kCodeBytes + kScaleBytes + g * 512 + 64 * cc);
+    const bool xrow = g < B;
+
+    float acc[kMT][NB][4];
+    unsigned xw[NB][16];
+#pragma unroll
+    for (int j = 0; j < NB; j++)
+#pragma unroll
+        for (int i = 0; i < 16; i++) xw[j][i] = 0u;
+
+    int s = 0, q = 0;  // ring position of the next stage, hand-over count (no divisions in the loop)
+    uint32_t ph = 0;
+    uint32_t st = sbase;
+    for (int p = p_begin; p < p_end; q++) {
+        const int r = p / UK2;
+        const int pe = min(p_end, (r + 1) * UK2);
+        const int h0 = p - r * UK2, h1 = pe - r * UK2;
+        // stages j whose half-unit 2j + kh lies in [h0, h1)
+        const int ja = (h0 - kh + 1) >> 1, jb = (h1 - 1 - kh) >> 1;
+#pragma unroll
+        for (int m = 0; m < kMT; m++)
+#pragma unroll
+            for (int j = 0; j < NB; j++) acc[m][j][0] = acc[m][j][1] = acc[m][j][2] = acc[m][j][3] = 0.0f;
+
+        for (int j = h0 >> 1; j < (h1 + 1) >> 1; j++) {
+            wait_phase(full + 8 * s, ph, flags);
+            if (j >= ja && j <= jb) {
+                uint4 ca[kMT], cb[kMT];
+                unsigned sA[kMT], sB[kMT];
+#pragma unroll
+                for (int m = 0; m < kMT; m++) {
+                    ca[m] = lds128(st + offA + 2048 * m);
+                    cb[m] = lds128(st + offA + 2048 * m + 1024);
+                    sA[m] = lds16(st + offS + 256 * m);
+                    sB[m] = lds16(st + offS + 256 * m + 128);
+                }
+                {
+#pragma unroll
+                    for (int jj = 0; jj < NB; jj++) {
+                        if (8 * jj + g < B && (NB > 1 || xrow)) {
+#pragma unroll
+                            for (int i = 0; i < 4; i++) {
+                                const uint4 v = lds128(st + offX + (uint32_t)(jj * 8 * 512 + 16 * i));
+                                xw[jj][4 * i] = v.x;
+                                xw[jj][4 * i + 1] = v.y;
+                                xw[jj][4 * i + 2] = v.z;
+                                xw[jj][4 * i + 3] = v.w;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int m = 0; m < kMT; m++) slice_mma<FMT, BF16, NB>(ca[m], cb[m], sA[m], sB[m], xw, acc[m]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + 8 * s);
+            st += (uint32_t)stage_sz;
+            if (++s == stages) {
+                s = 0;
+                ph ^= 1u;
+                st = sbase;
+            }
+        }
+
+        // hand the partial of this tile to the epilogue warp and go on
+        const int buf = q & 1;
+        wait_phase(pempty + 8 * buf, ((uint32_t)(q >> 1) & 1u) ^ 1u, flags);
+        float *dst = part + (buf * 2 + kh) * B * kTileRows;
+#pragma unroll
+        for (int m = 0; m < kMT; m++) {
+#pragma unroll
+            for (int jj = 0; jj < NB; jj++) {
+                const int b0 = 8 * jj + 2 * t;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int b = b0 + (i & 1), row = R0 + 16 * m + ((i & 2) ? 8 : 0);
+                    if (b < B) dst[b * kTileRows + row] = acc[m][jj][i];
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pfull + 8 * buf);
+        p = pe;
+    }
+}
+
+// Sums the workspace slots of the tiles shared by several CTAs, in CTA order.
+// Launched as a programmatic dependent of gemv_tma_kernel: it may become
+// resident early and waits here until that grid has completed.
+__global__ void __launch_bounds__(256) gemv_tma_reduce_kernel(const float *__restrict__ ws, int B, int N, int UK2, int U, int G, int T,
+                                                              const float *__restrict__ ts_p, float unbias, void *__restrict__ y, int out_dt)
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const float oscale = __fmul_rn(*ts_p, unbias);
+    const int slot_elems = B * kTileRows;
+    const int64_t total = (int64_t)T * slot_elems;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int r = (int)(i / slot_elems), e = (int)(i - (int64_t)r * slot_elems);
+        const int c_first = range_owner(r * UK2, U, G), c_last = range_owner((r + 1) * UK2 - 1, U, G);
+        const int row = r * kTileRows + (e & (kTileRows - 1));
+        if (c_first == c_last || row >= N) continue;  // whole tiles were written by the main kernel
+        const float *src = ws + (size_t)r * slot_elems + e;
+        float sum = 0.0f;
+        for (int k = c_first; k <= c_last; k++) sum += __ldcg(src + (size_t)k * slot_elems);
+        store_out(y, out_dt, (size_t)(e >> 7) * N + row, __fmul_rn(sum, oscale));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+struct Plan {
+    int64_t T, UK2, U, G;  // tiles, half-units per tile, half-units, CTAs
+    size_t total;  // workspace: one [B][128] fp32 slot per (CTA, tile) pair
+};
+
+static Plan plan(int64_t B, int64_t N, int64_t K)
+{
+    Plan p;
+    p.T = (N + kTileRows - 1) / kTileRows;
+    p.UK2 = K / 128;
+    p.U = p.T * p.UK2;
+    p.G = std::min<int64_t>(sm_count(), p.U);
+    p.total = (size_t)(p.G + p.T - 1) * (size_t)B * kTileRows * sizeof(float);
+    return p;
+}
+
+// launch with the programmatic-stream-serialization attribute: the kernel may
+// be scheduled before its predecessor in the stream has finished, and waits
+// for it with griddepcontrol.wait before touching memory the predecessor wrote
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+template <int FMT, bool BF16, int NB>
+static razer_status launch(const CUtensorMap &tc, const CUtensorMap &tsc, const CUtensorMap &tx, int B, int N, const Plan &pl,
+                           float *ws, const float *ts, float unbias, void *y, razer_dtype out_dt, cudaStream_t st)
+{
+    const int stages = num_stages(B), sz = stage_bytes(B), smem = smem_bytes(B);
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(gemv_tma_kernel<FMT, BF16, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
+            return RAZER_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int UK2 = (int)pl.UK2, U = (int)pl.U, G = (int)pl.G, T = (int)pl.T;
+    if (launch_pdl(gemv_tma_kernel<FMT, BF16, NB>, (unsigned)G, kThreads, (size_t)smem, st, tc, tsc, tx, B, N, UK2, U, stages, sz, ws, ts,
+                   unbias, y, (int)out_dt) != cudaSuccess)
+        return RAZER_ERR_CUDA;
+    // tiles shared by several CTAs exist unless every CTA range is whole tiles
+    bool shared = false;
+    for (int64_t r = 0; r < pl.T && !shared; r++)
+        shared = range_owner((int)(r * pl.UK2), U, G) != range_owner((int)((r + 1) * pl.UK2 - 1), U, G);
+    if (!shared) return RAZER_OK;
+    const int64_t total = pl.T * B * kTileRows;
+    const unsigned rgrid = (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 4);
+    if (launch_pdl(gemv_tma_reduce_kernel, rgrid, 256u, 0, st, (const float *)ws, B, N, UK2, U, G, T, ts, unbias, y, (int)out_dt) !=
+        cudaSuccess)
+        return RAZER_ERR_CUDA;
+    return RAZER_OK;
+}
+
+template <int FMT, bool BF16>
+static razer_status launch_nb(const CUtensorMap &tc, const CUtensorMap &tsc, const CUtensorMap &tx, int B, int N, const Plan &pl,
+                              float *ws, const float *ts, float unbias, void *y, razer_dtype out_dt, cudaStream_t st)
+{
+    if (B <= 8) return launch<FMT, BF16, 1>(tc, tsc, tx, B, N, pl, ws, ts, unbias, y, out_dt, st);
+    if (B <= 16) return launch<FMT, BF16, 2>(tc, tsc, tx, B, N, pl, ws, ts, unbias, y, out_dt, st);
+    return launch<FMT, BF16, 4>(tc, tsc, tx, B, N, pl, ws, ts, unbias, y, out_dt, st);
+}
+
+}  // namespace gemv_tma
+
+bool gemv_tma_eligible(int64_t B, int64_t N, int64_t K)
+{
+    // half-unit indices are 32-bit
+    return B >= 1 && B <= 32 && N >= 1 && K >= 256 && K % 256 == 0 && ((N + 127) / 128) * (K / 128) < (int64_t)INT32_MAX;
+}
+
+size_t gemv_tma_workspace_bytes(int64_t B, int64_t N, int64_t K) { return gemv_tma::plan(B, N, K).total; }
+
+razer_status run_gemv_tma(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                          razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st)
+{
+    using namespace gemv_tma;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return RAZER_ERR_CUDA;
+    const Plan pl = plan(B, N, K);
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUtensorMap tc, tsc, tx;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+        const cuuint32_t box[2] = {128u, (cuuint32_t)kTileRows};
+        if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return RAZER_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 16)};
+        const cuuint32_t box[2] = {16u, (cuuint32_t)kTileRows};
+        if (enc(&tsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(scales), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return RAZER_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)B};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {256u, (cuuint32_t)B};
+        if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return RAZER_ERR_CUDA;
+    }
+    float *ws = reinterpret_cast<float *>(workspace);
+    const float unbias = wfmt == RAZER_FMT_WEIGHT ? scale_f16_unbias<RAZER_FMT_WEIGHT>() : scale_f16_unbias<RAZER_FMT_ACT>();
+    const bool bf = act_dt == RAZER_BF16;
+    const int b = (int)B, n = (int)N;
+    if (wfmt == RAZER_FMT_WEIGHT)
+        return bf ? launch_nb<RAZER_FMT_WEIGHT, true>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st)
+                  : launch_nb<RAZER_FMT_WEIGHT, false>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st);
+    if (wfmt == RAZER_FMT_ACT)
+        return bf ? launch_nb<RAZER_FMT_ACT, true>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st)
+                  : launch_nb<RAZER_FMT_ACT, false>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st);
+    return bf ? launch_nb<RAZER_FMT_NVFP4, true>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st)
+              : launch_nb<RAZER_FMT_NVFP4, false>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st);
+}
+
+}  // namespace razer

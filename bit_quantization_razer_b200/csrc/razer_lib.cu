@@ -6,5 +6,6 @@
 #include "quantize.cu"
 #include "dequant.cu"
 #include "gemv.cu"
+#include "gemv_tma.cu"
 #include "gemm.cu"
 #include "gemv_noalloc.cu"

@@ -134,9 +134,12 @@ razer_status razer_dequant(const uint8_t *codes, const uint8_t *scales, const fl
  *   workspace  device scratch of at least
  *              razer_workspace_size(RAZER_OP_GEMV, B, N, K) bytes (16-byte
  *              aligned), or NULL when that size is 0.  Contents on entry are
- *              ignored.
+ *              ignored (it holds split-K partials while a call runs).
  * K must be a multiple of 128 (one 16-byte code chunk per 32 elements, four
- * chunks per row slice).
+ * chunks per row slice).  K % 256 == 0 with a 16-byte aligned scale pointer
+ * takes the bulk-tensor (TMA) kernel -- one persistent CTA per SM plus a small
+ * split-K reduction kernel launched as its programmatic dependent; other calls
+ * take a per-warp cp.async kernel and a reduction kernel.
  */
 razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes,
                         const uint8_t *scales, const float *ts, razer_format wfmt, int64_t N,
@@ -191,7 +194,7 @@ size_t razer_workspace_size(razer_op op, int64_t M_or_B, int64_t N, int64_t K);
 /*
  * razer_get_device_status -- the device-side error word of the current
  * device: RAZER_OK, or RAZER_ERR_TIMEOUT when a bounded wait inside a kernel
- * (pipeline barrier of razer_gemm) gave up.  Synchronises `stream`, then
+ * (pipeline barrier of razer_gemm or of the TMA razer_gemv) gave up.  Synchronises `stream`, then
  * reads and clears the word.
  */
 razer_status razer_get_device_status(razer_stream_t stream);

@@ -81,5 +81,18 @@ def test_gemv_gemm_validation(lib):
 
 def test_workspace_size_host_logic(lib):
     assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, 0, 64, 128) == 0
-    n = razer.razer_workspace_size(razer.RAZER_OP_GEMV, 4, 4096, 4096)
-    assert n > 0 and n % (4 * 4096 * 4) == 0
+    def split_k(B, N, K):  # per-warp kernel: ~8 CTAs per SM (148 without a GPU), >= 2 chunks per split
+        ctas = ((N + 15) // 16 + 3) // 4
+        chunks = K // 128
+        S = min(-(-148 * 8 // ctas), chunks // 2 if chunks >= 4 else chunks)
+        return max(S, 1) * B * N * 4
+    # K % 256 == 0: stream-K plan, one CTA per SM, 128-row tiles; one slot of
+    # B x 128 fp32 per (CTA, tile) pair, CTAs + tiles - 1 of them -- or the
+    # per-warp kernel's need if larger (it also serves 4-byte aligned scales)
+    for B, N, K in [(4, 4096, 4096), (1, 14336, 4096), (16, 4096, 14336), (32, 100, 256)]:
+        T = (N + 127) // 128
+        G = min(148, T * (K // 128))
+        tma = (G + T - 1) * B * 128 * 4
+        assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, B, N, K) == max(tma, split_k(B, N, K))
+    # other K: split-K partials of the per-warp kernel only
+    assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, 4, 4096, 4224) == split_k(4, 4096, 4224)

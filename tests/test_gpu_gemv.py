@@ -68,32 +68,83 @@ def test_gemv_one_hot_equals_dequant(orc):
         np.testing.assert_array_equal(y, deq[:, k])
 
 
-@pytest.mark.parametrize("N,K,B", [(4096, 4096, 1), (4096, 4096, 4), (14336, 4096, 16), (4096, 14336, 1),
-                                   (4096, 14336, 16), (8192, 8192, 32)])
-def test_gemv_config_shapes(orc, N, K, B):
-    codes, scales = workloads.random_packed(N, K, "weight", seed=N + K + B, max_scale_code=40)
+@pytest.mark.parametrize("N,K,B,fmt", [(4096, 4096, 1, "weight"), (4096, 4096, 4, "weight"), (14336, 4096, 16, "weight"),
+                                       (4096, 14336, 1, "weight"), (4096, 14336, 16, "weight"), (8192, 8192, 1, "weight"),
+                                       (8192, 8192, 8, "nvfp4"), (8192, 8192, 32, "weight"), (28672, 8192, 1, "weight"),
+                                       (8192, 28672, 32, "weight"), (28672, 8192, 8, "nvfp4")])
+def test_gemv_config_shapes(orc, N, K, B, fmt):
+    # the decode (Llama-3-8B) and 70B projection shapes, 512 sampled output columns
+    codes, scales = workloads.random_packed(N, K, fmt, seed=N + K + B, max_scale_code=40)
     x = workloads.vectors(B, K, seed=B)
     ts = 0.0045
-    y = gemv(x, codes, scales, ts, "weight").cpu().numpy()
+    y = gemv(x, codes, scales, ts, fmt).cpu().numpy()
     cols = np.random.default_rng(1).choice(N, 512, replace=False)
-    ref = orc.gemm_ref(x.numpy(), codes[cols].numpy(), scales[cols].numpy(), ts, 0)
+    ref = orc.gemm_ref(x.numpy(), codes[cols].numpy(), scales[cols].numpy(), ts, FMT_ID[fmt])
     assert rel_err(y[:, cols], ref) <= REL_TOL
 
 
-def test_gemv_k128_single_chunk(orc):
-    codes, scales = workloads.random_packed(48, 128, "act", seed=60)
-    x = workloads.vectors(2, 128, seed=61)
-    ref = orc.gemm_ref(x.numpy(), codes.numpy(), scales.numpy(), 1.5, 1)
-    y = gemv(x, codes, scales, 1.5, "act").cpu().numpy()
-    assert rel_err(y, ref) <= REL_TOL
+@pytest.mark.parametrize("fmt", ["weight", "act", "nvfp4"])
+@pytest.mark.parametrize("B", [1, 5, 9, 17, 32])
+@pytest.mark.parametrize("xdt", [torch.float16, torch.bfloat16])
+def test_gemv_tma_random_packed(orc, fmt, B, xdt):
+    # K % 256 == 0 (bulk-tensor kernel): ragged N over three 128-row tiles,
+    # 36 half-units shared unevenly by 36 CTAs
+    N, K = 300, 1536
+    codes, scales = workloads.random_packed(N, K, fmt, seed=140 + B)
+    x = workloads.vectors(B, K, seed=141 + B, dtype=xdt)
+    ts = 0.0371
+    ref = orc.gemm_ref(oracle_in(x), codes.numpy(), scales.numpy(), ts, FMT_ID[fmt])
+    y = gemv(x, codes, scales, ts, fmt)
+    assert rel_err(y.cpu().numpy(), ref) <= REL_TOL
 
 
-def test_gemv_workspace_errors():
-    codes, scales = workloads.random_packed(64, 256, "weight", seed=62)
-    x = torch.ones(4, 256, dtype=torch.float16, device=DEV)
-    ts = torch.ones(1, device=DEV)
-    need = R.razer_workspace_size(R.RAZER_OP_GEMV, 4, 64, 256)
-    small = torch.empty(max(need - 16, 16), dtype=torch.uint8, device=DEV)
-    with pytest.raises(R.RazerError) as e:
-        R.razer_gemv(x, codes.to(DEV), scales.to(DEV), ts, "weight", workspace=small)
-    assert "WORKSPACE" in str(e.value)
+@pytest.mark.parametrize("N,K,B", [(100, 256, 1), (128, 14336, 3), (129, 256, 2), (1, 4096, 1), (3000, 256, 7),
+                                   (640, 2304, 32), (1280, 4096, 8)])
+def test_gemv_stream_k_partitions(orc, N, K, B):
+    # fewer half-units than SMs; one tile shared by 112 CTAs; a one-row tail
+    # tile; N = 1; many tiles with one stage each; odd half-unit ranges
+    codes, scales = workloads.random_packed(N, K, "weight", seed=N * 7 + K + B)
+    x = workloads.vectors(B, K, seed=N + B)
+    ts = 0.0123
+    ref = orc.gemm_ref(x.numpy(), codes.numpy(), scales.numpy(), ts, 0)
+    y1 = gemv(x, codes, scales, ts, "weight")
+    y2 = gemv(x, codes, scales, ts, "weight")
+    assert rel_err(y1.cpu().numpy(), ref) <= REL_TOL
+    # the split-K partials are summed in a fixed order: repeat calls agree bit for bit
+    assert torch.equal(y1, y2)
+
+
+def test_gemv_workspace_garbage_and_reused(orc):
+    # one workspace full of garbage (NaN bytes) through calls of different
+    # shapes on both kernels (K % 256 == 0 and K % 256 == 128): its contents
+    # on entry never leak into y
+    shapes = [(4096, 4096, 4), (128, 14336, 2), (200, 1152, 3), (4096, 4096, 4), (300, 1536, 32)]
+    need = max(R.razer_workspace_size(R.RAZER_OP_GEMV, B, N, K) for N, K, B in shapes)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)
+    for i, (N, K, B) in enumerate(shapes):
+        codes, scales = workloads.random_packed(N, K, "weight", seed=600 + i, max_scale_code=40)
+        x = workloads.vectors(B, K, seed=610 + i)
+        ts = torch.tensor([0.02], dtype=torch.float32, device=DEV)
+        y = R.razer_gemv(x.to(DEV), codes.to(DEV), scales.to(DEV), ts, "weight", torch.float32, workspace=ws)
+        torch.cuda.synchronize()
+        assert R.razer_get_device_status() == 0
+        cols = np.arange(0, N, max(1, N // 64))
+        ref = orc.gemm_ref(x.numpy(), codes[cols].numpy(), scales[cols].numpy(), 0.02, 0)
+        assert rel_err(y.cpu().numpy()[:, cols], ref) <= REL_TOL
+        ws.fill_(0xFF)
+
+
+def test_gemv_scales_only_4byte_aligned(orc):
+    # a scale pointer that is 4- but not 16-byte aligned cannot back a tensor
+    # map: the per-warp kernel serves the call (same results)
+    N, K, B = 256, 1024, 2
+    codes, scales = workloads.random_packed(N, K, "weight", seed=77)
+    buf = torch.zeros(scales.numel() + 16, dtype=torch.uint8, device=DEV)
+    sc = buf[4:4 + scales.numel()].view(N, K // 16)
+    sc.copy_(scales.to(DEV))
+    assert sc.data_ptr() % 16 == 4
+    x = workloads.vectors(B, K, seed=78)
+    y = R.razer_gemv(x.to(DEV), codes.to(DEV), sc, torch.tensor([0.5], device=DEV), "weight", torch.float32)
+    torch.cuda.synchronize()
+    ref = orc.gemm_ref(x.numpy(), codes.numpy(), scales.numpy(), 0.5, 0)
+    assert rel_err(y.cpu().numpy(), ref) <= REL_TOL
