@@ -44,6 +44,15 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
 
 // Hardware E2M1 conversion (round to nearest even, saturating) of 8 values
 // into one word: nibble j holds the code of v[j].
+__device__ __forceinline__ float2 add2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{ .reg .b64 A, B, D; mov.b64 A, {%2, %3}; mov.b64 B, {%4, %5}; add.rn.f32x2 D, A, B; mov.b64 {%0, %1}, D; }"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 __device__ __forceinline__ unsigned cvt_e2m1x8(const float *v)
 {
     unsigned w;
@@ -141,14 +150,15 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], float t
         // 2^-20.  A = sum t and B = sum copysign(t, xs) are exact binary32 sums
         // (|A|, |B| <= 16); then the +5 sum is (A - B) / 2 and the -5 sum is
         // (A + B) / 2, both exact.
-        float A = 0.0f, Bs = 0.0f;
+        float2 AB = make_float2(0.0f, 0.0f);  // (A, B), one packed add per element
+        float ea[16];                           // 2|xs| - 10, reused by the final encode
 #pragma unroll
         for (int j = 0; j < 16; j++) {
-            const float e = __fmaf_rn(2.0f, fabsf(xs[j]), -10.0f);
-            const float t = fminf(__fadd_rn(fabsf(e), -1.0f), 0.0f);
-            A = __fadd_rn(A, t);
-            Bs = __fadd_rn(Bs, copysignf(t, xs[j]));
+            ea[j] = __fmaf_rn(2.0f, fabsf(xs[j]), -10.0f);
+            const float t = fminf(__fadd_rn(fabsf(ea[j]), -1.0f), 0.0f);
+            AB = add2(AB, make_float2(t, copysignf(t, xs[j])));
         }
+        const float A = AB.x, Bs = AB.y;
         const float dp5 = __fmul_rn(__fsub_rn(A, Bs), 0.5f);
         const float dn5 = __fmul_rn(__fadd_rn(A, Bs), 0.5f);
         float best = dp5;
@@ -182,25 +192,21 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], float t
         o.effective = best < 0.0f;
 
         // final encode against Q_FP4 u {v*}: elements nearest to v* take
-        // 0b1000.  For v* = +5 the region is xs in (4.5, 5.5], i.e.
-        // e = 2 xs - 10 in (-1, 1]; for v* = -5 it is [-5.5, -4.5), i.e.
-        // e = 2 xs + 10 in [-1, 1) (ties go to the smaller magnitude).  There e
-        // is an exact multiple of 2^-20, so the test is |e -+ 2^-22| < 1, the
-        // sign bit of r = |e -+ 2^-22| - 1.  The sign bits are gathered into
-        // the nibble mask with integer multiply-adds, keeping this pass off
-        // the half-rate ALU pipe.
+        // 0b1000.  For v* = +5 the region is xs in (4.5, 5.5], for v* = -5 it
+        // is [-5.5, -4.5) (ties go to the smaller magnitude): |xs| in
+        // (4.5, 5.5] with the sign of v*.  In terms of e = 2|xs| - 10 (exact
+        // there, a multiple of 2^-20) that is e in (-1, 1], i.e. the sign bit of
+        // r = |e - 2^-22| - 1.  The E2M1 convert keeps the sign of r in bit 3 of
+        // each nibble, which gathers the 16 tests with 4 converts; the sign of
+        // xs is the plain code's sign bit (the plain code is +-4 or +-6 there).
         unsigned o0 = 0u, o1 = 0u;
         if (meta < 2u) {
-            const float two_v = (meta & 1u) ? -10.0f : 10.0f;
-            const float nudge = (meta & 1u) ? 0x1p-22f : -0x1p-22f;
+            float r[16];
 #pragma unroll
-            for (int j = 0; j < 16; j++) {
-                const float e = __fmaf_rn(2.0f, xs[j], -two_v);
-                const float r = __fadd_rn(fabsf(__fadd_rn(e, nudge)), -1.0f);
-                const unsigned neg = __umulhi(__float_as_uint(r), 2u);  // sign bit of r
-                if (j < 8) o0 = neg * (8u << (4 * j)) + o0;
-                else o1 = neg * (8u << (4 * (j - 8))) + o1;
-            }
+            for (int j = 0; j < 16; j++) r[j] = __fadd_rn(fabsf(__fadd_rn(ea[j], -0x1p-22f)), -1.0f);
+            const unsigned in0 = cvt_e2m1x8(r) & 0x88888888u, in1 = cvt_e2m1x8(r + 8) & 0x88888888u;
+            o0 = in0 & ((meta & 1u) ? w0 : ~w0);
+            o1 = in1 & ((meta & 1u) ? w1 : ~w1);
         } else {
             // +8 (7, inf] / -8 [-inf, -7): one interval of bit patterns each
             const unsigned lo = 0x40E00001u | ((meta & 1u) << 31), span = 0x7F800000u - 0x40E00001u;
