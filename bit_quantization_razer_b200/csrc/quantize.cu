@@ -88,9 +88,18 @@ struct BlockOut {
     bool effective;  // the chosen special value strictly lowered the error
 };
 
+// Per-launch constants of the block quantizer: ts, 6*ts with its correctly
+// rounded reciprocal, and per scale code c the divisor d = dec(c) * ts and
+// RN(1/d) (0 where d is outside [2^-90, 2^90], where the IEEE divide is used).
+struct ScaleCtx {
+    float ts, six_ts, y6;
+    const float *tab_d, *tab_y;  // shared memory, one entry per magnitude code
+};
+
 template <int FMT>
-__device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], float ts)
+__device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const ScaleCtx &k)
 {
+    const float ts = k.ts;
     using F = Fmt<FMT>;
     BlockOut o;
     o.packed = make_uint2(0u, 0u);
@@ -103,17 +112,25 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], float t
     for (int j = 0; j < 16; j++) amax = fmaxf(amax, fabsf(x[j]));
     if (!(ts > 0.0f)) return o;
 
-    // block scale: s_f = amax_b / (6 ts), nearest scale code, exact decode
-    const float sf = __fdiv_rn(amax, __fmul_rn(6.0f, ts));
+    // block scale: s_f = RN(amax_b / RN(6 ts)), nearest scale code.  amax_b is
+    // an fp16/bf16 value, so Markstein's correction of amax_b * RN(1/(6 ts))
+    // is the IEEE quotient (the same proof as for X^scaled) while both
+    // operands stay well inside the normal range.
+    float sf;
+    if (k.y6 != 0.0f && amax >= 0x1p-60f && amax <= 0x1p60f) {
+        const float q = __fmul_rn(amax, k.y6);
+        sf = __fmaf_rn(__fmaf_rn(-q, k.six_ts, amax), k.y6, q);
+    } else {
+        sf = __fdiv_rn(amax, k.six_ts);
+    }
     const unsigned sc = encode_scale<FMT>(sf);
-    const float s = decode_scale<FMT>(sc);
-    const float d = __fmul_rn(s, ts);
+    const float d = k.tab_d[sc];  // dec(sc) * ts
     if (sc == 0u || d == 0.0f) return o;
 
     // X^scaled = RN(x / d)
     float xs[16];
-    if (d >= 0x1p-90f && d <= 0x1p90f) {
-        const float y = __frcp_rn(d);
+    const float y = k.tab_y[sc];  // RN(1/d), or 0 outside the Markstein range
+    if (y != 0.0f) {
         const float2 y2 = make_float2(y, y), nd2 = make_float2(-d, -d);
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
@@ -239,6 +256,20 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const TIn *__restri
     const float ts = ts_is_amax ? __fdiv_rn(tv, F::kC) : tv;
     unsigned cnt[4] = {0u, 0u, 0u, 0u};
 
+    __shared__ float tab_d[F::kMagMask + 1], tab_y[F::kMagMask + 1];
+    for (int c = threadIdx.x; c <= (int)F::kMagMask; c += blockDim.x) {
+        const float d = __fmul_rn(decode_scale<FMT>((unsigned)c), ts);
+        tab_d[c] = d;
+        tab_y[c] = (d >= 0x1p-90f && d <= 0x1p90f) ? __frcp_rn(d) : 0.0f;
+    }
+    ScaleCtx k;
+    k.ts = ts;
+    k.six_ts = __fmul_rn(6.0f, ts);
+    k.y6 = (k.six_ts >= 0x1p-60f && k.six_ts <= 0x1p60f) ? __frcp_rn(k.six_ts) : 0.0f;
+    k.tab_d = tab_d;
+    k.tab_y = tab_y;
+    __syncthreads();
+
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
         const uint4 *p = reinterpret_cast<const uint4 *>(x) + 2 * b;
@@ -252,7 +283,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const TIn *__restri
             xv[2 * i] = f.x;
             xv[2 * i + 1] = f.y;
         }
-        const BlockOut o = quantize_block<FMT>(xv, ts);
+        const BlockOut o = quantize_block<FMT>(xv, k);
         reinterpret_cast<uint2 *>(codes)[b] = o.packed;
         scales[b] = (uint8_t)o.sbyte;
         if constexpr (F::kSpecials > 0) {
