@@ -364,25 +364,6 @@ static Plan plan(int64_t B, int64_t N, int64_t K)
     return p;
 }
 
-// launch with the programmatic-stream-serialization attribute: the kernel may
-// be scheduled before its predecessor in the stream has finished, and waits
-// for it with griddepcontrol.wait before touching memory the predecessor wrote
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st, Args... args)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
 template <int FMT, bool BF16, int NB>
 static razer_status launch(const CUtensorMap &tc, const CUtensorMap &tsc, const CUtensorMap &tx, int B, int N, const Plan &pl,
                            float *ws, const float *ts, float unbias, void *y, razer_dtype out_dt, cudaStream_t st)

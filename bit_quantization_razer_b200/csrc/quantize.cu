@@ -252,6 +252,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const TIn *__restri
                                                              unsigned long long *__restrict__ hist)
 {
     using F = Fmt<FMT>;
+    pdl_wait();  // x, ts and the histogram come from earlier kernels in the stream
+    pdl_trigger();
     const float tv = *ts_src;
     const float ts = ts_is_amax ? __fdiv_rn(tv, F::kC) : tv;
     unsigned cnt[4] = {0u, 0u, 0u, 0u};
@@ -319,6 +321,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const TIn *__restri
 template <typename TIn>
 __global__ void __launch_bounds__(256) amax_kernel(const TIn *__restrict__ x, int64_t nvec, unsigned *__restrict__ out)
 {
+    pdl_wait();
+    pdl_trigger();
     float m = 0.0f;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const uint4 *p = reinterpret_cast<const uint4 *>(x);
@@ -346,11 +350,26 @@ __global__ void __launch_bounds__(256) amax_kernel(const TIn *__restrict__ x, in
 // ts = amax / (6 * S_max), written over the amax word.
 __global__ void finalize_ts_kernel(float *ts, float c)
 {
+    pdl_wait();
     const float amax = __uint_as_float(*reinterpret_cast<unsigned *>(ts));
     *ts = __fdiv_rn(amax, c);
 }
 
-__global__ void copy_ts_kernel(const float *src, float *dst) { *dst = *src; }
+__global__ void copy_ts_kernel(const float *src, float *dst)
+{
+    pdl_wait();
+    *dst = *src;
+}
+
+// zeroes the histogram and the amax accumulator of a quantizer call (one
+// launch instead of two memsets)
+__global__ void quant_init_kernel(unsigned long long *hist, unsigned *amax_bits)
+{
+    pdl_wait();
+    pdl_trigger();
+    if (hist && threadIdx.x < 4) hist[threadIdx.x] = 0ull;
+    if (amax_bits && threadIdx.x == 0) *amax_bits = 0u;
+}
 
 // ---------------------------------------------------------------------------
 // Host launchers.
@@ -367,15 +386,15 @@ template <typename TIn>
 static void launch_amax(const void *x, int64_t n, unsigned *out, cudaStream_t st)
 {
     const int64_t nvec = n / 8;
-    amax_kernel<TIn><<<quant_grid(nvec, 256, 8), 256, 0, st>>>(reinterpret_cast<const TIn *>(x), nvec, out);
+    launch_pdl(amax_kernel<TIn>, (unsigned)quant_grid(nvec, 256, 8), 256u, 0, st, reinterpret_cast<const TIn *>(x), nvec, out);
 }
 
 template <int FMT, typename TIn>
 static void launch_quant(const void *x, int64_t nblk, const float *ts_src, int is_amax, uint8_t *codes,
                          uint8_t *scales, unsigned long long *hist, cudaStream_t st)
 {
-    quantize_kernel<FMT, TIn><<<quant_grid(nblk, kQThreads, 8), kQThreads, 0, st>>>(
-        reinterpret_cast<const TIn *>(x), nblk, ts_src, is_amax, codes, scales, hist);
+    launch_pdl(quantize_kernel<FMT, TIn>, (unsigned)quant_grid(nblk, kQThreads, 8), (unsigned)kQThreads, 0, st,
+               reinterpret_cast<const TIn *>(x), nblk, ts_src, is_amax, codes, scales, hist);
 }
 
 template <int FMT>
@@ -394,11 +413,16 @@ razer_status run_quantize(const void *x, razer_dtype dt, int64_t R, int64_t K, c
     const int64_t n = R * K;
     const int64_t nblk = n / 16;
     const float C = fmt == RAZER_FMT_WEIGHT ? Fmt<RAZER_FMT_WEIGHT>::kC : Fmt<RAZER_FMT_ACT>::kC;
-    if (hist && cudaMemsetAsync(hist, 0, 4 * sizeof(unsigned long long), st) != cudaSuccess) return RAZER_ERR_CUDA;
+    // every kernel of the chain is a programmatic dependent of the previous one
+    // (it is scheduled early and waits before touching memory)
+    if (hist || !ts_in) {
+        if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, hist, ts_in ? (unsigned *)nullptr : reinterpret_cast<unsigned *>(ts_out)) !=
+            cudaSuccess)
+            return RAZER_ERR_CUDA;
+    }
     const float *ts_src = ts_in;
     int is_amax = 0;
     if (!ts_in) {
-        if (cudaMemsetAsync(ts_out, 0, sizeof(float), st) != cudaSuccess) return RAZER_ERR_CUDA;
         if (n > 0) {
             if (dt == RAZER_F16) launch_amax<__half>(x, n, reinterpret_cast<unsigned *>(ts_out), st);
             else launch_amax<__nv_bfloat16>(x, n, reinterpret_cast<unsigned *>(ts_out), st);
@@ -411,8 +435,11 @@ razer_status run_quantize(const void *x, razer_dtype dt, int64_t R, int64_t K, c
         else if (fmt == RAZER_FMT_ACT) launch_quant_dt<RAZER_FMT_ACT>(dt, x, nblk, ts_src, is_amax, codes, scales, hist, st);
         else launch_quant_dt<RAZER_FMT_NVFP4>(dt, x, nblk, ts_src, is_amax, codes, scales, nullptr, st);
     }
-    if (!ts_in) finalize_ts_kernel<<<1, 1, 0, st>>>(ts_out, C);
-    else if (ts_out != ts_in) copy_ts_kernel<<<1, 1, 0, st>>>(ts_in, ts_out);
+    if (!ts_in) {
+        if (launch_pdl(finalize_ts_kernel, 1u, 1u, 0, st, ts_out, C) != cudaSuccess) return RAZER_ERR_CUDA;
+    } else if (ts_out != ts_in) {
+        if (launch_pdl(copy_ts_kernel, 1u, 1u, 0, st, ts_in, ts_out) != cudaSuccess) return RAZER_ERR_CUDA;
+    }
     return last_launch_status();
 }
 

@@ -130,6 +130,30 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p)
 
 // Launch helpers shared by the host files --------------------------------------
 namespace razer {
+// launch with the programmatic-stream-serialization attribute: the kernel may
+// be scheduled before its predecessor in the stream has finished, and waits
+// for it with griddepcontrol.wait before touching memory the predecessor wrote
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// in a kernel launched that way: wait for the predecessor grid (no-op otherwise)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// let the dependent grid be scheduled (it still waits for this grid to finish)
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 int sm_count();
 razer_status last_launch_status();
 }  // namespace razer
