@@ -34,17 +34,33 @@
 namespace razer {
 namespace gemm {
 
-constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
+#ifndef RAZER_GEMM_BM
+#define RAZER_GEMM_BM 256
+#endif
+#ifndef RAZER_GEMM_BN
+#define RAZER_GEMM_BN 256
+#endif
+#ifndef RAZER_GEMM_STAGES
+#define RAZER_GEMM_STAGES 3
+#endif
+// CTA tile BM x BN x 64: BM / 128 UMMAs of M = 128 share each decoded BN-row
+// weight tile (every weight is decoded once per BM activation rows); the
+// accumulators fill (BM / 128) * BN = 512 TMEM columns.
+constexpr int BM = RAZER_GEMM_BM, BN = RAZER_GEMM_BN, BK = 64, STAGES = RAZER_GEMM_STAGES;
+constexpr int kMBlocks = BM / 128;
+static_assert(kMBlocks * BN == 512, "the accumulators fill the 512 TMEM columns");
 #ifndef RAZER_GEMM_DECODE_WARPS
 #define RAZER_GEMM_DECODE_WARPS 8
 #endif
 constexpr int kDecodeWarps = RAZER_GEMM_DECODE_WARPS;  // 8: a row per thread; 16: half a row per thread
-constexpr int kHalvesPerThread = 16 / kDecodeWarps;
+constexpr int kThreadsPerRow = 32 * kDecodeWarps / BN;   // decoder threads per weight row (1 or 2)
+constexpr int kHalvesPerThread = 2 / kThreadsPerRow;     // 32-code halves of a k-step per thread
+static_assert(kThreadsPerRow >= 1 && kThreadsPerRow <= 2, "one or two decoder threads per row");
 constexpr int kFirstDecodeWarp = 2;  // warp 0: X TMA, 1: MMA
 constexpr int kThreads = 32 * kFirstDecodeWarp + 32 * kDecodeWarps;
-constexpr uint32_t A_HALF_BYTES = 128 * BK * 2;               // 16 KB
-constexpr uint32_t B_BYTES = BN * BK * 2;                     // 32 KB (decoded weights)
-constexpr uint32_t STAGE_BYTES = 2 * A_HALF_BYTES + B_BYTES;  // 64 KB
+constexpr uint32_t A_HALF_BYTES = 128 * BK * 2;                      // 16 KB: one 128-row block of X
+constexpr uint32_t B_BYTES = BN * BK * 2;                            // decoded weights
+constexpr uint32_t STAGE_BYTES = kMBlocks * A_HALF_BYTES + B_BYTES;  // 64 KB (256x256) / 80 KB (512x128)
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -220,9 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
                 if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort_flag)) break;
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
-                mbar_expect_tx(full_a + 8 * s, 2 * A_HALF_BYTES);
-                tma_load_2d(a0, &tmap_x, kb * BK, m0, full_a + 8 * s);
-                tma_load_2d(a0 + A_HALF_BYTES, &tmap_x, kb * BK, m0 + 128, full_a + 8 * s);
+                mbar_expect_tx(full_a + 8 * s, kMBlocks * A_HALF_BYTES);
+#pragma unroll
+                for (int a = 0; a < kMBlocks; a++) tma_load_2d(a0 + a * A_HALF_BYTES, &tmap_x, kb * BK, m0 + 128 * a, full_a + 8 * s);
                 issued = kb + 1;
             }
             if (*abort_flag) {
@@ -248,13 +264,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
-                const uint32_t b0 = a0 + 2 * A_HALF_BYTES;
+                const uint32_t b0 = a0 + kMBlocks * A_HALF_BYTES;
 #pragma unroll
                 for (int k = 0; k < BK / 16; k++) {
                     const uint64_t bd = smem_desc_k128(b0 + 32 * k);
                     const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                    umma_f16(tmem, smem_desc_k128(a0 + 32 * k), bd, idesc, acc);
-                    umma_f16(tmem + 256, smem_desc_k128(a0 + A_HALF_BYTES + 32 * k), bd, idesc, acc);
+#pragma unroll
+                    for (int a = 0; a < kMBlocks; a++)
+                        umma_f16(tmem + a * BN, smem_desc_k128(a0 + a * A_HALF_BYTES + 32 * k), bd, idesc, acc);
                 }
                 umma_commit(empty + 8 * s);
             }
@@ -269,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---------------- decoders, then epilogue ----------------
         const int dt = threadIdx.x - 32 * kFirstDecodeWarp;  // 0 .. 32*kDecodeWarps-1
-        const int row = dt & (BN - 1);                      // 0..255
-        const int hk0 = kHalvesPerThread == 1 ? (dt >> 8) : 0;  // first 32-element half of the k-step
+        const int row = dt & (BN - 1);                                // weight row of the tile
+        const int hk0 = kHalvesPerThread == 1 ? (dt / BN) : 0;        // first 32-element half of the k-step
         const int n = n0 + row;
         const bool valid = n < N;
         const uint8_t *crow = codes + (size_t)(valid ? n : (N - 1)) * (K >> 1) + 16 * hk0;
@@ -305,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            uint8_t *rbase = smem + s * STAGE_BYTES + 2 * A_HALF_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+            uint8_t *rbase = smem + s * STAGE_BYTES + kMBlocks * A_HALF_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
             for (int h = 0; h < kHalvesPerThread; h++) {
                 const unsigned words[4] = {c0[h].x, c0[h].y, c0[h].z, c0[h].w};
@@ -335,12 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int cbeg = ((warp - kFirstDecodeWarp) >> 2) * (BN * 4 / kDecodeWarps);
             const float scale = __fmul_rn(*ts_p, unbias);
 #pragma unroll 1
-            for (int half = 0; half < 2; half++) {
+            for (int half = 0; half < kMBlocks; half++) {
                 const int m = m0 + half * 128 + q * 32 + lane;
 #pragma unroll 1
                 for (int c0 = cbeg; c0 < cbeg + BN * 4 / kDecodeWarps; c0 += 32) {
                     float v[32];
-                    tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 256 + c0), v);
+                    tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * BN + c0), v);
                     const int n = n0 + c0;
                     if (m < M && n < N && n + 32 > N) {
                         for (int i = 0; i < N - n; i++) {
