@@ -70,24 +70,30 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def source_hash():
+TRAFFIC_SOURCES = {  # the files each timed call's kernels are built from
+    "quantize_kernel": ["quantize.cu", "razer_internal.cuh"],
+    "gemv_kernel": ["gemv_tma.cu", "gemv.cu", "sm100_async.cuh", "razer_internal.cuh"],
+}
+
+
+def source_hash(files):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_quantization_razer_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in files:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources."""
+    """DRAM bytes per call from the committed ncu summary, if it was taken on
+    the current sources of that kernel."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    if d.get("source_hash") != source_hash():
+    e = json.load(open(p)).get("kernels", {}).get(kernel)
+    if not e or e.get("source_hash") != source_hash(TRAFFIC_SOURCES[kernel]):
         return None
-    return d.get("kernels", {}).get(kernel)
+    return e.get("bytes_per_call")
 
 
 class ClockSampler:

@@ -96,7 +96,12 @@ struct ScaleCtx {
     const float *tab_d, *tab_y;  // shared memory, one entry per magnitude code
 };
 
-template <int FMT>
+// FAST: the launch-wide preconditions of the fast path hold (ts in
+// [2^-62, 2^57]): RN(1/(6 ts)) and RN(1/d) of every non-zero scale code are
+// valid Markstein reciprocals, so the block needs no divide fallback and no
+// early exit (a zero scale code is zeroed by selects at the end).  F16IN: the
+// elements are fp16, whose amax is 0 or in [2^-24, 65504].
+template <int FMT, bool FAST, bool F16IN>
 __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const ScaleCtx &k)
 {
     const float ts = k.ts;
@@ -110,14 +115,14 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
     float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; j++) amax = fmaxf(amax, fabsf(x[j]));
-    if (!(ts > 0.0f)) return o;
+    if (!FAST && !(ts > 0.0f)) return o;
 
     // block scale: s_f = RN(amax_b / RN(6 ts)), nearest scale code.  amax_b is
     // an fp16/bf16 value, so Markstein's correction of amax_b * RN(1/(6 ts))
     // is the IEEE quotient (the same proof as for X^scaled) while both
     // operands stay well inside the normal range.
     float sf;
-    if (k.y6 != 0.0f && amax >= 0x1p-60f && amax <= 0x1p60f) {
+    if ((FAST && F16IN) || (k.y6 != 0.0f && ((amax >= 0x1p-60f && amax <= 0x1p60f) || amax == 0.0f))) {
         const float q = __fmul_rn(amax, k.y6);
         sf = __fmaf_rn(__fmaf_rn(-q, k.six_ts, amax), k.y6, q);
     } else {
@@ -125,12 +130,12 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
     }
     const unsigned sc = encode_scale<FMT>(sf);
     const float d = k.tab_d[sc];  // dec(sc) * ts
-    if (sc == 0u || d == 0.0f) return o;
+    if (!FAST && (sc == 0u || d == 0.0f)) return o;
 
     // X^scaled = RN(x / d)
     float xs[16];
     const float y = k.tab_y[sc];  // RN(1/d), or 0 outside the Markstein range
-    if (y != 0.0f) {
+    if (FAST || y != 0.0f) {
         const float2 y2 = make_float2(y, y), nd2 = make_float2(-d, -d);
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
@@ -180,12 +185,29 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
         const float dn5 = __fmul_rn(__fadd_rn(A, Bs), 0.5f);
         float best = dp5;
         if (dn5 < best) { best = dn5; meta = 1u; }
+        // final encode against Q_FP4 u {v*}: elements nearest to v* take
+        // 0b1000.  For v* = +5 the region is xs in (4.5, 5.5], for v* = -5 it
+        // is [-5.5, -4.5) (ties go to the smaller magnitude): |xs| in
+        // (4.5, 5.5] with the sign of v*.  In terms of e = 2|xs| - 10 (exact
+        // there, a multiple of 2^-20) that is e in (-1, 1], i.e. the sign bit of
+        // r = |e - 2^-22| - 1.  The E2M1 convert keeps the sign of r in bit 3 of
+        // each nibble, which gathers the 16 tests with 4 converts; the sign of
+        // xs is the plain code's sign bit (the plain code is +-4 or +-6 there).
+        unsigned o0, o1;
+        {
+            float r[16];
+#pragma unroll
+            for (int j = 0; j < 16; j++) r[j] = __fadd_rn(fabsf(__fadd_rn(ea[j], -0x1p-22f)), -1.0f);
+            const unsigned in0 = cvt_e2m1x8(r) & 0x88888888u, in1 = cvt_e2m1x8(r + 8) & 0x88888888u;
+            o0 = in0 & (meta ? w0 : ~w0);
+            o1 = in1 & (meta ? w1 : ~w1);
+        }
         if constexpr (F::kSpecials == 4) {
             // v = +8 / -8 changes an element only when |xs| > 7.  With a
             // normal scale code |xs| <= 6 / (1 - 2^-4) < 7, so only blocks with
-            // a subnormal scale code (sc < 8) can use them; there |xs| <= 9
+            // a subnormal scale code (0 < sc < 8) can use them; there |xs| <= 9
             // and the terms are summed exactly as integers in units of 2^-20.
-            if (sc < 8u) {
+            if (sc - 1u < 7u) {
                 int ip5 = 0, in5 = 0, ip8 = 0, in8 = 0;
 #pragma unroll
                 for (int j = 0; j < 16; j++) {
@@ -199,44 +221,35 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
                     in8 += __float2int_rn(__fmul_rn(t8n, 1048576.0f));
                 }
                 int ib = ip5;
-                meta = 0u;
-                if (in5 < ib) { ib = in5; meta = 1u; }
-                if (ip8 < ib) { ib = ip8; meta = 2u; }
-                if (in8 < ib) { ib = in8; meta = 3u; }
+                unsigned m8 = 0u;
+                if (in5 < ib) { ib = in5; m8 = 1u; }
+                if (ip8 < ib) { ib = ip8; m8 = 2u; }
+                if (in8 < ib) { ib = in8; m8 = 3u; }
                 best = (float)ib;
+                if (m8 >= 2u) {
+                    // +8 (7, inf] / -8 [-inf, -7): one interval of bit patterns each
+                    const unsigned lo = 0x40E00001u | ((m8 & 1u) << 31), span = 0x7F800000u - 0x40E00001u;
+                    o0 = o1 = 0u;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        o0 |= (__float_as_uint(xs[j]) - lo <= span) ? (8u << (4 * j)) : 0u;
+                        o1 |= (__float_as_uint(xs[j + 8]) - lo <= span) ? (8u << (4 * j)) : 0u;
+                    }
+                }
+                // below 2 the integer decision repeats the +-5 one (the same exact sums)
+                meta = m8;
             }
         }
         o.effective = best < 0.0f;
-
-        // final encode against Q_FP4 u {v*}: elements nearest to v* take
-        // 0b1000.  For v* = +5 the region is xs in (4.5, 5.5], for v* = -5 it
-        // is [-5.5, -4.5) (ties go to the smaller magnitude): |xs| in
-        // (4.5, 5.5] with the sign of v*.  In terms of e = 2|xs| - 10 (exact
-        // there, a multiple of 2^-20) that is e in (-1, 1], i.e. the sign bit of
-        // r = |e - 2^-22| - 1.  The E2M1 convert keeps the sign of r in bit 3 of
-        // each nibble, which gathers the 16 tests with 4 converts; the sign of
-        // xs is the plain code's sign bit (the plain code is +-4 or +-6 there).
-        unsigned o0 = 0u, o1 = 0u;
-        if (meta < 2u) {
-            float r[16];
-#pragma unroll
-            for (int j = 0; j < 16; j++) r[j] = __fadd_rn(fabsf(__fadd_rn(ea[j], -0x1p-22f)), -1.0f);
-            const unsigned in0 = cvt_e2m1x8(r) & 0x88888888u, in1 = cvt_e2m1x8(r + 8) & 0x88888888u;
-            o0 = in0 & ((meta & 1u) ? w0 : ~w0);
-            o1 = in1 & ((meta & 1u) ? w1 : ~w1);
-        } else {
-            // +8 (7, inf] / -8 [-inf, -7): one interval of bit patterns each
-            const unsigned lo = 0x40E00001u | ((meta & 1u) << 31), span = 0x7F800000u - 0x40E00001u;
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                o0 |= (__float_as_uint(xs[j]) - lo <= span) ? (8u << (4 * j)) : 0u;
-                o1 |= (__float_as_uint(xs[j + 8]) - lo <= span) ? (8u << (4 * j)) : 0u;
-            }
-        }
         w0 = (w0 & ~((o0 >> 3) * 15u)) | o0;
         w1 = (w1 & ~((o1 >> 3) * 15u)) | o1;
     }
 
+    if (FAST && sc == 0u) {  // amax_b rounds to a zero scale: all-zero block (selects, no branch)
+        w0 = w1 = 0u;
+        meta = 0u;
+        o.effective = false;
+    }
     o.packed = make_uint2(w0, w1);
     o.meta = meta;
     o.sbyte = sc | (meta << F::kMetaShift);
@@ -245,7 +258,37 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
 
 constexpr int kQThreads = 256;
 
-template <int FMT, typename TIn>
+template <int FMT, typename TIn, bool FAST, bool HIST>
+__device__ __forceinline__ void quant_loop(const TIn *__restrict__ x, int64_t nblk, const ScaleCtx &k, uint8_t *__restrict__ codes,
+                                           uint8_t *__restrict__ scales, unsigned (&cnt)[4])
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(x) + 2 * b;
+        const uint4 v0 = ldg_stream(p);
+        const uint4 v1 = ldg_stream(p + 1);
+        float xv[16];
+        const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float2 f = In16<TIn>::to_f2(wv[i]);
+            xv[2 * i] = f.x;
+            xv[2 * i + 1] = f.y;
+        }
+        const BlockOut o = quantize_block<FMT, FAST, std::is_same<TIn, __half>::value>(xv, k);
+        reinterpret_cast<uint2 *>(codes)[b] = o.packed;
+        scales[b] = (uint8_t)o.sbyte;
+        if constexpr (HIST) {
+            const unsigned m1 = o.meta & 1u, e = o.effective ? 1u : 0u;
+            cnt[0] += 1u - m1;
+            cnt[1] += m1;
+            cnt[2] += e & (1u - m1);
+            cnt[3] += e & m1;
+        }
+    }
+}
+
+template <int FMT, typename TIn, bool HIST>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(const TIn *__restrict__ x, int64_t nblk,
                                                              const float *__restrict__ ts_src, int ts_is_amax,
                                                              uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
@@ -272,47 +315,25 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const TIn *__restri
     k.tab_y = tab_y;
     __syncthreads();
 
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(x) + 2 * b;
-        const uint4 v0 = ldg_stream(p);
-        const uint4 v1 = ldg_stream(p + 1);
-        float xv[16];
-        const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    // launch-wide: with ts in [2^-62, 2^57] every reciprocal the blocks need
+    // is a valid Markstein reciprocal (d of a non-zero scale code lies in
+    // [2^-71, 2^66]), so the per-block fallbacks and early exits drop out
+    if (ts >= 0x1p-62f && ts <= 0x1p57f) quant_loop<FMT, TIn, true, HIST>(x, nblk, k, codes, scales, cnt);
+    else quant_loop<FMT, TIn, false, HIST>(x, nblk, k, codes, scales, cnt);
+
+    if constexpr (HIST) {
+        __shared__ unsigned long long sh[4];
+        if (threadIdx.x < 4) sh[threadIdx.x] = 0ull;
+        __syncthreads();
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const float2 f = In16<TIn>::to_f2(wv[i]);
-            xv[2 * i] = f.x;
-            xv[2 * i + 1] = f.y;
-        }
-        const BlockOut o = quantize_block<FMT>(xv, k);
-        reinterpret_cast<uint2 *>(codes)[b] = o.packed;
-        scales[b] = (uint8_t)o.sbyte;
-        if constexpr (F::kSpecials > 0) {
-            if (hist) {
-                const unsigned m1 = o.meta & 1u, e = o.effective ? 1u : 0u;
-                cnt[0] += 1u - m1;
-                cnt[1] += m1;
-                cnt[2] += e & (1u - m1);
-                cnt[3] += e & m1;
-            }
-        }
-    }
-    if constexpr (F::kSpecials > 0) {
-        if (hist) {
-            __shared__ unsigned long long sh[4];
-            if (threadIdx.x < 4) sh[threadIdx.x] = 0ull;
-            __syncthreads();
+        for (int i = 0; i < 4; i++) {
+            unsigned c = cnt[i];
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                unsigned c = cnt[i];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-                if ((threadIdx.x & 31) == 0 && c) atomicAdd(&sh[i], (unsigned long long)c);
-            }
-            __syncthreads();
-            if (threadIdx.x < 4 && sh[threadIdx.x]) atomicAdd(&hist[threadIdx.x], sh[threadIdx.x]);
+            for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+            if ((threadIdx.x & 31) == 0 && c) atomicAdd(&sh[i], (unsigned long long)c);
         }
+        __syncthreads();
+        if (threadIdx.x < 4 && sh[threadIdx.x]) atomicAdd(&hist[threadIdx.x], sh[threadIdx.x]);
     }
 }
 
@@ -393,8 +414,13 @@ template <int FMT, typename TIn>
 static void launch_quant(const void *x, int64_t nblk, const float *ts_src, int is_amax, uint8_t *codes,
                          uint8_t *scales, unsigned long long *hist, cudaStream_t st)
 {
-    launch_pdl(quantize_kernel<FMT, TIn>, (unsigned)quant_grid(nblk, kQThreads, 8), (unsigned)kQThreads, 0, st,
-               reinterpret_cast<const TIn *>(x), nblk, ts_src, is_amax, codes, scales, hist);
+    const unsigned grid = (unsigned)quant_grid(nblk, kQThreads, 8);
+    if (hist && Fmt<FMT>::kSpecials > 0)
+        launch_pdl(quantize_kernel<FMT, TIn, true>, grid, (unsigned)kQThreads, 0, st, reinterpret_cast<const TIn *>(x), nblk, ts_src,
+                   is_amax, codes, scales, hist);
+    else
+        launch_pdl(quantize_kernel<FMT, TIn, false>, grid, (unsigned)kQThreads, 0, st, reinterpret_cast<const TIn *>(x), nblk, ts_src,
+                   is_amax, codes, scales, hist);
 }
 
 template <int FMT>
