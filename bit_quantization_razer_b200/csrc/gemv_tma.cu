@@ -145,7 +145,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------- TMA producer -------------------------
         if (lane == 0) {
-            // inputs may come from the previous kernel in the stream
+            // the tensor maps are kernel parameters: fetch them while the
+            // previous kernel in the stream may still run; its outputs (which
+            // may be our inputs) are read only after griddepcontrol.wait
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_codes)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_scales)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
             asm volatile("griddepcontrol.wait;" ::: "memory");
             const uint32_t tx = (uint32_t)(kCodeBytes + kScaleBytes + B * 512);
             int s = 0, issued = 0;
@@ -330,6 +335,7 @@ __global__ void __launch_bounds__(256) gemv_tma_reduce_kernel(const float *__res
                                                               const float *__restrict__ ts_p, float unbias, void *__restrict__ y, int out_dt)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next call may become resident
     const float oscale = __fmul_rn(*ts_p, unbias);
     const int slot_elems = B * kTileRows;
     const int64_t total = (int64_t)T * slot_elems;
