@@ -461,9 +461,10 @@ def run_single_kernel(args):
         c, s, t = R.razer_quantize_weights(w)
         X = workloads.vectors(M, K, seed=4, dtype=torch.bfloat16).to(dev)
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        wsg = torch.empty(max(16, R.razer_workspace_size(R.RAZER_OP_GEMM, M, N, K)), dtype=torch.uint8, device=dev)
 
         def call():
-            R.razer_gemm(X, c, s, t, "weight", torch.bfloat16, out=Y)
+            R.razer_gemm(X, c, s, t, "weight", torch.bfloat16, out=Y, workspace=wsg)
     for _ in range(3):
         call()
     torch.cuda.synchronize()
@@ -529,12 +530,13 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
             w = workloads.weight(N, K, seed=401).to(dev)
             c, s, t = R.razer_quantize_weights(w)
             Yg = torch.empty((4096, N), dtype=torch.bfloat16, device=dev)
+            wsg = torch.empty(max(16, R.razer_workspace_size(R.RAZER_OP_GEMM, 4096, N, K)), dtype=torch.uint8, device=dev)
             for _ in range(3):
-                R.razer_gemm(Xg, c, s, t, "weight", torch.bfloat16, out=Yg)
+                R.razer_gemm(Xg, c, s, t, "weight", torch.bfloat16, out=Yg, workspace=wsg)
             reps = 20
             e0.record(stream)
             for _ in range(reps):
-                R.razer_gemm(Xg, c, s, t, "weight", torch.bfloat16, out=Yg)
+                R.razer_gemm(Xg, c, s, t, "weight", torch.bfloat16, out=Yg, workspace=wsg)
             e1.record(stream)
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / reps

@@ -26,6 +26,7 @@
 // normal range, which converts exactly to bf16 (at most 7 significant bits)
 // for bf16 activations.
 #include <cuda.h>
+#include <algorithm>
 #include <cstdlib>
 
 #include "razer_internal.cuh"
@@ -188,11 +189,15 @@ __device__ __forceinline__ uint4 decode_word(unsigned w, const BlockK &k)
     return make_uint4(p[0], p[1], p[2], p[3]);
 }
 
-template <int FMT, bool BF16>
+// DECODED: the weights were decoded once into a [N, K] 16-bit copy (q*s*2^-bias,
+// exact) that the producer loads by TMA like X; the decoder warps then only
+// run the epilogue.  CTA tiles are rasterised M-fastest so that the CTAs
+// sharing a weight tile run together and find it in L2.
+template <int FMT, bool BF16, bool DECODED>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
-                const float *__restrict__ ts_p, float unbias, int M, int N, int K, void *__restrict__ Y, int out_dt,
-                int inject_stall)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w, const uint8_t *__restrict__ codes,
+                const uint8_t *__restrict__ scales, const float *__restrict__ ts_p, float unbias, int M, int N, int K,
+                void *__restrict__ Y, int out_dt, int inject_stall)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 200);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+    const int n0 = (DECODED ? blockIdx.y : blockIdx.x) * BN, m0 = (DECODED ? blockIdx.x : blockIdx.y) * BM;
     const int KB = K / BK;
 
     if (threadIdx.x == 0) {
@@ -236,9 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
                 if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort_flag)) break;
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
-                mbar_expect_tx(full_a + 8 * s, kMBlocks * A_HALF_BYTES);
+                mbar_expect_tx(full_a + 8 * s, kMBlocks * A_HALF_BYTES + (DECODED ? B_BYTES : 0u));
 #pragma unroll
                 for (int a = 0; a < kMBlocks; a++) tma_load_2d(a0 + a * A_HALF_BYTES, &tmap_x, kb * BK, m0 + 128 * a, full_a + 8 * s);
+                if constexpr (DECODED) tma_load_2d(a0 + kMBlocks * A_HALF_BYTES, &tmap_w, kb * BK, n0, full_a + 8 * s);
                 issued = kb + 1;
             }
             if (*abort_flag) {
@@ -260,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < KB && ok; kb++) {
                 const int s = kb % STAGES;
                 const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-                ok = mbar_wait(full_a + 8 * s, ph, abort_flag) && mbar_wait(full_b + 8 * s, ph, abort_flag);
+                ok = mbar_wait(full_a + 8 * s, ph, abort_flag) && (DECODED || mbar_wait(full_b + 8 * s, ph, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
@@ -305,10 +311,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         : *reinterpret_cast<const unsigned *>(srow + (size_t)kb * 4);
         };
         Regs r0, r1;
-        load_stage(0, r0);
-        if (KB > 1) load_stage(1, r1);
         bool ok = true;
-        for (int kb = 0; kb < KB; kb++) {
+        if (!DECODED) {
+            load_stage(0, r0);
+            if (KB > 1) load_stage(1, r1);
+        }
+        for (int kb = 0; kb < (DECODED ? 0 : KB); kb++) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
             uint4 c0[kHalvesPerThread];
@@ -406,44 +414,80 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Decodes the packed weights once into a [N, K] 16-bit copy holding
+// q*s*2^-bias (the exact values the fused kernel writes to shared memory);
+// one thread per 16-element block.
+template <int FMT, bool BF16>
+__global__ void __launch_bounds__(256) decode_weights_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                                                             int64_t nblk, uint4 *__restrict__ out)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+        const uint2 c = ldg_stream_u2(reinterpret_cast<const uint2 *>(codes) + b);
+        const BlockK kc = block_consts<FMT>(scales[b]);
+        out[2 * b] = decode_word<FMT, BF16>(c.x, kc);
+        out[2 * b + 1] = decode_word<FMT, BF16>(c.y, kc);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int FMT, bool BF16>
-static razer_status launch(const CUtensorMap &map, const uint8_t *codes, const uint8_t *scales, const float *ts, float unbias,
-                           int M, int N, int K, void *Y, razer_dtype out_dt, cudaStream_t st)
+// decode once and run the plain 16-bit GEMM when M is large enough that the
+// fused kernel would decode every weight many times (M / BM) and the caller
+// provided the N x K x 2 bytes of workspace
+constexpr int64_t kDecodedMinM = 1024;
+
+template <int FMT, bool BF16, bool DECODED>
+static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                           float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, cudaStream_t st)
 {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(gemm_kernel<FMT, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_kernel<FMT, BF16, DECODED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+            cudaSuccess)
             return RAZER_ERR_CUDA;
         attr_set[dev] = true;
     }
-    dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+    const unsigned nt = (unsigned)((N + BN - 1) / BN), mt = (unsigned)((M + BM - 1) / BM);
+    const dim3 grid = DECODED ? dim3(mt, nt) : dim3(nt, mt);
     // RAZER_FAULT_INJECT_STALL=1 (tests only) withholds one decoder warp's
     // arrivals so that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
     const char *inj = getenv("RAZER_FAULT_INJECT_STALL");
     const int inject = (inj && inj[0] == '1') ? 1 : 0;
-    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt, inject);
+    gemm_kernel<FMT, BF16, DECODED><<<grid, kThreads, SMEM_BYTES, st>>>(map, wmap, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt,
+                                                                      inject);
     return last_launch_status();
+}
+
+template <int FMT, bool BF16>
+static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, bool decoded, const uint8_t *codes, const uint8_t *scales,
+                               const float *ts, float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, void *wdec, cudaStream_t st)
+{
+    if (!decoded) return launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, Y, out_dt, st);
+    const int64_t nblk = (int64_t)N * K / 16;
+    const int64_t g = std::min<int64_t>((nblk + 255) / 256, (int64_t)sm_count() * 8);
+    if (launch_pdl(decode_weights_kernel<FMT, BF16>, (unsigned)g, 256u, 0, st, codes, scales, nblk, reinterpret_cast<uint4 *>(wdec)) !=
+        cudaSuccess)
+        return RAZER_ERR_CUDA;
+    return launch<FMT, BF16, true>(map, wmap, codes, scales, ts, unbias, M, N, K, Y, out_dt, st);
 }
 
 }  // namespace gemm
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
-    (void)M;
-    (void)N;
-    (void)K;
-    return 0;
+    // the decoded weight copy, when the decode-once path applies
+    return M >= gemm::kDecodedMinM ? (size_t)N * (size_t)K * 2 : 0;
 }
 
 razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
                       razer_format wfmt, int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st)
 {
-    (void)workspace;
     using namespace gemm;
     if (K == 0) {
         const size_t esz = out_dt == RAZER_F32 ? 4 : 2;
@@ -463,15 +507,27 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
         return RAZER_ERR_CUDA;
     // the decoded q*s carries 2^-8 (E3M3) / 2^-4 (E4M3); undone in the epilogue
     const float unbias = wfmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f;
+    const bool decoded = M >= kDecodedMinM && workspace != nullptr;
+    CUtensorMap wmap = map;  // unused by the fused kernel
+    if (decoded) {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BN};
+        const cuuint32_t estr[2] = {1u, 1u};
+        if (enc(&wmap, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, workspace, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return RAZER_ERR_CUDA;
+    }
     const int m = (int)M, n = (int)N, k = (int)K;
     if (wfmt == RAZER_FMT_WEIGHT)
-        return bf ? launch<RAZER_FMT_WEIGHT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
-                  : launch<RAZER_FMT_WEIGHT, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
+        return bf ? launch_fmt<RAZER_FMT_WEIGHT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st)
+                  : launch_fmt<RAZER_FMT_WEIGHT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st);
     if (wfmt == RAZER_FMT_ACT)
-        return bf ? launch<RAZER_FMT_ACT, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
-                  : launch<RAZER_FMT_ACT, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
-    return bf ? launch<RAZER_FMT_NVFP4, true>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st)
-              : launch<RAZER_FMT_NVFP4, false>(map, codes, scales, ts, unbias, m, n, k, Y, out_dt, st);
+        return bf ? launch_fmt<RAZER_FMT_ACT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st)
+                  : launch_fmt<RAZER_FMT_ACT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st);
+    return bf ? launch_fmt<RAZER_FMT_NVFP4, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st)
+              : launch_fmt<RAZER_FMT_NVFP4, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st);
 }
 
 }  // namespace razer

@@ -117,6 +117,12 @@ template <> struct In16<__nv_bfloat16> {
     }
 };
 
+__device__ __forceinline__ uint2 ldg_stream_u2(const uint2 *p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint4 ldg_stream(const void *p)
 {
     uint4 v;
