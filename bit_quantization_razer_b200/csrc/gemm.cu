@@ -197,7 +197,7 @@ template <int FMT, bool BF16, bool DECODED>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w, const uint8_t *__restrict__ codes,
                 const uint8_t *__restrict__ scales, const float *__restrict__ ts_p, float unbias, int M, int N, int K,
-                void *__restrict__ Y, int out_dt, int inject_stall)
+                void *Y, int out_dt, int kb0, int nkb, const float *addend, int inject_stall)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -211,7 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = (DECODED ? blockIdx.y : blockIdx.x) * BN, m0 = (DECODED ? blockIdx.x : blockIdx.y) * BM;
-    const int KB = K / BK;
+    // this launch covers k-steps [kb0, kb0 + nkb) of the K / 64; a previous
+    // chunk's fp32 result (already scaled) is added in the epilogue
+    const int KB = nkb;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
@@ -243,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
                 mbar_expect_tx(full_a + 8 * s, kMBlocks * A_HALF_BYTES + (DECODED ? B_BYTES : 0u));
 #pragma unroll
-                for (int a = 0; a < kMBlocks; a++) tma_load_2d(a0 + a * A_HALF_BYTES, &tmap_x, kb * BK, m0 + 128 * a, full_a + 8 * s);
-                if constexpr (DECODED) tma_load_2d(a0 + kMBlocks * A_HALF_BYTES, &tmap_w, kb * BK, n0, full_a + 8 * s);
+                for (int a = 0; a < kMBlocks; a++) tma_load_2d(a0 + a * A_HALF_BYTES, &tmap_x, (kb0 + kb) * BK, m0 + 128 * a, full_a + 8 * s);
+                if constexpr (DECODED) tma_load_2d(a0 + kMBlocks * A_HALF_BYTES, &tmap_w, (kb0 + kb) * BK, n0, full_a + 8 * s);
                 issued = kb + 1;
             }
             if (*abort_flag) {
@@ -306,9 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto load_stage = [&](int kb, Regs &r) {
 #pragma unroll
-            for (int h = 0; h < kHalvesPerThread; h++) r.c[h] = ldg_stream(crow + (size_t)kb * 32 + 16 * h);
-            r.s = kHalvesPerThread == 1 ? (unsigned)*reinterpret_cast<const unsigned short *>(srow + (size_t)kb * 4)
-                                        : *reinterpret_cast<const unsigned *>(srow + (size_t)kb * 4);
+            for (int h = 0; h < kHalvesPerThread; h++) r.c[h] = ldg_stream(crow + (size_t)(kb0 + kb) * 32 + 16 * h);
+            r.s = kHalvesPerThread == 1 ? (unsigned)*reinterpret_cast<const unsigned short *>(srow + (size_t)(kb0 + kb) * 4)
+                                        : *reinterpret_cast<const unsigned *>(srow + (size_t)(kb0 + kb) * 4);
         };
         Regs r0, r1;
         bool ok = true;
@@ -367,19 +369,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float v[32];
                     tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * BN + c0), v);
                     const int n = n0 + c0;
-                    if (m < M && n < N && n + 32 > N) {
-                        for (int i = 0; i < N - n; i++) {
-                            const float a = v[i] * scale;
-                            if (out_dt == RAZER_F32) reinterpret_cast<float *>(Y)[(size_t)m * N + n + i] = a;
-                            else if (out_dt == RAZER_BF16) reinterpret_cast<__nv_bfloat16 *>(Y)[(size_t)m * N + n + i] = __float2bfloat16_rn(a);
-                            else reinterpret_cast<__half *>(Y)[(size_t)m * N + n + i] = __float2half_rn(a);
+                    if (m < M && n < N) {
+                        const int cnt = min(32, N - n);
+                        const float *add = addend ? addend + (size_t)m * N + n : nullptr;
+                        if (add && cnt == 32) {
+#pragma unroll
+                            for (int i = 0; i < 8; i++) {
+                                const float4 t = reinterpret_cast<const float4 *>(add)[i];
+                                v[4 * i] = __fmaf_rn(v[4 * i], scale, t.x);
+                                v[4 * i + 1] = __fmaf_rn(v[4 * i + 1], scale, t.y);
+                                v[4 * i + 2] = __fmaf_rn(v[4 * i + 2], scale, t.z);
+                                v[4 * i + 3] = __fmaf_rn(v[4 * i + 3], scale, t.w);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; i++) v[i] = (add && i < cnt) ? __fmaf_rn(v[i], scale, add[i]) : v[i] * scale;
                         }
-                    } else if (m < M && n < N) {
-                        if (out_dt == RAZER_F32) {
+                        if (cnt < 32) {
+                            for (int i = 0; i < cnt; i++) {
+                                const float a = v[i];
+                                if (out_dt == RAZER_F32) reinterpret_cast<float *>(Y)[(size_t)m * N + n + i] = a;
+                                else if (out_dt == RAZER_BF16) reinterpret_cast<__nv_bfloat16 *>(Y)[(size_t)m * N + n + i] = __float2bfloat16_rn(a);
+                                else reinterpret_cast<__half *>(Y)[(size_t)m * N + n + i] = __float2half_rn(a);
+                            }
+                        } else if (out_dt == RAZER_F32) {
                             float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(Y) + (size_t)m * N + n);
 #pragma unroll
-                            for (int i = 0; i < 8; i++)
-                                dst[i] = make_float4(v[4 * i] * scale, v[4 * i + 1] * scale, v[4 * i + 2] * scale, v[4 * i + 3] * scale);
+                            for (int i = 0; i < 8; i++) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                         } else {
                             uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(Y) + (size_t)m * N + n);
 #pragma unroll
@@ -387,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 unsigned p[4];
 #pragma unroll
                                 for (int e = 0; e < 4; e++) {
-                                    const float a = v[8 * i + 2 * e] * scale, b = v[8 * i + 2 * e + 1] * scale;
+                                    const float a = v[8 * i + 2 * e], b = v[8 * i + 2 * e + 1];
                                     if (out_dt == RAZER_BF16) {
                                         __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
                                         p[e] = *reinterpret_cast<unsigned *>(&h);
@@ -440,9 +456,25 @@ __global__ void __launch_bounds__(256) decode_weights_kernel(const uint8_t *__re
 // provided the N x K x 2 bytes of workspace
 constexpr int64_t kDecodedMinM = 1024;
 
+// Longest K one tensor-memory accumulation chain covers. The tcgen05 fp32
+// accumulator loses precision over long chains (measured on B200 with
+// decoded E3M3 weights: relative error ~5e-4 at K = 7168 but ~2.5e-3 at
+// K = 28672), so a longer K runs as equal chunks whose scaled partial sums
+// are added in fp32 through a [M, N] workspace buffer.
+#ifndef RAZER_GEMM_CHAIN_K
+#define RAZER_GEMM_CHAIN_K 16384
+#endif
+constexpr int64_t kMaxChainK = RAZER_GEMM_CHAIN_K;
+static_assert(kMaxChainK % BK == 0, "chain length must be whole k-steps");
+
+static int64_t num_chunks(int64_t K) { return (K + kMaxChainK - 1) / kMaxChainK; }
+static size_t decoded_bytes(int64_t M, int64_t N, int64_t K) { return M >= kDecodedMinM ? (size_t)N * (size_t)K * 2 : 0; }
+static size_t partial_bytes(int64_t M, int64_t N, int64_t K) { return num_chunks(K) > 1 ? (size_t)M * (size_t)N * 4 : 0; }
+
 template <int FMT, bool BF16, bool DECODED>
 static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, const uint8_t *codes, const uint8_t *scales, const float *ts,
-                           float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, cudaStream_t st)
+                           float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, int kb0, int nkb, const float *addend,
+                           cudaStream_t st)
 {
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -460,29 +492,44 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, cons
     const char *inj = getenv("RAZER_FAULT_INJECT_STALL");
     const int inject = (inj && inj[0] == '1') ? 1 : 0;
     gemm_kernel<FMT, BF16, DECODED><<<grid, kThreads, SMEM_BYTES, st>>>(map, wmap, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt,
-                                                                      inject);
+                                                                      kb0, nkb, addend, inject);
     return last_launch_status();
 }
 
 template <int FMT, bool BF16>
 static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, bool decoded, const uint8_t *codes, const uint8_t *scales,
-                               const float *ts, float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, void *wdec, cudaStream_t st)
+                               const float *ts, float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, void *wdec,
+                               float *partial, cudaStream_t st)
 {
-    if (!decoded) return launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, Y, out_dt, st);
-    const int64_t nblk = (int64_t)N * K / 16;
-    const int64_t g = std::min<int64_t>((nblk + 255) / 256, (int64_t)sm_count() * 8);
-    if (launch_pdl(decode_weights_kernel<FMT, BF16>, (unsigned)g, 256u, 0, st, codes, scales, nblk, reinterpret_cast<uint4 *>(wdec)) !=
-        cudaSuccess)
-        return RAZER_ERR_CUDA;
-    return launch<FMT, BF16, true>(map, wmap, codes, scales, ts, unbias, M, N, K, Y, out_dt, st);
+    if (decoded) {
+        const int64_t nblk = (int64_t)N * K / 16;
+        const int64_t g = std::min<int64_t>((nblk + 255) / 256, (int64_t)sm_count() * 8);
+        if (launch_pdl(decode_weights_kernel<FMT, BF16>, (unsigned)g, 256u, 0, st, codes, scales, nblk, reinterpret_cast<uint4 *>(wdec)) !=
+            cudaSuccess)
+            return RAZER_ERR_CUDA;
+    }
+    const int KB = K / BK;
+    const int nc = (int)num_chunks(K);
+    for (int c = 0; c < nc; c++) {
+        const int kb0 = (int)((int64_t)c * KB / nc), kb1 = (int)((int64_t)(c + 1) * KB / nc);
+        const bool last = c == nc - 1;
+        void *out = last ? Y : partial;
+        const razer_dtype odt = last ? out_dt : RAZER_F32;
+        const float *add = c > 0 ? partial : nullptr;
+        const razer_status r = decoded ? launch<FMT, BF16, true>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, kb0, kb1 - kb0, add, st)
+                                       : launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, kb0, kb1 - kb0, add, st);
+        if (r != RAZER_OK) return r;
+    }
+    return RAZER_OK;
 }
 
 }  // namespace gemm
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
-    // the decoded weight copy, when the decode-once path applies
-    return M >= gemm::kDecodedMinM ? (size_t)N * (size_t)K * 2 : 0;
+    // the decoded weight copy when the decode-once path applies, then the
+    // fp32 partial sums when K spans several accumulation chains
+    return gemm::decoded_bytes(M, N, K) + gemm::partial_bytes(M, N, K);
 }
 
 razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
@@ -507,7 +554,8 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
         return RAZER_ERR_CUDA;
     // the decoded q*s carries 2^-8 (E3M3) / 2^-4 (E4M3); undone in the epilogue
     const float unbias = wfmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f;
-    const bool decoded = M >= kDecodedMinM && workspace != nullptr;
+    const bool decoded = decoded_bytes(M, N, K) > 0;
+    float *partial = partial_bytes(M, N, K) ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + decoded_bytes(M, N, K)) : nullptr;
     CUtensorMap wmap = map;  // unused by the fused kernel
     if (decoded) {
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
@@ -521,13 +569,13 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
     }
     const int m = (int)M, n = (int)N, k = (int)K;
     if (wfmt == RAZER_FMT_WEIGHT)
-        return bf ? launch_fmt<RAZER_FMT_WEIGHT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st)
-                  : launch_fmt<RAZER_FMT_WEIGHT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st);
+        return bf ? launch_fmt<RAZER_FMT_WEIGHT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st)
+                  : launch_fmt<RAZER_FMT_WEIGHT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st);
     if (wfmt == RAZER_FMT_ACT)
-        return bf ? launch_fmt<RAZER_FMT_ACT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st)
-                  : launch_fmt<RAZER_FMT_ACT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st);
-    return bf ? launch_fmt<RAZER_FMT_NVFP4, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st)
-              : launch_fmt<RAZER_FMT_NVFP4, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, st);
+        return bf ? launch_fmt<RAZER_FMT_ACT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st)
+                  : launch_fmt<RAZER_FMT_ACT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st);
+    return bf ? launch_fmt<RAZER_FMT_NVFP4, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st)
+              : launch_fmt<RAZER_FMT_NVFP4, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st);
 }
 
 }  // namespace razer

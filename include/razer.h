@@ -152,7 +152,18 @@ razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint
  *   X   [M, K] activations, act_dt = RAZER_BF16 or RAZER_F16; the decoded
  *       weights use the same 16-bit type (q*s is exact in both).
  *   Y   [M, N] output, out_dt = RAZER_BF16, RAZER_F16 or RAZER_F32
- *   workspace  as for razer_gemv (size from razer_workspace_size(RAZER_OP_GEMM, M, N, K))
+ *   workspace  device scratch of razer_workspace_size(RAZER_OP_GEMM, M, N, K)
+ *              bytes (16-byte aligned; contents on entry ignored).  For
+ *              M >= 1024 that is N * K * 2 bytes: the packed weights are
+ *              decoded once into a 16-bit copy (exact q*s, the same type as
+ *              X) and the tensor-core pipeline loads both operands by TMA.
+ *              For smaller M it is 0 and the weights are decoded per CTA tile
+ *              into shared memory (each weight once per 256 rows of X).
+ *              When K > 16384 a further M * N * 4 bytes follow: K is then
+ *              split into equal chunks of at most 16384, each accumulated
+ *              in tensor memory on its own, and the scaled partial sums are
+ *              added in fp32 there (one accumulator chain over a longer K
+ *              loses precision).
  * K must be a multiple of 64 and N a multiple of 16.
  */
 razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes,

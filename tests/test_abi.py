@@ -96,3 +96,10 @@ def test_workspace_size_host_logic(lib):
         assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, B, N, K) == max(tma, split_k(B, N, K))
     # other K: split-K partials of the per-warp kernel only
     assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, 4, 4096, 4224) == split_k(4, 4096, 4224)
+    # GEMM: the decoded 16-bit weight copy for M >= 1024, plus fp32 partial
+    # sums of [M, N] when K is longer than one 16384-long accumulation chain
+    G = razer.RAZER_OP_GEMM
+    assert razer.razer_workspace_size(G, 1023, 4096, 16384) == 0
+    assert razer.razer_workspace_size(G, 1024, 4096, 16384) == 4096 * 16384 * 2
+    assert razer.razer_workspace_size(G, 512, 8192, 16448) == 512 * 8192 * 4
+    assert razer.razer_workspace_size(G, 2048, 8192, 28672) == 8192 * 28672 * 2 + 2048 * 8192 * 4

@@ -107,3 +107,36 @@ def test_gemm_bounded_wait_times_out_and_reports(monkeypatch):
     import oracle
     ref = oracle.gemm_ref(oracle_in(X.cpu()), codes.numpy(), scales.numpy(), 1.0, 0)
     assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
+
+
+@pytest.mark.parametrize("M,N,K,fmt", [(512, 28672, 8192, "weight"), (2048, 8192, 28672, "weight"), (8192, 8192, 8192, "nvfp4"),
+                                       (1024, 4096, 4096, "act")])
+def test_gemm_70b_sweep_sampled(orc, M, N, K, fmt):
+    # the 70B projection shapes of the sweep (M = 512 runs the fused decode,
+    # M >= 1024 the decode-once path); 32 sampled output rows against the oracle
+    codes, scales = workloads.random_packed(N, K, fmt, seed=M + N + K, max_scale_code=40)
+    X = workloads.vectors(M, K, seed=79, dtype=torch.bfloat16)
+    ts = 0.0031
+    Y = gemm(X, codes, scales, ts, fmt).cpu().numpy()
+    sel = np.sort(np.random.default_rng(3).choice(M, 32, replace=False))
+    ref = orc.gemm_ref(oracle_in(X[sel]), codes.numpy(), scales.numpy(), ts, FMT_ID[fmt])
+    assert rel_err(Y[sel], ref) <= REL_TOL
+
+
+@pytest.mark.parametrize("xdt", [torch.float16, torch.bfloat16])
+def test_gemm_decoded_path_f16_and_garbage_workspace(orc, xdt):
+    # decode-once path (M >= 1024) with both activation types; the workspace
+    # (the decoded weight copy) starts full of garbage and is sized by the API
+    M, N, K = 1100, 528, 320
+    codes, scales = workloads.random_packed(N, K, "weight", seed=81)
+    X = workloads.vectors(M, K, seed=82, dtype=xdt)
+    need = R.razer_workspace_size(R.RAZER_OP_GEMM, M, N, K)
+    assert need == N * K * 2
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)
+    Y = R.razer_gemm(X.to(DEV), codes.to(DEV), scales.to(DEV), torch.tensor([0.05], device=DEV), "weight", torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    assert R.razer_get_device_status() == 0
+    ref = orc.gemm_ref(oracle_in(X), codes.numpy(), scales.numpy(), 0.05, 0)
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
+    # below the threshold no workspace is needed (fused decode)
+    assert R.razer_workspace_size(R.RAZER_OP_GEMM, 1023, N, K) == 0
