@@ -81,6 +81,21 @@ __device__ __forceinline__ unsigned fix_codes(unsigned c1, unsigned c2)
     return w & ~z;
 }
 
+// Nearest scale code of s_f >= 0 (ties to even, saturating) from the hardware
+// E4M3 convert.  E4M3 (bias 7) codes are the activation scale codes; an E3M3
+// (bias 3) value times 2^-4 has the same exponent and mantissa fields in E4M3,
+// subnormals included, so the weight code is the E4M3 code of s_f * 2^-4
+// clamped to the largest E3M3 code (anything above it saturates there).
+template <int FMT> __device__ __forceinline__ unsigned encode_scale_cvt(float sf)
+{
+    using F = Fmt<FMT>;
+    const float v = FMT == RAZER_FMT_WEIGHT ? __fmul_rn(sf, 0.0625f) : sf;
+    unsigned short h;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(v));
+    const unsigned c = (unsigned)h & 0x7Fu;
+    return FMT == RAZER_FMT_WEIGHT ? min(c, (unsigned)F::kMagMask) : c;
+}
+
 struct BlockOut {
     uint2 packed;    // 16 nibbles
     unsigned sbyte;  // scale byte (meta | magnitude code)
@@ -128,7 +143,7 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
     } else {
         sf = __fdiv_rn(amax, k.six_ts);
     }
-    const unsigned sc = encode_scale<FMT>(sf);
+    const unsigned sc = FAST ? encode_scale_cvt<FMT>(sf) : encode_scale<FMT>(sf);
     const float d = k.tab_d[sc];  // dec(sc) * ts
     if (!FAST && (sc == 0u || d == 0.0f)) return o;
 
@@ -172,8 +187,36 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
         // 2^-20.  A = sum t and B = sum copysign(t, xs) are exact binary32 sums
         // (|A|, |B| <= 16); then the +5 sum is (A - B) / 2 and the -5 sum is
         // (A + B) / 2, both exact.
-        float2 AB = make_float2(0.0f, 0.0f);  // (A, B), one packed add per element
+#ifndef RAZER_Q_SAT
+#define RAZER_Q_SAT 1
+#endif
+#ifndef RAZER_Q_SCALAR_AB
+#define RAZER_Q_SCALAR_AB 0
+#endif
         float ea[16];                           // 2|xs| - 10, reused by the final encode
+#if RAZER_Q_SAT
+        // -t = sat(1 - |e|) in one saturating add
+        float Ap = 0.0f, Bp = 0.0f;
+        float2 AB = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+            ea[j] = __fmaf_rn(2.0f, fabsf(xs[j]), -10.0f);
+            const float nt = __saturatef(__fadd_rn(1.0f, -fabsf(ea[j])));
+#if RAZER_Q_SCALAR_AB
+            Ap = __fadd_rn(Ap, nt);
+            Bp = __fadd_rn(Bp, copysignf(nt, xs[j]));
+#else
+            AB = add2(AB, make_float2(nt, copysignf(nt, xs[j])));
+#endif
+        }
+#if !RAZER_Q_SCALAR_AB
+        Ap = AB.x;
+        Bp = AB.y;
+#endif
+        // copysign(-t, xs) = copysign(t, xs) for t <= 0: B is the same sum
+        const float A = -Ap, Bs = Bp;
+#else
+        float2 AB = make_float2(0.0f, 0.0f);  // (A, B), one packed add per element
 #pragma unroll
         for (int j = 0; j < 16; j++) {
             ea[j] = __fmaf_rn(2.0f, fabsf(xs[j]), -10.0f);
@@ -181,6 +224,7 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
             AB = add2(AB, make_float2(t, copysignf(t, xs[j])));
         }
         const float A = AB.x, Bs = AB.y;
+#endif
         const float dp5 = __fmul_rn(__fsub_rn(A, Bs), 0.5f);
         const float dn5 = __fmul_rn(__fadd_rn(A, Bs), 0.5f);
         float best = dp5;
@@ -188,17 +232,22 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
         // final encode against Q_FP4 u {v*}: elements nearest to v* take
         // 0b1000.  For v* = +5 the region is xs in (4.5, 5.5], for v* = -5 it
         // is [-5.5, -4.5) (ties go to the smaller magnitude): |xs| in
-        // (4.5, 5.5] with the sign of v*.  In terms of e = 2|xs| - 10 (exact
-        // there, a multiple of 2^-20) that is e in (-1, 1], i.e. the sign bit of
-        // r = |e - 2^-22| - 1.  The E2M1 convert keeps the sign of r in bit 3 of
-        // each nibble, which gathers the 16 tests with 4 converts; the sign of
-        // xs is the plain code's sign bit (the plain code is +-4 or +-6 there).
+        // (4.5, 5.5] with the sign of v*.  y = |xs|/2 - (1 + 2^-23) is exact
+        // for |xs| in [4, 8) (a multiple of 2^-23 in [1, 2)) and lies in
+        // (1.25, 1.75) -- the open interval the E2M1 convert sends to code
+        // 0b0011 -- exactly when |xs| is in (4.5, 5.5]; smaller |xs| give
+        // y < 1 and larger ones (<= 9) y > 1.75.  Four converts gather the 16
+        // tests; the sign of xs is the plain code's sign bit (the plain code is
+        // +-4 or +-6 there).
         unsigned o0, o1;
         {
-            float r[16];
+            float yv[16];
 #pragma unroll
-            for (int j = 0; j < 16; j++) r[j] = __fadd_rn(fabsf(__fadd_rn(ea[j], -0x1p-22f)), -1.0f);
-            const unsigned in0 = cvt_e2m1x8(r) & 0x88888888u, in1 = cvt_e2m1x8(r + 8) & 0x88888888u;
+            for (int j = 0; j < 16; j++) yv[j] = __fmaf_rn(fabsf(xs[j]), 0.5f, -(1.0f + 0x1p-23f));
+            const unsigned v0 = cvt_e2m1x8(yv) ^ 0x33333333u, v1 = cvt_e2m1x8(yv + 8) ^ 0x33333333u;
+            // bit 3 of every nibble equal to 0b0011
+            const unsigned in0 = ~(((v0 & 0x77777777u) + 0x77777777u) | v0) & 0x88888888u;
+            const unsigned in1 = ~(((v1 & 0x77777777u) + 0x77777777u) | v1) & 0x88888888u;
             o0 = in0 & (meta ? w0 : ~w0);
             o1 = in1 & (meta ? w1 : ~w1);
         }
@@ -259,33 +308,56 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
 constexpr int kQThreads = 256;
 
 template <int FMT, typename TIn, bool FAST, bool HIST>
+__device__ __forceinline__ void quant_one(const uint4 v0, const uint4 v1, int64_t b, const ScaleCtx &k, uint8_t *__restrict__ codes,
+                                          uint8_t *__restrict__ scales, unsigned (&cnt)[4])
+{
+    float xv[16];
+    const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const float2 f = In16<TIn>::to_f2(wv[i]);
+        xv[2 * i] = f.x;
+        xv[2 * i + 1] = f.y;
+    }
+    const BlockOut o = quantize_block<FMT, FAST, std::is_same<TIn, __half>::value>(xv, k);
+    reinterpret_cast<uint2 *>(codes)[b] = o.packed;
+    scales[b] = (uint8_t)o.sbyte;
+    if constexpr (HIST) {
+        const unsigned m1 = o.meta & 1u, e = o.effective ? 1u : 0u;
+        cnt[0] += 1u - m1;
+        cnt[1] += m1;
+        cnt[2] += e & (1u - m1);
+        cnt[3] += e & m1;
+    }
+}
+
+#ifndef RAZER_QPREFETCH
+#define RAZER_QPREFETCH 1
+#endif
+
+// Grid-stride over the 16-element blocks.  The next block's 32 bytes are
+// loaded before the current block is quantized, so every thread keeps one
+// load in flight while it computes.
+template <int FMT, typename TIn, bool FAST, bool HIST>
 __device__ __forceinline__ void quant_loop(const TIn *__restrict__ x, int64_t nblk, const ScaleCtx &k, uint8_t *__restrict__ codes,
                                            uint8_t *__restrict__ scales, unsigned (&cnt)[4])
 {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(x) + 2 * b;
-        const uint4 v0 = ldg_stream(p);
-        const uint4 v1 = ldg_stream(p + 1);
-        float xv[16];
-        const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const float2 f = In16<TIn>::to_f2(wv[i]);
-            xv[2 * i] = f.x;
-            xv[2 * i + 1] = f.y;
-        }
-        const BlockOut o = quantize_block<FMT, FAST, std::is_same<TIn, __half>::value>(xv, k);
-        reinterpret_cast<uint2 *>(codes)[b] = o.packed;
-        scales[b] = (uint8_t)o.sbyte;
-        if constexpr (HIST) {
-            const unsigned m1 = o.meta & 1u, e = o.effective ? 1u : 0u;
-            cnt[0] += 1u - m1;
-            cnt[1] += m1;
-            cnt[2] += e & (1u - m1);
-            cnt[3] += e & m1;
-        }
+    const uint4 *p = reinterpret_cast<const uint4 *>(x);
+    int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+#if RAZER_QPREFETCH
+    if (b >= nblk) return;
+    uint4 v0 = ldg_stream(p + 2 * b), v1 = ldg_stream(p + 2 * b + 1);
+    for (; b < nblk; b += stride) {
+        const int64_t bn = b + stride < nblk ? b + stride : b;
+        const uint4 n0 = ldg_stream(p + 2 * bn), n1 = ldg_stream(p + 2 * bn + 1);
+        quant_one<FMT, TIn, FAST, HIST>(v0, v1, b, k, codes, scales, cnt);
+        v0 = n0;
+        v1 = n1;
     }
+#else
+    for (; b < nblk; b += stride) quant_one<FMT, TIn, FAST, HIST>(ldg_stream(p + 2 * b), ldg_stream(p + 2 * b + 1), b, k, codes, scales, cnt);
+#endif
 }
 
 template <int FMT, typename TIn, bool HIST>
@@ -347,7 +419,23 @@ __global__ void __launch_bounds__(256) amax_kernel(const TIn *__restrict__ x, in
     float m = 0.0f;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const uint4 *p = reinterpret_cast<const uint4 *>(x);
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += stride) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // four independent 16-byte loads in flight per thread
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) v[u] = ldg_stream(p + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const unsigned w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const float2 f = In16<TIn>::to_f2(w[k]);
+                m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+    }
+    for (; i < nvec; i += stride) {
         const uint4 v = ldg_stream(p + i);
         const unsigned w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
