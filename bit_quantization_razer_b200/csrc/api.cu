@@ -22,6 +22,8 @@ razer_status last_launch_status() { return cudaGetLastError() == cudaSuccess ? R
 
 razer_status run_quantize(const void *x, razer_dtype dt, int64_t R, int64_t K, const float *ts_in, uint8_t *codes,
                           uint8_t *scales, float *ts_out, unsigned long long *hist, razer_format fmt, cudaStream_t st);
+razer_status run_quantize_batch(int count, const void *const *W, razer_dtype dt, const int64_t *R, const int64_t *K,
+                                uint8_t *const *codes, uint8_t *const *scales, float *ts, razer_format fmt, cudaStream_t st);
 razer_status run_dequant(const uint8_t *codes, const uint8_t *scales, const float *ts, razer_format fmt, int64_t R, int64_t K,
                          void *out, razer_dtype dt, cudaStream_t st);
 razer_status run_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
@@ -63,6 +65,26 @@ razer_status razer_quantize_weights(const void *W, razer_dtype in_dt, int64_t N,
     if (st != RAZER_OK) return st;
     if (!aligned(W, 16) || !aligned(tensor_scale, 4)) return RAZER_ERR_ALIGN;
     return run_quantize(W, in_dt, N, K, nullptr, codes, scales, tensor_scale, nullptr, fmt, (cudaStream_t)stream);
+}
+
+razer_status razer_quantize_weights_batch(int count, const void *const *W, razer_dtype in_dt, const int64_t *N, const int64_t *K,
+                                          uint8_t *const *codes, uint8_t *const *scales, float *tensor_scales, razer_format fmt,
+                                          razer_stream_t stream)
+{
+    if (count < 0) return RAZER_ERR_INVALID_ARG;
+    if (count == 0) return RAZER_OK;
+    if (!W || !N || !K || !codes || !scales || !tensor_scales) return RAZER_ERR_INVALID_ARG;
+    if (fmt != RAZER_FMT_WEIGHT && fmt != RAZER_FMT_NVFP4) return valid_fmt(fmt) ? RAZER_ERR_UNSUPPORTED : RAZER_ERR_INVALID_ARG;
+    if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(in_dt)) return RAZER_ERR_DTYPE;
+    if (!aligned(tensor_scales, 4)) return RAZER_ERR_ALIGN;
+    for (int i = 0; i < count; i++) {
+        if (!W[i] && N[i] * K[i] > 0) return RAZER_ERR_INVALID_ARG;
+        razer_status st = check_packed(codes[i], scales[i], N[i], K[i]);
+        if (st != RAZER_OK) return st;
+        if (!aligned(W[i], 16)) return RAZER_ERR_ALIGN;
+    }
+    return run_quantize_batch(count, W, in_dt, N, K, codes, scales, tensor_scales, fmt, (cudaStream_t)stream);
 }
 
 razer_status razer_quantize_acts(const void *X, razer_dtype in_dt, int64_t M, int64_t K, const float *ts_in, uint8_t *codes,

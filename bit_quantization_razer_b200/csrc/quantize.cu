@@ -331,33 +331,85 @@ __device__ __forceinline__ void quant_one(const uint4 v0, const uint4 v1, int64_
     }
 }
 
-#ifndef RAZER_QPREFETCH
-#define RAZER_QPREFETCH 1
-#endif
-
-// Grid-stride over the 16-element blocks.  The next block's 32 bytes are
+// Thread t of T quantizes blocks t, t + T, ...  The next block's 32 bytes are
 // loaded before the current block is quantized, so every thread keeps one
 // load in flight while it computes.
 template <int FMT, typename TIn, bool FAST, bool HIST>
-__device__ __forceinline__ void quant_loop(const TIn *__restrict__ x, int64_t nblk, const ScaleCtx &k, uint8_t *__restrict__ codes,
-                                           uint8_t *__restrict__ scales, unsigned (&cnt)[4])
+__device__ __forceinline__ void quant_range(const TIn *__restrict__ x, int64_t nblk, const ScaleCtx &k, uint8_t *__restrict__ codes,
+                                            uint8_t *__restrict__ scales, int64_t t, int64_t T, unsigned (&cnt)[4])
 {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const uint4 *p = reinterpret_cast<const uint4 *>(x);
-    int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-#if RAZER_QPREFETCH
+    int64_t b = t;
     if (b >= nblk) return;
     uint4 v0 = ldg_stream(p + 2 * b), v1 = ldg_stream(p + 2 * b + 1);
-    for (; b < nblk; b += stride) {
-        const int64_t bn = b + stride < nblk ? b + stride : b;
+    for (; b < nblk; b += T) {
+        const int64_t bn = b + T < nblk ? b + T : b;
         const uint4 n0 = ldg_stream(p + 2 * bn), n1 = ldg_stream(p + 2 * bn + 1);
         quant_one<FMT, TIn, FAST, HIST>(v0, v1, b, k, codes, scales, cnt);
         v0 = n0;
         v1 = n1;
     }
-#else
-    for (; b < nblk; b += stride) quant_one<FMT, TIn, FAST, HIST>(ldg_stream(p + 2 * b), ldg_stream(p + 2 * b + 1), b, k, codes, scales, cnt);
-#endif
+}
+
+template <int FMT, typename TIn, bool FAST, bool HIST>
+__device__ __forceinline__ void quant_loop(const TIn *__restrict__ x, int64_t nblk, const ScaleCtx &k, uint8_t *__restrict__ codes,
+                                           uint8_t *__restrict__ scales, unsigned (&cnt)[4])
+{
+    quant_range<FMT, TIn, FAST, HIST>(x, nblk, k, codes, scales, (int64_t)blockIdx.x * blockDim.x + threadIdx.x,
+                                      (int64_t)gridDim.x * blockDim.x, cnt);
+}
+
+// Fills the per-code tables (shared memory) and the launch constants for ts;
+// the caller synchronises the block before using them.
+template <int FMT>
+__device__ __forceinline__ ScaleCtx make_ctx(float ts, float *tab_d, float *tab_y)
+{
+    using F = Fmt<FMT>;
+    for (int c = threadIdx.x; c <= (int)F::kMagMask; c += blockDim.x) {
+        const float d = __fmul_rn(decode_scale<FMT>((unsigned)c), ts);
+        tab_d[c] = d;
+        tab_y[c] = (d >= 0x1p-90f && d <= 0x1p90f) ? __frcp_rn(d) : 0.0f;
+    }
+    ScaleCtx k;
+    k.ts = ts;
+    k.six_ts = __fmul_rn(6.0f, ts);
+    k.y6 = (k.six_ts >= 0x1p-60f && k.six_ts <= 0x1p60f) ? __frcp_rn(k.six_ts) : 0.0f;
+    k.tab_d = tab_d;
+    k.tab_y = tab_y;
+    return k;
+}
+
+// launch-wide: with ts in [2^-62, 2^57] every reciprocal the blocks need is a
+// valid Markstein reciprocal (d of a non-zero scale code lies in
+// [2^-71, 2^66]), so the per-block fallbacks and early exits drop out
+__device__ __forceinline__ bool fast_ts(float ts) { return ts >= 0x1p-62f && ts <= 0x1p57f; }
+
+// max(m, |x|) over the eight 16-bit values of one 16-byte vector
+template <typename TIn> __device__ __forceinline__ float amax_vec(float m, const uint4 v)
+{
+    const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const float2 f = In16<TIn>::to_f2(w[k]);
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+    return m;
+}
+
+// block-wide max of m, merged into *out as binary32 bits (atomicMax is
+// order-preserving for non-negative floats)
+__device__ __forceinline__ void commit_amax(float m, unsigned *out)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __shared__ float sm[32];
+    if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float r = sm[0];
+        for (int i = 1; i < (int)(blockDim.x >> 5); i++) r = fmaxf(r, sm[i]);
+        if (r > 0.0f) atomicMax(out, __float_as_uint(r));
+    }
 }
 
 template <int FMT, typename TIn, bool HIST>
@@ -374,23 +426,10 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const TIn *__restri
     unsigned cnt[4] = {0u, 0u, 0u, 0u};
 
     __shared__ float tab_d[F::kMagMask + 1], tab_y[F::kMagMask + 1];
-    for (int c = threadIdx.x; c <= (int)F::kMagMask; c += blockDim.x) {
-        const float d = __fmul_rn(decode_scale<FMT>((unsigned)c), ts);
-        tab_d[c] = d;
-        tab_y[c] = (d >= 0x1p-90f && d <= 0x1p90f) ? __frcp_rn(d) : 0.0f;
-    }
-    ScaleCtx k;
-    k.ts = ts;
-    k.six_ts = __fmul_rn(6.0f, ts);
-    k.y6 = (k.six_ts >= 0x1p-60f && k.six_ts <= 0x1p60f) ? __frcp_rn(k.six_ts) : 0.0f;
-    k.tab_d = tab_d;
-    k.tab_y = tab_y;
+    const ScaleCtx k = make_ctx<FMT>(ts, tab_d, tab_y);
     __syncthreads();
 
-    // launch-wide: with ts in [2^-62, 2^57] every reciprocal the blocks need
-    // is a valid Markstein reciprocal (d of a non-zero scale code lies in
-    // [2^-71, 2^66]), so the per-block fallbacks and early exits drop out
-    if (ts >= 0x1p-62f && ts <= 0x1p57f) quant_loop<FMT, TIn, true, HIST>(x, nblk, k, codes, scales, cnt);
+    if (fast_ts(ts)) quant_loop<FMT, TIn, true, HIST>(x, nblk, k, codes, scales, cnt);
     else quant_loop<FMT, TIn, false, HIST>(x, nblk, k, codes, scales, cnt);
 
     if constexpr (HIST) {
@@ -426,34 +465,77 @@ __global__ void __launch_bounds__(256) amax_kernel(const TIn *__restrict__ x, in
 #pragma unroll
         for (int u = 0; u < 4; u++) v[u] = ldg_stream(p + i + u * stride);
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const unsigned w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-                const float2 f = In16<TIn>::to_f2(w[k]);
-                m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
-        }
+        for (int u = 0; u < 4; u++) m = amax_vec<TIn>(m, v[u]);
     }
-    for (; i < nvec; i += stride) {
-        const uint4 v = ldg_stream(p + i);
-        const unsigned w[4] = {v.x, v.y, v.z, v.w};
+    for (; i < nvec; i += stride) m = amax_vec<TIn>(m, ldg_stream(p + i));
+    commit_amax(m, out);
+}
+
+// Thread t of T reduces max(m, |x|) over the 16-byte vectors t, t + T, ...
+// with eight loads in flight.
+template <typename TIn>
+__device__ __forceinline__ void amax_range(const TIn *__restrict__ x, int64_t nvec, int64_t t, int64_t T, float &m)
+{
+    const uint4 *p = reinterpret_cast<const uint4 *>(x);
+    int64_t i = t;
+    for (; i + 7 * T < nvec; i += 8 * T) {
+        uint4 v[8];
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
-            const float2 f = In16<TIn>::to_f2(w[k]);
-            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
+        for (int u = 0; u < 8; u++) v[u] = ldg_stream(p + i + u * T);
+#pragma unroll
+        for (int u = 0; u < 8; u++) m = amax_vec<TIn>(m, v[u]);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __shared__ float sm[8];
-    if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = m;
+    for (; i < nvec; i += T) m = amax_vec<TIn>(m, ldg_stream(p + i));
+}
+
+// One stage of the batched weight quantizer: quantizes tensor q, whose amax
+// an earlier kernel in the stream completed, while reducing amax(|x|) of the
+// next tensor a.  Quantization is arithmetic-bound and the amax pass is
+// bandwidth-bound, so each CTA splits its warps: the first amax_warps stream
+// tensor a (eight 16-byte loads in flight per thread, few instructions), the
+// others quantize tensor q with the prefetching loop.  The host picks the
+// split from the two parts' expected times so that both finish together.
+template <int FMT, typename TIn>
+__global__ void __launch_bounds__(kQThreads, 4) quant_amax_kernel(const TIn *__restrict__ xq, int64_t nblk, const float *__restrict__ amax_q,
+                                                                  uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                                                                  const TIn *__restrict__ xa, int64_t nva, unsigned *__restrict__ amax_a,
+                                                                  int amax_warps)
+{
+    using F = Fmt<FMT>;
+    pdl_wait();  // amax_q and the zeroed amax_a come from earlier kernels
+    pdl_trigger();
+    const float ts = __fdiv_rn(*amax_q, F::kC);
+    __shared__ float tab_d[F::kMagMask + 1], tab_y[F::kMagMask + 1];
+    const ScaleCtx k = make_ctx<FMT>(ts, tab_d, tab_y);
     __syncthreads();
-    if (threadIdx.x == 0) {
-        float r = sm[0];
-        for (int i = 1; i < (int)(blockDim.x >> 5); i++) r = fmaxf(r, sm[i]);
-        if (r > 0.0f) atomicMax(out, __float_as_uint(r));
+    float m = 0.0f;
+    const int warp = threadIdx.x >> 5;
+    if (warp < amax_warps) {
+        const int64_t per = 32 * amax_warps;
+        amax_range<TIn>(xa, nva, (int64_t)blockIdx.x * per + threadIdx.x, (int64_t)gridDim.x * per, m);
+    } else {
+        const int64_t per = kQThreads - 32 * amax_warps;
+        const int64_t t = (int64_t)blockIdx.x * per + threadIdx.x - 32 * amax_warps, T = (int64_t)gridDim.x * per;
+        unsigned cnt[4] = {0u, 0u, 0u, 0u};
+        if (fast_ts(ts)) quant_range<FMT, TIn, true, false>(xq, nblk, k, codes, scales, t, T, cnt);
+        else quant_range<FMT, TIn, false, false>(xq, nblk, k, codes, scales, t, T, cnt);
     }
+    commit_amax(m, amax_a);
+}
+
+// zeroes count amax words (one launch for a whole batch)
+__global__ void init_many_kernel(unsigned *bits, int count)
+{
+    pdl_wait();
+    pdl_trigger();
+    for (int i = threadIdx.x; i < count; i += blockDim.x) bits[i] = 0u;
+}
+
+// ts[i] = amax[i] / (6 * S_max) for a whole batch, written over the amax words
+__global__ void finalize_many_kernel(float *ts, int count, float c)
+{
+    pdl_wait();
+    for (int i = threadIdx.x; i < count; i += blockDim.x) ts[i] = __fdiv_rn(__uint_as_float(reinterpret_cast<unsigned *>(ts)[i]), c);
 }
 
 // ts = amax / (6 * S_max), written over the amax word.
@@ -483,6 +565,18 @@ __global__ void quant_init_kernel(unsigned long long *hist, unsigned *amax_bits)
 // ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
+// CTAs of kQThreads threads of kernel f resident per SM (cached per kernel)
+template <typename Kern> static int resident_ctas(Kern f)
+{
+    static int cached = 0;
+    if (!cached) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, f, kQThreads, 0) != cudaSuccess || n <= 0) n = 4;
+        cached = n;
+    }
+    return cached;
+}
+
 static int quant_grid(int64_t work, int threads, int per_sm)
 {
     int64_t g = (work + threads - 1) / threads;
@@ -555,6 +649,71 @@ razer_status run_quantize(const void *x, razer_dtype dt, int64_t R, int64_t K, c
         if (launch_pdl(copy_ts_kernel, 1u, 1u, 0, st, ts_in, ts_out) != cudaSuccess) return RAZER_ERR_CUDA;
     }
     return last_launch_status();
+}
+
+// Warps (of the 8 in a CTA) that stream the amax of the next tensor in a
+// batch stage: proportional to that part's expected share of the stage time,
+// at rates measured on this GPU (the amax warps ~8 TB/s of 16-byte vectors,
+// tuned so that the stage time is lowest; the quantizer ~92 G blocks/s).
+#ifndef RAZER_QSTAGE_AMAX_RATE
+#define RAZER_QSTAGE_AMAX_RATE 5.0e11  // 16-byte vectors per second
+#endif
+#ifndef RAZER_QSTAGE_QUANT_RATE
+#define RAZER_QSTAGE_QUANT_RATE 9.2e10  // 16-element blocks per second
+#endif
+static int stage_amax_warps(int64_t nblk, int64_t nva)
+{
+    if (nva == 0) return 0;
+    if (nblk == 0) return kQThreads / 32;
+    const double ta = (double)nva / RAZER_QSTAGE_AMAX_RATE, tq = (double)nblk / RAZER_QSTAGE_QUANT_RATE;
+    int aw = (int)(8.0 * ta / (ta + tq) + 0.5);
+    return aw < 1 ? 1 : (aw > 6 ? 6 : aw);
+}
+
+// Batched weight quantizer: tensors 0..count-1 with their amax words in
+// ts[0..count).  Stage 0 reduces amax of tensor 0; stage i (1 <= i < count)
+// quantizes tensor i-1 and reduces amax of tensor i in one kernel; the last
+// stage quantizes tensor count-1.  Each tensor's codes, scales and ts are
+// those of a separate run_quantize call.
+template <int FMT, typename TIn>
+static razer_status run_batch_t(int count, const void *const *W, const int64_t *R, const int64_t *K, uint8_t *const *codes,
+                                uint8_t *const *scales, float *ts, cudaStream_t st)
+{
+    const float C = Fmt<FMT>::kC;
+    unsigned *bits = reinterpret_cast<unsigned *>(ts);
+    if (launch_pdl(init_many_kernel, 1u, 256u, 0, st, bits, count) != cudaSuccess) return RAZER_ERR_CUDA;
+    if (R[0] * K[0] > 0) launch_amax<TIn>(W[0], R[0] * K[0], bits, st);
+    for (int i = 1; i < count; i++) {
+        const int64_t nblk = R[i - 1] * K[i - 1] / 16, nva = R[i] * K[i] / 8;
+        if (nblk + nva == 0) continue;
+        const int aw = stage_amax_warps(nblk, nva);
+        // one CTA per resident slot, fewer when a thread would otherwise get no work
+        const int qw = kQThreads / 32 - aw;
+        const int64_t need_q = qw ? (nblk + 32 * qw - 1) / (32 * qw) : 0, need_a = aw ? (nva + 32 * aw - 1) / (32 * aw) : 0;
+        const int64_t cap = (int64_t)sm_count() * resident_ctas(quant_amax_kernel<FMT, TIn>);
+        const int64_t need = need_q > need_a ? need_q : need_a;
+        const unsigned grid = (unsigned)(need < 1 ? 1 : (need > cap ? cap : need));
+        if (launch_pdl(quant_amax_kernel<FMT, TIn>, grid, (unsigned)kQThreads, 0, st, reinterpret_cast<const TIn *>(W[i - 1]), nblk,
+                       const_cast<const float *>(ts + i - 1), codes[i - 1], scales[i - 1], reinterpret_cast<const TIn *>(W[i]), nva,
+                       bits + i, aw) != cudaSuccess)
+            return RAZER_ERR_CUDA;
+    }
+    const int l = count - 1;
+    if (R[l] * K[l] > 0) launch_quant<FMT, TIn>(W[l], R[l] * K[l] / 16, ts + l, 1, codes[l], scales[l], nullptr, st);
+    if (launch_pdl(finalize_many_kernel, 1u, 256u, 0, st, ts, count, C) != cudaSuccess) return RAZER_ERR_CUDA;
+    return last_launch_status();
+}
+
+razer_status run_quantize_batch(int count, const void *const *W, razer_dtype dt, const int64_t *R, const int64_t *K,
+                                uint8_t *const *codes, uint8_t *const *scales, float *ts, razer_format fmt, cudaStream_t st)
+{
+    if (count == 0) return RAZER_OK;
+    const bool h = dt == RAZER_F16;
+    if (fmt == RAZER_FMT_WEIGHT)
+        return h ? run_batch_t<RAZER_FMT_WEIGHT, __half>(count, W, R, K, codes, scales, ts, st)
+                 : run_batch_t<RAZER_FMT_WEIGHT, __nv_bfloat16>(count, W, R, K, codes, scales, ts, st);
+    return h ? run_batch_t<RAZER_FMT_NVFP4, __half>(count, W, R, K, codes, scales, ts, st)
+             : run_batch_t<RAZER_FMT_NVFP4, __nv_bfloat16>(count, W, R, K, codes, scales, ts, st);
 }
 
 }  // namespace razer

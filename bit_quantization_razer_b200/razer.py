@@ -29,7 +29,7 @@ FORMATS = {"weight": RAZER_FMT_WEIGHT, "act": RAZER_FMT_ACT, "nvfp4": RAZER_FMT_
 _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZER_F32}
 
 EXPORTED = (
-    "razer_quantize_weights", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
     "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
 )
@@ -54,6 +54,8 @@ def load() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     L.razer_quantize_weights.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp]
+    L.razer_quantize_weights_batch.argtypes = [i32, ctypes.POINTER(vp), i32, ctypes.POINTER(i64), ctypes.POINTER(i64),
+                                               ctypes.POINTER(vp), ctypes.POINTER(vp), vp, i32, vp]
     L.razer_quantize_acts.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, vp, i32, vp]
     L.razer_dequant.argtypes = [vp, vp, vp, i32, i64, i64, vp, i32, vp]
     L.razer_gemv.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
@@ -68,7 +70,7 @@ def load() -> ctypes.CDLL:
     L.razer_status_string.argtypes = [i32]
     L.razer_status_string.restype = ctypes.c_char_p
     L.razer_version.argtypes = []
-    for fn in ("razer_quantize_weights", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    for fn in ("razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -104,6 +106,26 @@ def razer_quantize_weights(W: torch.Tensor, fmt="weight", *, codes=None, scales=
     st = load().razer_quantize_weights(_p(W), _DT.get(W.dtype, -1), N, K, _p(codes), _p(scales), _p(ts), _fmt(fmt), _stream(stream))
     _check("razer_quantize_weights", st)
     return codes, scales, ts
+
+
+def razer_quantize_weights_batch(Ws, fmt="weight", *, codes=None, scales=None, ts=None, stream=None):
+    """Quantize several weight matrices (same dtype and device) in one call.
+    Returns (list of codes, list of scales, ts [count] f32); matrix i's
+    results equal razer_quantize_weights(Ws[i])."""
+    n = len(Ws)
+    dev = Ws[0].device if n else torch.device("cuda")
+    dt = _DT.get(Ws[0].dtype, -1) if n else 0
+    codes = [torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=dev) for w in Ws] if codes is None else codes
+    scales = [torch.empty((w.shape[0], w.shape[1] // 16), dtype=torch.uint8, device=dev) for w in Ws] if scales is None else scales
+    ts = torch.empty(max(n, 1), dtype=torch.float32, device=dev) if ts is None else ts
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    arr = lambda ts_: (vp * max(n, 1))(*[t.data_ptr() for t in ts_])
+    Ns = (i64 * max(n, 1))(*[w.shape[0] for w in Ws])
+    Ks = (i64 * max(n, 1))(*[w.shape[1] for w in Ws])
+    st = load().razer_quantize_weights_batch(n, arr(Ws), dt, Ns, Ks, arr(codes), arr(scales), _p(ts), _fmt(fmt),
+                                             _stream(stream))
+    _check("razer_quantize_weights_batch", st)
+    return codes, scales, ts[:n]
 
 
 def razer_quantize_acts(X: torch.Tensor, ts_in: torch.Tensor | None = None, fmt="act", *, hist: bool = True,

@@ -95,6 +95,30 @@ razer_status razer_quantize_weights(const void *W, razer_dtype in_dt, int64_t N,
                                     razer_format fmt, razer_stream_t stream);
 
 /*
+ * razer_quantize_weights_batch -- razer_quantize_weights on count matrices in
+ * one call; matrix i gets exactly the codes, scales and ts a separate
+ * razer_quantize_weights call would give it.  The amax pass of matrix i + 1
+ * (bandwidth-bound) runs in the same kernel as the quantization of matrix i
+ * (arithmetic-bound), so a batch streams closer to the HBM rate than the
+ * separate calls.
+ *   count          number of matrices (0: nothing is done)
+ *   W, N, K        HOST arrays of count entries: device pointer of matrix i
+ *                  ([N[i], K[i]], in_dt = RAZER_F16 or RAZER_BF16) and sizes
+ *   codes, scales  HOST arrays of count device pointers ([N[i], K[i]/2] and
+ *                  [N[i], K[i]/16] outputs)
+ *   tensor_scales  DEVICE array of count floats, output: ts of each matrix
+ *                  (also the amax scratch during the call)
+ *   fmt            RAZER_FMT_WEIGHT or RAZER_FMT_NVFP4 (one format for all)
+ * The host arrays are read before the call returns.  Each matrix is checked
+ * like razer_quantize_weights' arguments; the first failure is returned and
+ * nothing is launched.
+ */
+razer_status razer_quantize_weights_batch(int count, const void *const *W, razer_dtype in_dt,
+                                          const int64_t *N, const int64_t *K, uint8_t *const *codes,
+                                          uint8_t *const *scales, float *tensor_scales,
+                                          razer_format fmt, razer_stream_t stream);
+
+/*
  * razer_quantize_acts -- online activation quantizer (关键设计 1-2; the
  * "double quantization" of 训练策略 / gist.science 2.2: each block is
  * quantized once per candidate in V_a = {+5, -5} and the smaller error wins).

@@ -55,6 +55,16 @@ def test_quantize_validation(lib):
     assert q(FAKE, 0, -1, 32, FAKE, FAKE, FAKE, 0, None) == 2
     assert q(ODD, 0, 4, 32, FAKE, FAKE, FAKE, 0, None) == 3
     assert q(FAKE, 0, 4, 32, ODD, FAKE, FAKE, 0, None) == 3
+    b = lib.razer_quantize_weights_batch
+    arr = lambda *v: (ctypes.c_void_p * len(v))(*v)
+    i64s = lambda *v: (ctypes.c_int64 * len(v))(*v)
+    assert b(0, None, 0, None, None, None, None, None, 0, None) == 0                     # empty batch
+    assert b(-1, None, 0, None, None, None, None, None, 0, None) == 1
+    assert b(2, arr(FAKE, FAKE), 0, i64s(4, 4), i64s(32, 32), arr(FAKE, FAKE), arr(FAKE, FAKE), None, 0, None) == 1
+    assert b(2, arr(FAKE, FAKE), 0, i64s(4, 4), i64s(32, 24), arr(FAKE, FAKE), arr(FAKE, FAKE), FAKE, 0, None) == 2
+    assert b(2, arr(FAKE, ODD), 0, i64s(4, 4), i64s(32, 32), arr(FAKE, FAKE), arr(FAKE, FAKE), FAKE, 0, None) == 3
+    assert b(2, arr(FAKE, FAKE), 0, i64s(4, 4), i64s(32, 32), arr(FAKE, FAKE), arr(FAKE, FAKE), FAKE, 1, None) == 6
+    assert b(1, arr(FAKE), 2, i64s(4), i64s(32), arr(FAKE), arr(FAKE), FAKE, 0, None) == 4
     a = lib.razer_quantize_acts
     assert a(FAKE, 1, 4, 32, None, FAKE, FAKE, None, None, 1, None) == 1
     assert a(FAKE, 1, 4, 32, None, FAKE, FAKE, FAKE, None, 0, None) == 6

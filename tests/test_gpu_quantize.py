@@ -83,6 +83,55 @@ def test_quantize_weights_subnormal_scales(orc):
     assert ((s >> 6) >= 2).any()
 
 
+def _subnormal_rows():
+    g = torch.Generator().manual_seed(11)
+    w = (torch.rand(48, 256, generator=g) * 2 - 1) * 0.3
+    w[:, ::64] = 180.0
+    w[::2, 1::64] = -180.0
+    return w
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("fmt", ["weight", "nvfp4"])
+def test_quantize_weights_batch_vs_oracle(orc, dtype, fmt):
+    # ragged row counts, an empty matrix inside the batch, a matrix whose
+    # blocks use subnormal scale codes (+-8 in play) and one larger than the
+    # next, so every stage mixes quantization and amax work of unequal size
+    Ws = [workloads.weight(256, 512, std=0.02, seed=21, dtype=dtype),
+          workloads.weight(100, 256, std=0.5, seed=22, dtype=dtype),
+          torch.empty(0, 64, dtype=dtype),
+          _subnormal_rows().to(dtype),
+          workloads.weight(7, 2048, std=3.0, seed=23, dtype=dtype)]
+    codes, scales, ts = R.razer_quantize_weights_batch([w.to(DEV) for w in Ws], fmt)
+    torch.cuda.synchronize()
+    ts = ts.cpu().numpy()
+    for i, w in enumerate(Ws):
+        oc, os_, ots, _ = orc.quantize(oracle_in(w), FMT_ID[fmt])
+        assert ts[i] == np.float32(ots), i
+        np.testing.assert_array_equal(codes[i].cpu().numpy(), oc.reshape(codes[i].shape))
+        np.testing.assert_array_equal(scales[i].cpu().numpy(), os_.reshape(scales[i].shape))
+
+
+def test_quantize_weights_batch_llama8b_equals_single_calls(orc):
+    # the decode-step projections in one batch: every byte equals the
+    # separate calls' output, ts equals the oracle's, sampled rows the oracle's
+    shapes = [(4096, 4096), (14336, 4096), (4096, 14336)]
+    Ws = [workloads.weight(N, K, std=0.02, seed=300 + i).to(DEV) for i, (N, K) in enumerate(shapes)]
+    codes, scales, ts = R.razer_quantize_weights_batch(Ws, "weight")
+    for i, w in enumerate(Ws):
+        c1, s1, t1 = R.razer_quantize_weights(w, "weight")
+        torch.cuda.synchronize()
+        assert torch.equal(codes[i], c1) and torch.equal(scales[i], s1)
+        assert float(ts[i]) == float(t1[0])
+        wc = w.cpu()
+        ots = orc.tensor_scale(wc.numpy(), 0)
+        assert float(ts[i]) == ots
+        rows = np.random.default_rng(i).choice(w.shape[0], 16, replace=False)
+        oc, os_, _, _ = orc.quantize(wc[rows].numpy(), 0, ts=ots)
+        np.testing.assert_array_equal(codes[i].cpu().numpy()[rows], oc)
+        np.testing.assert_array_equal(scales[i].cpu().numpy()[rows], os_)
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 def test_quantize_acts_dynamic(orc, dtype):
     x = workloads.outlier_activations(256, 4096, seed=300, dtype=dtype)
