@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 METRIC = "RaZeR W4A16 GEMV HBM GB/s & GEMM TFLOP/s vs B200 roofline; quantize GB/s"
 SHAPES = [(4096, 4096), (14336, 4096), (4096, 14336)]  # (N, K) of the Llama-3-8B projections
 BATCHES = [1, 4, 16]
-WORKLOAD = "llama3-8b-decode-w4a16: quantize 3 projections + GEMV B=1,4,16 (fp16)"
+WORKLOAD = "llama3-8b-decode-w4a16: quantize 3 projections (one batched call) + GEMV B=1,4,16 (fp16)"
 
 
 def quant_bytes(N, K):
@@ -71,7 +71,7 @@ def load_peaks():
 
 
 TRAFFIC_SOURCES = {  # the files each timed call's kernels are built from
-    "quantize_kernel": ["quantize.cu", "razer_internal.cuh"],
+    "quantize_batch": ["quantize.cu", "razer_internal.cuh"],
     "gemv_kernel": ["gemv_tma.cu", "gemv.cu", "sm100_async.cuh", "razer_internal.cuh"],
 }
 
@@ -94,6 +94,21 @@ def traffic_for(kernel: str):
     if not e or e.get("source_hash") != source_hash(TRAFFIC_SOURCES[kernel]):
         return None
     return e.get("bytes_per_call")
+
+
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured CUDA graph (every one is a launch of this
+    library's kernels in the bench step), or None if the graph cannot be read."""
+    try:
+        from cuda.bindings import runtime as rt
+
+        h = g.raw_cuda_graph()
+        err, _, n = rt.cudaGraphGetNodes(h, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(h, n)
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes[:n]]
+        return sum(1 for t in kinds if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return None
 
 
 class ClockSampler:
@@ -235,9 +250,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the breakdown / e2e / GEMM legs")
     ap.add_argument("--no-soak", action="store_true", help="skip the 1.5 s pre-timing load for the clock sampler")
-    ap.add_argument("--kernel", choices=["quantize", "act_quantize", "dequant", "gemv", "gemm"],
+    ap.add_argument("--kernel", choices=["quantize", "quantize_batch", "act_quantize", "dequant", "gemv", "gemm"],
                     help="profiling mode: run one call on --shape in a loop (for ncu)")
-    ap.add_argument("--shape", default="4096,4096", help="N,K (gemm: M,N,K)")
+    ap.add_argument("--shape", default="4096,4096", help="N,K (gemm: M,N,K; quantize_batch: N1,K1,N2,K2,...)")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()
@@ -276,19 +291,19 @@ def main():
     # inputs (host-generated, seeded), resident in HBM before timing
     W = [workloads.weight(N, K, seed=100 + i).to(dev) for i, (N, K) in enumerate(SHAPES)]
     X = {B: [workloads.vectors(B, K, seed=10 + B).to(dev) for _, K in SHAPES] for B in BATCHES}
-    packed = [[(torch.empty((N, K // 2), dtype=torch.uint8, device=dev), torch.empty((N, K // 16), dtype=torch.uint8, device=dev),
-                torch.empty(1, dtype=torch.float32, device=dev)) for N, K in SHAPES] for _ in range(2)]
+    # two packed sets (codes, scales, ts [3]) alternate between steps
+    packed = [([torch.empty((N, K // 2), dtype=torch.uint8, device=dev) for N, K in SHAPES],
+               [torch.empty((N, K // 16), dtype=torch.uint8, device=dev) for N, K in SHAPES],
+               torch.empty(len(SHAPES), dtype=torch.float32, device=dev)) for _ in range(2)]
     Y = {B: [torch.empty((B, N), dtype=torch.float16, device=dev) for N, _ in SHAPES] for B in BATCHES}
     wsz = max(R.razer_workspace_size(R.RAZER_OP_GEMV, B, N, K) for N, K in SHAPES for B in BATCHES)
     ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
 
     def step(s):
         cur, prev = packed[s % 2], packed[(s + 1) % 2]
+        R.razer_quantize_weights_batch(W, "weight", codes=cur[0], scales=cur[1], ts=cur[2])
         for i in range(len(SHAPES)):
-            c, sc, t = cur[i]
-            R.razer_quantize_weights(W[i], "weight", codes=c, scales=sc, ts=t)
-        for i in range(len(SHAPES)):
-            c, sc, t = prev[i]
+            c, sc, t = prev[0][i], prev[1][i], prev[2][i:i + 1]
             for B in BATCHES:
                 R.razer_gemv(X[B][i], c, sc, t, "weight", torch.float16, out=Y[B][i], workspace=ws)
 
@@ -301,10 +316,13 @@ def main():
     # host overhead; the work inside is unchanged)
     graphs = []
     for par in range(2):
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(g):
             step(par)
         graphs.append(g)
+    for g in graphs:
+        g.instantiate()
+    kernels_per_step = graph_kernel_nodes(graphs[0])
     for s in range(3):
         graphs[s % 2].replay()
     torch.cuda.synchronize()
@@ -346,7 +364,7 @@ def main():
     for i, (N, K) in enumerate(SHAPES):
         ncopy = max(2, -(-2 * l2 // (N * K * 2)))
         Wc = [W[i]] + [W[i].clone() for _ in range(ncopy - 1)]
-        outs = [(torch.empty_like(packed[0][i][0]), torch.empty_like(packed[0][i][1]), torch.empty_like(packed[0][i][2]))
+        outs = [(torch.empty_like(packed[0][0][i]), torch.empty_like(packed[0][1][i]), torch.empty(1, dtype=torch.float32, device=dev))
                 for _ in range(ncopy)]
         for r in range(ncopy):
             R.razer_quantize_weights(Wc[r], "weight", codes=outs[r][0], scales=outs[r][1], ts=outs[r][2])
@@ -354,10 +372,6 @@ def main():
                                  for r in range(ncopy)], ncopy, stream)
         nb = quant_bytes(N, K)
         breakdown[f"quantize_{N}x{K}"] = {"ms": ms, "GB/s": nb / ms / 1e6}
-        by_kind.setdefault("quantize", [0.0, 0.0, 0])
-        by_kind["quantize"][0] += ms
-        by_kind["quantize"][1] += nb
-        by_kind["quantize"][2] += 1
         del Wc
         npk = max(2, -(-2 * l2 // (N * K * 9 // 16)))
         pk = [outs[r % len(outs)] for r in range(npk)]
@@ -372,14 +386,26 @@ def main():
             by_kind["gemv"][1] += nb
             by_kind["gemv"][2] += 1
         del pk, outs
+    # the step's quantize call: all three projections in one batched call,
+    # two weight sets alternating (536 MB of fp16 input, > 2x L2)
+    Wsets = [W, [w.clone() for w in W]]
+    qouts = [([torch.empty_like(c) for c in packed[0][0]], [torch.empty_like(c) for c in packed[0][1]], torch.empty_like(packed[0][2]))
+             for _ in range(2)]
+    ms = time_graph(lambda: [R.razer_quantize_weights_batch(Wsets[r], "weight", codes=qouts[r][0], scales=qouts[r][1], ts=qouts[r][2])
+                             for r in range(2)], 2, stream)
+    nb = sum(quant_bytes(N, K) for N, K in SHAPES)
+    breakdown["quantize_batch_3proj"] = {"ms": ms, "GB/s": nb / ms / 1e6}
+    by_kind["quantize"] = [ms, nb, 1]
+    del Wsets, qouts
     torch.cuda.empty_cache()
     dominant = max(by_kind, key=lambda k: by_kind[k][0])
     dom_ms, dom_bytes, n_calls = by_kind[dominant]
     achieved = dom_bytes / dom_ms / 1e6  # GB/s over that kind's calls
-    kname = "quantize_kernel" if dominant == "quantize" else "gemv_kernel"
+    kname = "quantize_batch" if dominant == "quantize" else "gemv_kernel"
     traffic = traffic_for(kname)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": traffic, "kernel": ("razer_quantize_weights (amax + quantize kernels)" if dominant == "quantize"
+                "traffic": traffic, "kernel": ("razer_quantize_weights_batch of the 3 projections (amax, fused quantize + "
+                                               "next-amax, quantize kernels)" if dominant == "quantize"
                                                else "razer_gemv (gemv + split-K reduce kernels)"),
                 "algorithmic_bytes_per_call": dom_bytes / n_calls, "peak_source": peak_src,
                 "timing": "CUDA events around CUDA-graph replays of back-to-back calls on operand copies larger than L2"}
@@ -393,7 +419,9 @@ def main():
     if not args.no_extras:
         e2e = run_e2e(R, workloads, dev, stream, args, world, pg)
 
-    launches_per_step = len(SHAPES) * 3 + len(SHAPES) * len(BATCHES) * 2
+    # kernel nodes of the captured step graph: init + amax + 2 fused stages +
+    # quantize + finalize for the batch, main + reduction kernel per GEMV
+    launches_per_step = kernels_per_step if kernels_per_step is not None else 6 + len(SHAPES) * len(BATCHES) * 2
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -445,6 +473,12 @@ def run_single_kernel(args):
                 R.razer_dequant(c, s, t, "weight", torch.float16, out=out)
             else:
                 R.razer_gemv(x, c, s, t, "weight", torch.float16, out=y, workspace=ws)
+    elif args.kernel == "quantize_batch":
+        Ws = [workloads.weight(dims[2 * i], dims[2 * i + 1], seed=1 + i).to(dev) for i in range(len(dims) // 2)]
+        cs, ss, ts = R.razer_quantize_weights_batch(Ws)
+
+        def call():
+            R.razer_quantize_weights_batch(Ws, codes=cs, scales=ss, ts=ts)
     elif args.kernel == "act_quantize":
         M, K = dims
         xa = workloads.outlier_activations(M, K, seed=3).to(dev)
@@ -479,15 +513,19 @@ def run_single_kernel(args):
 
 
 def time_graph(fn, ncalls, stream, reps=5):
-    """Median device time of one call: fn() issues `ncalls` calls; they are
-    captured into one CUDA graph, replayed `reps` times between events."""
+    """Median device time of one call in a back-to-back sequence: fn() issues
+    `ncalls` calls; fn() is captured enough times for at least 8 calls per
+    CUDA graph (so the graph launch itself is amortised), and the graph is
+    replayed `reps` times between events."""
     import torch
 
+    inner = max(1, -(-8 // ncalls))
     fn()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        fn()
+        for _ in range(inner):
+            fn()
     g.replay()
     torch.cuda.synchronize()
     times = []
@@ -497,7 +535,7 @@ def time_graph(fn, ncalls, stream, reps=5):
         g.replay()
         e1.record(stream)
         torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1) / ncalls)
+        times.append(e0.elapsed_time(e1) / (ncalls * inner))
     del g
     return statistics.median(times)
 
@@ -562,14 +600,13 @@ def run_e2e(R, workloads, dev, stream, args, world, pg):
     d2h = sum(y.numel() * 2 for B in BATCHES for y in Yh[B])
 
     def step():
-        packed = []
         for i in range(len(SHAPES)):
             Wd[i].copy_(Wh[i], non_blocking=True)
-            packed.append(R.razer_quantize_weights(Wd[i]))
+        codes, scales, ts = R.razer_quantize_weights_batch(Wd, "weight")
         for i in range(len(SHAPES)):
             for B in BATCHES:
                 Xd[B][i].copy_(Xh[B][i], non_blocking=True)
-                y = R.razer_gemv(Xd[B][i], *packed[i], "weight", torch.float16)
+                y = R.razer_gemv(Xd[B][i], codes[i], scales[i], ts[i:i + 1], "weight", torch.float16)
                 Yh[B][i].copy_(y, non_blocking=True)
 
     for _ in range(3):
