@@ -38,7 +38,8 @@ sys.path.insert(0, ROOT)
 METRIC = "RaZeR W4A16 GEMV HBM GB/s & GEMM TFLOP/s vs B200 roofline; quantize GB/s"
 SHAPES = [(4096, 4096), (14336, 4096), (4096, 14336)]  # (N, K) of the Llama-3-8B projections
 BATCHES = [1, 4, 16]
-WORKLOAD = "llama3-8b-decode-w4a16: quantize 3 projections (one batched call) + GEMV B=1,4,16 (fp16)"
+WORKLOAD = ("llama3-8b-decode-w4a16: quantize the 3 projections (one batched call) + GEMV of the 3 projections at "
+            "B=1, 4, 16 (fp16; one batched call per B)")
 
 
 def quant_bytes(N, K):
@@ -72,7 +73,7 @@ def load_peaks():
 
 TRAFFIC_SOURCES = {  # the files each timed call's kernels are built from
     "quantize_batch": ["quantize.cu", "razer_internal.cuh"],
-    "gemv_kernel": ["gemv_tma.cu", "gemv.cu", "sm100_async.cuh", "razer_internal.cuh"],
+    "gemv_batch": ["gemv_tma.cu", "gemv.cu", "sm100_async.cuh", "razer_internal.cuh"],
 }
 
 
@@ -250,7 +251,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the breakdown / e2e / GEMM legs")
     ap.add_argument("--no-soak", action="store_true", help="skip the 1.5 s pre-timing load for the clock sampler")
-    ap.add_argument("--kernel", choices=["quantize", "quantize_batch", "act_quantize", "dequant", "gemv", "gemm"],
+    ap.add_argument("--kernel", choices=["quantize", "quantize_batch", "act_quantize", "dequant", "gemv", "gemv_batch", "gemm"],
                     help="profiling mode: run one call on --shape in a loop (for ncu)")
     ap.add_argument("--shape", default="4096,4096", help="N,K (gemm: M,N,K; quantize_batch: N1,K1,N2,K2,...)")
     ap.add_argument("--batch", type=int, default=1)
@@ -297,15 +298,21 @@ def main():
                torch.empty(len(SHAPES), dtype=torch.float32, device=dev)) for _ in range(2)]
     Y = {B: [torch.empty((B, N), dtype=torch.float16, device=dev) for N, _ in SHAPES] for B in BATCHES}
     wsz = max(R.razer_workspace_size(R.RAZER_OP_GEMV, B, N, K) for N, K in SHAPES for B in BATCHES)
+
+    # one batched GEMV call per B over the three (distinct) projections: the
+    # products of one call share no weights, so no call reads a matrix that
+    # another product of the same call also streams
+    def gemv_problems(pk, B):
+        return [(X[B][i], pk[0][i], pk[1][i], pk[2][i:i + 1]) for i in range(len(SHAPES))]
+
+    wsz = max([wsz] + [R.razer_gemv_batch_workspace_size(gemv_problems(packed[0], B)) for B in BATCHES])
     ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
 
     def step(s):
         cur, prev = packed[s % 2], packed[(s + 1) % 2]
         R.razer_quantize_weights_batch(W, "weight", codes=cur[0], scales=cur[1], ts=cur[2])
-        for i in range(len(SHAPES)):
-            c, sc, t = prev[0][i], prev[1][i], prev[2][i:i + 1]
-            for B in BATCHES:
-                R.razer_gemv(X[B][i], c, sc, t, "weight", torch.float16, out=Y[B][i], workspace=ws)
+        for B in BATCHES:
+            R.razer_gemv_batch(gemv_problems(prev, B), "weight", torch.float16, outs=Y[B], workspace=ws)
 
     # the first GEMVs read the second packed set: fill it; warm every path
     step(1)
@@ -381,10 +388,6 @@ def main():
                                      for r in range(npk)], npk, stream)
             nb = gemv_bytes(B, N, K)
             breakdown[f"gemv_{N}x{K}_b{B}"] = {"ms": ms, "GB/s": nb / ms / 1e6}
-            by_kind.setdefault("gemv", [0.0, 0.0, 0])
-            by_kind["gemv"][0] += ms
-            by_kind["gemv"][1] += nb
-            by_kind["gemv"][2] += 1
         del pk, outs
     # the step's quantize call: all three projections in one batched call,
     # two weight sets alternating (536 MB of fp16 input, > 2x L2)
@@ -396,17 +399,30 @@ def main():
     nb = sum(quant_bytes(N, K) for N, K in SHAPES)
     breakdown["quantize_batch_3proj"] = {"ms": ms, "GB/s": nb / ms / 1e6}
     by_kind["quantize"] = [ms, nb, 1]
-    del Wsets, qouts
+    # the step's GEMV calls: one batched call per B over the three
+    # projections, each on three copies of the packed weights (3 x 75 MB, > L2)
+    pks = [packed[0]] + [([c.clone() for c in packed[0][0]], [c.clone() for c in packed[0][1]], packed[0][2].clone()) for _ in range(2)]
+    by_kind["gemv"] = [0.0, 0.0, 0]
+    for B in BATCHES:
+        ms = time_graph(lambda: [R.razer_gemv_batch(gemv_problems(pks[r], B), "weight", torch.float16, outs=Y[B], workspace=ws)
+                                 for r in range(3)], 3, stream)
+        nb = sum(gemv_bytes(B, N, K) for N, K in SHAPES)
+        breakdown[f"gemv_batch_3proj_b{B}"] = {"ms": ms, "GB/s": nb / ms / 1e6}
+        by_kind["gemv"][0] += ms
+        by_kind["gemv"][1] += nb
+        by_kind["gemv"][2] += 1
+    del Wsets, qouts, pks
     torch.cuda.empty_cache()
     dominant = max(by_kind, key=lambda k: by_kind[k][0])
     dom_ms, dom_bytes, n_calls = by_kind[dominant]
     achieved = dom_bytes / dom_ms / 1e6  # GB/s over that kind's calls
-    kname = "quantize_batch" if dominant == "quantize" else "gemv_kernel"
+    kname = "quantize_batch" if dominant == "quantize" else "gemv_batch"
     traffic = traffic_for(kname)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": traffic, "kernel": ("razer_quantize_weights_batch of the 3 projections (amax, fused quantize + "
                                                "next-amax, quantize kernels)" if dominant == "quantize"
-                                               else "razer_gemv (gemv + split-K reduce kernels)"),
+                                               else "razer_gemv_batch of the 3 projections, per B (bulk-tensor + split-K "
+                                                    "reduce kernels)"),
                 "algorithmic_bytes_per_call": dom_bytes / n_calls, "peak_source": peak_src,
                 "timing": "CUDA events around CUDA-graph replays of back-to-back calls on operand copies larger than L2"}
 
@@ -420,8 +436,9 @@ def main():
         e2e = run_e2e(R, workloads, dev, stream, args, world, pg)
 
     # kernel nodes of the captured step graph: init + amax + 2 fused stages +
-    # quantize + finalize for the batch, main + reduction kernel per GEMV
-    launches_per_step = kernels_per_step if kernels_per_step is not None else 6 + len(SHAPES) * len(BATCHES) * 2
+    # quantize + finalize for the quantizer batch, main + reduction kernel per
+    # batched GEMV call
+    launches_per_step = kernels_per_step if kernels_per_step is not None else 6 + 2 * len(BATCHES)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -479,6 +496,18 @@ def run_single_kernel(args):
 
         def call():
             R.razer_quantize_weights_batch(Ws, codes=cs, scales=ss, ts=ts)
+    elif args.kernel == "gemv_batch":
+        # the GEMV at --batch on each N,K pair of --shape, one batched call
+        pairs = [(dims[2 * i], dims[2 * i + 1]) for i in range(len(dims) // 2)]
+        probs = []
+        for i, (N, K) in enumerate(pairs):
+            c, s, t = R.razer_quantize_weights(workloads.weight(N, K, seed=1 + i).to(dev))
+            probs.append((workloads.vectors(args.batch, K, seed=2 + i).to(dev), c, s, t))
+        ys = R.razer_gemv_batch(probs, "weight", torch.float16)
+        ws = torch.empty(max(16, R.razer_gemv_batch_workspace_size(probs)), dtype=torch.uint8, device=dev)
+
+        def call():
+            R.razer_gemv_batch(probs, "weight", torch.float16, outs=ys, workspace=ws)
     elif args.kernel == "act_quantize":
         M, K = dims
         xa = workloads.outlier_activations(M, K, seed=3).to(dev)
@@ -606,7 +635,10 @@ def run_e2e(R, workloads, dev, stream, args, world, pg):
         for i in range(len(SHAPES)):
             for B in BATCHES:
                 Xd[B][i].copy_(Xh[B][i], non_blocking=True)
-                y = R.razer_gemv(Xd[B][i], codes[i], scales[i], ts[i:i + 1], "weight", torch.float16)
+        for B in BATCHES:
+            ys = R.razer_gemv_batch([(Xd[B][i], codes[i], scales[i], ts[i:i + 1]) for i in range(len(SHAPES))], "weight",
+                                    torch.float16)
+            for i, y in enumerate(ys):
                 Yh[B][i].copy_(y, non_blocking=True)
 
     for _ in range(3):

@@ -29,6 +29,9 @@ razer_status run_dequant(const uint8_t *codes, const uint8_t *scales, const floa
 razer_status run_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
                       razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st);
 size_t gemv_workspace_bytes(int64_t B, int64_t N, int64_t K);
+razer_status run_gemv_batch(int count, const razer_gemv_problem *P, razer_dtype act_dt, razer_format wfmt, razer_dtype out_dt,
+                            void *workspace, cudaStream_t st);
+size_t gemv_batch_workspace_bytes(int count, const razer_gemv_problem *P);
 razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
                       razer_format wfmt, int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
@@ -142,6 +145,35 @@ razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint
         if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
     }
     return run_gemv(x, act_dt, B, codes, scales, ts, wfmt, N, K, y, out_dt, workspace, (cudaStream_t)stream);
+}
+
+size_t razer_gemv_batch_workspace_size(int count, const razer_gemv_problem *problems)
+{
+    if (count <= 0 || !problems) return 0;
+    return gemv_batch_workspace_bytes(count, problems);
+}
+
+razer_status razer_gemv_batch(int count, const razer_gemv_problem *problems, razer_dtype act_dt, razer_format wfmt, razer_dtype out_dt,
+                              void *workspace, size_t ws_bytes, razer_stream_t stream)
+{
+    if (count < 0 || (count > 0 && !problems)) return RAZER_ERR_INVALID_ARG;
+    if (count == 0) return RAZER_OK;
+    if (!valid_fmt(wfmt) || !valid_dt(act_dt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(act_dt)) return RAZER_ERR_DTYPE;
+    for (int i = 0; i < count; i++) {  // each problem as razer_gemv checks its arguments
+        const razer_gemv_problem &p = problems[i];
+        if (!p.ts || (!p.x && p.K > 0) || (!p.y && p.N > 0)) return RAZER_ERR_INVALID_ARG;
+        razer_status st = check_packed(p.codes, p.scales, p.N, p.K);
+        if (st != RAZER_OK) return st;
+        if (p.B < 1 || p.B > 32 || p.K % 128 != 0 || p.N > INT32_MAX || p.K > INT32_MAX) return RAZER_ERR_SHAPE;
+        if (!aligned(p.x, 16) || !aligned(p.y, 16) || !aligned(p.ts, 4)) return RAZER_ERR_ALIGN;
+    }
+    const size_t need = gemv_batch_workspace_bytes(count, problems);
+    if (need) {
+        if (!workspace || ws_bytes < need) return RAZER_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
+    }
+    return run_gemv_batch(count, problems, act_dt, wfmt, out_dt, workspace, (cudaStream_t)stream);
 }
 
 razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,

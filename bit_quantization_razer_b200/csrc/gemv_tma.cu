@@ -36,6 +36,8 @@
 //     arrivals) uniform, and the producer lets its in-flight loads land
 //     before it exits.
 #include <algorithm>
+#include <cstring>
+#include <vector>
 
 #include "razer_internal.cuh"
 #include "sm100_async.cuh"
@@ -68,6 +70,32 @@ __host__ __device__ constexpr int num_stages(int B)
                : (kSmemLimit - 1024 - kBarBytes - part_bytes(B)) / stage_bytes(B);
 }
 __host__ __device__ constexpr int smem_bytes(int B) { return num_stages(B) * stage_bytes(B) + part_bytes(B) + kBarBytes + 1024; }
+
+// A batch of independent problems y_i = ts_i * x_i * deq(W_i)^T (same
+// formats, same output type) run as one stream-K pass: their tiles are
+// concatenated in problem order, so one launch (one pipeline fill, one drain,
+// one reduction) serves all of them.  Problem i covers the global half-units
+// [unit0[i], unit0[i + 1]) and the global tiles [tile0[i], tile0[i + 1]).
+constexpr int kMaxProblems = 8;
+struct BatchInfo {
+    int count;
+    int B[kMaxProblems], N[kMaxProblems], UK2[kMaxProblems];
+    int unit0[kMaxProblems + 1], tile0[kMaxProblems + 1];
+    const float *ts[kMaxProblems];
+    void *y[kMaxProblems];
+};
+struct Batch {
+    CUtensorMap map[kMaxProblems][3];  // codes, scales and x of problem i
+    BatchInfo info;
+};
+
+// the problem whose half-units contain global half-unit p
+__device__ __forceinline__ int problem_of(const BatchInfo &I, int p)
+{
+    int i = 0;
+    while (i + 1 < I.count && p >= I.unit0[i + 1]) i++;
+    return i;
+}
 
 // first half-unit of CTA c's range
 __host__ __device__ __forceinline__ int range_start(int c, int U, int G) { return (int)((int64_t)c * U / G); }
@@ -111,14 +139,14 @@ __device__ __forceinline__ void wait_phase(uint32_t bar, uint32_t ph, volatile i
 
 template <int FMT, bool BF16, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemv_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
-                    const __grid_constant__ CUtensorMap tm_x, int B, int N, int UK2, int U, int stages, int stage_sz,
-                    float *__restrict__ ws, const float *__restrict__ ts_p, float unbias, void *__restrict__ y, int out_dt)
+    gemv_tma_kernel(const __grid_constant__ Batch A, int U, int stages, int stage_sz, int slot_elems, float *__restrict__ ws,
+                    float unbias, int out_dt)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *part = reinterpret_cast<float *>(smem + stages * stage_sz);  // [2 buffers][2 k-halves][B][128]
-    uint8_t *bars = smem + stages * stage_sz + 2 * 2 * B * kTileRows * 4;
+    const BatchInfo &I = A.info;
+    float *part = reinterpret_cast<float *>(smem + stages * stage_sz);  // [2 buffers][2 k-halves][Bmax][128]
+    uint8_t *bars = smem + stages * stage_sz + 2 * 2 * slot_elems * 4;
     const uint32_t full = smem_addr(bars), empty = full + 8 * kMaxStages;
     const uint32_t pfull = empty + 8 * kMaxStages, pempty = pfull + 16;
     volatile int *flags = reinterpret_cast<volatile int *>(bars + 16 * kMaxStages + 32);  // [0] abort
@@ -148,18 +176,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the tensor maps are kernel parameters: fetch them while the
             // previous kernel in the stream may still run; its outputs (which
             // may be our inputs) are read only after griddepcontrol.wait
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_codes)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_scales)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
+            for (int pi = problem_of(I, p_begin); pi <= problem_of(I, p_end - 1); pi++)
+#pragma unroll
+                for (int m = 0; m < 3; m++) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&A.map[pi][m])) : "memory");
             asm volatile("griddepcontrol.wait;" ::: "memory");
-            const uint32_t tx = (uint32_t)(kCodeBytes + kScaleBytes + B * 512);
             int s = 0, issued = 0;
             uint32_t ph = 0;
             bool ok = true;
             for (int p = p_begin; p < p_end && ok;) {
-                const int r = p / UK2;
-                const int pe = min(p_end, (r + 1) * UK2);
-                const int h0 = p - r * UK2, h1 = pe - r * UK2;
+                const int pi = problem_of(I, p), UK2 = I.UK2[pi], u0 = I.unit0[pi];
+                const int r = (p - u0) / UK2;
+                const int pe = min(p_end, u0 + (r + 1) * UK2);
+                const int h0 = p - u0 - r * UK2, h1 = pe - u0 - r * UK2;
+                const uint32_t tx = (uint32_t)(kCodeBytes + kScaleBytes + I.B[pi] * 512);
+                const CUtensorMap *tm_codes = &A.map[pi][0], *tm_scales = &A.map[pi][1], *tm_x = &A.map[pi][2];
                 for (int j = h0 >> 1; j < (h1 + 1) >> 1; j++) {
                     if (!mbar_wait(empty + 8 * s, ph ^ 1u, flags)) {
                         ok = false;
@@ -167,9 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const uint32_t dst = smem_addr(smem + s * stage_sz);
                     mbar_expect_tx(full + 8 * s, tx);
-                    tma_load_2d(dst, &tm_codes, j * 128, r * kTileRows, full + 8 * s);
-                    tma_load_2d(dst + kCodeBytes, &tm_scales, j * 16, r * kTileRows, full + 8 * s);
-                    tma_load_2d(dst + kCodeBytes + kScaleBytes, &tm_x, j * 256, 0, full + 8 * s);
+                    tma_load_2d(dst, tm_codes, j * 128, r * kTileRows, full + 8 * s);
+                    tma_load_2d(dst + kCodeBytes, tm_scales, j * 16, r * kTileRows, full + 8 * s);
+                    tma_load_2d(dst + kCodeBytes + kScaleBytes, tm_x, j * 256, 0, full + 8 * s);
                     issued++;
                     if (++s == stages) {
                         s = 0;
@@ -192,16 +222,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         // ------------------------- epilogue -------------------------
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        const float oscale = __fmul_rn(*ts_p, unbias);
-        const int slot_elems = B * kTileRows;
         int q = 0;
         for (int p = p_begin; p < p_end; q++) {
-            const int r = p / UK2;
-            const int pe = min(p_end, (r + 1) * UK2);
+            const int pi = problem_of(I, p), UK2 = I.UK2[pi], u0 = I.unit0[pi], B = I.B[pi], N = I.N[pi];
+            void *y = I.y[pi];
+            const float oscale = __fmul_rn(*I.ts[pi], unbias);
+            const int r = (p - u0) / UK2;
+            const int pe = min(p_end, u0 + (r + 1) * UK2);
             const int buf = q & 1;
             wait_phase(pfull + 8 * buf, (uint32_t)(q >> 1) & 1u, flags);
             const float *h0p = part + buf * 2 * slot_elems, *h1p = h0p + slot_elems;
-            const int c_first = range_owner(r * UK2, U, G), c_last = range_owner((r + 1) * UK2 - 1, U, G);
+            const int c_first = range_owner(u0 + r * UK2, U, G), c_last = range_owner(u0 + (r + 1) * UK2 - 1, U, G);
             const int row_base = r * kTileRows;
             // lane owns float4 e4 = lane + 32 i (i < B) of the [B][128] tile
             const float4 *h0v = reinterpret_cast<const float4 *>(h0p), *h1v = reinterpret_cast<const float4 *>(h1p);
@@ -218,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(pempty + 8 * buf);
             } else {
-                float4 *slot = reinterpret_cast<float4 *>(ws + (size_t)(c + r) * slot_elems);
+                float4 *slot = reinterpret_cast<float4 *>(ws + (size_t)(c + I.tile0[pi] + r) * slot_elems);
                 for (int i = 0; i < B; i++) {
                     const int e4 = lane + 32 * i;
                     const float4 a = h0v[e4], b4 = h1v[e4];
@@ -243,7 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t offA = (uint32_t)(R0 * 128 + ((cc ^ pr) << 4));  // + 1024 for row g + 8, + 2048 per 16-row tile
     const uint32_t offS = (uint32_t)(kCodeBytes + R0 * 16 + 2 * cc);  // + 128 for row g + 8, + 256 per tile
     const uint32_t offX = (uint32_t)(kCodeBytes + kScaleBytes + g * 512 + 64 * cc);
-    const bool xrow = g < B;
 
     float acc[kMT][NB][4];
     unsigned xw[NB][16];
@@ -256,9 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     uint32_t st = sbase;
     for (int p = p_begin; p < p_end; q++) {
-        const int r = p / UK2;
-        const int pe = min(p_end, (r + 1) * UK2);
-        const int h0 = p - r * UK2, h1 = pe - r * UK2;
+        const int pi = problem_of(I, p), UK2 = I.UK2[pi], u0 = I.unit0[pi], B = I.B[pi];
+        const bool xrow = g < B;
+        const int r = (p - u0) / UK2;
+        const int pe = min(p_end, u0 + (r + 1) * UK2);
+        const int h0 = p - u0 - r * UK2, h1 = pe - u0 - r * UK2;
         // stages j whose half-unit 2j + kh lies in [h0, h1)
         const int ja = (h0 - kh + 1) >> 1, jb = (h1 - 1 - kh) >> 1;
 #pragma unroll
@@ -309,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // hand the partial of this tile to the epilogue warp and go on
         const int buf = q & 1;
         wait_phase(pempty + 8 * buf, ((uint32_t)(q >> 1) & 1u) ^ 1u, flags);
-        float *dst = part + (buf * 2 + kh) * B * kTileRows;
+        float *dst = part + (buf * 2 + kh) * slot_elems;
 #pragma unroll
         for (int m = 0; m < kMT; m++) {
 #pragma unroll
@@ -331,50 +363,67 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Sums the workspace slots of the tiles shared by several CTAs, in CTA order.
 // Launched as a programmatic dependent of gemv_tma_kernel: it may become
 // resident early and waits here until that grid has completed.
-__global__ void __launch_bounds__(256) gemv_tma_reduce_kernel(const float *__restrict__ ws, int B, int N, int UK2, int U, int G, int T,
-                                                              const float *__restrict__ ts_p, float unbias, void *__restrict__ y, int out_dt)
+__global__ void __launch_bounds__(256) gemv_tma_reduce_kernel(const float *__restrict__ ws, const BatchInfo I, int slot_elems, int U,
+                                                              int G, float unbias, int out_dt)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next call may become resident
-    const float oscale = __fmul_rn(*ts_p, unbias);
-    const int slot_elems = B * kTileRows;
-    const int64_t total = (int64_t)T * slot_elems;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int r = (int)(i / slot_elems), e = (int)(i - (int64_t)r * slot_elems);
-        const int c_first = range_owner(r * UK2, U, G), c_last = range_owner((r + 1) * UK2 - 1, U, G);
-        const int row = r * kTileRows + (e & (kTileRows - 1));
-        if (c_first == c_last || row >= N) continue;  // whole tiles were written by the main kernel
-        const float *src = ws + (size_t)r * slot_elems + e;
+    const int64_t total = (int64_t)I.tile0[I.count] * slot_elems;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+        const int R = (int)(t / slot_elems), e = (int)(t - (int64_t)R * slot_elems);
+        int pi = 0;
+        while (pi + 1 < I.count && R >= I.tile0[pi + 1]) pi++;
+        const int r = R - I.tile0[pi], UK2 = I.UK2[pi], u0 = I.unit0[pi], N = I.N[pi];
+        const int c_first = range_owner(u0 + r * UK2, U, G), c_last = range_owner(u0 + (r + 1) * UK2 - 1, U, G);
+        const int row = r * kTileRows + (e & (kTileRows - 1)), b = e >> 7;
+        if (c_first == c_last || row >= N || b >= I.B[pi]) continue;  // whole tiles were written by the main kernel
+        // slot (cta + global tile) holds that CTA's part of the tile
+        const float *src = ws + (size_t)R * slot_elems + e;
         float sum = 0.0f;
         for (int k = c_first; k <= c_last; k++) sum += __ldcg(src + (size_t)k * slot_elems);
-        store_out(y, out_dt, (size_t)(e >> 7) * N + row, __fmul_rn(sum, oscale));
+        store_out(I.y[pi], out_dt, (size_t)b * N + row, __fmul_rn(sum, __fmul_rn(*I.ts[pi], unbias)));
     }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-struct Plan {
-    int64_t T, UK2, U, G;  // tiles, half-units per tile, half-units, CTAs
-    size_t total;  // workspace: one [B][128] fp32 slot per (CTA, tile) pair
+struct Problem {
+    const void *x;
+    int64_t B;
+    const uint8_t *codes, *scales;
+    const float *ts;
+    int64_t N, K;
+    void *y;
 };
 
-static Plan plan(int64_t B, int64_t N, int64_t K)
+struct Plan {
+    int64_t T, U, G, Bmax;  // tiles, half-units, CTAs, largest batch of the group
+    size_t total;           // workspace: one [Bmax][128] fp32 slot per (CTA, tile) pair
+};
+
+static Plan plan(const Problem *P, int n)
 {
-    Plan p;
-    p.T = (N + kTileRows - 1) / kTileRows;
-    p.UK2 = K / 128;
-    p.U = p.T * p.UK2;
+    Plan p = {0, 0, 0, 0, 0};
+    for (int i = 0; i < n; i++) {
+        const int64_t T = (P[i].N + kTileRows - 1) / kTileRows;
+        p.T += T;
+        p.U += T * (P[i].K / 128);
+        p.Bmax = std::max<int64_t>(p.Bmax, P[i].B);
+    }
     p.G = std::min<int64_t>(sm_count(), p.U);
-    p.total = (size_t)(p.G + p.T - 1) * (size_t)B * kTileRows * sizeof(float);
+    p.total = (size_t)(p.G + p.T - 1) * (size_t)p.Bmax * kTileRows * sizeof(float);
     return p;
 }
 
+// n-tiles of 8 columns the MMA needs for batch B
+static int nb_class(int64_t B) { return B <= 8 ? 1 : (B <= 16 ? 2 : 4); }
+
 template <int FMT, bool BF16, int NB>
-static razer_status launch(const CUtensorMap &tc, const CUtensorMap &tsc, const CUtensorMap &tx, int B, int N, const Plan &pl,
-                           float *ws, const float *ts, float unbias, void *y, razer_dtype out_dt, cudaStream_t st)
+static razer_status launch(const Batch &A, const Plan &pl, float *ws, float unbias, razer_dtype out_dt, cudaStream_t st)
 {
-    const int stages = num_stages(B), sz = stage_bytes(B), smem = smem_bytes(B);
+    const int Bmax = (int)pl.Bmax;
+    const int stages = num_stages(Bmax), sz = stage_bytes(Bmax), smem = smem_bytes(Bmax), slot_elems = Bmax * kTileRows;
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -383,30 +432,84 @@ static razer_status launch(const CUtensorMap &tc, const CUtensorMap &tsc, const 
             return RAZER_ERR_CUDA;
         attr_done[dev] = true;
     }
-    const int UK2 = (int)pl.UK2, U = (int)pl.U, G = (int)pl.G, T = (int)pl.T;
-    if (launch_pdl(gemv_tma_kernel<FMT, BF16, NB>, (unsigned)G, kThreads, (size_t)smem, st, tc, tsc, tx, B, N, UK2, U, stages, sz, ws, ts,
-                   unbias, y, (int)out_dt) != cudaSuccess)
+    const int U = (int)pl.U, G = (int)pl.G;
+    if (launch_pdl(gemv_tma_kernel<FMT, BF16, NB>, (unsigned)G, kThreads, (size_t)smem, st, A, U, stages, sz, slot_elems, ws, unbias,
+                   (int)out_dt) != cudaSuccess)
         return RAZER_ERR_CUDA;
     // tiles shared by several CTAs exist unless every CTA range is whole tiles
+    const BatchInfo &I = A.info;
     bool shared = false;
-    for (int64_t r = 0; r < pl.T && !shared; r++)
-        shared = range_owner((int)(r * pl.UK2), U, G) != range_owner((int)((r + 1) * pl.UK2 - 1), U, G);
+    for (int pi = 0; pi < I.count && !shared; pi++)
+        for (int r = 0; r < I.tile0[pi + 1] - I.tile0[pi] && !shared; r++)
+            shared = range_owner(I.unit0[pi] + r * I.UK2[pi], U, G) != range_owner(I.unit0[pi] + (r + 1) * I.UK2[pi] - 1, U, G);
     if (!shared) return RAZER_OK;
-    const int64_t total = pl.T * B * kTileRows;
+    const int64_t total = pl.T * slot_elems;
     const unsigned rgrid = (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 4);
-    if (launch_pdl(gemv_tma_reduce_kernel, rgrid, 256u, 0, st, (const float *)ws, B, N, UK2, U, G, T, ts, unbias, y, (int)out_dt) !=
-        cudaSuccess)
+    if (launch_pdl(gemv_tma_reduce_kernel, rgrid, 256u, 0, st, (const float *)ws, I, slot_elems, U, G, unbias, (int)out_dt) != cudaSuccess)
         return RAZER_ERR_CUDA;
     return RAZER_OK;
 }
 
 template <int FMT, bool BF16>
-static razer_status launch_nb(const CUtensorMap &tc, const CUtensorMap &tsc, const CUtensorMap &tx, int B, int N, const Plan &pl,
-                              float *ws, const float *ts, float unbias, void *y, razer_dtype out_dt, cudaStream_t st)
+static razer_status launch_nb(int nb, const Batch &A, const Plan &pl, float *ws, float unbias, razer_dtype out_dt, cudaStream_t st)
 {
-    if (B <= 8) return launch<FMT, BF16, 1>(tc, tsc, tx, B, N, pl, ws, ts, unbias, y, out_dt, st);
-    if (B <= 16) return launch<FMT, BF16, 2>(tc, tsc, tx, B, N, pl, ws, ts, unbias, y, out_dt, st);
-    return launch<FMT, BF16, 4>(tc, tsc, tx, B, N, pl, ws, ts, unbias, y, out_dt, st);
+    if (nb == 1) return launch<FMT, BF16, 1>(A, pl, ws, unbias, out_dt, st);
+    if (nb == 2) return launch<FMT, BF16, 2>(A, pl, ws, unbias, out_dt, st);
+    return launch<FMT, BF16, 4>(A, pl, ws, unbias, out_dt, st);
+}
+
+// The three tensor maps of one problem: codes [N, K/2] u8 in 128 x 128-byte
+// boxes (128-byte swizzle), scales [N, K/16] u8 in 128 x 16-byte boxes, x
+// [B, K] 16-bit in B x 256 boxes.
+static bool encode_problem(EncodeTiledFn enc, const Problem &P, CUtensorMap *m)
+{
+    const cuuint32_t estr[2] = {1u, 1u};
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(P.K / 2), (cuuint64_t)P.N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(P.K / 2)};
+        const cuuint32_t box[2] = {128u, (cuuint32_t)kTileRows};
+        if (enc(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(P.codes), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(P.K / 16), (cuuint64_t)P.N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(P.K / 16)};
+        const cuuint32_t box[2] = {16u, (cuuint32_t)kTileRows};
+        if (enc(&m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(P.scales), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)P.K, (cuuint64_t)P.B};
+        const cuuint64_t strides[1] = {(cuuint64_t)P.K * 2};
+        const cuuint32_t box[2] = {256u, (cuuint32_t)P.B};
+        if (enc(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(P.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    return true;
+}
+
+// Calls fn(group, n) for the launches of a batch: problems of the same
+// n-tile class, in their order, at most kMaxProblems per launch.
+template <typename Fn> static razer_status for_each_group(const Problem *P, int n, Fn fn)
+{
+    for (int nb = 1; nb <= 4; nb *= 2) {
+        Problem g[kMaxProblems];
+        int k = 0;
+        for (int i = 0; i <= n; i++) {
+            if (i < n && nb_class(P[i].B) == nb) g[k++] = P[i];
+            if (k > 0 && (k == kMaxProblems || i == n)) {
+                const razer_status r = fn(nb, g, k);
+                if (r != RAZER_OK) return r;
+                k = 0;
+            }
+        }
+    }
+    return RAZER_OK;
 }
 
 }  // namespace gemv_tma
@@ -417,54 +520,114 @@ bool gemv_tma_eligible(int64_t B, int64_t N, int64_t K)
     return B >= 1 && B <= 32 && N >= 1 && K >= 256 && K % 256 == 0 && ((N + 127) / 128) * (K / 128) < (int64_t)INT32_MAX;
 }
 
-size_t gemv_tma_workspace_bytes(int64_t B, int64_t N, int64_t K) { return gemv_tma::plan(B, N, K).total; }
+size_t gemv_tma_batch_workspace_bytes(const gemv_tma::Problem *P, int n)
+{
+    size_t need = 0;
+    gemv_tma::for_each_group(P, n, [&](int, const gemv_tma::Problem *g, int k) {
+        need = std::max(need, gemv_tma::plan(g, k).total);
+        return RAZER_OK;
+    });
+    return need;
+}
 
-razer_status run_gemv_tma(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
-                          razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st)
+size_t gemv_tma_workspace_bytes(int64_t B, int64_t N, int64_t K)
+{
+    gemv_tma::Problem P = {nullptr, B, nullptr, nullptr, nullptr, N, K, nullptr};
+    return gemv_tma_batch_workspace_bytes(&P, 1);
+}
+
+// Runs the problems (each gemv_tma_eligible, scales 16-byte aligned) in as few
+// launches as their n-tile classes allow; the launches reuse one workspace
+// (each waits for its predecessor in the stream before writing it).
+razer_status run_gemv_tma_batch(const gemv_tma::Problem *P, int n, razer_dtype act_dt, razer_format wfmt, razer_dtype out_dt,
+                                void *workspace, cudaStream_t st)
 {
     using namespace gemv_tma;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return RAZER_ERR_CUDA;
-    const Plan pl = plan(B, N, K);
-    const cuuint32_t estr[2] = {1u, 1u};
-    CUtensorMap tc, tsc, tx;
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
-        const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-        const cuuint32_t box[2] = {128u, (cuuint32_t)kTileRows};
-        if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return RAZER_ERR_CUDA;
-    }
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
-        const cuuint64_t strides[1] = {(cuuint64_t)(K / 16)};
-        const cuuint32_t box[2] = {16u, (cuuint32_t)kTileRows};
-        if (enc(&tsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(scales), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return RAZER_ERR_CUDA;
-    }
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)B};
-        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        const cuuint32_t box[2] = {256u, (cuuint32_t)B};
-        if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return RAZER_ERR_CUDA;
-    }
     float *ws = reinterpret_cast<float *>(workspace);
     const float unbias = wfmt == RAZER_FMT_WEIGHT ? scale_f16_unbias<RAZER_FMT_WEIGHT>() : scale_f16_unbias<RAZER_FMT_ACT>();
     const bool bf = act_dt == RAZER_BF16;
-    const int b = (int)B, n = (int)N;
-    if (wfmt == RAZER_FMT_WEIGHT)
-        return bf ? launch_nb<RAZER_FMT_WEIGHT, true>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st)
-                  : launch_nb<RAZER_FMT_WEIGHT, false>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st);
-    if (wfmt == RAZER_FMT_ACT)
-        return bf ? launch_nb<RAZER_FMT_ACT, true>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st)
-                  : launch_nb<RAZER_FMT_ACT, false>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st);
-    return bf ? launch_nb<RAZER_FMT_NVFP4, true>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st)
-              : launch_nb<RAZER_FMT_NVFP4, false>(tc, tsc, tx, b, n, pl, ws, ts, unbias, y, out_dt, st);
+    return for_each_group(P, n, [&](int nb, const Problem *g, int k) {
+        Batch A;
+        memset(&A, 0, sizeof(A));
+        BatchInfo &I = A.info;
+        I.count = k;
+        for (int i = 0; i < k; i++) {
+            if (!encode_problem(enc, g[i], A.map[i])) return RAZER_ERR_CUDA;
+            const int T = (int)((g[i].N + kTileRows - 1) / kTileRows), UK2 = (int)(g[i].K / 128);
+            I.B[i] = (int)g[i].B;
+            I.N[i] = (int)g[i].N;
+            I.UK2[i] = UK2;
+            I.unit0[i + 1] = I.unit0[i] + T * UK2;
+            I.tile0[i + 1] = I.tile0[i] + T;
+            I.ts[i] = g[i].ts;
+            I.y[i] = g[i].y;
+        }
+        const Plan pl = plan(g, k);
+        if (wfmt == RAZER_FMT_WEIGHT)
+            return bf ? launch_nb<RAZER_FMT_WEIGHT, true>(nb, A, pl, ws, unbias, out_dt, st)
+                      : launch_nb<RAZER_FMT_WEIGHT, false>(nb, A, pl, ws, unbias, out_dt, st);
+        if (wfmt == RAZER_FMT_ACT)
+            return bf ? launch_nb<RAZER_FMT_ACT, true>(nb, A, pl, ws, unbias, out_dt, st)
+                      : launch_nb<RAZER_FMT_ACT, false>(nb, A, pl, ws, unbias, out_dt, st);
+        return bf ? launch_nb<RAZER_FMT_NVFP4, true>(nb, A, pl, ws, unbias, out_dt, st)
+                  : launch_nb<RAZER_FMT_NVFP4, false>(nb, A, pl, ws, unbias, out_dt, st);
+    });
+}
+
+razer_status run_gemv_tma(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                          razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st)
+{
+    const gemv_tma::Problem P = {x, B, codes, scales, ts, N, K, y};
+    return run_gemv_tma_batch(&P, 1, act_dt, wfmt, out_dt, workspace, st);
+}
+
+// --- razer_gemv_batch: the bulk-tensor batch for every problem it can take,
+// the single-problem path for the rest (after it), empty problems handled
+// here.  Arguments were validated by the caller.
+static bool batch_tma_ok(const razer_gemv_problem &p)
+{
+    return p.N > 0 && p.K > 0 && gemv_tma_eligible(p.B, p.N, p.K) && (reinterpret_cast<uintptr_t>(p.scales) & 15) == 0;
+}
+
+size_t gemv_batch_workspace_bytes(int count, const razer_gemv_problem *P)
+{
+    std::vector<gemv_tma::Problem> t;
+    size_t other = 0;
+    for (int i = 0; i < count; i++) {
+        const razer_gemv_problem &p = P[i];
+        if (p.N == 0 || p.K == 0) continue;
+        if (batch_tma_ok(p)) t.push_back({p.x, p.B, p.codes, p.scales, p.ts, p.N, p.K, p.y});
+        else other = std::max(other, gemv_workspace_bytes(p.B, p.N, p.K));
+    }
+    return std::max(other, t.empty() ? (size_t)0 : gemv_tma_batch_workspace_bytes(t.data(), (int)t.size()));
+}
+
+razer_status run_gemv_batch(int count, const razer_gemv_problem *P, razer_dtype act_dt, razer_format wfmt, razer_dtype out_dt,
+                            void *workspace, cudaStream_t st)
+{
+    std::vector<gemv_tma::Problem> t;
+    for (int i = 0; i < count; i++) {
+        const razer_gemv_problem &p = P[i];
+        if (p.N > 0 && p.K > 0 && batch_tma_ok(p)) t.push_back({p.x, p.B, p.codes, p.scales, p.ts, p.N, p.K, p.y});
+    }
+    if (!t.empty()) {
+        const razer_status r = run_gemv_tma_batch(t.data(), (int)t.size(), act_dt, wfmt, out_dt, workspace, st);
+        if (r != RAZER_OK) return r;
+    }
+    for (int i = 0; i < count; i++) {
+        const razer_gemv_problem &p = P[i];
+        if (p.N == 0) continue;
+        if (p.K == 0) {  // empty sums: y = 0
+            if (cudaMemsetAsync(p.y, 0, (size_t)p.B * (size_t)p.N * (out_dt == RAZER_F32 ? 4 : 2), st) != cudaSuccess) return RAZER_ERR_CUDA;
+            continue;
+        }
+        if (batch_tma_ok(p)) continue;
+        const razer_status r = run_gemv(p.x, act_dt, p.B, p.codes, p.scales, p.ts, wfmt, p.N, p.K, p.y, out_dt, workspace, st);
+        if (r != RAZER_OK) return r;
+    }
+    return RAZER_OK;
 }
 
 }  // namespace razer

@@ -30,9 +30,16 @@ _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZE
 
 EXPORTED = (
     "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    "razer_gemv_batch", "razer_gemv_batch_workspace_size",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
     "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
 )
+
+
+class GemvProblem(ctypes.Structure):
+    """razer_gemv_problem of include/razer.h."""
+    _fields_ = [("x", ctypes.c_void_p), ("B", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("ts", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("y", ctypes.c_void_p)]
 
 
 class RazerError(RuntimeError):
@@ -60,6 +67,9 @@ def load() -> ctypes.CDLL:
     L.razer_dequant.argtypes = [vp, vp, vp, i32, i64, i64, vp, i32, vp]
     L.razer_gemv.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_gemm.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
+    L.razer_gemv_batch.argtypes = [i32, ctypes.POINTER(GemvProblem), i32, i32, i32, vp, sz, vp]
+    L.razer_gemv_batch_workspace_size.argtypes = [i32, ctypes.POINTER(GemvProblem)]
+    L.razer_gemv_batch_workspace_size.restype = sz
     L.razer_gemv_noalloc.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp]
     L.razer_gemv_noalloc.restype = ctypes.c_int
     L.razer_gemv_noalloc_max_scratch.argtypes = []
@@ -70,7 +80,7 @@ def load() -> ctypes.CDLL:
     L.razer_status_string.argtypes = [i32]
     L.razer_status_string.restype = ctypes.c_char_p
     L.razer_version.argtypes = []
-    for fn in ("razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    for fn in ("razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -177,6 +187,35 @@ def razer_gemv(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: t
                            _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
     _check("razer_gemv", st)
     return out
+
+
+def razer_gemv_batch(problems, fmt="weight", out_dtype=torch.float32, *, outs=None, workspace=None, stream=None):
+    """Several independent GEMVs in one call: problems = [(x, codes, scales,
+    ts), ...] (same activation dtype and device). Returns [y_i [B_i, N_i]]."""
+    n = len(problems)
+    if n == 0:
+        return []
+    dev = problems[0][0].device
+    outs = [torch.empty((x.shape[0], c.shape[0]), dtype=out_dtype, device=dev) for x, c, _, _ in problems] if outs is None else outs
+    arr = (GemvProblem * n)(*[GemvProblem(x.data_ptr(), x.shape[0], c.data_ptr(), s.data_ptr(), t.data_ptr(), c.shape[0], x.shape[1],
+                                          y.data_ptr()) for (x, c, s, t), y in zip(problems, outs)])
+    L = load()
+    need = int(L.razer_gemv_batch_workspace_size(n, arr))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.razer_gemv_batch(n, arr, _DT.get(problems[0][0].dtype, -1), _fmt(fmt), _DT.get(out_dtype, -1), _p(workspace), wsb,
+                            _stream(stream))
+    _check("razer_gemv_batch", st)
+    return outs
+
+
+def razer_gemv_batch_workspace_size(problems) -> int:
+    """Workspace bytes razer_gemv_batch needs for problems [(x, codes, scales, ts), ...]."""
+    n = len(problems)
+    arr = (GemvProblem * max(n, 1))(*[GemvProblem(x.data_ptr(), x.shape[0], c.data_ptr(), s.data_ptr(), t.data_ptr(), c.shape[0],
+                                                  x.shape[1], 0) for x, c, s, t in problems])
+    return int(load().razer_gemv_batch_workspace_size(n, arr))
 
 
 def razer_gemv_noalloc(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight",

@@ -196,6 +196,41 @@ razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint
                         razer_stream_t stream);
 
 /*
+ * razer_gemv_batch -- several independent razer_gemv products in one call
+ * (for example the projections of one layer that read the same activations):
+ *   y_i[b, n] = ts_i * sum_k x_i[b, k] * (q*s)_i[n, k]   for i < count.
+ * One activation type, weight format and output type for all problems.
+ * Problems that razer_gemv would run on its bulk-tensor kernel (K % 256 == 0,
+ * 16-byte aligned scales) share launches: their tiles are concatenated into
+ * one stream-K pass per group of up to 8 problems with the same n-tile class
+ * (B <= 8, B <= 16, B <= 32), so the pipeline fill, drain and split-K
+ * reduction are paid once per group instead of once per product.  The other
+ * problems run one by one after them.  Each y_i equals razer_gemv's result up
+ * to the order of the fp32 partial sums.
+ *   problems   HOST array of count razer_gemv_problem (device pointers in
+ *              it, each argument as for razer_gemv), read during the call
+ *   workspace  device scratch of razer_gemv_batch_workspace_size(count,
+ *              problems) bytes (16-byte aligned; contents on entry ignored),
+ *              or NULL when that size is 0
+ * Errors: those of razer_gemv for the first problem that fails a check
+ * (nothing is launched then); count < 0 or a NULL array -> INVALID_ARG.
+ */
+typedef struct {
+    const void *x;         /* [B, K] activations */
+    int64_t B;             /* 1 .. 32 */
+    const uint8_t *codes;  /* [N, K/2] */
+    const uint8_t *scales; /* [N, K/16] */
+    const float *ts;       /* device */
+    int64_t N, K;
+    void *y;               /* [B, N] */
+} razer_gemv_problem;
+
+razer_status razer_gemv_batch(int count, const razer_gemv_problem *problems, razer_dtype act_dt,
+                              razer_format wfmt, razer_dtype out_dt, void *workspace,
+                              size_t ws_bytes, razer_stream_t stream);
+size_t razer_gemv_batch_workspace_size(int count, const razer_gemv_problem *problems);
+
+/*
  * razer_gemv_noalloc -- razer_gemv for callers that cannot allocate device
  * memory (the paper has no counterpart: this is a deployment convenience).
  * Some callers cannot call cudaMalloc at all, e.g. a runtime that gives every

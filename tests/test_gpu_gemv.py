@@ -148,3 +148,60 @@ def test_gemv_scales_only_4byte_aligned(orc):
     torch.cuda.synchronize()
     ref = orc.gemm_ref(x.numpy(), codes.numpy(), scales.numpy(), 0.5, 0)
     assert rel_err(y.cpu().numpy(), ref) <= REL_TOL
+
+
+def _batch_problem(N, K, B, fmt, seed, xdt=torch.float16, ts=0.0312):
+    codes, scales = workloads.random_packed(N, K, fmt, seed=seed, max_scale_code=40)
+    x = workloads.vectors(B, K, seed=seed + 1, dtype=xdt)
+    return x, codes, scales, ts
+
+
+@pytest.mark.parametrize("fmt", ["weight", "nvfp4"])
+@pytest.mark.parametrize("xdt", [torch.float16, torch.bfloat16])
+def test_gemv_batch_mixed(orc, fmt, xdt):
+    # one call, every kind of problem: several of one n-tile class sharing a
+    # launch (ragged N, tiles split between CTAs), B of every class, a K that
+    # the bulk-tensor kernel does not take (K % 256 = 128: run on its own),
+    # an empty K (y = 0) and an empty N
+    specs = [(300, 512, 1), (1000, 256, 4), (130, 768, 8), (260, 1024, 16), (64, 1024, 32), (200, 384, 3), (70, 0, 2),
+             (0, 256, 5), (520, 2048, 2)]
+    probs = [_batch_problem(N, K, B, fmt, 100 + i, xdt, ts=0.02 + 0.01 * i) for i, (N, K, B) in enumerate(specs)]
+    dev = [(x.to(DEV), c.to(DEV), s.to(DEV), torch.tensor([t], dtype=torch.float32, device=DEV)) for x, c, s, t in probs]
+    ys = R.razer_gemv_batch(dev, fmt, torch.float32)
+    torch.cuda.synchronize()
+    for (x, c, s, t), y, (N, K, B) in zip(probs, ys, specs):
+        assert y.shape == (B, N)
+        if N == 0:
+            continue
+        if K == 0:
+            assert not y.any()
+            continue
+        ref = orc.gemm_ref(oracle_in(x), c.numpy(), s.numpy(), t, FMT_ID[fmt])
+        assert rel_err(y.cpu().numpy(), ref) <= REL_TOL, (N, K, B)
+
+
+def test_gemv_batch_more_problems_than_a_launch(orc):
+    # 11 problems of one class: two launches reuse the workspace; f16 output
+    probs = [_batch_problem(128 + 64 * i, 256 * (1 + i % 3), 1 + i % 8, "weight", 200 + i) for i in range(11)]
+    dev = [(x.to(DEV), c.to(DEV), s.to(DEV), torch.tensor([t], dtype=torch.float32, device=DEV)) for x, c, s, t in probs]
+    ws = torch.full((R.razer_gemv_batch_workspace_size(dev),), 0xFF, dtype=torch.uint8, device=DEV)  # garbage
+    ys = R.razer_gemv_batch(dev, "weight", torch.float16, workspace=ws)
+    torch.cuda.synchronize()
+    for (x, c, s, t), y in zip(probs, ys):
+        assert_close_typed(y, orc.gemm_ref(x.numpy(), c.numpy(), s.numpy(), t, 0))
+
+
+def test_gemv_batch_decode_projections_sampled(orc):
+    # the Llama-3-8B decode GEMVs of one step (3 projections x B = 1, 4, 16)
+    # in one call; 256 sampled output rows of each against the oracle
+    specs = [(N, K, B) for N, K in [(4096, 4096), (14336, 4096), (4096, 14336)] for B in (1, 4, 16)]
+    probs = [_batch_problem(N, K, B, "weight", 300 + i) for i, (N, K, B) in enumerate(specs)]
+    dev = [(x.to(DEV), c.to(DEV), s.to(DEV), torch.tensor([t], dtype=torch.float32, device=DEV)) for x, c, s, t in probs]
+    ys = R.razer_gemv_batch(dev, "weight", torch.float32)
+    y2 = R.razer_gemv_batch(dev, "weight", torch.float32)
+    torch.cuda.synchronize()
+    for i, ((x, c, s, t), y, (N, K, B)) in enumerate(zip(probs, ys, specs)):
+        assert torch.equal(y, y2[i])  # deterministic: same partition, same summation order
+        rows = np.random.default_rng(i).choice(N, 256, replace=False)
+        ref = orc.gemm_ref(x.numpy(), c.numpy()[rows], s.numpy()[rows], t, 0)
+        assert rel_err(y.cpu().numpy()[:, rows], ref) <= REL_TOL
