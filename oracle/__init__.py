@@ -86,6 +86,7 @@ def lib():
         L.ro_dequant.argtypes = [u8p, u8p, f32, ctypes.c_int, i64, i64, ctypes.c_int, vp]
         L.ro_dequant.restype = ctypes.c_int
         L.ro_gemm_ref.argtypes = [vp, ctypes.c_int, i64, u8p, u8p, f32, ctypes.c_int, i64, i64, vp, i64, vp]
+        L.ro_gemm_w4a4_ref.argtypes = [u8p, u8p, f32, ctypes.c_int, i64, u8p, u8p, f32, ctypes.c_int, i64, i64, vp, i64, vp]
         L.ro_gemm_ref.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -220,3 +221,23 @@ def gemm_ref(x, codes: np.ndarray, scales: np.ndarray, ts: float, fmt: int, rows
     if rc != 0:
         raise ValueError("oracle gemm_ref failed")
     return out
+
+
+def gemm_w4a4_ref(codes_a: np.ndarray, scales_a: np.ndarray, ts_a: float, afmt: int, codes_w: np.ndarray,
+                  scales_w: np.ndarray, ts_w: float, wfmt: int, rows=None) -> np.ndarray:
+    """r[m, n] = ts_a * ts_w * sum_k (q*s)_a[m, k] (q*s)_w[n, k] in double:
+    both operands RaZeR-packed ([M, K/2] / [M, K/16] and [N, K/2] / [N, K/16])."""
+    ca = np.ascontiguousarray(codes_a, dtype=np.uint8)
+    sa = np.ascontiguousarray(scales_a, dtype=np.uint8)
+    cw = np.ascontiguousarray(codes_w, dtype=np.uint8)
+    sw = np.ascontiguousarray(scales_w, dtype=np.uint8)
+    M, K = ca.shape[0], ca.shape[1] * 2
+    N = cw.shape[0]
+    r = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.zeros((M if r is None else r.size, N), np.float64)
+    rc = lib().ro_gemm_w4a4_ref(_ptr(ca), _ptr(sa), ts_a, afmt, M, _ptr(cw), _ptr(sw), ts_w, wfmt, N, K,
+                                None if r is None else _ptr(r), 0 if r is None else r.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle gemm_w4a4_ref failed")
+    return out
+

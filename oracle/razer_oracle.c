@@ -508,3 +508,46 @@ int ro_gemm_ref(const void *x, int x_dtype, int64_t M, const uint8_t *codes, con
     free(wrow);
     return 0;
 }
+
+/*
+ * W4A4 product (RaZeR notes, 局限与展望: on current Blackwell tensor cores the
+ * W4A4 multiply-add is emulated -- here by decoding both operands; gist.science
+ * summary 2.3: weight-activation kernels): both operands are RaZeR-packed,
+ *   r[m, n] = ts_a * ts_w * sum_k (q*s)_a[m, k] * (q*s)_w[n, k],
+ * every q*s exact, the sum accumulated in double, then one multiply by each
+ * tensor scale (in double).  rows: optional list of n_rows rows of A (NULL =
+ * all M); out is [n_rows or M, N].
+ */
+int ro_gemm_w4a4_ref(const uint8_t *codes_a, const uint8_t *scales_a, float ts_a, int afmt, int64_t M,
+                     const uint8_t *codes_w, const uint8_t *scales_w, float ts_w, int wfmt, int64_t N, int64_t K,
+                     const int64_t *rows, int64_t n_rows, double *out)
+{
+    if (K % 16 != 0)
+        return 1;
+    int64_t nm = rows ? n_rows : M;
+    double *arow = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+    double *wrows = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1) * (size_t)(N > 0 ? N : 1));
+    if (!arow || !wrows) {
+        free(arow);
+        free(wrows);
+        return 2;
+    }
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++)
+            wrows[n * K + k] = elem_qs(codes_w, scales_w, wfmt, K, n, k);
+    for (int64_t i = 0; i < nm; i++) {
+        int64_t m = rows ? rows[i] : i;
+        for (int64_t k = 0; k < K; k++)
+            arow[k] = elem_qs(codes_a, scales_a, afmt, K, m, k);
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += arow[k] * wrows[n * K + k];
+            out[i * N + n] = acc * (double)ts_a * (double)ts_w;
+        }
+    }
+    free(arow);
+    free(wrows);
+    return 0;
+}
+

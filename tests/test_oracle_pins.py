@@ -361,3 +361,33 @@ def test_zero_and_degenerate(orc):
     assert scales[0, 0] == 0 and codes[0, :8].sum() == 0
     with pytest.raises(ValueError):
         orc.quantize(np.zeros((1, 24), np.float16), 0)
+
+
+@pytest.mark.parametrize("afmt,wfmt", [("act", "weight"), ("nvfp4", "nvfp4"), ("act", "act"), ("weight", "nvfp4")])
+def test_w4a4_ref_matches_numpy(orc, afmt, wfmt):
+    # with power-of-two tensor scales the f32 dequant (pinned above) is exact,
+    # so a numpy float64 matmul of the two dequantized operands is the exact
+    # product up to the summation order; random packed operands reach every
+    # code, every meta value and the subnormal scale codes
+    M, N, K = 9, 21, 96
+    ca, sa = workloads.random_packed(M, K, afmt, seed=71)
+    cw, sw = workloads.random_packed(N, K, wfmt, seed=72)
+    ts_a, ts_w = 0.25, 2.0 ** -7
+    A = orc.dequant(ca.numpy(), sa.numpy(), ts_a, FMT[afmt], "f32").astype(np.float64)
+    W = orc.dequant(cw.numpy(), sw.numpy(), ts_w, FMT[wfmt], "f32").astype(np.float64)
+    ref = A @ W.T
+    got = orc.gemm_w4a4_ref(ca.numpy(), sa.numpy(), ts_a, FMT[afmt], cw.numpy(), sw.numpy(), ts_w, FMT[wfmt])
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    sub = orc.gemm_w4a4_ref(ca.numpy(), sa.numpy(), ts_a, FMT[afmt], cw.numpy(), sw.numpy(), ts_w, FMT[wfmt], rows=[7, 0])
+    np.testing.assert_array_equal(sub, got[[7, 0]])
+    # one non-zero activation picks the weight column: a special code of A
+    # (0b1000 -> its block's v) times W's dequantized column
+    ca2 = np.zeros_like(ca.numpy())
+    ca2[3, 5] = 0x80  # element 11 of row 3: code 0b1000
+    sa2 = np.zeros_like(sa.numpy())
+    sa2[3, 0] = (1 << 7 if afmt == "act" else 0) | 0x38  # meta 1 (-5 for activations), scale 1.0
+    one = orc.gemm_w4a4_ref(ca2, sa2, 1.0, FMT[afmt], cw.numpy(), sw.numpy(), ts_w, FMT[wfmt])
+    v = {"act": -5.0, "nvfp4": 0.0, "weight": None}[afmt]
+    if v is not None:
+        np.testing.assert_array_equal(one[3], v * W[:, 11])
+        assert not one[[i for i in range(M) if i != 3]].any()
