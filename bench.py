@@ -612,6 +612,29 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
         out["gemm"] = res
     except R.RazerError as e:
         out["gemm"] = {"unavailable": str(e)}
+    # W4A4: activations quantized online (E4M3 + 1-bit meta), weights offline;
+    # the call decodes both operands and runs the tcgen05 product
+    try:
+        M, N, K = 4096, 4096, 4096
+        ca, sa, ta, _ = R.razer_quantize_acts(workloads.outlier_activations(M, K, seed=402).to(dev), hist=False)
+        cw, sw, tw = R.razer_quantize_weights(workloads.weight(N, K, seed=403).to(dev))
+        Yw = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        wsw = torch.empty(R.razer_workspace_size(R.RAZER_OP_GEMM_W4A4, M, N, K), dtype=torch.uint8, device=dev)
+        call = lambda: R.razer_gemm_w4a4(ca, sa, ta, cw, sw, tw, "act", "weight", torch.bfloat16, out=Yw, workspace=wsw)
+        for _ in range(3):
+            call()
+        reps = 20
+        e0.record(stream)
+        for _ in range(reps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        tf = 2 * M * N * K / ms / 1e9
+        out["gemm_w4a4"] = {f"{M}x{N}x{K}": {"ms": ms, "TFLOP/s": tf, "frac": tf / bf16,
+                                              "includes": "decode of both operands + tcgen05 product"}}
+    except R.RazerError as e:
+        out["gemm_w4a4"] = {"unavailable": str(e)}
     return out
 
 

@@ -35,6 +35,10 @@ size_t gemv_batch_workspace_bytes(int count, const razer_gemv_problem *P);
 razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
                       razer_format wfmt, int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+razer_status run_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, const float *ts_a, razer_format afmt, int64_t M,
+                           const uint8_t *codes_w, const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K,
+                           void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st);
+size_t gemm_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 static bool valid_fmt(int f) { return f == RAZER_FMT_WEIGHT || f == RAZER_FMT_ACT || f == RAZER_FMT_NVFP4; }
@@ -120,6 +124,7 @@ size_t razer_workspace_size(razer_op op, int64_t M_or_B, int64_t N, int64_t K)
 {
     if (op == RAZER_OP_GEMV) return gemv_workspace_bytes(M_or_B, N, K);
     if (op == RAZER_OP_GEMM) return gemm_workspace_bytes(M_or_B, N, K);
+    if (op == RAZER_OP_GEMM_W4A4) return M_or_B > 0 && N > 0 && K > 0 ? gemm_w4a4_workspace_bytes(M_or_B, N, K) : 0;
     return 0;
 }
 
@@ -194,6 +199,28 @@ razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint
         if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
     }
     return run_gemm(X, act_dt, M, codes, scales, ts, wfmt, N, K, Y, out_dt, workspace, (cudaStream_t)stream);
+}
+
+razer_status razer_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, const float *ts_a, razer_format afmt, int64_t M,
+                             const uint8_t *codes_w, const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N,
+                             int64_t K, void *Y, razer_dtype out_dt, void *workspace, size_t ws_bytes, razer_stream_t stream)
+{
+    if (!ts_a || !ts_w || (!Y && M * N > 0)) return RAZER_ERR_INVALID_ARG;
+    if (!valid_fmt(afmt) || !valid_fmt(wfmt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    razer_status st = check_packed(codes_a, scales_a, M, K);
+    if (st != RAZER_OK) return st;
+    st = check_packed(codes_w, scales_w, N, K);
+    if (st != RAZER_OK) return st;
+    if (K % 64 != 0 || N % 16 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (!aligned(Y, 16) || !aligned(ts_a, 4) || !aligned(ts_w, 4)) return RAZER_ERR_ALIGN;
+    if (M == 0 || N == 0) return RAZER_OK;
+    const size_t need = K > 0 ? gemm_w4a4_workspace_bytes(M, N, K) : 0;
+    if (need) {
+        if (!workspace || ws_bytes < need) return RAZER_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
+    }
+    return run_gemm_w4a4(codes_a, scales_a, ts_a, afmt, M, codes_w, scales_w, ts_w, wfmt, N, K, Y, out_dt, workspace,
+                         (cudaStream_t)stream);
 }
 
 razer_status razer_get_device_status(razer_stream_t stream)

@@ -448,6 +448,14 @@ __global__ void __launch_bounds__(256) decode_weights_kernel(const uint8_t *__re
     }
 }
 
+// ts_a * ts_w (one binary32 rounding) for the epilogue of the W4A4 product
+__global__ void ts_product_kernel(const float *__restrict__ a, const float *__restrict__ b, float *__restrict__ out)
+{
+    pdl_wait();
+    pdl_trigger();
+    *out = __fmul_rn(*a, *b);
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -523,7 +531,88 @@ static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, 
     return RAZER_OK;
 }
 
+// decoded q*s*2^-bias of a packed [R, K] tensor into out (16-bit, [R, K])
+template <bool BF16>
+static razer_status decode_into(razer_format fmt, const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K, void *out,
+                                cudaStream_t st)
+{
+    const int64_t nblk = rows * K / 16;
+    const int64_t g = std::min<int64_t>((nblk + 255) / 256, (int64_t)sm_count() * 8);
+    uint4 *o = reinterpret_cast<uint4 *>(out);
+    cudaError_t e;
+    if (fmt == RAZER_FMT_WEIGHT) e = launch_pdl(decode_weights_kernel<RAZER_FMT_WEIGHT, BF16>, (unsigned)g, 256u, 0, st, codes, scales, nblk, o);
+    else if (fmt == RAZER_FMT_ACT) e = launch_pdl(decode_weights_kernel<RAZER_FMT_ACT, BF16>, (unsigned)g, 256u, 0, st, codes, scales, nblk, o);
+    else e = launch_pdl(decode_weights_kernel<RAZER_FMT_NVFP4, BF16>, (unsigned)g, 256u, 0, st, codes, scales, nblk, o);
+    return e == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
+}
+
+// 2^bias carried by the decoded q*s of a format (E3M3: 2^-8, E4M3: 2^-4)
+static float decode_unbias(razer_format fmt) { return fmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f; }
+
+static size_t w4a4_decoded_a_bytes(int64_t M, int64_t K) { return (size_t)M * (size_t)K * 2; }
+
 }  // namespace gemm
+
+size_t gemm_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    // decoded A [M, K] and W [N, K] (fp16), the fp32 partial sums when K spans
+    // several accumulation chains, then ts_a * ts_w
+    return gemm::w4a4_decoded_a_bytes(M, K) + (size_t)N * (size_t)K * 2 + gemm::partial_bytes(M, N, K) + 16;
+}
+
+// W4A4 product of two RaZeR-packed operands: both decoded exactly to fp16
+// (q*s*2^-bias) and multiplied on the tcgen05 pipeline of the decode-once
+// path; the epilogue applies ts_a * ts_w and both unbias factors.
+razer_status run_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, const float *ts_a, razer_format afmt, int64_t M,
+                           const uint8_t *codes_w, const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K,
+                           void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st)
+{
+    using namespace gemm;
+    if (K == 0) {
+        const size_t esz = out_dt == RAZER_F32 ? 4 : 2;
+        return cudaMemsetAsync(Y, 0, (size_t)M * (size_t)N * esz, st) == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return RAZER_ERR_CUDA;
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    uint8_t *wa = base, *ww = base + w4a4_decoded_a_bytes(M, K);
+    uint8_t *after_w = ww + (size_t)N * (size_t)K * 2;
+    float *partial = partial_bytes(M, N, K) ? reinterpret_cast<float *>(after_w) : nullptr;
+    float *tsp = reinterpret_cast<float *>(after_w + partial_bytes(M, N, K));
+    if (launch_pdl(ts_product_kernel, 1u, 1u, 0, st, ts_a, ts_w, tsp) != cudaSuccess) return RAZER_ERR_CUDA;
+    razer_status r = decode_into<false>(afmt, codes_a, scales_a, M, K, wa, st);
+    if (r != RAZER_OK) return r;
+    r = decode_into<false>(wfmt, codes_w, scales_w, N, K, ww, st);
+    if (r != RAZER_OK) return r;
+    CUtensorMap amap, wmap;
+    const cuuint32_t estr[2] = {1u, 1u};
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)BK, 128u};
+        if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, wa, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return RAZER_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BN};
+        if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ww, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return RAZER_ERR_CUDA;
+    }
+    const float unbias = decode_unbias(afmt) * decode_unbias(wfmt);  // a power of two: exact
+    const int m = (int)M, n = (int)N, k = (int)K, KB = k / BK, nc = (int)num_chunks(K);
+    for (int c = 0; c < nc; c++) {
+        const int kb0 = (int)((int64_t)c * KB / nc), kb1 = (int)((int64_t)(c + 1) * KB / nc);
+        const bool last = c == nc - 1;
+        r = launch<RAZER_FMT_WEIGHT, false, true>(amap, wmap, nullptr, nullptr, tsp, unbias, m, n, k, last ? Y : partial,
+                                                  last ? out_dt : RAZER_F32, kb0, kb1 - kb0, c > 0 ? partial : nullptr, st);
+        if (r != RAZER_OK) return r;
+    }
+    return RAZER_OK;
+}
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {

@@ -24,13 +24,13 @@ STATUS_NAMES = {
 }
 RAZER_F16, RAZER_BF16, RAZER_F32 = 0, 1, 2
 RAZER_FMT_WEIGHT, RAZER_FMT_ACT, RAZER_FMT_NVFP4 = 0, 1, 2
-RAZER_OP_GEMV, RAZER_OP_GEMM = 0, 1
+RAZER_OP_GEMV, RAZER_OP_GEMM, RAZER_OP_GEMM_W4A4 = 0, 1, 2
 FORMATS = {"weight": RAZER_FMT_WEIGHT, "act": RAZER_FMT_ACT, "nvfp4": RAZER_FMT_NVFP4}
 _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZER_F32}
 
 EXPORTED = (
     "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
-    "razer_gemv_batch", "razer_gemv_batch_workspace_size",
+    "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
     "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
 )
@@ -68,6 +68,7 @@ def load() -> ctypes.CDLL:
     L.razer_gemv.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_gemm.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_gemv_batch.argtypes = [i32, ctypes.POINTER(GemvProblem), i32, i32, i32, vp, sz, vp]
+    L.razer_gemm_w4a4.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_gemv_batch_workspace_size.argtypes = [i32, ctypes.POINTER(GemvProblem)]
     L.razer_gemv_batch_workspace_size.restype = sz
     L.razer_gemv_noalloc.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp]
@@ -80,7 +81,7 @@ def load() -> ctypes.CDLL:
     L.razer_status_string.argtypes = [i32]
     L.razer_status_string.restype = ctypes.c_char_p
     L.razer_version.argtypes = []
-    for fn in ("razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    for fn in ("razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -186,6 +187,20 @@ def razer_gemv(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: t
     st = load().razer_gemv(_p(x), _DT.get(x.dtype, -1), B, _p(codes), _p(scales), _p(ts), _fmt(fmt), N, K, _p(out),
                            _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
     _check("razer_gemv", st)
+    return out
+
+
+def razer_gemm_w4a4(codes_a: torch.Tensor, scales_a: torch.Tensor, ts_a: torch.Tensor, codes_w: torch.Tensor,
+                    scales_w: torch.Tensor, ts_w: torch.Tensor, afmt="act", wfmt="weight", out_dtype=torch.bfloat16, *,
+                    out=None, workspace=None, stream=None):
+    """Y [M, N] = ts_a * ts_w * deq(A [M, K]) . deq(W [N, K])^T, both operands RaZeR-packed."""
+    M, N, K = codes_a.shape[0], codes_w.shape[0], codes_w.shape[1] * 2
+    dev = codes_w.device
+    out = torch.empty((M, N), dtype=out_dtype, device=dev) if out is None else out
+    workspace, wsb = _workspace(RAZER_OP_GEMM_W4A4, M, N, K, dev, workspace)
+    st = load().razer_gemm_w4a4(_p(codes_a), _p(scales_a), _p(ts_a), _fmt(afmt), M, _p(codes_w), _p(scales_w), _p(ts_w),
+                                _fmt(wfmt), N, K, _p(out), _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
+    _check("razer_gemm_w4a4", st)
     return out
 
 

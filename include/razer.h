@@ -77,7 +77,7 @@ typedef enum { RAZER_F16 = 0, RAZER_BF16 = 1, RAZER_F32 = 2 } razer_dtype;
 
 typedef enum { RAZER_FMT_WEIGHT = 0, RAZER_FMT_ACT = 1, RAZER_FMT_NVFP4 = 2 } razer_format;
 
-typedef enum { RAZER_OP_GEMV = 0, RAZER_OP_GEMM = 1 } razer_op;
+typedef enum { RAZER_OP_GEMV = 0, RAZER_OP_GEMM = 1, RAZER_OP_GEMM_W4A4 = 2 } razer_op;
 
 /*
  * razer_quantize_weights -- offline weight quantizer (RaZeR notes, 关键设计
@@ -229,6 +229,31 @@ razer_status razer_gemv_batch(int count, const razer_gemv_problem *problems, raz
                               razer_format wfmt, razer_dtype out_dt, void *workspace,
                               size_t ws_bytes, razer_stream_t stream);
 size_t razer_gemv_batch_workspace_size(int count, const razer_gemv_problem *problems);
+
+/*
+ * razer_gemm_w4a4 -- W4A4 product of two RaZeR-packed operands (the
+ * weight-activation kernels of the gist.science summary 2.3; the RaZeR notes,
+ * 局限与展望, note that current Blackwell tensor cores run it only emulated):
+ *   Y[m, n] = ts_a * ts_w * sum_k (q*s)_a[m, k] * (q*s)_w[n, k],  fp32 accumulation.
+ *   codes_a, scales_a, ts_a, afmt   A [M, K] as razer_quantize_acts writes it
+ *                                   (any format; RAZER_FMT_ACT or NVFP4 for activations)
+ *   codes_w, scales_w, ts_w, wfmt   W [N, K] as razer_quantize_weights writes it
+ *   Y          [M, N], out_dt = RAZER_F32, RAZER_F16 or RAZER_BF16
+ *   workspace  razer_workspace_size(RAZER_OP_GEMM_W4A4, M, N, K) bytes
+ *              (16-byte aligned, contents on entry ignored): both operands
+ *              are decoded exactly to fp16 there (q*s*2^-bias is exact in
+ *              fp16 for every code and scale of the three formats), the
+ *              tcgen05 pipeline of razer_gemm multiplies them, and the
+ *              epilogue applies ts_a * ts_w (one fp32 rounding) and the
+ *              bias; K > 16384 runs in chunks as for razer_gemm.
+ * K must be a multiple of 64 and N a multiple of 16.  ts_a and ts_w are
+ * device floats.
+ */
+razer_status razer_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, const float *ts_a,
+                             razer_format afmt, int64_t M, const uint8_t *codes_w,
+                             const uint8_t *scales_w, const float *ts_w, razer_format wfmt,
+                             int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace,
+                             size_t ws_bytes, razer_stream_t stream);
 
 /*
  * razer_gemv_noalloc -- razer_gemv for callers that cannot allocate device

@@ -22,7 +22,7 @@ def lib():
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "razer.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(razer_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(razer_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -83,6 +83,16 @@ def test_gemv_gemm_validation(lib):
     assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 64, 96, FAKE, 1, None, 0, None) == 2   # K % 64
     assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 40, 128, FAKE, 1, None, 0, None) == 2  # N % 16
     assert m(None, 1, 64, FAKE, FAKE, FAKE, 0, 64, 128, FAKE, 1, None, 0, None) == 1
+    w = lib.razer_gemm_w4a4
+    wargs = lambda M, N, K, afmt=1, wfmt=0, ts=FAKE, y=FAKE: (FAKE, FAKE, ts, afmt, M, FAKE, FAKE, FAKE, wfmt, N, K, y, 1, None, 0,
+                                                              None)
+    assert w(*wargs(64, 64, 96)) == 2            # K % 64
+    assert w(*wargs(64, 40, 128)) == 2           # N % 16
+    assert w(*wargs(64, 64, 128, afmt=5)) == 1   # unknown format
+    assert w(*wargs(64, 64, 128, ts=None)) == 1
+    assert w(*wargs(64, 64, 128, y=ODD)) == 3
+    assert w(*wargs(64, 64, 128)) == 5           # workspace missing
+    assert w(*wargs(0, 64, 128)) == 0            # empty product
     d = lib.razer_dequant
     assert d(FAKE, FAKE, FAKE, 3, 4, 32, FAKE, 2, None) == 1
     assert d(FAKE, FAKE, FAKE, 0, 4, 32, FAKE, 5, None) == 1
@@ -113,3 +123,8 @@ def test_workspace_size_host_logic(lib):
     assert razer.razer_workspace_size(G, 1024, 4096, 16384) == 4096 * 16384 * 2
     assert razer.razer_workspace_size(G, 512, 8192, 16448) == 512 * 8192 * 4
     assert razer.razer_workspace_size(G, 2048, 8192, 28672) == 8192 * 28672 * 2 + 2048 * 8192 * 4
+    # W4A4: both decoded operands, the K-chunk partials, 16 bytes for ts_a * ts_w
+    W4 = razer.RAZER_OP_GEMM_W4A4
+    assert razer.razer_workspace_size(W4, 100, 64, 128) == 100 * 128 * 2 + 64 * 128 * 2 + 16
+    assert razer.razer_workspace_size(W4, 100, 64, 16448) == 100 * 16448 * 2 + 64 * 16448 * 2 + 100 * 64 * 4 + 16
+    assert razer.razer_workspace_size(W4, 0, 64, 128) == 0

@@ -140,3 +140,55 @@ def test_gemm_decoded_path_f16_and_garbage_workspace(orc, xdt):
     assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
     # below the threshold no workspace is needed (fused decode)
     assert R.razer_workspace_size(R.RAZER_OP_GEMM, 1023, N, K) == 0
+
+
+# --- W4A4 product of two RaZeR-packed operands ------------------------------
+def w4a4(ca, sa, ts_a, afmt, cw, sw, ts_w, wfmt, out_dtype=torch.float32, workspace=None):
+    t = lambda v: torch.tensor([v], dtype=torch.float32, device=DEV)
+    Y = R.razer_gemm_w4a4(ca.to(DEV), sa.to(DEV), t(ts_a), cw.to(DEV), sw.to(DEV), t(ts_w), afmt, wfmt, out_dtype,
+                          workspace=workspace)
+    torch.cuda.synchronize()
+    return Y
+
+
+@pytest.mark.parametrize("afmt,wfmt", [("act", "weight"), ("nvfp4", "nvfp4"), ("act", "act"), ("weight", "weight")])
+def test_w4a4_random_packed(orc, afmt, wfmt):
+    # ragged M and N over several 256 x 256 tiles, 5 k-steps; random packed
+    # operands reach every code, meta value and subnormal scale code
+    M, N, K = 300, 272, 320
+    ca, sa = workloads.random_packed(M, K, afmt, seed=61, max_scale_code=60)
+    cw, sw = workloads.random_packed(N, K, wfmt, seed=62, max_scale_code=60)
+    ts_a, ts_w = 0.0173, 0.00311
+    ref = orc.gemm_w4a4_ref(ca.numpy(), sa.numpy(), ts_a, FMT_ID[afmt], cw.numpy(), sw.numpy(), ts_w, FMT_ID[wfmt])
+    Y = w4a4(ca, sa, ts_a, afmt, cw, sw, ts_w, wfmt)
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
+    for odt in (torch.float16, torch.bfloat16):
+        assert_close_typed(w4a4(ca, sa, ts_a, afmt, cw, sw, ts_w, wfmt, odt), ref)
+
+
+def test_w4a4_oracle_quantized_pipeline(orc):
+    # activations with outlier channels and weights, both quantized by the
+    # oracle (activations: dynamic ts, E4M3 + 1-bit meta; weights: E3M3 +
+    # 2-bit meta); the GPU product of the packed tensors against the oracle's
+    M, N, K = 384, 512, 1024
+    x = workloads.outlier_activations(M, K, seed=63)
+    w = workloads.weight(N, K, std=0.02, seed=64)
+    ca, sa, ts_a, _ = orc.quantize(oracle_in(x), FMT_ID["act"])
+    cw, sw, ts_w, _ = orc.quantize(w.numpy(), FMT_ID["weight"])
+    ref = orc.gemm_w4a4_ref(ca, sa, ts_a, FMT_ID["act"], cw, sw, ts_w, FMT_ID["weight"])
+    Y = w4a4(torch.from_numpy(ca), torch.from_numpy(sa), ts_a, "act", torch.from_numpy(cw), torch.from_numpy(sw), ts_w, "weight")
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 4096, 4096), (1024, 1024, 28672)])
+def test_w4a4_full_size_sampled(orc, M, N, K):
+    # the prefill shape and a K that runs in two accumulation chains; 24
+    # sampled rows against the oracle, workspace full of garbage
+    ca, sa = workloads.random_packed(M, K, "act", seed=M + 1, max_scale_code=60)
+    cw, sw = workloads.random_packed(N, K, "weight", seed=N + 2, max_scale_code=40)
+    ts_a, ts_w = 0.011, 0.0042
+    ws = torch.full((R.razer_workspace_size(R.RAZER_OP_GEMM_W4A4, M, N, K),), 0xFF, dtype=torch.uint8, device=DEV)
+    Y = w4a4(ca, sa, ts_a, "act", cw, sw, ts_w, "weight", workspace=ws).cpu().numpy()
+    rows = np.random.default_rng(K).choice(M, 24, replace=False)
+    ref = orc.gemm_w4a4_ref(ca.numpy(), sa.numpy(), ts_a, FMT_ID["act"], cw.numpy(), sw.numpy(), ts_w, FMT_ID["weight"], rows=rows)
+    assert rel_err(Y[rows], ref) <= REL_TOL
