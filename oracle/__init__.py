@@ -86,6 +86,9 @@ def lib():
         L.ro_dequant.argtypes = [u8p, u8p, f32, ctypes.c_int, i64, i64, ctypes.c_int, vp]
         L.ro_dequant.restype = ctypes.c_int
         L.ro_gemm_ref.argtypes = [vp, ctypes.c_int, i64, u8p, u8p, f32, ctypes.c_int, i64, i64, vp, i64, vp]
+        L.ro_quantize_46.argtypes = [vp, ctypes.c_int, i64, i64, f32, u8p, u8p, vp]
+        L.ro_quant_sse.argtypes = [vp, ctypes.c_int, i64, i64, u8p, u8p, f32, ctypes.c_int]
+        L.ro_quant_sse.restype = f64
         L.ro_gemm_w4a4_ref.argtypes = [u8p, u8p, f32, ctypes.c_int, i64, u8p, u8p, f32, ctypes.c_int, i64, i64, vp, i64, vp]
         L.ro_gemm_ref.restype = ctypes.c_int
         _lib = L
@@ -240,4 +243,30 @@ def gemm_w4a4_ref(codes_a: np.ndarray, scales_a: np.ndarray, ts_a: float, afmt: 
     if rc != 0:
         raise ValueError("oracle gemm_w4a4_ref failed")
     return out
+
+
+def quantize_46(x, ts: float | None = None):
+    """FourOverSix quantization (plain NVFP4 encoding, per-block choice of
+    the amax -> 6 or amax -> 4 scale). ts None = amax / (6 * 448).
+    Returns (codes, scales, ts, blocks that took 4)."""
+    a, dt = _as_bits(x)
+    R, K = a.shape
+    if ts is None:
+        ts = tensor_scale(x, FMT_NVFP4)
+    codes = np.zeros((R, K // 2), np.uint8)
+    scales = np.zeros((R, K // 16), np.uint8)
+    n4 = np.zeros(1, np.uint64)
+    rc = lib().ro_quantize_46(_ptr(a), dt, R, K, ts, _ptr(codes), _ptr(scales), _ptr(n4))
+    if rc != 0:
+        raise ValueError("oracle quantize_46: K must be a multiple of 16")
+    return codes, scales, float(np.float32(ts)), int(n4[0])
+
+
+def quant_sse(x, codes: np.ndarray, scales: np.ndarray, ts: float, fmt: int) -> float:
+    """sum (x - q*s*ts)^2 over the tensor, in double, row-major order."""
+    a, dt = _as_bits(x)
+    R, K = a.shape
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    return float(lib().ro_quant_sse(_ptr(a), dt, R, K, _ptr(codes), _ptr(scales), ts, fmt))
 

@@ -551,3 +551,108 @@ int ro_gemm_w4a4_ref(const uint8_t *codes_a, const uint8_t *scales_a, float ts_a
     return 0;
 }
 
+/* ---------------------------------------------------------------------- */
+/* Accuracy ablations: FourOverSix and the quantization error.            */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * FourOverSix (Four Over Six summary page, 方法详解: 技术框架 and 关键创新):
+ * plain NVFP4 blocks, but each block may be scaled so that its amax maps to
+ * 4 instead of 6, whichever leaves the smaller error.  Reading R15: for
+ * c in {6, 4}: s_f = amax_b / fp32(c * ts), sc = nearest E4M3 code (R5),
+ * d = fp32(s * ts), codes by plain rounding of x / d (R6, R7, R9); the
+ * block's squared error is sum_j (x_j - q_j * d)^2 in double, each term and
+ * the running sum rounded in element order (q_j * d and x_j - q_j * d are
+ * exact in double).  The 4-candidate wins only with a strictly smaller error.
+ * A block whose scale code is 0 (or d = 0) is all zeros with error sum x^2.
+ * Output: NVFP4 encoding (scale byte = E4M3 code); n_four (may be NULL)
+ * counts the blocks that took 4.
+ */
+static double block_46(const float *x, float ts, float c, uint8_t *codes, int *sc_out)
+{
+    float amax_b = 0.0f;
+    for (int j = 0; j < 16; j++) {
+        float a = fabsf(x[j]);
+        if (a > amax_b)
+            amax_b = a;
+    }
+    float c_ts = c * ts;
+    float s_f = amax_b / c_ts;
+    int sc = ro_scale_encode(RO_FMT_NVFP4, s_f);
+    float d = (float)ro_scale_value(RO_FMT_NVFP4, sc) * ts;
+    double sse = 0.0;
+    *sc_out = sc;
+    if (sc == 0 || d == 0.0f) {
+        memset(codes, 0, 16);
+        *sc_out = 0;
+        for (int j = 0; j < 16; j++)
+            sse += (double)x[j] * (double)x[j];
+        return sse;
+    }
+    for (int j = 0; j < 16; j++) {
+        float xs = x[j] / d;
+        double pt;
+        int code = round_to_grid(xs, 0, 0.0, &pt);
+        if (pt == 0.0)
+            code = 0;
+        codes[j] = (uint8_t)code;
+        double t = (double)x[j] - pt * (double)d;
+        sse += t * t;
+    }
+    return sse;
+}
+
+int ro_quantize_46(const void *x, int dtype, int64_t R, int64_t K, float ts, uint8_t *codes, uint8_t *scales,
+                   uint64_t *n_four)
+{
+    if (K % 16 != 0)
+        return 1;
+    float blk[16];
+    uint8_t c6[16], c4[16];
+    if (n_four)
+        *n_four = 0;
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t b = 0; b < K / 16; b++) {
+            for (int j = 0; j < 16; j++)
+                blk[j] = load_elem(x, dtype, r * K + b * 16 + j);
+            int sc6 = 0, sc4 = 0;
+            const uint8_t *c = c6;
+            int sc = 0;
+            if (ts > 0.0f) { /* R10: ts <= 0 leaves the block zero */
+                double e6 = block_46(blk, ts, 6.0f, c6, &sc6);
+                double e4 = block_46(blk, ts, 4.0f, c4, &sc4);
+                sc = sc6;
+                if (e4 < e6) {
+                    c = c4;
+                    sc = sc4;
+                    if (n_four)
+                        (*n_four)++;
+                }
+            } else {
+                memset(c6, 0, 16);
+            }
+            for (int j = 0; j < 8; j++)
+                codes[r * (K / 2) + b * 8 + j] = (uint8_t)(c[2 * j] | (c[2 * j + 1] << 4));
+            scales[r * (K / 16) + b] = (uint8_t)sc;
+        }
+    return 0;
+}
+
+/*
+ * Quantization error of a packed tensor against its input:
+ * sum over [R, K] (row-major order) of (x - q*s*ts)^2 in double (q*s*ts is
+ * exact in double; each difference, square and running sum rounded).
+ */
+double ro_quant_sse(const void *x, int dtype, int64_t R, int64_t K, const uint8_t *codes, const uint8_t *scales, float ts,
+                    int fmt)
+{
+    double sse = 0.0;
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t k = 0; k < K; k++) {
+            double v = elem_qs(codes, scales, fmt, K, r, k) * (double)ts;
+            double t = (double)load_elem(x, dtype, r * K + k) - v;
+            sse += t * t;
+        }
+    return sse;
+}
+

@@ -391,3 +391,78 @@ def test_w4a4_ref_matches_numpy(orc, afmt, wfmt):
     if v is not None:
         np.testing.assert_array_equal(one[3], v * W[:, 11])
         assert not one[[i for i in range(M) if i != 3]].any()
+
+
+# ----------------------------------------------------------------------------
+# accuracy ablations: FourOverSix and the quantization error
+# ----------------------------------------------------------------------------
+_E2M1_MAGS = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3), Fraction(4), Fraction(6)]
+
+
+def _nearest_e2m1(xs: Fraction) -> tuple[int, Fraction]:
+    # brute force over the 8 magnitudes, ties to the smaller magnitude (R7)
+    a = abs(xs)
+    best = min(range(8), key=lambda c: (abs(a - _E2M1_MAGS[c]), c))
+    q = _E2M1_MAGS[best]
+    code = best | (8 if xs < 0 and q != 0 else 0)
+    return code, (-q if xs < 0 else q)
+
+
+def _block_46_exact(x16: np.ndarray, ts: float, c: float):
+    # library arithmetic for the float32 steps (numpy), torch for the E4M3
+    # rounding, exact rationals for the rounding to the grid and the error
+    amax = np.float32(np.max(np.abs(x16.astype(np.float32))))
+    s_f = np.float32(amax / np.float32(np.float32(c) * np.float32(ts)))
+    sc = int(torch.tensor([float(s_f)], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+    sc = 0x7E if sc >= 0x7F else sc  # saturate
+    s = float(torch.tensor([sc], dtype=torch.uint8).view(torch.float8_e4m3fn).float()[0])
+    d = np.float32(np.float32(s) * np.float32(ts))
+    xf = x16.astype(np.float32)
+    if sc == 0 or d == 0:
+        return [0] * 16, 0, sum(Fraction(float(v)) ** 2 for v in xf)
+    codes, err = [], Fraction(0)
+    for v in xf:
+        xs = np.float32(v / d)
+        code, q = _nearest_e2m1(Fraction(float(xs)))
+        codes.append(code)
+        err += (Fraction(float(v)) - q * Fraction(float(d))) ** 2
+    return codes, sc, err
+
+
+def test_four_over_six_bruteforce(orc):
+    # blocks of varied spread; the exact choice (strictly smaller error takes
+    # 4) against the oracle's double-precision one
+    rng = np.random.default_rng(5)
+    ts = 0.0037
+    n_four = 0
+    for trial in range(300):
+        scale = 10.0 ** rng.uniform(-1, 1)
+        x = (rng.standard_normal(16) * scale * (rng.random(16) ** rng.uniform(0, 3))).astype(np.float16)
+        c6, s6, e6 = _block_46_exact(x, ts, 6.0)
+        c4, s4, e4 = _block_46_exact(x, ts, 4.0)
+        codes, scales, _, n4 = orc.quantize_46(x.reshape(1, 16), ts)
+        got = [(codes[0, j // 2] >> (4 * (j & 1))) & 15 for j in range(16)]
+        exp_codes, exp_sc = (c4, s4) if e4 < e6 else (c6, s6)
+        assert got == exp_codes and int(scales[0, 0]) == exp_sc, trial
+        assert n4 == (1 if e4 < e6 else 0)
+        n_four += n4
+    assert 0 < n_four < 300  # both choices occur
+
+
+def test_quant_sse_and_ablation_invariants(orc):
+    w = workloads.weight(64, 512, std=0.02, seed=31)
+    # with a power-of-two tensor scale the f32 dequant (pinned above) is exact
+    for fmt in (0, 2):
+        codes, scales, _, _ = orc.quantize(w.numpy(), fmt, ts=2.0 ** -12)
+        deq = orc.dequant(codes, scales, 2.0 ** -12, fmt, "f32").astype(np.float64)
+        ref = float(np.sum((w.numpy().astype(np.float64) - deq) ** 2))
+        assert math.isclose(orc.quant_sse(w.numpy(), codes, scales, 2.0 ** -12, fmt), ref, rel_tol=1e-12)
+    # FourOverSix never does worse than plain NVFP4 (it includes its choice),
+    # and the blocks that keep 6 are plain NVFP4 blocks
+    cn, sn, ts, _ = orc.quantize(w.numpy(), 2)
+    c46, s46, ts46, n4 = orc.quantize_46(w.numpy())
+    assert ts46 == ts and n4 > 0
+    assert orc.quant_sse(w.numpy(), c46, s46, ts, 2) < orc.quant_sse(w.numpy(), cn, sn, ts, 2)
+    same = (s46 == sn)
+    blocks6 = np.repeat(same, 8, axis=1)
+    np.testing.assert_array_equal(c46[blocks6], cn[blocks6])
