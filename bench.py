@@ -635,6 +635,23 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
                                               "includes": "decode of both operands + tcgen05 product"}}
     except R.RazerError as e:
         out["gemm_w4a4"] = {"unavailable": str(e)}
+    # accuracy ablation: quantization MSE of RaZeR, plain NVFP4 and
+    # FourOverSix on a decode-shape weight matrix and on outlier activations
+    # (error sums on the GPU, razer_quant_error)
+    abl = {}
+    for name, X, razer_fmt in (("weights_14336x4096_fp16", workloads.weight(14336, 4096, seed=404).to(dev), "weight"),
+                               ("activations_2048x4096_bf16", workloads.outlier_activations(2048, 4096, seed=405).to(dev), "act")):
+        res = {}
+        for fmt, dec in (("nvfp4", "nvfp4"), ("four_over_six", "nvfp4"), (razer_fmt, razer_fmt)):
+            if fmt == "act":
+                c, s, t, _ = R.razer_quantize_acts(X, None, "act", hist=False)
+            else:
+                c, s, t = R.razer_quantize_weights(X, fmt)
+            res[fmt] = float(R.razer_quant_error(X, c, s, t, dec).cpu()[0]) / X.numel()
+        res["razer_over_nvfp4"] = res[razer_fmt] / res["nvfp4"]
+        res["four_over_six_over_nvfp4"] = res["four_over_six"] / res["nvfp4"]
+        abl[name] = res
+    out["accuracy_ablation_mse"] = abl
     return out
 
 

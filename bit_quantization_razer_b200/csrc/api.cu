@@ -22,6 +22,10 @@ razer_status last_launch_status() { return cudaGetLastError() == cudaSuccess ? R
 
 razer_status run_quantize(const void *x, razer_dtype dt, int64_t R, int64_t K, const float *ts_in, uint8_t *codes,
                           uint8_t *scales, float *ts_out, unsigned long long *hist, razer_format fmt, cudaStream_t st);
+razer_status run_quantize_46(const void *x, razer_dtype dt, int64_t R, int64_t K, uint8_t *codes, uint8_t *scales, float *ts_out,
+                             unsigned long long *n_four, cudaStream_t st);
+razer_status run_quant_sse(const void *x, razer_dtype dt, int64_t R, int64_t K, const uint8_t *codes, const uint8_t *scales,
+                           const float *ts, razer_format fmt, double *out, cudaStream_t st);
 razer_status run_quantize_batch(int count, const void *const *W, razer_dtype dt, const int64_t *R, const int64_t *K,
                                 uint8_t *const *codes, uint8_t *const *scales, float *ts, razer_format fmt, cudaStream_t st);
 razer_status run_dequant(const uint8_t *codes, const uint8_t *scales, const float *ts, razer_format fmt, int64_t R, int64_t K,
@@ -65,12 +69,15 @@ razer_status razer_quantize_weights(const void *W, razer_dtype in_dt, int64_t N,
                                     float *tensor_scale, razer_format fmt, razer_stream_t stream)
 {
     if (!tensor_scale || (!W && N * K > 0)) return RAZER_ERR_INVALID_ARG;
-    if (fmt != RAZER_FMT_WEIGHT && fmt != RAZER_FMT_NVFP4) return valid_fmt(fmt) ? RAZER_ERR_UNSUPPORTED : RAZER_ERR_INVALID_ARG;
+    if (fmt != RAZER_FMT_WEIGHT && fmt != RAZER_FMT_NVFP4 && fmt != RAZER_FMT_FOUR_OVER_SIX)
+        return valid_fmt(fmt) ? RAZER_ERR_UNSUPPORTED : RAZER_ERR_INVALID_ARG;
     if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
     if (!in16(in_dt)) return RAZER_ERR_DTYPE;
     razer_status st = check_packed(codes, scales, N, K);
     if (st != RAZER_OK) return st;
     if (!aligned(W, 16) || !aligned(tensor_scale, 4)) return RAZER_ERR_ALIGN;
+    if (fmt == RAZER_FMT_FOUR_OVER_SIX)
+        return run_quantize_46(W, in_dt, N, K, codes, scales, tensor_scale, nullptr, (cudaStream_t)stream);
     return run_quantize(W, in_dt, N, K, nullptr, codes, scales, tensor_scale, nullptr, fmt, (cudaStream_t)stream);
 }
 
@@ -221,6 +228,18 @@ razer_status razer_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, co
     }
     return run_gemm_w4a4(codes_a, scales_a, ts_a, afmt, M, codes_w, scales_w, ts_w, wfmt, N, K, Y, out_dt, workspace,
                          (cudaStream_t)stream);
+}
+
+razer_status razer_quant_error(const void *X, razer_dtype in_dt, int64_t R, int64_t K, const uint8_t *codes, const uint8_t *scales,
+                               const float *ts, razer_format fmt, double *sse, razer_stream_t stream)
+{
+    if (!ts || !sse || (!X && R * K > 0)) return RAZER_ERR_INVALID_ARG;
+    if (!valid_fmt(fmt) || !valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(in_dt)) return RAZER_ERR_DTYPE;
+    razer_status st = check_packed(codes, scales, R, K);
+    if (st != RAZER_OK) return st;
+    if (!aligned(X, 16) || !aligned(ts, 4) || !aligned(sse, 8)) return RAZER_ERR_ALIGN;
+    return run_quant_sse(X, in_dt, R, K, codes, scales, ts, fmt, sse, (cudaStream_t)stream);
 }
 
 razer_status razer_get_device_status(razer_stream_t stream)

@@ -4,6 +4,7 @@
 
 #include "api.cu"
 #include "quantize.cu"
+#include "ablation.cu"
 #include "dequant.cu"
 #include "gemv.cu"
 #include "gemv_tma.cu"

@@ -23,14 +23,14 @@ STATUS_NAMES = {
     7: "RAZER_ERR_TIMEOUT", 8: "RAZER_ERR_CUDA",
 }
 RAZER_F16, RAZER_BF16, RAZER_F32 = 0, 1, 2
-RAZER_FMT_WEIGHT, RAZER_FMT_ACT, RAZER_FMT_NVFP4 = 0, 1, 2
+RAZER_FMT_WEIGHT, RAZER_FMT_ACT, RAZER_FMT_NVFP4, RAZER_FMT_FOUR_OVER_SIX = 0, 1, 2, 3
 RAZER_OP_GEMV, RAZER_OP_GEMM, RAZER_OP_GEMM_W4A4 = 0, 1, 2
-FORMATS = {"weight": RAZER_FMT_WEIGHT, "act": RAZER_FMT_ACT, "nvfp4": RAZER_FMT_NVFP4}
+FORMATS = {"weight": RAZER_FMT_WEIGHT, "act": RAZER_FMT_ACT, "nvfp4": RAZER_FMT_NVFP4, "four_over_six": RAZER_FMT_FOUR_OVER_SIX}
 _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZER_F32}
 
 EXPORTED = (
     "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
-    "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4",
+    "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4", "razer_quant_error",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
     "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
 )
@@ -69,6 +69,7 @@ def load() -> ctypes.CDLL:
     L.razer_gemm.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_gemv_batch.argtypes = [i32, ctypes.POINTER(GemvProblem), i32, i32, i32, vp, sz, vp]
     L.razer_gemm_w4a4.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
+    L.razer_quant_error.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp]
     L.razer_gemv_batch_workspace_size.argtypes = [i32, ctypes.POINTER(GemvProblem)]
     L.razer_gemv_batch_workspace_size.restype = sz
     L.razer_gemv_noalloc.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp]
@@ -81,7 +82,7 @@ def load() -> ctypes.CDLL:
     L.razer_status_string.argtypes = [i32]
     L.razer_status_string.restype = ctypes.c_char_p
     L.razer_version.argtypes = []
-    for fn in ("razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    for fn in ("razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -201,6 +202,17 @@ def razer_gemm_w4a4(codes_a: torch.Tensor, scales_a: torch.Tensor, ts_a: torch.T
     st = load().razer_gemm_w4a4(_p(codes_a), _p(scales_a), _p(ts_a), _fmt(afmt), M, _p(codes_w), _p(scales_w), _p(ts_w),
                                 _fmt(wfmt), N, K, _p(out), _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
     _check("razer_gemm_w4a4", st)
+    return out
+
+
+def razer_quant_error(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight", *,
+                      out=None, stream=None) -> torch.Tensor:
+    """sum (X - deq(X))^2 over the tensor in double (device [1] f64)."""
+    R, K = X.shape
+    out = torch.empty(1, dtype=torch.float64, device=X.device) if out is None else out
+    st = load().razer_quant_error(_p(X), _DT.get(X.dtype, -1), R, K, _p(codes), _p(scales), _p(ts), _fmt(fmt), _p(out),
+                                  _stream(stream))
+    _check("razer_quant_error", st)
     return out
 
 

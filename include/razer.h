@@ -75,7 +75,17 @@ typedef enum {
 
 typedef enum { RAZER_F16 = 0, RAZER_BF16 = 1, RAZER_F32 = 2 } razer_dtype;
 
-typedef enum { RAZER_FMT_WEIGHT = 0, RAZER_FMT_ACT = 1, RAZER_FMT_NVFP4 = 2 } razer_format;
+typedef enum {
+    RAZER_FMT_WEIGHT = 0,
+    RAZER_FMT_ACT = 1,
+    RAZER_FMT_NVFP4 = 2,
+    /* razer_quantize_weights only (accuracy ablation): FourOverSix -- NVFP4
+     * encoding (decode it as RAZER_FMT_NVFP4), but each block is scaled so
+     * that its amax maps to 6 or to 4, whichever leaves the smaller squared
+     * error sum_j (x_j - q_j*d)^2 (double, element order; ties take 6).
+     * Four Over Six summary page, 方法详解. */
+    RAZER_FMT_FOUR_OVER_SIX = 3
+} razer_format;
 
 typedef enum { RAZER_OP_GEMV = 0, RAZER_OP_GEMM = 1, RAZER_OP_GEMM_W4A4 = 2 } razer_op;
 
@@ -254,6 +264,19 @@ razer_status razer_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, co
                              const uint8_t *scales_w, const float *ts_w, razer_format wfmt,
                              int64_t N, int64_t K, void *Y, razer_dtype out_dt, void *workspace,
                              size_t ws_bytes, razer_stream_t stream);
+
+/*
+ * razer_quant_error -- quantization error of a packed tensor (accuracy
+ * ablations): *sse = sum over [R, K] of (X - q*s*ts)^2 in double (q*s*ts is
+ * exact in double).  X is the tensor that was quantized (RAZER_F16 or
+ * RAZER_BF16), codes/scales/ts its packed form in format fmt (a tensor
+ * quantized with RAZER_FMT_FOUR_OVER_SIX is decoded as RAZER_FMT_NVFP4).  sse
+ * is a device double, overwritten; partial sums meet in atomic adds, so its
+ * last bits depend on the order the thread blocks finish in.
+ */
+razer_status razer_quant_error(const void *X, razer_dtype in_dt, int64_t R, int64_t K,
+                               const uint8_t *codes, const uint8_t *scales, const float *ts,
+                               razer_format fmt, double *sse, razer_stream_t stream);
 
 /*
  * razer_gemv_noalloc -- razer_gemv for callers that cannot allocate device
