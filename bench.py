@@ -631,8 +631,24 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / reps
         tf = 2 * M * N * K / ms / 1e9
-        out["gemm_w4a4"] = {f"{M}x{N}x{K}": {"ms": ms, "TFLOP/s": tf, "frac": tf / bf16,
-                                              "includes": "decode of both operands + tcgen05 product"}}
+        res = {f"{M}x{N}x{K}": {"ms": ms, "TFLOP/s": tf, "frac": tf / bf16, "includes": "decode of both operands + tcgen05 product"}}
+        # the online path from bf16 activations: quantize (dynamic ts) + product
+        Xa = workloads.outlier_activations(M, K, seed=402).to(dev)
+        online = lambda: R.razer_gemm_w4a4_online(Xa, cw, sw, tw, None, "act", "weight", torch.bfloat16, out=Yw, workspace=wsw)
+        two = lambda: (R.razer_quantize_acts(Xa, None, "act", codes=ca, scales=sa, ts_out=ta, hist=False),
+                       R.razer_gemm_w4a4(ca, sa, ta, cw, sw, tw, "act", "weight", torch.bfloat16, out=Yw, workspace=wsw))
+        for name, fn in (("online_fused", online), ("online_two_calls", two)):
+            for _ in range(3):
+                fn()
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            msn = e0.elapsed_time(e1) / reps
+            res[f"{M}x{N}x{K}_{name}"] = {"ms": msn, "TFLOP/s": 2 * M * N * K / msn / 1e9,
+                                           "includes": "activation quantization (dynamic ts) + decode + product"}
+        out["gemm_w4a4"] = res
     except R.RazerError as e:
         out["gemm_w4a4"] = {"unavailable": str(e)}
     # accuracy ablation: quantization MSE of RaZeR, plain NVFP4 and

@@ -43,6 +43,10 @@ razer_status run_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, cons
                            const uint8_t *codes_w, const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K,
                            void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st);
 size_t gemm_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+razer_status run_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, const float *ts_in, razer_format afmt, uint8_t *codes_a,
+                                  uint8_t *scales_a, float *ts_a_out, unsigned long long *hist, const uint8_t *codes_w,
+                                  const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K, void *Y,
+                                  razer_dtype out_dt, void *workspace, cudaStream_t st);
 
 static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 static bool valid_fmt(int f) { return f == RAZER_FMT_WEIGHT || f == RAZER_FMT_ACT || f == RAZER_FMT_NVFP4; }
@@ -228,6 +232,34 @@ razer_status razer_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, co
     }
     return run_gemm_w4a4(codes_a, scales_a, ts_a, afmt, M, codes_w, scales_w, ts_w, wfmt, N, K, Y, out_dt, workspace,
                          (cudaStream_t)stream);
+}
+
+razer_status razer_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, const float *ts_in, razer_format afmt,
+                                    uint8_t *codes_a, uint8_t *scales_a, float *ts_a_out, unsigned long long *meta_hist,
+                                    const uint8_t *codes_w, const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N,
+                                    int64_t K, void *Y, razer_dtype out_dt, void *workspace, size_t ws_bytes, razer_stream_t stream)
+{
+    if (!ts_a_out || !ts_w || (!X && M * K > 0) || (!Y && M * N > 0)) return RAZER_ERR_INVALID_ARG;
+    if (afmt != RAZER_FMT_ACT && afmt != RAZER_FMT_NVFP4) return valid_fmt(afmt) ? RAZER_ERR_UNSUPPORTED : RAZER_ERR_INVALID_ARG;
+    if (!valid_fmt(wfmt) || !valid_dt(x_dt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(x_dt)) return RAZER_ERR_DTYPE;
+    if ((codes_a == nullptr) != (scales_a == nullptr)) return RAZER_ERR_INVALID_ARG;
+    razer_status st = codes_a ? check_packed(codes_a, scales_a, M, K) : RAZER_OK;
+    if (st != RAZER_OK) return st;
+    st = check_packed(codes_w, scales_w, N, K);
+    if (st != RAZER_OK) return st;
+    if (M < 0 || K % 64 != 0 || N % 16 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ts_a_out, 4) || !aligned(ts_w, 4) || (ts_in && !aligned(ts_in, 4)) ||
+        (meta_hist && !aligned(meta_hist, 8)))
+        return RAZER_ERR_ALIGN;
+    if (M == 0 || N == 0) return RAZER_OK;
+    const size_t need = K > 0 ? gemm_w4a4_workspace_bytes(M, N, K) : 0;
+    if (need) {
+        if (!workspace || ws_bytes < need) return RAZER_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
+    }
+    return run_gemm_w4a4_online(X, x_dt, M, ts_in, afmt, codes_a, scales_a, ts_a_out, meta_hist, codes_w, scales_w, ts_w, wfmt, N, K, Y,
+                                out_dt, workspace, (cudaStream_t)stream);
 }
 
 razer_status razer_quant_error(const void *X, razer_dtype in_dt, int64_t R, int64_t K, const uint8_t *codes, const uint8_t *scales,

@@ -448,6 +448,75 @@ __global__ void __launch_bounds__(256) decode_weights_kernel(const uint8_t *__re
     }
 }
 
+// Online activation quantizer that also writes the decoded operand of the
+// W4A4 product: each block goes through the same block quantizer as
+// razer_quantize_acts (codes and scale byte, stored only when the caller asks
+// for them) and its codes are decoded at once to q*s*2^-bias in fp16 (exact),
+// so the activations are read once and the product needs no separate decode.
+template <int FMT, typename TIn, bool FAST, bool HIST>
+__device__ __forceinline__ void quantize_decode_loop(const TIn *__restrict__ x, int64_t nblk, const ScaleCtx &k, uint8_t *__restrict__ codes,
+                                                     uint8_t *__restrict__ scales, uint4 *__restrict__ dec, unsigned (&cnt)[4])
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const uint4 *p = reinterpret_cast<const uint4 *>(x);
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+        const uint4 v0 = ldg_stream(p + 2 * b), v1 = ldg_stream(p + 2 * b + 1);
+        const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float xv[16];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float2 f = In16<TIn>::to_f2(wv[i]);
+            xv[2 * i] = f.x;
+            xv[2 * i + 1] = f.y;
+        }
+        const BlockOut o = quantize_block<FMT, FAST, std::is_same<TIn, __half>::value>(xv, k);
+        if (codes) reinterpret_cast<uint2 *>(codes)[b] = o.packed;
+        if (scales) scales[b] = (uint8_t)o.sbyte;
+        const BlockK kc = block_consts<FMT>(o.sbyte);
+        dec[2 * b] = decode_word<FMT, false>(o.packed.x, kc);
+        dec[2 * b + 1] = decode_word<FMT, false>(o.packed.y, kc);
+        if constexpr (HIST) {
+            const unsigned m1 = o.meta & 1u, e = o.effective ? 1u : 0u;
+            cnt[0] += 1u - m1;
+            cnt[1] += m1;
+            cnt[2] += e & (1u - m1);
+            cnt[3] += e & m1;
+        }
+    }
+}
+
+template <int FMT, typename TIn, bool HIST>
+__global__ void __launch_bounds__(256) quantize_decode_kernel(const TIn *__restrict__ x, int64_t nblk, const float *__restrict__ ts_src,
+                                                             int ts_is_amax, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                                                             unsigned long long *__restrict__ hist, uint4 *__restrict__ dec)
+{
+    using F = Fmt<FMT>;
+    pdl_wait();
+    pdl_trigger();
+    const float tv = *ts_src;
+    const float ts = ts_is_amax ? __fdiv_rn(tv, F::kC) : tv;
+    __shared__ float tab_d[F::kMagMask + 1], tab_y[F::kMagMask + 1];
+    const ScaleCtx k = make_ctx<FMT>(ts, tab_d, tab_y);
+    __syncthreads();
+    unsigned cnt[4] = {0u, 0u, 0u, 0u};
+    if (fast_ts(ts)) quantize_decode_loop<FMT, TIn, true, HIST>(x, nblk, k, codes, scales, dec, cnt);
+    else quantize_decode_loop<FMT, TIn, false, HIST>(x, nblk, k, codes, scales, dec, cnt);
+    if constexpr (HIST) {
+        __shared__ unsigned long long sh[4];
+        if (threadIdx.x < 4) sh[threadIdx.x] = 0ull;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            unsigned c = cnt[i];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+            if ((threadIdx.x & 31) == 0 && c) atomicAdd(&sh[i], (unsigned long long)c);
+        }
+        __syncthreads();
+        if (threadIdx.x < 4 && sh[threadIdx.x]) atomicAdd(&hist[threadIdx.x], sh[threadIdx.x]);
+    }
+}
+
 // ts_a * ts_w (one binary32 rounding) for the epilogue of the W4A4 product
 __global__ void ts_product_kernel(const float *__restrict__ a, const float *__restrict__ b, float *__restrict__ out)
 {
@@ -563,15 +632,14 @@ size_t gemm_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K)
 // W4A4 product of two RaZeR-packed operands: both decoded exactly to fp16
 // (q*s*2^-bias) and multiplied on the tcgen05 pipeline of the decode-once
 // path; the epilogue applies ts_a * ts_w and both unbias factors.
-razer_status run_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, const float *ts_a, razer_format afmt, int64_t M,
-                           const uint8_t *codes_w, const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K,
-                           void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st)
+// The product half of the W4A4 path: the decoded A (fp16) sits at the start
+// of the workspace, written earlier on the stream; ts_a is the activations'
+// tensor scale (device).
+static razer_status w4a4_product(const float *ts_a, razer_format afmt, int64_t M, const uint8_t *codes_w,
+                                 const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K, void *Y,
+                                 razer_dtype out_dt, void *workspace, cudaStream_t st)
 {
     using namespace gemm;
-    if (K == 0) {
-        const size_t esz = out_dt == RAZER_F32 ? 4 : 2;
-        return cudaMemsetAsync(Y, 0, (size_t)M * (size_t)N * esz, st) == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
-    }
     EncodeTiledFn enc = encode_fn();
     if (!enc) return RAZER_ERR_CUDA;
     uint8_t *base = static_cast<uint8_t *>(workspace);
@@ -580,9 +648,7 @@ razer_status run_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, cons
     float *partial = partial_bytes(M, N, K) ? reinterpret_cast<float *>(after_w) : nullptr;
     float *tsp = reinterpret_cast<float *>(after_w + partial_bytes(M, N, K));
     if (launch_pdl(ts_product_kernel, 1u, 1u, 0, st, ts_a, ts_w, tsp) != cudaSuccess) return RAZER_ERR_CUDA;
-    razer_status r = decode_into<false>(afmt, codes_a, scales_a, M, K, wa, st);
-    if (r != RAZER_OK) return r;
-    r = decode_into<false>(wfmt, codes_w, scales_w, N, K, ww, st);
+    razer_status r = decode_into<false>(wfmt, codes_w, scales_w, N, K, ww, st);
     if (r != RAZER_OK) return r;
     CUtensorMap amap, wmap;
     const cuuint32_t estr[2] = {1u, 1u};
@@ -612,6 +678,89 @@ razer_status run_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, cons
         if (r != RAZER_OK) return r;
     }
     return RAZER_OK;
+}
+
+// W4A4 product of two RaZeR-packed operands: both decoded exactly to fp16
+// (q*s*2^-bias) and multiplied on the tcgen05 pipeline of the decode-once
+// path; the epilogue applies ts_a * ts_w and both unbias factors.
+razer_status run_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, const float *ts_a, razer_format afmt, int64_t M,
+                           const uint8_t *codes_w, const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K,
+                           void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st)
+{
+    using namespace gemm;
+    if (K == 0) {
+        const size_t esz = out_dt == RAZER_F32 ? 4 : 2;
+        return cudaMemsetAsync(Y, 0, (size_t)M * (size_t)N * esz, st) == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
+    }
+    uint8_t *wa = static_cast<uint8_t *>(workspace);
+    const razer_status r = decode_into<false>(afmt, codes_a, scales_a, M, K, wa, st);
+    if (r != RAZER_OK) return r;
+    return w4a4_product(ts_a, afmt, M, codes_w, scales_w, ts_w, wfmt, N, K, Y, out_dt, workspace, st);
+}
+
+// Online W4A4: the activations X are quantized (dynamic tensor scale when
+// ts_in is NULL, as razer_quantize_acts) by the fused quantize + decode
+// kernel, then multiplied as in run_gemm_w4a4.  codes_a / scales_a / hist may
+// be NULL; ts_a_out receives the activations' tensor scale.
+template <int FMT, typename TIn>
+static razer_status quantize_decode_t(const void *X, int64_t nblk, const float *ts_src, int is_amax, uint8_t *codes, uint8_t *scales,
+                                      unsigned long long *hist, void *dec, cudaStream_t st)
+{
+    const unsigned grid = (unsigned)std::min<int64_t>((nblk + 255) / 256, (int64_t)sm_count() * 8);
+    cudaError_t e;
+    if (hist && Fmt<FMT>::kSpecials > 0)
+        e = launch_pdl(gemm::quantize_decode_kernel<FMT, TIn, true>, grid, 256u, 0, st, reinterpret_cast<const TIn *>(X), nblk, ts_src,
+                       is_amax, codes, scales, hist, reinterpret_cast<uint4 *>(dec));
+    else
+        e = launch_pdl(gemm::quantize_decode_kernel<FMT, TIn, false>, grid, 256u, 0, st, reinterpret_cast<const TIn *>(X), nblk, ts_src,
+                       is_amax, codes, scales, (unsigned long long *)nullptr, reinterpret_cast<uint4 *>(dec));
+    return e == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
+}
+
+razer_status run_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, const float *ts_in, razer_format afmt, uint8_t *codes_a,
+                                  uint8_t *scales_a, float *ts_a_out, unsigned long long *hist, const uint8_t *codes_w,
+                                  const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K, void *Y,
+                                  razer_dtype out_dt, void *workspace, cudaStream_t st)
+{
+    const int64_t n = M * K, nblk = n / 16;
+    const float C = afmt == RAZER_FMT_WEIGHT ? Fmt<RAZER_FMT_WEIGHT>::kC : Fmt<RAZER_FMT_ACT>::kC;
+    if (hist || !ts_in) {
+        if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, hist, ts_in ? (unsigned *)nullptr : reinterpret_cast<unsigned *>(ts_a_out)) !=
+            cudaSuccess)
+            return RAZER_ERR_CUDA;
+    }
+    const float *ts_src = ts_in;
+    int is_amax = 0;
+    if (!ts_in) {
+        if (n > 0) {
+            if (x_dt == RAZER_F16) launch_amax<__half>(X, n, reinterpret_cast<unsigned *>(ts_a_out), st);
+            else launch_amax<__nv_bfloat16>(X, n, reinterpret_cast<unsigned *>(ts_a_out), st);
+        }
+        ts_src = ts_a_out;
+        is_amax = 1;
+    }
+    uint8_t *wa = static_cast<uint8_t *>(workspace);
+    if (nblk > 0) {
+        const bool h = x_dt == RAZER_F16;
+        razer_status r;
+        if (afmt == RAZER_FMT_ACT)
+            r = h ? quantize_decode_t<RAZER_FMT_ACT, __half>(X, nblk, ts_src, is_amax, codes_a, scales_a, hist, wa, st)
+                  : quantize_decode_t<RAZER_FMT_ACT, __nv_bfloat16>(X, nblk, ts_src, is_amax, codes_a, scales_a, hist, wa, st);
+        else
+            r = h ? quantize_decode_t<RAZER_FMT_NVFP4, __half>(X, nblk, ts_src, is_amax, codes_a, scales_a, hist, wa, st)
+                  : quantize_decode_t<RAZER_FMT_NVFP4, __nv_bfloat16>(X, nblk, ts_src, is_amax, codes_a, scales_a, hist, wa, st);
+        if (r != RAZER_OK) return r;
+    }
+    if (!ts_in) {
+        if (launch_pdl(finalize_ts_kernel, 1u, 1u, 0, st, ts_a_out, C) != cudaSuccess) return RAZER_ERR_CUDA;
+    } else if (ts_a_out != ts_in) {
+        if (launch_pdl(copy_ts_kernel, 1u, 1u, 0, st, ts_in, ts_a_out) != cudaSuccess) return RAZER_ERR_CUDA;
+    }
+    if (K == 0) {
+        const size_t esz = out_dt == RAZER_F32 ? 4 : 2;
+        return cudaMemsetAsync(Y, 0, (size_t)M * (size_t)N * esz, st) == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
+    }
+    return w4a4_product(ts_a_out, afmt, M, codes_w, scales_w, ts_w, wfmt, N, K, Y, out_dt, workspace, st);
 }
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)

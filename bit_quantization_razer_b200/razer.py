@@ -30,7 +30,7 @@ _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZE
 
 EXPORTED = (
     "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
-    "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4", "razer_quant_error",
+    "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4", "razer_gemm_w4a4_online", "razer_quant_error",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
     "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
 )
@@ -69,6 +69,7 @@ def load() -> ctypes.CDLL:
     L.razer_gemm.argtypes = [vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_gemv_batch.argtypes = [i32, ctypes.POINTER(GemvProblem), i32, i32, i32, vp, sz, vp]
     L.razer_gemm_w4a4.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
+    L.razer_gemm_w4a4_online.argtypes = [vp, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_quant_error.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp]
     L.razer_gemv_batch_workspace_size.argtypes = [i32, ctypes.POINTER(GemvProblem)]
     L.razer_gemv_batch_workspace_size.restype = sz
@@ -82,7 +83,7 @@ def load() -> ctypes.CDLL:
     L.razer_status_string.argtypes = [i32]
     L.razer_status_string.restype = ctypes.c_char_p
     L.razer_version.argtypes = []
-    for fn in ("razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    for fn in ("razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -203,6 +204,27 @@ def razer_gemm_w4a4(codes_a: torch.Tensor, scales_a: torch.Tensor, ts_a: torch.T
                                 _fmt(wfmt), N, K, _p(out), _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
     _check("razer_gemm_w4a4", st)
     return out
+
+
+def razer_gemm_w4a4_online(X: torch.Tensor, codes_w: torch.Tensor, scales_w: torch.Tensor, ts_w: torch.Tensor,
+                           ts_in: torch.Tensor | None = None, afmt="act", wfmt="weight", out_dtype=torch.bfloat16, *,
+                           keep_codes: bool = False, hist: bool = False, out=None, workspace=None, stream=None):
+    """Quantize activations X [M, K] and multiply with the packed weights W [N, K]
+    in one call. Returns (Y [M, N], ts_a [1], (codes_a, scales_a) or None, meta_hist or None)."""
+    M, K = X.shape
+    N = codes_w.shape[0]
+    dev = X.device
+    out = torch.empty((M, N), dtype=out_dtype, device=dev) if out is None else out
+    ts_a = torch.empty(1, dtype=torch.float32, device=dev)
+    ca = torch.empty((M, K // 2), dtype=torch.uint8, device=dev) if keep_codes else None
+    sa = torch.empty((M, K // 16), dtype=torch.uint8, device=dev) if keep_codes else None
+    mh = torch.empty(4, dtype=torch.int64, device=dev) if hist else None
+    workspace, wsb = _workspace(RAZER_OP_GEMM_W4A4, M, N, K, dev, workspace)
+    st = load().razer_gemm_w4a4_online(_p(X), _DT.get(X.dtype, -1), M, _p(ts_in), _fmt(afmt), _p(ca), _p(sa), _p(ts_a), _p(mh),
+                                       _p(codes_w), _p(scales_w), _p(ts_w), _fmt(wfmt), N, K, _p(out), _DT.get(out.dtype, -1),
+                                       _p(workspace), wsb, _stream(stream))
+    _check("razer_gemm_w4a4_online", st)
+    return out, ts_a, ((ca, sa) if keep_codes else None), mh
 
 
 def razer_quant_error(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight", *,

@@ -266,6 +266,29 @@ razer_status razer_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, co
                              size_t ws_bytes, razer_stream_t stream);
 
 /*
+ * razer_gemm_w4a4_online -- the online W4A4 path in one call: quantize the
+ * activations X [M, K] (fp16/bf16) as razer_quantize_acts does (ts_in = NULL:
+ * dynamic tensor scale; otherwise the given device scale) and multiply them
+ * with the packed weights as razer_gemm_w4a4 does.  The activation quantizer
+ * writes the decoded operand of the product directly (one pass over X; the
+ * codes are not read back), so
+ *   Y == razer_gemm_w4a4(razer_quantize_acts(X), W)   bit for bit.
+ *   afmt            RAZER_FMT_ACT or RAZER_FMT_NVFP4
+ *   codes_a, scales_a  optional outputs ([M, K/2], [M, K/16]); both NULL or
+ *                   both set
+ *   ts_a_out        device float, output: the activations' tensor scale
+ *   meta_hist       optional, as for razer_quantize_acts
+ *   W, Y, workspace as razer_gemm_w4a4 (razer_workspace_size(RAZER_OP_GEMM_W4A4, M, N, K))
+ */
+razer_status razer_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, const float *ts_in,
+                                    razer_format afmt, uint8_t *codes_a, uint8_t *scales_a,
+                                    float *ts_a_out, unsigned long long *meta_hist,
+                                    const uint8_t *codes_w, const uint8_t *scales_w,
+                                    const float *ts_w, razer_format wfmt, int64_t N, int64_t K,
+                                    void *Y, razer_dtype out_dt, void *workspace, size_t ws_bytes,
+                                    razer_stream_t stream);
+
+/*
  * razer_quant_error -- quantization error of a packed tensor (accuracy
  * ablations): *sse = sum over [R, K] of (X - q*s*ts)^2 in double (q*s*ts is
  * exact in double).  X is the tensor that was quantized (RAZER_F16 or

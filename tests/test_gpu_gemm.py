@@ -192,3 +192,47 @@ def test_w4a4_full_size_sampled(orc, M, N, K):
     rows = np.random.default_rng(K).choice(M, 24, replace=False)
     ref = orc.gemm_w4a4_ref(ca.numpy(), sa.numpy(), ts_a, FMT_ID["act"], cw.numpy(), sw.numpy(), ts_w, FMT_ID["weight"], rows=rows)
     assert rel_err(Y[rows], ref) <= REL_TOL
+
+
+@pytest.mark.parametrize("afmt", ["act", "nvfp4"])
+@pytest.mark.parametrize("xdt", [torch.bfloat16, torch.float16])
+def test_w4a4_online_equals_two_calls(orc, afmt, xdt):
+    # the fused quantize + decode path gives bit for bit what
+    # razer_quantize_acts followed by razer_gemm_w4a4 gives (dynamic ts, meta
+    # histogram, codes kept); both against the oracle's product of the
+    # oracle-quantized activations
+    M, N, K = 300, 272, 512
+    x = workloads.outlier_activations(M, K, seed=90, dtype=xdt)
+    cw, sw = workloads.random_packed(N, K, "weight", seed=91, max_scale_code=40)
+    xd, cwd, swd = x.to(DEV), cw.to(DEV), sw.to(DEV)
+    tw = torch.tensor([0.0043], dtype=torch.float32, device=DEV)
+    Y1, ts_a, kept, mh = R.razer_gemm_w4a4_online(xd, cwd, swd, tw, None, afmt, "weight", torch.float32, keep_codes=True,
+                                                  hist=afmt == "act")
+    ca, sa, t2, h2 = R.razer_quantize_acts(xd, None, afmt, hist=afmt == "act")
+    Y2 = R.razer_gemm_w4a4(ca, sa, t2, cwd, swd, tw, afmt, "weight", torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2) and torch.equal(ts_a, t2)
+    assert torch.equal(kept[0], ca) and torch.equal(kept[1], sa)
+    if afmt == "act":
+        assert torch.equal(mh, h2)
+    oca, osa, ots, _ = orc.quantize(oracle_in(x), FMT_ID[afmt])
+    assert float(ts_a.cpu()[0]) == ots
+    ref = orc.gemm_w4a4_ref(oca, osa, ots, FMT_ID[afmt], cw.numpy(), sw.numpy(), 0.0043, FMT_ID["weight"])
+    assert rel_err(Y1.cpu().numpy(), ref) <= REL_TOL
+
+
+def test_w4a4_online_static_scale(orc):
+    # a given activation scale (no amax pass); no codes kept, bf16 output
+    M, N, K = 256, 256, 1024
+    x = workloads.outlier_activations(M, K, seed=92)
+    w = workloads.weight(N, K, seed=93)
+    cw, sw, tw, _ = orc.quantize(w.numpy(), FMT_ID["weight"])
+    ts_in = 0.0371
+    oca, osa, _, _ = orc.quantize(oracle_in(x), FMT_ID["act"], ts=ts_in)
+    ref = orc.gemm_w4a4_ref(oca, osa, ts_in, FMT_ID["act"], cw, sw, tw, FMT_ID["weight"])
+    Y, ts_a, kept, _ = R.razer_gemm_w4a4_online(x.to(DEV), torch.from_numpy(cw).to(DEV), torch.from_numpy(sw).to(DEV),
+                                                torch.tensor([tw], dtype=torch.float32, device=DEV),
+                                                torch.tensor([ts_in], dtype=torch.float32, device=DEV), "act", "weight", torch.bfloat16)
+    torch.cuda.synchronize()
+    assert kept is None and float(ts_a.cpu()[0]) == np.float32(ts_in)
+    assert_close_typed(Y, ref)
