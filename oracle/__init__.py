@@ -89,6 +89,9 @@ def lib():
         L.ro_quantize_46.argtypes = [vp, ctypes.c_int, i64, i64, f32, u8p, u8p, vp]
         L.ro_quant_sse.argtypes = [vp, ctypes.c_int, i64, i64, u8p, u8p, f32, ctypes.c_int]
         L.ro_quant_sse.restype = f64
+        L.ro_quantize_generic.argtypes = [vp, ctypes.c_int, i64, i64, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, f32, u8p, u8p]
+        L.ro_quant_sse_generic.argtypes = [vp, ctypes.c_int, i64, i64, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, u8p, u8p, f32]
+        L.ro_quant_sse_generic.restype = f64
         L.ro_gemm_w4a4_ref.argtypes = [u8p, u8p, f32, ctypes.c_int, i64, u8p, u8p, f32, ctypes.c_int, i64, i64, vp, i64, vp]
         L.ro_gemm_ref.restype = ctypes.c_int
         _lib = L
@@ -269,4 +272,29 @@ def quant_sse(x, codes: np.ndarray, scales: np.ndarray, ts: float, fmt: int) -> 
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     return float(lib().ro_quant_sse(_ptr(a), dt, R, K, _ptr(codes), _ptr(scales), ts, fmt))
+
+
+def quantize_generic(x, block: int, sfmt: int, V, ts: float | None = None):
+    """RaZeR quantization with a block of `block` elements and special values
+    V (scale format sfmt: 0 = E3M3 + 2 meta bits, 1/2 = E4M3 + 1 meta bit).
+    ts None = amax / (6 * S_max(sfmt)). Returns (codes, scales [R, K/block], ts)."""
+    a, dt = _as_bits(x)
+    R, K = a.shape
+    if ts is None:
+        ts = tensor_scale(x, sfmt)
+    v = np.ascontiguousarray(np.asarray(V, dtype=np.float64).reshape(-1))
+    codes = np.zeros((R, K // 2), np.uint8)
+    scales = np.zeros((R, K // block), np.uint8)
+    rc = lib().ro_quantize_generic(_ptr(a), dt, R, K, block, sfmt, _ptr(v) if v.size else None, v.size, ts, _ptr(codes), _ptr(scales))
+    if rc != 0:
+        raise ValueError("oracle quantize_generic: bad block size")
+    return codes, scales, float(np.float32(ts))
+
+
+def quant_sse_generic(x, block: int, sfmt: int, V, codes: np.ndarray, scales: np.ndarray, ts: float) -> float:
+    a, dt = _as_bits(x)
+    R, K = a.shape
+    v = np.ascontiguousarray(np.asarray(V, dtype=np.float64).reshape(-1))
+    return float(lib().ro_quant_sse_generic(_ptr(a), dt, R, K, block, sfmt, _ptr(v) if v.size else None, v.size,
+                                            _ptr(np.ascontiguousarray(codes)), _ptr(np.ascontiguousarray(scales)), ts))
 

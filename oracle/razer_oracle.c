@@ -656,3 +656,103 @@ double ro_quant_sse(const void *x, int dtype, int64_t R, int64_t K, const uint8_
     return sse;
 }
 
+/* ---------------------------------------------------------------------- */
+/* Format variants (block size, special-value set) for accuracy studies.  */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * The RaZeR quantizer with a block of bs elements (16, 32, 64 or 128; the
+ * RaZeR notes, 主实验, report the block-size study) and a special-value set
+ * V[0..nv) given by the caller (multiples of 0.5 in [2.5, 9.5], the
+ * constraint of the gist.science summary 2.2).  Scale format sfmt:
+ * RO_FMT_WEIGHT (E3M3, meta in bits 7..6, nv <= 4) or RO_FMT_ACT /
+ * RO_FMT_NVFP4 (E4M3, meta in bit 7, nv <= 2; nv = 0 is plain NVFP4).  The
+ * steps are those of ro_quantize_block over bs elements: s_f = amax_b /
+ * fp32(6 ts), nearest scale code, d = fp32(s ts), xs = x / d, the candidate
+ * whose exact squared-error difference against plain rounding is smallest
+ * (ties: lowest index), the final encode against Q u {v*}.  scales is
+ * [R, K/bs].
+ */
+static void block_generic(const float *x, int bs, float ts, int sfmt, const double *V, int nv, uint8_t *codes, uint8_t *scale_byte)
+{
+    memset(codes, 0, (size_t)bs);
+    *scale_byte = 0;
+    float amax_b = 0.0f;
+    for (int j = 0; j < bs; j++) {
+        float a = fabsf(x[j]);
+        if (a > amax_b)
+            amax_b = a;
+    }
+    if (!(ts > 0.0f))
+        return;
+    float six_ts = 6.0f * ts;
+    float s_f = amax_b / six_ts;
+    int sc = ro_scale_encode(sfmt, s_f);
+    float d = (float)ro_scale_value(sfmt, sc) * ts;
+    if (sc == 0 || d == 0.0f)
+        return;
+    int meta = 0;
+    double best = 0.0;
+    for (int m = 0; m < nv; m++) {
+        double delta = 0.0;
+        for (int j = 0; j < bs; j++) {
+            float xs = x[j] / d;
+            double rp, rv;
+            round_to_grid(xs, 0, 0.0, &rp);
+            round_to_grid(xs, 1, V[m], &rv);
+            if (rv != rp)
+                delta += (rp - rv) * (2.0 * (double)xs - rv - rp);
+        }
+        if (m == 0 || delta < best) {
+            best = delta;
+            meta = m;
+        }
+    }
+    for (int j = 0; j < bs; j++) {
+        double pt;
+        int code = round_to_grid(x[j] / d, nv > 0, nv > 0 ? V[meta] : 0.0, &pt);
+        codes[j] = (uint8_t)(pt == 0.0 ? 0 : code);
+    }
+    *scale_byte = (uint8_t)(sc | (nv > 0 ? meta << (sfmt == RO_FMT_WEIGHT ? 6 : 7) : 0));
+}
+
+int ro_quantize_generic(const void *x, int dtype, int64_t R, int64_t K, int bs, int sfmt, const double *V, int nv, float ts,
+                        uint8_t *codes, uint8_t *scales)
+{
+    if (bs <= 0 || bs > 128 || K % bs != 0 || (bs & 15) != 0)
+        return 1;
+    float blk[128];
+    uint8_t c[128];
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t b = 0; b < K / bs; b++) {
+            for (int j = 0; j < bs; j++)
+                blk[j] = load_elem(x, dtype, r * K + b * bs + j);
+            uint8_t sb;
+            block_generic(blk, bs, ts, sfmt, V, nv, c, &sb);
+            for (int j = 0; j < bs / 2; j++)
+                codes[r * (K / 2) + b * (bs / 2) + j] = (uint8_t)(c[2 * j] | (c[2 * j + 1] << 4));
+            scales[r * (K / bs) + b] = sb;
+        }
+    return 0;
+}
+
+/* sum (x - q*s*ts)^2 for a tensor of ro_quantize_generic (row-major order, double) */
+double ro_quant_sse_generic(const void *x, int dtype, int64_t R, int64_t K, int bs, int sfmt, const double *V, int nv,
+                            const uint8_t *codes, const uint8_t *scales, float ts)
+{
+    double sse = 0.0;
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t k = 0; k < K; k++) {
+            uint8_t byte = codes[r * (K / 2) + k / 2];
+            int code = (k & 1) ? (byte >> 4) : (byte & 15);
+            uint8_t sb = scales[r * (K / bs) + k / bs];
+            int sc = sb & (sfmt == RO_FMT_WEIGHT ? 0x3f : 0x7f);
+            int meta = nv > 0 ? (sfmt == RO_FMT_WEIGHT ? sb >> 6 : sb >> 7) : 0;
+            double q = ro_fp4_value(code, nv > 0, nv > 0 ? V[meta] : 0.0);
+            double v = q * ro_scale_value(sfmt, sc) * (double)ts;
+            double t = (double)load_elem(x, dtype, r * K + k) - v;
+            sse += t * t;
+        }
+    return sse;
+}
+

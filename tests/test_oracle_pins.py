@@ -466,3 +466,86 @@ def test_quant_sse_and_ablation_invariants(orc):
     same = (s46 == sn)
     blocks6 = np.repeat(same, 8, axis=1)
     np.testing.assert_array_equal(c46[blocks6], cn[blocks6])
+
+
+# ----------------------------------------------------------------------------
+# format variants: block size and special-value set
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_generic_reduces_to_the_format(orc, fmt):
+    # block 16 with the format's own special values is the format's quantizer
+    w = workloads.weight(32, 256, std=0.02, seed=41)
+    V = [orc.special_value(fmt, m) for m in range(orc.num_specials(fmt))]
+    c, s, ts, _ = orc.quantize(w.numpy(), fmt)
+    cg, sg, tg = orc.quantize_generic(w.numpy(), 16, fmt, V)
+    assert tg == ts
+    np.testing.assert_array_equal(cg, c)
+    np.testing.assert_array_equal(sg, s)
+
+
+def _brute_force_generic(xs, specials):
+    # brute_force_block over any block length (zero entries fixed to code 0)
+    nz = [j for j in range(len(xs)) if xs[j] != 0]
+    best = None
+    for meta, v in (list(enumerate(specials)) if specials else [(0, None)]):
+        vv = Fraction(v) if v is not None else Fraction(0)
+        for assign in itertools.product(range(16), repeat=len(nz)):
+            sse = Fraction(0)
+            mags = []
+            for j, c in zip(nz, assign):
+                val = _code_value(c, vv)
+                sse += (Fraction(float(xs[j])) - val) ** 2
+                mags.append((abs(val), c))
+            key = (sse, meta, mags)
+            if best is None or key < best[0]:
+                best = (key, meta, dict(zip(nz, assign)))
+    _, meta, chosen = best
+    return meta, [chosen.get(j, 0) for j in range(len(xs))]
+
+
+@pytest.mark.parametrize("bs,sfmt,V", [(32, 0, [2.5, -2.5, 7.0, -7.0]), (64, 1, [3.5, -3.5]), (32, 0, [5.5, -5.5, 9.5, -9.5])])
+def test_generic_bruteforce(orc, bs, sfmt, V):
+    # sparse blocks of length bs, X^scaled near the custom special values;
+    # exact enumeration of (special value, codes) against the oracle
+    rng = random.Random(bs + 7 * sfmt)
+    ts = 0.125
+    step = Fraction(1, 32) / 8 if sfmt == 0 else Fraction(1, 64) / 8
+    checked = 0
+    for _ in range(80):
+        xs_t = [0.0] * bs
+        for p in rng.sample(range(bs), rng.randint(1, 3)):
+            a = float(np.float32(rng.choice([abs(V[0]) + d for d in (-0.6, -0.25, 0.0, 0.25, 0.6)] + [rng.uniform(0, 9.5)])))
+            xs_t[p] = a if rng.random() < 0.5 else -a
+        x = np.array([float(Fraction(t) * step) for t in xs_t], np.float32).reshape(1, bs)
+        codes, scales, _ = orc.quantize_generic(x, bs, sfmt, V, ts=ts)
+        sb = int(scales[0, 0])
+        sc = sb & (0x3F if sfmt == 0 else 0x7F)
+        got = [(int(codes[0, j // 2]) >> (4 * (j & 1))) & 15 for j in range(bs)]
+        if sc == 0:
+            assert not any(got)
+            continue
+        d = np.float32(np.float32(orc.scale_value(sfmt, sc)) * np.float32(ts))
+        xs = [float(np.float32(np.float32(v) / d)) for v in x[0]]
+        meta_bf, codes_bf = _brute_force_generic(xs, V)
+        meta = sb >> (6 if sfmt == 0 else 7)
+        assert meta == meta_bf and got == codes_bf, (xs, meta, meta_bf)
+        checked += 1
+    assert checked > 20
+
+
+def test_quant_sse_generic_matches_python_decode(orc):
+    # the error sum against a decode written here (value table + scale table)
+    # and a numpy sum; block 64, custom pair on E4M3
+    x = workloads.outlier_activations(8, 256, seed=43)
+    V = [4.5, -4.5]
+    codes, scales, ts = orc.quantize_generic(oracle_input(x), 64, 1, V)
+    vals = np.zeros((8, 256))
+    for r in range(8):
+        for k in range(256):
+            c = (int(codes[r, k // 2]) >> (4 * (k & 1))) & 15
+            sb = int(scales[r, k // 64])
+            q = V[sb >> 7] if c == 8 else _code_value(c, 0)
+            vals[r, k] = float(q) * orc.scale_value(1, sb & 0x7F) * ts
+    ref = float(np.sum((x.float().numpy().astype(np.float64) - vals) ** 2))
+    got = orc.quant_sse_generic(oracle_input(x), 64, 1, V, codes, scales, ts)
+    assert math.isclose(got, ref, rel_tol=1e-12)
