@@ -668,6 +668,21 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
         res["four_over_six_over_nvfp4"] = res["four_over_six"] / res["nvfp4"]
         abl[name] = res
     out["accuracy_ablation_mse"] = abl
+    # format variants on a 4096x4096 weight matrix: the block-size study
+    # (RaZeR with +-5/+-8 vs plain NVFP4 rounding at blocks of 16..128) and the
+    # weights-only search over special-value pairs +-a/+-b (E3M3, block 16)
+    Wv = workloads.weight(4096, 4096, seed=406).to(dev)
+    mse = lambda block, sfmt, V: float(R.razer_quant_error_variant(Wv, block, sfmt, V, *R.razer_quantize_variant(Wv, block, sfmt, V))
+                                       .cpu()[0]) / Wv.numel()
+    blocks = {}
+    for block in (16, 32, 64, 128):
+        blocks[f"block{block}"] = {"nvfp4": mse(block, "nvfp4", []), "razer_pm5_pm8": mse(block, "weight", [5.0, -5.0, 8.0, -8.0])}
+        blocks[f"block{block}"]["razer_over_nvfp4"] = blocks[f"block{block}"]["razer_pm5_pm8"] / blocks[f"block{block}"]["nvfp4"]
+    allowed = [2.5, 3.5, 4.5, 5.0, 5.5, 6.5, 7.0, 7.5, 8.0, 8.5, 9.0, 9.5]
+    pairs = sorted((mse(16, "weight", [a, -a, b, -b]), a, b) for i, a in enumerate(allowed) for b in allowed[i + 1:])
+    out["format_variants_4096x4096"] = {"block_size_study_mse": blocks,
+                                        "special_value_search_top5": [{"pair": f"+-{a}/+-{b}", "mse": m} for m, a, b in pairs[:5]],
+                                        "pairs_searched": len(pairs)}
     return out
 
 

@@ -167,6 +167,151 @@ __global__ void __launch_bounds__(256) quant_sse_kernel(const TIn *__restrict__ 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Format variants: any block size (16..128) and special-value set.
+// ---------------------------------------------------------------------------
+// nearest of the grid u {v} to xs, given the plain rounding rp: v wins when
+// strictly nearer, or equally near with the smaller magnitude (the grid tie
+// rule); distances are exact in binary32 (xs and the points are multiples of
+// xs's ulp, |xs| <= 16)
+__device__ __forceinline__ bool takes_v(float xs, float rp, float v)
+{
+    const float dv = fabsf(__fsub_rn(xs, v)), dp = fabsf(__fsub_rn(xs, rp));
+    return dv < dp || (dv == dp && fabsf(v) < fabsf(rp));
+}
+
+template <int SFMT>
+__device__ __forceinline__ unsigned variant_encode(float sf)
+{
+    return encode_scale<SFMT>(sf);
+}
+
+// One thread per 16 elements; the bs / 16 lanes of a block (consecutive,
+// inside one warp) reduce its amax and the candidates' exact error
+// differences with shuffles.  Decisions as the oracle's ro_quantize_generic.
+template <int SFMT, typename TIn>
+__global__ void __launch_bounds__(256) quantize_variant_kernel(const TIn *__restrict__ x, int64_t nsub, int group,
+                                                               const float *__restrict__ ts_src, int ts_is_amax, VariantV V,
+                                                               uint8_t *__restrict__ codes, uint8_t *__restrict__ scales)
+{
+    using F = Fmt<SFMT>;
+    pdl_wait();
+    pdl_trigger();
+    const float tv = *ts_src;
+    const float ts = ts_is_amax ? __fdiv_rn(tv, F::kC) : tv;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;  // a multiple of 32: groups never straddle warps
+    const int64_t nsub_pad = (nsub + 31) / 32 * 32;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < nsub_pad; t += stride) {
+        const bool live = t < nsub;
+        float xv[16];
+        if (live) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(x) + 2 * t;
+            const uint4 v0 = ldg_stream(p), v1 = ldg_stream(p + 1);
+            const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const float2 f = In16<TIn>::to_f2(wv[i]);
+                xv[2 * i] = f.x;
+                xv[2 * i + 1] = f.y;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; j++) xv[j] = 0.0f;
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; j++) amax = fmaxf(amax, fabsf(xv[j]));
+        for (int o = 1; o < group; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        // every lane of the warp runs the same shuffle sequence below; a
+        // block with a zero scale (or ts <= 0) contributes nothing and stays 0
+        const unsigned sc = ts > 0.0f ? variant_encode<SFMT>(__fdiv_rn(amax, __fmul_rn(6.0f, ts))) : 0u;
+        const float d = __fmul_rn(decode_scale<SFMT>(sc), ts);
+        const bool active = ts > 0.0f && sc != 0u && d != 0.0f;
+        const float dd = active ? d : 1.0f;
+        float xs[16], rp[16];
+        unsigned pc[16];
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+            xs[j] = active ? fminf(fmaxf(__fdiv_rn(xv[j], dd), -16.0f), 16.0f) : 0.0f;
+            pc[j] = e2m1_code_down(xs[j]);
+            rp[j] = e2m1_value(pc[j]);
+        }
+        int meta = 0;
+        double best = 0.0;
+        for (int m = 0; m < V.nv; m++) {
+            double delta = 0.0;
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+                if (takes_v(xs[j], rp[j], V.v[m])) {
+                    const double r0 = rp[j], r1 = V.v[m];
+                    delta = __dadd_rn(delta, __dmul_rn(__dsub_rn(r0, r1), __dsub_rn(__dsub_rn(2.0 * (double)xs[j], r1), r0)));
+                }
+            }
+            for (int o = 1; o < group; o <<= 1) delta += __shfl_xor_sync(0xffffffffu, delta, o);
+            if (m == 0 || delta < best) {
+                best = delta;
+                meta = m;
+            }
+        }
+        unsigned long long c = 0ull;
+        unsigned sb = 0u;
+        if (active) {
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+                const unsigned code = (V.nv > 0 && takes_v(xs[j], rp[j], V.v[meta])) ? 8u : pc[j];
+                c |= (unsigned long long)code << (4 * j);
+            }
+            sb = sc | (V.nv > 0 ? (unsigned)meta << F::kMetaShift : 0u);
+        }
+        if (live) {
+            reinterpret_cast<uint2 *>(codes)[t] = make_uint2((unsigned)c, (unsigned)(c >> 32));
+            if (t % group == 0) scales[t / group] = (uint8_t)sb;
+        }
+    }
+}
+
+template <int SFMT, typename TIn>
+__global__ void __launch_bounds__(256) quant_sse_variant_kernel(const TIn *__restrict__ x, int64_t nsub, int group,
+                                                                const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                                                                const float *__restrict__ ts_p, VariantV V, double *__restrict__ out)
+{
+    using F = Fmt<SFMT>;
+    pdl_wait();
+    pdl_trigger();
+    const double ts = (double)*ts_p;
+    double acc = 0.0;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < nsub; t += stride) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(x) + 2 * t;
+        const uint4 v0 = ldg_stream(p), v1 = ldg_stream(p + 1);
+        const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const uint2 cw = reinterpret_cast<const uint2 *>(codes)[t];
+        const unsigned long long c = (unsigned long long)cw.x | ((unsigned long long)cw.y << 32);
+        const unsigned sb = scales[t / group];
+        const double s = (double)decode_scale<SFMT>(sb & F::kMagMask);
+        const float vm = V.nv > 0 ? V.v[sb >> F::kMetaShift] : 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float2 f = In16<TIn>::to_f2(wv[i]);
+            const unsigned c0 = (unsigned)(c >> (8 * i)) & 15u, c1 = (unsigned)(c >> (8 * i + 4)) & 15u;
+            const double q0 = (V.nv > 0 && c0 == 8u) ? vm : e2m1_value(c0), q1 = (V.nv > 0 && c1 == 8u) ? vm : e2m1_value(c1);
+            const double t0 = __dsub_rn((double)f.x, __dmul_rn(__dmul_rn(q0, s), ts));
+            const double t1 = __dsub_rn((double)f.y, __dmul_rn(__dmul_rn(q1, s), ts));
+            acc = __dadd_rn(acc, __dadd_rn(__dmul_rn(t0, t0), __dmul_rn(t1, t1)));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    __shared__ double sm[8];
+    if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double r = 0.0;
+        for (int i = 0; i < (int)(blockDim.x >> 5); i++) r += sm[i];
+        atomicAdd(out, r);
+    }
+}
+
 __global__ void zero_u64_kernel(unsigned long long *a, unsigned long long *b)
 {
     pdl_wait();
@@ -228,6 +373,66 @@ razer_status run_quant_sse(const void *x, razer_dtype dt, int64_t R, int64_t K, 
     if (fmt == RAZER_FMT_WEIGHT) e = launch_sse<RAZER_FMT_WEIGHT>(dt, x, nblk, codes, scales, ts, out, st);
     else if (fmt == RAZER_FMT_ACT) e = launch_sse<RAZER_FMT_ACT>(dt, x, nblk, codes, scales, ts, out, st);
     else e = launch_sse<RAZER_FMT_NVFP4>(dt, x, nblk, codes, scales, ts, out, st);
+    return e == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
+}
+
+// Format-variant quantizer (block bs, special values V, scale format sfmt):
+// dynamic ts = amax / (6 * S_max(sfmt)).
+razer_status run_quantize_variant(const void *x, razer_dtype dt, int64_t R, int64_t K, int bs, razer_format sfmt, const VariantV &V,
+                                  uint8_t *codes, uint8_t *scales, float *ts_out, cudaStream_t st)
+{
+    const int64_t n = R * K, nsub = n / 16;
+    const float C = sfmt == RAZER_FMT_WEIGHT ? Fmt<RAZER_FMT_WEIGHT>::kC : Fmt<RAZER_FMT_ACT>::kC;
+    if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, (unsigned long long *)nullptr, reinterpret_cast<unsigned *>(ts_out)) != cudaSuccess)
+        return RAZER_ERR_CUDA;
+    if (n > 0) {
+        if (dt == RAZER_F16) launch_amax<__half>(x, n, reinterpret_cast<unsigned *>(ts_out), st);
+        else launch_amax<__nv_bfloat16>(x, n, reinterpret_cast<unsigned *>(ts_out), st);
+    }
+    if (nsub > 0) {
+        const unsigned grid = (unsigned)quant_grid((nsub + 31) / 32 * 32, 256, 8);
+        const int group = bs / 16;
+        const float *tsrc = ts_out;
+        cudaError_t e;
+        const bool h = dt == RAZER_F16;
+        if (sfmt == RAZER_FMT_WEIGHT)
+            e = h ? launch_pdl(quantize_variant_kernel<RAZER_FMT_WEIGHT, __half>, grid, 256u, 0, st, reinterpret_cast<const __half *>(x), nsub,
+                               group, tsrc, 1, V, codes, scales)
+                  : launch_pdl(quantize_variant_kernel<RAZER_FMT_WEIGHT, __nv_bfloat16>, grid, 256u, 0, st,
+                               reinterpret_cast<const __nv_bfloat16 *>(x), nsub, group, tsrc, 1, V, codes, scales);
+        else
+            e = h ? launch_pdl(quantize_variant_kernel<RAZER_FMT_ACT, __half>, grid, 256u, 0, st, reinterpret_cast<const __half *>(x), nsub,
+                               group, tsrc, 1, V, codes, scales)
+                  : launch_pdl(quantize_variant_kernel<RAZER_FMT_ACT, __nv_bfloat16>, grid, 256u, 0, st,
+                               reinterpret_cast<const __nv_bfloat16 *>(x), nsub, group, tsrc, 1, V, codes, scales);
+        if (e != cudaSuccess) return RAZER_ERR_CUDA;
+    }
+    if (launch_pdl(finalize_ts_kernel, 1u, 1u, 0, st, ts_out, C) != cudaSuccess) return RAZER_ERR_CUDA;
+    return last_launch_status();
+}
+
+razer_status run_quant_sse_variant(const void *x, razer_dtype dt, int64_t R, int64_t K, int bs, razer_format sfmt, const VariantV &V,
+                                   const uint8_t *codes, const uint8_t *scales, const float *ts, double *out, cudaStream_t st)
+{
+    const int64_t nsub = R * K / 16;
+    if (launch_pdl(zero_u64_kernel, 1u, 32u, 0, st, reinterpret_cast<unsigned long long *>(out), (unsigned long long *)nullptr) !=
+        cudaSuccess)
+        return RAZER_ERR_CUDA;
+    if (nsub == 0) return last_launch_status();
+    const unsigned grid = (unsigned)quant_grid(nsub, 256, 8);
+    const int group = bs / 16;
+    const bool h = dt == RAZER_F16;
+    cudaError_t e;
+    if (sfmt == RAZER_FMT_WEIGHT)
+        e = h ? launch_pdl(quant_sse_variant_kernel<RAZER_FMT_WEIGHT, __half>, grid, 256u, 0, st, reinterpret_cast<const __half *>(x), nsub,
+                           group, codes, scales, ts, V, out)
+              : launch_pdl(quant_sse_variant_kernel<RAZER_FMT_WEIGHT, __nv_bfloat16>, grid, 256u, 0, st,
+                           reinterpret_cast<const __nv_bfloat16 *>(x), nsub, group, codes, scales, ts, V, out);
+    else
+        e = h ? launch_pdl(quant_sse_variant_kernel<RAZER_FMT_ACT, __half>, grid, 256u, 0, st, reinterpret_cast<const __half *>(x), nsub,
+                           group, codes, scales, ts, V, out)
+              : launch_pdl(quant_sse_variant_kernel<RAZER_FMT_ACT, __nv_bfloat16>, grid, 256u, 0, st,
+                           reinterpret_cast<const __nv_bfloat16 *>(x), nsub, group, codes, scales, ts, V, out);
     return e == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
 }
 

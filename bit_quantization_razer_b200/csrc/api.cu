@@ -1,6 +1,8 @@
 // extern "C" surface of the RaZeR library: argument validation, then the
 // launches of the kernels in quantize.cu / dequant.cu / gemv.cu / gemm.cu.
 // No call allocates memory or synchronises (razer_get_device_status excepted).
+#include <cmath>
+
 #include "razer_internal.cuh"
 
 namespace razer {
@@ -26,6 +28,10 @@ razer_status run_quantize_46(const void *x, razer_dtype dt, int64_t R, int64_t K
                              unsigned long long *n_four, cudaStream_t st);
 razer_status run_quant_sse(const void *x, razer_dtype dt, int64_t R, int64_t K, const uint8_t *codes, const uint8_t *scales,
                            const float *ts, razer_format fmt, double *out, cudaStream_t st);
+razer_status run_quantize_variant(const void *x, razer_dtype dt, int64_t R, int64_t K, int bs, razer_format sfmt, const VariantV &V,
+                                  uint8_t *codes, uint8_t *scales, float *ts_out, cudaStream_t st);
+razer_status run_quant_sse_variant(const void *x, razer_dtype dt, int64_t R, int64_t K, int bs, razer_format sfmt, const VariantV &V,
+                                   const uint8_t *codes, const uint8_t *scales, const float *ts, double *out, cudaStream_t st);
 razer_status run_quantize_batch(int count, const void *const *W, razer_dtype dt, const int64_t *R, const int64_t *K,
                                 uint8_t *const *codes, uint8_t *const *scales, float *ts, razer_format fmt, cudaStream_t st);
 razer_status run_dequant(const uint8_t *codes, const uint8_t *scales, const float *ts, razer_format fmt, int64_t R, int64_t K,
@@ -260,6 +266,54 @@ razer_status razer_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, 
     }
     return run_gemm_w4a4_online(X, x_dt, M, ts_in, afmt, codes_a, scales_a, ts_a_out, meta_hist, codes_w, scales_w, ts_w, wfmt, N, K, Y,
                                 out_dt, workspace, (cudaStream_t)stream);
+}
+
+// checks of a format variant; fills V (scale format RAZER_FMT_ACT and NVFP4
+// both mean E4M3 with a 1-bit meta)
+static razer_status check_variant(int64_t R, int64_t K, int block, razer_format sfmt, const float *vals, int nv, VariantV &V)
+{
+    if (block != 16 && block != 32 && block != 64 && block != 128) return RAZER_ERR_SHAPE;
+    if (R < 0 || K < 0 || K % block != 0) return RAZER_ERR_SHAPE;
+    if (!valid_fmt(sfmt)) return RAZER_ERR_INVALID_ARG;
+    const int max_nv = sfmt == RAZER_FMT_WEIGHT ? 4 : 2;
+    if (nv < 0 || nv > max_nv || (nv > 0 && !vals)) return RAZER_ERR_INVALID_ARG;
+    V.nv = nv;
+    for (int i = 0; i < 4; i++) V.v[i] = 0.0f;
+    for (int i = 0; i < nv; i++) {
+        const float a = fabsf(vals[i]), h = a * 2.0f;
+        // a multiple of 0.5 in [2.5, 9.5], not an E2M1 magnitude (3, 4, 6)
+        if (!(a >= 2.5f && a <= 9.5f) || h != floorf(h) || a == 3.0f || a == 4.0f || a == 6.0f) return RAZER_ERR_INVALID_ARG;
+        V.v[i] = vals[i];
+    }
+    return RAZER_OK;
+}
+
+razer_status razer_quantize_variant(const void *X, razer_dtype in_dt, int64_t R, int64_t K, int block, razer_format scale_fmt,
+                                    const float *special_values, int n_special, uint8_t *codes, uint8_t *scales, float *ts_out,
+                                    razer_stream_t stream)
+{
+    VariantV V;
+    razer_status st = check_variant(R, K, block, scale_fmt, special_values, n_special, V);
+    if (st != RAZER_OK) return st;
+    if (!ts_out || (!X && R * K > 0) || (R * K > 0 && (!codes || !scales))) return RAZER_ERR_INVALID_ARG;
+    if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(in_dt)) return RAZER_ERR_DTYPE;
+    if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(ts_out, 4)) return RAZER_ERR_ALIGN;
+    return run_quantize_variant(X, in_dt, R, K, block, scale_fmt, V, codes, scales, ts_out, (cudaStream_t)stream);
+}
+
+razer_status razer_quant_error_variant(const void *X, razer_dtype in_dt, int64_t R, int64_t K, int block, razer_format scale_fmt,
+                                       const float *special_values, int n_special, const uint8_t *codes, const uint8_t *scales,
+                                       const float *ts, double *sse, razer_stream_t stream)
+{
+    VariantV V;
+    razer_status st = check_variant(R, K, block, scale_fmt, special_values, n_special, V);
+    if (st != RAZER_OK) return st;
+    if (!ts || !sse || (!X && R * K > 0) || (R * K > 0 && (!codes || !scales))) return RAZER_ERR_INVALID_ARG;
+    if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(in_dt)) return RAZER_ERR_DTYPE;
+    if (!aligned(X, 16) || !aligned(codes, 8) || !aligned(ts, 4) || !aligned(sse, 8)) return RAZER_ERR_ALIGN;
+    return run_quant_sse_variant(X, in_dt, R, K, block, scale_fmt, V, codes, scales, ts, sse, (cudaStream_t)stream);
 }
 
 razer_status razer_quant_error(const void *X, razer_dtype in_dt, int64_t R, int64_t K, const uint8_t *codes, const uint8_t *scales,

@@ -31,6 +31,7 @@ _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZE
 EXPORTED = (
     "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
     "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4", "razer_gemm_w4a4_online", "razer_quant_error",
+    "razer_quantize_variant", "razer_quant_error_variant",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
     "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
 )
@@ -70,6 +71,8 @@ def load() -> ctypes.CDLL:
     L.razer_gemv_batch.argtypes = [i32, ctypes.POINTER(GemvProblem), i32, i32, i32, vp, sz, vp]
     L.razer_gemm_w4a4.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_gemm_w4a4_online.argtypes = [vp, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
+    L.razer_quantize_variant.argtypes = [vp, i32, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_float), i32, vp, vp, vp, vp]
+    L.razer_quant_error_variant.argtypes = [vp, i32, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_float), i32, vp, vp, vp, vp, vp]
     L.razer_quant_error.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp]
     L.razer_gemv_batch_workspace_size.argtypes = [i32, ctypes.POINTER(GemvProblem)]
     L.razer_gemv_batch_workspace_size.restype = sz
@@ -83,7 +86,7 @@ def load() -> ctypes.CDLL:
     L.razer_status_string.argtypes = [i32]
     L.razer_status_string.restype = ctypes.c_char_p
     L.razer_version.argtypes = []
-    for fn in ("razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    for fn in ("razer_quantize_variant", "razer_quant_error_variant", "razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -225,6 +228,34 @@ def razer_gemm_w4a4_online(X: torch.Tensor, codes_w: torch.Tensor, scales_w: tor
                                        _p(workspace), wsb, _stream(stream))
     _check("razer_gemm_w4a4_online", st)
     return out, ts_a, ((ca, sa) if keep_codes else None), mh
+
+
+def _varr(V):
+    return (ctypes.c_float * max(len(V), 1))(*[float(v) for v in V])
+
+
+def razer_quantize_variant(X: torch.Tensor, block: int, scale_fmt, V, *, stream=None):
+    """RaZeR quantization with a `block`-element block and special values V.
+    Returns (codes [R, K/2], scales [R, K/block], ts [1])."""
+    R, K = X.shape
+    dev = X.device
+    codes = torch.empty((R, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((R, K // block), dtype=torch.uint8, device=dev)
+    ts = torch.empty(1, dtype=torch.float32, device=dev)
+    st = load().razer_quantize_variant(_p(X), _DT.get(X.dtype, -1), R, K, block, _fmt(scale_fmt), _varr(V), len(V), _p(codes),
+                                       _p(scales), _p(ts), _stream(stream))
+    _check("razer_quantize_variant", st)
+    return codes, scales, ts
+
+
+def razer_quant_error_variant(X: torch.Tensor, block: int, scale_fmt, V, codes, scales, ts, *, out=None, stream=None):
+    """sum (X - deq(X))^2 (double, device [1]) for a tensor of razer_quantize_variant."""
+    R, K = X.shape
+    out = torch.empty(1, dtype=torch.float64, device=X.device) if out is None else out
+    st = load().razer_quant_error_variant(_p(X), _DT.get(X.dtype, -1), R, K, block, _fmt(scale_fmt), _varr(V), len(V), _p(codes),
+                                          _p(scales), _p(ts), _p(out), _stream(stream))
+    _check("razer_quant_error_variant", st)
+    return out
 
 
 def razer_quant_error(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, fmt="weight", *,

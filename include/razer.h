@@ -302,6 +302,33 @@ razer_status razer_quant_error(const void *X, razer_dtype in_dt, int64_t R, int6
                                razer_format fmt, double *sse, razer_stream_t stream);
 
 /*
+ * razer_quantize_variant / razer_quant_error_variant -- format variants for
+ * accuracy studies (the block-size study of the RaZeR notes, 主实验, and the
+ * per-model special-value choice of 训练策略): the RaZeR quantizer with a
+ * block of `block` elements (16, 32, 64 or 128) and the special values
+ * special_values[0..n_special) (host array; each a multiple of 0.5 with
+ * magnitude in [2.5, 9.5] and not an E2M1 magnitude 3, 4 or 6; the
+ * gist.science summary 2.2 gives the constraint).  scale_fmt RAZER_FMT_WEIGHT:
+ * E3M3 scale, meta in bits 7..6 (n_special <= 4); RAZER_FMT_ACT or NVFP4:
+ * E4M3 scale, meta in bit 7 (n_special <= 2); n_special = 0 is plain NVFP4
+ * rounding.  Dynamic ts = amax / (6 * S_max).  codes [R, K/2] (16-byte
+ * aligned), scales [R, K/block].  The decision per block is exact (the
+ * candidates' squared-error differences are summed exactly).  The error
+ * variant writes sum (X - q*s*ts)^2 (double) to the device double *sse.
+ * These calls serve accuracy studies; the GEMV / GEMM decoders read the
+ * fixed 16-element formats only.
+ */
+razer_status razer_quantize_variant(const void *X, razer_dtype in_dt, int64_t R, int64_t K, int block,
+                                    razer_format scale_fmt, const float *special_values,
+                                    int n_special, uint8_t *codes, uint8_t *scales, float *ts_out,
+                                    razer_stream_t stream);
+razer_status razer_quant_error_variant(const void *X, razer_dtype in_dt, int64_t R, int64_t K,
+                                       int block, razer_format scale_fmt,
+                                       const float *special_values, int n_special,
+                                       const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                       double *sse, razer_stream_t stream);
+
+/*
  * razer_gemv_noalloc -- razer_gemv for callers that cannot allocate device
  * memory (the paper has no counterpart: this is a deployment convenience).
  * Some callers cannot call cudaMalloc at all, e.g. a runtime that gives every

@@ -93,6 +93,16 @@ def test_gemv_gemm_validation(lib):
     assert w(*wargs(64, 64, 128, y=ODD)) == 3
     assert w(*wargs(64, 64, 128)) == 5           # workspace missing
     assert w(*wargs(0, 64, 128)) == 0            # empty product
+    v = lib.razer_quantize_variant
+    vals = lambda *xs: (ctypes.c_float * max(len(xs), 1))(*xs)
+    vargs = lambda block, sfmt, V, K=128: (FAKE, 0, 4, K, block, sfmt, vals(*V), len(V), FAKE, FAKE, FAKE, None)
+    assert v(*vargs(24, 0, [5.0])) == 2                  # block size
+    assert v(*vargs(64, 0, [5.0], K=96)) == 2            # K % block
+    assert v(*vargs(32, 0, [3.0])) == 1                  # an E2M1 magnitude
+    assert v(*vargs(32, 0, [10.0])) == 1                 # above 9.5
+    assert v(*vargs(32, 0, [2.7])) == 1                  # not a multiple of 0.5
+    assert v(*vargs(32, 1, [5.0, -5.0, 7.0])) == 1       # E4M3 has one meta bit
+    assert v(*vargs(32, 0, [2.5, -2.5, 9.5, -9.5], K=128)[:4] + (32, 0, vals(2.5, -2.5, 9.5, -9.5), 4, FAKE, FAKE, None, None)) == 1
     d = lib.razer_dequant
     assert d(FAKE, FAKE, FAKE, 3, 4, 32, FAKE, 2, None) == 1
     assert d(FAKE, FAKE, FAKE, 0, 4, 32, FAKE, 5, None) == 1

@@ -68,3 +68,38 @@ def test_ablation_weights_ordering():
         err[fmt] = float(R.razer_quant_error(w, c, s, t, dec).cpu()[0])
     assert err["four_over_six"] < err["nvfp4"]
     assert all(math.isfinite(v) and v > 0 for v in err.values())
+
+
+VARIANTS = [(16, "weight", [5.0, -5.0, 8.0, -8.0]), (32, "weight", [2.5, -2.5, 7.0, -7.0]), (64, "act", [3.5, -3.5]),
+            (128, "act", []), (128, "weight", [5.0, -5.0, 8.0, -8.0]), (32, "nvfp4", [4.5, -4.5])]
+
+
+@pytest.mark.parametrize("block,sfmt,V", VARIANTS)
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_variant_matches_oracle(orc, block, sfmt, V, dtype):
+    # rows of very different spread (subnormal scales, zero rows) so every
+    # special value and the zero block occur
+    w = workloads.weight(96, 1024, std=0.02, seed=81, dtype=torch.float32)
+    w[::5] *= 30.0
+    w[2::9] *= 1e-5
+    w[7] = 0.0
+    w = w.to(dtype)
+    oc, os_, ots = orc.quantize_generic(oracle_in(w), block, FMT_ID[sfmt], V)
+    c, s, t = R.razer_quantize_variant(w.to(DEV), block, sfmt, V)
+    torch.cuda.synchronize()
+    assert float(t.cpu()[0]) == ots
+    np.testing.assert_array_equal(c.cpu().numpy(), oc)
+    np.testing.assert_array_equal(s.cpu().numpy(), os_)
+    ref = orc.quant_sse_generic(oracle_in(w), block, FMT_ID[sfmt], V, oc, os_, ots)
+    got = float(R.razer_quant_error_variant(w.to(DEV), block, sfmt, V, c, s, t).cpu()[0])
+    assert math.isclose(got, ref, rel_tol=1e-12)
+
+
+def test_variant_block16_equals_fast_quantizer():
+    # the variant path with the weight format's own set is the hot-path
+    # quantizer, byte for byte, at a decode shape
+    w = workloads.weight(4096, 4096, std=0.02, seed=82).to(DEV)
+    c1, s1, t1 = R.razer_quantize_weights(w, "weight")
+    c2, s2, t2 = R.razer_quantize_variant(w, 16, "weight", [5.0, -5.0, 8.0, -8.0])
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2) and torch.equal(s1, s2) and torch.equal(t1, t2)
