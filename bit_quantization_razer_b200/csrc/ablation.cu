@@ -16,6 +16,7 @@
 // is exact in double); the partial sums meet in an atomic add, so the last
 // bits depend on the order the blocks finish in.
 #include "razer_internal.cuh"
+#include "variant.cuh"
 
 namespace razer {
 

@@ -4,6 +4,7 @@
 #include <cmath>
 
 #include "razer_internal.cuh"
+#include "variant.cuh"
 
 namespace razer {
 

@@ -26,14 +26,6 @@ __device__ __forceinline__ void set_device_status(unsigned s) { atomicCAS(&g_dev
 // ---------------------------------------------------------------------------
 // Format traits.
 // ---------------------------------------------------------------------------
-// Special-value set of a format variant (block size and set chosen by the
-// caller for accuracy studies): up to 4 values, multiples of 0.5 in
-// [2.5, 9.5], none an E2M1 magnitude.
-struct VariantV {
-    float v[4];
-    int nv;  // 0 (plain) .. 4
-};
-
 template <int FMT> struct Fmt;
 
 template <> struct Fmt<RAZER_FMT_WEIGHT> {
