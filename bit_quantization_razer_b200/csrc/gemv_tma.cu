@@ -140,7 +140,7 @@ __device__ __forceinline__ void wait_phase(uint32_t bar, uint32_t ph, volatile i
 template <int FMT, bool BF16, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_tma_kernel(const __grid_constant__ Batch A, int U, int stages, int stage_sz, int slot_elems, float *__restrict__ ws,
-                    float unbias, int out_dt)
+                    float unbias, int out_dt, int inject_stall)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -194,6 +194,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!mbar_wait(empty + 8 * s, ph ^ 1u, flags)) {
                         ok = false;
                         break;
+                    }
+                    // fault injection (tests only): CTA 0 never fills its second
+                    // stage, so its consumers' bounded waits expire
+                    if (inject_stall && c == 0 && issued == 1) {
+                        inject_stall = 0;
+                        issued++;  // the ring position is used (the drain's bounded wait on it expires)
+                        if (++s == stages) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                        continue;
                     }
                     const uint32_t dst = smem_addr(smem + s * stage_sz);
                     mbar_expect_tx(full + 8 * s, tx);
@@ -433,8 +444,12 @@ static razer_status launch(const Batch &A, const Plan &pl, float *ws, float unbi
         attr_done[dev] = true;
     }
     const int U = (int)pl.U, G = (int)pl.G;
+    // RAZER_FAULT_INJECT_STALL=1 (tests only): one stage is never filled, so
+    // the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
+    const char *inj = getenv("RAZER_FAULT_INJECT_STALL");
+    const int inject = (inj && inj[0] == '1') ? 1 : 0;
     if (launch_pdl(gemv_tma_kernel<FMT, BF16, NB>, (unsigned)G, kThreads, (size_t)smem, st, A, U, stages, sz, slot_elems, ws, unbias,
-                   (int)out_dt) != cudaSuccess)
+                   (int)out_dt, inject) != cudaSuccess)
         return RAZER_ERR_CUDA;
     // tiles shared by several CTAs exist unless every CTA range is whole tiles
     const BatchInfo &I = A.info;

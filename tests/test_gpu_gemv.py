@@ -205,3 +205,25 @@ def test_gemv_batch_decode_projections_sampled(orc):
         rows = np.random.default_rng(i).choice(N, 256, replace=False)
         ref = orc.gemm_ref(x.numpy(), c.numpy()[rows], s.numpy()[rows], t, 0)
         assert rel_err(y.cpu().numpy()[:, rows], ref) <= REL_TOL
+
+
+def test_gemv_bounded_wait_times_out_and_reports(orc, monkeypatch):
+    """One stage that the producer never fills (host-side fault injection):
+    the consumers' bounded waits expire, the device status word reports
+    RAZER_ERR_TIMEOUT, the kernel ends, and the next call is correct."""
+    # 512 half-units over 148 CTAs: CTA 0 runs two stages, the second is skipped
+    N, K, B = 256, 32768, 1
+    codes, scales = workloads.random_packed(N, K, "weight", seed=95)
+    x = workloads.vectors(B, K, seed=96)
+    c, s, xd = codes.to(DEV), scales.to(DEV), x.to(DEV)
+    ts = torch.ones(1, device=DEV)
+    assert R.razer_get_device_status() == 0
+    monkeypatch.setenv("RAZER_FAULT_INJECT_STALL", "1")
+    R.razer_gemv(xd, c, s, ts, "weight", torch.float32)
+    assert R.razer_get_device_status() == 7  # RAZER_ERR_TIMEOUT, read and cleared
+    monkeypatch.delenv("RAZER_FAULT_INJECT_STALL")
+    y = R.razer_gemv(xd, c, s, ts, "weight", torch.float32)
+    torch.cuda.synchronize()
+    assert R.razer_get_device_status() == 0
+    ref = orc.gemm_ref(x.numpy(), codes.numpy(), scales.numpy(), 1.0, 0)
+    assert rel_err(y.cpu().numpy(), ref) <= REL_TOL
