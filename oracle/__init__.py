@@ -31,6 +31,7 @@ _LIB_PATH = os.path.join(_HERE, "librazer_oracle.so")
 FMT_WEIGHT = 0  # E3M3 scale + 2-bit meta, V_w = {+5, -5, +8, -8}
 FMT_ACT = 1  # E4M3 scale + 1-bit meta, V_a = {+5, -5}
 FMT_NVFP4 = 2  # E4M3 scale, no remap
+SCALE_F16 = 4  # format variants only: FP16 block scale, meta in bits 15..14, no tensor scale
 FORMATS = {"weight": FMT_WEIGHT, "act": FMT_ACT, "nvfp4": FMT_NVFP4}
 
 F16, BF16, F32 = 0, 1, 2
@@ -276,15 +277,17 @@ def quant_sse(x, codes: np.ndarray, scales: np.ndarray, ts: float, fmt: int) -> 
 
 def quantize_generic(x, block: int, sfmt: int, V, ts: float | None = None):
     """RaZeR quantization with a block of `block` elements and special values
-    V (scale format sfmt: 0 = E3M3 + 2 meta bits, 1/2 = E4M3 + 1 meta bit).
-    ts None = amax / (6 * S_max(sfmt)). Returns (codes, scales [R, K/block], ts)."""
+    V (scale format sfmt: 0 = E3M3 + 2 meta bits, 1/2 = E4M3 + 1 meta bit,
+    SCALE_F16 = FP16 scale words with the meta in bits 15..14 and no tensor
+    scale). ts None = amax / (6 * S_max(sfmt)) (1 for SCALE_F16). Returns
+    (codes, scales [R, K/block] bytes or [R, 2 K/block] for 16-bit words, ts)."""
     a, dt = _as_bits(x)
     R, K = a.shape
     if ts is None:
-        ts = tensor_scale(x, sfmt)
+        ts = 1.0 if sfmt == SCALE_F16 else tensor_scale(x, sfmt)
     v = np.ascontiguousarray(np.asarray(V, dtype=np.float64).reshape(-1))
     codes = np.zeros((R, K // 2), np.uint8)
-    scales = np.zeros((R, K // block), np.uint8)
+    scales = np.zeros((R, (K // block) * (2 if sfmt == SCALE_F16 else 1)), np.uint8)
     rc = lib().ro_quantize_generic(_ptr(a), dt, R, K, block, sfmt, _ptr(v) if v.size else None, v.size, ts, _ptr(codes), _ptr(scales))
     if rc != 0:
         raise ValueError("oracle quantize_generic: bad block size")

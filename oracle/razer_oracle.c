@@ -61,6 +61,7 @@
 #define RO_FMT_WEIGHT 0 /* E3M3 scale, 2-bit meta, V_w = {+5,-5,+8,-8} */
 #define RO_FMT_ACT 1    /* E4M3 scale, 1-bit meta, V_a = {+5,-5}       */
 #define RO_FMT_NVFP4 2  /* E4M3 scale, no remap (plain NVFP4)          */
+#define RO_SCALE_F16 4  /* format variants only: FP16 block scale, meta in bits 15..14 (R17) */
 
 /* input / output element types */
 #define RO_F16 0
@@ -673,22 +674,42 @@ double ro_quant_sse(const void *x, int dtype, int64_t R, int64_t K, const uint8_
  * (ties: lowest index), the final encode against Q u {v*}.  scales is
  * [R, K/bs].
  */
-static void block_generic(const float *x, int bs, float ts, int sfmt, const double *V, int nv, uint8_t *codes, uint8_t *scale_byte)
+/*
+ * Reading R17 (RaZeR notes, 关键设计 3: the authors' Blackwell kernels use
+ * blocks of 128 with an FP16 block scale whose sign bit and top exponent bit
+ * carry the meta): the scale is s = RN_fp16(amax_b / 6) with bits 15..14
+ * clear, saturating at 0x3FFF (the largest such value, 2 - 2^-10); no tensor
+ * scale (ts = 1); meta in bits 15..14 of the 16-bit scale word.
+ */
+static int f16_scale_code(float amax_b)
+{
+    uint16_t h = ro_float_to_f16(amax_b / 6.0f);
+    return h > 0x3FFF ? 0x3FFF : h;
+}
+
+static void block_generic(const float *x, int bs, float ts, int sfmt, const double *V, int nv, uint8_t *codes, uint16_t *scale_word)
 {
     memset(codes, 0, (size_t)bs);
-    *scale_byte = 0;
+    *scale_word = 0;
     float amax_b = 0.0f;
     for (int j = 0; j < bs; j++) {
         float a = fabsf(x[j]);
         if (a > amax_b)
             amax_b = a;
     }
-    if (!(ts > 0.0f))
-        return;
-    float six_ts = 6.0f * ts;
-    float s_f = amax_b / six_ts;
-    int sc = ro_scale_encode(sfmt, s_f);
-    float d = (float)ro_scale_value(sfmt, sc) * ts;
+    int sc;
+    float d;
+    if (sfmt == RO_SCALE_F16) {
+        sc = f16_scale_code(amax_b);
+        d = (float)ro_f16_to_double((uint16_t)sc);
+    } else {
+        if (!(ts > 0.0f))
+            return;
+        float six_ts = 6.0f * ts;
+        float s_f = amax_b / six_ts;
+        sc = ro_scale_encode(sfmt, s_f);
+        d = (float)ro_scale_value(sfmt, sc) * ts;
+    }
     if (sc == 0 || d == 0.0f)
         return;
     int meta = 0;
@@ -713,7 +734,10 @@ static void block_generic(const float *x, int bs, float ts, int sfmt, const doub
         int code = round_to_grid(x[j] / d, nv > 0, nv > 0 ? V[meta] : 0.0, &pt);
         codes[j] = (uint8_t)(pt == 0.0 ? 0 : code);
     }
-    *scale_byte = (uint8_t)(sc | (nv > 0 ? meta << (sfmt == RO_FMT_WEIGHT ? 6 : 7) : 0));
+    if (sfmt == RO_SCALE_F16)
+        *scale_word = (uint16_t)(sc | (nv > 0 ? meta << 14 : 0));
+    else
+        *scale_word = (uint16_t)(sc | (nv > 0 ? meta << (sfmt == RO_FMT_WEIGHT ? 6 : 7) : 0));
 }
 
 int ro_quantize_generic(const void *x, int dtype, int64_t R, int64_t K, int bs, int sfmt, const double *V, int nv, float ts,
@@ -727,11 +751,16 @@ int ro_quantize_generic(const void *x, int dtype, int64_t R, int64_t K, int bs, 
         for (int64_t b = 0; b < K / bs; b++) {
             for (int j = 0; j < bs; j++)
                 blk[j] = load_elem(x, dtype, r * K + b * bs + j);
-            uint8_t sb;
-            block_generic(blk, bs, ts, sfmt, V, nv, c, &sb);
+            uint16_t sw;
+            block_generic(blk, bs, ts, sfmt, V, nv, c, &sw);
             for (int j = 0; j < bs / 2; j++)
                 codes[r * (K / 2) + b * (bs / 2) + j] = (uint8_t)(c[2 * j] | (c[2 * j + 1] << 4));
-            scales[r * (K / bs) + b] = sb;
+            if (sfmt == RO_SCALE_F16) { /* 16-bit scale words, little-endian */
+                scales[2 * (r * (K / bs) + b)] = (uint8_t)(sw & 0xFF);
+                scales[2 * (r * (K / bs) + b) + 1] = (uint8_t)(sw >> 8);
+            } else {
+                scales[r * (K / bs) + b] = (uint8_t)sw;
+            }
         }
     return 0;
 }
@@ -745,11 +774,20 @@ double ro_quant_sse_generic(const void *x, int dtype, int64_t R, int64_t K, int 
         for (int64_t k = 0; k < K; k++) {
             uint8_t byte = codes[r * (K / 2) + k / 2];
             int code = (k & 1) ? (byte >> 4) : (byte & 15);
-            uint8_t sb = scales[r * (K / bs) + k / bs];
-            int sc = sb & (sfmt == RO_FMT_WEIGHT ? 0x3f : 0x7f);
-            int meta = nv > 0 ? (sfmt == RO_FMT_WEIGHT ? sb >> 6 : sb >> 7) : 0;
+            double sv;
+            int meta;
+            if (sfmt == RO_SCALE_F16) {
+                int64_t bi = r * (K / bs) + k / bs;
+                uint16_t sw = (uint16_t)(scales[2 * bi] | (scales[2 * bi + 1] << 8));
+                sv = ro_f16_to_double((uint16_t)(sw & 0x3FFF));
+                meta = nv > 0 ? sw >> 14 : 0;
+            } else {
+                uint8_t sb = scales[r * (K / bs) + k / bs];
+                sv = ro_scale_value(sfmt, sb & (sfmt == RO_FMT_WEIGHT ? 0x3f : 0x7f));
+                meta = nv > 0 ? (sfmt == RO_FMT_WEIGHT ? sb >> 6 : sb >> 7) : 0;
+            }
             double q = ro_fp4_value(code, nv > 0, nv > 0 ? V[meta] : 0.0);
-            double v = q * ro_scale_value(sfmt, sc) * (double)ts;
+            double v = q * sv * (double)ts;
             double t = (double)load_elem(x, dtype, r * K + k) - v;
             sse += t * t;
         }

@@ -549,3 +549,32 @@ def test_quant_sse_generic_matches_python_decode(orc):
     ref = float(np.sum((x.float().numpy().astype(np.float64) - vals) ** 2))
     got = orc.quant_sse_generic(oracle_input(x), 64, 1, V, codes, scales, ts)
     assert math.isclose(got, ref, rel_tol=1e-12)
+
+
+def test_generic_f16_scale_bruteforce(orc):
+    # the pages' kernel format (block 128, FP16 scale, meta in bits 15..14,
+    # no tensor scale): the scale from numpy's float16 rounding, the choice
+    # and codes by exact enumeration
+    rng = random.Random(17)
+    V = [5.0, -5.0, 8.0, -8.0]
+    checked = 0
+    for _ in range(30):
+        s_true = float(np.float16(rng.uniform(0.01, 0.5)))
+        xs_t = [0.0] * 128
+        xs_t[rng.randrange(128)] = 6.0  # fixes the block amax
+        for p in rng.sample(range(128), 2):
+            a = rng.choice([4.6, 4.9, 5.2, 5.4, rng.uniform(0, 6)])
+            xs_t[p] = a if rng.random() < 0.5 else -a
+        x = np.array([np.float32(t * s_true) for t in xs_t], np.float32).reshape(1, 128)
+        codes, scales, ts = orc.quantize_generic(x, 128, orc.SCALE_F16, V)
+        assert ts == 1.0
+        sw = int(scales[0, 0]) | (int(scales[0, 1]) << 8)
+        h = int(np.float16(np.float32(np.max(np.abs(x))) / np.float32(6.0)).view(np.uint16))
+        assert sw & 0x3FFF == min(h, 0x3FFF)
+        d = np.float32(np.uint16(sw & 0x3FFF).view(np.float16))
+        xs = [float(np.float32(v / d)) for v in x[0]]
+        meta_bf, codes_bf = _brute_force_generic(xs, V)
+        got = [(int(codes[0, j // 2]) >> (4 * (j & 1))) & 15 for j in range(128)]
+        assert (sw >> 14) == meta_bf and got == codes_bf
+        checked += 1
+    assert checked == 30
