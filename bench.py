@@ -680,6 +680,9 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
         blocks[f"block{block}"]["razer_over_nvfp4"] = blocks[f"block{block}"]["razer_pm5_pm8"] / blocks[f"block{block}"]["nvfp4"]
     allowed = [2.5, 3.5, 4.5, 5.0, 5.5, 6.5, 7.0, 7.5, 8.0, 8.5, 9.0, 9.5]
     pairs = sorted((mse(16, "weight", [a, -a, b, -b]), a, b) for i, a in enumerate(allowed) for b in allowed[i + 1:])
+    # the pages' own kernel format: blocks of 128 with an FP16 scale word
+    blocks["block128_f16_scale"] = {"razer_pm5_pm8": mse(128, "f16_scale", [5.0, -5.0, 8.0, -8.0]),
+                                    "plain": mse(128, "f16_scale", [])}
     out["format_variants_4096x4096"] = {"block_size_study_mse": blocks,
                                         "special_value_search_top5": [{"pair": f"+-{a}/+-{b}", "mse": m} for m, a, b in pairs[:5]],
                                         "pairs_searched": len(pairs)}

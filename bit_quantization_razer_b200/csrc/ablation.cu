@@ -181,11 +181,36 @@ __device__ __forceinline__ bool takes_v(float xs, float rp, float v)
     return dv < dp || (dv == dp && fabsf(v) < fabsf(rp));
 }
 
-template <int SFMT>
-__device__ __forceinline__ unsigned variant_encode(float sf)
-{
-    return encode_scale<SFMT>(sf);
-}
+// Scale formats of the variants: E3M3 / E4M3 codes (with the tensor scale),
+// or the FP16 word of the pages' kernel format (R17: s = RN_fp16(amax / 6)
+// with bits 15..14 clear, saturating at 0x3FFF; no tensor scale; meta in bits
+// 15..14).
+constexpr int kScaleF16 = RAZER_SCALE_F16;
+template <int SFMT> struct VarScale {
+    static constexpr float kC = Fmt<SFMT>::kC;
+    static constexpr int kMetaShift = Fmt<SFMT>::kMetaShift;
+    static constexpr unsigned kMagMask = Fmt<SFMT>::kMagMask;
+    static constexpr int kBytes = 1;
+    static __device__ __forceinline__ unsigned encode(float amax, float ts)
+    {
+        return ts > 0.0f ? encode_scale<SFMT>(__fdiv_rn(amax, __fmul_rn(6.0f, ts))) : 0u;
+    }
+    static __device__ __forceinline__ float value(unsigned code) { return decode_scale<SFMT>(code); }
+    static __device__ __forceinline__ float d(unsigned code, float ts) { return __fmul_rn(decode_scale<SFMT>(code), ts); }
+};
+template <> struct VarScale<kScaleF16> {
+    static constexpr float kC = 1.0f;
+    static constexpr int kMetaShift = 14;
+    static constexpr unsigned kMagMask = 0x3FFFu;
+    static constexpr int kBytes = 2;
+    static __device__ __forceinline__ unsigned encode(float amax, float)
+    {
+        const unsigned h = __half_as_ushort(__float2half_rn(__fdiv_rn(amax, 6.0f)));
+        return h > 0x3FFFu ? 0x3FFFu : h;
+    }
+    static __device__ __forceinline__ float value(unsigned code) { return __half2float(__ushort_as_half((unsigned short)code)); }
+    static __device__ __forceinline__ float d(unsigned code, float) { return value(code); }
+};
 
 // One thread per 16 elements; the bs / 16 lanes of a block (consecutive,
 // inside one warp) reduce its amax and the candidates' exact error
@@ -195,11 +220,11 @@ __global__ void __launch_bounds__(256) quantize_variant_kernel(const TIn *__rest
                                                                const float *__restrict__ ts_src, int ts_is_amax, VariantV V,
                                                                uint8_t *__restrict__ codes, uint8_t *__restrict__ scales)
 {
-    using F = Fmt<SFMT>;
+    using F = VarScale<SFMT>;
     pdl_wait();
     pdl_trigger();
-    const float tv = *ts_src;
-    const float ts = ts_is_amax ? __fdiv_rn(tv, F::kC) : tv;
+    const float tv = SFMT == kScaleF16 ? 1.0f : *ts_src;
+    const float ts = (ts_is_amax && SFMT != kScaleF16) ? __fdiv_rn(tv, F::kC) : tv;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;  // a multiple of 32: groups never straddle warps
     const int64_t nsub_pad = (nsub + 31) / 32 * 32;
     for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < nsub_pad; t += stride) {
@@ -225,8 +250,8 @@ __global__ void __launch_bounds__(256) quantize_variant_kernel(const TIn *__rest
         for (int o = 1; o < group; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         // every lane of the warp runs the same shuffle sequence below; a
         // block with a zero scale (or ts <= 0) contributes nothing and stays 0
-        const unsigned sc = ts > 0.0f ? variant_encode<SFMT>(__fdiv_rn(amax, __fmul_rn(6.0f, ts))) : 0u;
-        const float d = __fmul_rn(decode_scale<SFMT>(sc), ts);
+        const unsigned sc = F::encode(amax, ts);
+        const float d = F::d(sc, ts);
         const bool active = ts > 0.0f && sc != 0u && d != 0.0f;
         const float dd = active ? d : 1.0f;
         float xs[16], rp[16];
@@ -266,7 +291,10 @@ __global__ void __launch_bounds__(256) quantize_variant_kernel(const TIn *__rest
         }
         if (live) {
             reinterpret_cast<uint2 *>(codes)[t] = make_uint2((unsigned)c, (unsigned)(c >> 32));
-            if (t % group == 0) scales[t / group] = (uint8_t)sb;
+            if (t % group == 0) {
+                if (F::kBytes == 2) reinterpret_cast<uint16_t *>(scales)[t / group] = (uint16_t)sb;
+                else scales[t / group] = (uint8_t)sb;
+            }
         }
     }
 }
@@ -276,7 +304,7 @@ __global__ void __launch_bounds__(256) quant_sse_variant_kernel(const TIn *__res
                                                                 const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
                                                                 const float *__restrict__ ts_p, VariantV V, double *__restrict__ out)
 {
-    using F = Fmt<SFMT>;
+    using F = VarScale<SFMT>;
     pdl_wait();
     pdl_trigger();
     const double ts = (double)*ts_p;
@@ -288,8 +316,8 @@ __global__ void __launch_bounds__(256) quant_sse_variant_kernel(const TIn *__res
         const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         const uint2 cw = reinterpret_cast<const uint2 *>(codes)[t];
         const unsigned long long c = (unsigned long long)cw.x | ((unsigned long long)cw.y << 32);
-        const unsigned sb = scales[t / group];
-        const double s = (double)decode_scale<SFMT>(sb & F::kMagMask);
+        const unsigned sb = F::kBytes == 2 ? (unsigned)reinterpret_cast<const uint16_t *>(scales)[t / group] : (unsigned)scales[t / group];
+        const double s = (double)F::value(sb & F::kMagMask);
         const float vm = V.nv > 0 ? V.v[sb >> F::kMetaShift] : 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
@@ -311,6 +339,12 @@ __global__ void __launch_bounds__(256) quant_sse_variant_kernel(const TIn *__res
         for (int i = 0; i < (int)(blockDim.x >> 5); i++) r += sm[i];
         atomicAdd(out, r);
     }
+}
+
+__global__ void set_one_kernel(float *p)
+{
+    pdl_wait();
+    *p = 1.0f;
 }
 
 __global__ void zero_u64_kernel(unsigned long long *a, unsigned long long *b)
@@ -396,7 +430,12 @@ razer_status run_quantize_variant(const void *x, razer_dtype dt, int64_t R, int6
         const float *tsrc = ts_out;
         cudaError_t e;
         const bool h = dt == RAZER_F16;
-        if (sfmt == RAZER_FMT_WEIGHT)
+        if (sfmt == RAZER_SCALE_F16)
+            e = h ? launch_pdl(quantize_variant_kernel<kScaleF16, __half>, grid, 256u, 0, st, reinterpret_cast<const __half *>(x), nsub,
+                               group, tsrc, 1, V, codes, scales)
+                  : launch_pdl(quantize_variant_kernel<kScaleF16, __nv_bfloat16>, grid, 256u, 0, st, reinterpret_cast<const __nv_bfloat16 *>(x),
+                               nsub, group, tsrc, 1, V, codes, scales);
+        else if (sfmt == RAZER_FMT_WEIGHT)
             e = h ? launch_pdl(quantize_variant_kernel<RAZER_FMT_WEIGHT, __half>, grid, 256u, 0, st, reinterpret_cast<const __half *>(x), nsub,
                                group, tsrc, 1, V, codes, scales)
                   : launch_pdl(quantize_variant_kernel<RAZER_FMT_WEIGHT, __nv_bfloat16>, grid, 256u, 0, st,
@@ -408,7 +447,11 @@ razer_status run_quantize_variant(const void *x, razer_dtype dt, int64_t R, int6
                                reinterpret_cast<const __nv_bfloat16 *>(x), nsub, group, tsrc, 1, V, codes, scales);
         if (e != cudaSuccess) return RAZER_ERR_CUDA;
     }
-    if (launch_pdl(finalize_ts_kernel, 1u, 1u, 0, st, ts_out, C) != cudaSuccess) return RAZER_ERR_CUDA;
+    if (sfmt == RAZER_SCALE_F16) {  // no tensor scale: ts = 1
+        if (launch_pdl(set_one_kernel, 1u, 1u, 0, st, ts_out) != cudaSuccess) return RAZER_ERR_CUDA;
+    } else if (launch_pdl(finalize_ts_kernel, 1u, 1u, 0, st, ts_out, C) != cudaSuccess) {
+        return RAZER_ERR_CUDA;
+    }
     return last_launch_status();
 }
 
@@ -424,7 +467,12 @@ razer_status run_quant_sse_variant(const void *x, razer_dtype dt, int64_t R, int
     const int group = bs / 16;
     const bool h = dt == RAZER_F16;
     cudaError_t e;
-    if (sfmt == RAZER_FMT_WEIGHT)
+    if (sfmt == RAZER_SCALE_F16)
+        e = h ? launch_pdl(quant_sse_variant_kernel<kScaleF16, __half>, grid, 256u, 0, st, reinterpret_cast<const __half *>(x), nsub, group,
+                           codes, scales, ts, V, out)
+              : launch_pdl(quant_sse_variant_kernel<kScaleF16, __nv_bfloat16>, grid, 256u, 0, st, reinterpret_cast<const __nv_bfloat16 *>(x),
+                           nsub, group, codes, scales, ts, V, out);
+    else if (sfmt == RAZER_FMT_WEIGHT)
         e = h ? launch_pdl(quant_sse_variant_kernel<RAZER_FMT_WEIGHT, __half>, grid, 256u, 0, st, reinterpret_cast<const __half *>(x), nsub,
                            group, codes, scales, ts, V, out)
               : launch_pdl(quant_sse_variant_kernel<RAZER_FMT_WEIGHT, __nv_bfloat16>, grid, 256u, 0, st,

@@ -275,8 +275,8 @@ static razer_status check_variant(int64_t R, int64_t K, int block, razer_format 
 {
     if (block != 16 && block != 32 && block != 64 && block != 128) return RAZER_ERR_SHAPE;
     if (R < 0 || K < 0 || K % block != 0) return RAZER_ERR_SHAPE;
-    if (!valid_fmt(sfmt)) return RAZER_ERR_INVALID_ARG;
-    const int max_nv = sfmt == RAZER_FMT_WEIGHT ? 4 : 2;
+    if (!valid_fmt(sfmt) && sfmt != RAZER_SCALE_F16) return RAZER_ERR_INVALID_ARG;
+    const int max_nv = (sfmt == RAZER_FMT_WEIGHT || sfmt == RAZER_SCALE_F16) ? 4 : 2;
     if (nv < 0 || nv > max_nv || (nv > 0 && !vals)) return RAZER_ERR_INVALID_ARG;
     V.nv = nv;
     for (int i = 0; i < 4; i++) V.v[i] = 0.0f;
@@ -299,7 +299,8 @@ razer_status razer_quantize_variant(const void *X, razer_dtype in_dt, int64_t R,
     if (!ts_out || (!X && R * K > 0) || (R * K > 0 && (!codes || !scales))) return RAZER_ERR_INVALID_ARG;
     if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
     if (!in16(in_dt)) return RAZER_ERR_DTYPE;
-    if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(ts_out, 4)) return RAZER_ERR_ALIGN;
+    if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(ts_out, 4) || (scale_fmt == RAZER_SCALE_F16 && !aligned(scales, 2)))
+        return RAZER_ERR_ALIGN;
     return run_quantize_variant(X, in_dt, R, K, block, scale_fmt, V, codes, scales, ts_out, (cudaStream_t)stream);
 }
 
@@ -313,7 +314,9 @@ razer_status razer_quant_error_variant(const void *X, razer_dtype in_dt, int64_t
     if (!ts || !sse || (!X && R * K > 0) || (R * K > 0 && (!codes || !scales))) return RAZER_ERR_INVALID_ARG;
     if (!valid_dt(in_dt)) return RAZER_ERR_INVALID_ARG;
     if (!in16(in_dt)) return RAZER_ERR_DTYPE;
-    if (!aligned(X, 16) || !aligned(codes, 8) || !aligned(ts, 4) || !aligned(sse, 8)) return RAZER_ERR_ALIGN;
+    if (!aligned(X, 16) || !aligned(codes, 8) || !aligned(ts, 4) || !aligned(sse, 8) ||
+        (scale_fmt == RAZER_SCALE_F16 && !aligned(scales, 2)))
+        return RAZER_ERR_ALIGN;
     return run_quant_sse_variant(X, in_dt, R, K, block, scale_fmt, V, codes, scales, ts, sse, (cudaStream_t)stream);
 }
 

@@ -23,9 +23,10 @@ STATUS_NAMES = {
     7: "RAZER_ERR_TIMEOUT", 8: "RAZER_ERR_CUDA",
 }
 RAZER_F16, RAZER_BF16, RAZER_F32 = 0, 1, 2
-RAZER_FMT_WEIGHT, RAZER_FMT_ACT, RAZER_FMT_NVFP4, RAZER_FMT_FOUR_OVER_SIX = 0, 1, 2, 3
+RAZER_FMT_WEIGHT, RAZER_FMT_ACT, RAZER_FMT_NVFP4, RAZER_FMT_FOUR_OVER_SIX, RAZER_SCALE_F16 = 0, 1, 2, 3, 4
 RAZER_OP_GEMV, RAZER_OP_GEMM, RAZER_OP_GEMM_W4A4 = 0, 1, 2
-FORMATS = {"weight": RAZER_FMT_WEIGHT, "act": RAZER_FMT_ACT, "nvfp4": RAZER_FMT_NVFP4, "four_over_six": RAZER_FMT_FOUR_OVER_SIX}
+FORMATS = {"weight": RAZER_FMT_WEIGHT, "act": RAZER_FMT_ACT, "nvfp4": RAZER_FMT_NVFP4, "four_over_six": RAZER_FMT_FOUR_OVER_SIX,
+           "f16_scale": RAZER_SCALE_F16}
 _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZER_F32}
 
 EXPORTED = (
@@ -240,7 +241,8 @@ def razer_quantize_variant(X: torch.Tensor, block: int, scale_fmt, V, *, stream=
     R, K = X.shape
     dev = X.device
     codes = torch.empty((R, K // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((R, K // block), dtype=torch.uint8, device=dev)
+    wide = _fmt(scale_fmt) == RAZER_SCALE_F16
+    scales = torch.empty((R, (K // block) * (2 if wide else 1)), dtype=torch.uint8, device=dev)
     ts = torch.empty(1, dtype=torch.float32, device=dev)
     st = load().razer_quantize_variant(_p(X), _DT.get(X.dtype, -1), R, K, block, _fmt(scale_fmt), _varr(V), len(V), _p(codes),
                                        _p(scales), _p(ts), _stream(stream))

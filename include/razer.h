@@ -84,7 +84,12 @@ typedef enum {
      * that its amax maps to 6 or to 4, whichever leaves the smaller squared
      * error sum_j (x_j - q_j*d)^2 (double, element order; ties take 6).
      * Four Over Six summary page, 方法详解. */
-    RAZER_FMT_FOUR_OVER_SIX = 3
+    RAZER_FMT_FOUR_OVER_SIX = 3,
+    /* razer_quantize_variant / razer_quant_error_variant only: the FP16 block
+     * scale of the pages' kernel format (RaZeR notes, 关键设计 3) -- a 16-bit
+     * scale word per block, s = RN_fp16(amax_b / 6) in bits 13..0 (saturating
+     * at 0x3FFF), the meta in bits 15..14, no tensor scale (ts = 1). */
+    RAZER_SCALE_F16 = 4
 } razer_format;
 
 typedef enum { RAZER_OP_GEMV = 0, RAZER_OP_GEMM = 1, RAZER_OP_GEMM_W4A4 = 2 } razer_op;
@@ -310,9 +315,11 @@ razer_status razer_quant_error(const void *X, razer_dtype in_dt, int64_t R, int6
  * magnitude in [2.5, 9.5] and not an E2M1 magnitude 3, 4 or 6; the
  * gist.science summary 2.2 gives the constraint).  scale_fmt RAZER_FMT_WEIGHT:
  * E3M3 scale, meta in bits 7..6 (n_special <= 4); RAZER_FMT_ACT or NVFP4:
- * E4M3 scale, meta in bit 7 (n_special <= 2); n_special = 0 is plain NVFP4
- * rounding.  Dynamic ts = amax / (6 * S_max).  codes [R, K/2] (16-byte
- * aligned), scales [R, K/block].  The decision per block is exact (the
+ * E4M3 scale, meta in bit 7 (n_special <= 2); RAZER_SCALE_F16: the pages'
+ * kernel format, 16-bit scale words (n_special <= 4, ts = 1); n_special = 0
+ * is plain rounding.  Dynamic ts = amax / (6 * S_max).  codes [R, K/2]
+ * (16-byte aligned), scales [R, K/block] bytes ([R, K/block] 16-bit words,
+ * 2-byte aligned, for RAZER_SCALE_F16).  The decision per block is exact (the
  * candidates' squared-error differences are summed exactly).  The error
  * variant writes sum (X - q*s*ts)^2 (double) to the device double *sse.
  * These calls serve accuracy studies; the GEMV / GEMM decoders read the

@@ -7,7 +7,7 @@ from bit_quantization_razer_b200 import workloads
 
 cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 
-FMT_ID = {"weight": 0, "act": 1, "nvfp4": 2}
+FMT_ID = {"weight": 0, "act": 1, "nvfp4": 2, "f16_scale": 4}
 
 # Tolerance of the products (fp32 accumulation against the oracle's double
 # accumulation): max |y - r| / max(|r|, 0.01 * rms(r)) <= 2e-3.

@@ -71,7 +71,8 @@ def test_ablation_weights_ordering():
 
 
 VARIANTS = [(16, "weight", [5.0, -5.0, 8.0, -8.0]), (32, "weight", [2.5, -2.5, 7.0, -7.0]), (64, "act", [3.5, -3.5]),
-            (128, "act", []), (128, "weight", [5.0, -5.0, 8.0, -8.0]), (32, "nvfp4", [4.5, -4.5])]
+            (128, "act", []), (128, "weight", [5.0, -5.0, 8.0, -8.0]), (32, "nvfp4", [4.5, -4.5]),
+            (128, "f16_scale", [5.0, -5.0, 8.0, -8.0]), (64, "f16_scale", [])]
 
 
 @pytest.mark.parametrize("block,sfmt,V", VARIANTS)
