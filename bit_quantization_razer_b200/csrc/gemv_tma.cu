@@ -117,13 +117,6 @@ __device__ __forceinline__ unsigned lds16(uint32_t a)
     asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
     return v;
 }
-__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned *p, unsigned v)
-{
-    unsigned old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
-
 __device__ __forceinline__ void store_out(void *y, int out_dt, size_t i, float v)
 {
     if (out_dt == RAZER_F32) reinterpret_cast<float *>(y)[i] = v;

@@ -187,44 +187,17 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
         // 2^-20.  A = sum t and B = sum copysign(t, xs) are exact binary32 sums
         // (|A|, |B| <= 16); then the +5 sum is (A - B) / 2 and the -5 sum is
         // (A + B) / 2, both exact.
-#ifndef RAZER_Q_SAT
-#define RAZER_Q_SAT 1
-#endif
-#ifndef RAZER_Q_SCALAR_AB
-#define RAZER_Q_SCALAR_AB 0
-#endif
-        float ea[16];                           // 2|xs| - 10, reused by the final encode
-#if RAZER_Q_SAT
-        // -t = sat(1 - |e|) in one saturating add
-        float Ap = 0.0f, Bp = 0.0f;
-        float2 AB = make_float2(0.0f, 0.0f);
+        float ea[16];  // 2|xs| - 10, reused by the final encode
+        // -t = sat(1 - |e|) in one saturating add; copysign(-t, xs) =
+        // copysign(t, xs) for t <= 0, so the second sum is B itself
+        float2 AB = make_float2(0.0f, 0.0f);  // (-A, B), one packed add per element
 #pragma unroll
         for (int j = 0; j < 16; j++) {
             ea[j] = __fmaf_rn(2.0f, fabsf(xs[j]), -10.0f);
             const float nt = __saturatef(__fadd_rn(1.0f, -fabsf(ea[j])));
-#if RAZER_Q_SCALAR_AB
-            Ap = __fadd_rn(Ap, nt);
-            Bp = __fadd_rn(Bp, copysignf(nt, xs[j]));
-#else
             AB = add2(AB, make_float2(nt, copysignf(nt, xs[j])));
-#endif
         }
-#if !RAZER_Q_SCALAR_AB
-        Ap = AB.x;
-        Bp = AB.y;
-#endif
-        // copysign(-t, xs) = copysign(t, xs) for t <= 0: B is the same sum
-        const float A = -Ap, Bs = Bp;
-#else
-        float2 AB = make_float2(0.0f, 0.0f);  // (A, B), one packed add per element
-#pragma unroll
-        for (int j = 0; j < 16; j++) {
-            ea[j] = __fmaf_rn(2.0f, fabsf(xs[j]), -10.0f);
-            const float t = fminf(__fadd_rn(fabsf(ea[j]), -1.0f), 0.0f);
-            AB = add2(AB, make_float2(t, copysignf(t, xs[j])));
-        }
-        const float A = AB.x, Bs = AB.y;
-#endif
+        const float A = -AB.x, Bs = AB.y;
         const float dp5 = __fmul_rn(__fsub_rn(A, Bs), 0.5f);
         const float dn5 = __fmul_rn(__fadd_rn(A, Bs), 0.5f);
         float best = dp5;
