@@ -93,6 +93,10 @@ def lib():
         L.ro_quantize_generic.argtypes = [vp, ctypes.c_int, i64, i64, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, f32, u8p, u8p]
         L.ro_quant_sse_generic.argtypes = [vp, ctypes.c_int, i64, i64, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, u8p, u8p, f32]
         L.ro_quant_sse_generic.restype = f64
+        L.ro_dequant_generic.argtypes = [u8p, u8p, f32, i64, i64, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, ctypes.c_int, vp]
+        L.ro_dequant_generic.restype = ctypes.c_int
+        L.ro_gemv_generic.argtypes = [vp, ctypes.c_int, i64, u8p, u8p, f32, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, i64, i64, vp]
+        L.ro_gemv_generic.restype = ctypes.c_int
         L.ro_gemm_w4a4_ref.argtypes = [u8p, u8p, f32, ctypes.c_int, i64, u8p, u8p, f32, ctypes.c_int, i64, i64, vp, i64, vp]
         L.ro_gemm_ref.restype = ctypes.c_int
         _lib = L
@@ -292,6 +296,40 @@ def quantize_generic(x, block: int, sfmt: int, V, ts: float | None = None):
     if rc != 0:
         raise ValueError("oracle quantize_generic: bad block size")
     return codes, scales, float(np.float32(ts))
+
+
+def dequant_generic(codes: np.ndarray, scales: np.ndarray, ts: float, block: int, sfmt: int, V, out_dtype: str = "f32"):
+    """Decode a variant tensor (codes [R, K/2], scales as quantize_generic
+    returns them) to [R, K]: f32 values, or uint16 bit patterns for 'f16'/'bf16'."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    R, K2 = codes.shape
+    K = K2 * 2
+    v = np.ascontiguousarray(np.asarray(V, dtype=np.float64).reshape(-1))
+    odt = {"f16": F16, "bf16": BF16, "f32": F32}[out_dtype]
+    out = np.zeros((R, K), np.float32 if odt == F32 else np.uint16)
+    rc = lib().ro_dequant_generic(_ptr(codes), _ptr(scales), ts, R, K, block, sfmt, _ptr(v) if v.size else None, v.size, odt,
+                                  _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle dequant_generic: bad block size")
+    return out
+
+
+def gemv_generic(x, codes: np.ndarray, scales: np.ndarray, ts: float, block: int, sfmt: int, V) -> np.ndarray:
+    """r[b, n] = ts * sum_k x[b, k] * (q*s)[n, k] in double for a variant
+    weight tensor; x is [B, K] (fp16/bf16 torch tensor or numpy)."""
+    a, dt = _as_bits(x)
+    B, K = a.shape
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    N = codes.shape[0]
+    v = np.ascontiguousarray(np.asarray(V, dtype=np.float64).reshape(-1))
+    out = np.zeros((B, N), np.float64)
+    rc = lib().ro_gemv_generic(_ptr(a), dt, B, _ptr(codes), _ptr(scales), ts, block, sfmt, _ptr(v) if v.size else None, v.size,
+                               N, K, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle gemv_generic failed")
+    return out
 
 
 def quant_sse_generic(x, block: int, sfmt: int, V, codes: np.ndarray, scales: np.ndarray, ts: float) -> float:

@@ -765,6 +765,28 @@ int ro_quantize_generic(const void *x, int dtype, int64_t R, int64_t K, int bs, 
     return 0;
 }
 
+/* q*s of element (r, k) of a tensor of ro_quantize_generic (exact in double) */
+static double generic_qs(const uint8_t *codes, const uint8_t *scales, int64_t K, int bs, int sfmt, const double *V, int nv,
+                         int64_t r, int64_t k)
+{
+    uint8_t byte = codes[r * (K / 2) + k / 2];
+    int code = (k & 1) ? (byte >> 4) : (byte & 15);
+    double sv;
+    int meta;
+    if (sfmt == RO_SCALE_F16) {
+        int64_t bi = r * (K / bs) + k / bs;
+        uint16_t sw = (uint16_t)(scales[2 * bi] | (scales[2 * bi + 1] << 8));
+        sv = ro_f16_to_double((uint16_t)(sw & 0x3FFF));
+        meta = nv > 0 ? sw >> 14 : 0;
+    } else {
+        uint8_t sb = scales[r * (K / bs) + k / bs];
+        sv = ro_scale_value(sfmt, sb & (sfmt == RO_FMT_WEIGHT ? 0x3f : 0x7f));
+        meta = nv > 0 ? (sfmt == RO_FMT_WEIGHT ? sb >> 6 : sb >> 7) : 0;
+    }
+    double q = ro_fp4_value(code, nv > 0, nv > 0 ? V[meta] : 0.0);
+    return q * sv;
+}
+
 /* sum (x - q*s*ts)^2 for a tensor of ro_quantize_generic (row-major order, double) */
 double ro_quant_sse_generic(const void *x, int dtype, int64_t R, int64_t K, int bs, int sfmt, const double *V, int nv,
                             const uint8_t *codes, const uint8_t *scales, float ts)
@@ -772,25 +794,63 @@ double ro_quant_sse_generic(const void *x, int dtype, int64_t R, int64_t K, int 
     double sse = 0.0;
     for (int64_t r = 0; r < R; r++)
         for (int64_t k = 0; k < K; k++) {
-            uint8_t byte = codes[r * (K / 2) + k / 2];
-            int code = (k & 1) ? (byte >> 4) : (byte & 15);
-            double sv;
-            int meta;
-            if (sfmt == RO_SCALE_F16) {
-                int64_t bi = r * (K / bs) + k / bs;
-                uint16_t sw = (uint16_t)(scales[2 * bi] | (scales[2 * bi + 1] << 8));
-                sv = ro_f16_to_double((uint16_t)(sw & 0x3FFF));
-                meta = nv > 0 ? sw >> 14 : 0;
-            } else {
-                uint8_t sb = scales[r * (K / bs) + k / bs];
-                sv = ro_scale_value(sfmt, sb & (sfmt == RO_FMT_WEIGHT ? 0x3f : 0x7f));
-                meta = nv > 0 ? (sfmt == RO_FMT_WEIGHT ? sb >> 6 : sb >> 7) : 0;
-            }
-            double q = ro_fp4_value(code, nv > 0, nv > 0 ? V[meta] : 0.0);
-            double v = q * sv * (double)ts;
+            double v = generic_qs(codes, scales, K, bs, sfmt, V, nv, r, k) * (double)ts;
             double t = (double)load_elem(x, dtype, r * K + k) - v;
             sse += t * t;
         }
     return sse;
+}
+
+/*
+ * Decoder of the format variants, defined like ro_dequant: out[r, k] =
+ * round_out( fp32( (q*s) * ts ) ) -- q*s is exact in binary32 for every
+ * variant (at most 5 significant bits of q times at most 11 of s), one
+ * binary32 multiply by ts, one rounding to the output type.
+ */
+int ro_dequant_generic(const uint8_t *codes, const uint8_t *scales, float ts, int64_t R, int64_t K, int bs, int sfmt,
+                       const double *V, int nv, int out_dtype, void *out)
+{
+    if (bs <= 0 || bs > 128 || (bs & 15) != 0 || K % bs != 0)
+        return 1;
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t k = 0; k < K; k++) {
+            float qs = (float)generic_qs(codes, scales, K, bs, sfmt, V, nv, r, k);
+            float v = qs * ts;
+            int64_t i = r * K + k;
+            if (out_dtype == RO_F16)
+                ((uint16_t *)out)[i] = ro_float_to_f16(v);
+            else if (out_dtype == RO_BF16)
+                ((uint16_t *)out)[i] = ro_float_to_bf16(v);
+            else
+                ((float *)out)[i] = v;
+        }
+    return 0;
+}
+
+/*
+ * Reference W4A16 product on a variant weight tensor [N, K]:
+ * r[b, n] = ts * sum_k x[b, k] * (q*s)[n, k], accumulated in double (x is
+ * [B, K] of x_dtype); out is [B, N].
+ */
+int ro_gemv_generic(const void *x, int x_dtype, int64_t B, const uint8_t *codes, const uint8_t *scales, float ts, int bs,
+                    int sfmt, const double *V, int nv, int64_t N, int64_t K, double *out)
+{
+    if (bs <= 0 || bs > 128 || (bs & 15) != 0 || K % bs != 0)
+        return 1;
+    double *wrow = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+    if (!wrow)
+        return 2;
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t k = 0; k < K; k++)
+            wrow[k] = generic_qs(codes, scales, K, bs, sfmt, V, nv, n, k);
+        for (int64_t b = 0; b < B; b++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += (double)load_elem(x, x_dtype, b * K + k) * wrow[k];
+            out[b * N + n] = acc * (double)ts;
+        }
+    }
+    free(wrow);
+    return 0;
 }
 

@@ -578,3 +578,70 @@ def test_generic_f16_scale_bruteforce(orc):
         assert (sw >> 14) == meta_bf and got == codes_bf
         checked += 1
     assert checked == 30
+
+
+# ----------------------------------------------------------------------------
+# decoder and W4A16 reference of the format variants
+# ----------------------------------------------------------------------------
+_DEFAULT_V = {0: [5.0, -5.0, 8.0, -8.0], 1: [5.0, -5.0], 2: []}
+
+
+def _random_scale_bytes(rng, shape, fmt):
+    if fmt == 0:  # E3M3 magnitude (every 6-bit value valid) + 2 meta bits
+        return rng.integers(0, 256, shape, dtype=np.uint8)
+    mag = rng.integers(0, 0x7F, shape, dtype=np.uint8)  # E4M3 without the NaN code
+    if fmt == 1:
+        return mag | (rng.integers(0, 2, shape, dtype=np.uint8) << 7)
+    return mag
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_dequant_generic_reduces_to_the_format(orc, fmt):
+    # at block 16 with the format's own special values the variant decoder is
+    # the pinned decoder; at blocks 32 / 128 it equals the pinned decoder on
+    # scales repeated per 16 elements (the block index k / block)
+    rng = np.random.default_rng(60 + fmt)
+    R, K = 6, 256
+    codes = rng.integers(0, 256, (R, K // 2), dtype=np.uint8)
+    V = _DEFAULT_V[fmt]
+    ts = 0.0123
+    for bs in (16, 32, 128):
+        sc = _random_scale_bytes(rng, (R, K // bs), fmt)
+        sc16 = np.repeat(sc, bs // 16, axis=1)
+        for odt in ("f32", "f16", "bf16"):
+            np.testing.assert_array_equal(orc.dequant_generic(codes, sc, ts, bs, fmt, V, odt),
+                                          orc.dequant(codes, sc16, ts, fmt, odt))
+
+
+def test_dequant_generic_f16_scale_words(orc):
+    # FP16 scale words: bits 13..0 read by numpy's float16 decode, the meta in
+    # bits 15..14 selecting V like the E3M3 meta bits 7..6 (compared through an
+    # E3M3 scale of exactly 1.0, code 0b011000), little-endian 16-bit words
+    rng = np.random.default_rng(64)
+    R, K, bs = 5, 384, 128
+    V = [2.5, -7.0, 9.5, -3.5]
+    codes = rng.integers(0, 256, (R, K // 2), dtype=np.uint8)
+    mag = rng.integers(0, 0x4000, (R, K // bs), dtype=np.uint16)
+    meta = rng.integers(0, 4, (R, K // bs), dtype=np.uint16)
+    words = (mag | (meta << 14)).astype("<u2")
+    got = orc.dequant_generic(codes, words.view(np.uint8), 1.0, bs, orc.SCALE_F16, V, "f32")
+    unit = (24 | (meta.astype(np.uint8) << 6)).astype(np.uint8)
+    q = orc.dequant_generic(codes, unit, 1.0, bs, 0, V, "f32").astype(np.float64)
+    s = np.repeat(mag.view(np.float16).astype(np.float64), bs, axis=1)
+    np.testing.assert_array_equal(got, (q * s).astype(np.float32))
+    assert np.array_equal(q * s, (q * s).astype(np.float32).astype(np.float64))  # q*s exact in binary32
+
+
+def test_gemv_generic_matches_numpy(orc):
+    x = workloads.vectors(3, 256, seed=65)
+    w = workloads.weight(40, 256, seed=66)
+    for bs, sfmt, V in ((128, orc.SCALE_F16, [5.0, -5.0, 8.0, -8.0]), (32, 0, [5.0, -5.0, 7.0, -7.0]), (64, 1, [4.5, -4.5])):
+        codes, scales, ts = orc.quantize_generic(w.numpy(), bs, sfmt, V)
+        deq = orc.dequant_generic(codes, scales, 1.0, bs, sfmt, V, "f32").astype(np.float64)
+        ref = (x.numpy().astype(np.float64) @ deq.T) * ts
+        got = orc.gemv_generic(x.numpy(), codes, scales, ts, bs, sfmt, V)
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    # block 16 with the weight format's values is the pinned product reference
+    codes, scales, ts, _ = orc.quantize(w.numpy(), 0)
+    np.testing.assert_array_equal(orc.gemv_generic(x.numpy(), codes, scales, ts, 16, 0, _DEFAULT_V[0]),
+                                  orc.gemm_ref(x.numpy(), codes, scales, ts, 0))
