@@ -686,6 +686,28 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
     out["format_variants_4096x4096"] = {"block_size_study_mse": blocks,
                                         "special_value_search_top5": [{"pair": f"+-{a}/+-{b}", "mse": m} for m, a, b in pairs[:5]],
                                         "pairs_searched": len(pairs)}
+    # W4A16 GEMV on variant weights (14336x4096, fp16): the pages' kernel
+    # format (blocks of 128, FP16 scale words) and a per-model pair at block 16;
+    # 8 weight copies rotate so every call streams its weights from HBM
+    N, K = 14336, 4096
+    gv = {}
+    for name, block, sfmt, V in (("block128_f16_scale_pm5_pm8", 128, "f16_scale", [5.0, -5.0, 8.0, -8.0]),
+                                 ("block16_e3m3_pm5_pm7", 16, "weight", [5.0, -5.0, 7.0, -7.0])):
+        c0, s0 = workloads.random_packed_variant(N, K, block, sfmt, len(V), seed=407)
+        c0, s0 = c0.to(dev), s0.to(dev)
+        copies = [(c0.clone(), s0.clone()) for _ in range(8)]
+        tsv = torch.tensor([1.0 if sfmt == "f16_scale" else 2.0 ** -9], dtype=torch.float32, device=dev)
+        res = {}
+        for B in (1, 16):
+            xv = workloads.vectors(B, K, seed=408).to(dev)
+            yv = torch.empty((B, N), dtype=torch.float16, device=dev)
+            wsv = torch.empty(R.razer_workspace_size(R.RAZER_OP_GEMV, B, N, K), dtype=torch.uint8, device=dev)
+            ms = time_graph(lambda: [R.razer_gemv_variant(xv, cc, ss, tsv, block, sfmt, V, torch.float16, out=yv, workspace=wsv)
+                                     for cc, ss in copies], 8, stream)
+            nbytes = N * K // 2 + s0.numel() + 2 * B * K + 2 * B * N
+            res[f"B{B}"] = {"ms": ms, "GB/s": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm}
+        gv[name] = res
+    out["gemv_variant_14336x4096"] = gv
     return out
 
 

@@ -33,6 +33,12 @@ razer_status run_quantize_variant(const void *x, razer_dtype dt, int64_t R, int6
                                   uint8_t *codes, uint8_t *scales, float *ts_out, cudaStream_t st);
 razer_status run_quant_sse_variant(const void *x, razer_dtype dt, int64_t R, int64_t K, int bs, razer_format sfmt, const VariantV &V,
                                    const uint8_t *codes, const uint8_t *scales, const float *ts, double *out, cudaStream_t st);
+razer_status run_dequant_variant(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t R, int64_t K, int bs,
+                                 razer_format sfmt, const VariantV &V, void *out, razer_dtype dt, cudaStream_t st);
+razer_status run_gemv_variant(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                              int bs, razer_format sfmt, const VariantV &V, int64_t N, int64_t K, void *y, razer_dtype out_dt,
+                              void *workspace, cudaStream_t st);
+size_t gemv_variant_workspace_bytes(int64_t B, int64_t N, int64_t K);
 razer_status run_quantize_batch(int count, const void *const *W, razer_dtype dt, const int64_t *R, const int64_t *K,
                                 uint8_t *const *codes, uint8_t *const *scales, float *ts, razer_format fmt, cudaStream_t st);
 razer_status run_dequant(const uint8_t *codes, const uint8_t *scales, const float *ts, razer_format fmt, int64_t R, int64_t K,
@@ -318,6 +324,61 @@ razer_status razer_quant_error_variant(const void *X, razer_dtype in_dt, int64_t
         (scale_fmt == RAZER_SCALE_F16 && !aligned(scales, 2)))
         return RAZER_ERR_ALIGN;
     return run_quant_sse_variant(X, in_dt, R, K, block, scale_fmt, V, codes, scales, ts, sse, (cudaStream_t)stream);
+}
+
+razer_status razer_dequant_variant(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t R, int64_t K, int block,
+                                   razer_format scale_fmt, const float *special_values, int n_special, void *out, razer_dtype out_dt,
+                                   razer_stream_t stream)
+{
+    VariantV V;
+    razer_status st = check_variant(R, K, block, scale_fmt, special_values, n_special, V);
+    if (st != RAZER_OK) return st;
+    if (!ts || (R * K > 0 && (!codes || !scales || !out))) return RAZER_ERR_INVALID_ARG;
+    if (!valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!aligned(codes, 8) || !aligned(out, 16) || !aligned(ts, 4) || (scale_fmt == RAZER_SCALE_F16 && !aligned(scales, 2)))
+        return RAZER_ERR_ALIGN;
+    return run_dequant_variant(codes, scales, ts, R, K, block, scale_fmt, V, out, out_dt, (cudaStream_t)stream);
+}
+
+// a special value whose doubled magnitude has 5 significant bits (8.5, 9.5):
+// q * s then needs up to 9 bits, more than bf16 holds
+static bool needs_five_bits(const VariantV &V)
+{
+    for (int i = 0; i < V.nv; i++) {
+        int h = (int)(fabsf(V.v[i]) * 2.0f);
+        while (h > 0 && (h & 1) == 0) h >>= 1;
+        if (h >= 16) return true;
+    }
+    return false;
+}
+
+razer_status razer_gemv_variant(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                int block, razer_format scale_fmt, const float *special_values, int n_special, int64_t N, int64_t K,
+                                void *y, razer_dtype out_dt, void *workspace, size_t ws_bytes, razer_stream_t stream)
+{
+    VariantV V;
+    razer_status st = check_variant(N, K, block, scale_fmt, special_values, n_special, V);
+    if (st != RAZER_OK) return st;
+    if (!ts || (!x && K > 0) || (!y && N > 0) || (N * K > 0 && (!codes || !scales))) return RAZER_ERR_INVALID_ARG;
+    if (!valid_dt(act_dt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(act_dt)) return RAZER_ERR_DTYPE;
+    if (B < 1 || B > 32 || K % 128 != 0 || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (scale_fmt == RAZER_SCALE_F16 && block != 128) return RAZER_ERR_UNSUPPORTED;
+    if (scale_fmt != RAZER_SCALE_F16 && act_dt == RAZER_BF16 && needs_five_bits(V)) return RAZER_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ts, 4) || !aligned(codes, 16) ||
+        (scale_fmt == RAZER_SCALE_F16 && !aligned(scales, 2)))
+        return RAZER_ERR_ALIGN;
+    if (N == 0) return RAZER_OK;
+    if (K == 0)  // empty sums: y = 0
+        return cudaMemsetAsync(y, 0, (size_t)B * (size_t)N * (out_dt == RAZER_F32 ? 4 : 2), (cudaStream_t)stream) == cudaSuccess
+                   ? RAZER_OK
+                   : RAZER_ERR_CUDA;
+    const size_t need = gemv_variant_workspace_bytes(B, N, K);
+    if (need) {
+        if (!workspace || ws_bytes < need) return RAZER_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
+    }
+    return run_gemv_variant(x, act_dt, B, codes, scales, ts, block, scale_fmt, V, N, K, y, out_dt, workspace, (cudaStream_t)stream);
 }
 
 razer_status razer_quant_error(const void *X, razer_dtype in_dt, int64_t R, int64_t K, const uint8_t *codes, const uint8_t *scales,

@@ -8,5 +8,6 @@
 #include "dequant.cu"
 #include "gemv.cu"
 #include "gemv_tma.cu"
+#include "variant_decode.cu"
 #include "gemm.cu"
 #include "gemv_noalloc.cu"

@@ -32,7 +32,7 @@ _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZE
 EXPORTED = (
     "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
     "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4", "razer_gemm_w4a4_online", "razer_quant_error",
-    "razer_quantize_variant", "razer_quant_error_variant",
+    "razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
     "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
 )
@@ -74,6 +74,9 @@ def load() -> ctypes.CDLL:
     L.razer_gemm_w4a4_online.argtypes = [vp, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, vp, i32, vp, sz, vp]
     L.razer_quantize_variant.argtypes = [vp, i32, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_float), i32, vp, vp, vp, vp]
     L.razer_quant_error_variant.argtypes = [vp, i32, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_float), i32, vp, vp, vp, vp, vp]
+    L.razer_dequant_variant.argtypes = [vp, vp, vp, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_float), i32, vp, i32, vp]
+    L.razer_gemv_variant.argtypes = [vp, i32, i64, vp, vp, vp, i32, i32, ctypes.POINTER(ctypes.c_float), i32, i64, i64, vp, i32, vp,
+                                     sz, vp]
     L.razer_quant_error.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp]
     L.razer_gemv_batch_workspace_size.argtypes = [i32, ctypes.POINTER(GemvProblem)]
     L.razer_gemv_batch_workspace_size.restype = sz
@@ -87,7 +90,7 @@ def load() -> ctypes.CDLL:
     L.razer_status_string.argtypes = [i32]
     L.razer_status_string.restype = ctypes.c_char_p
     L.razer_version.argtypes = []
-    for fn in ("razer_quantize_variant", "razer_quant_error_variant", "razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    for fn in ("razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant", "razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -248,6 +251,31 @@ def razer_quantize_variant(X: torch.Tensor, block: int, scale_fmt, V, *, stream=
                                        _p(scales), _p(ts), _stream(stream))
     _check("razer_quantize_variant", st)
     return codes, scales, ts
+
+
+def razer_dequant_variant(codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, block: int, scale_fmt, V,
+                          out_dtype=torch.float32, *, out=None, stream=None):
+    """Decode a razer_quantize_variant tensor to [R, K]: (q*s)*ts rounded once to out_dtype."""
+    R, K2 = codes.shape
+    K = 2 * K2
+    out = torch.empty((R, K), dtype=out_dtype, device=codes.device) if out is None else out
+    st = load().razer_dequant_variant(_p(codes), _p(scales), _p(ts), R, K, block, _fmt(scale_fmt), _varr(V), len(V), _p(out),
+                                      _DT.get(out.dtype, -1), _stream(stream))
+    _check("razer_dequant_variant", st)
+    return out
+
+
+def razer_gemv_variant(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, block: int, scale_fmt, V,
+                       out_dtype=torch.float32, *, out=None, workspace=None, stream=None):
+    """y [B, N] = ts * x [B, K] . deq(W [N, K])^T for a razer_quantize_variant weight tensor, 1 <= B <= 32."""
+    B, K = x.shape
+    N = codes.shape[0]
+    out = torch.empty((B, N), dtype=out_dtype, device=x.device) if out is None else out
+    workspace, wsb = _workspace(RAZER_OP_GEMV, B, N, K, x.device, workspace)
+    st = load().razer_gemv_variant(_p(x), _DT.get(x.dtype, -1), B, _p(codes), _p(scales), _p(ts), block, _fmt(scale_fmt),
+                                   _varr(V), len(V), N, K, _p(out), _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
+    _check("razer_gemv_variant", st)
+    return out
 
 
 def razer_quant_error_variant(X: torch.Tensor, block: int, scale_fmt, V, codes, scales, ts, *, out=None, stream=None):

@@ -81,3 +81,27 @@ def random_packed(N: int, K: int, fmt: str, *, seed: int = 3, max_scale_code: in
         meta = torch.randint(0, 2, (N, K // 16), generator=g, dtype=torch.int32) if fmt == "act" else torch.zeros_like(mag)
         scales = (mag | (meta << 7)).to(torch.uint8)
     return codes, scales
+
+
+def random_packed_variant(N: int, K: int, block: int, scale_fmt: str, n_special: int, *, seed: int = 5):
+    """Random packed weights [N, K] of a format variant: uniform code bytes,
+    uniform valid scale magnitudes and meta values below n_special.  scale_fmt
+    "weight" (E3M3 bytes, meta bits 7..6), "act" / "nvfp4" (E4M3 bytes, meta
+    bit 7) or "f16_scale" (16-bit little-endian words: magnitude bits 13..0,
+    meta bits 15..14).  Returns (codes [N, K/2] u8, scales [N, K/block] u8 or
+    [N, 2 K/block] u8 for the 16-bit words) as CPU tensors."""
+    g = _gen(seed)
+    codes = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.int32).to(torch.uint8)
+    nb = K // block
+    meta = torch.randint(0, max(n_special, 1), (N, nb), generator=g, dtype=torch.int32)
+    if scale_fmt == "f16_scale":
+        mag = torch.randint(0, 0x4000, (N, nb), generator=g, dtype=torch.int32)
+        w = mag | (meta << 14)
+        scales = torch.stack([w & 0xFF, w >> 8], dim=2).reshape(N, 2 * nb).to(torch.uint8)
+    elif scale_fmt == "weight":
+        mag = torch.randint(0, 64, (N, nb), generator=g, dtype=torch.int32)
+        scales = (mag | (meta << 6)).to(torch.uint8)
+    else:
+        mag = torch.randint(0, 127, (N, nb), generator=g, dtype=torch.int32)
+        scales = (mag | (meta << 7)).to(torch.uint8)
+    return codes, scales

@@ -322,8 +322,8 @@ razer_status razer_quant_error(const void *X, razer_dtype in_dt, int64_t R, int6
  * 2-byte aligned, for RAZER_SCALE_F16).  The decision per block is exact (the
  * candidates' squared-error differences are summed exactly).  The error
  * variant writes sum (X - q*s*ts)^2 (double) to the device double *sse.
- * These calls serve accuracy studies; the GEMV / GEMM decoders read the
- * fixed 16-element formats only.
+ * razer_dequant_variant and razer_gemv_variant (below) decode these
+ * tensors; the hot-path GEMV / GEMM calls read the 16-element formats only.
  */
 razer_status razer_quantize_variant(const void *X, razer_dtype in_dt, int64_t R, int64_t K, int block,
                                     razer_format scale_fmt, const float *special_values,
@@ -334,6 +334,41 @@ razer_status razer_quant_error_variant(const void *X, razer_dtype in_dt, int64_t
                                        const float *special_values, int n_special,
                                        const uint8_t *codes, const uint8_t *scales, const float *ts,
                                        double *sse, razer_stream_t stream);
+
+/*
+ * razer_dequant_variant -- decoder of a razer_quantize_variant tensor (the
+ * same block, scale_fmt and special values; RaZeR notes, 关键设计 3: the FP4
+ * -0 code decodes to the special value the block's meta selects):
+ *   out[r, k] = round_out( (q * s) * ts ),
+ * q*s exact in binary32, one binary32 multiply by *ts, one rounding to out_dt
+ * (f16 / bf16 / f32).  Bit-exact.  codes [R, K/2] (8-byte aligned); scales
+ * as razer_quantize_variant writes them; out [R, K] (16-byte aligned).  A
+ * meta value at or past n_special decodes the 0b1000 code to 0.
+ */
+razer_status razer_dequant_variant(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t R, int64_t K,
+                                   int block, razer_format scale_fmt, const float *special_values, int n_special,
+                                   void *out, razer_dtype out_dt, razer_stream_t stream);
+
+/*
+ * razer_gemv_variant -- W4A16 small-batch product on a format-variant weight
+ * tensor (the per-model special values of the RaZeR notes, 训练策略, and the
+ * pages' own kernel format of 关键设计 3: blocks of 128, FP16 scale words):
+ *   y[b, n] = ts * sum_k x[b, k] * (q*s)[n, k],   1 <= B <= 32,
+ * fp32 accumulation.  Arguments as razer_gemv, plus block / scale_fmt /
+ * special_values / n_special as razer_quantize_variant.  workspace: at least
+ * razer_workspace_size(RAZER_OP_GEMV, B, N, K) bytes (16-byte aligned; NULL
+ * when that is 0), contents ignored.  K % 128 == 0; codes 16-byte aligned.
+ * Byte scales (RAZER_FMT_WEIGHT / ACT / NVFP4): any block; the decoded
+ * weights q*s enter the tensor-core MMA exactly, so bf16 activations with a
+ * special value of 5 significant bits (+-8.5, +-9.5) give
+ * RAZER_ERR_UNSUPPORTED (the operand would round in bf16).
+ * RAZER_SCALE_F16: block 128 only (others RAZER_ERR_UNSUPPORTED); the MMA
+ * sums q * x and each block's fp32 sum is multiplied by its scale.
+ */
+razer_status razer_gemv_variant(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes,
+                                const uint8_t *scales, const float *ts, int block, razer_format scale_fmt,
+                                const float *special_values, int n_special, int64_t N, int64_t K, void *y,
+                                razer_dtype out_dt, void *workspace, size_t ws_bytes, razer_stream_t stream);
 
 /*
  * razer_gemv_noalloc -- razer_gemv for callers that cannot allocate device

@@ -109,6 +109,38 @@ def test_gemv_gemm_validation(lib):
     assert d(FAKE, FAKE, FAKE, 0, 4, 32, ODD, 2, None) == 3
 
 
+def test_variant_decode_validation(lib):
+    vals = lambda *xs: (ctypes.c_float * max(len(xs), 1))(*xs)
+    g = lib.razer_gemv_variant
+
+    def gargs(block=32, sfmt=0, V=(5.0, -5.0), B=1, N=64, K=128, act=0, codes=FAKE, scales=FAKE):
+        return (FAKE, act, B, codes, scales, FAKE, block, sfmt, vals(*V), len(V), N, K, FAKE, 2, None, 0, None)
+
+    assert g(*gargs(block=24)) == 2                                   # block size
+    assert g(*gargs(block=32, K=96)) == 2                              # K % block
+    assert g(*gargs(block=32, K=64 * 3)) == 2                          # K % 128
+    assert g(*gargs(B=33)) == 2
+    assert g(*gargs(act=2)) == 4                                       # f32 activations
+    assert g(*gargs(block=64, sfmt=4)) == 6                            # FP16 scale words: block 128 only
+    assert g(*gargs(V=(5.0, -5.0, 9.5, -9.5), act=1)) == 6             # bf16 operand would round
+    assert g(*gargs(V=(5.0, -5.0, 8.5, -8.5), act=1)) == 6
+    assert g(*gargs(V=(5.0, -5.0, 9.0, -9.0), act=1)) == 5             # 4 significant bits: allowed (no workspace)
+    assert g(*gargs(V=(5.0, -5.0, 9.5, -9.5), act=0)) == 5             # fp16 operands are exact
+    assert g(*gargs(block=128, sfmt=4, V=(9.5, -9.5), act=1)) == 5     # q alone enters the MMA
+    assert g(*gargs(block=128, sfmt=4, scales=ODD)) == 3               # 16-bit scale words
+    assert g(*gargs(codes=ctypes.c_void_p(0x1008))) == 3
+    assert g(*gargs(N=0)) == 0                                         # empty product
+    d = lib.razer_dequant_variant
+    dargs = lambda block=32, sfmt=0, R=4, K=128, ts=FAKE, out=FAKE, odt=2: (FAKE, FAKE, ts, R, K, block, sfmt, vals(5.0, -5.0), 2,
+                                                                            out, odt, None)
+    assert d(*dargs(ts=None)) == 1
+    assert d(*dargs(out=ODD)) == 3
+    assert d(*dargs(odt=5)) == 1
+    assert d(*dargs(block=48)) == 2
+    assert d(*dargs(block=64, K=96)) == 2
+    assert d(*dargs(R=0)) == 0                                         # empty tensor
+
+
 def test_workspace_size_host_logic(lib):
     assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, 0, 64, 128) == 0
     def split_k(B, N, K):  # per-warp kernel: ~8 CTAs per SM (148 without a GPU), >= 2 chunks per split
