@@ -251,7 +251,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the breakdown / e2e / GEMM legs")
     ap.add_argument("--no-soak", action="store_true", help="skip the 1.5 s pre-timing load for the clock sampler")
-    ap.add_argument("--kernel", choices=["quantize", "quantize_batch", "act_quantize", "dequant", "gemv", "gemv_batch", "gemm"],
+    ap.add_argument("--kernel", choices=["quantize", "quantize_batch", "act_quantize", "dequant", "gemv", "gemv_batch", "gemv_variant",
+                             "gemm"],
                     help="profiling mode: run one call on --shape in a loop (for ncu)")
     ap.add_argument("--shape", default="4096,4096", help="N,K (gemm: M,N,K; quantize_batch: N1,K1,N2,K2,...)")
     ap.add_argument("--batch", type=int, default=1)
@@ -424,6 +425,7 @@ def main():
                                                else "razer_gemv_batch of the 3 projections, per B (bulk-tensor + split-K "
                                                     "reduce kernels)"),
                 "algorithmic_bytes_per_call": dom_bytes / n_calls, "peak_source": peak_src,
+                "nominal_peak": 8000.0, "frac_nominal": achieved / 8000.0,
                 "timing": "CUDA events around CUDA-graph replays of back-to-back calls on operand copies larger than L2"}
 
     extras = {}
@@ -508,6 +510,17 @@ def run_single_kernel(args):
 
         def call():
             R.razer_gemv_batch(probs, "weight", torch.float16, outs=ys, workspace=ws)
+    elif args.kernel == "gemv_variant":
+        # the pages' kernel format: blocks of 128, FP16 scale words, +-5/+-8
+        N, K = dims
+        V = [5.0, -5.0, 8.0, -8.0]
+        c, s, t = R.razer_quantize_variant(workloads.weight(N, K, seed=1).to(dev), 128, "f16_scale", V)
+        x = workloads.vectors(args.batch, K, seed=2).to(dev)
+        y = torch.empty((args.batch, N), dtype=torch.float16, device=dev)
+        ws = torch.empty(max(16, R.razer_workspace_size(R.RAZER_OP_GEMV, args.batch, N, K)), dtype=torch.uint8, device=dev)
+
+        def call():
+            R.razer_gemv_variant(x, c, s, t, 128, "f16_scale", V, torch.float16, out=y, workspace=ws)
     elif args.kernel == "act_quantize":
         M, K = dims
         xa = workloads.outlier_activations(M, K, seed=3).to(dev)
@@ -608,7 +621,7 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / reps
             tf = 2 * 4096 * N * K / ms / 1e9
-            res[f"{4096}x{N}x{K}"] = {"ms": ms, "TFLOP/s": tf, "frac": tf / bf16}
+            res[f"{4096}x{N}x{K}"] = {"ms": ms, "TFLOP/s": tf, "frac": tf / bf16, "frac_nominal_2250": tf / 2250.0}
         out["gemm"] = res
     except R.RazerError as e:
         out["gemm"] = {"unavailable": str(e)}
@@ -708,7 +721,78 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
             res[f"B{B}"] = {"ms": ms, "GB/s": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm}
         gv[name] = res
     out["gemv_variant_14336x4096"] = gv
+    out["llama3_70b_sweep"] = run_70b_sweep(R, workloads, dev, stream, hbm, bf16)
+    # the tiny case the oracle checks in full (launch-bound: time only)
+    Wt = workloads.weight(256, 512, seed=0).to(dev)
+    xt = workloads.vectors(1, 512, seed=1).to(dev)
+    ct, st_, tt = R.razer_quantize_weights(Wt)
+    yt = torch.empty((1, 256), dtype=torch.float16, device=dev)
+    wst = torch.empty(max(16, R.razer_workspace_size(R.RAZER_OP_GEMV, 1, 256, 512)), dtype=torch.uint8, device=dev)
+    out["tiny_256x512"] = {
+        "quantize_ms": time_graph(lambda: R.razer_quantize_weights(Wt, codes=ct, scales=st_, ts=tt), 1, stream),
+        "gemv_b1_ms": time_graph(lambda: R.razer_gemv(xt, ct, st_, tt, "weight", torch.float16, out=yt, workspace=wst), 1, stream),
+        "note": "launch-bound; parity case, no roofline fraction"}
+    # cuBLAS on the decoded weights, as an outside sanity reference only (a
+    # library run on bf16 operands, not a target)
+    Xc = workloads.vectors(4096, 4096, seed=400, dtype=torch.bfloat16).to(dev)
+    cub = {}
+    for N in (4096, 14336):
+        c, s, t = R.razer_quantize_weights(workloads.weight(N, 4096, seed=401).to(dev))
+        Wd = R.razer_dequant(c, s, t, "weight", torch.bfloat16)
+        Yc = torch.empty((4096, N), dtype=torch.bfloat16, device=dev)
+        ms = time_graph(lambda: torch.matmul(Xc, Wd.t(), out=Yc), 1, stream)
+        cub[f"4096x{N}x4096"] = {"ms": ms, "TFLOP/s": 2 * 4096 * N * 4096 / ms / 1e9}
+        del Wd, Yc
+    out["cublas_bf16_on_decoded_weights"] = cub
     return out
+
+
+def _rotation(nbytes, l2=126 * 2 ** 20):
+    """Operand copies for a back-to-back sequence that cannot hit L2:
+    ceil(2 L2 / bytes), at least 8 below 64 MB, at least 2."""
+    n = -(-2 * l2 // max(nbytes, 1))
+    if nbytes < 64 * 2 ** 20:
+        n = max(n, 8)
+    return max(n, 2)
+
+
+def run_70b_sweep(R, workloads, dev, stream, hbm, bf16):
+    """Llama-3-70B projections (N(0, 0.015^2), 0.1% x10): the W4A16 GEMV at
+    B = 1, 8, 32 and the prefill GEMM at M = 512, 2048, 8192, in the RaZeR
+    weight format and in plain NVFP4."""
+    import torch
+
+    shapes = [(8192, 8192), (28672, 8192), (8192, 28672)]
+    res = {}
+    for si, (N, K) in enumerate(shapes):
+        W = workloads.weight(N, K, std=0.015, seed=500 + si).to(dev)
+        for fmt in ("weight", "nvfp4"):
+            c, s, t = R.razer_quantize_weights(W, fmt)
+            packed = c.numel() + s.numel()
+            copies = [(c, s)] + [(c.clone(), s.clone()) for _ in range(_rotation(packed) - 1)]
+            key = f"{N}x{K}_{'razer' if fmt == 'weight' else 'nvfp4'}"
+            row = {}
+            for B in (1, 8, 32):
+                x = workloads.vectors(B, K, seed=510 + B).to(dev)
+                y = torch.empty((B, N), dtype=torch.float16, device=dev)
+                ws = torch.empty(max(16, R.razer_workspace_size(R.RAZER_OP_GEMV, B, N, K)), dtype=torch.uint8, device=dev)
+                ms = time_graph(lambda: [R.razer_gemv(x, cc, ss, t, fmt, torch.float16, out=y, workspace=ws) for cc, ss in copies],
+                                len(copies), stream)
+                nbytes = 0.5625 * N * K + 2 * B * K + 2 * B * N
+                row[f"gemv_B{B}"] = {"ms": ms, "GB/s": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm,
+                                     "frac_nominal_8TBs": nbytes / ms / 1e6 / 8000.0}
+            del copies
+            for M in (512, 2048, 8192):
+                X = workloads.vectors(M, K, seed=520 + M, dtype=torch.bfloat16).to(dev)
+                Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                ws = torch.empty(max(16, R.razer_workspace_size(R.RAZER_OP_GEMM, M, N, K)), dtype=torch.uint8, device=dev)
+                ms = time_graph(lambda: R.razer_gemm(X, c, s, t, fmt, torch.bfloat16, out=Y, workspace=ws), 1, stream, reps=3)
+                tf = 2 * M * N * K / ms / 1e9
+                row[f"gemm_M{M}"] = {"ms": ms, "TFLOP/s": tf, "frac": tf / bf16, "frac_nominal_2250": tf / 2250.0}
+                del X, Y, ws
+            res[key] = row
+        del W
+    return res
 
 
 def run_e2e(R, workloads, dev, stream, args, world, pg):

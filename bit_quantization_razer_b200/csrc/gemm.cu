@@ -212,8 +212,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = (DECODED ? blockIdx.y : blockIdx.x) * BN, m0 = (DECODED ? blockIdx.x : blockIdx.y) * BM;
     // this launch covers k-steps [kb0, kb0 + nkb) of the K / 64; a previous
-    // chunk's fp32 result (already scaled) is added in the epilogue
-    const int KB = nkb;
+    // chunk's fp32 result (already scaled) is added in the epilogue.  With
+    // gridDim.z > 1 the range is split further: split z takes its own part and
+    // writes its scaled fp32 sum to slice z of Y ([gridDim.z, M, N] fp32).
+    const int kbs = kb0 + (int)((int64_t)blockIdx.z * nkb / gridDim.z);
+    const int KB = kb0 + (int)((int64_t)(blockIdx.z + 1) * nkb / gridDim.z) - kbs;
+    if (gridDim.z > 1) Y = reinterpret_cast<float *>(Y) + (size_t)blockIdx.z * (size_t)M * (size_t)N;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
@@ -245,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
                 mbar_expect_tx(full_a + 8 * s, kMBlocks * A_HALF_BYTES + (DECODED ? B_BYTES : 0u));
 #pragma unroll
-                for (int a = 0; a < kMBlocks; a++) tma_load_2d(a0 + a * A_HALF_BYTES, &tmap_x, (kb0 + kb) * BK, m0 + 128 * a, full_a + 8 * s);
-                if constexpr (DECODED) tma_load_2d(a0 + kMBlocks * A_HALF_BYTES, &tmap_w, (kb0 + kb) * BK, n0, full_a + 8 * s);
+                for (int a = 0; a < kMBlocks; a++) tma_load_2d(a0 + a * A_HALF_BYTES, &tmap_x, (kbs + kb) * BK, m0 + 128 * a, full_a + 8 * s);
+                if constexpr (DECODED) tma_load_2d(a0 + kMBlocks * A_HALF_BYTES, &tmap_w, (kbs + kb) * BK, n0, full_a + 8 * s);
                 issued = kb + 1;
             }
             if (*abort_flag) {
@@ -308,9 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto load_stage = [&](int kb, Regs &r) {
 #pragma unroll
-            for (int h = 0; h < kHalvesPerThread; h++) r.c[h] = ldg_stream(crow + (size_t)(kb0 + kb) * 32 + 16 * h);
-            r.s = kHalvesPerThread == 1 ? (unsigned)*reinterpret_cast<const unsigned short *>(srow + (size_t)(kb0 + kb) * 4)
-                                        : *reinterpret_cast<const unsigned *>(srow + (size_t)(kb0 + kb) * 4);
+            for (int h = 0; h < kHalvesPerThread; h++) r.c[h] = ldg_stream(crow + (size_t)(kbs + kb) * 32 + 16 * h);
+            r.s = kHalvesPerThread == 1 ? (unsigned)*reinterpret_cast<const unsigned short *>(srow + (size_t)(kbs + kb) * 4)
+                                        : *reinterpret_cast<const unsigned *>(srow + (size_t)(kbs + kb) * 4);
         };
         Regs r0, r1;
         bool ok = true;
@@ -537,7 +541,8 @@ constexpr int64_t kDecodedMinM = 1024;
 // accumulator loses precision over long chains (measured on B200 with
 // decoded E3M3 weights: relative error ~5e-4 at K = 7168 but ~2.5e-3 at
 // K = 28672), so a longer K runs as equal chunks whose scaled partial sums
-// are added in fp32 through a [M, N] workspace buffer.
+// are added in fp32: as parallel splits with one [M, N] slice each in
+// razer_gemm, through one [M, N] buffer chunk after chunk in the W4A4 product.
 #ifndef RAZER_GEMM_CHAIN_K
 #define RAZER_GEMM_CHAIN_K 16384
 #endif
@@ -548,10 +553,55 @@ static int64_t num_chunks(int64_t K) { return (K + kMaxChainK - 1) / kMaxChainK;
 static size_t decoded_bytes(int64_t M, int64_t N, int64_t K) { return M >= kDecodedMinM ? (size_t)N * (size_t)K * 2 : 0; }
 static size_t partial_bytes(int64_t M, int64_t N, int64_t K) { return num_chunks(K) > 1 ? (size_t)M * (size_t)N * 4 : 0; }
 
+// Parallel K splits of razer_gemm: at least the number of accumulation chains
+// K needs, and more when the output tiles alone cannot occupy the SMs (each
+// split keeps at least kMinSplitSteps k-steps).  Every split writes its scaled
+// fp32 sum to its own [M, N] slice of the workspace; gemm_splits_reduce_kernel
+// adds the slices in split order (deterministic) and converts.
+constexpr int64_t kMinSplitSteps = 8;
+static int gemm_splits(int64_t M, int64_t N, int64_t K)
+{
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    int64_t s = num_chunks(K);
+    const int64_t sm = sm_count();
+    if (tiles > 0 && tiles < sm) s = std::max(s, std::min(sm / tiles, (K / BK) / kMinSplitSteps));
+    return (int)std::max<int64_t>(s, 1);
+}
+static size_t split_bytes(int64_t M, int64_t N, int64_t K)
+{
+    const int s = gemm_splits(M, N, K);
+    return s > 1 ? (size_t)s * (size_t)M * (size_t)N * 4 : 0;
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(256) gemm_splits_reduce_kernel(const float4 *__restrict__ part, int S, int64_t n4, TOut *__restrict__ Y)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+        float4 a = part[i];
+        for (int z = 1; z < S; z++) {
+            const float4 b = part[(size_t)z * (size_t)n4 + (size_t)i];
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+        if constexpr (sizeof(TOut) == 4) {
+            reinterpret_cast<float4 *>(Y)[i] = a;
+        } else if constexpr (std::is_same<TOut, __half>::value) {
+            __half2 lo = __floats2half2_rn(a.x, a.y), hi = __floats2half2_rn(a.z, a.w);
+            reinterpret_cast<uint2 *>(Y)[i] = make_uint2(*reinterpret_cast<unsigned *>(&lo), *reinterpret_cast<unsigned *>(&hi));
+        } else {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+            reinterpret_cast<uint2 *>(Y)[i] = make_uint2(*reinterpret_cast<unsigned *>(&lo), *reinterpret_cast<unsigned *>(&hi));
+        }
+    }
+}
+
 template <int FMT, bool BF16, bool DECODED>
 static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, const uint8_t *codes, const uint8_t *scales, const float *ts,
                            float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, int kb0, int nkb, const float *addend,
-                           cudaStream_t st)
+                           cudaStream_t st, int splits = 1)
 {
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -563,7 +613,7 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, cons
         attr_set[dev] = true;
     }
     const unsigned nt = (unsigned)((N + BN - 1) / BN), mt = (unsigned)((M + BM - 1) / BM);
-    const dim3 grid = DECODED ? dim3(mt, nt) : dim3(nt, mt);
+    const dim3 grid = DECODED ? dim3(mt, nt, (unsigned)splits) : dim3(nt, mt, (unsigned)splits);
     // RAZER_FAULT_INJECT_STALL=1 (tests only) withholds one decoder warp's
     // arrivals so that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
     const char *inj = getenv("RAZER_FAULT_INJECT_STALL");
@@ -576,7 +626,7 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, cons
 template <int FMT, bool BF16>
 static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, bool decoded, const uint8_t *codes, const uint8_t *scales,
                                const float *ts, float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, void *wdec,
-                               float *partial, cudaStream_t st)
+                               float *slices, cudaStream_t st)
 {
     if (decoded) {
         const int64_t nblk = (int64_t)N * K / 16;
@@ -586,18 +636,19 @@ static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, 
             return RAZER_ERR_CUDA;
     }
     const int KB = K / BK;
-    const int nc = (int)num_chunks(K);
-    for (int c = 0; c < nc; c++) {
-        const int kb0 = (int)((int64_t)c * KB / nc), kb1 = (int)((int64_t)(c + 1) * KB / nc);
-        const bool last = c == nc - 1;
-        void *out = last ? Y : partial;
-        const razer_dtype odt = last ? out_dt : RAZER_F32;
-        const float *add = c > 0 ? partial : nullptr;
-        const razer_status r = decoded ? launch<FMT, BF16, true>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, kb0, kb1 - kb0, add, st)
-                                       : launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, kb0, kb1 - kb0, add, st);
-        if (r != RAZER_OK) return r;
-    }
-    return RAZER_OK;
+    const int S = gemm_splits(M, N, K);
+    void *out = S > 1 ? static_cast<void *>(slices) : Y;
+    const razer_dtype odt = S > 1 ? RAZER_F32 : out_dt;
+    const razer_status r = decoded ? launch<FMT, BF16, true>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S)
+                                   : launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S);
+    if (r != RAZER_OK || S == 1) return r;
+    const int64_t n4 = (int64_t)M * N / 4;  // N % 16 == 0
+    const int64_t g = std::max<int64_t>(1, std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 8));
+    const float4 *part = reinterpret_cast<const float4 *>(slices);
+    if (out_dt == RAZER_F32) gemm_splits_reduce_kernel<float><<<(unsigned)g, 256, 0, st>>>(part, S, n4, reinterpret_cast<float *>(Y));
+    else if (out_dt == RAZER_F16) gemm_splits_reduce_kernel<__half><<<(unsigned)g, 256, 0, st>>>(part, S, n4, reinterpret_cast<__half *>(Y));
+    else gemm_splits_reduce_kernel<__nv_bfloat16><<<(unsigned)g, 256, 0, st>>>(part, S, n4, reinterpret_cast<__nv_bfloat16 *>(Y));
+    return last_launch_status();
 }
 
 // decoded q*s*2^-bias of a packed [R, K] tensor into out (16-bit, [R, K])
@@ -765,9 +816,9 @@ razer_status run_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, co
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
-    // the decoded weight copy when the decode-once path applies, then the
-    // fp32 partial sums when K spans several accumulation chains
-    return gemm::decoded_bytes(M, N, K) + gemm::partial_bytes(M, N, K);
+    // the decoded weight copy when the decode-once path applies, then one fp32
+    // [M, N] slice per parallel K split when there is more than one
+    return gemm::decoded_bytes(M, N, K) + gemm::split_bytes(M, N, K);
 }
 
 razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
@@ -793,7 +844,7 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
     // the decoded q*s carries 2^-8 (E3M3) / 2^-4 (E4M3); undone in the epilogue
     const float unbias = wfmt == RAZER_FMT_WEIGHT ? 256.0f : 16.0f;
     const bool decoded = decoded_bytes(M, N, K) > 0;
-    float *partial = partial_bytes(M, N, K) ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + decoded_bytes(M, N, K)) : nullptr;
+    float *slices = split_bytes(M, N, K) ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + decoded_bytes(M, N, K)) : nullptr;
     CUtensorMap wmap = map;  // unused by the fused kernel
     if (decoded) {
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
@@ -807,13 +858,13 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
     }
     const int m = (int)M, n = (int)N, k = (int)K;
     if (wfmt == RAZER_FMT_WEIGHT)
-        return bf ? launch_fmt<RAZER_FMT_WEIGHT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st)
-                  : launch_fmt<RAZER_FMT_WEIGHT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st);
+        return bf ? launch_fmt<RAZER_FMT_WEIGHT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
+                  : launch_fmt<RAZER_FMT_WEIGHT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
     if (wfmt == RAZER_FMT_ACT)
-        return bf ? launch_fmt<RAZER_FMT_ACT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st)
-                  : launch_fmt<RAZER_FMT_ACT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st);
-    return bf ? launch_fmt<RAZER_FMT_NVFP4, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st)
-              : launch_fmt<RAZER_FMT_NVFP4, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, partial, st);
+        return bf ? launch_fmt<RAZER_FMT_ACT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
+                  : launch_fmt<RAZER_FMT_ACT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
+    return bf ? launch_fmt<RAZER_FMT_NVFP4, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
+              : launch_fmt<RAZER_FMT_NVFP4, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
 }
 
 }  // namespace razer

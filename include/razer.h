@@ -198,11 +198,14 @@ razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint
  *              X) and the tensor-core pipeline loads both operands by TMA.
  *              For smaller M it is 0 and the weights are decoded per CTA tile
  *              into shared memory (each weight once per 256 rows of X).
- *              When K > 16384 a further M * N * 4 bytes follow: K is then
- *              split into equal chunks of at most 16384, each accumulated
- *              in tensor memory on its own, and the scaled partial sums are
- *              added in fp32 there (one accumulator chain over a longer K
- *              loses precision).
+ *              When K is split, a further S * M * N * 4 bytes follow.  S =
+ *              the number of 16384-long chunks K needs (one tensor-memory
+ *              accumulator chain over a longer K loses precision), raised
+ *              to min(SMs / tiles, K / 512) when the ceil(M/256) *
+ *              ceil(N/256) output tiles cannot occupy the SMs.  The S splits
+ *              run in parallel, each writes its scaled fp32 sum to its own
+ *              [M, N] slice, and a reduction kernel adds the slices in split
+ *              order (deterministic) and converts to out_dt.
  * K must be a multiple of 64 and N a multiple of 16.
  */
 razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes,

@@ -158,13 +158,33 @@ def test_workspace_size_host_logic(lib):
         assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, B, N, K) == max(tma, split_k(B, N, K))
     # other K: split-K partials of the per-warp kernel only
     assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, 4, 4096, 4224) == split_k(4, 4096, 4224)
-    # GEMM: the decoded 16-bit weight copy for M >= 1024, plus fp32 partial
-    # sums of [M, N] when K is longer than one 16384-long accumulation chain
+    # GEMM: the decoded 16-bit weight copy for M >= 1024, plus one fp32 [M, N]
+    # slice per parallel K split: as many splits as 16384-long accumulation
+    # chains K needs, more when the 256x256 output tiles leave SMs idle (each
+    # split keeps at least 8 k-steps of 64); 148 SMs without a GPU
     G = razer.RAZER_OP_GEMM
-    assert razer.razer_workspace_size(G, 1023, 4096, 16384) == 0
-    assert razer.razer_workspace_size(G, 1024, 4096, 16384) == 4096 * 16384 * 2
-    assert razer.razer_workspace_size(G, 512, 8192, 16448) == 512 * 8192 * 4
-    assert razer.razer_workspace_size(G, 2048, 8192, 28672) == 8192 * 28672 * 2 + 2048 * 8192 * 4
+
+    def splits(M, N, K):
+        tiles = -(-M // 256) * -(-N // 256)
+        s = -(-K // 16384)
+        if 0 < tiles < 148:
+            s = max(s, min(148 // tiles, (K // 64) // 8))
+        return max(s, 1)
+
+    def slices(M, N, K):
+        s = splits(M, N, K)
+        return s * M * N * 4 if s > 1 else 0
+
+    assert splits(1023, 4096, 16384) == 2 and splits(8192, 8192, 8192) == 1 and splits(256, 256, 256) == 1
+    assert splits(256, 256, 4096) == 8 and splits(512, 28672, 8192) == 1 and splits(2048, 8192, 28672) == 2
+    assert razer.razer_workspace_size(G, 8192, 8192, 8192) == 8192 * 8192 * 2
+    assert razer.razer_workspace_size(G, 4096, 14336, 4096) == 14336 * 4096 * 2
+    assert razer.razer_workspace_size(G, 256, 256, 256) == 0
+    for M, N, K in ((1023, 4096, 16384), (512, 8192, 16448), (512, 8192, 8192), (256, 256, 4096), (512, 28672, 8192),
+                    (512, 8192, 28672)):
+        assert razer.razer_workspace_size(G, M, N, K) == slices(M, N, K), (M, N, K)
+    assert razer.razer_workspace_size(G, 1024, 4096, 16384) == 4096 * 16384 * 2 + slices(1024, 4096, 16384)
+    assert razer.razer_workspace_size(G, 2048, 8192, 28672) == 8192 * 28672 * 2 + 2 * 2048 * 8192 * 4
     # W4A4: both decoded operands, the K-chunk partials, 16 bytes for ts_a * ts_w
     W4 = razer.RAZER_OP_GEMM_W4A4
     assert razer.razer_workspace_size(W4, 100, 64, 128) == 100 * 128 * 2 + 64 * 128 * 2 + 16
