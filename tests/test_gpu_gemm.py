@@ -28,6 +28,18 @@ def test_gemm_small_single_tile(orc):
     assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
 
 
+@pytest.mark.parametrize("M", [1, 8, 33, 129])
+def test_gemm_fewer_rows_than_a_tile(orc, M):
+    # M below the 128-row TMA box of the activations (the rows past M read
+    # as zeros) and 8192 columns of K split over several CTAs per tile
+    N, K = 512, 8192
+    codes, scales = workloads.random_packed(N, K, "weight", seed=84 + M, max_scale_code=40)
+    X = workloads.vectors(M, K, seed=85, dtype=torch.bfloat16)
+    ref = orc.gemm_ref(oracle_in(X), codes.numpy(), scales.numpy(), 0.03125, 0)
+    Y = gemm(X, codes, scales, 0.03125, "weight")
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
+
+
 @pytest.mark.parametrize("fmt", ["weight", "act", "nvfp4"])
 @pytest.mark.parametrize("xdt", [torch.bfloat16, torch.float16])
 def test_gemm_ragged_multi_tile(orc, fmt, xdt):
