@@ -147,7 +147,7 @@ __host__ __device__ constexpr int var_stage_bytes(int xrows) { return kCodeBytes
 // bs_shift = log2(block / 16).  Byte scales: [N, K / block] bytes; FP16 scale
 // words: [N, K / 128] 16-bit words.
 template <int SF, bool BF16, int NB>
-__global__ void __launch_bounds__(kGemvThreads) gemv_variant_kernel(const uint16_t *__restrict__ x, int B, const uint8_t *__restrict__ codes,
+__global__ void __launch_bounds__(kGemvThreads, NB == 1 ? 8 : (NB == 2 ? 5 : 3)) gemv_variant_kernel(const uint16_t *__restrict__ x, int B, const uint8_t *__restrict__ codes,
                                                                     const uint8_t *__restrict__ scales, int N, int K, int S, int bs_shift,
                                                                     VarTable T, float *__restrict__ ws)
 {
@@ -258,11 +258,25 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_variant_kernel(const uint16
     }
 }
 
-template <int SF, bool BF16>
-static void launch_gemv_variant(const void *x, int B, const uint8_t *codes, const uint8_t *scales, int N, int K, int S, int bs_shift,
-                                VarTable T, float *ws, cudaStream_t st)
+// Split count for a launch: every CTA of the grid resident at once (the
+// 4-warp CTAs have equal work, so a second partial wave would leave SMs
+// half idle), at most S_max (the count the workspace is sized for).
+template <typename Kern>
+static int one_wave_splits(Kern kern, int smem, int N, int S_max)
 {
-    dim3 grid((unsigned)(((N + 15) / 16 + kGemvWarps - 1) / kGemvWarps), (unsigned)S);
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreads, (size_t)smem) != cudaSuccess || occ < 1) occ = 1;
+    const int64_t ctas_x = ((N + 15) / 16 + kGemvWarps - 1) / kGemvWarps;
+    const int64_t s = (int64_t)sm_count() * occ / ctas_x;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(s, S_max));
+}
+
+// Launches the GEMV kernel; returns the split count it used (<= S_max).
+template <int SF, bool BF16>
+static int launch_gemv_variant(const void *x, int B, const uint8_t *codes, const uint8_t *scales, int N, int K, int S_max, int bs_shift,
+                               VarTable T, float *ws, cudaStream_t st)
+{
+    const unsigned gx = (unsigned)(((N + 15) / 16 + kGemvWarps - 1) / kGemvWarps);
     const uint16_t *xp = reinterpret_cast<const uint16_t *>(x);
     const int smem1 = kGemvWarps * kRing * var_stage_bytes(B), smem0 = kGemvWarps * kRing * var_stage_bytes(0);
     static bool attr_done[64] = {false};  // per device: up to 8 activation rows in the ring (> 48 KB)
@@ -273,9 +287,18 @@ static void launch_gemv_variant(const void *x, int B, const uint8_t *codes, cons
                              kGemvWarps * kRing * var_stage_bytes(8));
         attr_done[dev] = true;
     }
-    if (B <= 8) gemv_variant_kernel<SF, BF16, 1><<<grid, kGemvThreads, smem1, st>>>(xp, B, codes, scales, N, K, S, bs_shift, T, ws);
-    else if (B <= 16) gemv_variant_kernel<SF, BF16, 2><<<grid, kGemvThreads, smem0, st>>>(xp, B, codes, scales, N, K, S, bs_shift, T, ws);
-    else gemv_variant_kernel<SF, BF16, 4><<<grid, kGemvThreads, smem0, st>>>(xp, B, codes, scales, N, K, S, bs_shift, T, ws);
+    int S;
+    if (B <= 8) {
+        S = one_wave_splits(gemv_variant_kernel<SF, BF16, 1>, smem1, N, S_max);
+        gemv_variant_kernel<SF, BF16, 1><<<dim3(gx, S), kGemvThreads, smem1, st>>>(xp, B, codes, scales, N, K, S, bs_shift, T, ws);
+    } else if (B <= 16) {
+        S = one_wave_splits(gemv_variant_kernel<SF, BF16, 2>, smem0, N, S_max);
+        gemv_variant_kernel<SF, BF16, 2><<<dim3(gx, S), kGemvThreads, smem0, st>>>(xp, B, codes, scales, N, K, S, bs_shift, T, ws);
+    } else {
+        S = one_wave_splits(gemv_variant_kernel<SF, BF16, 4>, smem0, N, S_max);
+        gemv_variant_kernel<SF, BF16, 4><<<dim3(gx, S), kGemvThreads, smem0, st>>>(xp, B, codes, scales, N, K, S, bs_shift, T, ws);
+    }
+    return S;
 }
 
 static int var_sf(razer_format sfmt) { return sfmt == RAZER_SCALE_F16 ? kVarF16 : (sfmt == RAZER_FMT_WEIGHT ? kVarE3M3 : kVarE4M3); }
@@ -291,20 +314,21 @@ razer_status run_gemv_variant(const void *x, razer_dtype act_dt, int64_t B, cons
                               int bs, razer_format sfmt, const VariantV &V, int64_t N, int64_t K, void *y, razer_dtype out_dt,
                               void *workspace, cudaStream_t st)
 {
-    const int S = gemv_splits(B, N, K);
+    const int S_max = gemv_splits(B, N, K);  // the workspace holds S_max partial sets
     float *ws = reinterpret_cast<float *>(workspace);
     const VarTable T = var_table(V);
     const int sf = var_sf(sfmt), sh = bs_shift_of(bs);
     const bool bf = act_dt == RAZER_BF16;
-#define RAZER_VAR_LAUNCH(SFV)                                                                                                           \
-    do {                                                                                                                                \
-        if (bf) launch_gemv_variant<SFV, true>(x, (int)B, codes, scales, (int)N, (int)K, S, sh, T, ws, st);                            \
-        else launch_gemv_variant<SFV, false>(x, (int)B, codes, scales, (int)N, (int)K, S, sh, T, ws, st);                              \
-    } while (0)
-    if (sf == kVarE3M3) RAZER_VAR_LAUNCH(kVarE3M3);
-    else if (sf == kVarE4M3) RAZER_VAR_LAUNCH(kVarE4M3);
-    else RAZER_VAR_LAUNCH(kVarF16);
-#undef RAZER_VAR_LAUNCH
+    int S;
+    if (sf == kVarE3M3)
+        S = bf ? launch_gemv_variant<kVarE3M3, true>(x, (int)B, codes, scales, (int)N, (int)K, S_max, sh, T, ws, st)
+               : launch_gemv_variant<kVarE3M3, false>(x, (int)B, codes, scales, (int)N, (int)K, S_max, sh, T, ws, st);
+    else if (sf == kVarE4M3)
+        S = bf ? launch_gemv_variant<kVarE4M3, true>(x, (int)B, codes, scales, (int)N, (int)K, S_max, sh, T, ws, st)
+               : launch_gemv_variant<kVarE4M3, false>(x, (int)B, codes, scales, (int)N, (int)K, S_max, sh, T, ws, st);
+    else
+        S = bf ? launch_gemv_variant<kVarF16, true>(x, (int)B, codes, scales, (int)N, (int)K, S_max, sh, T, ws, st)
+               : launch_gemv_variant<kVarF16, false>(x, (int)B, codes, scales, (int)N, (int)K, S_max, sh, T, ws, st);
     const float unbias = sf == kVarE3M3 ? 4096.0f : (sf == kVarE4M3 ? 256.0f : 1.0f);
     const int64_t BN = B * N;
     int64_t g = (BN + 255) / 256;
