@@ -783,7 +783,8 @@ static double generic_qs(const uint8_t *codes, const uint8_t *scales, int64_t K,
         sv = ro_scale_value(sfmt, sb & (sfmt == RO_FMT_WEIGHT ? 0x3f : 0x7f));
         meta = nv > 0 ? (sfmt == RO_FMT_WEIGHT ? sb >> 6 : sb >> 7) : 0;
     }
-    double q = ro_fp4_value(code, nv > 0, nv > 0 ? V[meta] : 0.0);
+    /* a meta value at or past nv (never written by the quantizer) selects 0 */
+    double q = ro_fp4_value(code, nv > 0, (nv > 0 && meta < nv) ? V[meta] : 0.0);
     return q * sv;
 }
 

@@ -645,3 +645,13 @@ def test_gemv_generic_matches_numpy(orc):
     codes, scales, ts, _ = orc.quantize(w.numpy(), 0)
     np.testing.assert_array_equal(orc.gemv_generic(x.numpy(), codes, scales, ts, 16, 0, _DEFAULT_V[0]),
                                   orc.gemm_ref(x.numpy(), codes, scales, ts, 0))
+
+
+def test_dequant_generic_meta_past_the_set(orc):
+    # a scale byte whose meta names no special value (never written by the
+    # quantizer) decodes the 0b1000 code to 0 and leaves the other codes alone
+    codes = np.full((1, 16), 0x18, np.uint8)  # nibbles 8 (low) and 1 (high): 0b1000, 0.5
+    scales = np.array([[24 | (3 << 6), 24 | (1 << 6)]], np.uint8)  # E3M3 1.0, meta 3 / meta 1
+    got = orc.dequant_generic(codes, scales, 1.0, 16, 0, [5.0, -5.0], "f32")
+    np.testing.assert_array_equal(got[0, :16], np.tile([0.0, 0.5], 8).astype(np.float32))
+    np.testing.assert_array_equal(got[0, 16:], np.tile([-5.0, 0.5], 8).astype(np.float32))
