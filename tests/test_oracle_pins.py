@@ -122,6 +122,17 @@ def test_e3m3_encode(orc):
         assert orc.scale_encode(0, p) == 0x3F
 
 
+def test_e3m3_code_is_e4m3_code_of_sixteenth(orc):
+    # the GPU quantizer encodes an E3M3 scale with the hardware E4M3 convert:
+    # code = min(E4M3(s_f / 16), 63) -- the same grid scaled by 2^-4 in both
+    # the normal and the subnormal range (torch's float32 -> E4M3 is RNE)
+    pts = _adversarial_scales(30.0, 4000, 2) + [30.5, 31.0, 31.999]
+    t = torch.tensor(pts, dtype=torch.float32) / 16
+    c4 = t.to(torch.float8_e4m3fn).view(torch.uint8).numpy().astype(int)
+    for p, c in zip(pts, c4):
+        assert orc.scale_encode(0, p) == min(c, 0x3F), p
+
+
 # ----------------------------------------------------------------------------
 # element grid
 # ----------------------------------------------------------------------------
