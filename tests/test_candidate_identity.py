@@ -6,7 +6,8 @@ squared error of an element by
     d(xs) = (r5 - xs)^2 - (q - xs)^2,
 
 where q is the nearest grid point and r5 the nearest point of the grid plus
-5, both with ties to the smaller magnitude.  The kernel computes, in binary32,
+5, both with ties to the smaller magnitude.  The kernel computes, in
+binary32,
 
     t(xs) = sat(1 - |2|xs| - 10|)        (sat clamps to [0, 1])
 
@@ -15,6 +16,10 @@ for EVERY binary32 in [4, 8) (d is computed exactly in float64 from its
 definition) and that t vanishes on [2, 4) and [8, 16), where 5 is never the
 nearest point.  Every t is a multiple of 2^-20 in [0, 1], so a block's 16
 terms and their signed sums are exact binary32 sums in any order.
+
+For blocks with a subnormal scale code (|xs| <= 9) the kernel also tries
+v = 8, with the term min(28 - 4 xs, 0) from one FMA, and sums every term as
+an integer in units of 2^-20; the last test checks that form on [2, 16).
 """
 import numpy as np
 
@@ -67,3 +72,33 @@ def test_candidate_term_vanishes_outside():
 def test_candidate_term_values():
     a = np.array([4.5, 4.75, 5.0, 5.25, 5.5], np.float32)
     assert t_kernel(a).tolist() == [0.0, 0.5, 1.0, 0.5, 0.0]
+
+
+def delta_exact_v(a32, v):
+    a = a32.astype(np.float64)
+    q = nearest_ties_smaller(a, GRID)
+    r = nearest_ties_smaller(a, np.sort(np.append(GRID, v)))
+    return (r - a) ** 2 - (q - a) ** 2
+
+
+def t8_kernel(a32):
+    return np.minimum((np.float64(-4) * a32.astype(np.float64) + 28.0).astype(np.float32), np.float32(0))
+
+
+def t5_signed_kernel(a32):
+    # the integer-sum form of the +5 term: min(|2 xs - 10| - 1, 0)
+    e = (np.float32(2) * a32 - np.float32(10)).astype(np.float32)
+    return np.minimum((np.abs(e) - np.float32(1)).astype(np.float32), np.float32(0))
+
+
+def test_eight_term_exhaustive():
+    for e in (1, 2, 3):  # [2, 16): every binary32
+        a = binade(e)
+        t8 = t8_kernel(a)
+        assert np.array_equal(delta_exact_v(a, 8.0), t8.astype(np.float64))
+        units = t8.astype(np.float64) * 2.0 ** 20
+        assert np.array_equal(units, np.round(units))  # integers in units of 2^-20
+        t5 = t5_signed_kernel(a)
+        assert np.array_equal(delta_exact_v(a, 5.0), t5.astype(np.float64))
+        units5 = t5.astype(np.float64) * 2.0 ** 20
+        assert np.array_equal(units5, np.round(units5))
