@@ -340,14 +340,20 @@ razer_status razer_dequant_variant(const uint8_t *codes, const uint8_t *scales, 
     return run_dequant_variant(codes, scales, ts, R, K, block, scale_fmt, V, out, out_dt, (cudaStream_t)stream);
 }
 
-// a special value whose doubled magnitude has 5 significant bits (8.5, 9.5):
-// q * s then needs up to 9 bits, more than bf16 holds
-static bool needs_five_bits(const VariantV &V)
+// whether v * s can need more than the 8 significant bits of bf16 for some
+// scale: the odd part of 2|v| times every scale significand (1..15, the
+// E3M3 / E4M3 mantissa with its leading bit, or a subnormal one) must stay
+// below 256.  Of the allowed values only 9.5 (19 * 15 = 285) fails.
+static bool rounds_in_bf16(const VariantV &V)
 {
     for (int i = 0; i < V.nv; i++) {
         int h = (int)(fabsf(V.v[i]) * 2.0f);
         while (h > 0 && (h & 1) == 0) h >>= 1;
-        if (h >= 16) return true;
+        for (int m = 1; m <= 15; m++) {
+            int p = h * m;
+            while (p > 0 && (p & 1) == 0) p >>= 1;
+            if (p >= 256) return true;
+        }
     }
     return false;
 }
@@ -364,7 +370,7 @@ razer_status razer_gemv_variant(const void *x, razer_dtype act_dt, int64_t B, co
     if (!in16(act_dt)) return RAZER_ERR_DTYPE;
     if (B < 1 || B > 32 || K % 128 != 0 || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
     if (scale_fmt == RAZER_SCALE_F16 && block != 128) return RAZER_ERR_UNSUPPORTED;
-    if (scale_fmt != RAZER_SCALE_F16 && act_dt == RAZER_BF16 && needs_five_bits(V)) return RAZER_ERR_UNSUPPORTED;
+    if (scale_fmt != RAZER_SCALE_F16 && act_dt == RAZER_BF16 && rounds_in_bf16(V)) return RAZER_ERR_UNSUPPORTED;
     if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ts, 4) || !aligned(codes, 16) ||
         (scale_fmt == RAZER_SCALE_F16 && !aligned(scales, 2)))
         return RAZER_ERR_ALIGN;

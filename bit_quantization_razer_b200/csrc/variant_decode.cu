@@ -14,8 +14,8 @@
 //     significant bits, s at most 4) -- so the MMA sees exact operands and the
 //     scale is applied before it, as in the 16-element kernel.  For bf16
 //     activations the operand must be bf16 (8 significant bits), which holds
-//     only when no special value needs 5 bits (+-8.5, +-9.5); such sets are
-//     refused for bf16 activations;
+//     for every allowed value except +-9.5 (19 * 15 = 285 needs 9 bits); sets
+//     with it are refused for bf16 activations;
 //   * FP16 scale words (11 significant bits): q * s is not an fp16 value, so
 //     the MMA multiplies the exact q and the scale multiplies each block's
 //     fp32 partial sum afterwards.  A 128-k slice is one block, so every MMA

@@ -362,9 +362,10 @@ razer_status razer_dequant_variant(const uint8_t *codes, const uint8_t *scales, 
  * razer_workspace_size(RAZER_OP_GEMV, B, N, K) bytes (16-byte aligned; NULL
  * when that is 0), contents ignored.  K % 128 == 0; codes 16-byte aligned.
  * Byte scales (RAZER_FMT_WEIGHT / ACT / NVFP4): any block; the decoded
- * weights q*s enter the tensor-core MMA exactly, so bf16 activations with a
- * special value of 5 significant bits (+-8.5, +-9.5) give
- * RAZER_ERR_UNSUPPORTED (the operand would round in bf16).
+ * weights q*s enter the tensor-core MMA exactly, so bf16 activations with
+ * +-9.5 in the set give RAZER_ERR_UNSUPPORTED (9.5 times a scale of
+ * significand 1.875 needs 9 significant bits; every other allowed value
+ * fits the 8 of bf16).
  * RAZER_SCALE_F16: block 128 only (others RAZER_ERR_UNSUPPORTED); the MMA
  * sums q * x and each block's fp32 sum is multiplied by its scale.
  */

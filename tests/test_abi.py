@@ -122,9 +122,9 @@ def test_variant_decode_validation(lib):
     assert g(*gargs(B=33)) == 2
     assert g(*gargs(act=2)) == 4                                       # f32 activations
     assert g(*gargs(block=64, sfmt=4)) == 6                            # FP16 scale words: block 128 only
-    assert g(*gargs(V=(5.0, -5.0, 9.5, -9.5), act=1)) == 6             # bf16 operand would round
-    assert g(*gargs(V=(5.0, -5.0, 8.5, -8.5), act=1)) == 6
-    assert g(*gargs(V=(5.0, -5.0, 9.0, -9.0), act=1)) == 5             # 4 significant bits: allowed (no workspace)
+    assert g(*gargs(V=(5.0, -5.0, 9.5, -9.5), act=1)) == 6             # bf16 operand would round (19 * 15 = 285)
+    assert g(*gargs(V=(5.0, -5.0, 8.5, -8.5), act=1)) == 5             # 17 * 15 = 255 fits: allowed (no workspace)
+    assert g(*gargs(V=(5.0, -5.0, 9.0, -9.0), act=1)) == 5
     assert g(*gargs(V=(5.0, -5.0, 9.5, -9.5), act=0)) == 5             # fp16 operands are exact
     assert g(*gargs(block=128, sfmt=4, V=(9.5, -9.5), act=1)) == 5     # q alone enters the MMA
     assert g(*gargs(block=128, sfmt=4, scales=ODD)) == 3               # 16-bit scale words
