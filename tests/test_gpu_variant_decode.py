@@ -93,6 +93,17 @@ def test_gemv_variant_types(orc, block, fmt, V, xdt, out_dtype):
     assert_close_typed(y, r)
 
 
+def test_gemv_variant_bf16_with_eight_and_a_half(orc):
+    # 8.5 times every scale significand fits bf16's 8 bits: allowed and exact
+    N, K = 80, 512
+    V = [5.0, -5.0, 8.5, -8.5]
+    codes, scales = workloads.random_packed_variant(N, K, 16, "weight", 4, seed=103)
+    x = workloads.vectors(3, K, seed=104, dtype=torch.bfloat16)
+    y = R.razer_gemv_variant(x.to(DEV), *_dev(codes, scales), _ts(0.0625), 16, "weight", V)
+    r = orc.gemv_generic(oracle_in(x), codes.numpy(), scales.numpy(), 0.0625, 16, 0, V)
+    assert rel_err(y.cpu().numpy(), r) <= REL_TOL
+
+
 def test_gemv_variant_bf16_with_nine_and_a_half_is_refused():
     codes, scales = workloads.random_packed_variant(16, 128, 16, "weight", 4, seed=96)
     x = workloads.vectors(1, 128, seed=97, dtype=torch.bfloat16)
