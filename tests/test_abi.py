@@ -34,6 +34,21 @@ def test_exports_every_declared_symbol(lib):
         assert n in names
 
 
+def test_plain_c_consumer(lib, tmp_path):
+    # the header compiles as C99 with every warning an error, and a C program
+    # linked against the library gets the documented statuses
+    import subprocess
+
+    libdir = os.path.join(ROOT, "bit_quantization_razer_b200")
+    exe = str(tmp_path / "abi_consumer")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "abi_consumer.c"), "-L", libdir, "-lrazer", "-Wl,-rpath," + libdir,
+                    "-o", exe], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert "all checks passed" in out.stdout
+
+
 def test_status_strings(lib):
     for s in range(9):
         assert razer.razer_status_string(s)
