@@ -145,7 +145,9 @@ __device__ __forceinline__ void var_slice_postscaled(const uint4 &ca, const uint
 __host__ __device__ constexpr int var_stage_bytes(int xrows) { return kCodeBytes + xrows * kXRowBytes; }
 
 // bs_shift = log2(block / 16).  Byte scales: [N, K / block] bytes; FP16 scale
-// words: [N, K / 128] 16-bit words.
+// words: [N, K / 128] 16-bit words.  Launch bounds: the B <= 8 kernel fits 64
+// registers without spilling (8 CTAs per SM); the B <= 16 and B <= 32 kernels
+// keep their natural register counts (about 90 and 150).
 template <int SF, bool BF16, int NB>
 __global__ void __launch_bounds__(kGemvThreads, NB == 1 ? 8 : (NB == 2 ? 5 : 3)) gemv_variant_kernel(const uint16_t *__restrict__ x, int B, const uint8_t *__restrict__ codes,
                                                                     const uint8_t *__restrict__ scales, int N, int K, int S, int bs_shift,
