@@ -666,3 +666,56 @@ def test_dequant_generic_meta_past_the_set(orc):
     got = orc.dequant_generic(codes, scales, 1.0, 16, 0, [5.0, -5.0], "f32")
     np.testing.assert_array_equal(got[0, :16], np.tile([0.0, 0.5], 8).astype(np.float32))
     np.testing.assert_array_equal(got[0, 16:], np.tile([-5.0, 0.5], 8).astype(np.float32))
+
+
+def _nearest_with_tie_rule(xs: Fraction, v):
+    """Nearest point of Q_FP4 (and v when given) to xs; ties to the smaller
+    magnitude.  Returns (value, code) with 0 encoded as 0b0000 and v as 0b1000."""
+    cands = [(m, c) for c, m in enumerate(MAGS)] + [(-m, c | 8) for c, m in enumerate(MAGS) if m != 0]
+    if v is not None:
+        cands.append((Fraction(v), 8))
+    best = min(cands, key=lambda pc: (abs(xs - pc[0]), abs(pc[0])))
+    return best[0], (0 if best[0] == 0 else best[1])
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_full_blocks_exact_argmin(orc, fmt):
+    # all 16 elements in play: given v each element's best point is
+    # independent, so the exact SSE of every candidate is a sum of per-element
+    # minima (rationals); the oracle's meta must be the argmin (ties: lowest
+    # index) and its codes the nearest points under the tie rule
+    rng = np.random.default_rng(70 + fmt)
+    specials = [orc.special_value(fmt, m) for m in range(orc.num_specials(fmt))]
+    mids = np.array(ADV, np.float32)
+    checked, picks = 0, {}
+    for i in range(300):
+        x = rng.standard_normal(16).astype(np.float32)
+        k = rng.integers(0, 8)  # some elements on grid midpoints (+-1 ulp) of xs
+        x[:k] = rng.choice(mids, k) * rng.choice([-1.0, 1.0], k)
+        x *= np.float32(rng.uniform(0.2, 1.5))
+        if fmt == 0 and i % 2:
+            # s_f just below a subnormal code midpoint, (m + 0.3..0.49) / 32 with
+            # m = 1, 2: the scale rounds down to m / 32, so the block amax
+            # lands at |xs| in (7, 9) and +-8 competes
+            m = int(rng.integers(1, 3))
+            ts = np.float32(np.abs(x).max() / (6 * (m + rng.uniform(0.3, 0.49)) / 32))
+        else:
+            ts = np.float32(rng.uniform(0.05, 0.5))
+        codes, sb, xs, _ = orc.quantize_block(x, float(ts), fmt)
+        if (sb & (0x3F if fmt == 0 else 0x7F)) == 0:
+            assert all(c == 0 for c in codes)
+            continue
+        xsf = [Fraction(float(t)) for t in xs]
+        sse = []
+        for v in (specials or [None]):
+            sse.append(sum((t - _nearest_with_tie_rule(t, v)[0]) ** 2 for t in xsf))
+        meta = min(range(len(sse)), key=lambda m: (sse[m], m))
+        got_meta = (sb >> 6) if fmt == 0 else ((sb >> 7) if fmt == 1 else 0)
+        assert got_meta == meta, (i, sse)
+        v = specials[meta] if specials else None
+        assert list(codes) == [_nearest_with_tie_rule(t, v)[1] for t in xsf], i
+        picks[meta] = picks.get(meta, 0) + 1
+        checked += 1
+    assert checked > 250
+    if fmt == 0:
+        assert picks.get(2, 0) + picks.get(3, 0) >= 10, picks  # +-8 really competes
