@@ -1,7 +1,9 @@
 // extern "C" surface of the RaZeR library: argument validation, then the
 // launches of the kernels in quantize.cu / dequant.cu / gemv.cu / gemm.cu.
 // No call allocates memory or synchronises (razer_get_device_status excepted).
+#include <atomic>
 #include <cmath>
+#include <cstdlib>
 
 #include "razer_internal.cuh"
 #include "variant.cuh"
@@ -22,6 +24,15 @@ int sm_count()
 }
 
 razer_status last_launch_status() { return cudaGetLastError() == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA; }
+
+// Off unless razer_debug_set_fault_injection turns it on; the environment
+// variable RAZER_FAULT_INJECT_STALL=1 sets the initial value, read once when
+// the library is loaded.
+static std::atomic<int> g_fault_injection{[] {
+    const char *v = getenv("RAZER_FAULT_INJECT_STALL");
+    return (v && v[0] == '1') ? 1 : 0;
+}()};
+bool fault_injection_enabled() { return g_fault_injection.load(std::memory_order_relaxed) != 0; }
 
 razer_status run_quantize(const void *x, razer_dtype dt, int64_t R, int64_t K, const float *ts_in, uint8_t *codes,
                           uint8_t *scales, float *ts_out, unsigned long long *hist, razer_format fmt, cudaStream_t st);
@@ -424,6 +435,11 @@ const char *razer_status_string(razer_status s)
     return "unknown status";
 }
 
-int razer_version(void) { return 100; }
+int razer_version(void) { return 200; }
+
+int razer_debug_set_fault_injection(int on)
+{
+    return g_fault_injection.exchange(on ? 1 : 0, std::memory_order_relaxed);
+}
 
 }  // extern "C"

@@ -614,10 +614,9 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, cons
     }
     const unsigned nt = (unsigned)((N + BN - 1) / BN), mt = (unsigned)((M + BM - 1) / BM);
     const dim3 grid = DECODED ? dim3(mt, nt, (unsigned)splits) : dim3(nt, mt, (unsigned)splits);
-    // RAZER_FAULT_INJECT_STALL=1 (tests only) withholds one decoder warp's
-    // arrivals so that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
-    const char *inj = getenv("RAZER_FAULT_INJECT_STALL");
-    const int inject = (inj && inj[0] == '1') ? 1 : 0;
+    // fault injection (tests only) withholds one decoder warp's arrivals so
+    // that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
+    const int inject = fault_injection_enabled() ? 1 : 0;
     gemm_kernel<FMT, BF16, DECODED><<<grid, kThreads, SMEM_BYTES, st>>>(map, wmap, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt,
                                                                       kb0, nkb, addend, inject);
     return last_launch_status();

@@ -147,10 +147,14 @@ __device__ __forceinline__ BlockOut quantize_block(const float (&x)[16], const S
     const float d = k.tab_d[sc];  // dec(sc) * ts
     if (!FAST && (sc == 0u || d == 0.0f)) return o;
 
-    // X^scaled = RN(x / d)
+    // X^scaled = RN(x / d).  Markstein's correction needs its intermediates in
+    // the normal range: with a caller-given ts a saturated block scale can
+    // leave x / d near or past the binary32 maximum (bf16 input only: an fp16
+    // amax is at most 65504), so such blocks take the IEEE divide (which
+    // overflows to inf like the oracle's quotient).
     float xs[16];
     const float y = k.tab_y[sc];  // RN(1/d), or 0 outside the Markstein range
-    if (FAST || y != 0.0f) {
+    if ((FAST || y != 0.0f) && (F16IN || __fmul_rn(amax, y) <= 0x1p126f)) {
         const float2 y2 = make_float2(y, y), nd2 = make_float2(-d, -d);
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {

@@ -162,4 +162,7 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 
 int sm_count();
 razer_status last_launch_status();
+// Test-only fault injection (razer_debug_set_fault_injection): a plain load
+// on the launch path, no environment lookup per call.
+bool fault_injection_enabled();
 }  // namespace razer

@@ -34,7 +34,7 @@ EXPORTED = (
     "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4", "razer_gemm_w4a4_online", "razer_quant_error",
     "razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
-    "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch",
+    "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch", "razer_debug_set_fault_injection",
 )
 
 
@@ -90,6 +90,8 @@ def load() -> ctypes.CDLL:
     L.razer_status_string.argtypes = [i32]
     L.razer_status_string.restype = ctypes.c_char_p
     L.razer_version.argtypes = []
+    L.razer_debug_set_fault_injection.argtypes = [i32]
+    L.razer_debug_set_fault_injection.restype = ctypes.c_int
     for fn in ("razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant", "razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
@@ -369,3 +371,9 @@ def razer_status_string(status: int) -> str:
 
 def razer_version() -> int:
     return int(load().razer_version())
+
+
+def razer_debug_set_fault_injection(on: bool) -> bool:
+    """Test-only: turns the GEMV / GEMM stall injection on or off; returns
+    the previous setting."""
+    return bool(load().razer_debug_set_fault_injection(1 if on else 0))

@@ -384,8 +384,11 @@ razer_status razer_gemv_variant(const void *x, razer_dtype act_dt, int64_t B, co
  * inside the library instead (razer_gemv_noalloc_max_scratch() bytes, held on
  * every GPU that loads the library until the process exits).
  *   - It allocates nothing.  Its first call on a device looks up the device
- *     address of the array (with that device current); make that first call
- *     before any stream capture.
+ *     address of the array (with that device current), and so does its first
+ *     call after the device's context is re-created (e.g. by cudaDeviceReset);
+ *     make that first call before any stream capture.
+ *   - Arguments are checked as razer_gemv checks them; K = 0 writes y = 0 and
+ *     N = 0 writes nothing (null x / y are then allowed).
  *   - Sizes whose scratch need (razer_workspace_size(RAZER_OP_GEMV, B, N, K))
  *     exceeds the maximum are rejected with RAZER_ERR_WORKSPACE.
  *   - All calls on a device share the array and it keeps the last call's
@@ -418,6 +421,20 @@ const char *razer_status_string(razer_status status);
 
 /* Library version, as major*10000 + minor*100 + patch. */
 int razer_version(void);
+
+/*
+ * razer_debug_set_fault_injection -- for tests of the failure path only (the
+ * paper has no counterpart).  While on (on != 0), each launch of the
+ * bulk-tensor razer_gemv kernel leaves one pipeline stage of one CTA unfilled
+ * and each razer_gemm launch withholds one decoder warp's arrivals, so their
+ * bounded waits expire: the call still returns RAZER_OK and
+ * razer_get_device_status then reports RAZER_ERR_TIMEOUT; outputs of such a
+ * call are void.  No GPU fault, trap or hang results.  Returns the previous
+ * setting.  The initial setting is 1 when the environment variable
+ * RAZER_FAULT_INJECT_STALL is "1" when the library is loaded, else 0.
+ * Process-wide; not meant to be toggled while other threads launch.
+ */
+int razer_debug_set_fault_injection(int on);
 
 #ifdef __cplusplus
 }

@@ -98,7 +98,7 @@ def test_gemm_k_zero_and_errors():
         R.razer_gemm(torch.zeros(8, 96, dtype=torch.bfloat16, device=DEV), c.to(DEV), s.to(DEV), torch.ones(1, device=DEV))
 
 
-def test_gemm_bounded_wait_times_out_and_reports(monkeypatch):
+def test_gemm_bounded_wait_times_out_and_reports():
     """A decoder warp that never arrives (host-side fault injection) makes the
     MMA thread's bounded wait expire: the kernel stops, frees its tensor
     memory, and the device status word reports RAZER_ERR_TIMEOUT; the context
@@ -108,10 +108,12 @@ def test_gemm_bounded_wait_times_out_and_reports(monkeypatch):
     c, s = codes.to(DEV), scales.to(DEV)
     ts = torch.ones(1, device=DEV)
     assert R.razer_get_device_status() == 0
-    monkeypatch.setenv("RAZER_FAULT_INJECT_STALL", "1")
-    R.razer_gemm(X, c, s, ts, "weight", torch.float32)
+    R.razer_debug_set_fault_injection(True)
+    try:
+        R.razer_gemm(X, c, s, ts, "weight", torch.float32)
+    finally:
+        R.razer_debug_set_fault_injection(False)
     assert R.razer_get_device_status() == 7  # RAZER_ERR_TIMEOUT, read and cleared
-    monkeypatch.delenv("RAZER_FAULT_INJECT_STALL")
     assert R.razer_get_device_status() == 0
     # the next call works normally
     Y = R.razer_gemm(X, c, s, ts, "weight", torch.float32)

@@ -170,6 +170,25 @@ def test_quantize_acts_static_scale(orc):
         np.testing.assert_array_equal(h, oh[[0, 1, 4, 5]].astype(np.int64))
 
 
+def test_quantize_acts_static_scale_huge_bf16(orc):
+    # a caller-given ts far below the data: every block scale saturates and
+    # X^scaled of the blocks scaled by 2^100 overflows binary32 (inf, rounded
+    # to +-6 like any value above the grid); ts = 2^-60 is inside the
+    # launch-wide fast range, 2^-80 outside it with divisors still inside the
+    # corrected-reciprocal range
+    x = workloads.outlier_activations(64, 1024, seed=304).float()
+    x[::3, 16:48] *= 2.0 ** 100
+    x[1::5, 512:528] *= -(2.0 ** 120)
+    x = x.to(torch.bfloat16)
+    for ts_val in (2.0 ** -60, 2.0 ** -80):
+        oc, os_, _, oh = orc.quantize(oracle_in(x), 1, ts=ts_val)
+        ts_in = torch.tensor([ts_val], dtype=torch.float32, device=DEV)
+        c, s, t, h = quantize_gpu(x, "act", ts_in=ts_in)
+        np.testing.assert_array_equal(c, oc)
+        np.testing.assert_array_equal(s, os_)
+        np.testing.assert_array_equal(h, oh[[0, 1, 4, 5]].astype(np.int64))
+
+
 def test_quantize_acts_nvfp4(orc):
     x = workloads.outlier_activations(64, 1024, seed=303)
     oc, os_, ots, _ = orc.quantize(oracle_in(x), 2)
