@@ -244,7 +244,40 @@ def cpu_baseline_sample():
         res["all_cores"] = cpu_baseline_all_cores(ws, x, rows)
     except Exception as e:  # the single-thread figure stands on its own
         res["all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"}
+    try:
+        res["gemm"] = cpu_gemm_sample()
+    except Exception as e:
+        res["gemm"] = {"unavailable": f"{type(e).__name__}: {e}"}
     return res
+
+
+def cpu_gemm_sample():
+    """The oracle's GEMM reference (double accumulation, single thread) on the
+    prefill GEMM shapes: timed on two sampled row counts, and the full
+    product's time extrapolated from the fit (a fixed part -- the oracle
+    decodes the weights once per call -- plus a part per row of X), labelled
+    as an extrapolation."""
+    import oracle
+    import torch
+    from bit_quantization_razer_b200 import workloads
+
+    out = {}
+    for M, N, K, r1, r2 in ((4096, 4096, 4096, 4, 20), (4096, 14336, 4096, 2, 6)):
+        codes, scales = workloads.random_packed(N, K, "weight", seed=N + K, max_scale_code=40)
+        t = []
+        for rows in (r1, r2):
+            X = workloads.vectors(rows, K, seed=M + rows, dtype=torch.bfloat16)
+            xb = oracle.Bf16Bits(workloads.to_numpy_bits(X))
+            t0 = time.perf_counter()
+            oracle.gemm_ref(xb, codes.numpy(), scales.numpy(), 0.01, 0)
+            t.append(time.perf_counter() - t0)
+        per_row = max((t[1] - t[0]) / (r2 - r1), 1e-12)
+        fixed = max(t[0] - r1 * per_row, 0.0)
+        full = fixed + M * per_row
+        out[f"{M}x{N}x{K}"] = {"value": 2.0 * M * N * K / full / 1e9, "unit": "GFLOP/s", "cores": 1, "kind": "oracle",
+                               "extrapolated": True, "extrapolated_full_s": full,
+                               "sample": f"{r1} and {r2} rows of {M} timed ({t[0]:.2f} s, {t[1]:.2f} s), fixed + per-row fit"}
+    return out
 
 
 def _oracle_rows_worker(rank, nproc, ws, x, rows, tsbuf, start, mid, done):
@@ -489,7 +522,13 @@ def main():
                                                     "reduce kernels)"),
                 "algorithmic_bytes_per_call": dom_bytes / n_calls, "peak_source": peak_src,
                 "nominal_peak": 8000.0, "frac_nominal": achieved / 8000.0,
-                "timing": "CUDA events around CUDA-graph replays of back-to-back calls on operand copies larger than L2"}
+                "timing": "CUDA events around CUDA-graph replays of at least 50 back-to-back calls on operand copies "
+                          "larger than L2 (median of 5 replays)"}
+    if traffic:
+        # the same time against the DRAM bytes ncu counted for one call (a
+        # pass may find part of its matrix still in L2 from the previous pass)
+        dram = traffic / (dom_ms / n_calls) / 1e6
+        roofline.update({"dram_achieved": dram, "dram_frac": dram / hbm, "dram_frac_nominal": dram / 8000.0})
 
     extras = {}
     if not args.no_extras and rank == 0:
@@ -619,12 +658,12 @@ def run_single_kernel(args):
 
 def time_graph(fn, ncalls, stream, reps=5):
     """Median device time of one call in a back-to-back sequence: fn() issues
-    `ncalls` calls; fn() is captured enough times for at least 8 calls per
+    `ncalls` calls; fn() is captured enough times for at least 50 calls per
     CUDA graph (so the graph launch itself is amortised), and the graph is
     replayed `reps` times between events."""
     import torch
 
-    inner = max(1, -(-8 // ncalls))
+    inner = max(1, -(-50 // ncalls))
     fn()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()

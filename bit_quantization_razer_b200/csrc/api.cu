@@ -172,7 +172,7 @@ razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint
     if (!in16(act_dt)) return RAZER_ERR_DTYPE;
     razer_status st = check_packed(codes, scales, N, K);
     if (st != RAZER_OK) return st;
-    if (B < 1 || B > 32 || K % 128 != 0 || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (B < 1 || B > 32 || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
     if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ts, 4)) return RAZER_ERR_ALIGN;
     if (N == 0) return RAZER_OK;
     if (K == 0)  // empty sums: y = 0
@@ -205,7 +205,7 @@ razer_status razer_gemv_batch(int count, const razer_gemv_problem *problems, raz
         if (!p.ts || (!p.x && p.K > 0) || (!p.y && p.N > 0)) return RAZER_ERR_INVALID_ARG;
         razer_status st = check_packed(p.codes, p.scales, p.N, p.K);
         if (st != RAZER_OK) return st;
-        if (p.B < 1 || p.B > 32 || p.K % 128 != 0 || p.N > INT32_MAX || p.K > INT32_MAX) return RAZER_ERR_SHAPE;
+        if (p.B < 1 || p.B > 32 || p.N > INT32_MAX || p.K > INT32_MAX) return RAZER_ERR_SHAPE;
         if (!aligned(p.x, 16) || !aligned(p.y, 16) || !aligned(p.ts, 4)) return RAZER_ERR_ALIGN;
     }
     const size_t need = gemv_batch_workspace_bytes(count, problems);
@@ -225,7 +225,7 @@ razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint
     if (!in16(act_dt)) return RAZER_ERR_DTYPE;
     razer_status st = check_packed(codes, scales, N, K);
     if (st != RAZER_OK) return st;
-    if (M < 0 || K % 64 != 0 || N % 16 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (M < 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
     if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ts, 4)) return RAZER_ERR_ALIGN;
     if (M == 0 || N == 0) return RAZER_OK;
     const size_t need = gemm_workspace_bytes(M, N, K);
@@ -246,7 +246,7 @@ razer_status razer_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, co
     if (st != RAZER_OK) return st;
     st = check_packed(codes_w, scales_w, N, K);
     if (st != RAZER_OK) return st;
-    if (K % 64 != 0 || N % 16 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
     if (!aligned(Y, 16) || !aligned(ts_a, 4) || !aligned(ts_w, 4)) return RAZER_ERR_ALIGN;
     if (M == 0 || N == 0) return RAZER_OK;
     const size_t need = K > 0 ? gemm_w4a4_workspace_bytes(M, N, K) : 0;
@@ -272,7 +272,7 @@ razer_status razer_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, 
     if (st != RAZER_OK) return st;
     st = check_packed(codes_w, scales_w, N, K);
     if (st != RAZER_OK) return st;
-    if (M < 0 || K % 64 != 0 || N % 16 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (M < 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
     if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ts_a_out, 4) || !aligned(ts_w, 4) || (ts_in && !aligned(ts_in, 4)) ||
         (meta_hist && !aligned(meta_hist, 8)))
         return RAZER_ERR_ALIGN;

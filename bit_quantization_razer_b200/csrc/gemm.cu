@@ -375,8 +375,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int n = n0 + c0;
                     if (m < M && n < N) {
                         const int cnt = min(32, N - n);
+                        // 16-byte vector accesses need rows of N % 4 (fp32) / N % 8 (16-bit) elements
+                        const bool vec = out_dt == RAZER_F32 ? (N & 3) == 0 : (N & 7) == 0;
                         const float *add = addend ? addend + (size_t)m * N + n : nullptr;
-                        if (add && cnt == 32) {
+                        if (add && cnt == 32 && (N & 3) == 0) {
 #pragma unroll
                             for (int i = 0; i < 8; i++) {
                                 const float4 t = reinterpret_cast<const float4 *>(add)[i];
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int i = 0; i < 32; i++) v[i] = (add && i < cnt) ? __fmaf_rn(v[i], scale, add[i]) : v[i] * scale;
                         }
-                        if (cnt < 32) {
+                        if (cnt < 32 || !vec) {
                             for (int i = 0; i < cnt; i++) {
                                 const float a = v[i];
                                 if (out_dt == RAZER_F32) reinterpret_cast<float *>(Y)[(size_t)m * N + n + i] = a;
@@ -550,7 +552,14 @@ constexpr int64_t kMaxChainK = RAZER_GEMM_CHAIN_K;
 static_assert(kMaxChainK % BK == 0, "chain length must be whole k-steps");
 
 static int64_t num_chunks(int64_t K) { return (K + kMaxChainK - 1) / kMaxChainK; }
-static size_t decoded_bytes(int64_t M, int64_t N, int64_t K) { return M >= kDecodedMinM ? (size_t)N * (size_t)K * 2 : 0; }
+// Shapes the fused decoders cannot stream (K % 64 != 0: a row's last k-step
+// is partial; N % 16 != 0) take the decode-once path: the bulk-tensor copies
+// zero-fill past K and past N, so the k-steps simply run to ceil(K / 64).
+static bool gemm_generic(int64_t N, int64_t K) { return K % BK != 0 || N % 16 != 0; }
+static size_t decoded_bytes(int64_t M, int64_t N, int64_t K)
+{
+    return (M >= kDecodedMinM || gemm_generic(N, K)) ? (size_t)N * (size_t)K * 2 : 0;
+}
 static size_t partial_bytes(int64_t M, int64_t N, int64_t K) { return num_chunks(K) > 1 ? (size_t)M * (size_t)N * 4 : 0; }
 
 // Parallel K splits of razer_gemm: at least the number of accumulation chains
@@ -598,6 +607,21 @@ __global__ void __launch_bounds__(256) gemm_splits_reduce_kernel(const float4 *_
     }
 }
 
+// the same for any element count (rows of N % 4 != 0 elements are not
+// 16-byte aligned)
+template <typename TOut>
+__global__ void __launch_bounds__(256) gemm_splits_reduce1_kernel(const float *__restrict__ part, int S, int64_t n, TOut *__restrict__ Y)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        float a = part[i];
+        for (int z = 1; z < S; z++) a += part[(size_t)z * (size_t)n + (size_t)i];
+        if constexpr (sizeof(TOut) == 4) Y[i] = a;
+        else if constexpr (std::is_same<TOut, __half>::value) Y[i] = __float2half_rn(a);
+        else Y[i] = __float2bfloat16_rn(a);
+    }
+}
+
 template <int FMT, bool BF16, bool DECODED>
 static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, const uint8_t *codes, const uint8_t *scales, const float *ts,
                            float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, int kb0, int nkb, const float *addend,
@@ -634,14 +658,22 @@ static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, 
             cudaSuccess)
             return RAZER_ERR_CUDA;
     }
-    const int KB = K / BK;
+    const int KB = (K + BK - 1) / BK;  // the last k-step of a generic K is zero-filled past K
     const int S = gemm_splits(M, N, K);
     void *out = S > 1 ? static_cast<void *>(slices) : Y;
     const razer_dtype odt = S > 1 ? RAZER_F32 : out_dt;
     const razer_status r = decoded ? launch<FMT, BF16, true>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S)
                                    : launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S);
     if (r != RAZER_OK || S == 1) return r;
-    const int64_t n4 = (int64_t)M * N / 4;  // N % 16 == 0
+    if (N % 4 != 0) {
+        const int64_t n1 = (int64_t)M * N;
+        const int64_t g = std::max<int64_t>(1, std::min<int64_t>((n1 + 255) / 256, (int64_t)sm_count() * 8));
+        if (out_dt == RAZER_F32) gemm_splits_reduce1_kernel<float><<<(unsigned)g, 256, 0, st>>>(slices, S, n1, reinterpret_cast<float *>(Y));
+        else if (out_dt == RAZER_F16) gemm_splits_reduce1_kernel<__half><<<(unsigned)g, 256, 0, st>>>(slices, S, n1, reinterpret_cast<__half *>(Y));
+        else gemm_splits_reduce1_kernel<__nv_bfloat16><<<(unsigned)g, 256, 0, st>>>(slices, S, n1, reinterpret_cast<__nv_bfloat16 *>(Y));
+        return last_launch_status();
+    }
+    const int64_t n4 = (int64_t)M * N / 4;  // N % 4 == 0
     const int64_t g = std::max<int64_t>(1, std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 8));
     const float4 *part = reinterpret_cast<const float4 *>(slices);
     if (out_dt == RAZER_F32) gemm_splits_reduce_kernel<float><<<(unsigned)g, 256, 0, st>>>(part, S, n4, reinterpret_cast<float *>(Y));
@@ -719,7 +751,7 @@ static razer_status w4a4_product(const float *ts_a, razer_format afmt, int64_t M
             return RAZER_ERR_CUDA;
     }
     const float unbias = decode_unbias(afmt) * decode_unbias(wfmt);  // a power of two: exact
-    const int m = (int)M, n = (int)N, k = (int)K, KB = k / BK, nc = (int)num_chunks(K);
+    const int m = (int)M, n = (int)N, k = (int)K, KB = (k + BK - 1) / BK, nc = (int)num_chunks(K);
     for (int c = 0; c < nc; c++) {
         const int kb0 = (int)((int64_t)c * KB / nc), kb1 = (int)((int64_t)(c + 1) * KB / nc);
         const bool last = c == nc - 1;

@@ -324,6 +324,71 @@ int gemv_splits(int64_t B, int64_t N, int64_t K)
     return (int)S;
 }
 
+// ---------------------------------------------------------------------------
+// Any K % 16 == 0 (K % 128 != 0 has no 128-k chunking): one thread per weight
+// row, every block decoded exactly in binary32 (q*s, or v*s for the
+// redundant-zero code) and multiplied into B fp32 accumulators; y = ts * sum.
+// The activations are read through the read-only cache (every thread of a
+// warp reads the same element).  No workspace.
+// ---------------------------------------------------------------------------
+template <int FMT, typename TIn>
+__global__ void __launch_bounds__(128) gemv_generic_kernel(const TIn *__restrict__ x, int B, const uint8_t *__restrict__ codes,
+                                                           const uint8_t *__restrict__ scales, const float *__restrict__ ts_p, int N, int K,
+                                                           void *y, int out_dt)
+{
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    float acc[32];
+#pragma unroll
+    for (int b = 0; b < 32; b++) acc[b] = 0.0f;
+    const int nb = K >> 4;
+    const uint2 *crow = reinterpret_cast<const uint2 *>(codes + (size_t)n * (K >> 1));  // 8 bytes per block (K/2 % 8 == 0)
+    const uint8_t *srow = scales + (size_t)n * nb;
+    for (int kb = 0; kb < nb; kb++) {
+        const uint2 cw = __ldg(crow + kb);
+        const unsigned sb = srow[kb];
+        const float s = decode_scale<FMT>(sb);
+        float v = 0.0f;
+        if constexpr (Fmt<FMT>::kSpecials > 0) v = special_value((int)(sb >> Fmt<FMT>::kMetaShift));
+#pragma unroll
+        for (int e = 0; e < 16; e++) {
+            const unsigned c = ((e < 8 ? cw.x : cw.y) >> (4 * (e & 7))) & 0xFu;
+            float q = fp4_mag(c & 7u);
+            if (c & 8u) q = (Fmt<FMT>::kSpecials > 0 && c == 8u) ? v : -q;
+            const float w = __fmul_rn(q, s);  // exact
+            const size_t k = (size_t)kb * 16 + e;
+            for (int b = 0; b < B; b++) {
+                const TIn xv = x[(size_t)b * K + k];
+                float xf;
+                if constexpr (std::is_same<TIn, __half>::value) xf = __half2float(xv);
+                else xf = __bfloat162float(xv);
+                acc[b] = fmaf(xf, w, acc[b]);
+            }
+        }
+    }
+    const float ts = *ts_p;
+    for (int b = 0; b < B; b++) {
+        const float a = __fmul_rn(acc[b], ts);
+        const size_t i = (size_t)b * N + n;
+        if (out_dt == RAZER_F32) reinterpret_cast<float *>(y)[i] = a;
+        else if (out_dt == RAZER_F16) reinterpret_cast<__half *>(y)[i] = __float2half_rn(a);
+        else reinterpret_cast<__nv_bfloat16 *>(y)[i] = __float2bfloat16_rn(a);
+    }
+}
+
+template <int FMT>
+static razer_status launch_gemv_generic(const void *x, razer_dtype act_dt, int B, const uint8_t *codes, const uint8_t *scales,
+                                        const float *ts, int N, int K, void *y, razer_dtype out_dt, cudaStream_t st)
+{
+    const unsigned grid = (unsigned)((N + 127) / 128);
+    if (act_dt == RAZER_F16)
+        gemv_generic_kernel<FMT, __half><<<grid, 128, 0, st>>>(reinterpret_cast<const __half *>(x), B, codes, scales, ts, N, K, y, (int)out_dt);
+    else
+        gemv_generic_kernel<FMT, __nv_bfloat16><<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), B, codes, scales, ts, N, K, y,
+                                                                     (int)out_dt);
+    return last_launch_status();
+}
+
 bool gemv_tma_eligible(int64_t B, int64_t N, int64_t K);
 size_t gemv_tma_workspace_bytes(int64_t B, int64_t N, int64_t K);
 razer_status run_gemv_tma(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
@@ -331,7 +396,7 @@ razer_status run_gemv_tma(const void *x, razer_dtype act_dt, int64_t B, const ui
 
 size_t gemv_workspace_bytes(int64_t B, int64_t N, int64_t K)
 {
-    if (B <= 0 || N <= 0 || K <= 0) return 0;
+    if (B <= 0 || N <= 0 || K <= 0 || K % 128 != 0) return 0;  // K % 128 != 0: the generic kernel, no workspace
     // the per-warp kernel also serves eligible shapes whose scale pointer is
     // only 4-byte aligned (a tensor map needs 16), so size for both
     const size_t split = (size_t)gemv_splits(B, N, K) * (size_t)B * (size_t)N * sizeof(float);
@@ -361,6 +426,11 @@ static void launch_gemv_fmt(const void *x, int B, const uint8_t *codes, const ui
 razer_status run_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,
                       razer_format wfmt, int64_t N, int64_t K, void *y, razer_dtype out_dt, void *workspace, cudaStream_t st)
 {
+    if (K % 128 != 0) {
+        if (wfmt == RAZER_FMT_WEIGHT) return launch_gemv_generic<RAZER_FMT_WEIGHT>(x, act_dt, (int)B, codes, scales, ts, (int)N, (int)K, y, out_dt, st);
+        if (wfmt == RAZER_FMT_ACT) return launch_gemv_generic<RAZER_FMT_ACT>(x, act_dt, (int)B, codes, scales, ts, (int)N, (int)K, y, out_dt, st);
+        return launch_gemv_generic<RAZER_FMT_NVFP4>(x, act_dt, (int)B, codes, scales, ts, (int)N, (int)K, y, out_dt, st);
+    }
     if (gemv_tma_eligible(B, N, K) && (reinterpret_cast<uintptr_t>(scales) & 15) == 0)
         return run_gemv_tma(x, act_dt, B, codes, scales, ts, wfmt, N, K, y, out_dt, workspace, st);
     const int S = gemv_splits(B, N, K);

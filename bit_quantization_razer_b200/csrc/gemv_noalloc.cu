@@ -97,7 +97,7 @@ extern "C" razer_status razer_gemv_noalloc(const void *x, razer_dtype act_dt, in
         if (!codes || !scales) return RAZER_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(codes) % 16 || reinterpret_cast<uintptr_t>(scales) % 4) return RAZER_ERR_ALIGN;
     }
-    if (B < 1 || B > 32 || K % 128 != 0 || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    if (B < 1 || B > 32 || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) % 16 || reinterpret_cast<uintptr_t>(ts) % 4)
         return RAZER_ERR_ALIGN;
     if (N == 0) return RAZER_OK;

@@ -174,11 +174,12 @@ razer_status razer_dequant(const uint8_t *codes, const uint8_t *scales, const fl
  *              razer_workspace_size(RAZER_OP_GEMV, B, N, K) bytes (16-byte
  *              aligned), or NULL when that size is 0.  Contents on entry are
  *              ignored (it holds split-K partials while a call runs).
- * K must be a multiple of 128 (one 16-byte code chunk per 32 elements, four
- * chunks per row slice).  K % 256 == 0 with a 16-byte aligned scale pointer
- * takes the bulk-tensor (TMA) kernel -- one persistent CTA per SM plus a small
- * split-K reduction kernel launched as its programmatic dependent; other calls
- * take a per-warp cp.async kernel and a reduction kernel.
+ * Any K % 16 == 0.  K % 256 == 0 with a 16-byte aligned scale pointer takes
+ * the bulk-tensor (TMA) kernel -- one persistent CTA per SM plus a small
+ * split-K reduction kernel launched as its programmatic dependent; other
+ * K % 128 == 0 calls take a per-warp cp.async kernel and a reduction kernel;
+ * K % 128 != 0 takes a row-per-thread kernel that decodes each block exactly
+ * in fp32 (no workspace: razer_workspace_size returns 0).
  */
 razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes,
                         const uint8_t *scales, const float *ts, razer_format wfmt, int64_t N,
@@ -206,7 +207,9 @@ razer_status razer_gemv(const void *x, razer_dtype act_dt, int64_t B, const uint
  *              run in parallel, each writes its scaled fp32 sum to its own
  *              [M, N] slice, and a reduction kernel adds the slices in split
  *              order (deterministic) and converts to out_dt.
- * K must be a multiple of 64 and N a multiple of 16.
+ * Any K % 16 == 0 and any N, M.  K % 64 != 0 or N % 16 != 0 take the
+ * decode-once path whatever M (workspace N * K * 2 bytes first): the
+ * bulk-tensor copies zero-fill the last, partial k-step of both operands.
  */
 razer_status razer_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes,
                         const uint8_t *scales, const float *ts, razer_format wfmt, int64_t N,
@@ -264,8 +267,8 @@ size_t razer_gemv_batch_workspace_size(int count, const razer_gemv_problem *prob
  *              tcgen05 pipeline of razer_gemm multiplies them, and the
  *              epilogue applies ts_a * ts_w (one fp32 rounding) and the
  *              bias; K > 16384 runs in chunks as for razer_gemm.
- * K must be a multiple of 64 and N a multiple of 16.  ts_a and ts_w are
- * device floats.
+ * Any K % 16 == 0 and any N (a partial last k-step is zero-filled as for
+ * razer_gemm).  ts_a and ts_w are device floats.
  */
 razer_status razer_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, const float *ts_a,
                              razer_format afmt, int64_t M, const uint8_t *codes_w,

@@ -91,18 +91,23 @@ def test_gemv_gemm_validation(lib):
     args = lambda B, N, K, ws=None, wsb=0: (FAKE, 0, B, FAKE, FAKE, FAKE, 0, N, K, FAKE, 2, ws, wsb, None)
     assert g(*args(0, 64, 128)) == 2
     assert g(*args(33, 64, 128)) == 2
-    assert g(*args(1, 64, 96)) == 2          # K % 128
+    assert g(*args(1, 64, 24)) == 2          # K % 16 (the only K-shape error)
+    assert g(*args(33, 64, 96)) == 2         # B, with a K outside the 128-k chunking
     assert g(*args(1, 64, 128)) == 5         # workspace missing
     assert g(FAKE, 2, 1, FAKE, FAKE, FAKE, 0, 64, 128, FAKE, 2, None, 0, None) == 4
     m = lib.razer_gemm
-    assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 64, 96, FAKE, 1, None, 0, None) == 2   # K % 64
-    assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 40, 128, FAKE, 1, None, 0, None) == 2  # N % 16
+    assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 64, 24, FAKE, 1, None, 0, None) == 2   # K % 16
+    # K % 64 != 0 and N % 16 != 0 are served (decode-once path): they need its workspace
+    assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 64, 96, FAKE, 1, None, 0, None) == 5
+    assert m(FAKE, 1, 64, FAKE, FAKE, FAKE, 0, 40, 128, FAKE, 1, None, 0, None) == 5
+    assert razer.razer_workspace_size(razer.RAZER_OP_GEMM, 64, 40, 96) == 40 * 96 * 2
     assert m(None, 1, 64, FAKE, FAKE, FAKE, 0, 64, 128, FAKE, 1, None, 0, None) == 1
     w = lib.razer_gemm_w4a4
     wargs = lambda M, N, K, afmt=1, wfmt=0, ts=FAKE, y=FAKE: (FAKE, FAKE, ts, afmt, M, FAKE, FAKE, FAKE, wfmt, N, K, y, 1, None, 0,
                                                               None)
-    assert w(*wargs(64, 64, 96)) == 2            # K % 64
-    assert w(*wargs(64, 40, 128)) == 2           # N % 16
+    assert w(*wargs(64, 64, 24)) == 2            # K % 16
+    assert w(*wargs(64, 64, 96)) == 5            # K % 64 != 0 is served: workspace missing
+    assert w(*wargs(64, 40, 128)) == 5           # N % 16 != 0 likewise
     assert w(*wargs(64, 64, 128, afmt=5)) == 1   # unknown format
     assert w(*wargs(64, 64, 128, ts=None)) == 1
     assert w(*wargs(64, 64, 128, y=ODD)) == 3

@@ -93,9 +93,41 @@ def test_gemm_k_zero_and_errors():
     Y = R.razer_gemm(X, codes, scales, torch.ones(1, device=DEV), "weight", torch.float32)
     torch.cuda.synchronize()
     assert not Y.any()
-    c, s = workloads.random_packed(48, 96, "weight", seed=1)
-    with pytest.raises(R.RazerError):  # K % 64
-        R.razer_gemm(torch.zeros(8, 96, dtype=torch.bfloat16, device=DEV), c.to(DEV), s.to(DEV), torch.ones(1, device=DEV))
+    with pytest.raises(R.RazerError):  # K % 16
+        R.razer_gemm(torch.zeros(8, 24, dtype=torch.bfloat16, device=DEV), torch.zeros(48, 12, dtype=torch.uint8, device=DEV),
+                     torch.zeros(48, 2, dtype=torch.uint8, device=DEV), torch.ones(1, device=DEV))
+
+
+@pytest.mark.parametrize("M,N,K,fmt,xdt,odt", [(1, 17, 16, "weight", torch.bfloat16, torch.float32),
+                                               (100, 40, 80, "act", torch.float16, torch.float16),
+                                               (33, 100, 208, "nvfp4", torch.bfloat16, torch.bfloat16),
+                                               (300, 24, 16400, "weight", torch.bfloat16, torch.float32),
+                                               (1100, 18, 144, "weight", torch.float16, torch.float16),
+                                               (130, 300, 1040, "weight", torch.bfloat16, torch.bfloat16)])
+def test_gemm_generic_shapes(orc, M, N, K, fmt, xdt, odt):
+    # K % 64 != 0 and N % 16 != 0 (rows not 16-byte aligned, a ragged last
+    # k-step, a K spanning two accumulation chains, M above the decode-once
+    # threshold) against the oracle
+    codes, scales = workloads.random_packed(N, K, fmt, seed=M + N + K, max_scale_code=40)
+    X = workloads.vectors(M, K, seed=M + 1, dtype=xdt)
+    ts = 0.0213
+    Y = R.razer_gemm(X.to(DEV), codes.to(DEV), scales.to(DEV), torch.tensor([ts], device=DEV), fmt, odt)
+    torch.cuda.synchronize()
+    rows = np.arange(M) if M <= 256 else np.random.default_rng(M).choice(M, 64, replace=False)
+    ref = orc.gemm_ref(oracle_in(X[rows]), codes.numpy(), scales.numpy(), ts, FMT_ID[fmt])
+    assert_close_typed(Y[rows], ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(50, 24, 80), (7, 100, 16)])
+def test_gemm_w4a4_generic_shapes(orc, M, N, K):
+    xa = workloads.vectors(M, K, seed=M, dtype=torch.bfloat16)
+    ca, sa, ta, _ = R.razer_quantize_acts(xa.to(DEV), None, "act", hist=False)
+    cw, sw = workloads.random_packed(N, K, "weight", seed=N + K, max_scale_code=40)
+    tw = torch.tensor([0.031], device=DEV)
+    Y = R.razer_gemm_w4a4(ca, sa, ta, cw.to(DEV), sw.to(DEV), tw, "act", "weight", torch.float32)
+    torch.cuda.synchronize()
+    ref = orc.gemm_w4a4_ref(ca.cpu().numpy(), sa.cpu().numpy(), float(ta.cpu()[0]), 1, cw.numpy(), sw.numpy(), 0.031, 0)
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
 
 
 def test_gemm_bounded_wait_times_out_and_reports():

@@ -98,6 +98,22 @@ def test_gemv_tma_random_packed(orc, fmt, B, xdt):
     assert rel_err(y.cpu().numpy(), ref) <= REL_TOL
 
 
+@pytest.mark.parametrize("N,K,B,fmt,xdt,odt", [(17, 16, 1, "weight", torch.float16, torch.float32),
+                                               (200, 48, 3, "act", torch.bfloat16, torch.float16),
+                                               (130, 144, 17, "nvfp4", torch.float16, torch.bfloat16),
+                                               (64, 4112, 32, "weight", torch.bfloat16, torch.float32),
+                                               (300, 400, 5, "weight", torch.float16, torch.float16)])
+def test_gemv_generic_k(orc, N, K, B, fmt, xdt, odt):
+    # K % 128 != 0 (the only K-shape error is K % 16 != 0): no 128-k chunking
+    codes, scales = workloads.random_packed(N, K, fmt, seed=N + K + B, max_scale_code=40)
+    x = workloads.vectors(B, K, seed=B + 7, dtype=xdt)
+    ts = 0.0371
+    ref = orc.gemm_ref(oracle_in(x), codes.numpy(), scales.numpy(), ts, FMT_ID[fmt])
+    assert R.razer_workspace_size(R.RAZER_OP_GEMV, B, N, K) == 0
+    y = gemv(x, codes, scales, ts, fmt, odt)
+    assert_close_typed(y, ref)
+
+
 @pytest.mark.parametrize("N,K,B", [(100, 256, 1), (128, 14336, 3), (129, 256, 2), (1, 4096, 1), (3000, 256, 7),
                                    (640, 2304, 32), (1280, 4096, 8)])
 def test_gemv_stream_k_partitions(orc, N, K, B):
