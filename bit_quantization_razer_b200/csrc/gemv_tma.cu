@@ -45,28 +45,31 @@
 namespace razer {
 namespace gemv_tma {
 
+#ifndef RAZER_GEMV_MT
+#define RAZER_GEMV_MT 2
+#endif
+constexpr int kMT = RAZER_GEMV_MT;                  // 16-row MMA tiles per consumer warp (1 or 2)
 constexpr int kTileRows = 128;
+constexpr int kRowGroups = kTileRows / (16 * kMT);  // consumer warps per k-half
+constexpr int kConsumerWarps = 2 * kRowGroups;      // one per (row group, 128-k half of a stage)
 constexpr int kFirstConsumer = 2;                   // warp 0: TMA producer, warp 1: epilogue
+constexpr int kThreads = 32 * (kFirstConsumer + kConsumerWarps);
 constexpr int kCodeBytes = kTileRows * 128;         // 128 rows x 256 codes
 constexpr int kScaleBytes = kTileRows * 16;         // 128 rows x 16 blocks
 constexpr int kMaxStages = 8;
 constexpr int kBarBytes = 256;
-constexpr int kTableBytes = 2048;                   // 256 (s, v*s) fp32 pairs, one per scale byte
 constexpr int kSmemLimit = 227 * 1024;
-// consumer warps: one per (group of 16 * MT rows of the tile, 128-k half of a stage)
-__host__ __device__ constexpr int consumer_warps(int MT) { return 2 * (kTileRows / (16 * MT)); }
-__host__ __device__ constexpr int cta_threads(int MT) { return 32 * (kFirstConsumer + consumer_warps(MT)); }
 
 __host__ __device__ constexpr int stage_bytes(int B) { return (kCodeBytes + kScaleBytes + B * 512 + 1023) / 1024 * 1024; }
 // two hand-over buffers of [k-half][B][128 rows] fp32 partials
 __host__ __device__ constexpr int part_bytes(int B) { return 2 * 2 * B * kTileRows * 4; }
-// dynamic shared memory: 2 KB alignment slack | scale table | stages | hand-over | barriers
-__host__ __device__ constexpr int fixed_bytes(int B) { return 2047 + kTableBytes + part_bytes(B) + kBarBytes; }
 __host__ __device__ constexpr int num_stages(int B)
 {
-    return (kSmemLimit - fixed_bytes(B)) / stage_bytes(B) > kMaxStages ? kMaxStages : (kSmemLimit - fixed_bytes(B)) / stage_bytes(B);
+    return (kSmemLimit - 1024 - kBarBytes - part_bytes(B)) / stage_bytes(B) > kMaxStages
+               ? kMaxStages
+               : (kSmemLimit - 1024 - kBarBytes - part_bytes(B)) / stage_bytes(B);
 }
-__host__ __device__ constexpr int smem_bytes(int B) { return num_stages(B) * stage_bytes(B) + fixed_bytes(B); }
+__host__ __device__ constexpr int smem_bytes(int B) { return num_stages(B) * stage_bytes(B) + part_bytes(B) + kBarBytes + 1024; }
 
 // A batch of independent problems y_i = ts_i * x_i * deq(W_i)^T (same
 // formats, same output type) run as one stream-K pass: their tiles are
@@ -127,266 +130,13 @@ __device__ __forceinline__ void wait_phase(uint32_t bar, uint32_t ph, volatile i
     if (!mbar_try_wait(bar, ph)) (void)mbar_wait(bar, ph, flags);  // on abort: carry on, results are void
 }
 
-// ---------------------------------------------------------------------------
-// Block-column decode (B <= 4, fp16 activations).
-//
-// The per-element decode is reduced to one hardware E2M1 convert per code
-// pair: neither the block scale nor the special value is applied to the
-// decoded operand.
-//   * The 8 output columns of each m16n8k16 MMA carry (block, batch row)
-//     pairs instead of batch rows: the activation operand is block-diagonal
-//     (column n only sees the k of its block), so after the MMAs of one group
-//     column n holds the unscaled dot product of one 16-element block.  The
-//     block scale s is then applied once per (row, block) with an fp32 FMA on
-//     the MMA output.  BP = padded batch (1, 2 or 4); a group of 8 / BP MMAs
-//     covers 8 / BP blocks.
-//   * The redundant-zero codes (0b1000) convert to -0, so the plain MMA adds
-//     nothing for them.  A second MMA multiplies a 0/1 indicator operand
-//     (the E2M1 code of 1.0 exactly where the code is 0b1000, found with
-//     three integer operations per 8 codes) by the same activations; its
-//     output, times v*s, is the special values' share of the block
-//     (RaZeR notes 关键设计 2: the -0 code carries the special value).
-//   * s and v*s of every scale byte come from a 256-entry fp32 table in
-//     shared memory built at kernel start (one 8-byte load per block).
-// Each fp32 product s*(q.x) equals the exact sum up to the MMA's fp32
-// accumulation, and q*x, v*x are exact in the MMA, so the result carries
-// the same rounding as decoding q*s first.
-// ---------------------------------------------------------------------------
-
-// E2M1 pair -> f16x2 of byte lane L of w (L a compile-time constant after unrolling)
-__device__ __forceinline__ unsigned cvt_byte(unsigned w, int L)
-{
-    unsigned r;
-    if (L == 0) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b0; }" : "=r"(r) : "r"(w));
-    else if (L == 1) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b1; }" : "=r"(r) : "r"(w));
-    else if (L == 2) asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b2; }" : "=r"(r) : "r"(w));
-    else asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %1; cvt.rn.f16x2.e2m1x2 %0, b3; }" : "=r"(r) : "r"(w));
-    return r;
-}
-
-// E2M1 codes of 1.0 (0b0010) exactly where a nibble of w is 0b1000, 0 elsewhere
-__device__ __forceinline__ unsigned indicator_codes(unsigned w)
-{
-    const unsigned t = (w & 0x77777777u) + 0x77777777u;  // bit 3 set where the magnitude bits are non-zero
-    const unsigned is8 = w & ~t & 0x88888888u;           // bit 3 set where the code is 0b1000
-    return __umulhi(is8, 0x40000000u);                   // >> 2 on the multiply pipe
-}
-
-// not volatile: a pure function of its operands, so the compiler may
-// interleave the MMAs of independent row tiles and groups
-__device__ __forceinline__ void mma_f16(float (&d)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3, unsigned b0, unsigned b1)
-{
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// (s, v*s) of byte lane L of w
-__device__ __forceinline__ float2 table_entry(unsigned w, int L, const float2 *tbl) { return tbl[(w >> (8 * L)) & 0xFFu]; }
-
-// Shared-memory loads as plain C++ loads (not volatile asm): the compiler
-// schedules them freely between the pipeline-barrier waits, whose asm
-// carries a memory clobber, so no load moves above the wait for its stage.
-template <typename T> __device__ __forceinline__ T sld(const uint8_t *p) { return *reinterpret_cast<const T *>(p); }
-
-// MMA row g of a 16-row tile -> tile row (0..7), chosen so that the code
-// loads of one shared-memory phase hit distinct banks under the 128-byte swizzle
-template <int BP> __device__ __forceinline__ int bc_row(int g) { return BP == 2 ? (((g & 3) << 1) | (g >> 2)) : tile_row(g); }
-
-// One 128-k slice of one 16-row tile: the codes of rows r and r + 8 (tile
-// rows; r & 7 == pr) through the block-column MMAs, accumulated into acc
-// (BP = 1: [row g, row g+8]; BP = 2, 4: [row g: 2 batch columns, row g+8: 2]).
-template <int FMT, int BP>
-__device__ __forceinline__ void bc_tile(const uint8_t *st, const uint8_t *scl, const float2 *tbl, int r, int pr, int kh, int t,
-                                        const unsigned (&xb0)[16], const unsigned (&xb1)[16], float (&acc)[4])
-{
-    constexpr bool kSpecial = Fmt<FMT>::kSpecials > 0;
-    const uint8_t *rowA = st + r * 128, *rowB = rowA + 8 * 128;
-    // this half's 8 scale bytes of rows r and r + 8
-    const uint2 sA = sld<uint2>(scl + r * 16 + 8 * kh), sB = sld<uint2>(scl + (r + 8) * 16 + 8 * kh);
-    if constexpr (BP == 1) {
-        // lane t: blocks 2t, 2t+1 (16 bytes, one swizzled chunk); MMA i takes pair i of both
-        const int off = ((4 * kh + t) ^ pr) << 4;
-        const uint4 cA = sld<uint4>(rowA + off), cB = sld<uint4>(rowB + off);
-        const unsigned wA[4] = {cA.x, cA.y, cA.z, cA.w}, wB[4] = {cB.x, cB.y, cB.z, cB.w};
-        unsigned iA[4], iB[4];
-        if constexpr (kSpecial) {
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-                iA[k] = indicator_codes(wA[k]);
-                iB[k] = indicator_codes(wB[k]);
-            }
-        }
-        float dq[4] = {0.f, 0.f, 0.f, 0.f}, di[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const int lo = i >> 2, hi = 2 + (i >> 2), L = i & 3;
-            mma_f16(dq, cvt_byte(wA[lo], L), cvt_byte(wB[lo], L), cvt_byte(wA[hi], L), cvt_byte(wB[hi], L), xb0[i], xb1[i]);
-            if constexpr (kSpecial)
-                mma_f16(di, cvt_byte(iA[lo], L), cvt_byte(iB[lo], L), cvt_byte(iA[hi], L), cvt_byte(iB[hi], L), xb0[i], xb1[i]);
-        }
-        // scale bytes 2t, 2t+1 of the half: word t >> 1, byte lanes 2(t & 1), +1
-        const unsigned wsA = (t >> 1) ? sA.y : sA.x, wsB = (t >> 1) ? sB.y : sB.x;
-        const unsigned shA = wsA >> (16 * (t & 1)), shB = wsB >> (16 * (t & 1));
-        const float2 e0 = (table_entry(shA, 0, tbl)), e1 = (table_entry(shA, 1, tbl));
-        const float2 e2 = (table_entry(shB, 0, tbl)), e3 = (table_entry(shB, 1, tbl));
-        acc[0] = fmaf(e0.x, dq[0], acc[0]);
-        acc[0] = fmaf(e1.x, dq[1], acc[0]);
-        acc[1] = fmaf(e2.x, dq[2], acc[1]);
-        acc[1] = fmaf(e3.x, dq[3], acc[1]);
-        if constexpr (kSpecial) {
-            acc[0] = fmaf(e0.y, di[0], acc[0]);
-            acc[0] = fmaf(e1.y, di[1], acc[0]);
-            acc[1] = fmaf(e2.y, di[2], acc[1]);
-            acc[1] = fmaf(e3.y, di[3], acc[1]);
-        }
-    } else if constexpr (BP == 2) {
-        // group gm (blocks 4gm .. 4gm+3): lane t decodes block 4gm + t (8 bytes);
-        // MMA i takes its pairs 2i, 2i+1
-#pragma unroll
-        for (int gm = 0; gm < 2; gm++) {
-            const int off = (((4 * kh + 2 * gm + (t >> 1)) ^ pr) << 4) + 8 * (t & 1);
-            const uint2 cA = sld<uint2>(rowA + off), cB = sld<uint2>(rowB + off);
-            const unsigned wA[2] = {cA.x, cA.y}, wB[2] = {cB.x, cB.y};
-            unsigned iA[2], iB[2];
-            if constexpr (kSpecial) {
-#pragma unroll
-                for (int k = 0; k < 2; k++) {
-                    iA[k] = indicator_codes(wA[k]);
-                    iB[k] = indicator_codes(wB[k]);
-                }
-            }
-            float dq[4] = {0.f, 0.f, 0.f, 0.f}, di[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const int w = i >> 1, L0 = 2 * (i & 1), L1 = L0 + 1;
-                mma_f16(dq, cvt_byte(wA[w], L0), cvt_byte(wB[w], L0), cvt_byte(wA[w], L1), cvt_byte(wB[w], L1), xb0[4 * gm + i],
-                        xb1[4 * gm + i]);
-                if constexpr (kSpecial)
-                    mma_f16(di, cvt_byte(iA[w], L0), cvt_byte(iB[w], L0), cvt_byte(iA[w], L1), cvt_byte(iB[w], L1), xb0[4 * gm + i],
-                            xb1[4 * gm + i]);
-            }
-            // scale byte 4gm + t of the half: word gm, byte lane t
-            const unsigned wsA = gm ? sA.y : sA.x, wsB = gm ? sB.y : sB.x;
-            const unsigned shA = wsA >> (8 * t), shB = wsB >> (8 * t);
-            const float2 ea = (table_entry(shA, 0, tbl)), eb = (table_entry(shB, 0, tbl));
-            // columns 2t, 2t+1 = (block t, batch 0), (block t, batch 1)
-            acc[0] = fmaf(ea.x, dq[0], acc[0]);
-            acc[1] = fmaf(ea.x, dq[1], acc[1]);
-            acc[2] = fmaf(eb.x, dq[2], acc[2]);
-            acc[3] = fmaf(eb.x, dq[3], acc[3]);
-            if constexpr (kSpecial) {
-                acc[0] = fmaf(ea.y, di[0], acc[0]);
-                acc[1] = fmaf(ea.y, di[1], acc[1]);
-                acc[2] = fmaf(eb.y, di[2], acc[2]);
-                acc[3] = fmaf(eb.y, di[3], acc[3]);
-            }
-        }
-    } else {
-        // group gm (blocks 2gm, 2gm+1): lane t decodes word t & 1 of block
-        // 2gm + (t >> 1); MMA i takes its byte lanes 2i, 2i+1
-#pragma unroll
-        for (int gm = 0; gm < 4; gm++) {
-            const int off = (((4 * kh + gm) ^ pr) << 4) + 4 * t;
-            const unsigned wA = sld<unsigned>(rowA + off), wB = sld<unsigned>(rowB + off);
-            unsigned iA = 0u, iB = 0u;
-            if constexpr (kSpecial) {
-                iA = indicator_codes(wA);
-                iB = indicator_codes(wB);
-            }
-            float dq[4] = {0.f, 0.f, 0.f, 0.f}, di[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 2; i++) {
-                mma_f16(dq, cvt_byte(wA, 2 * i), cvt_byte(wB, 2 * i), cvt_byte(wA, 2 * i + 1), cvt_byte(wB, 2 * i + 1), xb0[2 * gm + i],
-                        xb1[2 * gm + i]);
-                if constexpr (kSpecial)
-                    mma_f16(di, cvt_byte(iA, 2 * i), cvt_byte(iB, 2 * i), cvt_byte(iA, 2 * i + 1), cvt_byte(iB, 2 * i + 1),
-                            xb0[2 * gm + i], xb1[2 * gm + i]);
-            }
-            // scale byte 2gm + (t >> 1) of the half: word gm >> 1, byte lane 2(gm & 1) + (t >> 1)
-            const unsigned wsA = (gm >> 1) ? sA.y : sA.x, wsB = (gm >> 1) ? sB.y : sB.x;
-            const int L = 2 * (gm & 1);
-            const unsigned shA = wsA >> (8 * (t >> 1)), shB = wsB >> (8 * (t >> 1));
-            const float2 ea = (table_entry(shA, L, tbl)), eb = (table_entry(shB, L, tbl));
-            // columns 2t, 2t+1 = (block t >> 1, batch 2(t & 1)), (.., batch 2(t & 1) + 1)
-            acc[0] = fmaf(ea.x, dq[0], acc[0]);
-            acc[1] = fmaf(ea.x, dq[1], acc[1]);
-            acc[2] = fmaf(eb.x, dq[2], acc[2]);
-            acc[3] = fmaf(eb.x, dq[3], acc[3]);
-            if constexpr (kSpecial) {
-                acc[0] = fmaf(ea.y, di[0], acc[0]);
-                acc[1] = fmaf(ea.y, di[1], acc[1]);
-                acc[2] = fmaf(eb.y, di[2], acc[2]);
-                acc[3] = fmaf(eb.y, di[3], acc[3]);
-            }
-        }
-    }
-}
-
-// The activation operand of one 128-k slice for the block-column MMAs:
-// lanes that hold a (block, batch row) column load its values, every other
-// lane holds zeros.  xs = shared address of batch row 0 of this k-half.
-template <int BP>
-__device__ __forceinline__ void bc_activations(const uint8_t *xs, int g, int t, int B, unsigned (&xb0)[16], unsigned (&xb1)[16])
-{
-#pragma unroll
-    for (int i = 0; i < 16; i++) xb0[i] = xb1[i] = 0u;
-    if constexpr (BP == 1) {
-        // column g = block g: kk-pair t is block 2t, kk-pair t+4 block 2t+1
-        if (t == (g >> 1)) {
-            const uint4 v0 = sld<uint4>(xs + 32 * g), v1 = sld<uint4>(xs + 32 * g + 16);
-            const unsigned xr[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                if (g & 1) xb1[i] = xr[i];
-                else xb0[i] = xr[i];
-            }
-        }
-    } else if constexpr (BP == 2) {
-        // column g = (block g >> 1 of the group, batch row g & 1)
-        const int b = g & 1;
-        if (t == (g >> 1) && b < B) {
-#pragma unroll
-            for (int gm = 0; gm < 2; gm++) {
-                const uint8_t *a = xs + 512 * b + 32 * (4 * gm + t);
-                const uint4 v0 = sld<uint4>(a), v1 = sld<uint4>(a + 16);
-                const unsigned xr[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    xb0[4 * gm + i] = xr[2 * i];
-                    xb1[4 * gm + i] = xr[2 * i + 1];
-                }
-            }
-        }
-    } else {
-        // column g = (block g >> 2 of the group, batch row g & 3)
-        const int b = g & 3;
-        if ((t >> 1) == (g >> 2) && b < B) {
-#pragma unroll
-            for (int gm = 0; gm < 4; gm++) {
-                const uint4 v = sld<uint4>(xs + 512 * b + 32 * (2 * gm + (t >> 1)) + 16 * (t & 1));
-                xb0[2 * gm] = v.x;
-                xb1[2 * gm] = v.y;
-                xb0[2 * gm + 1] = v.z;
-                xb1[2 * gm + 1] = v.w;
-            }
-        }
-    }
-}
-
-// BP = 0: the per-element decode of the split-K kernel (scale and special
-// value folded into the MMA operand; every B <= 32, fp16 or bf16).
-// BP = 1, 2, 4: the block-column decode above (B <= BP, fp16).
-template <int FMT, bool BF16, int NB, int BP, int MT>
-__global__ void __launch_bounds__(cta_threads(MT), 1)
+template <int FMT, bool BF16, int NB>
+__global__ void __launch_bounds__(kThreads, 1)
     gemv_tma_kernel(const __grid_constant__ Batch A, int U, int stages, int stage_sz, int slot_elems, float *__restrict__ ws,
                     float unbias, int out_dt, int inject_stall)
 {
-    constexpr int kConsumerWarps = consumer_warps(MT);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 2047) & ~uintptr_t(2047));
-    float2 *table = reinterpret_cast<float2 *>(base);
-    uint8_t *smem = base + kTableBytes;
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const BatchInfo &I = A.info;
     float *part = reinterpret_cast<float *>(smem + stages * stage_sz);  // [2 buffers][2 k-halves][Bmax][128]
     uint8_t *bars = smem + stages * stage_sz + 2 * 2 * slot_elems * 4;
@@ -408,16 +158,6 @@ __global__ void __launch_bounds__(cta_threads(MT), 1)
         }
         flags[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if constexpr (BP > 0) {
-        // (s, v * s) of every scale byte: exact binary32 values
-        if (threadIdx.x < 256) {
-            const unsigned code = threadIdx.x;
-            const float s = decode_scale<FMT>(code);
-            float vs = 0.0f;
-            if constexpr (Fmt<FMT>::kSpecials > 0) vs = special_value((int)(code >> Fmt<FMT>::kMetaShift)) * s;
-            table[code] = make_float2(s, vs);
-        }
     }
     __syncthreads();
     // the reduction kernel may be scheduled now (it waits for this grid to finish)
@@ -528,131 +268,53 @@ __global__ void __launch_bounds__(cta_threads(MT), 1)
     }
 
     // ------------------------- consumers -------------------------
-    // warp (rg, kh): rows 16 MT rg .. 16 MT (rg + 1) - 1 of the tile, k-half kh
+    // warp (rg, kh): rows 16 kMT rg .. 16 kMT (rg + 1) - 1 of the tile, k-half kh
     // of every 256-k stage
     const int cw = warp - kFirstConsumer, rg = cw >> 1, kh = cw & 1, g = lane >> 2, t = lane & 3;
+    const int pr = tile_row(g);
+    const int cc = t + 4 * kh;  // this lane's 16-byte chunk of the 128-byte code row
+    const int R0 = 16 * kMT * rg + pr;  // tile row of MMA row g of the first 16-row tile
     const uint32_t sbase = smem_addr(smem);
+    const uint32_t offA = (uint32_t)(R0 * 128 + ((cc ^ pr) << 4));  // + 1024 for row g + 8, + 2048 per 16-row tile
+    const uint32_t offS = (uint32_t)(kCodeBytes + R0 * 16 + 2 * cc);  // + 128 for row g + 8, + 256 per tile
+    const uint32_t offX = (uint32_t)(kCodeBytes + kScaleBytes + g * 512 + 64 * cc);
+
+    float acc[kMT][NB][4];
+    unsigned xw[NB][16];
+#pragma unroll
+    for (int j = 0; j < NB; j++)
+#pragma unroll
+        for (int i = 0; i < 16; i++) xw[j][i] = 0u;
+
     int s = 0, q = 0;  // ring position of the next stage, hand-over count (no divisions in the loop)
     uint32_t ph = 0;
     uint32_t st = sbase;
-
-    if constexpr (BP > 0) {
-        const int pr = bc_row<BP>(g);
-        const int R0 = 16 * MT * rg + pr;  // tile row of MMA row g of the first 16-row tile
-        const float2 *tbl = table;
-        float acc[MT][4];
-        unsigned xb0[16], xb1[16];
-        const uint8_t *sp = smem;  // generic pointer of the current stage
-        for (int p = p_begin; p < p_end; q++) {
-            const int pi = problem_of(I, p), UK2 = I.UK2[pi], u0 = I.unit0[pi], B = I.B[pi];
-            const int r = (p - u0) / UK2;
-            const int pe = min(p_end, u0 + (r + 1) * UK2);
-            const int h0 = p - u0 - r * UK2, h1 = pe - u0 - r * UK2;
-            const int ja = (h0 - kh + 1) >> 1, jb = (h1 - 1 - kh) >> 1;
+    for (int p = p_begin; p < p_end; q++) {
+        const int pi = problem_of(I, p), UK2 = I.UK2[pi], u0 = I.unit0[pi], B = I.B[pi];
+        const bool xrow = g < B;
+        const int r = (p - u0) / UK2;
+        const int pe = min(p_end, u0 + (r + 1) * UK2);
+        const int h0 = p - u0 - r * UK2, h1 = pe - u0 - r * UK2;
+        // stages j whose half-unit 2j + kh lies in [h0, h1)
+        const int ja = (h0 - kh + 1) >> 1, jb = (h1 - 1 - kh) >> 1;
 #pragma unroll
-            for (int m = 0; m < MT; m++) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.0f;
-
-            for (int j = h0 >> 1; j < (h1 + 1) >> 1; j++) {
-                wait_phase(full + 8 * s, ph, flags);
-                if (j >= ja && j <= jb) {
-                    bc_activations<BP>(sp + kCodeBytes + kScaleBytes + 256 * kh, g, t, B, xb0, xb1);
+        for (int m = 0; m < kMT; m++)
 #pragma unroll
-                    for (int m = 0; m < MT; m++)
-                        bc_tile<FMT, BP>(sp, sp + kCodeBytes, tbl, R0 + 16 * m, pr, kh, t, xb0, xb1, acc[m]);
+            for (int j = 0; j < NB; j++) acc[m][j][0] = acc[m][j][1] = acc[m][j][2] = acc[m][j][3] = 0.0f;
+
+        for (int j = h0 >> 1; j < (h1 + 1) >> 1; j++) {
+            wait_phase(full + 8 * s, ph, flags);
+            if (j >= ja && j <= jb) {
+                uint4 ca[kMT], cb[kMT];
+                unsigned sA[kMT], sB[kMT];
+#pragma unroll
+                for (int m = 0; m < kMT; m++) {
+                    ca[m] = lds128(st + offA + 2048 * m);
+                    cb[m] = lds128(st + offA + 2048 * m + 1024);
+                    sA[m] = lds16(st + offS + 256 * m);
+                    sB[m] = lds16(st + offS + 256 * m + 128);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty + 8 * s);
-                sp += stage_sz;
-                if (++s == stages) {
-                    s = 0;
-                    ph ^= 1u;
-                    sp = smem;
-                }
-            }
-
-            // hand the partial of this tile to the epilogue warp and go on
-            const int buf = q & 1;
-            wait_phase(pempty + 8 * buf, ((uint32_t)(q >> 1) & 1u) ^ 1u, flags);
-            float *dst = part + (buf * 2 + kh) * slot_elems;
-#pragma unroll
-            for (int m = 0; m < MT; m++) {
-                const int row = R0 + 16 * m;
-                if constexpr (BP == 1) {
-                    float a0 = acc[m][0], a1 = acc[m][1];
-                    a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
-                    a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
-                    a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
-                    a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
-                    if (t == 0) {
-                        dst[row] = a0;
-                        dst[row + 8] = a1;
-                    }
-                } else {
-                    float a[4] = {acc[m][0], acc[m][1], acc[m][2], acc[m][3]};
-#pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        if (BP == 2) a[u] += __shfl_xor_sync(0xffffffffu, a[u], 1);
-                        a[u] += __shfl_xor_sync(0xffffffffu, a[u], 2);
-                    }
-                    // BP = 2: lane t = 0 holds batch rows 0, 1; BP = 4: lanes t = 0, 1 hold 2t, 2t+1
-                    if ((BP == 2 && t == 0) || (BP == 4 && t < 2)) {
-                        const int b0 = BP == 2 ? 0 : 2 * t;
-                        if (b0 < B) {
-                            dst[b0 * kTileRows + row] = a[0];
-                            dst[b0 * kTileRows + row + 8] = a[2];
-                        }
-                        if (b0 + 1 < B) {
-                            dst[(b0 + 1) * kTileRows + row] = a[1];
-                            dst[(b0 + 1) * kTileRows + row + 8] = a[3];
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(pfull + 8 * buf);
-            p = pe;
-        }
-        return;
-    } else {
-        const int pr = tile_row(g);
-        const int cc = t + 4 * kh;  // this lane's 16-byte chunk of the 128-byte code row
-        const int R0 = 16 * MT * rg + pr;  // tile row of MMA row g of the first 16-row tile
-        const uint32_t offA = (uint32_t)(R0 * 128 + ((cc ^ pr) << 4));  // + 1024 for row g + 8, + 2048 per 16-row tile
-        const uint32_t offS = (uint32_t)(kCodeBytes + R0 * 16 + 2 * cc);  // + 128 for row g + 8, + 256 per tile
-        const uint32_t offX = (uint32_t)(kCodeBytes + kScaleBytes + g * 512 + 64 * cc);
-
-        float acc[MT][NB][4];
-        unsigned xw[NB][16];
-#pragma unroll
-        for (int j = 0; j < NB; j++)
-#pragma unroll
-            for (int i = 0; i < 16; i++) xw[j][i] = 0u;
-
-        for (int p = p_begin; p < p_end; q++) {
-            const int pi = problem_of(I, p), UK2 = I.UK2[pi], u0 = I.unit0[pi], B = I.B[pi];
-            const bool xrow = g < B;
-            const int r = (p - u0) / UK2;
-            const int pe = min(p_end, u0 + (r + 1) * UK2);
-            const int h0 = p - u0 - r * UK2, h1 = pe - u0 - r * UK2;
-            // stages j whose half-unit 2j + kh lies in [h0, h1)
-            const int ja = (h0 - kh + 1) >> 1, jb = (h1 - 1 - kh) >> 1;
-#pragma unroll
-            for (int m = 0; m < MT; m++)
-#pragma unroll
-                for (int j = 0; j < NB; j++) acc[m][j][0] = acc[m][j][1] = acc[m][j][2] = acc[m][j][3] = 0.0f;
-
-            for (int j = h0 >> 1; j < (h1 + 1) >> 1; j++) {
-                wait_phase(full + 8 * s, ph, flags);
-                if (j >= ja && j <= jb) {
-                    uint4 ca[MT], cb[MT];
-                    unsigned sA[MT], sB[MT];
-#pragma unroll
-                    for (int m = 0; m < MT; m++) {
-                        ca[m] = lds128(st + offA + 2048 * m);
-                        cb[m] = lds128(st + offA + 2048 * m + 1024);
-                        sA[m] = lds16(st + offS + 256 * m);
-                        sB[m] = lds16(st + offS + 256 * m + 128);
-                    }
+                {
 #pragma unroll
                     for (int jj = 0; jj < NB; jj++) {
                         if (8 * jj + g < B && (NB > 1 || xrow)) {
@@ -667,38 +329,38 @@ __global__ void __launch_bounds__(cta_threads(MT), 1)
                         }
                     }
 #pragma unroll
-                    for (int m = 0; m < MT; m++) slice_mma<FMT, BF16, NB>(ca[m], cb[m], sA[m], sB[m], xw, acc[m]);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty + 8 * s);
-                st += (uint32_t)stage_sz;
-                if (++s == stages) {
-                    s = 0;
-                    ph ^= 1u;
-                    st = sbase;
-                }
-            }
-
-            // hand the partial of this tile to the epilogue warp and go on
-            const int buf = q & 1;
-            wait_phase(pempty + 8 * buf, ((uint32_t)(q >> 1) & 1u) ^ 1u, flags);
-            float *dst = part + (buf * 2 + kh) * slot_elems;
-#pragma unroll
-            for (int m = 0; m < MT; m++) {
-#pragma unroll
-                for (int jj = 0; jj < NB; jj++) {
-                    const int b0 = 8 * jj + 2 * t;
-#pragma unroll
-                    for (int i = 0; i < 4; i++) {
-                        const int b = b0 + (i & 1), row = R0 + 16 * m + ((i & 2) ? 8 : 0);
-                        if (b < B) dst[b * kTileRows + row] = acc[m][jj][i];
-                    }
+                    for (int m = 0; m < kMT; m++) slice_mma<FMT, BF16, NB>(ca[m], cb[m], sA[m], sB[m], xw, acc[m]);
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(pfull + 8 * buf);
-            p = pe;
+            if (lane == 0) mbar_arrive(empty + 8 * s);
+            st += (uint32_t)stage_sz;
+            if (++s == stages) {
+                s = 0;
+                ph ^= 1u;
+                st = sbase;
+            }
         }
+
+        // hand the partial of this tile to the epilogue warp and go on
+        const int buf = q & 1;
+        wait_phase(pempty + 8 * buf, ((uint32_t)(q >> 1) & 1u) ^ 1u, flags);
+        float *dst = part + (buf * 2 + kh) * slot_elems;
+#pragma unroll
+        for (int m = 0; m < kMT; m++) {
+#pragma unroll
+            for (int jj = 0; jj < NB; jj++) {
+                const int b0 = 8 * jj + 2 * t;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int b = b0 + (i & 1), row = R0 + 16 * m + ((i & 2) ? 8 : 0);
+                    if (b < B) dst[b * kTileRows + row] = acc[m][jj][i];
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pfull + 8 * buf);
+        p = pe;
     }
 }
 
@@ -758,18 +420,10 @@ static Plan plan(const Problem *P, int n)
     return p;
 }
 
-// Launch classes: problems of one class share a launch.  With fp16
-// activations, B = 1, B = 2 and B = 3..4 take the block-column kernels
-// (padded batch 1, 2, 4); every other case takes the per-element decode
-// with 1, 2 or 4 n8 MMA tiles (B <= 8, <= 16, <= 32).
-enum { kClassBC1 = 0, kClassBC2, kClassBC4, kClassNB1, kClassNB2, kClassNB4, kNumClasses };
-static int launch_class(int64_t B, bool bc)
-{
-    if (bc && B <= 4) return B == 1 ? kClassBC1 : (B == 2 ? kClassBC2 : kClassBC4);
-    return B <= 8 ? kClassNB1 : (B <= 16 ? kClassNB2 : kClassNB4);
-}
+// n-tiles of 8 columns the MMA needs for batch B
+static int nb_class(int64_t B) { return B <= 8 ? 1 : (B <= 16 ? 2 : 4); }
 
-template <int FMT, bool BF16, int NB, int BP, int MT>
+template <int FMT, bool BF16, int NB>
 static razer_status launch(const Batch &A, const Plan &pl, float *ws, float unbias, razer_dtype out_dt, cudaStream_t st)
 {
     const int Bmax = (int)pl.Bmax;
@@ -778,8 +432,7 @@ static razer_status launch(const Batch &A, const Plan &pl, float *ws, float unbi
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        if (cudaFuncSetAttribute(gemv_tma_kernel<FMT, BF16, NB, BP, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(gemv_tma_kernel<FMT, BF16, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
             return RAZER_ERR_CUDA;
         attr_done[dev] = true;
     }
@@ -787,8 +440,8 @@ static razer_status launch(const Batch &A, const Plan &pl, float *ws, float unbi
     // fault injection (tests only): one stage is never filled, so the
     // kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
     const int inject = fault_injection_enabled() ? 1 : 0;
-    if (launch_pdl(gemv_tma_kernel<FMT, BF16, NB, BP, MT>, (unsigned)G, (unsigned)cta_threads(MT), (size_t)smem, st, A, U, stages, sz,
-                   slot_elems, ws, unbias, (int)out_dt, inject) != cudaSuccess)
+    if (launch_pdl(gemv_tma_kernel<FMT, BF16, NB>, (unsigned)G, kThreads, (size_t)smem, st, A, U, stages, sz, slot_elems, ws, unbias,
+                   (int)out_dt, inject) != cudaSuccess)
         return RAZER_ERR_CUDA;
     // tiles shared by several CTAs exist unless every CTA range is whole tiles
     const BatchInfo &I = A.info;
@@ -804,27 +457,12 @@ static razer_status launch(const Batch &A, const Plan &pl, float *ws, float unbi
     return RAZER_OK;
 }
 
-#ifndef RAZER_GEMV_BC_MT
-#define RAZER_GEMV_BC_MT 2
-#endif
-constexpr int kLegacyMT = 2;             // per-element decode: 2 row tiles per consumer warp
-constexpr int kBcMT = RAZER_GEMV_BC_MT;  // block-column decode
-
 template <int FMT, bool BF16>
-static razer_status launch_class_fmt(int cls, const Batch &A, const Plan &pl, float *ws, razer_format wfmt, razer_dtype out_dt,
-                                     cudaStream_t st)
+static razer_status launch_nb(int nb, const Batch &A, const Plan &pl, float *ws, float unbias, razer_dtype out_dt, cudaStream_t st)
 {
-    // the per-element decode carries q*s*2^-bias; the block-column one exact s
-    const float unbias = wfmt == RAZER_FMT_WEIGHT ? scale_f16_unbias<RAZER_FMT_WEIGHT>() : scale_f16_unbias<RAZER_FMT_ACT>();
-    if constexpr (!BF16) {
-        if (cls == kClassBC1) return launch<FMT, false, 1, 1, kBcMT>(A, pl, ws, 1.0f, out_dt, st);
-        if (cls == kClassBC2) return launch<FMT, false, 1, 2, kBcMT>(A, pl, ws, 1.0f, out_dt, st);
-        if (cls == kClassBC4) return launch<FMT, false, 1, 4, kBcMT>(A, pl, ws, 1.0f, out_dt, st);
-    }
-    if (cls == kClassNB1) return launch<FMT, BF16, 1, 0, kLegacyMT>(A, pl, ws, unbias, out_dt, st);
-    if (cls == kClassNB2) return launch<FMT, BF16, 2, 0, kLegacyMT>(A, pl, ws, unbias, out_dt, st);
-    if (cls == kClassNB4) return launch<FMT, BF16, 4, 0, kLegacyMT>(A, pl, ws, unbias, out_dt, st);
-    return RAZER_ERR_UNSUPPORTED;
+    if (nb == 1) return launch<FMT, BF16, 1>(A, pl, ws, unbias, out_dt, st);
+    if (nb == 2) return launch<FMT, BF16, 2>(A, pl, ws, unbias, out_dt, st);
+    return launch<FMT, BF16, 4>(A, pl, ws, unbias, out_dt, st);
 }
 
 // The three tensor maps of one problem: codes [N, K/2] u8 in 128 x 128-byte
@@ -862,17 +500,17 @@ static bool encode_problem(EncodeTiledFn enc, const Problem &P, CUtensorMap *m)
     return true;
 }
 
-// Calls fn(class, group, n) for the launches of a batch: problems of the
-// same launch class, in their order, at most kMaxProblems per launch.
-template <typename Fn> static razer_status for_each_group(const Problem *P, int n, bool bc, Fn fn)
+// Calls fn(group, n) for the launches of a batch: problems of the same
+// n-tile class, in their order, at most kMaxProblems per launch.
+template <typename Fn> static razer_status for_each_group(const Problem *P, int n, Fn fn)
 {
-    for (int cls = 0; cls < kNumClasses; cls++) {
+    for (int nb = 1; nb <= 4; nb *= 2) {
         Problem g[kMaxProblems];
         int k = 0;
         for (int i = 0; i <= n; i++) {
-            if (i < n && launch_class(P[i].B, bc) == cls) g[k++] = P[i];
+            if (i < n && nb_class(P[i].B) == nb) g[k++] = P[i];
             if (k > 0 && (k == kMaxProblems || i == n)) {
-                const razer_status r = fn(cls, g, k);
+                const razer_status r = fn(nb, g, k);
                 if (r != RAZER_OK) return r;
                 k = 0;
             }
@@ -891,13 +529,11 @@ bool gemv_tma_eligible(int64_t B, int64_t N, int64_t K)
 
 size_t gemv_tma_batch_workspace_bytes(const gemv_tma::Problem *P, int n)
 {
-    // the grouping depends on the activation type: size for both
     size_t need = 0;
-    for (int bc = 0; bc < 2; bc++)
-        gemv_tma::for_each_group(P, n, bc != 0, [&](int, const gemv_tma::Problem *g, int k) {
-            need = std::max(need, gemv_tma::plan(g, k).total);
-            return RAZER_OK;
-        });
+    gemv_tma::for_each_group(P, n, [&](int, const gemv_tma::Problem *g, int k) {
+        need = std::max(need, gemv_tma::plan(g, k).total);
+        return RAZER_OK;
+    });
     return need;
 }
 
@@ -917,8 +553,9 @@ razer_status run_gemv_tma_batch(const gemv_tma::Problem *P, int n, razer_dtype a
     EncodeTiledFn enc = encode_fn();
     if (!enc) return RAZER_ERR_CUDA;
     float *ws = reinterpret_cast<float *>(workspace);
+    const float unbias = wfmt == RAZER_FMT_WEIGHT ? scale_f16_unbias<RAZER_FMT_WEIGHT>() : scale_f16_unbias<RAZER_FMT_ACT>();
     const bool bf = act_dt == RAZER_BF16;
-    return for_each_group(P, n, !bf, [&](int cls, const Problem *g, int k) {
+    return for_each_group(P, n, [&](int nb, const Problem *g, int k) {
         Batch A;
         memset(&A, 0, sizeof(A));
         BatchInfo &I = A.info;
@@ -936,13 +573,13 @@ razer_status run_gemv_tma_batch(const gemv_tma::Problem *P, int n, razer_dtype a
         }
         const Plan pl = plan(g, k);
         if (wfmt == RAZER_FMT_WEIGHT)
-            return bf ? launch_class_fmt<RAZER_FMT_WEIGHT, true>(cls, A, pl, ws, wfmt, out_dt, st)
-                      : launch_class_fmt<RAZER_FMT_WEIGHT, false>(cls, A, pl, ws, wfmt, out_dt, st);
+            return bf ? launch_nb<RAZER_FMT_WEIGHT, true>(nb, A, pl, ws, unbias, out_dt, st)
+                      : launch_nb<RAZER_FMT_WEIGHT, false>(nb, A, pl, ws, unbias, out_dt, st);
         if (wfmt == RAZER_FMT_ACT)
-            return bf ? launch_class_fmt<RAZER_FMT_ACT, true>(cls, A, pl, ws, wfmt, out_dt, st)
-                      : launch_class_fmt<RAZER_FMT_ACT, false>(cls, A, pl, ws, wfmt, out_dt, st);
-        return bf ? launch_class_fmt<RAZER_FMT_NVFP4, true>(cls, A, pl, ws, wfmt, out_dt, st)
-                  : launch_class_fmt<RAZER_FMT_NVFP4, false>(cls, A, pl, ws, wfmt, out_dt, st);
+            return bf ? launch_nb<RAZER_FMT_ACT, true>(nb, A, pl, ws, unbias, out_dt, st)
+                      : launch_nb<RAZER_FMT_ACT, false>(nb, A, pl, ws, unbias, out_dt, st);
+        return bf ? launch_nb<RAZER_FMT_NVFP4, true>(nb, A, pl, ws, unbias, out_dt, st)
+                  : launch_nb<RAZER_FMT_NVFP4, false>(nb, A, pl, ws, unbias, out_dt, st);
     });
 }
 
