@@ -700,8 +700,13 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
     n = 2048 * 4096
     h = hist.cpu().tolist()
     nblk = n // 16
-    out["act_quantize"] = {"ms": ms, "GB/s_two_pass": n * 4.5625 / ms / 1e6, "GB/s_single_pass_bytes": n * 2.5625 / ms / 1e6,
-                           "frac_two_pass": n * 4.5625 / ms / 1e6 / hbm,
+    # the library takes the single-pass kernel (X read once: 2 B in, 0.5625 B
+    # out per element) when each SM's slice of blocks fits its shared memory
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    single = nblk >= sms and -(-nblk // sms) * 32 <= 224 * 1024
+    bpe = 2.5625 if single else 4.5625
+    out["act_quantize"] = {"ms": ms, "path": "single_pass" if single else "two_pass", "bytes_per_elt": bpe,
+                           "GB/s": n * bpe / ms / 1e6, "frac": n * bpe / ms / 1e6 / hbm,
                            "meta_fraction": {"+5": h[0] / nblk, "-5": h[1] / nblk},
                            "effective_fraction": {"+5": h[2] / nblk, "-5": h[3] / nblk}}
     # tcgen05 GEMM on the prefill shapes

@@ -365,7 +365,8 @@ razer_status run_quantize_46(const void *x, razer_dtype dt, int64_t R, int64_t K
 {
     const int64_t n = R * K, nblk = n / 16;
     if (launch_pdl(zero_u64_kernel, 1u, 32u, 0, st, n_four, (unsigned long long *)nullptr) != cudaSuccess) return RAZER_ERR_CUDA;
-    if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, (unsigned long long *)nullptr, reinterpret_cast<unsigned *>(ts_out)) != cudaSuccess)
+    if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, (unsigned long long *)nullptr, reinterpret_cast<unsigned *>(ts_out), (unsigned *)nullptr) !=
+        cudaSuccess)
         return RAZER_ERR_CUDA;
     if (n > 0) {
         if (dt == RAZER_F16) launch_amax<__half>(x, n, reinterpret_cast<unsigned *>(ts_out), st);
@@ -418,7 +419,8 @@ razer_status run_quantize_variant(const void *x, razer_dtype dt, int64_t R, int6
 {
     const int64_t n = R * K, nsub = n / 16;
     const float C = sfmt == RAZER_FMT_WEIGHT ? Fmt<RAZER_FMT_WEIGHT>::kC : Fmt<RAZER_FMT_ACT>::kC;
-    if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, (unsigned long long *)nullptr, reinterpret_cast<unsigned *>(ts_out)) != cudaSuccess)
+    if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, (unsigned long long *)nullptr, reinterpret_cast<unsigned *>(ts_out), (unsigned *)nullptr) !=
+        cudaSuccess)
         return RAZER_ERR_CUDA;
     if (n > 0) {
         if (dt == RAZER_F16) launch_amax<__half>(x, n, reinterpret_cast<unsigned *>(ts_out), st);

@@ -807,7 +807,8 @@ razer_status run_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, co
     const int64_t n = M * K, nblk = n / 16;
     const float C = afmt == RAZER_FMT_WEIGHT ? Fmt<RAZER_FMT_WEIGHT>::kC : Fmt<RAZER_FMT_ACT>::kC;
     if (hist || !ts_in) {
-        if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, hist, ts_in ? (unsigned *)nullptr : reinterpret_cast<unsigned *>(ts_a_out)) !=
+        if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, hist, ts_in ? (unsigned *)nullptr : reinterpret_cast<unsigned *>(ts_a_out),
+                   (unsigned *)nullptr) !=
             cudaSuccess)
             return RAZER_ERR_CUDA;
     }

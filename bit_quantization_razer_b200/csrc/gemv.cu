@@ -297,8 +297,16 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float *__restric
     const float scale = __fmul_rn(*ts_p, unbias);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < BN; i += stride) {
+        // independent loads, eight at a time, added in split order
         float a = 0.0f;
-        for (int s = 0; s < S; s++) a += ws[(size_t)s * BN + i];
+        for (int s0 = 0; s0 < S; s0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int k = 0; k < 8; k++) v[k] = s0 + k < S ? ws[(size_t)(s0 + k) * BN + i] : 0.0f;
+#pragma unroll
+            for (int k = 0; k < 8; k++)
+                if (s0 + k < S) a += v[k];
+        }
         a = __fmul_rn(a, scale);
         if constexpr (sizeof(TOut) == 4) y[i] = a;
         else if constexpr (std::is_same<TOut, __half>::value) y[i] = __float2half_rn(a);

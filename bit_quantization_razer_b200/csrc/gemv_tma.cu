@@ -367,25 +367,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Sums the workspace slots of the tiles shared by several CTAs, in CTA order.
 // Launched as a programmatic dependent of gemv_tma_kernel: it may become
 // resident early and waits here until that grid has completed.
-__global__ void __launch_bounds__(256) gemv_tma_reduce_kernel(const float *__restrict__ ws, const BatchInfo I, int slot_elems, int U,
-                                                              int G, float unbias, int out_dt)
+__global__ void __launch_bounds__(kTileRows) gemv_tma_reduce_kernel(const float *__restrict__ ws, const BatchInfo I, int slot_elems, int U,
+                                                                    int G, float unbias, int out_dt)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next call may become resident
-    const int64_t total = (int64_t)I.tile0[I.count] * slot_elems;
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
-        const int R = (int)(t / slot_elems), e = (int)(t - (int64_t)R * slot_elems);
-        int pi = 0;
-        while (pi + 1 < I.count && R >= I.tile0[pi + 1]) pi++;
-        const int r = R - I.tile0[pi], UK2 = I.UK2[pi], u0 = I.unit0[pi], N = I.N[pi];
-        const int c_first = range_owner(u0 + r * UK2, U, G), c_last = range_owner(u0 + (r + 1) * UK2 - 1, U, G);
-        const int row = r * kTileRows + (e & (kTileRows - 1)), b = e >> 7;
-        if (c_first == c_last || row >= N || b >= I.B[pi]) continue;  // whole tiles were written by the main kernel
-        // slot (cta + global tile) holds that CTA's part of the tile
-        const float *src = ws + (size_t)R * slot_elems + e;
+    // CTA R: global tile R (thread = tile row); its contributing CTAs are
+    // found once per tile, and whole tiles were written by the main kernel
+    const int R = blockIdx.x;
+    int pi = 0;
+    while (pi + 1 < I.count && R >= I.tile0[pi + 1]) pi++;
+    const int r = R - I.tile0[pi], UK2 = I.UK2[pi], u0 = I.unit0[pi], N = I.N[pi], B = I.B[pi];
+    const int c_first = range_owner(u0 + r * UK2, U, G), c_last = range_owner(u0 + (r + 1) * UK2 - 1, U, G);
+    const int row = r * kTileRows + threadIdx.x;
+    if (c_first == c_last || row >= N) return;
+    const float oscale = __fmul_rn(*I.ts[pi], unbias);
+    for (int b = 0; b < B; b++) {
+        // slot (cta + global tile) holds that CTA's part of the tile; the slots
+        // are loaded eight at a time (independent loads) and added in CTA order
+        const float *src = ws + (size_t)R * slot_elems + b * kTileRows + threadIdx.x;
         float sum = 0.0f;
-        for (int k = c_first; k <= c_last; k++) sum += __ldcg(src + (size_t)k * slot_elems);
-        store_out(I.y[pi], out_dt, (size_t)b * N + row, __fmul_rn(sum, __fmul_rn(*I.ts[pi], unbias)));
+        for (int k0 = c_first; k0 <= c_last; k0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) v[i] = k0 + i <= c_last ? __ldcg(src + (size_t)(k0 + i) * slot_elems) : 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                if (k0 + i <= c_last) sum += v[i];
+        }
+        store_out(I.y[pi], out_dt, (size_t)b * N + row, __fmul_rn(sum, oscale));
     }
 }
 
@@ -450,9 +460,8 @@ static razer_status launch(const Batch &A, const Plan &pl, float *ws, float unbi
         for (int r = 0; r < I.tile0[pi + 1] - I.tile0[pi] && !shared; r++)
             shared = range_owner(I.unit0[pi] + r * I.UK2[pi], U, G) != range_owner(I.unit0[pi] + (r + 1) * I.UK2[pi] - 1, U, G);
     if (!shared) return RAZER_OK;
-    const int64_t total = pl.T * slot_elems;
-    const unsigned rgrid = (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 4);
-    if (launch_pdl(gemv_tma_reduce_kernel, rgrid, 256u, 0, st, (const float *)ws, I, slot_elems, U, G, unbias, (int)out_dt) != cudaSuccess)
+    if (launch_pdl(gemv_tma_reduce_kernel, (unsigned)pl.T, (unsigned)kTileRows, 0, st, (const float *)ws, I, slot_elems, U, G, unbias,
+                   (int)out_dt) != cudaSuccess)
         return RAZER_ERR_CUDA;
     return RAZER_OK;
 }

@@ -21,6 +21,7 @@
 //     is a multiple of 2^-20 computed exactly in binary32, and the partial
 //     sums stay exact (see the notes on each accumulator below).
 #include "razer_internal.cuh"
+#include "sm100_async.cuh"
 
 namespace razer {
 
@@ -530,13 +531,157 @@ __global__ void copy_ts_kernel(const float *src, float *dst)
 }
 
 // zeroes the histogram and the amax accumulator of a quantizer call (one
-// launch instead of two memsets)
-__global__ void quant_init_kernel(unsigned long long *hist, unsigned *amax_bits)
+// launch instead of two memsets), and the two barrier words of the
+// single-pass kernel when it runs (the first 8 code bytes)
+__global__ void quant_init_kernel(unsigned long long *hist, unsigned *amax_bits, unsigned *bar_words)
 {
     pdl_wait();
     pdl_trigger();
     if (hist && threadIdx.x < 4) hist[threadIdx.x] = 0ull;
     if (amax_bits && threadIdx.x == 0) *amax_bits = 0u;
+    if (bar_words && threadIdx.x < 2) bar_words[threadIdx.x] = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// Single-pass quantizer with a dynamic tensor scale: X is read from HBM once.
+// One CTA per SM, all co-resident (cooperative launch), each holding its
+// contiguous slice of blocks in shared memory:
+//   1. bulk copies bring the slice in (8 chunks at most, one mbarrier each);
+//      the block-wide amax is reduced chunk by chunk as they land and merged
+//      into the amax word (*ts_out, zeroed by the init kernel);
+//   2. a grid barrier: arrivals count up in bar[0], bounded wait for all G;
+//   3. every CTA reads the tensor amax, ts = amax / (6 S_max) (the same fp32
+//      divide as the two-pass path), counts itself out in bar[1], and
+//      quantizes its slice from shared memory with the same block quantizer;
+//   4. CTA 0 waits (bounded) until every CTA has counted out, then writes
+//      what the barrier words overlay -- the code bytes of block 0 -- and ts.
+// bar[] is the first 8 bytes of this call's code output: no state outlives
+// the call, and concurrent calls do not share it.  On a timeout the device
+// status word records RAZER_ERR_TIMEOUT and the outputs are void.
+// ---------------------------------------------------------------------------
+constexpr int kOneThreads = 1024;
+constexpr int kOneChunk = 32768;                  // bytes per bulk copy
+constexpr int kOneMaxChunks = 7;
+constexpr int kOneMaxSlice = kOneChunk * kOneMaxChunks;  // 224 KB of blocks per CTA
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+template <int FMT, typename TIn, bool HIST>
+__global__ void __launch_bounds__(kOneThreads, 1)
+    quantize_onepass_kernel(const TIn *__restrict__ x, int64_t nblk, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                            float *ts_out, unsigned long long *__restrict__ hist, int inject_stall)
+{
+    using F = Fmt<FMT>;
+    extern __shared__ __align__(128) uint8_t slice[];
+    __shared__ __align__(8) uint64_t bars[kOneMaxChunks];
+    __shared__ int s_abort;
+    __shared__ float s_amax;
+    __shared__ float tab_d[F::kMagMask + 1], tab_y[F::kMagMask + 1];
+    const int G = gridDim.x, c = blockIdx.x;
+    const int64_t b0 = (int64_t)c * nblk / G, b1 = (int64_t)(c + 1) * nblk / G;
+    const int nb = (int)(b1 - b0), bytes = nb * 32, nch = (bytes + kOneChunk - 1) / kOneChunk;
+    unsigned *bar = reinterpret_cast<unsigned *>(codes);  // [0] arrived, [1] departed (zeroed by the init kernel)
+    unsigned *amax_bits = reinterpret_cast<unsigned *>(ts_out);
+    const uint32_t bar0 = smem_addr(bars), sl = smem_addr(slice);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < nch; i++) mbar_init(bar0 + 8 * i, 1);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(x) + b0 * 32;
+        for (int i = 0; i < nch; i++) {
+            const uint32_t sz = (uint32_t)min(kOneChunk, bytes - i * kOneChunk);
+            mbar_expect_tx(bar0 + 8 * i, sz);
+            bulk_load(sl + (uint32_t)(i * kOneChunk), src + (size_t)i * kOneChunk, sz, bar0 + 8 * i);
+        }
+    }
+    // 1. amax of the slice, chunk by chunk
+    float m = 0.0f;
+    for (int i = 0; i < nch; i++) {
+        if (!mbar_try_wait(bar0 + 8 * i, 0)) (void)mbar_wait(bar0 + 8 * i, 0, &s_abort);
+        const int nv = min(kOneChunk, bytes - i * kOneChunk) / 16;
+        const uint4 *v = reinterpret_cast<const uint4 *>(slice + i * kOneChunk);
+        for (int j = threadIdx.x; j < nv; j += kOneThreads) m = amax_vec<TIn>(m, v[j]);
+    }
+    commit_amax(m, amax_bits);  // ends with thread 0's atomicMax (after a block barrier)
+    // 2. grid barrier
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (!(inject_stall && c == 0)) atomicAdd(&bar[0], 1u);  // fault injection (tests only): CTA 0 never arrives
+        const uint64_t t0 = globaltimer();
+        while (ld_acquire_u32(&bar[0]) < (unsigned)G) {
+            if (globaltimer() - t0 > kTimeoutNs) {
+                set_device_status(RAZER_ERR_TIMEOUT);
+                s_abort = 1;
+                break;
+            }
+            __nanosleep(64);
+        }
+        // 3. the tensor amax, read once; then this CTA counts itself out (it
+        // touches neither the barrier words nor the amax word again)
+        s_amax = __uint_as_float(ld_acquire_u32(amax_bits));
+        atomicAdd(&bar[1], 1u);
+    }
+    __syncthreads();
+    const float ts = __fdiv_rn(s_amax, F::kC);
+    const ScaleCtx k = make_ctx<FMT>(ts, tab_d, tab_y);
+    __syncthreads();
+    unsigned cnt[4] = {0u, 0u, 0u, 0u};
+    uint2 block0 = make_uint2(0u, 0u);  // CTA 0's first block: written last
+    const bool fast = fast_ts(ts);
+    for (int j = threadIdx.x; j < nb; j += kOneThreads) {
+        const uint4 *v = reinterpret_cast<const uint4 *>(slice + j * 32);
+        const uint4 v0 = v[0], v1 = v[1];
+        float xv[16];
+        const unsigned wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float2 f = In16<TIn>::to_f2(wv[i]);
+            xv[2 * i] = f.x;
+            xv[2 * i + 1] = f.y;
+        }
+        const BlockOut o = fast ? quantize_block<FMT, true, std::is_same<TIn, __half>::value>(xv, k)
+                                : quantize_block<FMT, false, std::is_same<TIn, __half>::value>(xv, k);
+        const int64_t b = b0 + j;
+        if (b == 0) block0 = o.packed;
+        else reinterpret_cast<uint2 *>(codes)[b] = o.packed;
+        scales[b] = (uint8_t)o.sbyte;
+        if constexpr (HIST) {
+            const unsigned m1 = o.meta & 1u, e = o.effective ? 1u : 0u;
+            cnt[0] += 1u - m1;
+            cnt[1] += m1;
+            cnt[2] += e & (1u - m1);
+            cnt[3] += e & m1;
+        }
+    }
+    if constexpr (HIST) {
+        __shared__ unsigned long long sh[4];
+        if (threadIdx.x < 4) sh[threadIdx.x] = 0ull;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            unsigned cc = cnt[i];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cc += __shfl_xor_sync(0xffffffffu, cc, o);
+            if ((threadIdx.x & 31) == 0 && cc) atomicAdd(&sh[i], (unsigned long long)cc);
+        }
+        __syncthreads();
+        if (threadIdx.x < 4 && sh[threadIdx.x]) atomicAdd(&hist[threadIdx.x], sh[threadIdx.x]);
+    }
+    // 4. block 0's codes and ts, once no CTA reads the barrier words or the amax word
+    if (c == 0 && threadIdx.x == 0) {
+        const uint64_t t0 = globaltimer();
+        while (ld_acquire_u32(&bar[1]) < (unsigned)G && globaltimer() - t0 < kTimeoutNs) __nanosleep(64);
+        if (nb > 0) reinterpret_cast<uint2 *>(codes)[0] = block0;
+        *ts_out = ts;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -590,18 +735,79 @@ static void launch_quant_dt(razer_dtype dt, const void *x, int64_t nblk, const f
     else launch_quant<FMT, __nv_bfloat16>(x, nblk, ts_src, is_amax, codes, scales, hist, st);
 }
 
+// the single-pass kernel takes the call when each SM's slice fits in shared
+// memory (dynamic scale only: a given scale needs no amax pass)
+static bool onepass_eligible(int64_t nblk)
+{
+    const int64_t G = sm_count();
+    return nblk >= G && (nblk + G - 1) / G * 32 <= kOneMaxSlice;
+}
+
+template <int FMT, typename TIn>
+static razer_status launch_onepass(const void *x, int64_t nblk, uint8_t *codes, uint8_t *scales, float *ts_out, unsigned long long *hist,
+                                   cudaStream_t st)
+{
+    const int G = sm_count();
+    const int64_t slice = (nblk + G - 1) / G * 32;
+    static bool attr_done[2][64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool h = hist && Fmt<FMT>::kSpecials > 0;
+    auto kern = h ? quantize_onepass_kernel<FMT, TIn, true> : quantize_onepass_kernel<FMT, TIn, false>;
+    if (dev >= 0 && dev < 64 && !attr_done[h][dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kOneMaxSlice) != cudaSuccess) return RAZER_ERR_CUDA;
+        attr_done[h][dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)G);
+    cfg.blockDim = dim3((unsigned)kOneThreads);
+    cfg.dynamicSmemBytes = (size_t)slice;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident at once: the grid barrier cannot wait on an unscheduled CTA
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int inject = fault_injection_enabled() ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const TIn *>(x), nblk, codes, scales, ts_out, hist, inject);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        (void)cudaGetLastError();
+        return RAZER_ERR_UNSUPPORTED;  // fewer SMs than the device reports (a partitioned GPU): the caller takes the two-pass path
+    }
+    return e == cudaSuccess ? RAZER_OK : RAZER_ERR_CUDA;
+}
+
 // Runs the whole quantizer on one stream.  ts_in == nullptr: dynamic scale
-// (memset + amax + quantize + finalize into ts_out); otherwise static.
+// (the single-pass kernel when each SM's slice fits in shared memory, else
+// memset + amax + quantize + finalize into ts_out); otherwise static.
 razer_status run_quantize(const void *x, razer_dtype dt, int64_t R, int64_t K, const float *ts_in, uint8_t *codes,
                           uint8_t *scales, float *ts_out, unsigned long long *hist, razer_format fmt, cudaStream_t st)
 {
     const int64_t n = R * K;
     const int64_t nblk = n / 16;
     const float C = fmt == RAZER_FMT_WEIGHT ? Fmt<RAZER_FMT_WEIGHT>::kC : Fmt<RAZER_FMT_ACT>::kC;
+    if (!ts_in && onepass_eligible(nblk)) {
+        if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, hist, reinterpret_cast<unsigned *>(ts_out), reinterpret_cast<unsigned *>(codes)) !=
+            cudaSuccess)
+            return RAZER_ERR_CUDA;
+        const bool h = dt == RAZER_F16;
+        razer_status r;
+        if (fmt == RAZER_FMT_WEIGHT)
+            r = h ? launch_onepass<RAZER_FMT_WEIGHT, __half>(x, nblk, codes, scales, ts_out, nullptr, st)
+                  : launch_onepass<RAZER_FMT_WEIGHT, __nv_bfloat16>(x, nblk, codes, scales, ts_out, nullptr, st);
+        else if (fmt == RAZER_FMT_ACT)
+            r = h ? launch_onepass<RAZER_FMT_ACT, __half>(x, nblk, codes, scales, ts_out, hist, st)
+                  : launch_onepass<RAZER_FMT_ACT, __nv_bfloat16>(x, nblk, codes, scales, ts_out, hist, st);
+        else
+            r = h ? launch_onepass<RAZER_FMT_NVFP4, __half>(x, nblk, codes, scales, ts_out, nullptr, st)
+                  : launch_onepass<RAZER_FMT_NVFP4, __nv_bfloat16>(x, nblk, codes, scales, ts_out, nullptr, st);
+        if (r != RAZER_ERR_UNSUPPORTED) return r;
+    }
     // every kernel of the chain is a programmatic dependent of the previous one
     // (it is scheduled early and waits before touching memory)
     if (hist || !ts_in) {
-        if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, hist, ts_in ? (unsigned *)nullptr : reinterpret_cast<unsigned *>(ts_out)) !=
+        if (launch_pdl(quant_init_kernel, 1u, 32u, 0, st, hist, ts_in ? (unsigned *)nullptr : reinterpret_cast<unsigned *>(ts_out),
+                   (unsigned *)nullptr) !=
             cudaSuccess)
             return RAZER_ERR_CUDA;
     }

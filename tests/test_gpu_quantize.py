@@ -143,6 +143,52 @@ def test_quantize_acts_dynamic(orc, dtype):
     np.testing.assert_array_equal(h, oh[[0, 1, 4, 5]].astype(np.int64))
 
 
+def test_quantize_acts_single_pass_matches_given_scale():
+    # the single-pass kernel (dynamic scale; every SM's slice in shared memory)
+    # against the streaming quantizer given the same scale: the full tensor,
+    # bit for bit, with the histogram
+    x = workloads.outlier_activations(2048, 4096, seed=305)
+    c1, s1, t1, h1 = quantize_gpu(x, "act")
+    ts_in = torch.tensor([t1], dtype=torch.float32, device=DEV)
+    c2, s2, t2, h2 = quantize_gpu(x, "act", ts_in=ts_in)
+    assert t2 == t1
+    np.testing.assert_array_equal(c1, c2)
+    np.testing.assert_array_equal(s1, s2)
+    np.testing.assert_array_equal(h1, h2)
+
+
+@pytest.mark.parametrize("R,K", [(1, 148 * 16), (3, 149 * 16), (37, 4096)])
+def test_quantize_acts_single_pass_small_slices(orc, R, K):
+    # one block per SM, one SM with one more block, ragged slices
+    x = workloads.outlier_activations(R, K, seed=R + K)
+    oc, os_, ots, oh = orc.quantize(oracle_in(x), 1)
+    c, s, t, h = quantize_gpu(x, "act")
+    assert t == ots
+    np.testing.assert_array_equal(c, oc)
+    np.testing.assert_array_equal(s, os_)
+    np.testing.assert_array_equal(h, oh[[0, 1, 4, 5]].astype(np.int64))
+
+
+def test_quantize_single_pass_barrier_times_out_and_reports(orc):
+    """One CTA that never reaches the grid barrier (host-side fault
+    injection): the others' bounded waits expire, the device status word
+    reports RAZER_ERR_TIMEOUT, and the next call is correct."""
+    x = workloads.outlier_activations(256, 4096, seed=306)
+    assert R.razer_get_device_status() == 0
+    R.razer_debug_set_fault_injection(True)
+    try:
+        quantize_gpu(x, "act")
+    finally:
+        R.razer_debug_set_fault_injection(False)
+    assert R.razer_get_device_status() == 7  # RAZER_ERR_TIMEOUT, read and cleared
+    oc, os_, ots, _ = orc.quantize(oracle_in(x), 1)
+    c, s, t, _ = quantize_gpu(x, "act")
+    assert R.razer_get_device_status() == 0
+    assert t == ots
+    np.testing.assert_array_equal(c, oc)
+    np.testing.assert_array_equal(s, os_)
+
+
 def test_quantize_acts_full_config_sampled(orc):
     # 2048 tokens x 4096, rows N(0,1), 8 channels x50, bf16
     x = workloads.outlier_activations(2048, 4096, seed=301)
