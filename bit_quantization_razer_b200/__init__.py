@@ -12,5 +12,5 @@ from .razer import (  # noqa: F401
     RAZER_FMT_FOUR_OVER_SIX, RAZER_SCALE_F16,
     razer_get_device_status, razer_quantize_acts, razer_quantize_weights, razer_quantize_weights_batch,
     razer_status_string,
-    razer_version, razer_workspace_size, razer_debug_set_fault_injection,
+    razer_version, razer_workspace_size, razer_debug_set_fault_injection, razer_set_quantize_path,
 )

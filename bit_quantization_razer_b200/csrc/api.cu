@@ -437,6 +437,12 @@ const char *razer_status_string(razer_status s)
 
 int razer_version(void) { return 200; }
 
+int razer_set_quantize_path(int path)
+{
+    if (path != RAZER_QPATH_TWO_PASS && path != RAZER_QPATH_SINGLE_PASS) return -1;
+    return set_single_pass_quantizer(path == RAZER_QPATH_SINGLE_PASS) ? RAZER_QPATH_SINGLE_PASS : RAZER_QPATH_TWO_PASS;
+}
+
 int razer_debug_set_fault_injection(int on)
 {
     return g_fault_injection.exchange(on ? 1 : 0, std::memory_order_relaxed);

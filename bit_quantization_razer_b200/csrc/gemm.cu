@@ -436,6 +436,260 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Persistent GEMM on two bulk-tensor-loaded 16-bit operands (the decode-once
+// path, and the W4A4 product): Y[m, n] = ts * unbias * sum_k X[m, k] Wd[n, k].
+// One CTA per SM walks the work units u = blockIdx.x, + gridDim.x, ... of the
+// (256 x 256 output tile, K split) grid, m-tile fastest so that consecutive
+// units share their weight tile in L2:
+//   * warp 0, lane 0: the bulk-tensor producer.  It runs ahead across units:
+//     while the epilogue drains one unit's accumulator it fills the stages
+//     of the next;
+//   * warp 1, lane 0: the MMA issuer (two M = 128 UMMAs per k-substep share
+//     the B tile); it returns each stage to the producer and hands each
+//     finished accumulator to the epilogue;
+//   * warps 2-9: the epilogue.  Each warp drains its TMEM lane quarter in
+//     32-column chunks, scales them, stages each chunk in shared memory
+//     (16-byte units XOR-swizzled by row, conflict-free both ways) and reads it
+//     back row-contiguous, so every warp store writes whole row segments of
+//     four rows (128 bytes per row in fp32, 64 in 16-bit) instead of sixteen
+//     bytes in each of 32 rows.  The accumulator goes back to the MMA issuer
+//     as soon as every warp has read its last chunk.
+// Every wait is bounded as in gemm_kernel; a timeout stops all roles.
+// ---------------------------------------------------------------------------
+constexpr int kEpiWarps = 8;
+constexpr int kTmaThreads = 32 * (2 + kEpiWarps);
+constexpr uint32_t kTmaStageBytes = 2 * A_HALF_BYTES + (uint32_t)BN * BK * 2;  // X 256 x 64 + W 256 x 64
+constexpr uint32_t kEpiStageBytes = 32 * 128;                                  // one warp's 32 x 32 fp32 chunk
+constexpr uint32_t kTmaSmemBytes = STAGES * kTmaStageBytes + kEpiWarps * kEpiStageBytes + BAR_BYTES + 1024;
+static_assert(kTmaSmemBytes <= 232448, "shared memory of the persistent GEMM");
+
+struct TmaUnit {
+    int m0, n0, kbs, nk, z;
+};
+__device__ __forceinline__ TmaUnit tma_unit(int u, int mt, int T, int S, int kb0, int nkb)
+{
+    TmaUnit w;
+    w.z = u / T;
+    const int t = u - w.z * T;
+    w.m0 = (t % mt) * 256;
+    w.n0 = (t / mt) * BN;
+    w.kbs = kb0 + (int)((int64_t)w.z * nkb / S);
+    w.nk = kb0 + (int)((int64_t)(w.z + 1) * nkb / S) - w.kbs;
+    return w;
+}
+
+template <typename TOut>
+__device__ __forceinline__ void store4(TOut *p, float4 a);
+template <> __device__ __forceinline__ void store4<float>(float *p, float4 a) { *reinterpret_cast<float4 *>(p) = a; }
+template <> __device__ __forceinline__ void store4<__half>(__half *p, float4 a)
+{
+    __half2 lo = __floats2half2_rn(a.x, a.y), hi = __floats2half2_rn(a.z, a.w);
+    *reinterpret_cast<uint2 *>(p) = make_uint2(*reinterpret_cast<unsigned *>(&lo), *reinterpret_cast<unsigned *>(&hi));
+}
+template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, float4 a)
+{
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+    *reinterpret_cast<uint2 *>(p) = make_uint2(*reinterpret_cast<unsigned *>(&lo), *reinterpret_cast<unsigned *>(&hi));
+}
+template <typename TOut> __device__ __forceinline__ void store1(TOut *p, float a);
+template <> __device__ __forceinline__ void store1<float>(float *p, float a) { *p = a; }
+template <> __device__ __forceinline__ void store1<__half>(__half *p, float a) { *p = __float2half_rn(a); }
+template <> __device__ __forceinline__ void store1<__nv_bfloat16>(__nv_bfloat16 *p, float a) { *p = __float2bfloat16_rn(a); }
+
+// One epilogue warp's row-contiguous write of a staged 32 x 32 chunk whose
+// top-left output element is (m, n): lane l writes 4 elements of row
+// 4 p + l / 8, for p = 0..7.
+template <typename TOut>
+__device__ __forceinline__ void epi_write(const uint8_t *stage, int lane, int m, int n, int M, int N, TOut *Y, const float *addend)
+{
+    const int u = lane & 7;
+    const bool vec = (N & 3) == 0;  // rows of whole 4-element groups: 16-byte (fp32) / 8-byte (16-bit) aligned
+#pragma unroll
+    for (int p = 0; p < 8; p++) {
+        const int r = 4 * p + (lane >> 3);
+        float4 a = *reinterpret_cast<const float4 *>(stage + r * 128 + ((u ^ (r & 7)) << 4));
+        const int mm = m + r, nn = n + 4 * u;
+        if (mm >= M || nn >= N) continue;
+        const size_t off = (size_t)mm * (size_t)N + (size_t)nn;
+        if (vec && nn + 4 <= N) {
+            if (addend) {
+                const float4 t = *reinterpret_cast<const float4 *>(addend + off);
+                a.x += t.x;
+                a.y += t.y;
+                a.z += t.z;
+                a.w += t.w;
+            }
+            store4<TOut>(Y + off, a);
+        } else {
+            const float e[4] = {a.x, a.y, a.z, a.w};
+            for (int i = 0; i < 4 && nn + i < N; i++) store1<TOut>(Y + off + i, addend ? e[i] + addend[off + i] : e[i]);
+        }
+    }
+}
+
+template <bool BF16, typename TOut>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    gemm_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w, const float *__restrict__ ts_p,
+                    float unbias, int M, int N, int mt, int T, int S, int kb0, int nkb, TOut *Y, const float *addend, int inject_stall)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *epi = smem + STAGES * kTmaStageBytes;
+    uint8_t *bars = epi + kEpiWarps * kEpiStageBytes;
+    const uint32_t full = smem_addr(bars);       // STAGES x 8
+    const uint32_t empty = full + 8 * STAGES;     // STAGES x 8
+    const uint32_t acc_full = empty + 8 * STAGES;  // 8
+    const uint32_t acc_empty = acc_full + 8;       // 8
+    const uint32_t drained = acc_empty + 8;        // 8: the MMA issuer's own wait after a timeout
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(bars + 192);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 200);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int U = T * S, G = gridDim.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; s++) {
+            mbar_init(full + 8 * s, 1);
+            mbar_init(empty + 8 * s, 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kEpiWarps);
+        mbar_init(drained, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_addr((const void *)tmem_slot)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the decoded operands come from earlier kernels in the stream
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- bulk-tensor producer ----------------
+            uint32_t g = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < U && ok; u += G) {
+                const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb);
+                for (int kb = 0; kb < w.nk; kb++, g++) {
+                    const uint32_t s = g % STAGES, ph = (g / STAGES) & 1u;
+                    if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    // fault injection (tests only): CTA 0 never fills its first stage
+                    if (inject_stall && blockIdx.x == 0 && g == 0) continue;
+                    const uint32_t a0 = smem_addr(smem + s * kTmaStageBytes);
+                    mbar_expect_tx(full + 8 * s, kTmaStageBytes);
+                    tma_load_2d(a0, &tmap_x, (w.kbs + kb) * BK, w.m0, full + 8 * s);
+                    tma_load_2d(a0 + A_HALF_BYTES, &tmap_x, (w.kbs + kb) * BK, w.m0 + 128, full + 8 * s);
+                    tma_load_2d(a0 + 2 * A_HALF_BYTES, &tmap_w, (w.kbs + kb) * BK, w.n0, full + 8 * s);
+                }
+            }
+            if (!ok) {
+                // let the loads already issued land before the CTA exits (bounded)
+                const uint64_t t0 = globaltimer();
+                for (uint32_t gg = g > (uint32_t)STAGES ? g - STAGES : 0u; gg < g; gg++) {
+                    if (inject_stall && blockIdx.x == 0 && gg == 0) continue;
+                    while (!mbar_try_wait(full + 8 * (gg % STAGES), (gg / STAGES) & 1u) && globaltimer() - t0 < kTimeoutNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            const uint32_t idesc = idesc_f16(BF16, 128, BN);
+            uint32_t g = 0, ti = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < U && ok; u += G, ti++) {
+                const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb);
+                // the epilogue has drained the previous unit's accumulator
+                if (!mbar_wait(acc_empty, (ti & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < w.nk; kb++, g++) {
+                    const uint32_t s = g % STAGES, ph = (g / STAGES) & 1u;
+                    if (!mbar_wait(full + 8 * s, ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_addr(smem + s * kTmaStageBytes);
+                    const uint32_t b0 = a0 + 2 * A_HALF_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; k++) {
+                        const uint64_t bd = smem_desc_k128(b0 + 32 * k);
+                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                        umma_f16(tmem, smem_desc_k128(a0 + 32 * k), bd, idesc, acc);
+                        umma_f16(tmem + BN, smem_desc_k128(a0 + A_HALF_BYTES + 32 * k), bd, idesc, acc);
+                    }
+                    umma_commit(empty + 8 * s);
+                }
+                if (ok) umma_commit(acc_full);
+            }
+            // every MMA issued has completed before the TMEM is freed (bounded)
+            umma_commit(drained);
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(drained, 0) && globaltimer() - t0 < kTimeoutNs) {
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int q = warp & 3;                          // TMEM lane quarter this warp may access
+        const int cbeg = ((warp - 2) >> 2) * (BN / 2);   // the two warps of a quarter split the columns
+        uint8_t *stage = epi + (warp - 2) * kEpiStageBytes;
+        const float scale = __fmul_rn(*ts_p, unbias);
+        TOut *Yz = Y;
+        uint32_t ti = 0;
+        for (int u = blockIdx.x; u < U; u += G, ti++) {
+            const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb);
+            if (!mbar_wait_warp(acc_full, ti & 1u, abort_flag)) break;
+            tc_fence_after();
+            Yz = Y + (S > 1 ? (size_t)w.z * (size_t)M * (size_t)N : 0);
+#pragma unroll 1
+            for (int c = 0; c < 2 * (BN / 2) / 32; c++) {
+                const int half = c / ((BN / 2) / 32), col = cbeg + 32 * (c % ((BN / 2) / 32));
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * BN + col), v);
+                if (c == 2 * (BN / 2) / 32 - 1) {
+                    // this warp has read the whole accumulator: hand it back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(acc_empty);
+                }
+                // an empty K range leaves the accumulator unwritten: its sum is 0
+                if (w.nk == 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; i++) v[i] = 0.0f;
+                }
+                // stage row `lane` (16-byte unit j at j ^ (lane & 7))
+#pragma unroll
+                for (int j = 0; j < 8; j++)
+                    *reinterpret_cast<float4 *>(stage + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                        make_float4(v[4 * j] * scale, v[4 * j + 1] * scale, v[4 * j + 2] * scale, v[4 * j + 3] * scale);
+                __syncwarp();
+                epi_write<TOut>(stage, lane, w.m0 + half * 128 + q * 32, w.n0 + col, M, N, Yz, S > 1 ? nullptr : addend);
+                __syncwarp();
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncwarp();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    }
+}
+
 // Decodes the packed weights once into a [N, K] 16-bit copy holding
 // q*s*2^-bias (the exact values the fused kernel writes to shared memory);
 // one thread per 16-element block.
@@ -646,6 +900,43 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, cons
     return last_launch_status();
 }
 
+// the persistent GEMM on two decoded 16-bit operands; S > 1 writes fp32
+// slices (out = the slice buffer, out_dt = RAZER_F32)
+template <bool BF16, typename TOut>
+static razer_status launch_tma_t(const CUtensorMap &map, const CUtensorMap &wmap, const float *ts, float unbias, int M, int N, TOut *out,
+                                 int kb0, int nkb, const float *addend, cudaStream_t st, int S)
+{
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(gemm_tma_kernel<BF16, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTmaSmemBytes) !=
+            cudaSuccess)
+            return RAZER_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    const int mt = (M + 255) / 256, nt = (N + BN - 1) / BN, T = mt * nt;
+    const int G = (int)std::min<int64_t>((int64_t)T * S, sm_count());
+    // fault injection (tests only): CTA 0 leaves its first stage unfilled so
+    // that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
+    const int inject = fault_injection_enabled() ? 1 : 0;
+    if (launch_pdl(gemm_tma_kernel<BF16, TOut>, (unsigned)G, (unsigned)kTmaThreads, (size_t)kTmaSmemBytes, st, map, wmap, ts, unbias, M, N,
+                   mt, T, S, kb0, nkb, out, addend, inject) != cudaSuccess)
+        return RAZER_ERR_CUDA;
+    return RAZER_OK;
+}
+
+template <bool BF16>
+static razer_status launch_tma(const CUtensorMap &map, const CUtensorMap &wmap, const float *ts, float unbias, int M, int N, void *out,
+                               razer_dtype out_dt, int kb0, int nkb, const float *addend, cudaStream_t st, int S)
+{
+    if (out_dt == RAZER_F32)
+        return launch_tma_t<BF16, float>(map, wmap, ts, unbias, M, N, reinterpret_cast<float *>(out), kb0, nkb, addend, st, S);
+    if (out_dt == RAZER_F16)
+        return launch_tma_t<BF16, __half>(map, wmap, ts, unbias, M, N, reinterpret_cast<__half *>(out), kb0, nkb, addend, st, S);
+    return launch_tma_t<BF16, __nv_bfloat16>(map, wmap, ts, unbias, M, N, reinterpret_cast<__nv_bfloat16 *>(out), kb0, nkb, addend, st, S);
+}
+
 template <int FMT, bool BF16>
 static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, bool decoded, const uint8_t *codes, const uint8_t *scales,
                                const float *ts, float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, void *wdec,
@@ -662,7 +953,7 @@ static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, 
     const int S = gemm_splits(M, N, K);
     void *out = S > 1 ? static_cast<void *>(slices) : Y;
     const razer_dtype odt = S > 1 ? RAZER_F32 : out_dt;
-    const razer_status r = decoded ? launch<FMT, BF16, true>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S)
+    const razer_status r = decoded ? launch_tma<BF16>(map, wmap, ts, unbias, M, N, out, odt, 0, KB, nullptr, st, S)
                                    : launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S);
     if (r != RAZER_OK || S == 1) return r;
     if (N % 4 != 0) {
@@ -755,8 +1046,8 @@ static razer_status w4a4_product(const float *ts_a, razer_format afmt, int64_t M
     for (int c = 0; c < nc; c++) {
         const int kb0 = (int)((int64_t)c * KB / nc), kb1 = (int)((int64_t)(c + 1) * KB / nc);
         const bool last = c == nc - 1;
-        r = launch<RAZER_FMT_WEIGHT, false, true>(amap, wmap, nullptr, nullptr, tsp, unbias, m, n, k, last ? Y : partial,
-                                                  last ? out_dt : RAZER_F32, kb0, kb1 - kb0, c > 0 ? partial : nullptr, st);
+        r = launch_tma<false>(amap, wmap, tsp, unbias, m, n, last ? Y : partial, last ? out_dt : RAZER_F32, kb0, kb1 - kb0,
+                              c > 0 ? partial : nullptr, st, 1);
         if (r != RAZER_OK) return r;
     }
     return RAZER_OK;

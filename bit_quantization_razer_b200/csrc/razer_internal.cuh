@@ -165,4 +165,6 @@ razer_status last_launch_status();
 // Test-only fault injection (razer_debug_set_fault_injection): a plain load
 // on the launch path, no environment lookup per call.
 bool fault_injection_enabled();
+// dynamic-scale quantizer path (false: two-pass); returns the previous value
+bool set_single_pass_quantizer(bool on);
 }  // namespace razer

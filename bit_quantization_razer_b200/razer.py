@@ -34,7 +34,7 @@ EXPORTED = (
     "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4", "razer_gemm_w4a4_online", "razer_quant_error",
     "razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
-    "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch", "razer_debug_set_fault_injection",
+    "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch", "razer_debug_set_fault_injection", "razer_set_quantize_path",
 )
 
 
@@ -92,6 +92,8 @@ def load() -> ctypes.CDLL:
     L.razer_version.argtypes = []
     L.razer_debug_set_fault_injection.argtypes = [i32]
     L.razer_debug_set_fault_injection.restype = ctypes.c_int
+    L.razer_set_quantize_path.argtypes = [i32]
+    L.razer_set_quantize_path.restype = ctypes.c_int
     for fn in ("razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant", "razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
@@ -373,7 +375,20 @@ def razer_version() -> int:
     return int(load().razer_version())
 
 
+RAZER_QPATH_TWO_PASS, RAZER_QPATH_SINGLE_PASS = 0, 1
+QUANTIZE_PATHS = {"two_pass": RAZER_QPATH_TWO_PASS, "single_pass": RAZER_QPATH_SINGLE_PASS}
+
+
+def razer_set_quantize_path(path: str) -> str:
+    """Selects the dynamic-scale quantizer path ("two_pass", the default, or
+    "single_pass"); returns the previous one."""
+    if path not in QUANTIZE_PATHS:
+        raise ValueError(f"unknown quantizer path {path!r}")
+    prev = int(load().razer_set_quantize_path(QUANTIZE_PATHS[path]))
+    return "single_pass" if prev == RAZER_QPATH_SINGLE_PASS else "two_pass"
+
+
 def razer_debug_set_fault_injection(on: bool) -> bool:
-    """Test-only: turns the GEMV / GEMM stall injection on or off; returns
-    the previous setting."""
+    """Test-only: turns the GEMV / GEMM / single-pass quantizer stall
+    injection on or off; returns the previous setting."""
     return bool(load().razer_debug_set_fault_injection(1 if on else 0))

@@ -426,10 +426,37 @@ const char *razer_status_string(razer_status status);
 int razer_version(void);
 
 /*
+ * razer_set_quantize_path -- how razer_quantize_weights and
+ * razer_quantize_acts compute a DYNAMIC tensor scale (ts_in == NULL);
+ * process-wide, default RAZER_QPATH_TWO_PASS.  Both paths write identical
+ * codes, scales, ts and histogram.
+ *   RAZER_QPATH_TWO_PASS     an amax kernel, then the block quantizer reads X
+ *                            again (from L2 when X fits there).
+ *   RAZER_QPATH_SINGLE_PASS  one cooperative kernel, one CTA per SM: each CTA
+ *                            copies its contiguous slice of blocks into shared
+ *                            memory, the CTAs merge their amax and meet at a
+ *                            grid barrier (bounded wait: on expiry the outputs
+ *                            are void and razer_get_device_status reports
+ *                            RAZER_ERR_TIMEOUT), then each quantizes its slice
+ *                            from shared memory: X is read from HBM once.
+ *                            Taken when at least one block per SM exists and
+ *                            each slice fits in 224 KB (X of at most
+ *                            SMs x 224 KB); other sizes and partitioned GPUs
+ *                            that cannot hold every CTA at once use the
+ *                            two-pass path.  The batched weight quantizer is
+ *                            not affected.
+ * Returns the previous setting, or -1 (and changes nothing) for an unknown
+ * value.  Not meant to be changed while other threads launch quantizers.
+ */
+typedef enum { RAZER_QPATH_TWO_PASS = 0, RAZER_QPATH_SINGLE_PASS = 1 } razer_qpath;
+int razer_set_quantize_path(int path);
+
+/*
  * razer_debug_set_fault_injection -- for tests of the failure path only (the
  * paper has no counterpart).  While on (on != 0), each launch of the
- * bulk-tensor razer_gemv kernel leaves one pipeline stage of one CTA unfilled
- * and each razer_gemm launch withholds one decoder warp's arrivals, so their
+ * bulk-tensor razer_gemv kernel leaves one pipeline stage of one CTA unfilled,
+ * each razer_gemm launch withholds one decoder warp's arrivals and one CTA of
+ * the single-pass quantizer never arrives at its grid barrier, so their
  * bounded waits expire: the call still returns RAZER_OK and
  * razer_get_device_status then reports RAZER_ERR_TIMEOUT; outputs of such a
  * call are void.  No GPU fault, trap or hang results.  Returns the previous

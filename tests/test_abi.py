@@ -161,6 +161,18 @@ def test_variant_decode_validation(lib):
     assert d(*dargs(R=0)) == 0                                         # empty tensor
 
 
+def test_quantize_path_selector(lib):
+    # host-side setting only: no kernel runs
+    lib.razer_set_quantize_path.restype = ctypes.c_int
+    lib.razer_set_quantize_path.argtypes = [ctypes.c_int]
+    assert lib.razer_set_quantize_path(7) == -1
+    assert lib.razer_set_quantize_path(-1) == -1
+    prev = lib.razer_set_quantize_path(1)
+    assert prev == 0  # two-pass is the default
+    assert lib.razer_set_quantize_path(0) == 1
+    assert lib.razer_set_quantize_path(0) == 0
+
+
 def test_workspace_size_host_logic(lib):
     assert razer.razer_workspace_size(razer.RAZER_OP_GEMV, 0, 64, 128) == 0
     def split_k(B, N, K):  # per-warp kernel: ~8 CTAs per SM (148 without a GPU), >= 2 chunks per split

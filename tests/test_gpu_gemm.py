@@ -155,6 +155,51 @@ def test_gemm_bounded_wait_times_out_and_reports():
     assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
 
 
+def test_gemm_persistent_bounded_wait_times_out_and_reports():
+    """The decode-once path's persistent kernel: one CTA never fills its first
+    stage (host-side fault injection), the MMA issuer's bounded wait expires,
+    every role stops, the tensor memory is freed and the status word reports
+    RAZER_ERR_TIMEOUT; the next call is correct."""
+    M, N, K = 1024, 512, 256
+    codes, scales = workloads.random_packed(N, K, "weight", seed=92)
+    X = workloads.vectors(M, K, seed=93, dtype=torch.bfloat16).to(DEV)
+    c, s = codes.to(DEV), scales.to(DEV)
+    ts = torch.ones(1, device=DEV)
+    assert R.razer_get_device_status() == 0
+    R.razer_debug_set_fault_injection(True)
+    try:
+        R.razer_gemm(X, c, s, ts, "weight", torch.float32)
+    finally:
+        R.razer_debug_set_fault_injection(False)
+    assert R.razer_get_device_status() == 7
+    assert R.razer_get_device_status() == 0
+    Y = R.razer_gemm(X, c, s, ts, "weight", torch.float32)
+    torch.cuda.synchronize()
+    import oracle
+    rows = np.arange(0, M, 37)
+    ref = oracle.gemm_ref(oracle_in(X.cpu()[rows]), codes.numpy(), scales.numpy(), 1.0, 0)
+    assert rel_err(Y.cpu().numpy()[rows], ref) <= REL_TOL
+
+
+@pytest.mark.parametrize("M,N,K", [(1024, 256, 64), (1280, 640, 192), (4096, 4096, 512), (1100, 300, 128), (1024, 258, 4096)])
+def test_gemm_persistent_units(M, N, K):
+    """Unit walk of the persistent kernel: fewer units than SMs, several
+    units per CTA with ragged last tiles (M, N not multiples of 256), and
+    rows of N % 4 != 0 elements (scalar stores); every row is checked."""
+    codes, scales = workloads.random_packed(N, K, "weight", seed=M + N + K, max_scale_code=40)
+    X = workloads.vectors(M, K, seed=94, dtype=torch.bfloat16)
+    ts = torch.tensor([0.02], device=DEV)
+    Y = R.razer_gemm(X.to(DEV), codes.to(DEV), scales.to(DEV), ts, "weight", torch.float32)
+    torch.cuda.synchronize()
+    import oracle
+    ref = oracle.gemm_ref(oracle_in(X), codes.numpy(), scales.numpy(), 0.02, 0)
+    assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
+    # the bf16 output is the fp32 result rounded once
+    Yb = R.razer_gemm(X.to(DEV), codes.to(DEV), scales.to(DEV), ts, "weight", torch.bfloat16)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(Yb.cpu().float().numpy(), torch.from_numpy(Y.cpu().numpy()).to(torch.bfloat16).float().numpy())
+
+
 @pytest.mark.parametrize("M,N,K,fmt", [(512, 28672, 8192, "weight"), (2048, 8192, 28672, "weight"), (8192, 8192, 8192, "nvfp4"),
                                        (1024, 4096, 4096, "act")])
 def test_gemm_70b_sweep_sampled(orc, M, N, K, fmt):

@@ -13,6 +13,26 @@ pytestmark = [pytest.mark.gpu, cuda]
 DEV = "cuda:0"
 
 
+@pytest.fixture(params=["two_pass", "single_pass"])
+def qpath(request):
+    """Runs a dynamic-scale test once per quantizer path (both must give the
+    oracle's bits)."""
+    prev = R.razer_set_quantize_path(request.param)
+    try:
+        yield request.param
+    finally:
+        R.razer_set_quantize_path(prev)
+
+
+@pytest.fixture
+def single_pass():
+    prev = R.razer_set_quantize_path("single_pass")
+    try:
+        yield
+    finally:
+        R.razer_set_quantize_path(prev)
+
+
 def quantize_gpu(x: torch.Tensor, fmt: str, ts_in=None):
     x = x.to(DEV)
     if fmt == "act":
@@ -41,7 +61,7 @@ def test_worked_rows_gpu(orc, case):
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("fmt", ["weight", "nvfp4"])
-def test_quantize_weights_tiny_config(orc, dtype, fmt):
+def test_quantize_weights_tiny_config(orc, dtype, fmt, qpath):
     # 256 x 512, N(0, 0.02^2), 0.1% x10 outliers, seed 0
     w = workloads.weight(256, 512, std=0.02, seed=0, dtype=dtype)
     oc, os_, ots, _ = orc.quantize(oracle_in(w), FMT_ID[fmt])
@@ -133,7 +153,7 @@ def test_quantize_weights_batch_llama8b_equals_single_calls(orc):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-def test_quantize_acts_dynamic(orc, dtype):
+def test_quantize_acts_dynamic(orc, dtype, qpath):
     x = workloads.outlier_activations(256, 4096, seed=300, dtype=dtype)
     oc, os_, ots, oh = orc.quantize(oracle_in(x), 1)
     c, s, t, h = quantize_gpu(x, "act")
@@ -143,7 +163,7 @@ def test_quantize_acts_dynamic(orc, dtype):
     np.testing.assert_array_equal(h, oh[[0, 1, 4, 5]].astype(np.int64))
 
 
-def test_quantize_acts_single_pass_matches_given_scale():
+def test_quantize_acts_single_pass_matches_given_scale(single_pass):
     # the single-pass kernel (dynamic scale; every SM's slice in shared memory)
     # against the streaming quantizer given the same scale: the full tensor,
     # bit for bit, with the histogram
@@ -157,10 +177,11 @@ def test_quantize_acts_single_pass_matches_given_scale():
     np.testing.assert_array_equal(h1, h2)
 
 
-@pytest.mark.parametrize("R,K", [(1, 148 * 16), (3, 149 * 16), (37, 4096)])
-def test_quantize_acts_single_pass_small_slices(orc, R, K):
-    # one block per SM, one SM with one more block, ragged slices
-    x = workloads.outlier_activations(R, K, seed=R + K)
+@pytest.mark.parametrize("M,K", [(1, 148 * 16), (3, 149 * 16), (37, 4096), (1, 147 * 16)])
+def test_quantize_acts_small_slices(orc, M, K, qpath):
+    # one block per SM, one SM with one more block, ragged slices, fewer
+    # blocks than SMs (the single-pass path hands that to the two-pass one)
+    x = workloads.outlier_activations(M, K, seed=M + K)
     oc, os_, ots, oh = orc.quantize(oracle_in(x), 1)
     c, s, t, h = quantize_gpu(x, "act")
     assert t == ots
@@ -169,7 +190,7 @@ def test_quantize_acts_single_pass_small_slices(orc, R, K):
     np.testing.assert_array_equal(h, oh[[0, 1, 4, 5]].astype(np.int64))
 
 
-def test_quantize_single_pass_barrier_times_out_and_reports(orc):
+def test_quantize_single_pass_barrier_times_out_and_reports(orc, single_pass):
     """One CTA that never reaches the grid barrier (host-side fault
     injection): the others' bounded waits expire, the device status word
     reports RAZER_ERR_TIMEOUT, and the next call is correct."""
@@ -189,7 +210,7 @@ def test_quantize_single_pass_barrier_times_out_and_reports(orc):
     np.testing.assert_array_equal(s, os_)
 
 
-def test_quantize_acts_full_config_sampled(orc):
+def test_quantize_acts_full_config_sampled(orc, qpath):
     # 2048 tokens x 4096, rows N(0,1), 8 channels x50, bf16
     x = workloads.outlier_activations(2048, 4096, seed=301)
     xin = oracle_in(x)
