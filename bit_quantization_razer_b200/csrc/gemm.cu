@@ -788,10 +788,15 @@ __global__ void ts_product_kernel(const float *__restrict__ a, const float *__re
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-// decode once and run the plain 16-bit GEMM when M is large enough that the
-// fused kernel would decode every weight many times (M / BM) and the caller
-// provided the N x K x 2 bytes of workspace
+// decode once and run the persistent 16-bit GEMM when M is large enough that
+// the fused kernel would decode every weight many times (M / BM), and for
+// M >= 256 when the weight matrix is small enough that its decoded copy is
+// cheap: measured on a B200 (bf16 out), M = 512: 4096 x 4096 47.1 -> 37.6 us,
+// but 14336 x 4096 83.2 -> 92.7 us and 28672 x 8192 292 -> 342 us; M = 256:
+// 4096 x 4096 38.4 -> 32.5 us, 14336 x 4096 63.1 -> 77.2 us
 constexpr int64_t kDecodedMinM = 1024;
+constexpr int64_t kDecodedSmallMinM = 256;
+constexpr int64_t kDecodedSmallMaxNK = int64_t(1) << 25;
 
 // Longest K one tensor-memory accumulation chain covers. The tcgen05 fp32
 // accumulator loses precision over long chains (measured on B200 with
@@ -812,7 +817,8 @@ static int64_t num_chunks(int64_t K) { return (K + kMaxChainK - 1) / kMaxChainK;
 static bool gemm_generic(int64_t N, int64_t K) { return K % BK != 0 || N % 16 != 0; }
 static size_t decoded_bytes(int64_t M, int64_t N, int64_t K)
 {
-    return (M >= kDecodedMinM || gemm_generic(N, K)) ? (size_t)N * (size_t)K * 2 : 0;
+    const bool small_w = M >= kDecodedSmallMinM && N * K <= kDecodedSmallMaxNK;
+    return (M >= kDecodedMinM || small_w || gemm_generic(N, K)) ? (size_t)N * (size_t)K * 2 : 0;
 }
 static size_t partial_bytes(int64_t M, int64_t N, int64_t K) { return num_chunks(K) > 1 ? (size_t)M * (size_t)N * 4 : 0; }
 

@@ -211,9 +211,13 @@ def test_workspace_size_host_logic(lib):
     assert splits(256, 256, 4096) == 8 and splits(512, 28672, 8192) == 1 and splits(2048, 8192, 28672) == 2
     assert razer.razer_workspace_size(G, 8192, 8192, 8192) == 8192 * 8192 * 2
     assert razer.razer_workspace_size(G, 4096, 14336, 4096) == 14336 * 4096 * 2
-    assert razer.razer_workspace_size(G, 256, 256, 256) == 0
-    for M, N, K in ((1023, 4096, 16384), (512, 8192, 16448), (512, 8192, 8192), (256, 256, 4096), (512, 28672, 8192),
-                    (512, 8192, 28672)):
+    # M >= 256 with at most 2^25 weights also decodes once
+    assert razer.razer_workspace_size(G, 256, 256, 256) == 256 * 256 * 2
+    assert razer.razer_workspace_size(G, 255, 256, 256) == 0
+    assert razer.razer_workspace_size(G, 256, 256, 4096) == 256 * 4096 * 2 + slices(256, 256, 4096)
+    assert razer.razer_workspace_size(G, 512, 4096, 8192) == 4096 * 8192 * 2 + slices(512, 4096, 8192)
+    for M, N, K in ((1023, 4096, 16384), (512, 8192, 16448), (512, 8192, 8192), (255, 256, 4096), (512, 28672, 8192),
+                    (512, 8192, 28672), (512, 4112, 8192)):
         assert razer.razer_workspace_size(G, M, N, K) == slices(M, N, K), (M, N, K)
     assert razer.razer_workspace_size(G, 1024, 4096, 16384) == 4096 * 16384 * 2 + slices(1024, 4096, 16384)
     assert razer.razer_workspace_size(G, 2048, 8192, 28672) == 8192 * 28672 * 2 + 2 * 2048 * 8192 * 4

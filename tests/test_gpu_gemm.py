@@ -40,11 +40,14 @@ def test_gemm_fewer_rows_than_a_tile(orc, M):
     assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
 
 
+@pytest.mark.parametrize("M", [200, 300])
 @pytest.mark.parametrize("fmt", ["weight", "act", "nvfp4"])
 @pytest.mark.parametrize("xdt", [torch.bfloat16, torch.float16])
-def test_gemm_ragged_multi_tile(orc, fmt, xdt):
-    # M tail (300 rows), N not a multiple of 32, 3 k-steps (one pass over the stages)
-    M, N, K = 300, 272, 192
+def test_gemm_ragged_multi_tile(orc, fmt, xdt, M):
+    # M tail (200 rows: the fused in-shared-memory decode; 300 rows: the
+    # decode-once path), N not a multiple of 32, 3 k-steps (one pass over the
+    # stages)
+    N, K = 272, 192
     codes, scales = workloads.random_packed(N, K, fmt, seed=72, max_scale_code=None)
     X = workloads.vectors(M, K, seed=73, dtype=xdt)
     ts = 0.0371
@@ -53,11 +56,13 @@ def test_gemm_ragged_multi_tile(orc, fmt, xdt):
     assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
 
 
-def test_gemm_oracle_quantized_weights(orc):
-    # realistic weights quantized by the oracle; 8 k-steps wrap the 3-stage ring
+@pytest.mark.parametrize("M", [240, 512])
+def test_gemm_oracle_quantized_weights(orc, M):
+    # realistic weights quantized by the oracle; 8 k-steps wrap the 3-stage
+    # ring (M = 240: fused decode, M = 512: decode-once)
     w = workloads.weight(512, 512, std=0.02, seed=74)
     codes, scales, ts, _ = orc.quantize(w.numpy(), 0)
-    X = workloads.vectors(512, 512, seed=75, dtype=torch.bfloat16)
+    X = workloads.vectors(M, 512, seed=75, dtype=torch.bfloat16)
     ref = orc.gemm_ref(oracle_in(X), codes, scales, ts, 0)
     for odt in (torch.float32, torch.bfloat16, torch.float16):
         Y = gemm(X, torch.from_numpy(codes), torch.from_numpy(scales), ts, "weight", odt)
@@ -136,7 +141,7 @@ def test_gemm_bounded_wait_times_out_and_reports():
     memory, and the device status word reports RAZER_ERR_TIMEOUT; the context
     stays usable."""
     codes, scales = workloads.random_packed(256, 64, "weight", seed=90)
-    X = workloads.vectors(256, 64, seed=91, dtype=torch.bfloat16).to(DEV)
+    X = workloads.vectors(128, 64, seed=91, dtype=torch.bfloat16).to(DEV)  # M < 256: the fused kernel
     c, s = codes.to(DEV), scales.to(DEV)
     ts = torch.ones(1, device=DEV)
     assert R.razer_get_device_status() == 0
@@ -229,8 +234,11 @@ def test_gemm_decoded_path_f16_and_garbage_workspace(orc, xdt):
     assert R.razer_get_device_status() == 0
     ref = orc.gemm_ref(oracle_in(X), codes.numpy(), scales.numpy(), 0.05, 0)
     assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
-    # below the threshold no workspace is needed (fused decode)
-    assert R.razer_workspace_size(R.RAZER_OP_GEMM, 1023, N, K) == 0
+    # below M = 256, and below M = 1024 for weight matrices of more than 2^25
+    # elements, no workspace is needed (fused decode)
+    assert R.razer_workspace_size(R.RAZER_OP_GEMM, 255, N, K) == 0
+    assert R.razer_workspace_size(R.RAZER_OP_GEMM, 1023, 8192, 8192) == 0
+    assert R.razer_workspace_size(R.RAZER_OP_GEMM, 1023, N, K) == N * K * 2
 
 
 # --- W4A4 product of two RaZeR-packed operands ------------------------------
