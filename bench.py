@@ -710,6 +710,7 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
             R.razer_set_quantize_path(prev)
         paths[path] = ms_p
     ms = paths["two_pass"]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n = 2048 * 4096
     h = hist.cpu().tolist()
     nblk = n // 16
@@ -838,6 +839,23 @@ def run_extras(R, workloads, dev, stream, hbm, bf16):
             res[f"B{B}"] = {"ms": ms, "GB/s": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm}
         gv[name] = res
     out["gemv_variant_14336x4096"] = gv
+    # prefill GEMM on variant weights (M = 4096, 4096 x 4096): the pages'
+    # format with fp16 activations and a per-model pair at block 16 with bf16
+    # activations; the time includes the decode of the weight copy
+    M, N, K = 4096, 4096, 4096
+    gmv = {}
+    for name, block, sfmt, V, xdt in (("block128_f16_scale_pm5_pm8_fp16", 128, "f16_scale", [5.0, -5.0, 8.0, -8.0], torch.float16),
+                                      ("block16_e3m3_pm5_pm7_bf16", 16, "weight", [5.0, -5.0, 7.0, -7.0], torch.bfloat16)):
+        c0, s0 = workloads.random_packed_variant(N, K, block, sfmt, len(V), seed=409)
+        c0, s0 = c0.to(dev), s0.to(dev)
+        tsv = torch.tensor([1.0 if sfmt == "f16_scale" else 2.0 ** -9], dtype=torch.float32, device=dev)
+        Xv = workloads.vectors(M, K, seed=410, dtype=xdt).to(dev)
+        Yv = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        wsv = torch.empty(R.razer_workspace_size(R.RAZER_OP_GEMM_VARIANT, M, N, K), dtype=torch.uint8, device=dev)
+        ms = time_graph(lambda: R.razer_gemm_variant(Xv, c0, s0, tsv, block, sfmt, V, torch.bfloat16, out=Yv, workspace=wsv), 1, stream)
+        tf = 2 * M * N * K / ms / 1e9
+        gmv[name] = {"ms": ms, "TFLOP/s": tf, "frac": tf / bf16}
+    out["gemm_variant_4096x4096x4096"] = gmv
     out["llama3_70b_sweep"] = run_70b_sweep(R, workloads, dev, stream, hbm, bf16)
     # the tiny case the oracle checks in full (launch-bound: time only)
     Wt = workloads.weight(256, 512, seed=0).to(dev)

@@ -67,6 +67,10 @@ razer_status run_gemm_w4a4(const uint8_t *codes_a, const uint8_t *scales_a, cons
                            const uint8_t *codes_w, const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K,
                            void *Y, razer_dtype out_dt, void *workspace, cudaStream_t st);
 size_t gemm_w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+size_t gemm_variant_workspace_bytes(int64_t M, int64_t N, int64_t K);
+razer_status run_gemm_variant(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                              int block, razer_format sfmt, const VariantV &V, int64_t N, int64_t K, void *Y, razer_dtype out_dt,
+                              void *workspace, cudaStream_t st);
 razer_status run_gemm_w4a4_online(const void *X, razer_dtype x_dt, int64_t M, const float *ts_in, razer_format afmt, uint8_t *codes_a,
                                   uint8_t *scales_a, float *ts_a_out, unsigned long long *hist, const uint8_t *codes_w,
                                   const uint8_t *scales_w, const float *ts_w, razer_format wfmt, int64_t N, int64_t K, void *Y,
@@ -160,6 +164,7 @@ size_t razer_workspace_size(razer_op op, int64_t M_or_B, int64_t N, int64_t K)
     if (op == RAZER_OP_GEMV) return gemv_workspace_bytes(M_or_B, N, K);
     if (op == RAZER_OP_GEMM) return gemm_workspace_bytes(M_or_B, N, K);
     if (op == RAZER_OP_GEMM_W4A4) return M_or_B > 0 && N > 0 && K > 0 ? gemm_w4a4_workspace_bytes(M_or_B, N, K) : 0;
+    if (op == RAZER_OP_GEMM_VARIANT) return gemm_variant_workspace_bytes(M_or_B, N, K);
     return 0;
 }
 
@@ -367,6 +372,34 @@ static bool rounds_in_bf16(const VariantV &V)
         }
     }
     return false;
+}
+
+razer_status razer_gemm_variant(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                int block, razer_format scale_fmt, const float *special_values, int n_special, int64_t N, int64_t K,
+                                void *Y, razer_dtype out_dt, void *workspace, size_t ws_bytes, razer_stream_t stream)
+{
+    VariantV V;
+    razer_status st = check_variant(N, K, block, scale_fmt, special_values, n_special, V);
+    if (st != RAZER_OK) return st;
+    if (!ts || (!X && M * K > 0) || (!Y && M * N > 0) || (N * K > 0 && (!codes || !scales))) return RAZER_ERR_INVALID_ARG;
+    if (!valid_dt(act_dt) || !valid_dt(out_dt)) return RAZER_ERR_INVALID_ARG;
+    if (!in16(act_dt)) return RAZER_ERR_DTYPE;
+    if (M < 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return RAZER_ERR_SHAPE;
+    // the 16-bit weight copy must hold q*s: bf16 holds it exactly for byte
+    // scales without +-9.5 (FP16 scale words take two terms in either type)
+    if (act_dt == RAZER_BF16 && scale_fmt != RAZER_SCALE_F16 && rounds_in_bf16(V)) return RAZER_ERR_UNSUPPORTED;
+    if (scale_fmt == RAZER_SCALE_F16 && K % 64 != 0) return RAZER_ERR_UNSUPPORTED;  // the two-term copy takes whole k-steps
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ts, 4) || !aligned(codes, 8) || (scale_fmt == RAZER_SCALE_F16 && !aligned(scales, 2)))
+        return RAZER_ERR_ALIGN;
+    if (M == 0 || N == 0) return RAZER_OK;
+    if (K == 0)  // empty sums: Y = 0
+        return cudaMemsetAsync(Y, 0, (size_t)M * (size_t)N * (out_dt == RAZER_F32 ? 4 : 2), (cudaStream_t)stream) == cudaSuccess
+                   ? RAZER_OK
+                   : RAZER_ERR_CUDA;
+    const size_t need = gemm_variant_workspace_bytes(M, N, K);
+    if (!workspace || ws_bytes < need) return RAZER_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return RAZER_ERR_ALIGN;
+    return run_gemm_variant(X, act_dt, M, codes, scales, ts, block, scale_fmt, V, N, K, Y, out_dt, workspace, (cudaStream_t)stream);
 }
 
 razer_status razer_gemv_variant(const void *x, razer_dtype act_dt, int64_t B, const uint8_t *codes, const uint8_t *scales, const float *ts,

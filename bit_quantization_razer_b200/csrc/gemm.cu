@@ -31,6 +31,7 @@
 
 #include "razer_internal.cuh"
 #include "sm100_async.cuh"
+#include "variant.cuh"
 
 namespace razer {
 namespace gemm {
@@ -531,7 +532,8 @@ __device__ __forceinline__ void epi_write(const uint8_t *stage, int lane, int m,
 template <bool BF16, typename TOut>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     gemm_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w, const float *__restrict__ ts_p,
-                    float unbias, int M, int N, int mt, int T, int S, int kb0, int nkb, TOut *Y, const float *addend, int inject_stall)
+                    float unbias, int M, int N, int mt, int T, int S, int kb0, int nkb, TOut *Y, const float *addend, int inject_stall,
+                    int kx_wrap)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -584,9 +586,12 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                     // fault injection (tests only): CTA 0 never fills its first stage
                     if (inject_stall && blockIdx.x == 0 && g == 0) continue;
                     const uint32_t a0 = smem_addr(smem + s * kTmaStageBytes);
+                    // kx_wrap > 0: the weight operand has kx_wrap k-steps per X pass
+                    // ([W_hi | W_lo] against [X | X])
+                    const int kx = kx_wrap > 0 ? (w.kbs + kb) % kx_wrap : w.kbs + kb;
                     mbar_expect_tx(full + 8 * s, kTmaStageBytes);
-                    tma_load_2d(a0, &tmap_x, (w.kbs + kb) * BK, w.m0, full + 8 * s);
-                    tma_load_2d(a0 + A_HALF_BYTES, &tmap_x, (w.kbs + kb) * BK, w.m0 + 128, full + 8 * s);
+                    tma_load_2d(a0, &tmap_x, kx * BK, w.m0, full + 8 * s);
+                    tma_load_2d(a0 + A_HALF_BYTES, &tmap_x, kx * BK, w.m0 + 128, full + 8 * s);
                     tma_load_2d(a0 + 2 * A_HALF_BYTES, &tmap_w, (w.kbs + kb) * BK, w.n0, full + 8 * s);
                 }
             }
@@ -910,7 +915,7 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, cons
 // slices (out = the slice buffer, out_dt = RAZER_F32)
 template <bool BF16, typename TOut>
 static razer_status launch_tma_t(const CUtensorMap &map, const CUtensorMap &wmap, const float *ts, float unbias, int M, int N, TOut *out,
-                                 int kb0, int nkb, const float *addend, cudaStream_t st, int S)
+                                 int kb0, int nkb, const float *addend, cudaStream_t st, int S, int kx_wrap)
 {
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -927,21 +932,24 @@ static razer_status launch_tma_t(const CUtensorMap &map, const CUtensorMap &wmap
     // that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
     const int inject = fault_injection_enabled() ? 1 : 0;
     if (launch_pdl(gemm_tma_kernel<BF16, TOut>, (unsigned)G, (unsigned)kTmaThreads, (size_t)kTmaSmemBytes, st, map, wmap, ts, unbias, M, N,
-                   mt, T, S, kb0, nkb, out, addend, inject) != cudaSuccess)
+                   mt, T, S, kb0, nkb, out, addend, inject, kx_wrap) != cudaSuccess)
         return RAZER_ERR_CUDA;
     return RAZER_OK;
 }
 
 template <bool BF16>
 static razer_status launch_tma(const CUtensorMap &map, const CUtensorMap &wmap, const float *ts, float unbias, int M, int N, void *out,
-                               razer_dtype out_dt, int kb0, int nkb, const float *addend, cudaStream_t st, int S)
+                               razer_dtype out_dt, int kb0, int nkb, const float *addend, cudaStream_t st, int S, int kx_wrap = 0)
 {
     if (out_dt == RAZER_F32)
-        return launch_tma_t<BF16, float>(map, wmap, ts, unbias, M, N, reinterpret_cast<float *>(out), kb0, nkb, addend, st, S);
+        return launch_tma_t<BF16, float>(map, wmap, ts, unbias, M, N, reinterpret_cast<float *>(out), kb0, nkb, addend, st, S, kx_wrap);
     if (out_dt == RAZER_F16)
-        return launch_tma_t<BF16, __half>(map, wmap, ts, unbias, M, N, reinterpret_cast<__half *>(out), kb0, nkb, addend, st, S);
-    return launch_tma_t<BF16, __nv_bfloat16>(map, wmap, ts, unbias, M, N, reinterpret_cast<__nv_bfloat16 *>(out), kb0, nkb, addend, st, S);
+        return launch_tma_t<BF16, __half>(map, wmap, ts, unbias, M, N, reinterpret_cast<__half *>(out), kb0, nkb, addend, st, S, kx_wrap);
+    return launch_tma_t<BF16, __nv_bfloat16>(map, wmap, ts, unbias, M, N, reinterpret_cast<__nv_bfloat16 *>(out), kb0, nkb, addend, st, S,
+                                             kx_wrap);
 }
+
+static razer_status reduce_splits(const float *slices, int S, int M, int N, void *Y, razer_dtype out_dt, cudaStream_t st);
 
 template <int FMT, bool BF16>
 static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, bool decoded, const uint8_t *codes, const uint8_t *scales,
@@ -962,6 +970,12 @@ static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, 
     const razer_status r = decoded ? launch_tma<BF16>(map, wmap, ts, unbias, M, N, out, odt, 0, KB, nullptr, st, S)
                                    : launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S);
     if (r != RAZER_OK || S == 1) return r;
+    return reduce_splits(slices, S, M, N, Y, out_dt, st);
+}
+
+// adds the S fp32 [M, N] slices in split order and converts to out_dt
+static razer_status reduce_splits(const float *slices, int S, int M, int N, void *Y, razer_dtype out_dt, cudaStream_t st)
+{
     if (N % 4 != 0) {
         const int64_t n1 = (int64_t)M * N;
         const int64_t g = std::max<int64_t>(1, std::min<int64_t>((n1 + 255) / 256, (int64_t)sm_count() * 8));
@@ -1194,6 +1208,96 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
                   : launch_fmt<RAZER_FMT_ACT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
     return bf ? launch_fmt<RAZER_FMT_NVFP4, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
               : launch_fmt<RAZER_FMT_NVFP4, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
+}
+
+
+// ---------------------------------------------------------------------------
+// Prefill GEMM on a format-variant weight tensor (blocks of 16-128 elements, a
+// caller-chosen special-value set, or the pages' FP16-scale words; RaZeR
+// notes, 关键设计 3 and 训练策略).  The weights are decoded once into a 16-bit
+// copy and the persistent tcgen05 GEMM multiplies it, applying ts in the
+// epilogue.
+//   * byte scales: the decoder of razer_dequant_variant, given a device 1.0
+//     in place of ts, writes round16(q*s) -- exact: q*s has at most 5 + 4
+//     significant bits and lies in [2^-10, 4256], inside fp16's normal range;
+//     in bf16 as well unless +-9.5 is in the set (refused by the caller);
+//   * FP16 scale words: q*s has up to 16 significant bits, more than a 16-bit
+//     operand holds, so the copy is two 16-bit terms of q*s*2^11 side by side
+//     ([N, 2 K]: hi, then lo; see decode_f16w_split_kernel) and the GEMM runs
+//     over 2 K with the activations' k-steps taken twice, then scales by
+//     ts * 2^-11.  Twice the MMA work of the byte-scale formats, for a
+//     product within fp32 accumulation of the exact one (bf16: hi + lo is
+//     q*s*2^11 exactly; fp16: to within 2^-25 where lo is subnormal).
+// ---------------------------------------------------------------------------
+razer_status run_dequant_variant(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t R, int64_t K, int bs,
+                                 razer_format sfmt, const VariantV &V, void *out, razer_dtype dt, cudaStream_t st);
+razer_status run_decode_f16w_split(const uint8_t *codes, const uint8_t *scales, int64_t N, int64_t K, int bs, const VariantV &V, void *out,
+                                   bool bf16, cudaStream_t st);
+
+namespace gemm {
+__global__ void unit_scale_kernel(float *p) { *p = 1.0f; }
+}  // namespace gemm
+
+size_t gemm_variant_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    // sized for the FP16-word layout (two terms, 2 K columns; the byte-scale
+    // formats use the first half): the decoded copy, the fp32 slices of the
+    // parallel K splits, one float
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    return (size_t)N * (size_t)K * 4 + gemm::split_bytes(M, N, 2 * K) + 16;
+}
+
+razer_status run_gemm_variant(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes, const uint8_t *scales, const float *ts,
+                              int block, razer_format sfmt, const VariantV &V, int64_t N, int64_t K, void *Y, razer_dtype out_dt,
+                              void *workspace, cudaStream_t st)
+{
+    using namespace gemm;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return RAZER_ERR_CUDA;
+    const bool bf = act_dt == RAZER_BF16, two = sfmt == RAZER_SCALE_F16;
+    const int64_t Kw = two ? 2 * K : K;  // columns of the weight copy
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    const size_t dec = (size_t)N * (size_t)Kw * 2, sb = split_bytes(M, N, Kw);
+    float *slices = sb ? reinterpret_cast<float *>(base + dec) : nullptr;
+    razer_status r;
+    if (two) {
+        r = run_decode_f16w_split(codes, scales, N, K, block, V, base, bf, st);
+    } else {
+        float *one = reinterpret_cast<float *>(base + dec + sb);
+        unit_scale_kernel<<<1, 1, 0, st>>>(one);
+        r = run_dequant_variant(codes, scales, one, N, K, block, sfmt, V, base, bf ? RAZER_BF16 : RAZER_F16, st);
+    }
+    if (r != RAZER_OK) return r;
+    CUtensorMap map, wmap;
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUtensorMapDataType tdt = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)BK, 128u};
+        if (enc(&map, tdt, 2, const_cast<void *>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return RAZER_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)Kw, (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)Kw * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BN};
+        if (enc(&wmap, tdt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return RAZER_ERR_CUDA;
+    }
+    // two terms: K % 64 == 0 (checked by the caller), so the hi and lo halves
+    // are whole k-steps and X's k-steps repeat after KB
+    const int m = (int)M, n = (int)N, KB = (int)((K + BK - 1) / BK), KBw = two ? 2 * KB : KB;
+    const int S = gemm_splits(M, N, Kw);
+    const float unbias = two ? 1.0f / 2048.0f : 1.0f;  // a power of two: exact
+    void *out = S > 1 ? static_cast<void *>(slices) : Y;
+    const razer_dtype odt = S > 1 ? RAZER_F32 : out_dt;
+    r = bf ? launch_tma<true>(map, wmap, ts, unbias, m, n, out, odt, 0, KBw, nullptr, st, S, two ? KB : 0)
+           : launch_tma<false>(map, wmap, ts, unbias, m, n, out, odt, 0, KBw, nullptr, st, S, two ? KB : 0);
+    if (r != RAZER_OK || S == 1) return r;
+    return reduce_splits(slices, S, m, n, Y, out_dt, st);
 }
 
 }  // namespace razer

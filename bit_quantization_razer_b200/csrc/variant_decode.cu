@@ -429,4 +429,82 @@ razer_status run_dequant_variant(const uint8_t *codes, const uint8_t *scales, co
     return last_launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Two-term 16-bit copy of a weight tensor with FP16 scale words, for the
+// prefill GEMM: v = q*s*2^11 (exact in binary32: at most 5 + 11 significant
+// bits; in [2^-14, 38912] for every nonzero q and scale word, inside fp16's
+// normal range), hi = RN16(v), lo = RN16(v - hi) (v - hi is exact in binary32
+// and at most half a 16-bit ulp of hi).  Row n of the [N, 2 K] output holds hi
+// in columns [0, K) and lo in [K, 2 K), so a GEMM over 2 K columns against
+// [X | X] sums x * (hi + lo).  bf16: hi keeps 8 of v's at most 16 significant
+// bits and lo the other at most 8, so hi + lo == v exactly.  fp16: exact
+// unless lo falls below fp16's normal range (v < 2^-3), and then off by at
+// most 2^-25 -- where one fp16 term would be off by up to 2^-11 relative.
+// One thread per 16-element sub-block.
+// ---------------------------------------------------------------------------
+template <bool BF>
+__global__ void __launch_bounds__(256) decode_f16w_split_kernel(const uint2 *__restrict__ codes, const uint8_t *__restrict__ scales,
+                                                                int64_t nsub, int64_t sub_per_row, int bs_shift, VariantV V,
+                                                                uint4 *__restrict__ out)
+{
+    pdl_wait();
+    const int64_t per_row = sub_per_row >> bs_shift;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nsub; b += stride) {
+        const int64_t r = b / sub_per_row, u = b - r * sub_per_row;
+        const unsigned sw = reinterpret_cast<const unsigned short *>(scales)[r * per_row + (u >> bs_shift)];
+        const float s = __half2float(__ushort_as_half((unsigned short)(sw & 0x3FFFu)));
+        const unsigned meta = sw >> 14;
+        const float v = meta == 0 ? V.v[0] : (meta == 1 ? V.v[1] : (meta == 2 ? V.v[2] : V.v[3]));
+        const uint2 c = codes[b];
+        unsigned hw[8], lw[8];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+            float hv[2], lv[2];
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+                const unsigned code = ((j + e < 8 ? c.x : c.y) >> (4 * ((j + e) & 7))) & 15u;
+                float q;
+                if (code == 8u) q = V.nv > 0 ? v : 0.0f;
+                else q = (code & 8u) ? -fp4_mag(code & 7u) : fp4_mag(code & 7u);
+                const float w = __fmul_rn(__fmul_rn(q, s), 2048.0f);
+                const float h = BF ? __bfloat162float(__float2bfloat16_rn(w)) : __half2float(__float2half_rn(w));
+                hv[e] = w;
+                lv[e] = __fsub_rn(w, h);
+            }
+            if constexpr (BF) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(hv[0], hv[1]), l2 = __floats2bfloat162_rn(lv[0], lv[1]);
+                hw[j / 2] = *reinterpret_cast<const unsigned *>(&h2);
+                lw[j / 2] = *reinterpret_cast<const unsigned *>(&l2);
+            } else {
+                const __half2 h2 = __floats2half2_rn(hv[0], hv[1]), l2 = __floats2half2_rn(lv[0], lv[1]);
+                hw[j / 2] = *reinterpret_cast<const unsigned *>(&h2);
+                lw[j / 2] = *reinterpret_cast<const unsigned *>(&l2);
+            }
+        }
+        // sub-block u of row r: 16 halves at column 16 u of the hi and lo halves
+        uint4 *oh = out + r * (sub_per_row * 4) + 2 * u;
+        uint4 *ol = oh + sub_per_row * 2;
+        oh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        oh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+        ol[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        ol[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    }
+}
+
+razer_status run_decode_f16w_split(const uint8_t *codes, const uint8_t *scales, int64_t N, int64_t K, int bs, const VariantV &V, void *out,
+                                   bool bf16, cudaStream_t st)
+{
+    const int64_t nsub = N * K / 16;
+    if (nsub == 0) return RAZER_OK;
+    int64_t g = (nsub + 255) / 256;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (g > cap) g = cap;
+    if (launch_pdl(bf16 ? decode_f16w_split_kernel<true> : decode_f16w_split_kernel<false>, (unsigned)g, 256u, 0, st,
+                   reinterpret_cast<const uint2 *>(codes), scales, nsub, K / 16, bs_shift_of(bs), V, reinterpret_cast<uint4 *>(out)) !=
+        cudaSuccess)
+        return RAZER_ERR_CUDA;
+    return RAZER_OK;
+}
+
 }  // namespace razer

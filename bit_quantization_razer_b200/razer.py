@@ -24,7 +24,7 @@ STATUS_NAMES = {
 }
 RAZER_F16, RAZER_BF16, RAZER_F32 = 0, 1, 2
 RAZER_FMT_WEIGHT, RAZER_FMT_ACT, RAZER_FMT_NVFP4, RAZER_FMT_FOUR_OVER_SIX, RAZER_SCALE_F16 = 0, 1, 2, 3, 4
-RAZER_OP_GEMV, RAZER_OP_GEMM, RAZER_OP_GEMM_W4A4 = 0, 1, 2
+RAZER_OP_GEMV, RAZER_OP_GEMM, RAZER_OP_GEMM_W4A4, RAZER_OP_GEMM_VARIANT = 0, 1, 2, 3
 FORMATS = {"weight": RAZER_FMT_WEIGHT, "act": RAZER_FMT_ACT, "nvfp4": RAZER_FMT_NVFP4, "four_over_six": RAZER_FMT_FOUR_OVER_SIX,
            "f16_scale": RAZER_SCALE_F16}
 _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZER_F32}
@@ -32,7 +32,7 @@ _DT = {torch.float16: RAZER_F16, torch.bfloat16: RAZER_BF16, torch.float32: RAZE
 EXPORTED = (
     "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
     "razer_gemv_batch", "razer_gemv_batch_workspace_size", "razer_gemm_w4a4", "razer_gemm_w4a4_online", "razer_quant_error",
-    "razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant",
+    "razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant", "razer_gemm_variant",
     "razer_workspace_size", "razer_get_device_status", "razer_status_string", "razer_version",
     "razer_gemv_noalloc", "razer_gemv_noalloc_max_scratch", "razer_debug_set_fault_injection", "razer_set_quantize_path",
 )
@@ -77,6 +77,8 @@ def load() -> ctypes.CDLL:
     L.razer_dequant_variant.argtypes = [vp, vp, vp, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_float), i32, vp, i32, vp]
     L.razer_gemv_variant.argtypes = [vp, i32, i64, vp, vp, vp, i32, i32, ctypes.POINTER(ctypes.c_float), i32, i64, i64, vp, i32, vp,
                                      sz, vp]
+    L.razer_gemm_variant.argtypes = [vp, i32, i64, vp, vp, vp, i32, i32, ctypes.POINTER(ctypes.c_float), i32, i64, i64, vp, i32, vp,
+                                     sz, vp]
     L.razer_quant_error.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp]
     L.razer_gemv_batch_workspace_size.argtypes = [i32, ctypes.POINTER(GemvProblem)]
     L.razer_gemv_batch_workspace_size.restype = sz
@@ -94,7 +96,8 @@ def load() -> ctypes.CDLL:
     L.razer_debug_set_fault_injection.restype = ctypes.c_int
     L.razer_set_quantize_path.argtypes = [i32]
     L.razer_set_quantize_path.restype = ctypes.c_int
-    for fn in ("razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant", "razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
+    for fn in ("razer_quantize_variant", "razer_quant_error_variant", "razer_dequant_variant", "razer_gemv_variant", "razer_gemm_variant",
+               "razer_gemm_w4a4_online", "razer_quant_error", "razer_gemm_w4a4", "razer_gemv_batch", "razer_quantize_weights", "razer_quantize_weights_batch", "razer_quantize_acts", "razer_dequant", "razer_gemv", "razer_gemm",
                "razer_get_device_status", "razer_version"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -279,6 +282,19 @@ def razer_gemv_variant(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tenso
     st = load().razer_gemv_variant(_p(x), _DT.get(x.dtype, -1), B, _p(codes), _p(scales), _p(ts), block, _fmt(scale_fmt),
                                    _varr(V), len(V), N, K, _p(out), _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
     _check("razer_gemv_variant", st)
+    return out
+
+
+def razer_gemm_variant(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, ts: torch.Tensor, block: int, scale_fmt, V,
+                       out_dtype=torch.bfloat16, *, out=None, workspace=None, stream=None):
+    """Y [M, N] = ts * X [M, K] . deq(W [N, K])^T for a razer_quantize_variant weight tensor (tcgen05 GEMM)."""
+    M, K = X.shape
+    N = codes.shape[0]
+    out = torch.empty((M, N), dtype=out_dtype, device=X.device) if out is None else out
+    workspace, wsb = _workspace(RAZER_OP_GEMM_VARIANT, M, N, K, X.device, workspace)
+    st = load().razer_gemm_variant(_p(X), _DT.get(X.dtype, -1), M, _p(codes), _p(scales), _p(ts), block, _fmt(scale_fmt),
+                                   _varr(V), len(V), N, K, _p(out), _DT.get(out.dtype, -1), _p(workspace), wsb, _stream(stream))
+    _check("razer_gemm_variant", st)
     return out
 
 

@@ -92,7 +92,7 @@ typedef enum {
     RAZER_SCALE_F16 = 4
 } razer_format;
 
-typedef enum { RAZER_OP_GEMV = 0, RAZER_OP_GEMM = 1, RAZER_OP_GEMM_W4A4 = 2 } razer_op;
+typedef enum { RAZER_OP_GEMV = 0, RAZER_OP_GEMM = 1, RAZER_OP_GEMM_W4A4 = 2, RAZER_OP_GEMM_VARIANT = 3 } razer_op;
 
 /*
  * razer_quantize_weights -- offline weight quantizer (RaZeR notes, 关键设计
@@ -378,6 +378,32 @@ razer_status razer_gemv_variant(const void *x, razer_dtype act_dt, int64_t B, co
                                 razer_dtype out_dt, void *workspace, size_t ws_bytes, razer_stream_t stream);
 
 /*
+ * razer_gemm_variant -- prefill GEMM on a format-variant weight tensor (RaZeR
+ * notes, 关键设计 3: the pages' W4A16 kernels on group-128 FP16-scale
+ * weights; 训练策略: per-model special values):
+ *   Y[m, n] = ts * sum_k X[m, k] * (q*s)[n, k],   fp32 accumulation,
+ * on the tcgen05 tensor cores.  Arguments as razer_gemm, plus block /
+ * scale_fmt / special_values / n_special as razer_quantize_variant.  codes
+ * 8-byte aligned; FP16 scale words 2-byte aligned.
+ *   workspace  at least razer_workspace_size(RAZER_OP_GEMM_VARIANT, M, N, K)
+ *              bytes, 16-byte aligned (a decoded [N, K] 16-bit copy of q*s,
+ *              the partial sums of long or split K, one float); contents
+ *              ignored.  M = 0, N = 0 or K = 0 need none.
+ * The weights are decoded once to the activations' 16-bit type.  Byte-scale
+ * formats: q*s is exact in fp16, and in bf16 unless +-9.5 is in the set
+ * (bf16 activations with +-9.5 give RAZER_ERR_UNSUPPORTED).  FP16 scale
+ * words: q*s has up to 16 significant bits, so the copy holds two 16-bit
+ * terms hi + lo of q*s*2^11 (exact in bf16; in fp16 to within 2^-25 where lo
+ * is subnormal) and the product runs over 2 K (twice the tensor-core work);
+ * K % 64 == 0 (else RAZER_ERR_UNSUPPORTED).  Any M >= 0, N, and K a multiple
+ * of block.
+ */
+razer_status razer_gemm_variant(const void *X, razer_dtype act_dt, int64_t M, const uint8_t *codes,
+                                const uint8_t *scales, const float *ts, int block, razer_format scale_fmt,
+                                const float *special_values, int n_special, int64_t N, int64_t K, void *Y,
+                                razer_dtype out_dt, void *workspace, size_t ws_bytes, razer_stream_t stream);
+
+/*
  * razer_gemv_noalloc -- razer_gemv for callers that cannot allocate device
  * memory (the paper has no counterpart: this is a deployment convenience).
  * Some callers cannot call cudaMalloc at all, e.g. a runtime that gives every
@@ -407,8 +433,10 @@ razer_status razer_gemv_noalloc(const void *x, razer_dtype act_dt, int64_t B, co
 /* Size in bytes of the fixed scratch array used by razer_gemv_noalloc. */
 size_t razer_gemv_noalloc_max_scratch(void);
 
-/* Bytes of workspace razer_gemv / razer_gemm need for these sizes (0 when
- * none); M_or_B is B for RAZER_OP_GEMV and M for RAZER_OP_GEMM. */
+/* Bytes of workspace razer_gemv (RAZER_OP_GEMV; M_or_B = B), razer_gemm
+ * (RAZER_OP_GEMM), razer_gemm_w4a4 / razer_gemm_w4a4_online
+ * (RAZER_OP_GEMM_W4A4) and razer_gemm_variant (RAZER_OP_GEMM_VARIANT) need
+ * for these sizes (M_or_B = M for the GEMMs); 0 when none. */
 size_t razer_workspace_size(razer_op op, int64_t M_or_B, int64_t N, int64_t K);
 
 /*

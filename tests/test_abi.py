@@ -221,6 +221,12 @@ def test_workspace_size_host_logic(lib):
         assert razer.razer_workspace_size(G, M, N, K) == slices(M, N, K), (M, N, K)
     assert razer.razer_workspace_size(G, 1024, 4096, 16384) == 4096 * 16384 * 2 + slices(1024, 4096, 16384)
     assert razer.razer_workspace_size(G, 2048, 8192, 28672) == 8192 * 28672 * 2 + 2 * 2048 * 8192 * 4
+    # variant GEMM: the decoded copy sized for two 16-bit terms (FP16 scale
+    # words), the split slices over 2 K, one float
+    GV = razer.RAZER_OP_GEMM_VARIANT
+    assert razer.razer_workspace_size(GV, 4096, 4096, 4096) == 4096 * 4096 * 4 + slices(4096, 4096, 8192) + 16
+    assert razer.razer_workspace_size(GV, 64, 200, 384) == 200 * 384 * 4 + slices(64, 200, 768) + 16
+    assert razer.razer_workspace_size(GV, 0, 200, 384) == 0 and razer.razer_workspace_size(GV, 8, 200, 0) == 0
     # W4A4: both decoded operands, the K-chunk partials, 16 bytes for ts_a * ts_w
     W4 = razer.RAZER_OP_GEMM_W4A4
     assert razer.razer_workspace_size(W4, 100, 64, 128) == 100 * 128 * 2 + 64 * 128 * 2 + 16

@@ -150,3 +150,85 @@ def test_gemv_variant_empty_and_zero_k():
     y0 = R.razer_gemv_variant(x0, c0, s0, _ts(1.0), 128, "f16_scale", [5.0, -5.0], out=torch.full((2, 8), 7.0, device=DEV))
     torch.cuda.synchronize()
     assert not y0.any()
+
+
+# --- prefill GEMM on variant weights -----------------------------------------
+@pytest.mark.parametrize("M", [64, 300])
+@pytest.mark.parametrize("block,fmt,V", VARIANTS, ids=IDS)
+def test_gemm_variant_quantized(orc, block, fmt, V, M):
+    # oracle-quantized weights (zero and tiny rows), ragged N and M tiles
+    N, K = 200, 384
+    codes, scales, ts = _quantized(orc, N, K, block, fmt, V, seed=92)
+    X = workloads.vectors(M, K, seed=110)
+    Y = R.razer_gemm_variant(X.to(DEV), *_dev(codes, scales), _ts(ts), block, fmt, V, torch.float32)
+    r = orc.gemv_generic(X.numpy(), codes, scales, ts, block, FMT_ID[fmt], V)
+    assert rel_err(Y.cpu().numpy(), r) <= REL_TOL
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("block,fmt,V", [VARIANTS[0], VARIANTS[2], VARIANTS[3], VARIANTS[5], VARIANTS[6], VARIANTS[7]],
+                         ids=[IDS[0], IDS[2], IDS[3], IDS[5], IDS[6], IDS[7]])
+def test_gemm_variant_bf16_random_packed(orc, block, fmt, V, out_dtype):
+    # bf16 activations (the weight copy is bf16: exact without +-9.5; FP16
+    # scale words as two exact bf16 terms), every code under every scale
+    # magnitude, K spanning several k-steps
+    M, N, K = 320, 96, 1024
+    codes, scales = workloads.random_packed_variant(N, K, block, fmt, len(V), seed=111)
+    X = workloads.vectors(M, K, seed=112, dtype=torch.bfloat16)
+    Y = R.razer_gemm_variant(X.to(DEV), *_dev(codes, scales), _ts(0.0193), block, fmt, V, out_dtype)
+    r = orc.gemv_generic(oracle_in(X), codes.numpy(), scales.numpy(), 0.0193, block, FMT_ID[fmt], V)
+    assert_close_typed(Y, r)
+
+
+def test_gemm_variant_refusals():
+    codes, scales = workloads.random_packed_variant(16, 256, 16, "weight", 4, seed=113)
+    X = workloads.vectors(8, 256, seed=114, dtype=torch.bfloat16)
+    with pytest.raises(R.RazerError):  # bf16 cannot hold 9.5 x every scale
+        R.razer_gemm_variant(X.to(DEV), *_dev(codes, scales), _ts(1.0), 16, "weight", [5.0, -5.0, 9.5, -9.5])
+    c2, s2 = workloads.random_packed_variant(16, 96, 32, "f16_scale", 4, seed=115)
+    with pytest.raises(R.RazerError):  # FP16 scale words need whole 64-element k-steps
+        R.razer_gemm_variant(workloads.vectors(8, 96).to(DEV), *_dev(c2, s2), _ts(1.0), 32, "f16_scale", [5.0, -5.0, 8.0, -8.0])
+    with pytest.raises(R.RazerError):  # K not a multiple of the block
+        R.razer_gemm_variant(workloads.vectors(8, 96).to(DEV), *_dev(c2, s2), _ts(1.0), 64, "f16_scale", [5.0])
+
+
+@pytest.mark.parametrize("M", [100, 1100])
+def test_gemm_variant_hot_path_format_equals_razer_gemm(M):
+    # block 16, E3M3 scales, V = +-5/+-8 is the hot-path weight format: the
+    # variant GEMM's exact q*s copy and razer_gemm's q*s*2^-8 copy differ by a
+    # power of two that the epilogue undoes exactly, so the outputs are equal
+    N, K = 272, 640
+    codes, scales = workloads.random_packed(N, K, "weight", seed=116, max_scale_code=40)
+    X = workloads.vectors(M, K, seed=117, dtype=torch.bfloat16).to(DEV)
+    c, s = _dev(codes, scales)
+    a = R.razer_gemm_variant(X, c, s, _ts(0.037), 16, "weight", [5.0, -5.0, 8.0, -8.0], torch.float32)
+    b = R.razer_gemm(X, c, s, _ts(0.037), "weight", torch.float32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(a.cpu().numpy(), b.cpu().numpy())
+
+
+def test_gemm_variant_pages_format_sampled(orc):
+    # the pages' kernel format (blocks of 128, FP16 scale words, +-5/+-8) on a
+    # prefill shape, fp16 activations; sampled rows against the oracle
+    M, N, K = 2048, 4096, 4096
+    codes, scales = workloads.random_packed_variant(N, K, 128, "f16_scale", 4, seed=118)
+    X = workloads.vectors(M, K, seed=119)
+    Y = R.razer_gemm_variant(X.to(DEV), *_dev(codes, scales), _ts(1.0), 128, "f16_scale", [5.0, -5.0, 8.0, -8.0],
+                             torch.float32).cpu().numpy()
+    rows = np.sort(np.random.default_rng(120).choice(M, 24, replace=False))
+    r = orc.gemv_generic(X.numpy()[rows], codes.numpy(), scales.numpy(), 1.0, 128, FMT_ID["f16_scale"], [5.0, -5.0, 8.0, -8.0])
+    assert rel_err(Y[rows], r) <= REL_TOL
+
+
+def test_gemm_variant_empty_shapes():
+    c, s = workloads.random_packed_variant(8, 128, 128, "f16_scale", 2, seed=121)
+    X0 = torch.zeros((0, 128), device=DEV).half()
+    Y0 = R.razer_gemm_variant(X0, *_dev(c, s), _ts(1.0), 128, "f16_scale", [5.0, -5.0], torch.float32)
+    assert Y0.shape == (0, 8)
+    c0 = torch.zeros((8, 0), dtype=torch.uint8, device=DEV)
+    s0 = torch.zeros((8, 0), dtype=torch.uint8, device=DEV)
+    X = torch.zeros((3, 0), device=DEV).half()
+    Y = R.razer_gemm_variant(X, c0, s0, _ts(1.0), 128, "f16_scale", [5.0, -5.0], torch.float32,
+                             out=torch.full((3, 8), 7.0, device=DEV))
+    torch.cuda.synchronize()
+    assert not Y.any()
