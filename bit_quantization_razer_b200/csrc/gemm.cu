@@ -460,21 +460,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 constexpr int kEpiWarps = 8;
 constexpr int kTmaThreads = 32 * (2 + kEpiWarps);
-constexpr uint32_t kTmaStageBytes = 2 * A_HALF_BYTES + (uint32_t)BN * BK * 2;  // X 256 x 64 + W 256 x 64
+// the tile is 256 x TBN with TBN = 256 or 224: the host takes the width whose
+// rounds of tiles over the SMs cost least (4096 x 14336: 896 tiles of 256 are
+// 7 rounds, the last with 8 tiles; 1024 tiles of 224 are 7 full rounds)
+__host__ __device__ constexpr uint32_t tma_stage_bytes(int tbn) { return 2 * A_HALF_BYTES + (uint32_t)tbn * BK * 2; }  // X 256 x 64 + W tbn x 64
 constexpr uint32_t kEpiStageBytes = 32 * 128;                                  // one warp's 32 x 32 fp32 chunk
-constexpr uint32_t kTmaSmemBytes = STAGES * kTmaStageBytes + kEpiWarps * kEpiStageBytes + BAR_BYTES + 1024;
-static_assert(kTmaSmemBytes <= 232448, "shared memory of the persistent GEMM");
+__host__ __device__ constexpr uint32_t tma_smem_bytes(int tbn) { return STAGES * tma_stage_bytes(tbn) + kEpiWarps * kEpiStageBytes + BAR_BYTES + 1024; }
+static_assert(tma_smem_bytes(256) <= 232448, "shared memory of the persistent GEMM");
 
 struct TmaUnit {
     int m0, n0, kbs, nk, z;
 };
-__device__ __forceinline__ TmaUnit tma_unit(int u, int mt, int T, int S, int kb0, int nkb)
+__device__ __forceinline__ TmaUnit tma_unit(int u, int mt, int T, int S, int kb0, int nkb, int tbn)
 {
     TmaUnit w;
     w.z = u / T;
     const int t = u - w.z * T;
     w.m0 = (t % mt) * 256;
-    w.n0 = (t / mt) * BN;
+    w.n0 = (t / mt) * tbn;
     w.kbs = kb0 + (int)((int64_t)w.z * nkb / S);
     w.nk = kb0 + (int)((int64_t)(w.z + 1) * nkb / S) - w.kbs;
     return w;
@@ -529,12 +532,13 @@ __device__ __forceinline__ void epi_write(const uint8_t *stage, int lane, int m,
     }
 }
 
-template <bool BF16, typename TOut>
+template <bool BF16, typename TOut, int TBN>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     gemm_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w, const float *__restrict__ ts_p,
                     float unbias, int M, int N, int mt, int T, int S, int kb0, int nkb, TOut *Y, const float *addend, int inject_stall,
                     int kx_wrap)
 {
+    constexpr uint32_t kTmaStageBytes = tma_stage_bytes(TBN);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *epi = smem + STAGES * kTmaStageBytes;
@@ -576,7 +580,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             uint32_t g = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < U && ok; u += G) {
-                const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb);
+                const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb, TBN);
                 for (int kb = 0; kb < w.nk; kb++, g++) {
                     const uint32_t s = g % STAGES, ph = (g / STAGES) & 1u;
                     if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort_flag)) {
@@ -608,11 +612,11 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            const uint32_t idesc = idesc_f16(BF16, 128, BN);
+            const uint32_t idesc = idesc_f16(BF16, 128, TBN);
             uint32_t g = 0, ti = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < U && ok; u += G, ti++) {
-                const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb);
+                const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb, TBN);
                 // the epilogue has drained the previous unit's accumulator
                 if (!mbar_wait(acc_empty, (ti & 1u) ^ 1u, abort_flag)) {
                     ok = false;
@@ -633,7 +637,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                         const uint64_t bd = smem_desc_k128(b0 + 32 * k);
                         const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
                         umma_f16(tmem, smem_desc_k128(a0 + 32 * k), bd, idesc, acc);
-                        umma_f16(tmem + BN, smem_desc_k128(a0 + A_HALF_BYTES + 32 * k), bd, idesc, acc);
+                        umma_f16(tmem + TBN, smem_desc_k128(a0 + A_HALF_BYTES + 32 * k), bd, idesc, acc);
                     }
                     umma_commit(empty + 8 * s);
                 }
@@ -647,23 +651,24 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         }
     } else {
         // ---------------- epilogue ----------------
-        const int q = warp & 3;                          // TMEM lane quarter this warp may access
-        const int cbeg = ((warp - 2) >> 2) * (BN / 2);   // the two warps of a quarter split the columns
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        // the two warps of a quarter split each half's columns: [0, 128) and [128, TBN)
+        const int wb = (warp - 2) >> 2, cbeg = wb * 128, nch = (wb ? TBN - 128 : 128) / 32;
         uint8_t *stage = epi + (warp - 2) * kEpiStageBytes;
         const float scale = __fmul_rn(*ts_p, unbias);
         TOut *Yz = Y;
         uint32_t ti = 0;
         for (int u = blockIdx.x; u < U; u += G, ti++) {
-            const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb);
+            const TmaUnit w = tma_unit(u, mt, T, S, kb0, nkb, TBN);
             if (!mbar_wait_warp(acc_full, ti & 1u, abort_flag)) break;
             tc_fence_after();
             Yz = Y + (S > 1 ? (size_t)w.z * (size_t)M * (size_t)N : 0);
 #pragma unroll 1
-            for (int c = 0; c < 2 * (BN / 2) / 32; c++) {
-                const int half = c / ((BN / 2) / 32), col = cbeg + 32 * (c % ((BN / 2) / 32));
+            for (int c = 0; c < 2 * nch; c++) {
+                const int half = c / nch, col = cbeg + 32 * (c % nch);
                 float v[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * BN + col), v);
-                if (c == 2 * (BN / 2) / 32 - 1) {
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * TBN + col), v);
+                if (c == 2 * nch - 1) {
                     // this warp has read the whole accumulator: hand it back
                     tc_fence_before();
                     __syncwarp();
@@ -911,9 +916,26 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, cons
     return last_launch_status();
 }
 
+// tile width of the persistent GEMM: the candidate whose rounds of units over
+// the SMs (each round as long as one tile of that width) cost least
+static int choose_tbn(int64_t M, int64_t N, int S)
+{
+    const int64_t sm = sm_count(), mt = (M + 255) / 256;
+    int best = 256;
+    int64_t best_cost = 0;
+    for (int c : {256, 224}) {
+        const int64_t units = mt * ((N + c - 1) / c) * S, cost = (units + sm - 1) / sm * c;
+        if (c == 256 || cost < best_cost) {
+            best = c;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
 // the persistent GEMM on two decoded 16-bit operands; S > 1 writes fp32
-// slices (out = the slice buffer, out_dt = RAZER_F32)
-template <bool BF16, typename TOut>
+// slices (out = the slice buffer, out_dt = RAZER_F32); wmap's box is tbn rows
+template <bool BF16, typename TOut, int TBN>
 static razer_status launch_tma_t(const CUtensorMap &map, const CUtensorMap &wmap, const float *ts, float unbias, int M, int N, TOut *out,
                                  int kb0, int nkb, const float *addend, cudaStream_t st, int S, int kx_wrap)
 {
@@ -921,40 +943,49 @@ static razer_status launch_tma_t(const CUtensorMap &map, const CUtensorMap &wmap
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(gemm_tma_kernel<BF16, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTmaSmemBytes) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_tma_kernel<BF16, TOut, TBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tma_smem_bytes(TBN)) != cudaSuccess)
             return RAZER_ERR_CUDA;
         attr_set[dev] = true;
     }
-    const int mt = (M + 255) / 256, nt = (N + BN - 1) / BN, T = mt * nt;
+    const int mt = (M + 255) / 256, nt = (N + TBN - 1) / TBN, T = mt * nt;
     const int G = (int)std::min<int64_t>((int64_t)T * S, sm_count());
     // fault injection (tests only): CTA 0 leaves its first stage unfilled so
     // that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
     const int inject = fault_injection_enabled() ? 1 : 0;
-    if (launch_pdl(gemm_tma_kernel<BF16, TOut>, (unsigned)G, (unsigned)kTmaThreads, (size_t)kTmaSmemBytes, st, map, wmap, ts, unbias, M, N,
-                   mt, T, S, kb0, nkb, out, addend, inject, kx_wrap) != cudaSuccess)
+    if (launch_pdl(gemm_tma_kernel<BF16, TOut, TBN>, (unsigned)G, (unsigned)kTmaThreads, (size_t)tma_smem_bytes(TBN), st, map, wmap, ts,
+                   unbias, M, N, mt, T, S, kb0, nkb, out, addend, inject, kx_wrap) != cudaSuccess)
         return RAZER_ERR_CUDA;
     return RAZER_OK;
 }
 
+template <bool BF16, typename TOut>
+static razer_status launch_tma_w(const CUtensorMap &map, const CUtensorMap &wmap, int tbn, const float *ts, float unbias, int M, int N,
+                                 TOut *out, int kb0, int nkb, const float *addend, cudaStream_t st, int S, int kx_wrap)
+{
+    if (tbn == 224) return launch_tma_t<BF16, TOut, 224>(map, wmap, ts, unbias, M, N, out, kb0, nkb, addend, st, S, kx_wrap);
+    return launch_tma_t<BF16, TOut, 256>(map, wmap, ts, unbias, M, N, out, kb0, nkb, addend, st, S, kx_wrap);
+}
+
 template <bool BF16>
-static razer_status launch_tma(const CUtensorMap &map, const CUtensorMap &wmap, const float *ts, float unbias, int M, int N, void *out,
-                               razer_dtype out_dt, int kb0, int nkb, const float *addend, cudaStream_t st, int S, int kx_wrap = 0)
+static razer_status launch_tma(const CUtensorMap &map, const CUtensorMap &wmap, int tbn, const float *ts, float unbias, int M, int N,
+                               void *out, razer_dtype out_dt, int kb0, int nkb, const float *addend, cudaStream_t st, int S,
+                               int kx_wrap = 0)
 {
     if (out_dt == RAZER_F32)
-        return launch_tma_t<BF16, float>(map, wmap, ts, unbias, M, N, reinterpret_cast<float *>(out), kb0, nkb, addend, st, S, kx_wrap);
+        return launch_tma_w<BF16, float>(map, wmap, tbn, ts, unbias, M, N, reinterpret_cast<float *>(out), kb0, nkb, addend, st, S, kx_wrap);
     if (out_dt == RAZER_F16)
-        return launch_tma_t<BF16, __half>(map, wmap, ts, unbias, M, N, reinterpret_cast<__half *>(out), kb0, nkb, addend, st, S, kx_wrap);
-    return launch_tma_t<BF16, __nv_bfloat16>(map, wmap, ts, unbias, M, N, reinterpret_cast<__nv_bfloat16 *>(out), kb0, nkb, addend, st, S,
-                                             kx_wrap);
+        return launch_tma_w<BF16, __half>(map, wmap, tbn, ts, unbias, M, N, reinterpret_cast<__half *>(out), kb0, nkb, addend, st, S, kx_wrap);
+    return launch_tma_w<BF16, __nv_bfloat16>(map, wmap, tbn, ts, unbias, M, N, reinterpret_cast<__nv_bfloat16 *>(out), kb0, nkb, addend, st,
+                                             S, kx_wrap);
 }
 
 static razer_status reduce_splits(const float *slices, int S, int M, int N, void *Y, razer_dtype out_dt, cudaStream_t st);
 
 template <int FMT, bool BF16>
-static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, bool decoded, const uint8_t *codes, const uint8_t *scales,
-                               const float *ts, float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, void *wdec,
-                               float *slices, cudaStream_t st)
+static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, int tbn, bool decoded, const uint8_t *codes,
+                               const uint8_t *scales, const float *ts, float unbias, int M, int N, int K, void *Y, razer_dtype out_dt,
+                               void *wdec, float *slices, cudaStream_t st)
 {
     if (decoded) {
         const int64_t nblk = (int64_t)N * K / 16;
@@ -967,7 +998,7 @@ static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, 
     const int S = gemm_splits(M, N, K);
     void *out = S > 1 ? static_cast<void *>(slices) : Y;
     const razer_dtype odt = S > 1 ? RAZER_F32 : out_dt;
-    const razer_status r = decoded ? launch_tma<BF16>(map, wmap, ts, unbias, M, N, out, odt, 0, KB, nullptr, st, S)
+    const razer_status r = decoded ? launch_tma<BF16>(map, wmap, tbn, ts, unbias, M, N, out, odt, 0, KB, nullptr, st, S)
                                    : launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S);
     if (r != RAZER_OK || S == 1) return r;
     return reduce_splits(slices, S, M, N, Y, out_dt, st);
@@ -1053,10 +1084,11 @@ static razer_status w4a4_product(const float *ts_a, razer_format afmt, int64_t M
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return RAZER_ERR_CUDA;
     }
+    const int tbn = choose_tbn(M, N, 1);
     {
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
         const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BN};
+        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)tbn};
         if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ww, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return RAZER_ERR_CUDA;
@@ -1066,7 +1098,7 @@ static razer_status w4a4_product(const float *ts_a, razer_format afmt, int64_t M
     for (int c = 0; c < nc; c++) {
         const int kb0 = (int)((int64_t)c * KB / nc), kb1 = (int)((int64_t)(c + 1) * KB / nc);
         const bool last = c == nc - 1;
-        r = launch_tma<false>(amap, wmap, tsp, unbias, m, n, last ? Y : partial, last ? out_dt : RAZER_F32, kb0, kb1 - kb0,
+        r = launch_tma<false>(amap, wmap, tbn, tsp, unbias, m, n, last ? Y : partial, last ? out_dt : RAZER_F32, kb0, kb1 - kb0,
                               c > 0 ? partial : nullptr, st, 1);
         if (r != RAZER_OK) return r;
     }
@@ -1189,10 +1221,11 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
     const bool decoded = decoded_bytes(M, N, K) > 0;
     float *slices = split_bytes(M, N, K) ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + decoded_bytes(M, N, K)) : nullptr;
     CUtensorMap wmap = map;  // unused by the fused kernel
+    const int tbn = choose_tbn(M, N, gemm_splits(M, N, K));
     if (decoded) {
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
         const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BN};
+        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)tbn};
         const cuuint32_t estr[2] = {1u, 1u};
         if (enc(&wmap, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, workspace, dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1201,13 +1234,13 @@ razer_status run_gemm(const void *X, razer_dtype act_dt, int64_t M, const uint8_
     }
     const int m = (int)M, n = (int)N, k = (int)K;
     if (wfmt == RAZER_FMT_WEIGHT)
-        return bf ? launch_fmt<RAZER_FMT_WEIGHT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
-                  : launch_fmt<RAZER_FMT_WEIGHT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
+        return bf ? launch_fmt<RAZER_FMT_WEIGHT, true>(map, wmap, tbn, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
+                  : launch_fmt<RAZER_FMT_WEIGHT, false>(map, wmap, tbn, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
     if (wfmt == RAZER_FMT_ACT)
-        return bf ? launch_fmt<RAZER_FMT_ACT, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
-                  : launch_fmt<RAZER_FMT_ACT, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
-    return bf ? launch_fmt<RAZER_FMT_NVFP4, true>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
-              : launch_fmt<RAZER_FMT_NVFP4, false>(map, wmap, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
+        return bf ? launch_fmt<RAZER_FMT_ACT, true>(map, wmap, tbn, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
+                  : launch_fmt<RAZER_FMT_ACT, false>(map, wmap, tbn, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
+    return bf ? launch_fmt<RAZER_FMT_NVFP4, true>(map, wmap, tbn, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st)
+              : launch_fmt<RAZER_FMT_NVFP4, false>(map, wmap, tbn, decoded, codes, scales, ts, unbias, m, n, k, Y, out_dt, workspace, slices, st);
 }
 
 
@@ -1279,10 +1312,11 @@ razer_status run_gemm_variant(const void *X, razer_dtype act_dt, int64_t M, cons
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return RAZER_ERR_CUDA;
     }
+    const int tbn = choose_tbn(M, N, gemm_splits(M, N, Kw));
     {
         const cuuint64_t dims[2] = {(cuuint64_t)Kw, (cuuint64_t)N};
         const cuuint64_t strides[1] = {(cuuint64_t)Kw * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BN};
+        const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)tbn};
         if (enc(&wmap, tdt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return RAZER_ERR_CUDA;
@@ -1294,8 +1328,8 @@ razer_status run_gemm_variant(const void *X, razer_dtype act_dt, int64_t M, cons
     const float unbias = two ? 1.0f / 2048.0f : 1.0f;  // a power of two: exact
     void *out = S > 1 ? static_cast<void *>(slices) : Y;
     const razer_dtype odt = S > 1 ? RAZER_F32 : out_dt;
-    r = bf ? launch_tma<true>(map, wmap, ts, unbias, m, n, out, odt, 0, KBw, nullptr, st, S, two ? KB : 0)
-           : launch_tma<false>(map, wmap, ts, unbias, m, n, out, odt, 0, KBw, nullptr, st, S, two ? KB : 0);
+    r = bf ? launch_tma<true>(map, wmap, tbn, ts, unbias, m, n, out, odt, 0, KBw, nullptr, st, S, two ? KB : 0)
+           : launch_tma<false>(map, wmap, tbn, ts, unbias, m, n, out, odt, 0, KBw, nullptr, st, S, two ? KB : 0);
     if (r != RAZER_OK || S == 1) return r;
     return reduce_splits(slices, S, m, n, Y, out_dt, st);
 }
