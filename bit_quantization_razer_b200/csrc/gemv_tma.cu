@@ -45,15 +45,20 @@
 namespace razer {
 namespace gemv_tma {
 
-#ifndef RAZER_GEMV_MT
-#define RAZER_GEMV_MT 2
-#endif
-constexpr int kMT = RAZER_GEMV_MT;                  // 16-row MMA tiles per consumer warp (1 or 2)
 constexpr int kTileRows = 128;
-constexpr int kRowGroups = kTileRows / (16 * kMT);  // consumer warps per k-half
-constexpr int kConsumerWarps = 2 * kRowGroups;      // one per (row group, 128-k half of a stage)
-constexpr int kFirstConsumer = 2;                   // warp 0: TMA producer, warp 1: epilogue
-constexpr int kThreads = 32 * (kFirstConsumer + kConsumerWarps);
+constexpr int kFirstConsumer = 2;  // warp 0: TMA producer, warp 1: epilogue
+// Consumer layout per n8 activation tile count NB: B <= 8 (NB = 1) runs 16
+// consumer warps of one 16-row MMA tile each (more warps to hide the decode's
+// latencies: the three 8B projections at B = 1 / 4 took 30.3 / 32.3 us
+// against 32.0 / 34.1 us with 8 warps); larger B runs 8 warps of two tiles
+// that share the activation fragments (16 warps: 51.8 against 46.8 us at
+// B = 16, and spills at B = 32).
+template <int NB> struct Cfg {
+    static constexpr int MT = NB == 1 ? 1 : 2;                   // 16-row MMA tiles per consumer warp
+    static constexpr int RowGroups = kTileRows / (16 * MT);      // consumer warps per k-half
+    static constexpr int ConsumerWarps = 2 * RowGroups;          // one per (row group, 128-k half of a stage)
+    static constexpr int Threads = 32 * (kFirstConsumer + ConsumerWarps);
+};
 constexpr int kCodeBytes = kTileRows * 128;         // 128 rows x 256 codes
 constexpr int kScaleBytes = kTileRows * 16;         // 128 rows x 16 blocks
 constexpr int kMaxStages = 8;
@@ -131,10 +136,11 @@ __device__ __forceinline__ void wait_phase(uint32_t bar, uint32_t ph, volatile i
 }
 
 template <int FMT, bool BF16, int NB>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<NB>::Threads, 1)
     gemv_tma_kernel(const __grid_constant__ Batch A, int U, int stages, int stage_sz, int slot_elems, float *__restrict__ ws,
                     float unbias, int out_dt, int inject_stall)
 {
+    constexpr int kMT = Cfg<NB>::MT, kConsumerWarps = Cfg<NB>::ConsumerWarps;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const BatchInfo &I = A.info;
@@ -450,7 +456,7 @@ static razer_status launch(const Batch &A, const Plan &pl, float *ws, float unbi
     // fault injection (tests only): one stage is never filled, so the
     // kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
     const int inject = fault_injection_enabled() ? 1 : 0;
-    if (launch_pdl(gemv_tma_kernel<FMT, BF16, NB>, (unsigned)G, kThreads, (size_t)smem, st, A, U, stages, sz, slot_elems, ws, unbias,
+    if (launch_pdl(gemv_tma_kernel<FMT, BF16, NB>, (unsigned)G, (unsigned)Cfg<NB>::Threads, (size_t)smem, st, A, U, stages, sz, slot_elems, ws, unbias,
                    (int)out_dt, inject) != cudaSuccess)
         return RAZER_ERR_CUDA;
     // tiles shared by several CTAs exist unless every CTA range is whole tiles
