@@ -56,6 +56,20 @@ def test_gemm_ragged_multi_tile(orc, fmt, xdt, M):
     assert rel_err(Y.cpu().numpy(), ref) <= REL_TOL
 
 
+@pytest.mark.parametrize("M,rows", [(4096, 32), (200, 200)])
+def test_gemm_oracle_quantized_weights_full_size(orc, M, rows):
+    # a realistic 4096 x 4096 weight matrix (N(0, 0.02^2), 0.1% x10 outliers)
+    # quantized by the oracle, at the prefill M (persistent decode-once path,
+    # sampled rows) and at M = 200 (fused decode, every row)
+    w = workloads.weight(4096, 4096, std=0.02, seed=123)
+    codes, scales, ts, _ = orc.quantize(w.numpy(), 0)
+    X = workloads.vectors(M, 4096, seed=124, dtype=torch.bfloat16)
+    Y = gemm(X, torch.from_numpy(codes), torch.from_numpy(scales), ts, "weight", torch.float32).cpu().numpy()
+    sel = np.sort(np.random.default_rng(125).choice(M, rows, replace=False))
+    ref = orc.gemm_ref(oracle_in(X[sel]), codes, scales, ts, 0)
+    assert rel_err(Y[sel], ref) <= REL_TOL
+
+
 @pytest.mark.parametrize("M", [240, 512])
 def test_gemm_oracle_quantized_weights(orc, M):
     # realistic weights quantized by the oracle; 8 k-steps wrap the 3-stage
