@@ -587,6 +587,10 @@ __global__ void __launch_bounds__(kOneThreads, 1)
     __shared__ int s_abort;
     __shared__ float s_amax;
     __shared__ float tab_d[F::kMagMask + 1], tab_y[F::kMagMask + 1];
+    // launched as a programmatic dependent of the init kernel: resident early,
+    // it touches no global memory before that kernel (and the stream's earlier
+    // work) has completed
+    pdl_wait();
     const int G = gridDim.x, c = blockIdx.x;
     const int64_t b0 = (int64_t)c * nblk / G, b1 = (int64_t)(c + 1) * nblk / G;
     const int nb = (int)(b1 - b0), bytes = nb * 32, nch = (bytes + kOneChunk - 1) / kOneChunk;
@@ -789,11 +793,13 @@ static razer_status launch_onepass(const void *x, int64_t nblk, uint8_t *codes, 
     cfg.blockDim = dim3((unsigned)kOneThreads);
     cfg.dynamicSmemBytes = (size_t)slice;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident at once: the grid barrier cannot wait on an unscheduled CTA
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const int inject = fault_injection_enabled() ? 1 : 0;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const TIn *>(x), nblk, codes, scales, ts_out, hist, inject);
     if (e == cudaErrorCooperativeLaunchTooLarge) {
