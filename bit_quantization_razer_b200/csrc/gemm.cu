@@ -4,7 +4,13 @@
 //
 // (RaZeR notes 关键设计 3: weight-only kernels that decode the remapped codes
 // on the fly; gist.science summary 2.3.)  The contraction is dense, so it runs
-// on the 5th-generation tensor cores:
+// on the 5th-generation tensor cores, by one of two kernels:
+//   * gemm_kernel (below): each CTA decodes its weight tile into shared memory
+//     every k-step -- for small M, where that decode is not repeated often;
+//   * gemm_tma_kernel (further down): the weights are decoded once into a
+//     16-bit copy in HBM and a persistent kernel multiplies two TMA-fed
+//     operands -- for large M, and for M >= 256 on small weight matrices.
+// gemm_kernel:
 //   * CTA tile 256 (M) x 256 (N), k-step 64.  Two UMMA instructions of
 //     M = 128 share one decoded weight tile, so every weight is decoded once
 //     per 256 activation rows (half the decode work per SM of a 128-row tile).
@@ -190,13 +196,11 @@ __device__ __forceinline__ uint4 decode_word(unsigned w, const BlockK &k)
     return make_uint4(p[0], p[1], p[2], p[3]);
 }
 
-// DECODED: the weights were decoded once into a [N, K] 16-bit copy (q*s*2^-bias,
-// exact) that the producer loads by TMA like X; the decoder warps then only
-// run the epilogue.  CTA tiles are rasterised M-fastest so that the CTAs
-// sharing a weight tile run together and find it in L2.
-template <int FMT, bool BF16, bool DECODED>
+// The fused kernel: the decoder warps write each k-step's weight tile into
+// shared memory (the decode-once path runs gemm_tma_kernel instead).
+template <int FMT, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w, const uint8_t *__restrict__ codes,
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t *__restrict__ codes,
                 const uint8_t *__restrict__ scales, const float *__restrict__ ts_p, float unbias, int M, int N, int K,
                 void *Y, int out_dt, int kb0, int nkb, const float *addend, int inject_stall)
 {
@@ -211,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 200);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = (DECODED ? blockIdx.y : blockIdx.x) * BN, m0 = (DECODED ? blockIdx.x : blockIdx.y) * BM;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
     // this launch covers k-steps [kb0, kb0 + nkb) of the K / 64; a previous
     // chunk's fp32 result (already scaled) is added in the epilogue.  With
     // gridDim.z > 1 the range is split further: split z takes its own part and
@@ -248,10 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
                 if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort_flag)) break;
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
-                mbar_expect_tx(full_a + 8 * s, kMBlocks * A_HALF_BYTES + (DECODED ? B_BYTES : 0u));
+                mbar_expect_tx(full_a + 8 * s, kMBlocks * A_HALF_BYTES);
 #pragma unroll
                 for (int a = 0; a < kMBlocks; a++) tma_load_2d(a0 + a * A_HALF_BYTES, &tmap_x, (kbs + kb) * BK, m0 + 128 * a, full_a + 8 * s);
-                if constexpr (DECODED) tma_load_2d(a0 + kMBlocks * A_HALF_BYTES, &tmap_w, (kbs + kb) * BK, n0, full_a + 8 * s);
                 issued = kb + 1;
             }
             if (*abort_flag) {
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < KB && ok; kb++) {
                 const int s = kb % STAGES;
                 const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-                ok = mbar_wait(full_a + 8 * s, ph, abort_flag) && (DECODED || mbar_wait(full_b + 8 * s, ph, abort_flag));
+                ok = mbar_wait(full_a + 8 * s, ph, abort_flag) && mbar_wait(full_b + 8 * s, ph, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t a0 = smem_addr(smem + s * STAGE_BYTES);
@@ -319,11 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         Regs r0, r1;
         bool ok = true;
-        if (!DECODED) {
-            load_stage(0, r0);
-            if (KB > 1) load_stage(1, r1);
-        }
-        for (int kb = 0; kb < (DECODED ? 0 : KB); kb++) {
+        load_stage(0, r0);
+        if (KB > 1) load_stage(1, r1);
+        for (int kb = 0; kb < KB; kb++) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
             uint4 c0[kHalvesPerThread];
@@ -892,8 +893,8 @@ __global__ void __launch_bounds__(256) gemm_splits_reduce1_kernel(const float *_
     }
 }
 
-template <int FMT, bool BF16, bool DECODED>
-static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, const uint8_t *codes, const uint8_t *scales, const float *ts,
+template <int FMT, bool BF16>
+static razer_status launch(const CUtensorMap &map, const uint8_t *codes, const uint8_t *scales, const float *ts,
                            float unbias, int M, int N, int K, void *Y, razer_dtype out_dt, int kb0, int nkb, const float *addend,
                            cudaStream_t st, int splits = 1)
 {
@@ -901,18 +902,18 @@ static razer_status launch(const CUtensorMap &map, const CUtensorMap &wmap, cons
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(gemm_kernel<FMT, BF16, DECODED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+        if (cudaFuncSetAttribute(gemm_kernel<FMT, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
             cudaSuccess)
             return RAZER_ERR_CUDA;
         attr_set[dev] = true;
     }
     const unsigned nt = (unsigned)((N + BN - 1) / BN), mt = (unsigned)((M + BM - 1) / BM);
-    const dim3 grid = DECODED ? dim3(mt, nt, (unsigned)splits) : dim3(nt, mt, (unsigned)splits);
+    const dim3 grid(nt, mt, (unsigned)splits);
     // fault injection (tests only) withholds one decoder warp's arrivals so
     // that the kernel's bounded waits expire (RAZER_ERR_TIMEOUT)
     const int inject = fault_injection_enabled() ? 1 : 0;
-    gemm_kernel<FMT, BF16, DECODED><<<grid, kThreads, SMEM_BYTES, st>>>(map, wmap, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt,
-                                                                      kb0, nkb, addend, inject);
+    gemm_kernel<FMT, BF16><<<grid, kThreads, SMEM_BYTES, st>>>(map, codes, scales, ts, unbias, M, N, K, Y, (int)out_dt, kb0, nkb, addend,
+                                                             inject);
     return last_launch_status();
 }
 
@@ -999,7 +1000,7 @@ static razer_status launch_fmt(const CUtensorMap &map, const CUtensorMap &wmap, 
     void *out = S > 1 ? static_cast<void *>(slices) : Y;
     const razer_dtype odt = S > 1 ? RAZER_F32 : out_dt;
     const razer_status r = decoded ? launch_tma<BF16>(map, wmap, tbn, ts, unbias, M, N, out, odt, 0, KB, nullptr, st, S)
-                                   : launch<FMT, BF16, false>(map, wmap, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S);
+                                   : launch<FMT, BF16>(map, codes, scales, ts, unbias, M, N, K, out, odt, 0, KB, nullptr, st, S);
     if (r != RAZER_OK || S == 1) return r;
     return reduce_splits(slices, S, M, N, Y, out_dt, st);
 }
