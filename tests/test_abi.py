@@ -159,6 +159,29 @@ def test_variant_decode_validation(lib):
     assert d(*dargs(block=48)) == 2
     assert d(*dargs(block=64, K=96)) == 2
     assert d(*dargs(R=0)) == 0                                         # empty tensor
+    # the prefill GEMM on variant weights: every refusal happens before a launch
+    m = lib.razer_gemm_variant
+    m.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                  ctypes.c_int, ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    m.restype = ctypes.c_int
+
+    def margs(block=32, sfmt=0, V=(5.0, -5.0), M=256, N=64, K=128, act=0, codes=FAKE, scales=FAKE, ts=FAKE, ws=None, wsb=0, Y=FAKE):
+        return (FAKE, act, M, codes, scales, ts, block, sfmt, vals(*V), len(V), N, K, Y, 2, ws, wsb, None)
+
+    assert m(*margs(ts=None)) == 1
+    assert m(*margs(block=24)) == 2                                   # block size
+    assert m(*margs(block=64, K=96)) == 2                              # K % block
+    assert m(*margs(M=-1)) == 2
+    assert m(*margs(act=2)) == 4                                       # f32 activations
+    assert m(*margs(V=(5.0, -5.0, 9.5, -9.5), act=1)) == 6             # a bf16 copy would round 9.5 x the scale
+    assert m(*margs(block=32, sfmt=4, K=96)) == 6                      # FP16 words: whole 64-element k-steps
+    assert m(*margs(block=128, sfmt=4, scales=ODD)) == 3               # 16-bit scale words
+    assert m(*margs(codes=ctypes.c_void_p(0x1004))) == 3               # 8-byte aligned codes
+    assert m(*margs(Y=ODD)) == 3
+    assert m(*margs()) == 5                                            # no workspace
+    assert m(*margs(ws=ctypes.c_void_p(0x1000), wsb=16)) == 5          # too small
+    assert m(*margs(M=0)) == 0 and m(*margs(N=0)) == 0                 # empty products
 
 
 def test_quantize_path_selector(lib):
