@@ -91,7 +91,12 @@ __device__ __forceinline__ void decode_word(unsigned w, unsigned s2, unsigned vs
 {
     unsigned q[4] = {cvt_lane<0>(w), cvt_lane<1>(w), cvt_lane<2>(w), cvt_lane<3>(w)};
     if constexpr (Fmt<FMT>::kSpecials > 0) {
-        const unsigned t = (w & 0x77777777u) + 0x77777777u;       // bit 3 set where the magnitude is non-zero
+        // bit 3 set where the magnitude is non-zero; the add is issued as an
+        // integer multiply-add so that it runs on the FMA pipe -- the ALU pipe
+        // (converts, logic) bounds this decode (three 8B projections at
+        // B = 1: 30.3 -> 29.1 us)
+        unsigned t;
+        asm("mad.lo.u32 %0, %1, 1, 0x77777777;" : "=r"(t) : "r"(w & 0x77777777u));
         const unsigned is8 = w & ~t & 0x88888888u;                 // bit 3 set where the code is 0b1000
         const unsigned ind = __umulhi(is8, 0x40000000u);          // is8 >> 2: nibble 0b0010 (= 1.0)
         const unsigned i[4] = {cvt_lane<0>(ind), cvt_lane<1>(ind), cvt_lane<2>(ind), cvt_lane<3>(ind)};
